@@ -1,0 +1,482 @@
+"""Pins of the CPU oracle to facts fixed outside the oracle itself: the pages'
+printed memory figures, hand-worked closed forms, brute force on tiny inputs
+and the invariants the pages state.  CPU only."""
+import math
+import os
+
+import numpy as np
+import pytest
+
+import synthetic as syn
+from oracle import tinyloop_oracle as o
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden_memory():
+    out = {}
+    with open(os.path.join(GOLDEN, "memory_numbers.txt")) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, val, unit = line.split("|")[0].split()
+            out[key] = (float(val), unit)
+    return out
+
+
+# ---------------------------------------------------------------- quantisation
+
+def _f16_hex(x):
+    return np.float16(x).view(np.uint16).item()
+
+
+@pytest.mark.parametrize("bits,weights,scale_hex,codes", [
+    # absmax 0.7: 0.7/7 rounds to fp16 0x2E66 = 0.0999755859375; the ratios
+    # w/s are 7.0017, -3.5009, 1.0002, 0, 2.4996, -7.0017, 0.50012, 3.5009
+    (4, [0.7, -0.35, 0.1, 0, 0.2499, -0.7, 0.05, 0.35], 0x2E66, [7, -4, 1, 0, 2, -7, 1, 4]),
+    # absmax 7 gives scale 1.0 exactly; exact halves round to even
+    (4, [7, 2.5, -2.5, 3.5, -0.5, 0.5, 1.5, 0], 0x3C00, [7, 2, -2, 4, 0, 0, 2, 0]),
+    # an all-zero group has scale 0 and codes 0
+    (4, [0] * 8, 0x0000, [0] * 8),
+    # INT3: absmax 3 gives scale 1.0, codes stay in [-4, 3]
+    (3, [3, 1.5, -1.5, 2.5, -0.5, 0.5, -3, 0], 0x3C00, [3, 2, -2, 2, 0, 0, -3, 0]),
+    # negative absmax element maps to -qmax, never to -qmax-1; scale fp16(0.1),
+    # ratios -3.0007, 1.0002, 0.50012
+    (3, [-0.3, 0.1, 0.05, 0, 0, 0, 0, 0], 0x2E66, [-3, 1, 1, 0, 0, 0, 0, 0]),
+])
+def test_quantize_hand_worked(bits, weights, scale_hex, codes):
+    w = np.array([weights], dtype=np.float32)
+    c, s = o.quantize_groupwise(w, bits, group=8)
+    assert s.view(np.uint16)[0, 0] == scale_hex
+    assert c[0].tolist() == codes
+
+
+def test_pack_layout_int4_nibble_order():
+    # offset binary u = code + 8, lowest k in the lowest nibble
+    codes = np.array([[-8, -7, -6, -5, -4, -3, -2, -1, 0, 1, 2, 3, 4, 5, 6, 7]], np.int8)
+    words = o.pack_codes(codes, 4)
+    assert words.tolist() == [[0x76543210, 0xFEDCBA98]]
+
+
+def test_pack_layout_int3_ten_per_word():
+    # u = code + 4 at bits 3i: the octal digits of the word are u9..u0
+    codes = np.array([[-4, -3, -2, -1, 0, 1, 2, 3, -4, -3, 3]], np.int8)
+    words = o.pack_codes(codes, 3)
+    pad = int("4444444444", 8)
+    assert words.shape == (1, 4)                  # ceil(11/10) = 2 words, padded to 4
+    assert words[0, 0] == 0o1076543210
+    assert words[0, 1] == int("4444444447", 8)    # k=10 holds u=7, the rest padding u=4
+    assert words[0, 2] == pad and words[0, 3] == pad
+    assert int(words.max()) < (1 << 30)           # bits 30-31 zero
+
+
+def test_int3_words_per_row():
+    assert o.int3_words_per_row(2048) == 208       # 205 words padded to 208
+    assert o.int3_words_per_row(8192) == 820
+    assert o.int3_words_per_row(10) == 4
+
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (4, 128), (3, 128), (3, 64)])
+def test_quantize_properties(bits, group):
+    rng = np.random.default_rng(1)
+    w = (rng.standard_normal((37, 4 * group)) * 0.02).astype(np.float32)
+    w[3, :group] = 0.0                                   # all-zero group
+    w[5, group:2 * group] = 1e-3                         # constant group
+    codes, s16 = o.quantize_groupwise(w, bits, group)
+    qmax = o.QMAX[bits]
+    assert codes.min() >= -qmax and codes.max() <= qmax     # -qmax-1 never produced
+    # round trip through the packed words
+    assert np.array_equal(o.unpack_codes(o.pack_codes(codes, bits), w.shape[1], bits), codes)
+    s = np.repeat(s16.astype(np.float64), group, axis=1)
+    err = np.abs(w.astype(np.float64) - codes * s)
+    assert np.all(err <= s / 2 * (1 + 1e-6) + 1e-12)
+    # the largest-magnitude element of each group maps to +-qmax
+    g = np.abs(w).reshape(37, -1, group)
+    am = g.argmax(axis=2)
+    cg = codes.reshape(37, -1, group)
+    top = np.take_along_axis(np.abs(cg), am[..., None], axis=2)[..., 0]
+    nz = s16 != 0
+    assert np.all(top[nz] == qmax)
+    assert np.all(s16[3, 0] == 0) and np.all(codes[3, :group] == 0)
+
+
+def test_dequantize_uses_group_of_each_column():
+    codes = np.ones((1, 8), np.int8)
+    s16 = np.array([[1.0, 2.0, 4.0, 8.0]], np.float16)
+    assert o.dequantize(codes, s16, 2).tolist() == [[1, 1, 2, 2, 4, 4, 8, 8]]
+
+
+# ---------------------------------------------------------------- INT8 KV
+
+def test_kv_int8_hand_worked():
+    # absmax 127 * 2^-7: scale = 2^-7 exactly, codes = 128 x; fp16(0.1) = 0.0999755859375
+    x = np.array([[0.9921875, -0.5, 0.25, 0.00390625, 0.01171875, -0.9921875, 0.1, 0.0]], np.float16)
+    c, s = o.kv_quant_int8(x)
+    assert s[0] == np.float16(2.0 ** -7)
+    assert c[0].tolist() == [127, -64, 32, 0, 2, -127, 13, 0]
+
+
+def test_kv_int8_properties():
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((64, 16, 128)).astype(np.float16)
+    x[0, 0] = 0
+    c, s = o.kv_quant_int8(x)
+    assert c.shape == x.shape and s.shape == (64, 16)
+    assert s[0, 0] == 0 and np.all(c[0, 0] == 0)
+    am = np.abs(x.astype(np.float32)).max(-1)
+    assert np.array_equal(s, (am / np.float32(127)).astype(np.float16))   # one scale per (token, head)
+    err = np.abs(x.astype(np.float64) - o.kv_dequant_int8(c, s))
+    assert np.all(err <= s.astype(np.float64)[..., None] / 2 * (1 + 1e-6) + 1e-12)
+    assert np.all(np.abs(c).max(-1)[s != 0] == 127)
+
+
+# ---------------------------------------------------------------- memory figures
+
+def test_kv_bytes_match_pages():
+    g = _golden_memory()
+    fp16 = o.kv_cache_bytes(10, 2048, 16, 128, "fp16")
+    int8 = o.kv_cache_bytes(10, 2048, 16, 128, "int8")
+    assert round(fp16 / 1e6, 1) == g["kv_fp16_max_seq_2048_10_layers"][0]
+    assert round(int8 / 1e6, 1) == g["kv_int8_max_seq_2048_10_layers"][0]
+    assert round((int8 / fp16 - 1) * 100, 1) == g["kv_int8_delta_percent"][0]
+
+
+def test_weight_counts_match_pages():
+    g = _golden_memory()
+    per_block = o.block_weight_count(2048, 8192)
+    assert per_block == 64 * 2 ** 20
+    params = 3 * per_block + 2 * syn.VOCAB * 2048               # 3 blocks + embedding + head
+    assert round(params / 1e6) == g["model_params"][0]
+    # the FP16 body cache adds 2 bytes per body weight: 216 -> 619 MB
+    delta = g["weight_vram_int4_plus_fp16_body"][0] - g["weight_vram_int4"][0]
+    assert abs(3 * per_block * 2 / 1e6 - delta) < 1.0
+    # weight bytes of one packed INT4 block (group 128) and INT3 block
+    assert o.packed_block_bytes(2048, 8192, 4, 128) == 32 * 2 ** 20 + 2 ** 20
+    assert o.packed_block_bytes(2048, 8192, 3, 128) < o.packed_block_bytes(2048, 8192, 4, 128)
+
+
+# ---------------------------------------------------------------- RMSNorm / RoPE / SwiGLU
+
+def test_rmsnorm_closed_form():
+    rng = np.random.default_rng(3)
+    h = rng.standard_normal((5, 64)) * 3
+    gam = 1 + 0.1 * rng.standard_normal(64)
+    y = o.rmsnorm(h, gam, 1e-5)
+    ms = (h * h).mean(-1)
+    rms_unscaled = np.sqrt(((y / gam) ** 2).mean(-1))
+    assert np.allclose(rms_unscaled, np.sqrt(ms / (ms + 1e-5)), rtol=1e-12)
+    # per element, against a plain loop
+    for t in range(5):
+        s = sum(float(v) * float(v) for v in h[t]) / 64
+        for i in range(64):
+            assert abs(y[t, i] - h[t, i] / math.sqrt(s + 1e-5) * gam[i]) < 1e-12
+
+
+def test_rope_hand_values():
+    # hd = 2: inv_freq = 1, so pos 1 rotates the pair by 1 rad
+    y = o.rope(np.array([[[1.0, 0.0]]]), np.array([1]), 10000.0)
+    assert np.allclose(y[0, 0], [math.cos(1), math.sin(1)], atol=1e-15)
+    y = o.rope(np.array([[[0.0, 1.0]]]), np.array([2]), 10000.0)
+    assert np.allclose(y[0, 0], [-math.sin(2), math.cos(2)], atol=1e-15)
+    # hd = 4: pair (1, 3) has inv_freq 10000^(-2/4) = 0.01, so pos 100 turns it by 1 rad
+    y = o.rope(np.array([[[0.0, 1.0, 0.0, 0.0]]]), np.array([100]), 10000.0)
+    assert np.allclose(y[0, 0], [0, math.cos(1), 0, math.sin(1)], atol=1e-12)
+
+
+def test_rope_properties():
+    rng = np.random.default_rng(4)
+    hd = 64
+    q = rng.standard_normal((1, 3, hd))
+    k = rng.standard_normal((1, 3, hd))
+    assert np.array_equal(o.rope(q, np.array([0]), 1e4), q)             # pos 0 is identity
+    r = o.rope(q, np.array([777]), 1e4)
+    half = hd // 2
+    assert np.allclose(r[..., :half] ** 2 + r[..., half:] ** 2, q[..., :half] ** 2 + q[..., half:] ** 2)
+    # <R_m q, R_n k> depends only on m - n
+    dots = [np.sum(o.rope(q, np.array([m]), 1e4) * o.rope(k, np.array([m - 5]), 1e4)) for m in (5, 40, 900)]
+    assert np.allclose(dots, dots[0], rtol=1e-9)
+    # complex-number form: z_i = x_i + j x_{i+hd/2} multiplied by exp(j pos theta^(-2i/hd))
+    z = q[..., :half] + 1j * q[..., half:]
+    w = z * np.exp(1j * 321 * 1e4 ** (-2 * np.arange(half) / hd))
+    r = o.rope(q, np.array([321]), 1e4)
+    assert np.allclose(r[..., :half], w.real) and np.allclose(r[..., half:], w.imag)
+
+
+def test_silu_identities():
+    z = np.linspace(-30, 30, 121)
+    s = o.silu(z)
+    assert o.silu(np.array([0.0]))[0] == 0
+    assert np.allclose(s - o.silu(-z), z)                      # silu(x) - silu(-x) = x
+    assert np.allclose(o.silu(np.array([40.0])), 40.0)
+    assert abs(o.silu(np.array([1.0]))[0] - 1 / (1 + math.exp(-1))) < 1e-15
+
+
+# ---------------------------------------------------------------- attention
+
+def _attention_brute(q, k, v, q_pos):
+    tq, nh, hd = q.shape
+    out = np.zeros_like(q, dtype=np.float64)
+    for t in range(tq):
+        for h in range(nh):
+            sc = [sum(q[t, h, e] * k[j, h, e] for e in range(hd)) / math.sqrt(hd) for j in range(q_pos[t] + 1)]
+            m = max(sc)
+            p = [math.exp(x - m) for x in sc]
+            z = sum(p)
+            for e in range(hd):
+                out[t, h, e] = sum(p[j] * v[j, h, e] for j in range(len(p))) / z
+    return out
+
+
+@pytest.mark.parametrize("t,nh,hd", [(1, 1, 4), (5, 2, 4), (9, 3, 8), (16, 1, 16)])
+def test_attention_brute_force(t, nh, hd):
+    rng = np.random.default_rng(t * 100 + hd)
+    q, k, v = (rng.standard_normal((t, nh, hd)) for _ in range(3))
+    pos = np.arange(t)
+    assert np.allclose(o.causal_attention(q, k, v, pos), _attention_brute(q, k, v, pos), atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(5)
+    k, v = rng.standard_normal((7, 2, 8)), rng.standard_normal((7, 2, 8))
+    # a single key returns its value
+    assert np.allclose(o.causal_attention(rng.standard_normal((1, 2, 8)), k[:1], v[:1], np.array([0])), v[:1])
+    # q = 0 gives the mean of the visible values (causal prefix means)
+    out = o.causal_attention(np.zeros((7, 2, 8)), k, v, np.arange(7))
+    pref = np.cumsum(v, axis=0) / np.arange(1, 8)[:, None, None]
+    assert np.allclose(out, pref)
+    # a decode query at position p sees keys 0..p
+    out = o.causal_attention(rng.standard_normal((1, 2, 8)), k, v, np.array([3]))
+    out2 = o.causal_attention(out * 0 + 0, k[:4], v[:4], np.array([3]))
+    assert np.allclose(out2[0], v[:4].mean(0))
+
+
+# ---------------------------------------------------------------- whole block, brute force
+
+def _tiny_cfg():
+    return {"d_model": 8, "n_heads": 2, "head_dim": 4, "ffn": 16, "bits": 4, "group": 8,
+            "eps": 1e-5, "rope_theta": 10000.0}
+
+
+def _tiny_weights(seed):
+    shape = syn.BlockShape(8, 2, 4, 16)
+    w = syn.block_weights(shape, seed, "tiny")
+    for k in list(w):
+        if k.startswith("w_"):
+            w[k] = (w[k] * 10).astype(np.float32)
+    return w
+
+
+def _block_brute(blk, h, pos0=0):
+    """One block by explicit loops over indices, from the dequantised weights."""
+    c = blk.cfg
+    d, nh, hd, f = c["d_model"], c["n_heads"], c["head_dim"], c["ffn"]
+    W = blk.W
+    t = len(h)
+
+    def norm(row, g):
+        ms = sum(x * x for x in row) / d
+        return [row[i] / math.sqrt(ms + c["eps"]) * g[i] for i in range(d)]
+
+    def mv(m, x):
+        return [sum(m[n][kk] * x[kk] for kk in range(len(x))) for n in range(len(m))]
+
+    q = [[[0.0] * hd for _ in range(nh)] for _ in range(t)]
+    k = [[[0.0] * hd for _ in range(nh)] for _ in range(t)]
+    v = [[[0.0] * hd for _ in range(nh)] for _ in range(t)]
+    for ti in range(t):
+        x = norm(list(h[ti]), blk.gamma_attn)
+        y = mv(W["qkv"], x)
+        for hh in range(nh):
+            for e in range(hd):
+                q[ti][hh][e] = y[hh * hd + e]
+                k[ti][hh][e] = y[d + hh * hd + e]
+                v[ti][hh][e] = y[2 * d + hh * hd + e]
+        for arr in (q, k):
+            for hh in range(nh):
+                vec = list(arr[ti][hh])
+                for i in range(hd // 2):
+                    a = (pos0 + ti) * c["rope_theta"] ** (-2.0 * i / hd)
+                    arr[ti][hh][i] = vec[i] * math.cos(a) - vec[i + hd // 2] * math.sin(a)
+                    arr[ti][hh][i + hd // 2] = vec[i + hd // 2] * math.cos(a) + vec[i] * math.sin(a)
+    out = []
+    for ti in range(t):
+        att = []
+        for hh in range(nh):
+            sc = [sum(q[ti][hh][e] * k[j][hh][e] for e in range(hd)) / math.sqrt(hd) for j in range(ti + 1)]
+            m = max(sc)
+            p = [math.exp(s - m) for s in sc]
+            z = sum(p)
+            att += [sum(p[j] * v[j][hh][e] for j in range(ti + 1)) / z for e in range(hd)]
+        o1 = mv(W["o"], att)
+        r = [h[ti][i] + o1[i] for i in range(d)]
+        x = norm(r, blk.gamma_ffn)
+        g = mv(W["gate"], x)
+        u = mv(W["up"], x)
+        a = [g[i] / (1 + math.exp(-g[i])) * u[i] for i in range(f)]
+        dn = mv(W["down"], a)
+        out.append([r[i] + dn[i] for i in range(d)])
+    return np.array(out)
+
+
+def _apply_block(blk, h):
+    pos = np.arange(len(h))
+    q, k, v = blk.qkv(h, pos)
+    return blk.finish(h, o.causal_attention(q, k, v, pos))
+
+
+def test_block_brute_force():
+    blk = o.Block.from_fp32(_tiny_weights(7), _tiny_cfg())
+    h = np.random.default_rng(8).standard_normal((3, 8))
+    assert np.allclose(_apply_block(blk, h), _block_brute(blk, h), atol=1e-12)
+
+
+def test_zero_weights_block_is_identity():
+    w = _tiny_weights(9)
+    for k in list(w):
+        if k.startswith("w_"):
+            w[k] = np.zeros_like(w[k])
+    blk = o.Block.from_fp32(w, _tiny_cfg())
+    h = np.random.default_rng(10).standard_normal((4, 8))
+    assert np.array_equal(_apply_block(blk, h), h)
+
+
+# ---------------------------------------------------------------- model invariants
+
+def _tiny_model(L_seed=11, n_pre=1):
+    cfg = _tiny_cfg()
+    pre = [o.Block.from_fp32(_tiny_weights(L_seed + i), cfg) for i in range(n_pre)]
+    loop = o.Block.from_fp32(_tiny_weights(L_seed + 50), cfg)
+    gam = 1 + 0.1 * np.random.default_rng(L_seed).standard_normal(8)
+    emb = (np.random.default_rng(L_seed + 1).standard_normal((20, 8))).astype(np.float16)
+    return o.LoopedModel(pre, loop, gam, emb)
+
+
+def test_schedule_reuses_loop_block():
+    m = _tiny_model()
+    sched = m.schedule(5)
+    assert len(sched) == 6 and all(b is m.loop for b in sched[1:])
+
+
+def test_L_copies_equal_L_iterations():
+    m = _tiny_model()
+    ids = np.array([1, 5, 7, 2, 19])
+    for L in (1, 3, 6):
+        looped = m.prefill(ids, L)
+        deep = o.unrolled_copy(m, L).prefill(ids, L)
+        assert np.array_equal(looped, deep)
+
+
+def test_cached_decode_matches_uncached_forward():
+    m = _tiny_model()
+    ids = np.array([3, 1, 4, 1, 5, 9, 2, 6, 5, 3])
+    L = 3
+    full = m.prefill(ids, L)
+    kv = m.new_kv(L, "exact")
+    m.prefill(ids[:4], L, kv=kv)
+    for t in range(4, 10):
+        y = m.decode_step(ids[t], L, kv)
+        assert np.allclose(y, full[t], atol=1e-12)
+    # with FP16 storage the cached path stays within the float tolerance
+    kv16 = m.new_kv(L, "fp16")
+    m.prefill(ids[:4], L, kv=kv16)
+    for t in range(4, 10):
+        y = m.decode_step(ids[t], L, kv16)
+        cos = y @ full[t] / np.linalg.norm(y) / np.linalg.norm(full[t])
+        assert cos > 0.9999
+
+
+def test_per_lane_L_is_its_own_run():
+    m = _tiny_model()
+    ids = np.array([4, 8, 15, 16])
+    outs = {}
+    for L in (1, 2, 4):
+        kv = m.new_kv(L, "fp16")
+        m.prefill(ids, L, kv=kv)
+        outs[L] = m.decode_step(np.int64(7), L, kv)
+    assert not np.allclose(outs[1], outs[4])          # depth changes the result
+    kv = m.new_kv(2, "fp16")
+    m.prefill(ids, 2, kv=kv)
+    assert np.array_equal(m.decode_step(np.int64(7), 2, kv), outs[2])
+
+
+def test_kv_slot_count_is_pre_plus_L():
+    m = _tiny_model(n_pre=2)
+    kv = m.new_kv(5, "fp16")
+    m.prefill(np.array([1, 2, 3]), 5, kv=kv)
+    assert len(kv) == 7 and all(len(s) == 3 for s in kv)
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _pins_pass():
+    """Run the cheap pins; returns False if any fails."""
+    checks = [test_block_brute_force, test_rope_hand_values, test_rope_properties,
+              lambda: test_attention_brute_force(5, 2, 4), test_attention_special_cases,
+              test_rmsnorm_closed_form, test_cached_decode_matches_uncached_forward,
+              test_zero_weights_block_is_identity, test_dequantize_uses_group_of_each_column]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def _mutants():
+    orig_rope, orig_attn, orig_finish, orig_norm, orig_deq = (
+        o.rope, o.causal_attention, o.Block.finish, o.rmsnorm, o.dequantize)
+
+    def rope_sign(x, pos, theta):             # wrong sign of the sine term
+        return orig_rope(x, -np.asarray(pos), theta)
+
+    def rope_pairs(x, pos, theta):            # interleaved instead of rotate-half pairing
+        y = np.asarray(x, float)
+        hd = y.shape[-1]
+        perm = np.concatenate([np.arange(0, hd, 2), np.arange(1, hd, 2)])
+        inv = np.argsort(perm)
+        return orig_rope(y[..., perm], pos, theta)[..., inv]
+
+    def attn_no_mask(q, k, v, q_pos):         # causal mask dropped
+        return orig_attn(q, k, v, np.full(len(q_pos), k.shape[0] - 1))
+
+    def attn_no_scale(q, k, v, q_pos):        # 1/sqrt(hd) dropped
+        return orig_attn(np.asarray(q) * math.sqrt(q.shape[-1]), k, v, q_pos)
+
+    def finish_no_residual(self, h, attn):    # residual add dropped
+        return orig_finish(self, h, attn) - h
+
+    def finish_transposed_o(self, h, attn):   # W_o used transposed
+        w = self.W["o"]
+        self.W["o"] = w.T
+        try:
+            return orig_finish(self, h, attn)
+        finally:
+            self.W["o"] = w
+
+    def norm_no_gain(h, gamma, eps):          # gain ignored
+        return orig_norm(h, np.ones_like(gamma), eps)
+
+    def norm_no_eps(h, gamma, eps):           # mean of squares replaced by mean of abs
+        hh = np.asarray(h, float)
+        return hh / np.mean(np.abs(hh), axis=-1, keepdims=True) * gamma
+
+    def deq_wrong_group(codes, s, g):         # group index k % n_groups instead of k // g
+        return codes.astype(float) * np.tile(s.astype(float), (1, codes.shape[1] // s.shape[1]))
+
+    return [("rope", rope_sign), ("rope", rope_pairs), ("causal_attention", attn_no_mask),
+            ("causal_attention", attn_no_scale), ("finish", finish_no_residual),
+            ("finish", finish_transposed_o), ("rmsnorm", norm_no_gain), ("rmsnorm", norm_no_eps),
+            ("dequantize", deq_wrong_group)]
+
+
+@pytest.mark.parametrize("idx", range(9))
+def test_planted_mistake_is_caught(monkeypatch, idx):
+    """Each plausible mistake planted in the oracle makes at least one pin fail."""
+    # the pins compare against brute force built on the (possibly mutated) Block
+    # weights, so mutate the module-level functions the oracle itself calls
+    name, fn = _mutants()[idx]
+    if name == "finish":
+        monkeypatch.setattr(o.Block, "finish", fn)
+    else:
+        monkeypatch.setattr(o, name, fn)
+    assert not _pins_pass()
