@@ -1,0 +1,275 @@
+/*
+ * tl.h - C ABI of the B200 looped-block library (libtinyloop_b200.so).
+ *
+ * The library runs the hot path of a weight-shared looped transformer: embed,
+ * a few pre-blocks applied once, one shared block applied L times with the same
+ * weights, final RMSNorm, no logits ("TinyLoop Framework", the four-step list of
+ * the architectural family; "Performance and Memory", "Benchmark Shape
+ * Matters").  Prefill and KV-cached decode are both covered ("Production
+ * Roadmap", Stage 1: default-on KV-cache decode).
+ *
+ * Conventions (every function):
+ *   - Returns tl_status.  Nothing aborts or exits.  On failure a description is
+ *     available from tl_last_error() (thread-local, valid until the next call
+ *     on the same thread).
+ *   - Argument checks (null pointers, shapes, L range, context overflow, bit
+ *     width) happen on the host before any launch; a rejected call launches
+ *     nothing and changes no state.
+ *   - "device pointer" arguments are caller-owned CUDA device memory (for
+ *     example allocated by PyTorch).  The library never frees caller memory.
+ *     Where a pointer may be host or device memory it says so.
+ *   - Handles (tl_block, tl_model, tl_kv) are library-owned and released by the
+ *     matching *_destroy.  A tl_model owns its workspace, RoPE table and CUDA
+ *     graphs; a tl_kv owns nothing on the device (its storage is the caller's).
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL is the legacy default
+ *     stream) and is asynchronous.  Device-side errors (a bounded wait that ran
+ *     out, a non-finite output) are recorded in the model's status word and
+ *     returned by tl_sync_status().
+ *   - All matrices are row-major.  fp16/bf16 values travel as uint16_t bits.
+ */
+#ifndef TINYLOOP_B200_TL_H
+#define TINYLOOP_B200_TL_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* tl_stream; /* same type as cudaStream_t */
+
+typedef enum tl_status {
+  TL_OK = 0,
+  TL_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, L out of range, overflow */
+  TL_ERR_CUDA = 2,         /* a CUDA runtime/driver call failed */
+  TL_ERR_OOM = 3,          /* a library-owned allocation failed */
+  TL_ERR_TIMEOUT = 4,      /* a bounded device-side wait ran out */
+  TL_ERR_UNSUPPORTED = 5,  /* valid request outside what this build implements */
+  TL_ERR_NUMERIC = 6       /* a non-finite value reached an output */
+} tl_status;
+
+typedef enum tl_kv_dtype {
+  TL_KV_FP16 = 0,  /* K and V as fp16 */
+  TL_KV_INT8 = 1   /* int8 codes + one fp16 scale per (token, head) */
+} tl_kv_dtype;
+
+/* Description of the last failure on this thread ("" if none). */
+const char* tl_last_error(void);
+
+/* ABI version of this header (major * 100 + minor). */
+int tl_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Weight packing.  Group-wise symmetric quantisation along K with one fp16
+ * scale per group: INT4 ("TinyLoop Framework", "What Makes It Different":
+ * INT2/INT4 low-bit execution) and INT3 ("Current Status", core inference
+ * table, INT3 GEMM row: 8 levels, 3 bits per weight, 10 values per 32-bit word,
+ * converter --bits 3).
+ *
+ * Quantisation (both widths, all in IEEE fp32):
+ *   scale = fp16_rne(max|w| over the group / qmax)      qmax = 7 (INT4), 3 (INT3)
+ *   code  = clamp(rint(w / float(scale)), -qmax-1, qmax)  (rint ties to even;
+ *           scale == 0 gives code 0)
+ * Canonical packed layout (row n of an [N, K] matrix, row-major):
+ *   INT4: K/8 uint32 words per row; u = code + 8; word j holds k = 8j..8j+7,
+ *         element 8j+i in bits 4i..4i+3.
+ *   INT3: W3 = ceil(K/10) rounded up to a multiple of 4 words per row;
+ *         u = code + 4; word j holds k = 10j..10j+9, element 10j+i in bits
+ *         3i..3i+2; bits 30-31 zero; unused slots hold u = 4 (code 0).
+ *   Scales: fp16 [N, K/group], row-major.
+ * ------------------------------------------------------------------------ */
+
+/* Words per packed row for K columns at `bits` (3 or 4). */
+tl_status tl_packed_words_per_row(int K, int bits, int* words);
+
+/* Bytes of the packed codes and of the fp16 scales of an [N, K] matrix.
+ * Requirements: N >= 1, K >= 1, bits in {3, 4}, group in {64, 128},
+ * K % group == 0, and K % 8 == 0 for INT4. */
+tl_status tl_packed_bytes(int N, int K, int bits, int group,
+                          size_t* code_bytes, size_t* scale_bytes);
+
+/* Quantise and pack an fp32 [N, K] matrix on the device.
+ *   w       device pointer, fp32 [N, K]; must be finite.
+ *   packed  device pointer, uint32 [N, words_per_row]  (written)
+ *   scales  device pointer, fp16   [N, K/group]        (written)
+ * Bit-exact with the definition above.  Runs once per matrix, at load time. */
+tl_status tl_pack_weights(const float* w, int N, int K, int bits, int group,
+                          uint32_t* packed, uint16_t* scales, tl_stream stream);
+
+/* Test hook: unpack canonical packed words back to int8 codes [N, K]
+ * (device pointers). */
+tl_status tl_unpack_codes(const uint32_t* packed, int N, int K, int bits,
+                          int8_t* codes, tl_stream stream);
+
+/* Per-(token, head) symmetric INT8 KV quantisation ("Performance and Memory",
+ * "KV cache INT8" table and the sentence under it: per-token per-head
+ * symmetric INT8 with one FP16 scale per (token, head)).  For each row of hd
+ * fp16 values x:  scale = fp16_rne(max|x| / 127),  code = clamp(rint(x /
+ * float(scale)), -127, 127), scale == 0 gives codes 0; dequantised value is
+ * code * scale.
+ *   x       device pointer, fp16 [rows, hd]
+ *   codes   device pointer, int8 [rows, hd]   (written)
+ *   scales  device pointer, fp16 [rows]       (written)
+ * Requirements: rows >= 0, 1 <= hd <= 256. */
+tl_status tl_kv_quant_int8(const uint16_t* x, int rows, int hd, int8_t* codes,
+                           uint16_t* scales, tl_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Blocks.  One pre-norm transformer block: RMSNorm -> fused QKV -> RoPE on q
+ * and k -> causal attention -> O projection + residual -> RMSNorm -> SwiGLU
+ * (silu(gate) * up) -> down projection + residual.  RoPE is applied on every
+ * forward path ("Current Status", model architecture table, RoPE row); the
+ * pairing is rotate-half (i, i + head_dim/2), angle = pos * theta^(-2i/hd).
+ * The residual stream is fp32 ("Current Status", core inference table: the
+ * FP16 residual stream is opt-in, so FP32 is the default).
+ * ------------------------------------------------------------------------ */
+typedef struct tl_block_desc {
+  int d_model;     /* d; multiple of 256, at most 8192 */
+  int n_heads;     /* H; n_heads * head_dim == d_model (multi-head, no GQA) */
+  int head_dim;    /* 64 or 128 */
+  int ffn;         /* F; multiple of 128 */
+  int bits;        /* 4 or 3 */
+  int group;       /* 64 or 128 */
+  float eps;       /* RMSNorm epsilon, e.g. 1e-5 */
+  float rope_theta;/* e.g. 10000 */
+  /* Canonical packed weights (see tl_pack_weights), device pointers.  Rows
+   * are output features.  w_qkv is [3d, d] with rows [Q; K; V], head-major. */
+  const uint32_t* w_qkv;  const uint16_t* s_qkv;   /* [3d, d] */
+  const uint32_t* w_o;    const uint16_t* s_o;     /* [d, d]  */
+  const uint32_t* w_gate; const uint16_t* s_gate;  /* [F, d]  */
+  const uint32_t* w_up;   const uint16_t* s_up;    /* [F, d]  */
+  const uint32_t* w_down; const uint16_t* s_down;  /* [d, F]  */
+  const float* gamma_attn;                          /* [d] RMSNorm gain before QKV */
+  const float* gamma_ffn;                           /* [d] RMSNorm gain before SwiGLU */
+} tl_block_desc;
+
+typedef struct tl_block tl_block;
+
+/* Validate a block description and wrap it.  The block references the caller's
+ * device memory (no copy); that memory must outlive the block and every model
+ * built from it. */
+tl_status tl_block_create(const tl_block_desc* desc, tl_block** out);
+tl_status tl_block_destroy(tl_block* block);
+
+/* ------------------------------------------------------------------------
+ * Models.  Weight memory is tied to unique blocks, not to effective depth
+ * ("TinyLoop Framework", "What Makes It Different"): a model references its
+ * n_pre + 1 blocks once and L is an argument of every forward call ("Loop count
+ * is a runtime knob").
+ * ------------------------------------------------------------------------ */
+typedef struct tl_model_desc {
+  const tl_block* const* pre; /* n_pre blocks applied once each, in order */
+  int n_pre;                  /* >= 0 */
+  const tl_block* loop;       /* the shared block applied L times */
+  const uint16_t* embed;      /* device fp16 [vocab, d] or NULL (hidden-state input only) */
+  int vocab;
+  const float* gamma_final;   /* device fp32 [d], final RMSNorm gain */
+  int max_tokens;             /* largest seq passed to tl_prefill, >= 1 */
+  int max_lanes;              /* largest n_lanes passed to tl_decode_step, 1..8 */
+  int max_ctx;                /* largest position + 1 any call may reach */
+  int max_L;                  /* largest loop count any call may use, 1..64 */
+} tl_model_desc;
+
+typedef struct tl_model tl_model;
+
+/* Build a model: allocates the library-owned workspace (sized by max_tokens,
+ * max_lanes), the RoPE table (max_ctx) and the status word on the current
+ * device.  All blocks must share d_model, n_heads, head_dim and ffn. */
+tl_status tl_model_create(const tl_model_desc* desc, tl_model** out);
+tl_status tl_model_destroy(tl_model* model);
+
+/* Library-owned device bytes of a model (workspace + tables).  Independent of
+ * any L. */
+tl_status tl_model_device_bytes(const tl_model* model, size_t* bytes);
+
+/* Enable (default) or disable CUDA-graph replay of the forward calls. */
+tl_status tl_model_set_graphs(tl_model* model, int enable);
+
+/* ------------------------------------------------------------------------
+ * KV cache.  Every layer application keeps its own K/V slot: n_pre slots for
+ * the pre-blocks and one per loop iteration ("Performance and Memory", "KV
+ * cache INT8" table: 10 layers for 2 pre-blocks + L=8).  Lane b has
+ * n_pre + L_per_lane[b] slots.
+ *
+ * Storage is caller-owned: tl_kv_bytes gives the size, the caller allocates
+ * one device buffer (256-byte aligned) and tl_kv_create lays the cache out in
+ * it.  Layout inside the buffer: a 4 KiB header (per-lane positions), then for
+ * each lane b, for each layer l < n_pre + L_b: K [H][max_ctx][hd], V
+ * [H][max_ctx][hd] (fp16, or int8 codes), then for INT8 the scales K
+ * [H][max_ctx], V [H][max_ctx] (fp16); every region starts on 256 bytes.
+ * K is stored after RoPE.
+ * ------------------------------------------------------------------------ */
+typedef struct tl_kv tl_kv;
+
+/* Bytes of one (lane, layer) slot: 2 * align256(H * max_ctx * hd * elem)
+ * plus, for INT8, 2 * align256(H * max_ctx * 2) of fp16 scales.  Host-only. */
+tl_status tl_kv_layer_bytes(int n_heads, int head_dim, int max_ctx, tl_kv_dtype dtype,
+                            size_t* bytes);
+
+tl_status tl_kv_bytes(const tl_model* model, int n_lanes, int max_ctx,
+                      const int* L_per_lane /* host [n_lanes] */,
+                      tl_kv_dtype dtype, size_t* bytes);
+tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
+                       const int* L_per_lane /* host [n_lanes] */,
+                       tl_kv_dtype dtype, void* buffer, size_t buffer_bytes,
+                       tl_kv** out);
+tl_status tl_kv_destroy(tl_kv* kv);
+/* Set the position of one lane (lane >= 0) or of every lane (lane == -1) to
+ * 0.  Enqueued on `stream`. */
+tl_status tl_kv_reset(tl_kv* kv, int lane, tl_stream stream);
+/* Host-side position (number of cached tokens) of a lane. */
+tl_status tl_kv_position(const tl_kv* kv, int lane, int* pos);
+/* Declare that positions 0..pos-1 of a lane already hold valid entries (for a
+ * cache filled by the caller through tl_kv_layer_ptrs). */
+tl_status tl_kv_set_position(tl_kv* kv, int lane, int pos, tl_stream stream);
+/* Device pointers of one (lane, layer) slot: K, V ([H][max_ctx][hd]) and, for
+ * INT8, the scales ([H][max_ctx]; NULL for FP16). */
+tl_status tl_kv_layer_ptrs(const tl_kv* kv, int lane, int layer, void** k,
+                           void** v, uint16_t** k_scale, uint16_t** v_scale);
+
+/* ------------------------------------------------------------------------
+ * Forward calls.  Input and output pointers may be host or device memory
+ * (copies to and from the model's workspace are enqueued on `stream`; host
+ * memory should be pinned for asynchronous copies).
+ * ------------------------------------------------------------------------ */
+
+/* Causal prefill of `seq` tokens at positions 0..seq-1 of one lane.
+ *   ids      int32 [seq] token ids (needs an embedding), or NULL
+ *   h_in     fp16 [seq, d] input hidden states, or NULL (exactly one of the two)
+ *   L        loop count, 1..max_L (and <= the lane's L when kv is given)
+ *   kv       cache to fill (positions 0..seq-1 of `lane`, position set to seq),
+ *            or NULL for an uncached forward
+ *   y_out    fp32 [seq, d]: final RMSNorm of the residual stream (no logits)
+ *   h_trace  NULL, or fp32 [n_pre + L, seq, d]: the residual stream after each
+ *            block application (a test hook)
+ * The sequence is processed as one CUDA graph per (seq, L, lane, kv). */
+tl_status tl_prefill(tl_model* model, const int32_t* ids, const uint16_t* h_in,
+                     int seq, int L, tl_kv* kv, int lane, float* y_out,
+                     float* h_trace, tl_stream stream);
+
+/* One cached decode step for lanes 0..n_lanes-1 of `kv`: each lane appends
+ * one token at its current position and runs with its own loop count
+ * ("Current Status", architecture-unique table, L-aware batching row:
+ * per-lane loops, each lane bit-exact with its own run).
+ *   ids         int32 [n_lanes], or NULL
+ *   h_in        fp16 [n_lanes, d], or NULL (exactly one of the two)
+ *   L_per_lane  host int [n_lanes]; 1 <= L_b <= the L the lane's cache holds
+ *   y_out       fp32 [n_lanes, d]
+ *   h_trace     NULL, or fp32 [n_pre + max_b L_b, n_lanes, d]; rows of lanes
+ *               that ran fewer iterations keep their last value
+ * A lane's result does not depend on the other lanes or on n_lanes. */
+tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
+                         const uint16_t* h_in, const int* L_per_lane,
+                         int n_lanes, float* y_out, float* h_trace,
+                         tl_stream stream);
+
+/* Synchronise `stream`, then return and clear the model's device status word
+ * (TL_OK, TL_ERR_TIMEOUT or TL_ERR_NUMERIC). */
+tl_status tl_sync_status(tl_model* model, tl_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TINYLOOP_B200_TL_H */

@@ -298,12 +298,14 @@ def pack_block(weights: Dict[str, np.ndarray], bits: int, group: int) -> Dict[st
 class KVSlot:
     """K/V of one layer (one pre-block or one loop iteration) for one lane, in
     the cache's storage dtype: "fp16", "int8" or "exact" (fp64, used only to
-    check the cached path against the uncached one without storage rounding)."""
+    check the cached path against the uncached one without storage rounding).
+    Stored values are kept dequantised, positions 0..len-1."""
 
     def __init__(self, dtype: str):
         self.dtype = dtype
-        self.k: List[np.ndarray] = []     # per position, [H, hd] as stored
-        self.v: List[np.ndarray] = []
+        self._k: Optional[np.ndarray] = None
+        self._v: Optional[np.ndarray] = None
+        self.n = 0
 
     def _store(self, x: np.ndarray) -> np.ndarray:
         if self.dtype == "exact":
@@ -316,18 +318,43 @@ class KVSlot:
             return kv_dequant_int8(codes, scale)
         raise ValueError(self.dtype)
 
+    def _reserve(self, n: int, shape) -> None:
+        if self._k is None or self._k.shape[0] < n:
+            cap = max(n, 2 * (0 if self._k is None else self._k.shape[0]), 16)
+            k = np.empty((cap,) + tuple(shape), F64)
+            v = np.empty((cap,) + tuple(shape), F64)
+            if self._k is not None:
+                k[:self.n] = self._k[:self.n]
+                v[:self.n] = self._v[:self.n]
+            self._k, self._v = k, v
+
     def append(self, k: np.ndarray, v: np.ndarray) -> None:
-        for t in range(k.shape[0]):
-            self.k.append(self._store(k[t]))
-            self.v.append(self._store(v[t]))
+        """Append T positions: k, v [T, H, hd], stored in the cache dtype."""
+        t = k.shape[0]
+        self._reserve(self.n + t, k.shape[1:])
+        self._k[self.n:self.n + t] = self._store(k)
+        self._v[self.n:self.n + t] = self._store(v)
+        self.n += t
 
     def load_stored(self, k_values: np.ndarray, v_values: np.ndarray) -> None:
-        """Set the slot to already-stored values [T, H, hd] (dequantised)."""
-        self.k = [np.asarray(x, F64) for x in k_values]
-        self.v = [np.asarray(x, F64) for x in v_values]
+        """Set the slot to already-stored (dequantised) values [T, H, hd]."""
+        self._k = self._v = None
+        self.n = 0
+        self._reserve(k_values.shape[0] + 64, k_values.shape[1:])
+        self._k[:k_values.shape[0]] = k_values
+        self._v[:v_values.shape[0]] = v_values
+        self.n = k_values.shape[0]
+
+    @property
+    def k(self) -> np.ndarray:
+        return self._k[:self.n]
+
+    @property
+    def v(self) -> np.ndarray:
+        return self._v[:self.n]
 
     def __len__(self) -> int:
-        return len(self.k)
+        return self.n
 
 
 class LoopedModel:
@@ -379,9 +406,7 @@ class LoopedModel:
             q, k, v = blk.qkv(h, pos)
             slot = kv[layer]
             slot.append(k, v)
-            keys = np.stack(slot.k)          # [pos+1, H, hd]
-            vals = np.stack(slot.v)
-            h = blk.finish(h, causal_attention(q, keys, vals, pos))
+            h = blk.finish(h, causal_attention(q, slot.k, slot.v, pos))   # keys 0..pos
             if trace is not None:
                 trace.append(h.copy())
         return rmsnorm(h, self.gamma_final, self.cfg["eps"])[0]

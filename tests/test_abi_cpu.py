@@ -1,0 +1,137 @@
+"""The C-ABI library loads, exports every entry point the header declares, and
+its host-only logic (sizes, argument checks) behaves as documented.  No
+compute calls: these run without a GPU."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import weight_shared_looped_b200 as tl
+from oracle import tinyloop_oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(tl_[a-z0-9_]+)\s*\(", src))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert {"tl_pack_weights", "tl_block_create", "tl_prefill", "tl_decode_step"} <= names
+    for n in sorted(names):
+        assert hasattr(tl.lib, n), n
+
+
+def test_only_tl_symbols_exported():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", tl.LIB_PATH], capture_output=True,
+                         text=True).stdout
+    syms = [line.split()[-1] for line in out.splitlines() if line.strip()]
+    assert syms and all(s.startswith("tl_") or s.startswith("_") for s in syms), syms
+
+
+def test_abi_version():
+    assert tl.tl_abi_version() == 100
+
+
+@pytest.mark.parametrize("K", [64, 256, 2048, 8192, 10, 11, 4000])
+def test_words_per_row_matches_oracle(K):
+    assert tl.tl_packed_words_per_row(K, 3) == o.int3_words_per_row(K)
+    if K % 8 == 0:
+        assert tl.tl_packed_words_per_row(K, 4) == K // 8
+
+
+def test_packed_bytes_match_oracle_block_bytes():
+    d, f = 2048, 8192
+    for bits in (3, 4):
+        total = 0
+        for n, k in ((3 * d, d), (d, d), (f, d), (f, d), (d, f)):
+            c, s = tl.tl_packed_bytes(n, k, bits, 128)
+            total += c + s
+        assert total == o.packed_block_bytes(d, f, bits, 128)
+
+
+def test_kv_layer_bytes_match_pages_figures():
+    # 10 layers (2 pre-blocks + L=8), max_seq 2048, 16 heads x 128
+    fp16 = 10 * tl.tl_kv_layer_bytes(16, 128, 2048, tl.TL_KV_FP16)
+    int8 = 10 * tl.tl_kv_layer_bytes(16, 128, 2048, tl.TL_KV_INT8)
+    assert fp16 == o.kv_cache_bytes(10, 2048, 16, 128, "fp16")
+    assert int8 == o.kv_cache_bytes(10, 2048, 16, 128, "int8")
+    assert round(fp16 / 1e6, 1) == 167.8 and round(int8 / 1e6, 1) == 85.2
+
+
+@pytest.mark.parametrize("args,status", [
+    ((64, 128, 5, 64), tl.TL_ERR_UNSUPPORTED),     # bits
+    ((64, 128, 4, 32), tl.TL_ERR_UNSUPPORTED),     # group
+    ((64, 96, 4, 64), tl.TL_ERR_INVALID_ARG),      # K % group
+    ((0, 128, 4, 64), tl.TL_ERR_INVALID_ARG),      # empty N
+])
+def test_pack_rejects_before_launch(args, status):
+    n, k, bits, group = args
+    rc = tl.lib.tl_pack_weights(ctypes.c_void_p(16), n, k, bits, group, ctypes.c_void_p(16),
+                                ctypes.c_void_p(16), None)
+    assert rc == status
+    assert tl.lib.tl_last_error()
+
+
+def test_null_pointers_rejected():
+    assert tl.lib.tl_pack_weights(None, 8, 64, 4, 64, None, None, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_kv_quant_int8(None, 4, 128, None, None, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_kv_quant_int8(None, 0, 128, None, None, None) == tl.TL_OK   # empty: no-op
+    assert tl.lib.tl_kv_quant_int8(None, 4, 0, None, None, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_prefill(None, None, None, 1, 1, None, 0, None, None, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_sync_status(None, None) == tl.TL_ERR_INVALID_ARG
+
+
+def _desc(**over):
+    cfg = dict(d_model=256, n_heads=4, head_dim=64, ffn=768, bits=4, group=64, eps=1e-5,
+               rope_theta=1e4)
+    cfg.update(over)
+    ptrs = [16] * 12
+    return tl.BlockDesc(cfg["d_model"], cfg["n_heads"], cfg["head_dim"], cfg["ffn"], cfg["bits"],
+                        cfg["group"], cfg["eps"], cfg["rope_theta"], *ptrs)
+
+
+@pytest.mark.parametrize("over,status", [
+    ({"d_model": 200}, tl.TL_ERR_INVALID_ARG),
+    ({"head_dim": 96, "n_heads": 2, "d_model": 192}, tl.TL_ERR_INVALID_ARG),
+    ({"head_dim": 32, "n_heads": 8}, tl.TL_ERR_UNSUPPORTED),
+    ({"n_heads": 3}, tl.TL_ERR_INVALID_ARG),
+    ({"ffn": 700}, tl.TL_ERR_INVALID_ARG),
+    ({"bits": 2}, tl.TL_ERR_UNSUPPORTED),
+    ({"eps": 0.0}, tl.TL_ERR_INVALID_ARG),
+])
+def test_block_create_validation(over, status):
+    out = ctypes.c_void_p()
+    assert tl.lib.tl_block_create(ctypes.byref(_desc(**over)), ctypes.byref(out)) == status
+    assert not out.value
+
+
+def test_int4_block_wraps_without_device_work():
+    out = ctypes.c_void_p()
+    assert tl.lib.tl_block_create(ctypes.byref(_desc()), ctypes.byref(out)) == tl.TL_OK
+    assert out.value
+    assert tl.lib.tl_block_destroy(out) == tl.TL_OK
+
+
+def test_model_create_validation():
+    blk = ctypes.c_void_p()
+    assert tl.lib.tl_block_create(ctypes.byref(_desc()), ctypes.byref(blk)) == tl.TL_OK
+    bad = [dict(max_tokens=0), dict(max_lanes=9), dict(max_L=65), dict(max_ctx=4)]
+    for b in bad:
+        kw = dict(max_tokens=16, max_lanes=1, max_ctx=64, max_L=8)
+        kw.update(b)
+        d = tl.ModelDesc(None, 0, blk, None, 0, ctypes.c_void_p(16), kw["max_tokens"],
+                         kw["max_lanes"], kw["max_ctx"], kw["max_L"])
+        out = ctypes.c_void_p()
+        assert tl.lib.tl_model_create(ctypes.byref(d), ctypes.byref(out)) == tl.TL_ERR_INVALID_ARG
+    tl.lib.tl_block_destroy(blk)

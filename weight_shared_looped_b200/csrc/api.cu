@@ -1,0 +1,910 @@
+// C ABI of the looped-block library: argument checks, library-owned objects,
+// the loop driver and CUDA-graph replay.
+//
+// Forward order ("TinyLoop Framework", the four steps of the architectural
+// family): embed, the pre-blocks once each, the shared loop block L times with
+// the same weights (each application with its own KV slot, "Performance and
+// Memory", "KV cache INT8": 10 layers = 2 pre-blocks + L=8), final RMSNorm and
+// no output head.  L is an argument of every call ("Loop count is a runtime
+// knob"); the weights a model references do not depend on it.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <memory>
+#include <string>
+#include <tuple>
+#include <vector>
+#include <algorithm>
+
+#include "tl_internal.cuh"
+
+#define TL_API extern "C" __attribute__((visibility("default")))
+
+namespace tl {
+
+static thread_local std::string g_last_error;
+
+tl_status set_error(tl_status st, const char* fmt, ...) {
+  char buf[1024];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+tl_status ok() { return TL_OK; }
+
+static size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+static int words_per_row(int K, int bits) {
+  return bits == 4 ? K / 8 : ((K + 9) / 10 + 3) / 4 * 4;
+}
+
+static tl_status check_matrix(int N, int K, int bits, int group) {
+  TL_CHECK_ARG(N >= 1 && K >= 1, "matrix shape [%d, %d] must be positive", N, K);
+  if (bits != 3 && bits != 4)
+    return set_error(TL_ERR_UNSUPPORTED, "bits = %d: only 3 and 4 are supported", bits);
+  if (group != 64 && group != 128)
+    return set_error(TL_ERR_UNSUPPORTED, "group = %d: only 64 and 128 are supported", group);
+  TL_CHECK_ARG(K % group == 0, "K = %d is not a multiple of group %d", K, group);
+  TL_CHECK_ARG(bits != 4 || K % 8 == 0, "INT4 needs K %% 8 == 0 (K = %d)", K);
+  return ok();
+}
+
+}  // namespace tl
+
+using namespace tl;
+
+// ============================================================================
+// Objects
+// ============================================================================
+struct tl_block {
+  tl_block_desc d;
+  // INT4 canonical words the GEMM kernels read: the caller's words for an
+  // INT4 block, a library-owned INT4 copy of the same codes for an INT3 block.
+  const uint32_t* w4[5];
+  std::vector<void*> owned;
+};
+
+struct tl_kv {
+  const tl_model* model;
+  int n_lanes, max_ctx, dtype;
+  int L[kMaxLanes];
+  int pos[kMaxLanes];
+  char* buffer;
+  size_t layer_bytes, region_bytes;
+};
+
+struct GraphEntry {
+  cudaGraphExec_t exec = nullptr;
+  int32_t* lane_of_row = nullptr;   // device, decode graphs
+};
+
+struct tl_model {
+  tl_model_desc desc;
+  std::vector<const tl_block*> pre;
+  const tl_block* loop;
+  int d, H, hd, F, Tmax;
+  float eps;
+  bool graphs = true;
+  cudaStream_t cap_stream = nullptr;
+  // workspace
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  int32_t* ids;
+  __half* hin;
+  float* h;
+  __half* x;
+  __half* attn;
+  __half *q, *k, *v;
+  __half* u;
+  float* part;
+  float* y;
+  int32_t* lane_map;
+  float* dec_scratch;
+  int max_chunks;
+  int* status;
+  float2* rope;
+  std::map<std::string, GraphEntry> graphs_cache;
+};
+
+// ============================================================================
+// Misc
+// ============================================================================
+TL_API const char* tl_last_error(void) { return g_last_error.c_str(); }
+TL_API int tl_abi_version(void) { return 100; }
+
+// ============================================================================
+// Packing
+// ============================================================================
+TL_API tl_status tl_packed_words_per_row(int K, int bits, int* words) {
+  TL_CHECK_ARG(words != nullptr, "words is NULL");
+  TL_CHECK_ARG(K >= 1, "K = %d must be positive", K);
+  if (bits != 3 && bits != 4)
+    return set_error(TL_ERR_UNSUPPORTED, "bits = %d: only 3 and 4 are supported", bits);
+  TL_CHECK_ARG(bits != 4 || K % 8 == 0, "INT4 needs K %% 8 == 0 (K = %d)", K);
+  *words = words_per_row(K, bits);
+  return ok();
+}
+
+TL_API tl_status tl_packed_bytes(int N, int K, int bits, int group, size_t* code_bytes,
+                                 size_t* scale_bytes) {
+  TL_TRY(check_matrix(N, K, bits, group));
+  TL_CHECK_ARG(code_bytes && scale_bytes, "output pointer is NULL");
+  *code_bytes = (size_t)N * words_per_row(K, bits) * 4;
+  *scale_bytes = (size_t)N * (K / group) * 2;
+  return ok();
+}
+
+TL_API tl_status tl_pack_weights(const float* w, int N, int K, int bits, int group,
+                                 uint32_t* packed, uint16_t* scales, tl_stream stream) {
+  TL_TRY(check_matrix(N, K, bits, group));
+  TL_CHECK_ARG(w && packed && scales, "NULL device pointer");
+  return launch_pack(w, N, K, bits, group, packed, scales, (cudaStream_t)stream);
+}
+
+TL_API tl_status tl_unpack_codes(const uint32_t* packed, int N, int K, int bits, int8_t* codes,
+                                 tl_stream stream) {
+  TL_CHECK_ARG(packed && codes, "NULL device pointer");
+  TL_CHECK_ARG(N >= 1 && K >= 1, "matrix shape [%d, %d] must be positive", N, K);
+  if (bits != 3 && bits != 4)
+    return set_error(TL_ERR_UNSUPPORTED, "bits = %d: only 3 and 4 are supported", bits);
+  TL_CHECK_ARG(bits != 4 || K % 8 == 0, "INT4 needs K %% 8 == 0 (K = %d)", K);
+  return launch_unpack(packed, N, K, bits, codes, (cudaStream_t)stream);
+}
+
+TL_API tl_status tl_kv_quant_int8(const uint16_t* x, int rows, int hd, int8_t* codes,
+                                  uint16_t* scales, tl_stream stream) {
+  TL_CHECK_ARG(rows >= 0, "rows = %d must be >= 0", rows);
+  TL_CHECK_ARG(hd >= 1 && hd <= 256, "hd = %d must be in [1, 256]", hd);
+  if (rows == 0) return ok();
+  TL_CHECK_ARG(x && codes && scales, "NULL device pointer");
+  return launch_kv_quant_int8(reinterpret_cast<const __half*>(x), rows, hd, codes,
+                              reinterpret_cast<__half*>(scales), (cudaStream_t)stream);
+}
+
+// ============================================================================
+// Blocks
+// ============================================================================
+TL_API tl_status tl_block_create(const tl_block_desc* desc, tl_block** out) {
+  TL_CHECK_ARG(desc && out, "NULL argument");
+  *out = nullptr;
+  const tl_block_desc& d = *desc;
+  TL_CHECK_ARG(d.d_model >= 256 && d.d_model % 256 == 0 && d.d_model <= 8192,
+               "d_model = %d must be a multiple of 256 in [256, 8192]", d.d_model);
+  if (d.head_dim != 64 && d.head_dim != 128)
+    return set_error(TL_ERR_UNSUPPORTED, "head_dim = %d: only 64 and 128", d.head_dim);
+  TL_CHECK_ARG(d.n_heads * d.head_dim == d.d_model,
+               "n_heads * head_dim = %d must equal d_model = %d", d.n_heads * d.head_dim,
+               d.d_model);
+  TL_CHECK_ARG(d.ffn >= 128 && d.ffn % 128 == 0, "ffn = %d must be a multiple of 128", d.ffn);
+  TL_TRY(check_matrix(3 * d.d_model, d.d_model, d.bits, d.group));
+  TL_TRY(check_matrix(d.ffn, d.d_model, d.bits, d.group));
+  TL_TRY(check_matrix(d.d_model, d.ffn, d.bits, d.group));
+  TL_CHECK_ARG(d.eps > 0.f && std::isfinite(d.eps), "eps must be positive");
+  TL_CHECK_ARG(d.rope_theta > 1.f && std::isfinite(d.rope_theta), "rope_theta must be > 1");
+  TL_CHECK_ARG(d.w_qkv && d.s_qkv && d.w_o && d.s_o && d.w_gate && d.s_gate && d.w_up &&
+                   d.s_up && d.w_down && d.s_down && d.gamma_attn && d.gamma_ffn,
+               "NULL weight pointer in block description");
+  std::unique_ptr<tl_block> b(new tl_block());
+  b->d = d;
+  const uint32_t* src[5] = {d.w_qkv, d.w_o, d.w_gate, d.w_up, d.w_down};
+  const int Ns[5] = {3 * d.d_model, d.d_model, d.ffn, d.ffn, d.d_model};
+  const int Ks[5] = {d.d_model, d.d_model, d.d_model, d.d_model, d.ffn};
+  if (d.bits == 4) {
+    for (int i = 0; i < 5; ++i) b->w4[i] = src[i];
+  } else {
+    cudaStream_t s;
+    TL_CUDA(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
+    for (int i = 0; i < 5; ++i) {
+      void* p = nullptr;
+      if (cudaMalloc(&p, (size_t)Ns[i] * (Ks[i] / 8) * 4) != cudaSuccess) {
+        for (void* q : b->owned) cudaFree(q);
+        cudaStreamDestroy(s);
+        return set_error(TL_ERR_OOM, "cannot allocate the INT4 copy of an INT3 matrix");
+      }
+      b->owned.push_back(p);
+      tl_status st = launch_int3_to_int4(src[i], Ns[i], Ks[i], (uint32_t*)p, s);
+      if (st != TL_OK) {
+        for (void* q : b->owned) cudaFree(q);
+        cudaStreamDestroy(s);
+        return st;
+      }
+      b->w4[i] = (const uint32_t*)p;
+    }
+    cudaError_t e = cudaStreamSynchronize(s);
+    cudaStreamDestroy(s);
+    if (e != cudaSuccess) {
+      for (void* q : b->owned) cudaFree(q);
+      return set_error(TL_ERR_CUDA, "INT3 conversion failed: %s", cudaGetErrorString(e));
+    }
+  }
+  *out = b.release();
+  return ok();
+}
+
+TL_API tl_status tl_block_destroy(tl_block* block) {
+  if (!block) return ok();
+  for (void* p : block->owned) cudaFree(p);
+  delete block;
+  return ok();
+}
+
+// ============================================================================
+// Models
+// ============================================================================
+namespace {
+
+struct GemmShape {
+  int N, K;
+};
+
+size_t part_floats(const tl_model* m, int T) {
+  const GemmShape gs[4] = {{3 * m->d, m->d}, {m->d, m->d}, {2 * m->F, m->d}, {m->d, m->F}};
+  size_t best = 0;
+  for (auto& g : gs) best = std::max(best, (size_t)gemm_splits(g.N, g.K, T) * T * g.N);
+  return best;
+}
+
+void free_graphs(tl_model* m) {
+  for (auto& kv : m->graphs_cache) {
+    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
+    if (kv.second.lane_of_row) cudaFree(kv.second.lane_of_row);
+  }
+  m->graphs_cache.clear();
+}
+
+}  // namespace
+
+TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
+  TL_CHECK_ARG(desc && out, "NULL argument");
+  *out = nullptr;
+  const tl_model_desc& md = *desc;
+  TL_CHECK_ARG(md.loop != nullptr, "loop block is NULL");
+  TL_CHECK_ARG(md.n_pre >= 0 && md.n_pre <= 16, "n_pre = %d must be in [0, 16]", md.n_pre);
+  TL_CHECK_ARG(md.n_pre == 0 || md.pre != nullptr, "pre is NULL");
+  TL_CHECK_ARG(md.gamma_final != nullptr, "gamma_final is NULL");
+  TL_CHECK_ARG(md.max_tokens >= 1 && md.max_tokens <= 8192, "max_tokens = %d out of [1, 8192]",
+               md.max_tokens);
+  TL_CHECK_ARG(md.max_lanes >= 1 && md.max_lanes <= kMaxLanes, "max_lanes = %d out of [1, %d]",
+               md.max_lanes, kMaxLanes);
+  TL_CHECK_ARG(md.max_ctx >= md.max_tokens && md.max_ctx <= 65536,
+               "max_ctx = %d must be in [max_tokens, 65536]", md.max_ctx);
+  TL_CHECK_ARG(md.max_L >= 1 && md.max_L <= kMaxL, "max_L = %d out of [1, %d]", md.max_L, kMaxL);
+  TL_CHECK_ARG(md.embed == nullptr || md.vocab >= 1, "vocab must be >= 1 with an embedding");
+  const tl_block_desc& ld = md.loop->d;
+  for (int i = 0; i < md.n_pre; ++i) {
+    TL_CHECK_ARG(md.pre[i] != nullptr, "pre[%d] is NULL", i);
+    const tl_block_desc& pd = md.pre[i]->d;
+    TL_CHECK_ARG(pd.d_model == ld.d_model && pd.n_heads == ld.n_heads &&
+                     pd.head_dim == ld.head_dim && pd.ffn == ld.ffn && pd.eps == ld.eps &&
+                     pd.rope_theta == ld.rope_theta,
+                 "pre[%d] shape differs from the loop block", i);
+  }
+  std::unique_ptr<tl_model> m(new tl_model());
+  m->desc = md;
+  for (int i = 0; i < md.n_pre; ++i) m->pre.push_back(md.pre[i]);
+  m->loop = md.loop;
+  m->d = ld.d_model;
+  m->H = ld.n_heads;
+  m->hd = ld.head_dim;
+  m->F = ld.ffn;
+  m->eps = ld.eps;
+  m->Tmax = std::max(md.max_tokens, md.max_lanes);
+  m->max_chunks = (md.max_ctx + kDecodeChunk - 1) / kDecodeChunk;
+  const int T = m->Tmax, d = m->d, F = m->F;
+  size_t maxpart = 0;
+  for (int t = 1; t <= T; ++t) maxpart = std::max(maxpart, part_floats(m.get(), t));
+  // workspace layout
+  struct Slot {
+    void** ptr;
+    size_t bytes;
+  };
+  void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
+  void* p_u; void* p_part; void* p_y; void* p_lid; void* p_dec; void* p_status; void* p_rope;
+  Slot slots[] = {
+      {&p_ids, (size_t)T * 4},
+      {&p_hin, (size_t)T * d * 2},
+      {&p_h, (size_t)T * d * 4},
+      {&p_x, (size_t)T * d * 2},
+      {&p_attn, (size_t)T * d * 2},
+      {&p_q, (size_t)T * d * 2},
+      {&p_k, (size_t)T * d * 2},
+      {&p_v, (size_t)T * d * 2},
+      {&p_u, (size_t)T * F * 2},
+      {&p_part, maxpart * 4},
+      {&p_y, (size_t)T * d * 4},
+      {&p_lid, (size_t)kMaxLanes * 4},
+      {&p_dec, (size_t)kMaxLanes * m->H * m->max_chunks * (m->hd + 2) * 4},
+      {&p_status, 256},
+      {&p_rope, (size_t)md.max_ctx * (m->hd / 2) * sizeof(float2)},
+  };
+  size_t total = 0;
+  for (auto& s : slots) total += align256(s.bytes);
+  if (cudaMalloc(&m->ws, total) != cudaSuccess)
+    return set_error(TL_ERR_OOM, "cannot allocate %zu bytes of model workspace", total);
+  m->ws_bytes = total;
+  char* base = (char*)m->ws;
+  for (auto& s : slots) {
+    *s.ptr = base;
+    base += align256(s.bytes);
+  }
+  m->ids = (int32_t*)p_ids;
+  m->hin = (__half*)p_hin;
+  m->h = (float*)p_h;
+  m->x = (__half*)p_x;
+  m->attn = (__half*)p_attn;
+  m->q = (__half*)p_q;
+  m->k = (__half*)p_k;
+  m->v = (__half*)p_v;
+  m->u = (__half*)p_u;
+  m->part = (float*)p_part;
+  m->y = (float*)p_y;
+  m->lane_map = (int32_t*)p_lid;
+  m->dec_scratch = (float*)p_dec;
+  m->status = (int*)p_status;
+  m->rope = (float2*)p_rope;
+  // RoPE table: angle = pos * theta^(-2i/hd), computed in double, rounded to fp32
+  {
+    const int half = m->hd / 2;
+    std::vector<float2> tab((size_t)md.max_ctx * half);
+    for (int p = 0; p < md.max_ctx; ++p)
+      for (int i = 0; i < half; ++i) {
+        double inv = std::pow((double)ld.rope_theta, -2.0 * i / m->hd);
+        double a = (double)p * inv;
+        tab[(size_t)p * half + i] = make_float2((float)std::cos(a), (float)std::sin(a));
+      }
+    int32_t ident[kMaxLanes];
+    for (int i = 0; i < kMaxLanes; ++i) ident[i] = i;
+    cudaError_t e1 = cudaMemcpy(m->rope, tab.data(), tab.size() * sizeof(float2),
+                                cudaMemcpyHostToDevice);
+    cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
+    cudaError_t e3 = cudaMemset(m->status, 0, 256);
+    if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
+      cudaFree(m->ws);
+      return set_error(TL_ERR_CUDA, "model initialisation copy failed");
+    }
+  }
+  if (cudaStreamCreateWithFlags(&m->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaFree(m->ws);
+    return set_error(TL_ERR_CUDA, "cannot create the capture stream");
+  }
+  *out = m.release();
+  return ok();
+}
+
+TL_API tl_status tl_model_destroy(tl_model* model) {
+  if (!model) return ok();
+  free_graphs(model);
+  if (model->cap_stream) cudaStreamDestroy(model->cap_stream);
+  if (model->ws) cudaFree(model->ws);
+  delete model;
+  return ok();
+}
+
+TL_API tl_status tl_model_device_bytes(const tl_model* model, size_t* bytes) {
+  TL_CHECK_ARG(model && bytes, "NULL argument");
+  *bytes = model->ws_bytes;
+  return ok();
+}
+
+TL_API tl_status tl_model_set_graphs(tl_model* model, int enable) {
+  TL_CHECK_ARG(model, "NULL model");
+  model->graphs = enable != 0;
+  if (!model->graphs) free_graphs(model);
+  return ok();
+}
+
+// ============================================================================
+// KV cache
+// ============================================================================
+namespace {
+
+void kv_geometry_hd(int H, int hd, int max_ctx, int dtype, size_t* layer, size_t* region) {
+  size_t esz = dtype == TL_KV_INT8 ? 1 : 2;
+  size_t r = align256((size_t)H * max_ctx * hd * esz);
+  size_t l = 2 * r;
+  if (dtype == TL_KV_INT8) l += 2 * align256((size_t)H * max_ctx * 2);
+  *layer = l;
+  *region = r;
+}
+
+void kv_geometry(const tl_model* m, int max_ctx, int dtype, size_t* layer, size_t* region) {
+  kv_geometry_hd(m->H, m->hd, max_ctx, dtype, layer, region);
+}
+
+tl_status check_kv_args(const tl_model* m, int n_lanes, int max_ctx, const int* L, int dtype) {
+  TL_CHECK_ARG(m, "NULL model");
+  TL_CHECK_ARG(n_lanes >= 1 && n_lanes <= kMaxLanes, "n_lanes = %d out of [1, %d]", n_lanes,
+               kMaxLanes);
+  TL_CHECK_ARG(max_ctx >= 1 && max_ctx <= m->desc.max_ctx,
+               "max_ctx = %d out of [1, model max_ctx %d]", max_ctx, m->desc.max_ctx);
+  TL_CHECK_ARG(L != nullptr, "L_per_lane is NULL");
+  for (int b = 0; b < n_lanes; ++b)
+    TL_CHECK_ARG(L[b] >= 1 && L[b] <= m->desc.max_L, "L_per_lane[%d] = %d out of [1, %d]", b,
+                 L[b], m->desc.max_L);
+  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8, "unknown KV dtype %d", dtype);
+  return ok();
+}
+
+}  // namespace
+
+TL_API tl_status tl_kv_layer_bytes(int n_heads, int head_dim, int max_ctx, tl_kv_dtype dtype,
+                                   size_t* bytes) {
+  TL_CHECK_ARG(bytes, "bytes is NULL");
+  TL_CHECK_ARG(n_heads >= 1 && head_dim >= 1 && max_ctx >= 1, "sizes must be positive");
+  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8, "unknown KV dtype %d", dtype);
+  size_t region;
+  kv_geometry_hd(n_heads, head_dim, max_ctx, dtype, bytes, &region);
+  return ok();
+}
+
+TL_API tl_status tl_kv_bytes(const tl_model* model, int n_lanes, int max_ctx,
+                             const int* L_per_lane, tl_kv_dtype dtype, size_t* bytes) {
+  TL_TRY(check_kv_args(model, n_lanes, max_ctx, L_per_lane, dtype));
+  TL_CHECK_ARG(bytes, "bytes is NULL");
+  size_t layer, region;
+  kv_geometry(model, max_ctx, dtype, &layer, &region);
+  size_t layers = 0;
+  for (int b = 0; b < n_lanes; ++b) layers += (size_t)model->desc.n_pre + L_per_lane[b];
+  *bytes = kKvHeaderBytes + layers * layer;
+  return ok();
+}
+
+TL_API tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
+                              const int* L_per_lane, tl_kv_dtype dtype, void* buffer,
+                              size_t buffer_bytes, tl_kv** out) {
+  TL_CHECK_ARG(out, "out is NULL");
+  *out = nullptr;
+  size_t need = 0;
+  TL_TRY(tl_kv_bytes(model, n_lanes, max_ctx, L_per_lane, dtype, &need));
+  TL_CHECK_ARG(buffer != nullptr, "buffer is NULL");
+  TL_CHECK_ARG(((uintptr_t)buffer & 255) == 0, "buffer must be 256-byte aligned");
+  TL_CHECK_ARG(buffer_bytes >= need, "buffer has %zu bytes, %zu needed", buffer_bytes, need);
+  std::unique_ptr<tl_kv> kv(new tl_kv());
+  kv->model = model;
+  kv->n_lanes = n_lanes;
+  kv->max_ctx = max_ctx;
+  kv->dtype = dtype;
+  kv->buffer = (char*)buffer;
+  kv_geometry(model, max_ctx, dtype, &kv->layer_bytes, &kv->region_bytes);
+  KvHeader hdr;
+  memset(&hdr, 0, sizeof(hdr));
+  int cum = 0;
+  for (int b = 0; b < kMaxLanes; ++b) {
+    kv->L[b] = b < n_lanes ? L_per_lane[b] : 0;
+    kv->pos[b] = 0;
+    hdr.cum_layers[b] = cum;
+    if (b < n_lanes) cum += model->desc.n_pre + L_per_lane[b];
+  }
+  TL_CUDA(cudaMemcpy(buffer, &hdr, sizeof(hdr), cudaMemcpyHostToDevice));
+  *out = kv.release();
+  return ok();
+}
+
+TL_API tl_status tl_kv_destroy(tl_kv* kv) {
+  delete kv;
+  return ok();
+}
+
+TL_API tl_status tl_kv_reset(tl_kv* kv, int lane, tl_stream stream) {
+  TL_CHECK_ARG(kv, "NULL kv");
+  TL_CHECK_ARG(lane >= -1 && lane < kv->n_lanes, "lane = %d out of [-1, %d)", lane, kv->n_lanes);
+  TL_TRY(launch_set_pos((KvHeader*)kv->buffer, lane, 0, (cudaStream_t)stream));
+  for (int b = 0; b < kv->n_lanes; ++b)
+    if (lane < 0 || b == lane) kv->pos[b] = 0;
+  return ok();
+}
+
+TL_API tl_status tl_kv_position(const tl_kv* kv, int lane, int* pos) {
+  TL_CHECK_ARG(kv && pos, "NULL argument");
+  TL_CHECK_ARG(lane >= 0 && lane < kv->n_lanes, "lane = %d out of [0, %d)", lane, kv->n_lanes);
+  *pos = kv->pos[lane];
+  return ok();
+}
+
+TL_API tl_status tl_kv_set_position(tl_kv* kv, int lane, int pos, tl_stream stream) {
+  TL_CHECK_ARG(kv, "NULL kv");
+  TL_CHECK_ARG(lane >= 0 && lane < kv->n_lanes, "lane = %d out of [0, %d)", lane, kv->n_lanes);
+  TL_CHECK_ARG(pos >= 0 && pos <= kv->max_ctx, "pos = %d out of [0, %d]", pos, kv->max_ctx);
+  TL_TRY(launch_set_pos((KvHeader*)kv->buffer, lane, pos, (cudaStream_t)stream));
+  kv->pos[lane] = pos;
+  return ok();
+}
+
+TL_API tl_status tl_kv_layer_ptrs(const tl_kv* kv, int lane, int layer, void** k, void** v,
+                                  uint16_t** k_scale, uint16_t** v_scale) {
+  TL_CHECK_ARG(kv && k && v && k_scale && v_scale, "NULL argument");
+  TL_CHECK_ARG(lane >= 0 && lane < kv->n_lanes, "lane = %d out of [0, %d)", lane, kv->n_lanes);
+  const int layers = kv->model->desc.n_pre + kv->L[lane];
+  TL_CHECK_ARG(layer >= 0 && layer < layers, "layer = %d out of [0, %d)", layer, layers);
+  int cum = 0;
+  for (int b = 0; b < lane; ++b) cum += kv->model->desc.n_pre + kv->L[b];
+  char* base = kv->buffer + kKvHeaderBytes + (size_t)(cum + layer) * kv->layer_bytes;
+  *k = base;
+  *v = base + kv->region_bytes;
+  if (kv->dtype == TL_KV_INT8) {
+    size_t sreg = (kv->layer_bytes - 2 * kv->region_bytes) / 2;
+    *k_scale = (uint16_t*)(base + 2 * kv->region_bytes);
+    *v_scale = (uint16_t*)(base + 2 * kv->region_bytes + sreg);
+  } else {
+    *k_scale = nullptr;
+    *v_scale = nullptr;
+  }
+  return ok();
+}
+
+// ============================================================================
+// Loop driver
+// ============================================================================
+namespace {
+
+const tl_block* block_at(const tl_model* m, int layer) {
+  return layer < (int)m->pre.size() ? m->pre[layer] : m->loop;
+}
+
+GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half* x, int T) {
+  const tl_block_desc& d = b->d;
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.G = d.group;
+  a.x = x;
+  a.T = T;
+  a.part = m->part;
+  switch (which) {
+    case 0:  // QKV
+      a.w0 = a.w1 = b->w4[0];
+      a.s0 = a.s1 = (const __half*)d.s_qkv;
+      a.N = a.n_split = 3 * m->d;
+      a.K = m->d;
+      break;
+    case 1:  // O
+      a.w0 = a.w1 = b->w4[1];
+      a.s0 = a.s1 = (const __half*)d.s_o;
+      a.N = a.n_split = m->d;
+      a.K = m->d;
+      break;
+    case 2:  // gate | up
+      a.w0 = b->w4[2];
+      a.s0 = (const __half*)d.s_gate;
+      a.w1 = b->w4[3];
+      a.s1 = (const __half*)d.s_up;
+      a.n_split = m->F;
+      a.N = 2 * m->F;
+      a.K = m->d;
+      break;
+    default:  // down
+      a.w0 = a.w1 = b->w4[4];
+      a.s0 = a.s1 = (const __half*)d.s_down;
+      a.N = a.n_split = m->d;
+      a.K = m->F;
+      break;
+  }
+  a.splits = gemm_splits(a.N, a.K, T);
+  return a;
+}
+
+NormArgs norm_args(const tl_model* m, int rows) {
+  NormArgs n;
+  memset(&n, 0, sizeof(n));
+  n.h = m->h;
+  n.d = m->d;
+  n.rows = rows;
+  n.x = m->x;
+  n.y = m->y;
+  n.eps = m->eps;
+  n.status = m->status;
+  return n;
+}
+
+// One block application (everything after the input RMSNorm, up to and
+// including the down projection; the residual add of the down projection is
+// done by the next norm).  `rows` rows are active.
+tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
+                             int lane, bool decode, const int32_t* lane_of_row, cudaStream_t s) {
+  // QKV
+  GemmArgs g = gemm_args(m, b, 0, m->x, rows);
+  TL_TRY(launch_gemm(g, s));
+  RopeKvArgs r;
+  memset(&r, 0, sizeof(r));
+  r.part = m->part;
+  r.S = g.splits;
+  r.rows = rows;
+  r.d = m->d;
+  r.H = m->H;
+  r.hd = m->hd;
+  r.rope_cs = m->rope;
+  r.q = m->q;
+  r.k = decode ? nullptr : m->k;
+  r.v = decode ? nullptr : m->v;
+  if (kv) {
+    r.kv_base = kv->buffer + kKvHeaderBytes;
+    r.hdr = (const KvHeader*)kv->buffer;
+    r.layer_bytes = kv->layer_bytes;
+    r.kv_region_bytes = kv->region_bytes;
+    r.layer = layer;
+    r.max_ctx = kv->max_ctx;
+    r.kv_int8 = kv->dtype == TL_KV_INT8;
+  }
+  r.lane_of_row = lane_of_row;
+  r.lane = lane;
+  r.decode = decode ? 1 : 0;
+  TL_TRY(launch_rope_kv(r, s));
+  // attention
+  if (!decode) {
+    TL_TRY(launch_attn_prefill(m->q, m->k, m->v, m->attn, rows, m->H, m->hd, s));
+  } else {
+    DecodeAttnArgs da;
+    memset(&da, 0, sizeof(da));
+    da.q = m->q;
+    da.out = m->attn;
+    da.rows = rows;
+    da.H = m->H;
+    da.hd = m->hd;
+    da.d = m->d;
+    da.kv_base = kv->buffer + kKvHeaderBytes;
+    da.hdr = (const KvHeader*)kv->buffer;
+    da.layer_bytes = kv->layer_bytes;
+    da.kv_region_bytes = kv->region_bytes;
+    da.layer = layer;
+    da.max_ctx = kv->max_ctx;
+    da.kv_int8 = kv->dtype == TL_KV_INT8;
+    da.lane_of_row = lane_of_row;
+    da.scratch = m->dec_scratch;
+    da.max_chunks = (kv->max_ctx + kDecodeChunk - 1) / kDecodeChunk;
+    TL_TRY(launch_attn_decode(da, s));
+  }
+  // O projection, residual, RMSNorm before the MLP
+  g = gemm_args(m, b, 1, m->attn, rows);
+  TL_TRY(launch_gemm(g, s));
+  NormArgs n = norm_args(m, rows);
+  n.part = m->part;
+  n.part_rows = rows;
+  n.S = g.splits;
+  n.n_add = rows;
+  n.gamma_next = b->d.gamma_ffn;
+  n.n_next = rows;
+  n.out_row = lane_of_row;
+  TL_TRY(launch_residual_norm(n, s));
+  // SwiGLU MLP
+  g = gemm_args(m, b, 2, m->x, rows);
+  TL_TRY(launch_gemm(g, s));
+  TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
+  g = gemm_args(m, b, 3, m->u, rows);
+  TL_TRY(launch_gemm(g, s));
+  return ok();
+}
+
+tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, int lane,
+                          float* trace, cudaStream_t s) {
+  const int n_layers = (int)m->pre.size() + L;
+  EmbedArgs e;
+  memset(&e, 0, sizeof(e));
+  e.ids = use_ids ? m->ids : nullptr;
+  e.h_in = m->hin;
+  e.embed = (const __half*)m->desc.embed;
+  e.vocab = m->desc.vocab;
+  e.d = m->d;
+  e.rows = seq;
+  e.h = m->h;
+  e.status = m->status;
+  TL_TRY(launch_embed(e, s));
+  NormArgs n = norm_args(m, seq);
+  n.gamma_next = block_at(m, 0)->d.gamma_attn;
+  n.n_next = seq;
+  TL_TRY(launch_residual_norm(n, s));
+  for (int layer = 0; layer < n_layers; ++layer) {
+    const tl_block* b = block_at(m, layer);
+    TL_TRY(enqueue_block_body(m, b, layer, seq, kv, lane, false, nullptr, s));
+    NormArgs en = norm_args(m, seq);
+    en.part = m->part;
+    en.part_rows = seq;
+    en.S = gemm_splits(m->d, m->F, seq);
+    en.n_add = seq;
+    if (layer + 1 < n_layers) {
+      en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
+      en.n_next = seq;
+    } else {
+      en.gamma_final = m->desc.gamma_final;
+      en.fin_lo = 0;
+      en.fin_hi = seq;
+    }
+    if (trace) en.trace = trace + (size_t)layer * seq * m->d;
+    TL_TRY(launch_residual_norm(en, s));
+  }
+  if (kv) TL_TRY(launch_set_pos((KvHeader*)kv->buffer, lane, seq, s));
+  return ok();
+}
+
+// rows are lanes sorted by L descending; active rows at loop iteration i are
+// those with L > i (a prefix).
+tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int* L_sorted,
+                         const int32_t* lane_of_row, float* trace, cudaStream_t s) {
+  const int n_pre = (int)m->pre.size();
+  const int Lmax = L_sorted[0];
+  const int n_layers = n_pre + Lmax;
+  auto active = [&](int layer) {
+    if (layer < n_pre) return B;
+    int it = layer - n_pre, c = 0;
+    for (int i = 0; i < B; ++i) c += L_sorted[i] > it;
+    return c;
+  };
+  EmbedArgs e;
+  memset(&e, 0, sizeof(e));
+  e.ids = use_ids ? m->ids : nullptr;
+  e.h_in = m->hin;
+  e.embed = (const __half*)m->desc.embed;
+  e.vocab = m->desc.vocab;
+  e.d = m->d;
+  e.rows = B;
+  e.src_row = lane_of_row;
+  e.h = m->h;
+  e.status = m->status;
+  TL_TRY(launch_embed(e, s));
+  NormArgs n = norm_args(m, B);
+  n.gamma_next = block_at(m, 0)->d.gamma_attn;
+  n.n_next = B;
+  n.out_row = lane_of_row;
+  TL_TRY(launch_residual_norm(n, s));
+  for (int layer = 0; layer < n_layers; ++layer) {
+    const int act = active(layer);
+    const tl_block* b = block_at(m, layer);
+    TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, s));
+    const int nxt = layer + 1 < n_layers ? active(layer + 1) : 0;
+    NormArgs en = norm_args(m, trace ? B : act);
+    en.part = m->part;
+    en.part_rows = act;
+    en.S = gemm_splits(m->d, m->F, act);
+    en.n_add = act;
+    en.n_next = nxt;
+    if (nxt > 0) en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
+    en.gamma_final = m->desc.gamma_final;
+    en.fin_lo = nxt;
+    en.fin_hi = act;
+    en.out_row = lane_of_row;
+    if (trace) en.trace = trace + (size_t)layer * B * m->d;
+    TL_TRY(launch_residual_norm(en, s));
+  }
+  TL_TRY(launch_advance_pos((KvHeader*)kv->buffer, B, s));
+  return ok();
+}
+
+template <typename F>
+tl_status run_graph(tl_model* m, const std::string& key, cudaStream_t stream, F&& enqueue,
+                    GraphEntry** entry_out = nullptr, const int32_t* lane_map = nullptr) {
+  if (!m->graphs) return enqueue(stream, nullptr);
+  auto it = m->graphs_cache.find(key);
+  if (it == m->graphs_cache.end()) {
+    if (m->graphs_cache.size() >= 64) free_graphs(m);
+    GraphEntry ge;
+    if (lane_map) {
+      if (cudaMalloc(&ge.lane_of_row, kMaxLanes * 4) != cudaSuccess)
+        return set_error(TL_ERR_OOM, "cannot allocate a graph lane map");
+      if (cudaMemcpy(ge.lane_of_row, lane_map, kMaxLanes * 4, cudaMemcpyHostToDevice) !=
+          cudaSuccess) {
+        cudaFree(ge.lane_of_row);
+        return set_error(TL_ERR_CUDA, "cannot upload a graph lane map");
+      }
+    }
+    TL_CUDA(cudaStreamBeginCapture(m->cap_stream, cudaStreamCaptureModeThreadLocal));
+    tl_status st = enqueue(m->cap_stream, ge.lane_of_row);
+    cudaGraph_t graph = nullptr;
+    cudaError_t ce = cudaStreamEndCapture(m->cap_stream, &graph);
+    if (st != TL_OK || ce != cudaSuccess) {
+      if (graph) cudaGraphDestroy(graph);
+      if (ge.lane_of_row) cudaFree(ge.lane_of_row);
+      if (st != TL_OK) return st;
+      return set_error(TL_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(ce));
+    }
+    ce = cudaGraphInstantiate(&ge.exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (ce != cudaSuccess) {
+      if (ge.lane_of_row) cudaFree(ge.lane_of_row);
+      return set_error(TL_ERR_CUDA, "graph instantiation failed: %s", cudaGetErrorString(ce));
+    }
+    it = m->graphs_cache.emplace(key, ge).first;
+  }
+  TL_CUDA(cudaGraphLaunch(it->second.exec, stream));
+  if (entry_out) *entry_out = &it->second;
+  return ok();
+}
+
+}  // namespace
+
+TL_API tl_status tl_prefill(tl_model* model, const int32_t* ids, const uint16_t* h_in, int seq,
+                            int L, tl_kv* kv, int lane, float* y_out, float* h_trace,
+                            tl_stream stream) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG((ids == nullptr) != (h_in == nullptr), "give exactly one of ids and h_in");
+  TL_CHECK_ARG(ids == nullptr || model->desc.embed != nullptr, "ids given but no embedding");
+  TL_CHECK_ARG(seq >= 1 && seq <= model->desc.max_tokens, "seq = %d out of [1, %d]", seq,
+               model->desc.max_tokens);
+  TL_CHECK_ARG(L >= 1 && L <= model->desc.max_L, "L = %d out of [1, %d]", L, model->desc.max_L);
+  TL_CHECK_ARG(y_out != nullptr, "y_out is NULL");
+  if (kv) {
+    TL_CHECK_ARG(kv->model == model, "kv was created for another model");
+    TL_CHECK_ARG(lane >= 0 && lane < kv->n_lanes, "lane = %d out of [0, %d)", lane, kv->n_lanes);
+    TL_CHECK_ARG(L <= kv->L[lane], "L = %d exceeds the %d loop slots of lane %d", L, kv->L[lane],
+                 lane);
+    TL_CHECK_ARG(seq <= kv->max_ctx, "seq = %d exceeds the cache context %d", seq, kv->max_ctx);
+  }
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = model->d;
+  if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)seq * 4, cudaMemcpyDefault, s));
+  else TL_CUDA(cudaMemcpyAsync(model->hin, h_in, (size_t)seq * d * 2, cudaMemcpyDefault, s));
+  char key[256];
+  snprintf(key, sizeof(key), "P|%d|%d|%p|%d|%d|%p", seq, L, (void*)kv, lane, ids ? 1 : 0,
+           (void*)h_trace);
+  const bool use_ids = ids != nullptr;
+  TL_TRY(run_graph(model, key, s, [&](cudaStream_t cs, int32_t*) {
+    return enqueue_prefill(model, use_ids, seq, L, kv, lane, h_trace, cs);
+  }));
+  TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)seq * d * 4, cudaMemcpyDefault, s));
+  if (kv) kv->pos[lane] = seq;
+  return ok();
+}
+
+TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
+                                const uint16_t* h_in, const int* L_per_lane, int n_lanes,
+                                float* y_out, float* h_trace, tl_stream stream) {
+  TL_CHECK_ARG(model && kv, "NULL model or kv");
+  TL_CHECK_ARG(kv->model == model, "kv was created for another model");
+  TL_CHECK_ARG((ids == nullptr) != (h_in == nullptr), "give exactly one of ids and h_in");
+  TL_CHECK_ARG(ids == nullptr || model->desc.embed != nullptr, "ids given but no embedding");
+  TL_CHECK_ARG(n_lanes >= 1 && n_lanes <= kv->n_lanes && n_lanes <= model->desc.max_lanes,
+               "n_lanes = %d out of [1, %d]", n_lanes, std::min(kv->n_lanes, model->desc.max_lanes));
+  TL_CHECK_ARG(L_per_lane != nullptr && y_out != nullptr, "NULL L_per_lane or y_out");
+  for (int b = 0; b < n_lanes; ++b) {
+    TL_CHECK_ARG(L_per_lane[b] >= 1 && L_per_lane[b] <= kv->L[b],
+                 "L_per_lane[%d] = %d out of [1, %d]", b, L_per_lane[b], kv->L[b]);
+    TL_CHECK_ARG(kv->pos[b] + 1 <= kv->max_ctx, "lane %d is full (%d of %d positions)", b,
+                 kv->pos[b], kv->max_ctx);
+  }
+  // sort lanes by L, descending and stable
+  int32_t order[kMaxLanes];
+  for (int b = 0; b < kMaxLanes; ++b) order[b] = b < n_lanes ? b : 0;
+  std::stable_sort(order, order + n_lanes,
+                   [&](int a, int b) { return L_per_lane[a] > L_per_lane[b]; });
+  int L_sorted[kMaxLanes];
+  for (int i = 0; i < n_lanes; ++i) L_sorted[i] = L_per_lane[order[i]];
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = model->d;
+  if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)n_lanes * 4, cudaMemcpyDefault, s));
+  else TL_CUDA(cudaMemcpyAsync(model->hin, h_in, (size_t)n_lanes * d * 2, cudaMemcpyDefault, s));
+  std::string key = "D|" + std::to_string((uintptr_t)kv) + "|" + std::to_string(n_lanes) + "|" +
+                    std::to_string(ids ? 1 : 0) + "|" + std::to_string((uintptr_t)h_trace);
+  for (int b = 0; b < n_lanes; ++b) key += "|" + std::to_string(L_per_lane[b]);
+  const bool use_ids = ids != nullptr;
+  if (model->graphs) {
+    TL_TRY(run_graph(
+        model, key, s,
+        [&](cudaStream_t cs, int32_t* lmap) {
+          return enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, lmap, h_trace, cs);
+        },
+        nullptr, order));
+  } else {
+    // without graphs the lane map lives in the model workspace
+    TL_CUDA(cudaMemcpyAsync(model->lane_map, order, sizeof(order), cudaMemcpyHostToDevice, s));
+    TL_TRY(enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, model->lane_map, h_trace, s));
+  }
+  TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)n_lanes * d * 4, cudaMemcpyDefault, s));
+  for (int b = 0; b < n_lanes; ++b) kv->pos[b] += 1;
+  return ok();
+}
+
+TL_API tl_status tl_sync_status(tl_model* model, tl_stream stream) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+  int code = 0;
+  TL_CUDA(cudaMemcpy(&code, model->status, 4, cudaMemcpyDeviceToHost));
+  TL_CUDA(cudaMemset(model->status, 0, 4));
+  if (code == 0) return ok();
+  if (code == TL_ERR_TIMEOUT) return set_error(TL_ERR_TIMEOUT, "a bounded device wait ran out");
+  if (code == TL_ERR_NUMERIC) return set_error(TL_ERR_NUMERIC, "a non-finite value reached an output");
+  if (code == TL_ERR_INVALID_ARG) return set_error(TL_ERR_INVALID_ARG, "a token id was out of range");
+  return set_error((tl_status)code, "device status %d", code);
+}

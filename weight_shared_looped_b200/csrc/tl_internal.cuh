@@ -1,0 +1,154 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+
+#include "../../include/tl.h"
+
+namespace tl {
+
+// ---------------------------------------------------------------- errors
+tl_status set_error(tl_status st, const char* fmt, ...);
+tl_status ok();
+
+#define TL_CHECK_ARG(cond, ...)                                   \
+  do {                                                            \
+    if (!(cond)) return ::tl::set_error(TL_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define TL_CUDA(call)                                                         \
+  do {                                                                        \
+    cudaError_t e_ = (call);                                                  \
+    if (e_ != cudaSuccess)                                                    \
+      return ::tl::set_error(TL_ERR_CUDA, "%s failed: %s (%s:%d)", #call,    \
+                             cudaGetErrorString(e_), __FILE__, __LINE__);    \
+  } while (0)
+
+#define TL_LAUNCH_CHECK() TL_CUDA(cudaGetLastError())
+
+#define TL_TRY(expr)                         \
+  do {                                       \
+    tl_status s_ = (expr);                   \
+    if (s_ != TL_OK) return s_;              \
+  } while (0)
+
+// ---------------------------------------------------------------- limits
+constexpr int kMaxLanes = 8;
+constexpr int kMaxL = 64;
+constexpr int kMaxLayers = 16 + kMaxL;   // pre-blocks + loop iterations
+constexpr int kKvHeaderBytes = 4096;
+constexpr int kDecodeChunk = 64;         // keys per decode-attention split (fixed by position)
+
+// Device status codes written by kernels (same numbers as tl_status).
+constexpr int kDevTimeout = TL_ERR_TIMEOUT;
+constexpr int kDevNumeric = TL_ERR_NUMERIC;
+
+// KV header at the start of the caller's KV buffer.
+struct KvHeader {
+  int32_t pos[kMaxLanes];         // cached tokens per lane
+  int32_t cum_layers[kMaxLanes];  // layers of all lanes before this one
+};
+
+// ---------------------------------------------------------------- kernels (host launchers)
+
+// packing (pack.cu)
+tl_status launch_pack(const float* w, int N, int K, int bits, int group, uint32_t* packed,
+                      uint16_t* scales, cudaStream_t s);
+tl_status launch_unpack(const uint32_t* packed, int N, int K, int bits, int8_t* codes,
+                        cudaStream_t s);
+tl_status launch_kv_quant_int8(const __half* x, int rows, int hd, int8_t* codes, __half* scales,
+                               cudaStream_t s);
+// INT3 canonical rows -> INT4 canonical rows (same codes), for the GEMM kernels
+tl_status launch_int3_to_int4(const uint32_t* src, int N, int K, uint32_t* dst, cudaStream_t s);
+
+// quantised-weight GEMM (gemm_mma.cu): part[z][t][n] = sum_{k in split z} x[t][k] * W[n][k]
+struct GemmArgs {
+  const uint32_t* w0;   // INT4 canonical words, rows [0, n_split)
+  const __half* s0;
+  const uint32_t* w1;   // rows [n_split, N) (may equal w0 when n_split == N)
+  const __half* s1;
+  int n_split;
+  int N, K, G;
+  const __half* x;      // fp16 [T][K]
+  int T;
+  float* part;          // fp32 [S][T][N]
+  int splits;           // S
+};
+int gemm_splits(int N, int K, int T);
+tl_status launch_gemm(const GemmArgs& a, cudaStream_t s);
+
+// elementwise (elementwise.cu)
+struct EmbedArgs {
+  const int32_t* ids;        // [rows] or null
+  const __half* h_in;        // [rows][d] or null
+  const __half* embed;       // [vocab][d]
+  int vocab, d, rows;
+  const int32_t* src_row;    // row t reads input row src_row[t] (null = identity)
+  float* h;                  // [rows][d]
+  int* status;
+};
+tl_status launch_embed(const EmbedArgs& a, cudaStream_t s);
+
+struct NormArgs {
+  float* h;                  // [rows][d] residual
+  int d, rows;               // rows: all rows (trace writes cover all)
+  const float* part;         // [S][part_rows][d] partials to add (S may be 0)
+  int part_rows;
+  int S, n_add;              // rows < n_add get h += sum_s part[s]
+  const float* gamma_next;   // rows < n_next: x = fp16(rmsnorm(h) * gamma_next)
+  __half* x;
+  int n_next;
+  const float* gamma_final;  // rows in [fin_lo, fin_hi): y[out_row] = rmsnorm(h) * gamma_final
+  float* y;
+  int fin_lo, fin_hi;
+  float* trace;              // null or [rows][d] (indexed by out_row)
+  const int32_t* out_row;    // null = identity
+  float eps;
+  int* status;
+};
+tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s);
+
+struct RopeKvArgs {
+  const float* part;         // [S][rows][3d] QKV partials
+  int S, rows, d, H, hd;
+  const float2* rope_cs;     // [max_ctx][hd/2] (cos, sin)
+  __half* q;                 // [rows][d]
+  __half* k;                 // [rows][d] or null
+  __half* v;                 // [rows][d] or null
+  // cache (null kv_base = uncached)
+  char* kv_base;             // start of lane data (after the header)
+  const KvHeader* hdr;
+  size_t layer_bytes, kv_region_bytes;   // region = K or V array bytes (256-aligned)
+  int layer, max_ctx, kv_int8;
+  const int32_t* lane_of_row;  // decode: lane of each row; null = prefill of `lane`
+  int lane;
+  int decode;                  // 1: position = hdr->pos[lane]; 0: position = row index
+};
+tl_status launch_rope_kv(const RopeKvArgs& a, cudaStream_t s);
+
+tl_status launch_swiglu(const float* part, int S, int rows, int F, __half* u, cudaStream_t s);
+tl_status launch_set_pos(KvHeader* hdr, int lane, int value, cudaStream_t s);
+tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s);
+
+// attention (attention.cu)
+tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
+                              int T, int H, int hd, cudaStream_t s);
+struct DecodeAttnArgs {
+  const __half* q;           // [rows][d]
+  __half* out;               // [rows][d]
+  int rows, H, hd, d;
+  const char* kv_base;
+  const KvHeader* hdr;
+  size_t layer_bytes, kv_region_bytes;
+  int layer, max_ctx, kv_int8;
+  const int32_t* lane_of_row;
+  float* scratch;            // [rows][H][max_chunks][hd + 2]
+  int max_chunks;
+};
+tl_status launch_attn_decode(const DecodeAttnArgs& a, cudaStream_t s);
+
+}  // namespace tl
