@@ -1,0 +1,505 @@
+#!/usr/bin/env python
+"""Benchmark of the looped-block hot path on B200.
+
+Headline: one looped forward of the 407M-shaped model (d_model 2048, 16 heads
+x 128, ffn 8192, INT4 group 128, 2 pre-blocks + 1 shared loop block run L=8,
+seq 128, batch 1, final RMSNorm, no logits) per step; value = tokens/s over the
+whole job.  Secondary lines (inside the same JSON object) time KV-cached
+decode: batch 1 with FP16 KV, batch 8 at context 2048 with INT8 KV, and the
+mixed-depth INT3 lanes L=[4,16,32].
+
+Inputs are seeded synthetic weights and token ids.  The model's weights (about
+104 MB) fit in the 126 MB L2, so L2 is flushed (a 256 MiB write) before every
+timed step; the flush is outside the timed interval.
+
+Multi-GPU: replicas only (each rank runs the same workload on its own GPU, no
+data-path collective); value = all ranks' tokens / the slowest rank's time.
+
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "looped forward ms & tokens/s (seq=128,L=8; decode tok/s) + % of roofline"
+WORKLOAD = ("prefill407m: d_model 2048, 16 heads x 128, SwiGLU ffn 8192, INT4 group 128 fp16 "
+            "scales, 2 pre-blocks + shared loop block L=8, seq 128, batch 1, no logits")
+FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-decode", action="store_true", help="skip the decode sub-measurements")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.err = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
+        except OSError as e:
+            self.err = str(e)
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        time.sleep(0.15)
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        if self.err or not self.out:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": self.err or "no nvidia-smi samples"}
+        sms, mx, reasons, n = [], None, set(), 0
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sms.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            n += 1
+            for name, val in zip(names, f[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": n}
+
+
+def gpu_uuid(torch, dev):
+    u = str(torch.cuda.get_device_properties(dev).uuid)
+    return u if u.startswith("GPU-") else "GPU-" + u
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+
+def oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline_prefill(seconds: float = 10.0):
+    """The oracle's full seq-128 L=8 forward on the host cores, repeated for
+    about `seconds` (at least 2 forwards) after one untimed forward."""
+    import numpy as np
+    import synthetic as syn
+    from oracle.workloads import build_oracle_model
+    w = syn.WORKLOADS["prefill407m"]
+    om = build_oracle_model("prefill407m")
+    ids = syn.prompt_ids(w)
+    om.prefill(ids, w.L[0])
+    n, t0 = 0, time.perf_counter()
+    while n < 2 or time.perf_counter() - t0 < seconds:
+        om.prefill(ids, w.L[0])
+        n += 1
+    dt = time.perf_counter() - t0
+    return {"value": round(w.seq * n / dt, 2), "unit": "tokens/s", "cores": oracle_threads(),
+            "kind": "oracle",
+            "sample": f"{n} full forwards (seq 128, L=8, fp64 numpy oracle), {dt:.1f} s; "
+                      f"model build untimed"}
+
+
+def run_reference(args, rank, world):
+    """CPU oracle arm: each step is one of the 10 block applications of the
+    seq-128 L=8 forward (cycling pre0, pre1, loop x 8 on the inputs that layer
+    sees), so K steps are K/10 forwards of work."""
+    if rank != 0:
+        return
+    import numpy as np
+    import synthetic as syn
+    from oracle import tinyloop_oracle as o
+    from oracle.workloads import build_oracle_model
+    w = syn.WORKLOADS["prefill407m"]
+    L = w.L[0]
+    om = build_oracle_model("prefill407m")
+    ids = syn.prompt_ids(w)
+    trace = []
+    om.prefill(ids, L, trace=trace)
+    inputs = [om.embed(ids)] + trace[:-1]
+    sched = om.schedule(L)
+    pos = np.arange(w.seq)
+
+    def step(i):
+        layer = i % len(sched)
+        blk, h = sched[layer], inputs[layer]
+        q, k, v = blk.qkv(h, pos)
+        return blk.finish(h, o.causal_attention(q, k, v, pos))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    layers = len(sched)
+    fwd_s = dt / args.steps * layers
+    value = round(w.seq / fwd_s, 3)
+    sample = (f"{args.steps} block applications = {args.steps / layers:.1f} forwards "
+              f"(seq 128, L=8) on the fp64 numpy oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "step": "one block application (1/10 forward)"},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": oracle_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def source_hash(*files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_file: str, src_files):
+    """Per-launch DRAM bytes of a kernel from its committed ncu summary, if the
+    summary was taken on the current source (matching hash); else None."""
+    path = os.path.join(ROOT, "profiles", kernel_file)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("source_sha256_16") != source_hash(*src_files):
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def run_ours(args, rank, world, dist):
+    import numpy as np
+    import torch
+
+    from weight_shared_looped_b200 import build as _build
+    _build.build()
+    import synthetic as syn
+    import weight_shared_looped_b200 as tl
+    from oracle import tinyloop_oracle as o   # noqa: F401  (block_cfg helper only)
+    from weight_shared_looped_b200.model import DeviceBlock, DeviceModel
+
+    dev = int(os.environ.get("LOCAL_RANK", 0))
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    w = syn.WORKLOADS["prefill407m"]
+    L, seq = w.L[0], w.seq
+
+    def cfg(bits):
+        return {"d_model": 2048, "n_heads": 16, "head_dim": 128, "ffn": 8192, "bits": bits,
+                "group": 128, "eps": 1e-5, "rope_theta": 10000.0}
+
+    blocks = {n: DeviceBlock(cfg(4), weights=syn.block_weights(w.shape, w.seed, n))
+              for n in syn.block_names(w)}
+    embed = syn.embedding(w.shape, w.seed)
+    gamma_f = syn.final_gain(w.shape, w.seed)
+    model = DeviceModel([blocks["pre0"], blocks["pre1"]], blocks["loop"], gamma_f, embed,
+                        max_tokens=2048, max_lanes=8, max_ctx=2048 + 64, max_L=32)
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    ids = torch.from_numpy(syn.prompt_ids(w).astype(np.int32)).cuda()
+    y = torch.empty(seq, 2048, dtype=torch.float32, device="cuda")
+
+    def step():
+        model.prefill(ids, L=L, y_out=y)
+
+    def timed(fn, k, warm):
+        for _ in range(warm):
+            flush.zero_()
+            fn()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(k)]
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        return sum(a.elapsed_time(b) for a, b in evs) / 1e3   # seconds
+
+    # headline: prefill forward
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    assert model.sync_status() == tl.TL_OK
+    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+        t = timed(step, args.steps, 0)
+    assert model.sync_status() == tl.TL_OK
+    if dist:
+        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t = float(tt.item())
+    tokens = seq * args.steps * world
+    value = tokens / t
+    ms_per_step = t / args.steps * 1e3
+    n_layers = 2 + L
+    launches_per_fwd = 2 + 9 * n_layers
+
+    # e2e: host (pinned) ids in, host y out, through the C-ABI call
+    ids_h = torch.from_numpy(syn.prompt_ids(w).astype(np.int32)).pin_memory()
+    y_h = torch.empty(seq, 2048, dtype=torch.float32).pin_memory()
+    k_e2e = max(10, min(args.steps, 500))
+    t_e2e = timed(lambda: model.prefill(ids_h, L=L, y_out=y_h), k_e2e, 3)
+    if dist:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device="cuda")
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = float(tt.item())
+    e2e = {"value": round(seq * k_e2e * world / t_e2e, 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": ids_h.numel() * 4, "d2h_bytes_per_step": y_h.numel() * 4}
+
+    # roofline of the dominant kernel: the gate|up GEMM launch (N 16384, K 2048, T 128)
+    xg = torch.randn(seq, 2048, device="cuda").half()
+    wg = torch.cat([blocks["loop"].t["w_gate"], blocks["loop"].t["w_up"]])
+    sg = torch.cat([blocks["loop"].t["s_gate"], blocks["loop"].t["s_up"]])
+    yg = torch.empty(seq, 16384, dtype=torch.float32, device="cuda")
+    ws_b = tl.tl_linear_workspace_bytes(16384, 2048, seq)
+    wsg = torch.empty(max(ws_b, 1), dtype=torch.uint8, device="cuda")
+    k_gemm = 200
+    t_gemm = timed(lambda: tl.tl_linear(wg, sg, 16384, 2048, 128, xg, yg, wsg), k_gemm, 5)
+    flops = 2.0 * seq * 16384 * 2048
+    achieved = flops * k_gemm / t_gemm / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
+            "traffic": ncu_traffic("gemm_w4_mma_gateup_T128.txt",
+                                   ["weight_shared_looped_b200/csrc/gemm_mma.cu"]),
+            "kernel": "gemm_w4_mma_kernel<64> (gate|up, N 16384, K 2048, T 128; cold L2)",
+            "peak_kind": f"bf16 dense burst, {pk['source']} (fp16 operands run at the same rate)",
+            "us_per_launch": round(t_gemm / k_gemm * 1e6, 2),
+            "forward_tflops": round(172.5e9 * args.steps / (t / world) / 1e12, 2),
+            "forward_frac": round(172.5e9 * args.steps / (t / world) / 1e12 / pk["bf16_tflops"], 4)}
+
+    decode = None
+    if not args.no_decode:
+        decode = run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
+                            cfg)
+
+    line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "l2": "flushed before every timed step (256 MiB write)",
+                       "parallelism": "replicas" if world > 1 else "single",
+                       "graphs": "one CUDA graph per (seq, L)"},
+            "roofline": roof, "e2e": e2e, "gpu_launches": launches_per_fwd * args.steps,
+            "clocks": clk.summary()}
+    if decode is not None:
+        line["decode"] = decode
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline_prefill()
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    model.close()
+    return line
+
+
+def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg):
+    """KV-cached decode throughput: B=1 FP16 KV (prompt 256, 128 steps), B=8
+    INT8 KV at context 2048 (64 steps), mixed-depth INT3 lanes (ctx 1024, 32
+    steps).  Each timed step is one tl_decode_step; caches are filled by GPU
+    prefill of seeded prompt ids."""
+    from weight_shared_looped_b200.model import DeviceBlock, DeviceModel
+    out = {}
+    hbm = pk["hbm_gbs"]
+    blk_bytes = 34.6e6
+
+    def ids_t(x):
+        return torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).cuda()
+
+    def max_t(t):
+        if dist:
+            tt = torch.tensor([t], dtype=torch.float64, device="cuda")
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            return float(tt.item())
+        return t
+
+    # B = 1, FP16 KV, prompt 256 -> 384
+    w = syn.WORKLOADS["decode407m"]
+    kv = model.new_kv([8], max_ctx=w.max_ctx)
+    model.prefill(ids_t(syn.prompt_ids(w)), L=8, kv=kv, lane=0)
+    dids = [ids_t(syn.decode_ids(w)[i:i + 1]) for i in range(w.steps)]
+    it = iter(range(10 ** 9))
+    y1 = torch.empty(1, 2048, dtype=torch.float32, device="cuda")
+
+    def dstep():
+        model.decode(kv, dids[next(it) % w.steps], L_per_lane=[8], y_out=y1)
+
+    # warm the graph, then rewind the cache so every timed step is at 256..383
+    dstep()
+    kv.set_position(0, w.seq)
+    it = iter(range(10 ** 9))
+    t = max_t(timed(dstep, w.steps, 0))
+    avg_ctx = w.seq + (w.steps + 1) / 2
+    kv_bytes = 10 * avg_ctx * 2048 * 2 * 2
+    step_bytes = 3 * blk_bytes + kv_bytes
+    out["b1_fp16kv"] = {"tok_s": round(w.steps * world / t, 1),
+                        "ms_per_step": round(t / w.steps * 1e3, 4),
+                        "hbm_bytes_per_step": int(step_bytes),
+                        "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                        "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
+    kv.close()
+    torch.cuda.synchronize()
+
+    # B = 8, INT8 KV, context 2048 -> 2112
+    w = syn.WORKLOADS["longctx_int8"]
+    kv = model.new_kv(list(w.L), max_ctx=w.max_ctx, dtype="int8")
+    for b in range(8):
+        model.prefill(ids_t(syn.token_ids(w.seq, w.seed, f"ctxprompt.lane{b}")), L=8, kv=kv,
+                      lane=b)
+    ids8 = [ids_t(np.array([syn.decode_ids(w, b)[s] for b in range(8)])) for s in range(w.steps)]
+    y8 = torch.empty(8, 2048, dtype=torch.float32, device="cuda")
+    it2 = iter(range(10 ** 9))
+
+    def dstep8():
+        model.decode(kv, ids8[next(it2) % w.steps], L_per_lane=list(w.L), y_out=y8)
+
+    dstep8()
+    for b in range(8):
+        kv.set_position(b, w.seq)
+    t = max_t(timed(dstep8, w.steps, 0))
+    avg_ctx = w.seq + (w.steps + 1) / 2
+    kv_bytes = 8 * 10 * avg_ctx * 16 * (2 * 128 + 2 * 2)
+    step_bytes = 3 * blk_bytes + kv_bytes
+    out["b8_int8kv_ctx2048"] = {"tok_s": round(8 * w.steps * world / t, 1),
+                                "ms_per_step": round(t / w.steps * 1e3, 4),
+                                "hbm_bytes_per_step": int(step_bytes),
+                                "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                                "workload": "batch 8, context 2048 + 64 steps, L=8, INT8 KV"}
+    kv.close()
+    torch.cuda.synchronize()
+
+    # mixed-depth INT3 loop block, lanes L = [4, 16, 32], context 1024
+    w = syn.WORKLOADS["mixed_int3"]
+    loop3 = DeviceBlock(cfg(3), weights=syn.block_weights(w.shape, w.seed, "loop"))
+    m3 = DeviceModel([blocks["pre0"], blocks["pre1"]], loop3, syn.final_gain(w.shape, w.seed),
+                     syn.embedding(w.shape, w.seed), max_tokens=1024, max_lanes=3,
+                     max_ctx=w.max_ctx, max_L=32)
+    kv = m3.new_kv(list(w.L), max_ctx=w.max_ctx)
+    for b in range(3):
+        m3.prefill(ids_t(syn.prompt_ids(w, b)), L=w.L[b], kv=kv, lane=b)
+    ids3 = [ids_t(np.array([syn.decode_ids(w, b)[s] for b in range(3)])) for s in range(w.steps)]
+    y3 = torch.empty(3, 2048, dtype=torch.float32, device="cuda")
+    it3 = iter(range(10 ** 9))
+
+    def dstep3():
+        m3.decode(kv, ids3[next(it3) % w.steps], L_per_lane=list(w.L), y_out=y3)
+
+    dstep3()
+    for b in range(3):
+        kv.set_position(b, w.seq)
+    t = max_t(timed(dstep3, w.steps, 0))
+    avg_ctx = w.seq + (w.steps + 1) / 2
+    slots = sum(2 + L for L in w.L)
+    kv_bytes = slots * avg_ctx * 2048 * 2 * 2
+    step_bytes = 2 * blk_bytes + 28.2e6 + kv_bytes
+    out["b3_int3_mixedL"] = {"tok_s": round(3 * w.steps * world / t, 1),
+                             "ms_per_step": round(t / w.steps * 1e3, 4),
+                             "hbm_bytes_per_step": int(step_bytes),
+                             "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                             "workload": "lanes L=[4,16,32], INT3 loop block, context 1024 + "
+                                         "32 steps, FP16 KV"}
+    kv.close()
+    m3.close()
+    loop3.close()
+    return out
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    line = run_ours(args, rank, world, dist)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -264,6 +264,23 @@ tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
                          int n_lanes, float* y_out, float* h_trace,
                          tl_stream stream);
 
+/* ------------------------------------------------------------------------
+ * Quantised-weight linear layer (test and measurement hook).  The GEMM every
+ * block projection uses:  y[t, n] = sum_k x[t, k] * code[n, k] * scale[n, k/G]
+ * for one canonical INT4 matrix (see tl_pack_weights), fp32 accumulation;
+ * split-K partial sums, when the kernel uses them, are added in a fixed order.
+ *   packed, scales  device, INT4 canonical [N, K/8] words and fp16 [N, K/G]
+ *   x               device fp16 [T, K]
+ *   y               device fp32 [T, N]   (written)
+ *   workspace       device scratch of tl_linear_workspace_bytes(N, K, T) bytes
+ *                   (may be NULL when that size is 0)
+ * Requirements: N % 64 == 0, K % 64 == 0, group in {64, 128}, 1 <= T <= 8192.
+ * bits must be 4 (an INT3 matrix is converted by tl_block_create). */
+tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes);
+tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K,
+                    int group, const uint16_t* x, int T, float* y,
+                    void* workspace, tl_stream stream);
+
 /* Synchronise `stream`, then return and clear the model's device status word
  * (TL_OK, TL_ERR_TIMEOUT or TL_ERR_NUMERIC). */
 tl_status tl_sync_status(tl_model* model, tl_stream stream);

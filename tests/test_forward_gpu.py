@@ -214,3 +214,20 @@ def test_non_finite_input_reports_numeric_status(model):
     model.prefill(h_in=to_dev(x, torch.float16), L=1)
     assert model.sync_status() == tl.TL_ERR_NUMERIC
     assert model.sync_status() == tl.TL_OK           # the status word is cleared
+
+
+def test_new_cache_after_destroy_uses_its_own_graphs(model):
+    """A cache created after another was destroyed (possibly at the same host
+    address) must not replay graphs captured for the old one."""
+    x = to_dev(syn.hidden_input(W, 8, name="reuse.prompt"), torch.float16)
+    step = to_dev(syn.hidden_input(W, 1, name="reuse.step"), torch.float16)
+    outs = []
+    for lanes in ([2, 1, 2], [2]):
+        kv = model.new_kv(lanes, max_ctx=9)
+        for b in range(len(lanes)):
+            model.prefill(h_in=x, L=lanes[b], kv=kv, lane=b)
+        outs.append(model.decode(kv, h_in=step.repeat(len(lanes), 1),
+                                 L_per_lane=lanes).cpu().numpy())
+        kv.close()
+    assert np.array_equal(outs[0][0], outs[1][0])
+    assert np.array_equal(outs[0][2], outs[1][0])

@@ -79,6 +79,8 @@ _SIGS = {
     "tl_prefill": ([P, P, P, I, I, P, I, P, P, P], I),
     "tl_decode_step": ([P, P, P, P, P, I, P, P, P], I),
     "tl_sync_status": ([P, P], I),
+    "tl_linear_workspace_bytes": ([I, I, I, ctypes.POINTER(SZ)], I),
+    "tl_linear": ([P, P, I, I, I, P, I, P, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -255,6 +257,19 @@ def tl_decode_step(model: int, kv: int, ids=None, h_in=None, *, L_per_lane: Sequ
     arr = _int_array(L_per_lane)
     _check(lib.tl_decode_step(model, kv, _ptr(ids), _ptr(h_in), ctypes.cast(arr, P),
                               len(L_per_lane), _ptr(y_out), _ptr(h_trace), _stream(stream)))
+
+
+def tl_linear_workspace_bytes(N: int, K: int, T: int) -> int:
+    b = SZ()
+    _check(lib.tl_linear_workspace_bytes(N, K, T, ctypes.byref(b)))
+    return b.value
+
+
+def tl_linear(packed, scales, N: int, K: int, group: int, x, y, workspace=None,
+              stream=None) -> None:
+    T = x.shape[0]
+    _check(lib.tl_linear(_ptr(packed), _ptr(scales), N, K, group, _ptr(x), T, _ptr(y),
+                         _ptr(workspace), _stream(stream)))
 
 
 def tl_sync_status(model: int, stream=None) -> int:

@@ -17,6 +17,7 @@
 #include <tuple>
 #include <vector>
 #include <algorithm>
+#include <atomic>
 
 #include "tl_internal.cuh"
 
@@ -71,6 +72,7 @@ struct tl_block {
 };
 
 struct tl_kv {
+  uint64_t id;            // unique per created cache; graphs are keyed on it
   const tl_model* model;
   int n_lanes, max_ctx, dtype;
   int L[kMaxLanes];
@@ -82,6 +84,7 @@ struct tl_kv {
 struct GraphEntry {
   cudaGraphExec_t exec = nullptr;
   int32_t* lane_of_row = nullptr;   // device, decode graphs
+  uint64_t kv_id = 0;               // cache the graph writes (0 = none)
 };
 
 struct tl_model {
@@ -250,12 +253,31 @@ size_t part_floats(const tl_model* m, int T) {
   return best;
 }
 
+void free_graph(GraphEntry& g) {
+  if (g.exec) cudaGraphExecDestroy(g.exec);
+  if (g.lane_of_row) cudaFree(g.lane_of_row);
+}
+
 void free_graphs(tl_model* m) {
-  for (auto& kv : m->graphs_cache) {
-    if (kv.second.exec) cudaGraphExecDestroy(kv.second.exec);
-    if (kv.second.lane_of_row) cudaFree(kv.second.lane_of_row);
-  }
+  for (auto& kv : m->graphs_cache) free_graph(kv.second);
   m->graphs_cache.clear();
+}
+
+// Graphs bake in a cache's buffer and geometry: drop them with the cache.
+void free_kv_graphs(tl_model* m, uint64_t kv_id) {
+  for (auto it = m->graphs_cache.begin(); it != m->graphs_cache.end();) {
+    if (it->second.kv_id == kv_id) {
+      free_graph(it->second);
+      it = m->graphs_cache.erase(it);
+    } else {
+      ++it;
+    }
+  }
+}
+
+uint64_t next_kv_id() {
+  static std::atomic<uint64_t> counter{1};
+  return counter.fetch_add(1);
 }
 
 }  // namespace
@@ -466,6 +488,7 @@ TL_API tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
   TL_CHECK_ARG(((uintptr_t)buffer & 255) == 0, "buffer must be 256-byte aligned");
   TL_CHECK_ARG(buffer_bytes >= need, "buffer has %zu bytes, %zu needed", buffer_bytes, need);
   std::unique_ptr<tl_kv> kv(new tl_kv());
+  kv->id = next_kv_id();
   kv->model = model;
   kv->n_lanes = n_lanes;
   kv->max_ctx = max_ctx;
@@ -487,6 +510,8 @@ TL_API tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
 }
 
 TL_API tl_status tl_kv_destroy(tl_kv* kv) {
+  if (!kv) return ok();
+  free_kv_graphs(const_cast<tl_model*>(kv->model), kv->id);
   delete kv;
   return ok();
 }
@@ -774,13 +799,14 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
 }
 
 template <typename F>
-tl_status run_graph(tl_model* m, const std::string& key, cudaStream_t stream, F&& enqueue,
-                    GraphEntry** entry_out = nullptr, const int32_t* lane_map = nullptr) {
+tl_status run_graph(tl_model* m, const std::string& key, uint64_t kv_id, cudaStream_t stream,
+                    F&& enqueue, const int32_t* lane_map = nullptr) {
   if (!m->graphs) return enqueue(stream, nullptr);
   auto it = m->graphs_cache.find(key);
   if (it == m->graphs_cache.end()) {
     if (m->graphs_cache.size() >= 64) free_graphs(m);
     GraphEntry ge;
+    ge.kv_id = kv_id;
     if (lane_map) {
       if (cudaMalloc(&ge.lane_of_row, kMaxLanes * 4) != cudaSuccess)
         return set_error(TL_ERR_OOM, "cannot allocate a graph lane map");
@@ -809,7 +835,6 @@ tl_status run_graph(tl_model* m, const std::string& key, cudaStream_t stream, F&
     it = m->graphs_cache.emplace(key, ge).first;
   }
   TL_CUDA(cudaGraphLaunch(it->second.exec, stream));
-  if (entry_out) *entry_out = &it->second;
   return ok();
 }
 
@@ -837,10 +862,11 @@ TL_API tl_status tl_prefill(tl_model* model, const int32_t* ids, const uint16_t*
   if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)seq * 4, cudaMemcpyDefault, s));
   else TL_CUDA(cudaMemcpyAsync(model->hin, h_in, (size_t)seq * d * 2, cudaMemcpyDefault, s));
   char key[256];
-  snprintf(key, sizeof(key), "P|%d|%d|%p|%d|%d|%p", seq, L, (void*)kv, lane, ids ? 1 : 0,
-           (void*)h_trace);
+  const uint64_t kv_id = kv ? kv->id : 0;
+  snprintf(key, sizeof(key), "P|%d|%d|%llu|%d|%d|%p", seq, L, (unsigned long long)kv_id, lane,
+           ids ? 1 : 0, (void*)h_trace);
   const bool use_ids = ids != nullptr;
-  TL_TRY(run_graph(model, key, s, [&](cudaStream_t cs, int32_t*) {
+  TL_TRY(run_graph(model, key, kv_id, s, [&](cudaStream_t cs, int32_t*) {
     return enqueue_prefill(model, use_ids, seq, L, kv, lane, h_trace, cs);
   }));
   TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)seq * d * 4, cudaMemcpyDefault, s));
@@ -875,17 +901,17 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
   const int d = model->d;
   if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)n_lanes * 4, cudaMemcpyDefault, s));
   else TL_CUDA(cudaMemcpyAsync(model->hin, h_in, (size_t)n_lanes * d * 2, cudaMemcpyDefault, s));
-  std::string key = "D|" + std::to_string((uintptr_t)kv) + "|" + std::to_string(n_lanes) + "|" +
+  std::string key = "D|" + std::to_string(kv->id) + "|" + std::to_string(n_lanes) + "|" +
                     std::to_string(ids ? 1 : 0) + "|" + std::to_string((uintptr_t)h_trace);
   for (int b = 0; b < n_lanes; ++b) key += "|" + std::to_string(L_per_lane[b]);
   const bool use_ids = ids != nullptr;
   if (model->graphs) {
     TL_TRY(run_graph(
-        model, key, s,
+        model, key, kv->id, s,
         [&](cudaStream_t cs, int32_t* lmap) {
           return enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, lmap, h_trace, cs);
         },
-        nullptr, order));
+        order));
   } else {
     // without graphs the lane map lives in the model workspace
     TL_CUDA(cudaMemcpyAsync(model->lane_map, order, sizeof(order), cudaMemcpyHostToDevice, s));
@@ -893,6 +919,53 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
   }
   TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)n_lanes * d * 4, cudaMemcpyDefault, s));
   for (int b = 0; b < n_lanes; ++b) kv->pos[b] += 1;
+  return ok();
+}
+
+// ============================================================================
+// Linear-layer hook
+// ============================================================================
+namespace {
+tl_status check_linear(int N, int K, int group, int T) {
+  TL_CHECK_ARG(N >= 64 && N % 64 == 0, "N = %d must be a positive multiple of 64", N);
+  TL_CHECK_ARG(K >= 64 && K % 64 == 0, "K = %d must be a positive multiple of 64", K);
+  if (group != 64 && group != 128)
+    return set_error(TL_ERR_UNSUPPORTED, "group = %d: only 64 and 128 are supported", group);
+  TL_CHECK_ARG(T >= 1 && T <= 8192, "T = %d out of [1, 8192]", T);
+  return ok();
+}
+}  // namespace
+
+TL_API tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes) {
+  TL_CHECK_ARG(bytes, "bytes is NULL");
+  TL_TRY(check_linear(N, K, 64, T));
+  const int S = gemm_splits(N, K, T);
+  *bytes = S > 1 ? (size_t)S * T * N * 4 : 0;
+  return ok();
+}
+
+TL_API tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K,
+                           int group, const uint16_t* x, int T, float* y, void* workspace,
+                           tl_stream stream) {
+  TL_TRY(check_linear(N, K, group, T));
+  TL_CHECK_ARG(packed && scales && x && y, "NULL device pointer");
+  const int S = gemm_splits(N, K, T);
+  TL_CHECK_ARG(S == 1 || workspace, "workspace is NULL but %zu bytes are needed",
+               (size_t)S * T * N * 4);
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.w0 = a.w1 = packed;
+  a.s0 = a.s1 = (const __half*)scales;
+  a.n_split = a.N = N;
+  a.K = K;
+  a.G = group;
+  a.x = (const __half*)x;
+  a.T = T;
+  a.splits = S;
+  a.part = S > 1 ? (float*)workspace : y;
+  cudaStream_t s = (cudaStream_t)stream;
+  TL_TRY(launch_gemm(a, s));
+  if (S > 1) TL_TRY(launch_split_sum((const float*)workspace, S, (long)T * N, y, s));
   return ok();
 }
 

@@ -159,6 +159,15 @@ __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
   }
 }
 
+__global__ void split_sum_kernel(const float* __restrict__ part, int S, long n,
+                                 float* __restrict__ y) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  float acc = part[i];
+  for (int s = 1; s < S; ++s) acc += part[(long)s * n + i];
+  y[i] = acc;
+}
+
 int token_tile(int T) { return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : 64; }
 
 }  // namespace
@@ -174,6 +183,13 @@ int gemm_splits(int N, int K, int T) {
   while (tiles * s < 2 * 148 && s * 2 <= 16 && n_chunks % (s * 2) == 0 && n_chunks / (s * 2) >= 2)
     s *= 2;
   return s;
+}
+
+tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s) {
+  if (n == 0) return ok();
+  split_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, n, y);
+  TL_LAUNCH_CHECK();
+  return ok();
 }
 
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {

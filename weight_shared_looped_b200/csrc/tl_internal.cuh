@@ -80,6 +80,8 @@ struct GemmArgs {
 };
 int gemm_splits(int N, int K, int T);
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s);
+// y[t][n] = sum_{s < S} part[s][t][n], in order s = 0, 1, ...
+tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s);
 
 // elementwise (elementwise.cu)
 struct EmbedArgs {
