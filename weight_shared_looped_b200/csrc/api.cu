@@ -307,6 +307,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
                      pd.rope_theta == ld.rope_theta,
                  "pre[%d] shape differs from the loop block", i);
   }
+  TL_TRY(gemm_tc_init());
   std::unique_ptr<tl_model> m(new tl_model());
   m->desc = md;
   for (int i = 0; i < md.n_pre; ++i) m->pre.push_back(md.pre[i]);
@@ -610,6 +611,7 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
       break;
   }
   a.splits = gemm_splits(a.N, a.K, T);
+  a.status = m->status;
   return a;
 }
 
@@ -949,6 +951,7 @@ TL_API tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N
                            tl_stream stream) {
   TL_TRY(check_linear(N, K, group, T));
   TL_CHECK_ARG(packed && scales && x && y, "NULL device pointer");
+  TL_TRY(gemm_tc_init());
   const int S = gemm_splits(N, K, T);
   TL_CHECK_ARG(S == 1 || workspace, "workspace is NULL but %zu bytes are needed",
                (size_t)S * T * N * 4);

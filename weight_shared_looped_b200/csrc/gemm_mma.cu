@@ -176,7 +176,7 @@ int token_tile(int T) { return T <= 8 ? 8 : T <= 16 ? 16 : T <= 32 ? 32 : 64; }
 // 64-wide chunks and gives at least two CTAs per SM.  Decode-sized calls
 // (T <= 8) always use the T <= 8 branch, so a lane's reduction order does not
 // depend on how many lanes are active.
-int gemm_splits(int N, int K, int T) {
+int gemm_mma_splits(int N, int K, int T) {
   int n_chunks = K / KC;
   int tiles = (N / ROWS_CTA) * ((T + token_tile(T) - 1) / token_tile(T));
   int s = 1;
@@ -192,7 +192,16 @@ tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStrea
   return ok();
 }
 
+int gemm_splits(int N, int K, int T) {
+  return gemm_tc_eligible(N, K, T) ? gemm_tc_splits(N, K, T) : gemm_mma_splits(N, K, T);
+}
+
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (gemm_tc_eligible(a.N, a.K, a.T)) return launch_gemm_tc(a, s);
+  return launch_gemm_mma(a, s);
+}
+
+tl_status launch_gemm_mma(const GemmArgs& a, cudaStream_t s) {
   if (a.T == 0) return ok();
   const int nt = token_tile(a.T);
   dim3 grid(a.N / ROWS_CTA, (a.T + nt - 1) / nt, a.splits);

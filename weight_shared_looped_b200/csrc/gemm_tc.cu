@@ -1,0 +1,451 @@
+// Quantised-weight GEMM on the 5th-generation tensor cores (tcgen05), for
+// prefill-sized token counts:
+//   part[z][t][n] = sum over k in split z of x[t][k] * W[n][k],
+//   W[n][k] = code[n][k] * scale[n][k / G]  (group-wise symmetric INT4).
+//
+// One CTA computes 128 weight rows x BN tokens over a range of 64-wide k
+// blocks.  Per k block:
+//   * a TMA warp loads the activation tile x[BN tokens][64 k] (fp16, 128-byte
+//     swizzled, rows past T read as zero) and the packed weight tile
+//     [128 rows][8 words] into a shared-memory stage;
+//   * four dequantisation warps (one TMEM lane quadrant each, one thread per
+//     weight row) turn the row's 64 codes into fp16 code*scale pairs and store
+//     them straight into tensor memory with tcgen05.st: the weight tile is the
+//     A operand of the MMA and never passes through shared memory;
+//   * one thread issues four tcgen05.mma kind::f16 (M 128, N BN, K 16), A from
+//     TMEM, B from the swizzled shared-memory tile, fp32 accumulation in TMEM,
+//     and commits to the stage's "empty" barrier.
+// The same four warps then read the accumulator back with tcgen05.ld and store
+// it as fp32 partial sums.  Every wait on an mbarrier is bounded: when a wait
+// runs out the CTA records TL_ERR_TIMEOUT in the status word, stops issuing
+// work, waits (bounded) for its copies in flight, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "tl_internal.cuh"
+
+namespace tl {
+namespace {
+
+constexpr int BM = 128;            // weight rows per CTA (MMA M)
+constexpr int BK = 64;             // k per stage
+constexpr int STAGES = 4;
+constexpr int THREADS = 256;       // warp 0 TMA, warp 1 MMA, warps 4..7 dequant + epilogue
+constexpr int A_COLS = BK / 2;     // TMEM columns per A stage (two fp16 per column)
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a bounded wait gives up after 2 s
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait for the phase with the given parity to complete: false after
+// kWaitLimitNs of global time.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  uint64_t start = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((i & 255) == 0) {
+      const uint64_t now = globaltimer_ns();
+      if (i == 0) start = now;
+      else if (now - start > kWaitLimitNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
+      "%3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+  // K-major, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused for this layout)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset
+  d |= (uint64_t)1 << 46;                 // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;                 // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                       uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t dequant_code_pair(uint32_t w, uint32_t sel) {
+  // byte b of w holds the codes of k = 2b (low nibble) and 2b + 1 (high nibble)
+  uint32_t x, h;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(w), "r"(0u), "r"(sel));
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
+  const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
+  const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+struct TcArgs {
+  int N, K, G, T, n_split;   // n_split % 128 == 0
+  int kblocks_per_split;
+  const __half* s0;
+  const __half* s1;
+  float* part;
+  int* status;
+};
+
+template <int BN>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x,
+                      const __grid_constant__ CUtensorMap map_w0,
+                      const __grid_constant__ CUtensorMap map_w1, TcArgs a) {
+  constexpr uint32_t B_BYTES = BN * 128;          // BN rows x 64 fp16
+  constexpr uint32_t W_BYTES = BM * 32;           // 128 rows x 8 words
+  constexpr uint32_t TMEM_COLS = (BN + STAGES * A_COLS) <= 256 ? 256 : 512;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-align the dynamic shared memory base
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* sB = smem;                                        // STAGES x B_BYTES
+  uint8_t* sW = sB + STAGES * B_BYTES;                       // STAGES x W_BYTES
+  __half* sScale = reinterpret_cast<__half*>(sW + STAGES * W_BYTES);   // [BM][groups]
+  const int kb_begin = blockIdx.z * a.kblocks_per_split;
+  const int nkb = a.kblocks_per_split;
+  const int groups = (nkb * BK + a.G - 1) / a.G;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sScale + BM * groups + 8);
+  bars = reinterpret_cast<uint64_t*>(((uintptr_t)bars + 7) & ~(uintptr_t)7);
+  uint64_t* full = bars;                 // TMA landed
+  uint64_t* empty = bars + STAGES;       // MMA done with the stage
+  uint64_t* afull = bars + 2 * STAGES;   // A stage written to TMEM
+  uint64_t* accb = bars + 3 * STAGES;    // accumulator complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+  int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * BM;
+  const int t0 = blockIdx.y * BN;
+  const bool second = m0 >= a.n_split;
+  const CUtensorMap* map_w = second ? &map_w1 : &map_w0;
+  const int wrow0 = second ? m0 - a.n_split : m0;
+  const __half* scales = second ? a.s1 : a.s0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 4);
+    }
+    mbar_init(accb, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(map_w) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  // scales of this CTA's rows and k range -> shared memory
+  {
+    const int gpr = a.K / a.G;
+    const int g0 = (kb_begin * BK) / a.G;
+    for (int i = threadIdx.x; i < BM * groups; i += THREADS) {
+      int r = i / groups, g = i % groups;
+      sScale[r * groups + g] =
+          g0 + g < gpr ? scales[(size_t)(wrow0 + r) * gpr + g0 + g] : __float2half_rn(0.f);
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t acc_col = 0;
+  const uint32_t a_col0 = BN;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA
+    if (lane == 0) {
+      int issued = 0;
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % STAGES;
+        if (i >= STAGES) {
+          if (!mbar_wait(&empty[s], ((i / STAGES) - 1) & 1)) {
+            atomicExch(abort_flag, 1);
+            break;
+          }
+        }
+        if (*(volatile int*)abort_flag) break;
+        mbar_expect_tx(&full[s], B_BYTES + W_BYTES);
+        const int kb = kb_begin + i;
+        tma_load_2d(sB + s * B_BYTES, &map_x, kb * BK, t0, &full[s]);
+        tma_load_2d(sW + s * W_BYTES, map_w, kb * (BK / 8), wrow0, &full[s]);
+        issued = i + 1;
+      }
+      // on abort, let every copy already issued land before the CTA exits
+      if (*(volatile int*)abort_flag) {
+        for (int i = 0; i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA
+    if (lane == 0) {
+      const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      bool ok = true;
+      for (int i = 0; i < nkb && ok; ++i) {
+        const int s = i % STAGES;
+        if (!mbar_wait(&full[s], (i / STAGES) & 1) || !mbar_wait(&afull[s], (i / STAGES) & 1) ||
+            *(volatile int*)abort_flag) {
+          atomicExch(abort_flag, 1);
+          ok = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_BYTES));
+        const uint32_t a_tm = tmem_base + a_col0 + s * A_COLS;
+#pragma unroll
+        for (int j = 0; j < BK / 16; ++j)
+          mma_ts(tmem_base + acc_col, a_tm + j * 8, bdesc + (uint64_t)(2 * j), idesc,
+                 (i > 0 || j > 0) ? 1u : 0u);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(accb);   // arrives once all issued MMAs are complete
+    }
+  } else if (warp >= 4) {
+    // ---------------------------------------------------------------- dequant + epilogue
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;             // weight row within the tile = TMEM lane
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % STAGES;
+      if (!mbar_wait(&full[s], (i / STAGES) & 1) || *(volatile int*)abort_flag) {
+        atomicExch(abort_flag, 1);
+        break;
+      }
+      const uint4* wp = reinterpret_cast<const uint4*>(sW + s * W_BYTES + r * 32);
+      const uint4 wa = wp[0], wb = wp[1];
+      const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+      const int g = ((kb_begin + i) * BK) / a.G - (kb_begin * BK) / a.G;
+      const __half sc = sScale[r * groups + g];
+      const __half2 s2 = __halves2half2(sc, sc);
+      uint32_t v[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const uint32_t b = c & 3;
+        const uint32_t sel = b | 0x40u | (b << 8) | 0x4000u;
+        uint32_t code = dequant_code_pair(words[c >> 2], sel);
+        __half2 wv = __hmul2(*reinterpret_cast<__half2*>(&code), s2);
+        v[c] = *reinterpret_cast<uint32_t*>(&wv);
+      }
+      const uint32_t taddr = tmem_base + lane_addr + a_col0 + s * A_COLS;
+      asm volatile(
+          "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+          "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+          "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+          "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+          "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+          "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+          "r"(v[29]), "r"(v[30]), "r"(v[31])
+          : "memory");
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[s]);
+    }
+    // epilogue: accumulator rows = weight rows, columns = tokens
+    const bool ok = mbar_wait(accb, 0) && !*(volatile int*)abort_flag;
+    if (!ok) atomicExch(abort_flag, 1);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (ok) {
+      float* out = a.part + (size_t)blockIdx.z * a.T * a.N + (size_t)(m0 + r);
+#pragma unroll 1
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        if (t0 + cc * 32 >= a.T) break;   // warp-uniform
+        uint32_t u[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+            "%27, %28, %29, %30, %31}, [%32];"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+              "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+              "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
+              "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
+              "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
+              "=r"(u[31])
+            : "r"(tmem_base + lane_addr + acc_col + cc * 32));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int t = t0 + cc * 32 + e;
+          if (t < a.T) out[(size_t)t * a.N] = __uint_as_float(u[e]);
+        }
+      }
+    }
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+  __syncthreads();
+  if (*(volatile int*)abort_flag && threadIdx.x == 0 && a.status)
+    atomicCAS(a.status, 0, kDevTimeout);
+  if (warp == 1) {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+tl_status get_encoder() {
+  if (g_encode) return ok();
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return set_error(TL_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
+  g_encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+  return ok();
+}
+
+tl_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                    uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+                    CUtensorMapSwizzle swz) {
+  TL_TRY(get_encoder());
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return set_error(TL_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return ok();
+}
+
+int tc_tile_n(int T) {
+  if (T >= 256) return 256;
+  return T <= 64 ? 64 : 128;
+}
+
+template <int BN>
+size_t tc_smem_bytes(int kblocks_per_split, int G) {
+  int groups = (kblocks_per_split * BK + G - 1) / G + 1;
+  return 1024 + (size_t)STAGES * (BN * 128 + BM * 32) + (size_t)BM * groups * 2 + 16 +
+         (4 * STAGES + 1) * 8 + 16;
+}
+
+template <int BN>
+tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
+  CUtensorMap mx, mw0, mw1;
+  TL_TRY(encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.x, g.K, g.T, (uint64_t)g.K * 2, BK, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B));
+  const int n1 = g.n_split, n2 = g.N - g.n_split;
+  TL_TRY(encode_2d(&mw0, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w0, g.K / 8, n1, (uint64_t)g.K / 8 * 4,
+                   BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE));
+  if (n2 > 0) {
+    TL_TRY(encode_2d(&mw1, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w1, g.K / 8, n2,
+                     (uint64_t)g.K / 8 * 4, BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE));
+  } else {
+    mw1 = mw0;
+  }
+  TcArgs a;
+  a.N = g.N;
+  a.K = g.K;
+  a.G = g.G;
+  a.T = g.T;
+  a.n_split = g.n_split;
+  a.kblocks_per_split = (g.K / BK) / g.splits;
+  a.s0 = g.s0;
+  a.s1 = g.s1;
+  a.part = g.part;
+  a.status = g.status;
+  const size_t smem = tc_smem_bytes<BN>(a.kblocks_per_split, g.G);
+  dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
+  gemm_w4_tc_kernel<BN><<<grid, THREADS, smem, s>>>(mx, mw0, mw1, a);
+  TL_LAUNCH_CHECK();
+  return ok();
+}
+
+}  // namespace
+
+// One-time set-up (driver entry point, shared-memory limit); called outside
+// any stream capture.
+tl_status gemm_tc_init() {
+  static bool done = false;
+  if (done) return ok();
+  TL_TRY(get_encoder());
+  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               232448));
+  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<256>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+  done = true;
+  return ok();
+}
+
+// Split-K factor for the tensor-core kernel: enough CTAs to cover the SMs
+// once, at least 4 k blocks per split.
+int gemm_tc_splits(int N, int K, int T) {
+  const int nkb = K / BK;
+  const int tiles = (N / BM) * ((T + tc_tile_n(T) - 1) / tc_tile_n(T));
+  int s = 1;
+  while (tiles * s < 148 && s * 2 <= 16 && nkb % (s * 2) == 0 && nkb / (s * 2) >= 4) s *= 2;
+  return s;
+}
+
+bool gemm_tc_eligible(int N, int K, int T) { return T >= 64 && N % BM == 0 && K % BK == 0; }
+
+tl_status launch_gemm_tc(const GemmArgs& g, cudaStream_t s) {
+  if (g.T == 0) return ok();
+  if (g.n_split % BM != 0)
+    return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs row split %% 128 == 0");
+  const int bn = tc_tile_n(g.T);
+  if (bn == 256) return launch_tc_bn<256>(g, s);
+  if (bn == 128) return launch_tc_bn<128>(g, s);
+  return launch_tc_bn<64>(g, s);
+}
+
+}  // namespace tl

@@ -76,10 +76,20 @@ struct GemmArgs {
   const __half* x;      // fp16 [T][K]
   int T;
   float* part;          // fp32 [S][T][N]
-  int splits;           // S
+  int splits;           // S (from gemm_splits)
+  int* status;          // device status word for bounded-wait timeouts (may be null)
 };
+// Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
+// kernel for T >= 64, the mma.sync register-dequant kernel below that.
 int gemm_splits(int N, int K, int T);
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s);
+// the two kernels
+int gemm_mma_splits(int N, int K, int T);
+tl_status launch_gemm_mma(const GemmArgs& a, cudaStream_t s);
+bool gemm_tc_eligible(int N, int K, int T);
+int gemm_tc_splits(int N, int K, int T);
+tl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t s);
+tl_status gemm_tc_init();
 // y[t][n] = sum_{s < S} part[s][t][n], in order s = 0, 1, ...
 tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s);
 
