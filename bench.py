@@ -335,9 +335,9 @@ def run_ours(args, rank, world, dist):
     achieved = flops * k_gemm / t_gemm / 1e12
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16_tflops"],
             "unit": "TFLOP/s", "frac": round(achieved / pk["bf16_tflops"], 4),
-            "traffic": ncu_traffic("gemm_w4_mma_gateup_T128.txt",
-                                   ["weight_shared_looped_b200/csrc/gemm_mma.cu"]),
-            "kernel": "gemm_w4_mma_kernel<64> (gate|up, N 16384, K 2048, T 128; cold L2)",
+            "traffic": ncu_traffic("gemm_w4_tc_gateup_T128.md",
+                                   ["weight_shared_looped_b200/csrc/gemm_tc.cu"]),
+            "kernel": "gemm_w4_tc_kernel<128> (gate|up, N 16384, K 2048, T 128; cold L2)",
             "peak_kind": f"bf16 dense burst, {pk['source']} (fp16 operands run at the same rate)",
             "us_per_launch": round(t_gemm / k_gemm * 1e6, 2),
             "forward_tflops": round(172.5e9 * args.steps / (t / world) / 1e12, 2),

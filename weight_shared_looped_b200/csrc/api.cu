@@ -106,6 +106,8 @@ struct tl_model {
   __half *q, *k, *v;
   __half* u;
   float* part;
+  float* part2;          // decode: gate|up partials read by the down projection
+  int* attn_counters;    // decode: merge tickets [kMaxLanes][H], zero between launches
   float* y;
   int32_t* lane_map;
   float* dec_scratch;
@@ -329,6 +331,10 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
   void* p_u; void* p_part; void* p_y; void* p_lid; void* p_dec; void* p_status; void* p_rope;
+  void* p_part2; void* p_ctr;
+  size_t part2_floats = 0;
+  for (int t = 1; t <= md.max_lanes; ++t)
+    part2_floats = std::max(part2_floats, (size_t)gemm_splits(2 * F, d, t) * t * 2 * F);
   Slot slots[] = {
       {&p_ids, (size_t)T * 4},
       {&p_hin, (size_t)T * d * 2},
@@ -340,6 +346,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_v, (size_t)T * d * 2},
       {&p_u, (size_t)T * F * 2},
       {&p_part, maxpart * 4},
+      {&p_part2, part2_floats * 4},
+      {&p_ctr, (size_t)kMaxLanes * m->H * 4},
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
       {&p_dec, (size_t)kMaxLanes * m->H * m->max_chunks * (m->hd + 2) * 4},
@@ -366,6 +374,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->v = (__half*)p_v;
   m->u = (__half*)p_u;
   m->part = (float*)p_part;
+  m->part2 = (float*)p_part2;
+  m->attn_counters = (int*)p_ctr;
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
   m->dec_scratch = (float*)p_dec;
@@ -387,6 +397,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
                                 cudaMemcpyHostToDevice);
     cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
+    if (e3 == cudaSuccess) e3 = cudaMemset(m->attn_counters, 0, (size_t)kMaxLanes * m->H * 4);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
       return set_error(TL_ERR_CUDA, "model initialisation copy failed");
@@ -636,38 +647,35 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   // QKV
   GemmArgs g = gemm_args(m, b, 0, m->x, rows);
   TL_TRY(launch_gemm(g, s));
-  RopeKvArgs r;
-  memset(&r, 0, sizeof(r));
-  r.part = m->part;
-  r.S = g.splits;
-  r.rows = rows;
-  r.d = m->d;
-  r.H = m->H;
-  r.hd = m->hd;
-  r.rope_cs = m->rope;
-  r.q = m->q;
-  r.k = decode ? nullptr : m->k;
-  r.v = decode ? nullptr : m->v;
-  if (kv) {
-    r.kv_base = kv->buffer + kKvHeaderBytes;
-    r.hdr = (const KvHeader*)kv->buffer;
-    r.layer_bytes = kv->layer_bytes;
-    r.kv_region_bytes = kv->region_bytes;
-    r.layer = layer;
-    r.max_ctx = kv->max_ctx;
-    r.kv_int8 = kv->dtype == TL_KV_INT8;
-  }
-  r.lane_of_row = lane_of_row;
-  r.lane = lane;
-  r.decode = decode ? 1 : 0;
-  TL_TRY(launch_rope_kv(r, s));
-  // attention
   if (!decode) {
+    RopeKvArgs r;
+    memset(&r, 0, sizeof(r));
+    r.part = m->part;
+    r.S = g.splits;
+    r.rows = rows;
+    r.d = m->d;
+    r.H = m->H;
+    r.hd = m->hd;
+    r.rope_cs = m->rope;
+    r.q = m->q;
+    r.k = m->k;
+    r.v = m->v;
+    if (kv) {
+      r.kv_base = kv->buffer + kKvHeaderBytes;
+      r.hdr = (const KvHeader*)kv->buffer;
+      r.layer_bytes = kv->layer_bytes;
+      r.kv_region_bytes = kv->region_bytes;
+      r.layer = layer;
+      r.max_ctx = kv->max_ctx;
+      r.kv_int8 = kv->dtype == TL_KV_INT8;
+    }
+    r.lane = lane;
+    TL_TRY(launch_rope_kv(r, s));
     TL_TRY(launch_attn_prefill(m->q, m->k, m->v, m->attn, rows, m->H, m->hd, s));
   } else {
+    // RoPE, KV append, split attention and merge in one launch
     DecodeAttnArgs da;
     memset(&da, 0, sizeof(da));
-    da.q = m->q;
     da.out = m->attn;
     da.rows = rows;
     da.H = m->H;
@@ -683,7 +691,11 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     da.lane_of_row = lane_of_row;
     da.scratch = m->dec_scratch;
     da.max_chunks = (kv->max_ctx + kDecodeChunk - 1) / kDecodeChunk;
-    TL_TRY(launch_attn_decode(da, s));
+    da.qkv_part = m->part;
+    da.qkv_S = g.splits;
+    da.rope_cs = m->rope;
+    da.counters = m->attn_counters;
+    TL_TRY(launch_attn_decode_fused(da, s));
   }
   // O projection, residual, RMSNorm before the MLP
   g = gemm_args(m, b, 1, m->attn, rows);
@@ -699,10 +711,22 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   TL_TRY(launch_residual_norm(n, s));
   // SwiGLU MLP
   g = gemm_args(m, b, 2, m->x, rows);
-  TL_TRY(launch_gemm(g, s));
-  TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
-  g = gemm_args(m, b, 3, m->u, rows);
-  TL_TRY(launch_gemm(g, s));
+  if (decode) {
+    // gate|up partials go to their own buffer; the down projection's
+    // activation staging forms silu(gate) * up from them
+    g.part = m->part2;
+    TL_TRY(launch_gemm(g, s));
+    GemmArgs dn = gemm_args(m, b, 3, m->u, rows);
+    dn.x_part = m->part2;
+    dn.x_S = g.splits;
+    dn.x_F = m->F;
+    TL_TRY(launch_gemm(dn, s));
+  } else {
+    TL_TRY(launch_gemm(g, s));
+    TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
+    g = gemm_args(m, b, 3, m->u, rows);
+    TL_TRY(launch_gemm(g, s));
+  }
   return ok();
 }
 

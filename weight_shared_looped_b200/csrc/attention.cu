@@ -27,100 +27,178 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // ------------------------------------------------------------------ prefill
-constexpr int PQ = 16;     // queries per CTA (4 warps x 4)
-constexpr int PK = 64;     // keys per tile
+// Tensor cores (mma.sync m16n8k16, fp16 in, fp32 accumulate): each warp
+// owns 16 queries; S = Q K^T and O += P V run on the tensor cores with the
+// score fragment reused in registers as the A operand of P V; V fragments come
+// from shared memory through ldmatrix.trans.  Online softmax in base 2 with
+// the 1/sqrt(hd) scale folded into log2(e).
+constexpr int FQ = 64;   // queries per CTA (4 warps x 16)
+constexpr int FK = 64;   // keys per tile
+
+__device__ __forceinline__ void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
 template <int HD>
-__global__ void __launch_bounds__(128) attn_prefill_kernel(const __half* __restrict__ q,
-                                                           const __half* __restrict__ k,
-                                                           const __half* __restrict__ v,
-                                                           __half* __restrict__ out, int T,
-                                                           int H, float scale) {
-  __shared__ __align__(16) __half Ks[PK][HD + 2];
-  __shared__ __align__(16) __half Vs[PK][HD + 8];
-  __shared__ float Qs[PQ][HD];
+__global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __restrict__ q,
+                                                              const __half* __restrict__ k,
+                                                              const __half* __restrict__ v,
+                                                              __half* __restrict__ out, int T,
+                                                              int H, float scale_log2) {
+  constexpr int LD = HD + 8;                 // halves per smem row (16-byte aligned, no conflicts)
+  __shared__ __align__(16) __half Ks[FK][LD];
+  __shared__ __align__(16) __half Vs[FK][LD];
   const int head = blockIdx.y;
-  const int q0 = blockIdx.x * PQ;
+  const int q0 = blockIdx.x * FQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
   const int d = H * HD;
-  constexpr int DPL = HD / 32;   // output dims per lane
+  const int qw = q0 + warp * 16;             // first query of this warp
+  constexpr int KS = HD / 16;                // k steps over head_dim
+  constexpr int NT = HD / 8;                 // output n tiles over head_dim
 
-  for (int i = threadIdx.x; i < PQ * HD; i += 128) {
-    int r = i / HD, e = i % HD;
-    int t = q0 + r;
-    Qs[r][e] = t < T ? __half2float(q[(size_t)t * d + head * HD + e]) * scale : 0.f;
-  }
-  float m[4], l[4], acc[4][DPL];
+  // Q fragments (A operand, 16 x HD), rows qw+g and qw+g+8
+  uint32_t qa[KS][4];
+  {
+    const int r0 = qw + g, r1 = qw + g + 8;
 #pragma unroll
-  for (int qi = 0; qi < 4; ++qi) {
-    m[qi] = -INFINITY;
-    l[qi] = 0.f;
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[qi][e] = 0.f;
+    for (int ks = 0; ks < KS; ++ks) {
+      const int c = ks * 16 + 2 * t;
+      auto ld = [&](int r, int col) -> uint32_t {
+        if (r >= T) return 0u;
+        return *reinterpret_cast<const uint32_t*>(q + (size_t)r * d + head * HD + col);
+      };
+      qa[ks][0] = ld(r0, c);
+      qa[ks][1] = ld(r1, c);
+      qa[ks][2] = ld(r0, c + 8);
+      qa[ks][3] = ld(r1, c + 8);
+    }
   }
-  const int q_last = min(q0 + PQ, T) - 1;   // highest query position in this CTA
-  for (int k0 = 0; k0 <= q_last; k0 += PK) {
+  float o[NT][4];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  const int q_hi = min(q0 + FQ, T) - 1;
+  for (int k0 = 0; k0 <= q_hi; k0 += FK) {
     __syncthreads();
-    for (int i = threadIdx.x; i < PK * (HD / 2); i += 128) {
-      int r = i / (HD / 2), e2 = (i % (HD / 2)) * 2;
-      int t = k0 + r;
-      __half2 kk = __float2half2_rn(0.f), vv = __float2half2_rn(0.f);
-      if (t < T) {
-        kk = *reinterpret_cast<const __half2*>(k + (size_t)t * d + head * HD + e2);
-        vv = *reinterpret_cast<const __half2*>(v + (size_t)t * d + head * HD + e2);
+    for (int i = threadIdx.x; i < FK * (HD / 8); i += 128) {
+      const int r = i / (HD / 8), c = (i % (HD / 8)) * 8;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
+      if (k0 + r < T) {
+        kv = *reinterpret_cast<const uint4*>(k + (size_t)(k0 + r) * d + head * HD + c);
+        vv = *reinterpret_cast<const uint4*>(v + (size_t)(k0 + r) * d + head * HD + c);
       }
-      *reinterpret_cast<__half2*>(&Ks[r][e2]) = kk;
-      *reinterpret_cast<__half2*>(&Vs[r][e2]) = vv;
+      *reinterpret_cast<uint4*>(&Ks[r][c]) = kv;
+      *reinterpret_cast<uint4*>(&Vs[r][c]) = vv;
     }
     __syncthreads();
+    if (k0 > qw + 15) continue;              // this warp's queries all precede the tile
+    // S = Q K^T : 16 x 64
+    float sc[FK / 8][4];
 #pragma unroll
-    for (int qi = 0; qi < 4; ++qi) {
-      const int qr = warp * 4 + qi;
-      const int qpos = q0 + qr;
-      if (qpos >= T) continue;   // warp-uniform
-      float s[2];
+    for (int nt = 0; nt < FK / 8; ++nt) {
+      sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int j = lane + 32 * jj;
-        float dot = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < HD; e += 2) {
-          float2 kf = __half22float2(*reinterpret_cast<const __half2*>(&Ks[j][e]));
-          dot = fmaf(Qs[qr][e], kf.x, dot);
-          dot = fmaf(Qs[qr][e + 1], kf.y, dot);
-        }
-        s[jj] = (k0 + j <= qpos) ? dot : -INFINITY;
+      for (int ks = 0; ks < KS; ++ks) {
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(&Ks[nt * 8 + g][ks * 16 + 2 * t]);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(&Ks[nt * 8 + g][ks * 16 + 2 * t + 8]);
+        mma_f16(sc[nt], qa[ks], b0, b1);
       }
-      float mt = warp_max(fmaxf(s[0], s[1]));
-      float m_new = fmaxf(m[qi], mt);
-      float corr = __expf(m[qi] - m_new);
-      float p0 = __expf(s[0] - m_new), p1 = __expf(s[1] - m_new);
-      l[qi] = l[qi] * corr + warp_sum(p0 + p1);
-      m[qi] = m_new;
+    }
+    // causal mask (key index > query index) and running max
+    const int r0 = qw + g, r1 = qw + g + 8;
+    float mx0 = m0, mx1 = m1;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[qi][e] *= corr;
-      const int jmax = min(PK, qpos - k0 + 1);
-      for (int j = 0; j < jmax; ++j) {
-        float pj = __shfl_sync(0xffffffffu, j < 32 ? p0 : p1, j & 31);
+    for (int nt = 0; nt < FK / 8; ++nt) {
 #pragma unroll
-        for (int e = 0; e < DPL; e += 2) {
-          float2 vf = __half22float2(*reinterpret_cast<const __half2*>(&Vs[j][lane * DPL + e]));
-          acc[qi][e] = fmaf(pj, vf.x, acc[qi][e]);
-          acc[qi][e + 1] = fmaf(pj, vf.y, acc[qi][e + 1]);
-        }
+      for (int e = 0; e < 2; ++e) {
+        const int key = k0 + nt * 8 + 2 * t + e;
+        float s0 = sc[nt][e] * scale_log2, s1 = sc[nt][2 + e] * scale_log2;
+        if (key > r0 || key >= T) s0 = -INFINITY;
+        if (key > r1 || key >= T) s1 = -INFINITY;
+        sc[nt][e] = s0;
+        sc[nt][2 + e] = s1;
+        mx0 = fmaxf(mx0, s0);
+        mx1 = fmaxf(mx1, s1);
+      }
+    }
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    // rows past T have no valid key at all: keep their state finite
+    const float base0 = mx0 == -INFINITY ? 0.f : mx0;
+    const float base1 = mx1 == -INFINITY ? 0.f : mx1;
+    const float corr0 = exp2f(m0 - base0), corr1 = exp2f(m1 - base1);
+    m0 = mx0;
+    m1 = mx1;
+    float ps0 = 0.f, ps1 = 0.f;
+    uint32_t pa[FK / 16][4];
+#pragma unroll
+    for (int nt = 0; nt < FK / 8; ++nt) {
+      const float p00 = exp2f(sc[nt][0] - base0), p01 = exp2f(sc[nt][1] - base0);
+      const float p10 = exp2f(sc[nt][2] - base1), p11 = exp2f(sc[nt][3] - base1);
+      ps0 += p00 + p01;
+      ps1 += p10 + p11;
+      const int kk = nt >> 1;
+      if ((nt & 1) == 0) {
+        pa[kk][0] = pack_half2(p00, p01);
+        pa[kk][1] = pack_half2(p10, p11);
+      } else {
+        pa[kk][2] = pack_half2(p00, p01);
+        pa[kk][3] = pack_half2(p10, p11);
+      }
+    }
+    l0 = l0 * corr0 + ps0;
+    l1 = l1 * corr1 + ps1;
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      o[i][0] *= corr0;
+      o[i][1] *= corr0;
+      o[i][2] *= corr1;
+      o[i][3] *= corr1;
+    }
+    // O += P V
+#pragma unroll
+    for (int kk = 0; kk < FK / 16; ++kk) {
+#pragma unroll
+      for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
+        // four 8x8 tiles: keys kk*16 + {0..7, 8..15} x dims nt2*16 + {0..7, 8..15}
+        const int mi = lane >> 3, ri = lane & 7;
+        const __half* src = &Vs[kk * 16 + (mi & 1) * 8 + ri][nt2 * 16 + (mi >> 1) * 8];
+        uint32_t b0, b1, b2, b3;
+        asm volatile(
+            "ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+            : "=r"(b0), "=r"(b1), "=r"(b2), "=r"(b3)
+            : "r"((uint32_t)__cvta_generic_to_shared(src)));
+        mma_f16(o[2 * nt2], pa[kk], b0, b1);
+        mma_f16(o[2 * nt2 + 1], pa[kk], b2, b3);
       }
     }
   }
+  // row sums across the quad, normalise, store
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const int r0 = qw + g, r1 = qw + g + 8;
+  const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
 #pragma unroll
-  for (int qi = 0; qi < 4; ++qi) {
-    const int qpos = q0 + warp * 4 + qi;
-    if (qpos >= T) continue;
-    const float inv = 1.0f / l[qi];
-#pragma unroll
-    for (int e = 0; e < DPL; e += 2) {
-      __half2 o = __floats2half2_rn(acc[qi][e] * inv, acc[qi][e + 1] * inv);
-      *reinterpret_cast<__half2*>(out + (size_t)qpos * d + head * HD + lane * DPL + e) = o;
-    }
+  for (int nt = 0; nt < NT; ++nt) {
+    const int c = head * HD + nt * 8 + 2 * t;
+    if (r0 < T)
+      *reinterpret_cast<uint32_t*>(out + (size_t)r0 * d + c) = pack_half2(o[nt][0] * i0, o[nt][1] * i0);
+    if (r1 < T)
+      *reinterpret_cast<uint32_t*>(out + (size_t)r1 * d + c) = pack_half2(o[nt][2] * i1, o[nt][3] * i1);
   }
 }
 
@@ -237,19 +315,233 @@ __global__ void __launch_bounds__(HD) attn_decode_merge_kernel(DecodeAttnArgs a)
   a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
 }
 
+// Fused decode attention for one (row, head, 64-key chunk):
+//   * q = sum of the QKV split-K partials, RoPE at the lane's position;
+//   * the CTA holding the lane's newest position also forms k and v, applies
+//     RoPE to k and appends both to the cache (fp16, or INT8 codes + fp16 scale
+//     per (token, head)); positions before it are only read;
+//   * scores, max-subtracted exponentials and the weighted V sum of the chunk
+//     go to scratch; the last CTA of the (row, head) to finish (an atomic
+//     ticket, no waiting) merges all chunks in chunk order and writes the
+//     output, then resets the ticket for the next launch.
+template <int HD>
+__global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a) {
+  constexpr int DPL = HD / 32;
+  constexpr int HALF = HD / 2;
+  __shared__ float qs[HD], kn[HD], vn[HD];
+  __shared__ float sc[kDecodeChunk];
+  __shared__ float wacc[4][HD];
+  __shared__ float wl[4];
+  __shared__ float red[4];
+  __shared__ int is_last;
+  const int chunk = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
+  const int lane_id = a.lane_of_row[row];
+  const int pos = a.hdr->pos[lane_id];
+  const int n_keys = pos + 1;
+  const int n_chunks = (n_keys + kDecodeChunk - 1) / kDecodeChunk;
+  if (chunk >= n_chunks) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool owner = chunk == n_chunks - 1;    // holds position pos
+  const size_t split_stride = (size_t)a.rows * 3 * a.d;
+  const float* prow = a.qkv_part + (size_t)row * 3 * a.d + (size_t)head * HD;
+
+  // q (and k, v for the owner) from the partial sums
+  for (int i = threadIdx.x; i < HD; i += 128) {
+    float sq = 0.f, sk = 0.f, sv = 0.f;
+    for (int sp = 0; sp < a.qkv_S; ++sp) {
+      const float* p = prow + sp * split_stride;
+      sq += p[i];
+      if (owner) {
+        sk += p[a.d + i];
+        sv += p[2 * a.d + i];
+      }
+    }
+    qs[i] = sq;
+    kn[i] = sk;
+    vn[i] = sv;
+  }
+  __syncthreads();
+  float qr = 0.f, kr = 0.f;
+  const int i = threadIdx.x;
+  if (i < HD) {
+    const float2 cs = a.rope_cs[(size_t)pos * HALF + (i % HALF)];
+    if (i < HALF) {
+      qr = qs[i] * cs.x - qs[i + HALF] * cs.y;
+      kr = kn[i] * cs.x - kn[i + HALF] * cs.y;
+    } else {
+      qr = qs[i] * cs.x + qs[i - HALF] * cs.y;
+      kr = kn[i] * cs.x + kn[i - HALF] * cs.y;
+    }
+  }
+  __syncthreads();
+  const char* layer_c =
+      a.kv_base + (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
+  char* layer = const_cast<char*>(layer_c);
+  const size_t head_off = (size_t)head * a.max_ctx;
+  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
+  if (i < HD) {
+    // the query is rounded to fp16 as in the unfused path
+    qs[i] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
+  }
+  if (owner) {
+    // append k (after RoPE) and v at position pos
+    const __half kh = __float2half_rn(kr);
+    const __half vh = __float2half_rn(i < HD ? vn[i] : 0.f);
+    if (!a.kv_int8) {
+      if (i < HD) {
+        reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + i] = kh;
+        reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = vh;
+      }
+    } else {
+      float km = i < HD ? fabsf(__half2float(kh)) : 0.f;
+      float vm = i < HD ? fabsf(__half2float(vh)) : 0.f;
+      km = warp_max(km);
+      vm = warp_max(vm);
+      if (lane == 0) {
+        red[warp] = km;
+        wl[warp] = vm;
+      }
+      __syncthreads();
+      km = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+      vm = fmaxf(fmaxf(wl[0], wl[1]), fmaxf(wl[2], wl[3]));
+      const __half ksh = __float2half_rn(__fdiv_rn(km, 127.0f));
+      const __half vsh = __float2half_rn(__fdiv_rn(vm, 127.0f));
+      const float ks = __half2float(ksh), vs = __half2float(vsh);
+      if (i < HD) {
+        const float kx = __half2float(kh), vx = __half2float(vh);
+        const int kc = ks == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ks)), -127.f), 127.f);
+        const int vc = vs == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vs)), -127.f), 127.f);
+        reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + i] = (int8_t)kc;
+        reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = (int8_t)vc;
+      }
+      if (i == 0) {
+        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
+        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] =
+            vsh;
+      }
+    }
+  }
+  __syncthreads();   // the appended entry and qs are visible to the whole CTA
+
+  const __half* ksc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
+  const __half* vsc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
+  auto load_row = [&](int which, int p, float* out) {
+    const size_t eoff = (head_off + p) * HD + lane * DPL;
+    if (!a.kv_int8) {
+      const __half* src = reinterpret_cast<const __half*>(layer + which * a.kv_region_bytes) + eoff;
+#pragma unroll
+      for (int e = 0; e < DPL; e += 2) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(src + e));
+        out[e] = f.x;
+        out[e + 1] = f.y;
+      }
+    } else {
+      const int8_t* src = reinterpret_cast<const int8_t*>(layer + which * a.kv_region_bytes) + eoff;
+      const float sc_ = __half2float((which == 0 ? ksc : vsc)[head_off + p]);
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) out[e] = (float)src[e] * sc_;
+    }
+  };
+  float qv[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) qv[e] = qs[lane * DPL + e];
+  const int base = chunk * kDecodeChunk;
+  for (int j0 = 0; j0 < kDecodeChunk / 4; ++j0) {
+    const int j = warp * (kDecodeChunk / 4) + j0;
+    const int p = base + j;
+    float sv = -INFINITY;
+    if (p < n_keys) {
+      float kr2[DPL];
+      load_row(0, p, kr2);
+      float dot = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) dot = fmaf(qv[e], kr2[e], dot);
+      sv = warp_sum(dot);
+    }
+    if (lane == 0) sc[j] = sv;
+  }
+  __syncthreads();
+  float m = -INFINITY;
+  for (int j = 0; j < kDecodeChunk; ++j) m = fmaxf(m, sc[j]);
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  float lsum = 0.f;
+  for (int j0 = 0; j0 < kDecodeChunk / 4; ++j0) {
+    const int j = warp * (kDecodeChunk / 4) + j0;
+    const int p = base + j;
+    if (p >= n_keys) break;
+    const float pr = __expf(sc[j] - m);
+    lsum += pr;
+    float vr[DPL];
+    load_row(1, p, vr);
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pr, vr[e], acc[e]);
+  }
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
+  if (lane == 0) wl[warp] = lsum;
+  __syncthreads();
+  float* part = a.scratch + ((size_t)row * a.H + head) * a.max_chunks * (HD + 2);
+  float* dst = part + (size_t)chunk * (HD + 2);
+  for (int e = threadIdx.x; e < HD; e += 128)
+    dst[e] = wacc[0][e] + wacc[1][e] + wacc[2][e] + wacc[3][e];
+  if (threadIdx.x == 0) {
+    dst[HD] = m;
+    dst[HD + 1] = wl[0] + wl[1] + wl[2] + wl[3];
+  }
+  // last CTA of this (row, head) merges
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* ctr = a.counters + (size_t)lane_id * a.H + head;
+    const int ticket = atomicAdd(ctr, 1);
+    is_last = ticket == n_chunks - 1;
+    if (is_last) *ctr = 0;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  float M = -INFINITY;
+  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, __ldcg(part + (size_t)c * (HD + 2) + HD));
+  for (int e = threadIdx.x; e < HD; e += 128) {
+    float L = 0.f, o = 0.f;
+    for (int c = 0; c < n_chunks; ++c) {
+      const float* pc = part + (size_t)c * (HD + 2);
+      const float w = __expf(__ldcg(pc + HD) - M);
+      L = fmaf(__ldcg(pc + HD + 1), w, L);
+      o = fmaf(__ldcg(pc + e), w, o);
+    }
+    a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
+  }
+}
+
 }  // namespace
 
 tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
                               int T, int H, int hd, cudaStream_t s) {
   if (T == 0) return ok();
-  dim3 grid((T + PQ - 1) / PQ, H);
-  const float scale = 1.0f / sqrtf((float)hd);
+  dim3 grid((T + FQ - 1) / FQ, H);
+  const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
   if (hd == 128)
-    attn_prefill_kernel<128><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale);
+    attn_prefill_tc_kernel<128><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale_log2);
   else if (hd == 64)
-    attn_prefill_kernel<64><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale);
+    attn_prefill_tc_kernel<64><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale_log2);
   else
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", hd);
+  TL_LAUNCH_CHECK();
+  return ok();
+}
+
+tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
+  if (a.rows == 0) return ok();
+  dim3 grid(a.max_chunks, a.H, a.rows);
+  if (a.hd == 128)
+    attn_decode_fused_kernel<128><<<grid, 128, 0, s>>>(a);
+  else if (a.hd == 64)
+    attn_decode_fused_kernel<64><<<grid, 128, 0, s>>>(a);
+  else
+    return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
   TL_LAUNCH_CHECK();
   return ok();
 }

@@ -159,6 +159,156 @@ __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- decode GEMV
+// T <= 8 tokens.  The k order inside the MMA is a free choice as long as A and
+// B use the same one, so each lane owns two whole packed words (16 k) of its
+// two rows per 64-wide chunk: lane (g, t) loads words 2t and 2t+1 of rows g
+// and g+8 (8 distinct bytes each, no duplicate loads).  A word's nibble pairs
+// (i, i+4) come out of one lop3 each after a shift: (w >> 4i) & 0x000F000F |
+// 0x6400_6400 is the fp16 pair (1024 + u_i, 1024 + u_{i+4}), and one HSUB2 of
+// 1032 leaves the exact codes.  The activations are staged once per CTA with
+// every 8-k group stored in the order 0 4 1 5 2 6 3 7, so the matching B pairs
+// are adjacent and one 8-byte shared load feeds a k step.
+constexpr int GV_ROWS = 128;      // 8 warps x 16 rows
+constexpr int GV_THREADS = 256;
+constexpr int GV_BATCH = 8;       // 64-k chunks loaded ahead per batch
+
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
+  uint32_t h;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
+  __half2 r = __hsub2(*reinterpret_cast<__half2*>(&h),
+                      __halves2half2(__float2half_rn(1032.0f), __float2half_rn(1032.0f)));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+
+__global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
+  extern __shared__ __align__(16) __half gv_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int m0 = blockIdx.x * GV_ROWS;
+  const int n_chunks = a.K / KC;
+  const int per = n_chunks / a.splits;
+  const int c0 = blockIdx.z * per;
+  const int krange = per * KC;
+  const int xstride = krange + 4;             // halves; row stride = 2 (mod 32) words
+  __half* xs = gv_smem;                       // [8][xstride], k-permuted
+  const int gpr = a.K / a.G;
+  const int g_lo = (c0 * KC) / a.G;
+  const int n_groups = (krange + a.G - 1) / a.G + 1;
+  __half* ss = xs + 8 * xstride;              // [128][n_groups] scales of this CTA
+
+  // stage x (rows >= T are zero), permuting each 8-k group to 0 4 1 5 2 6 3 7
+  for (int i = threadIdx.x; i < 8 * (krange / 8); i += GV_THREADS) {
+    const int r = i / (krange / 8), q = i % (krange / 8);
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (r < a.T) {
+      if (a.x_part) {
+        // SwiGLU of the gate|up partial sums, rounded to fp16 like the unfused path
+        __half hv[8];
+        const size_t stride = (size_t)a.T * 2 * a.x_F;
+        for (int e = 0; e < 8; ++e) {
+          const size_t kk = (size_t)c0 * KC + q * 8 + e;
+          float gs = 0.f, us = 0.f;
+          for (int sp = 0; sp < a.x_S; ++sp) {
+            const float* p = a.x_part + sp * stride + (size_t)r * 2 * a.x_F;
+            gs += p[kk];
+            us += p[a.x_F + kk];
+          }
+          hv[e] = __float2half_rn(gs / (1.0f + __expf(-gs)) * us);
+        }
+        v = *reinterpret_cast<const uint4*>(hv);
+      } else {
+        v = *reinterpret_cast<const uint4*>(a.x + (size_t)r * a.K + c0 * KC + q * 8);
+      }
+    }
+    const __half* e = reinterpret_cast<const __half*>(&v);
+    __half2 p0 = __halves2half2(e[0], e[4]), p1 = __halves2half2(e[1], e[5]);
+    __half2 p2 = __halves2half2(e[2], e[6]), p3 = __halves2half2(e[3], e[7]);
+    uint2* d = reinterpret_cast<uint2*>(xs + r * xstride + q * 8);   // 8-byte aligned
+    d[0] = make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
+    d[1] = make_uint2(*reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+  }
+  for (int i = threadIdx.x; i < GV_ROWS * n_groups; i += GV_THREADS) {
+    const int r = i / n_groups, gg = i % n_groups;
+    const int row = m0 + r;
+    const __half* sp = row < a.n_split ? a.s0 + (size_t)row * gpr
+                                       : a.s1 + (size_t)(row - a.n_split) * gpr;
+    ss[i] = g_lo + gg < gpr ? sp[g_lo + gg] : __float2half_rn(0.f);
+  }
+
+  const int rowA = m0 + warp * 16 + g;
+  const uint2* wr[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = rowA + 8 * r;
+    const uint32_t* base = row < a.n_split ? a.w0 + (size_t)row * (a.K / 8)
+                                           : a.w1 + (size_t)(row - a.n_split) * (a.K / 8);
+    wr[r] = reinterpret_cast<const uint2*>(base + c0 * 8) + t;   // words 2t, 2t+1 of chunk 0
+  }
+  const __half* srow0 = ss + (warp * 16 + g) * n_groups;
+  const __half* srow1 = srow0 + 8 * n_groups;
+  __syncthreads();
+
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  uint2 cur[GV_BATCH][2], nxt[GV_BATCH][2];
+#pragma unroll
+  for (int b = 0; b < GV_BATCH; ++b) {
+    const bool in = b < per;
+    nxt[b][0] = in ? __ldg(wr[0] + b * 4) : make_uint2(0u, 0u);
+    nxt[b][1] = in ? __ldg(wr[1] + b * 4) : make_uint2(0u, 0u);
+  }
+  for (int cb = 0; cb < per; cb += GV_BATCH) {
+#pragma unroll
+    for (int b = 0; b < GV_BATCH; ++b) {
+      cur[b][0] = nxt[b][0];
+      cur[b][1] = nxt[b][1];
+    }
+#pragma unroll
+    for (int b = 0; b < GV_BATCH; ++b) {
+      const int c = cb + GV_BATCH + b;
+      const bool in = c < per;
+      nxt[b][0] = in ? __ldg(wr[0] + c * 4) : make_uint2(0u, 0u);
+      nxt[b][1] = in ? __ldg(wr[1] + c * 4) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int b = 0; b < GV_BATCH; ++b) {
+      const int c = cb + b;
+      if (c >= per) break;
+      float cacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w0 = (j < 2) ? cur[b][0].x : cur[b][0].y;   // row g
+        const uint32_t w1 = (j < 2) ? cur[b][1].x : cur[b][1].y;   // row g + 8
+        const int sh = (j & 1) * 8;                                  // nibble pairs 0,1 or 2,3
+        uint32_t A[4];
+        A[0] = nib_pair(w0 >> sh);
+        A[1] = nib_pair(w1 >> sh);
+        A[2] = nib_pair(w0 >> (sh + 4));
+        A[3] = nib_pair(w1 >> (sh + 4));
+        const uint2 bx =
+            *reinterpret_cast<const uint2*>(xs + g * xstride + c * KC + 16 * t + 4 * j);
+        mma16816(cacc, A, bx.x, bx.y);
+      }
+      const float s0 = __half2float(srow0[((c0 + c) * KC) / a.G - g_lo]);
+      const float s1 = __half2float(srow1[((c0 + c) * KC) / a.G - g_lo]);
+      acc[0] = fmaf(cacc[0], s0, acc[0]);
+      acc[1] = fmaf(cacc[1], s0, acc[1]);
+      acc[2] = fmaf(cacc[2], s1, acc[2]);
+      acc[3] = fmaf(cacc[3], s1, acc[3]);
+    }
+  }
+  float* out = a.part + (size_t)blockIdx.z * a.T * a.N;
+  const int tk = 2 * t;
+  if (tk < a.T) {
+    out[(size_t)tk * a.N + rowA] = acc[0];
+    out[(size_t)tk * a.N + rowA + 8] = acc[2];
+  }
+  if (tk + 1 < a.T) {
+    out[(size_t)(tk + 1) * a.N + rowA] = acc[1];
+    out[(size_t)(tk + 1) * a.N + rowA + 8] = acc[3];
+  }
+}
+
 __global__ void split_sum_kernel(const float* __restrict__ part, int S, long n,
                                  float* __restrict__ y) {
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -192,11 +342,40 @@ tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStrea
   return ok();
 }
 
+bool gemv_eligible(int N, int K, int T) { return T <= 8 && N % GV_ROWS == 0 && K % KC == 0; }
+
+// Decode split count: each split covers at most 2048 k (the staged activations
+// then fit in 33 KB of shared memory) and at least 4 chunks; splits double
+// until there are two CTAs per SM.  Depends on (N, K) only.
+int gemv_splits(int N, int K) {
+  const int n_chunks = K / KC;
+  int s = 1;
+  while (n_chunks / s > 32 && n_chunks % (2 * s) == 0) s *= 2;
+  while ((N / GV_ROWS) * s < 2 * 148 && n_chunks % (2 * s) == 0 && n_chunks / (2 * s) >= 4) s *= 2;
+  return s;
+}
+
 int gemm_splits(int N, int K, int T) {
+  if (gemv_eligible(N, K, T)) return gemv_splits(N, K);
   return gemm_tc_eligible(N, K, T) ? gemm_tc_splits(N, K, T) : gemm_mma_splits(N, K, T);
 }
 
+tl_status launch_gemv(const GemmArgs& a, cudaStream_t s) {
+  if (a.T == 0) return ok();
+  const int per = (a.K / KC) / a.splits;
+  const int krange = per * KC;
+  const int n_groups = (krange + a.G - 1) / a.G + 1;
+  const size_t smem = (size_t)8 * (krange + 4) * 2 + (size_t)GV_ROWS * n_groups * 2;
+  if (smem > 48 * 1024) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV split too wide");
+  dim3 grid(a.N / GV_ROWS, 1, a.splits);
+  gemv_w4_kernel<<<grid, GV_THREADS, smem, s>>>(a);
+  TL_LAUNCH_CHECK();
+  return ok();
+}
+
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (gemv_eligible(a.N, a.K, a.T)) return launch_gemv(a, s);
+  if (a.x_part) return set_error(TL_ERR_UNSUPPORTED, "SwiGLU staging needs the decode GEMV");
   if (gemm_tc_eligible(a.N, a.K, a.T)) return launch_gemm_tc(a, s);
   return launch_gemm_mma(a, s);
 }

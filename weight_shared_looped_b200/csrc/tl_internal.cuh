@@ -78,6 +78,11 @@ struct GemmArgs {
   float* part;          // fp32 [S][T][N]
   int splits;           // S (from gemm_splits)
   int* status;          // device status word for bounded-wait timeouts (may be null)
+  // decode GEMV only: when x_part is set the activations are
+  // silu(sum_s x_part[s][t][k]) * sum_s x_part[s][t][x_F + k] (SwiGLU of the
+  // gate|up partial sums) instead of x
+  const float* x_part;
+  int x_S, x_F;
 };
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
 // kernel for T >= 64, the mma.sync register-dequant kernel below that.
@@ -150,9 +155,14 @@ tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s);
 tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
                               int T, int H, int hd, cudaStream_t s);
 struct DecodeAttnArgs {
-  const __half* q;           // [rows][d]
+  const __half* q;           // [rows][d] (unfused path)
   __half* out;               // [rows][d]
   int rows, H, hd, d;
+  // fused path: q/k/v from the QKV split-K partials, RoPE, KV append, merge
+  const float* qkv_part;     // [S][rows][3d]
+  int qkv_S;
+  const float2* rope_cs;     // [max_ctx][hd/2]
+  int* counters;             // [kMaxLanes][H], zero between launches
   const char* kv_base;
   const KvHeader* hdr;
   size_t layer_bytes, kv_region_bytes;
@@ -162,5 +172,6 @@ struct DecodeAttnArgs {
   int max_chunks;
 };
 tl_status launch_attn_decode(const DecodeAttnArgs& a, cudaStream_t s);
+tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
 
 }  // namespace tl
