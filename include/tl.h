@@ -281,6 +281,22 @@ tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K
                     int group, const uint16_t* x, int T, float* y,
                     void* workspace, tl_stream stream);
 
+/* tl_linear without a caller workspace, for callers that cannot allocate
+ * device memory while they run (memory reserved up front by another
+ * allocator, work issued inside someone else's open stream capture, fixed
+ * real-time budgets).  The TinyLoop pages have no counterpart of this call.
+ * Same arguments and result as tl_linear minus the workspace: the split-K
+ * partial sums go to a 4 MiB buffer compiled into the library (held on every
+ * GPU that loads it until exit).  Calls needing more than 4 MiB of partial
+ * sums (S * T * N * 4 bytes) return TL_ERR_INVALID_ARG before any launch.
+ * Allocates nothing.  All calls share the buffer, so calls that overlap on the
+ * GPU race; each call overwrites what it reads, so nothing needs clearing.
+ * The first call on a device looks up the buffer's device address; make it
+ * before any stream capture. */
+tl_status tl_linear_noalloc(const uint32_t* packed, const uint16_t* scales, int N,
+                            int K, int group, const uint16_t* x, int T, float* y,
+                            tl_stream stream);
+
 /* Synchronise `stream`, then return and clear the model's device status word
  * (TL_OK, TL_ERR_TIMEOUT or TL_ERR_NUMERIC). */
 tl_status tl_sync_status(tl_model* model, tl_stream stream);

@@ -81,6 +81,7 @@ _SIGS = {
     "tl_sync_status": ([P, P], I),
     "tl_linear_workspace_bytes": ([I, I, I, ctypes.POINTER(SZ)], I),
     "tl_linear": ([P, P, I, I, I, P, I, P, P, P], I),
+    "tl_linear_noalloc": ([P, P, I, I, I, P, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -270,6 +271,12 @@ def tl_linear(packed, scales, N: int, K: int, group: int, x, y, workspace=None,
     T = x.shape[0]
     _check(lib.tl_linear(_ptr(packed), _ptr(scales), N, K, group, _ptr(x), T, _ptr(y),
                          _ptr(workspace), _stream(stream)))
+
+
+def tl_linear_noalloc(packed, scales, N: int, K: int, group: int, x, y, stream=None) -> None:
+    T = x.shape[0]
+    _check(lib.tl_linear_noalloc(_ptr(packed), _ptr(scales), N, K, group, _ptr(x), T, _ptr(y),
+                                 _stream(stream)))
 
 
 def tl_sync_status(model: int, stream=None) -> int:
