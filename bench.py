@@ -206,6 +206,24 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------------------- replicas
+
+def max_over_ranks(t: float, dist, device) -> float:
+    """The slowest rank's time (seconds); t itself on a single process."""
+    if dist is None:
+        return t
+    import torch
+    tt = torch.tensor([t], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_value(units_per_rank: float, world: int, t_max: float) -> float:
+    """Whole-job throughput of N independent replicas: every rank's units over
+    the slowest rank's time."""
+    return units_per_rank * world / t_max
+
+
 # ----------------------------------------------------------------------------- GPU arm
 
 def source_hash(*files):
@@ -300,12 +318,8 @@ def run_ours(args, rank, world, dist):
     with ClockSampler(gpu_uuid(torch, dev)) as clk:
         t = timed(step, args.steps, 0)
     assert model.sync_status() == tl.TL_OK
-    if dist:
-        tt = torch.tensor([t], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t = float(tt.item())
-    tokens = seq * args.steps * world
-    value = tokens / t
+    t = max_over_ranks(t, dist, "cuda")
+    value = job_value(seq * args.steps, world, t)
     ms_per_step = t / args.steps * 1e3
     n_layers = 2 + L
     launches_per_fwd = 2 + 9 * n_layers
@@ -314,12 +328,9 @@ def run_ours(args, rank, world, dist):
     ids_h = torch.from_numpy(syn.prompt_ids(w).astype(np.int32)).pin_memory()
     y_h = torch.empty(seq, 2048, dtype=torch.float32).pin_memory()
     k_e2e = max(10, min(args.steps, 500))
-    t_e2e = timed(lambda: model.prefill(ids_h, L=L, y_out=y_h), k_e2e, 3)
-    if dist:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device="cuda")
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = float(tt.item())
-    e2e = {"value": round(seq * k_e2e * world / t_e2e, 1), "unit": "tokens/s",
+    t_e2e = max_over_ranks(timed(lambda: model.prefill(ids_h, L=L, y_out=y_h), k_e2e, 3), dist,
+                           "cuda")
+    e2e = {"value": round(job_value(seq * k_e2e, world, t_e2e), 1), "unit": "tokens/s",
            "h2d_bytes_per_step": ids_h.numel() * 4, "d2h_bytes_per_step": y_h.numel() * 4}
 
     # roofline of the dominant kernel: the gate|up GEMM launch (N 16384, K 2048, T 128)
@@ -381,11 +392,7 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
         return torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).cuda()
 
     def max_t(t):
-        if dist:
-            tt = torch.tensor([t], dtype=torch.float64, device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            return float(tt.item())
-        return t
+        return max_over_ranks(t, dist, "cuda")
 
     # B = 1, FP16 KV, prompt 256 -> 384
     w = syn.WORKLOADS["decode407m"]

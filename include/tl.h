@@ -125,7 +125,7 @@ tl_status tl_kv_quant_int8(const uint16_t* x, int rows, int hd, int8_t* codes,
  * FP16 residual stream is opt-in, so FP32 is the default).
  * ------------------------------------------------------------------------ */
 typedef struct tl_block_desc {
-  int d_model;     /* d; multiple of 256, at most 8192 */
+  int d_model;     /* d; 256 * 2^k, at most 8192 */
   int n_heads;     /* H; n_heads * head_dim == d_model (multi-head, no GQA) */
   int head_dim;    /* 64 or 128 */
   int ffn;         /* F; multiple of 128 */
@@ -296,6 +296,13 @@ tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K
 tl_status tl_linear_noalloc(const uint32_t* packed, const uint16_t* scales, int N,
                             int K, int group, const uint16_t* x, int T, float* y,
                             tl_stream stream);
+
+/* Test hook for the bounded device waits: runs one kernel whose mbarrier wait
+ * can never complete (nothing arrives on it).  The wait gives up after
+ * limit_us microseconds (1 .. 2e6) and records TL_ERR_TIMEOUT in the model's
+ * status word; read it with tl_sync_status.  The kernel returns normally: no
+ * trap, no fault, the context stays usable. */
+tl_status tl_check_bounded_wait(tl_model* model, unsigned limit_us, tl_stream stream);
 
 /* Synchronise `stream`, then return and clear the model's device status word
  * (TL_OK, TL_ERR_TIMEOUT or TL_ERR_NUMERIC). */

@@ -231,3 +231,17 @@ def test_new_cache_after_destroy_uses_its_own_graphs(model):
         kv.close()
     assert np.array_equal(outs[0][0], outs[1][0])
     assert np.array_equal(outs[0][2], outs[1][0])
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(model):
+    """A device wait that can never complete gives up after its limit and
+    reports TL_ERR_TIMEOUT; the context keeps working afterwards."""
+    import time
+    t0 = time.perf_counter()
+    tl.tl_check_bounded_wait(model.handle, 2000)          # 2 ms limit
+    assert model.sync_status() == tl.TL_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 5.0
+    assert model.sync_status() == tl.TL_OK               # cleared
+    x = to_dev(syn.hidden_input(W, 4), torch.float16)
+    y = model.prefill(h_in=x, L=1)
+    assert model.sync_status() == tl.TL_OK and torch.isfinite(y).all()

@@ -82,6 +82,7 @@ _SIGS = {
     "tl_linear_workspace_bytes": ([I, I, I, ctypes.POINTER(SZ)], I),
     "tl_linear": ([P, P, I, I, I, P, I, P, P, P], I),
     "tl_linear_noalloc": ([P, P, I, I, I, P, I, P, P], I),
+    "tl_check_bounded_wait": ([P, ctypes.c_uint, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -277,6 +278,10 @@ def tl_linear_noalloc(packed, scales, N: int, K: int, group: int, x, y, stream=N
     T = x.shape[0]
     _check(lib.tl_linear_noalloc(_ptr(packed), _ptr(scales), N, K, group, _ptr(x), T, _ptr(y),
                                  _stream(stream)))
+
+
+def tl_check_bounded_wait(model: int, limit_us: int, stream=None) -> None:
+    _check(lib.tl_check_bounded_wait(model, limit_us, _stream(stream)))
 
 
 def tl_sync_status(model: int, stream=None) -> int:

@@ -108,6 +108,7 @@ struct tl_model {
   float* part;
   float* part2;          // decode: gate|up partials read by the down projection
   int* attn_counters;    // decode: merge tickets [kMaxLanes][H], zero between launches
+  int* gemv_tickets;     // decode: residual-add tickets per 128-row block, zero between launches
   float* y;
   int32_t* lane_map;
   float* dec_scratch;
@@ -179,8 +180,9 @@ TL_API tl_status tl_block_create(const tl_block_desc* desc, tl_block** out) {
   TL_CHECK_ARG(desc && out, "NULL argument");
   *out = nullptr;
   const tl_block_desc& d = *desc;
-  TL_CHECK_ARG(d.d_model >= 256 && d.d_model % 256 == 0 && d.d_model <= 8192,
-               "d_model = %d must be a multiple of 256 in [256, 8192]", d.d_model);
+  TL_CHECK_ARG(d.d_model >= 256 && d.d_model <= 8192 && d.d_model % 256 == 0 &&
+                   ((d.d_model / 256) & (d.d_model / 256 - 1)) == 0,
+               "d_model = %d must be 256 * 2^k, at most 8192", d.d_model);
   if (d.head_dim != 64 && d.head_dim != 128)
     return set_error(TL_ERR_UNSUPPORTED, "head_dim = %d: only 64 and 128", d.head_dim);
   TL_CHECK_ARG(d.n_heads * d.head_dim == d.d_model,
@@ -331,7 +333,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
   void* p_u; void* p_part; void* p_y; void* p_lid; void* p_dec; void* p_status; void* p_rope;
-  void* p_part2; void* p_ctr;
+  void* p_part2; void* p_ctr; void* p_gtk;
   size_t part2_floats = 0;
   for (int t = 1; t <= md.max_lanes; ++t)
     part2_floats = std::max(part2_floats, (size_t)gemm_splits(2 * F, d, t) * t * 2 * F);
@@ -348,6 +350,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_part, maxpart * 4},
       {&p_part2, part2_floats * 4},
       {&p_ctr, (size_t)kMaxLanes * m->H * 4},
+      {&p_gtk, (size_t)1024 * 4},
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
       {&p_dec, (size_t)kMaxLanes * m->H * m->max_chunks * (m->hd + 2) * 4},
@@ -376,6 +379,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->part = (float*)p_part;
   m->part2 = (float*)p_part2;
   m->attn_counters = (int*)p_ctr;
+  m->gemv_tickets = (int*)p_gtk;
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
   m->dec_scratch = (float*)p_dec;
@@ -398,6 +402,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
     cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
     if (e3 == cudaSuccess) e3 = cudaMemset(m->attn_counters, 0, (size_t)kMaxLanes * m->H * 4);
+    if (e3 == cudaSuccess) e3 = cudaMemset(m->gemv_tickets, 0, (size_t)1024 * 4);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
       return set_error(TL_ERR_CUDA, "model initialisation copy failed");
@@ -697,13 +702,18 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     da.counters = m->attn_counters;
     TL_TRY(launch_attn_decode_fused(da, s));
   }
-  // O projection, residual, RMSNorm before the MLP
+  // O projection, residual, RMSNorm before the MLP (decode: the GEMV's last
+  // CTA per row block adds the residual, the norm reads h only)
   g = gemm_args(m, b, 1, m->attn, rows);
+  if (decode) {
+    g.h = m->h;
+    g.tickets = m->gemv_tickets;
+  }
   TL_TRY(launch_gemm(g, s));
   NormArgs n = norm_args(m, rows);
   n.part = m->part;
   n.part_rows = rows;
-  n.S = g.splits;
+  n.S = decode ? 0 : g.splits;
   n.n_add = rows;
   n.gamma_next = b->d.gamma_ffn;
   n.n_next = rows;
@@ -720,6 +730,8 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     dn.x_part = m->part2;
     dn.x_S = g.splits;
     dn.x_F = m->F;
+    dn.h = m->h;
+    dn.tickets = m->gemv_tickets;
     TL_TRY(launch_gemm(dn, s));
   } else {
     TL_TRY(launch_gemm(g, s));
@@ -807,9 +819,7 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
     TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, s));
     const int nxt = layer + 1 < n_layers ? active(layer + 1) : 0;
     NormArgs en = norm_args(m, trace ? B : act);
-    en.part = m->part;
-    en.part_rows = act;
-    en.S = gemm_splits(m->d, m->F, act);
+    en.S = 0;   // the down projection already added its sums into h
     en.n_add = act;
     en.n_next = nxt;
     if (nxt > 0) en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
@@ -994,6 +1004,14 @@ TL_API tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N
   TL_TRY(launch_gemm(a, s));
   if (S > 1) TL_TRY(launch_split_sum((const float*)workspace, S, (long)T * N, y, s));
   return ok();
+}
+
+TL_API tl_status tl_check_bounded_wait(tl_model* model, unsigned limit_us, tl_stream stream) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG(limit_us >= 1 && limit_us <= 2000000, "limit_us = %u out of [1, 2000000]",
+               limit_us);
+  return launch_bounded_wait_check(model->status, (uint64_t)limit_us * 1000ull,
+                                   (cudaStream_t)stream);
 }
 
 TL_API tl_status tl_sync_status(tl_model* model, tl_stream stream) {

@@ -6,7 +6,7 @@
 //
 // Every reduction runs in a fixed order that depends only on the row length,
 // so a row's result never depends on how many rows share the launch.
-#include "tl_internal.cuh"
+#include "tl_launch.cuh"
 
 namespace tl {
 namespace {
@@ -28,6 +28,7 @@ __device__ __forceinline__ void set_status(int* status, int code) {
 
 // ------------------------------------------------------------------ embed
 __global__ void embed_kernel(EmbedArgs a) {
+  pdl_enter();
   const int row = blockIdx.x;
   const int src = a.src_row ? a.src_row[row] : row;
   float* h = a.h + (size_t)row * a.d;
@@ -47,45 +48,50 @@ __global__ void embed_kernel(EmbedArgs a) {
 
 // ------------------------------------------------------------------ residual + RMSNorm
 constexpr int NORM_THREADS = 256;
-constexpr int NORM_MAX_PER_THREAD = 32;   // d <= 8192
 
+// PER = d / 256 elements per thread.  Partial sums are loaded four splits at a
+// time (independent loads in flight) and added in split order.
+template <int PER>
 __global__ void __launch_bounds__(NORM_THREADS) residual_norm_kernel(NormArgs a) {
+  pdl_enter();
   __shared__ float red[NORM_THREADS / 32];
   const int row = blockIdx.x;
-  const int per = a.d / NORM_THREADS;   // d % 256 == 0 checked on the host
   float* h = a.h + (size_t)row * a.d;
   const int out_row = a.out_row ? a.out_row[row] : row;
-  float v[NORM_MAX_PER_THREAD];
+  float v[PER];
   const bool add = row < a.n_add && a.S > 0;
 #pragma unroll
-  for (int e = 0; e < NORM_MAX_PER_THREAD; ++e) {
-    if (e < per) {
-      int i = threadIdx.x + e * NORM_THREADS;
-      float x = h[i];
-      if (add) {
-        for (int s = 0; s < a.S; ++s) x += a.part[((size_t)s * a.part_rows + row) * a.d + i];
-      }
-      v[e] = x;
-    }
-  }
+  for (int e = 0; e < PER; ++e) v[e] = h[threadIdx.x + e * NORM_THREADS];
   if (add) {
+    const size_t sstride = (size_t)a.part_rows * a.d;
+    const float* p0 = a.part + (size_t)row * a.d + threadIdx.x;
+    int sp = 0;
+    for (; sp + 4 <= a.S; sp += 4) {
+      float t[4][PER];
 #pragma unroll
-    for (int e = 0; e < NORM_MAX_PER_THREAD; ++e)
-      if (e < per) h[threadIdx.x + e * NORM_THREADS] = v[e];
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < PER; ++e) t[q][e] = p0[(sp + q) * sstride + e * NORM_THREADS];
+#pragma unroll
+      for (int e = 0; e < PER; ++e) v[e] = (((v[e] + t[0][e]) + t[1][e]) + t[2][e]) + t[3][e];
+    }
+    for (; sp < a.S; ++sp)
+#pragma unroll
+      for (int e = 0; e < PER; ++e) v[e] += p0[sp * sstride + e * NORM_THREADS];
+#pragma unroll
+    for (int e = 0; e < PER; ++e) h[threadIdx.x + e * NORM_THREADS] = v[e];
   }
   if (a.trace) {
     float* tr = a.trace + (size_t)out_row * a.d;
 #pragma unroll
-    for (int e = 0; e < NORM_MAX_PER_THREAD; ++e)
-      if (e < per) tr[threadIdx.x + e * NORM_THREADS] = v[e];
+    for (int e = 0; e < PER; ++e) tr[threadIdx.x + e * NORM_THREADS] = v[e];
   }
   const bool want_x = row < a.n_next;
   const bool want_y = row >= a.fin_lo && row < a.fin_hi;
   if (!want_x && !want_y) return;
   float ss = 0.0f;
 #pragma unroll
-  for (int e = 0; e < NORM_MAX_PER_THREAD; ++e)
-    if (e < per) ss = fmaf(v[e], v[e], ss);
+  for (int e = 0; e < PER; ++e) ss = fmaf(v[e], v[e], ss);
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -96,23 +102,19 @@ __global__ void __launch_bounds__(NORM_THREADS) residual_norm_kernel(NormArgs a)
   if (want_x) {
     __half* x = a.x + (size_t)row * a.d;
 #pragma unroll
-    for (int e = 0; e < NORM_MAX_PER_THREAD; ++e) {
-      if (e < per) {
-        int i = threadIdx.x + e * NORM_THREADS;
-        x[i] = __float2half_rn(v[e] * r * a.gamma_next[i]);
-      }
+    for (int e = 0; e < PER; ++e) {
+      const int i = threadIdx.x + e * NORM_THREADS;
+      x[i] = __float2half_rn(v[e] * r * a.gamma_next[i]);
     }
   } else {
     float* y = a.y + (size_t)out_row * a.d;
     bool bad = false;
 #pragma unroll
-    for (int e = 0; e < NORM_MAX_PER_THREAD; ++e) {
-      if (e < per) {
-        int i = threadIdx.x + e * NORM_THREADS;
-        float o = v[e] * r * a.gamma_final[i];
-        bad |= !isfinite(o);
-        y[i] = o;
-      }
+    for (int e = 0; e < PER; ++e) {
+      const int i = threadIdx.x + e * NORM_THREADS;
+      const float o = v[e] * r * a.gamma_final[i];
+      bad |= !isfinite(o);
+      y[i] = o;
     }
     if (bad) set_status(a.status, TL_ERR_NUMERIC);
   }
@@ -122,6 +124,7 @@ __global__ void __launch_bounds__(NORM_THREADS) residual_norm_kernel(NormArgs a)
 // One warp per (row, head).  Lane l handles rotate-half pairs (i, i + hd/2)
 // for i = l, l + 32 (hd = 128) or i = l (hd = 64).
 __global__ void rope_kv_kernel(RopeKvArgs a) {
+  pdl_enter();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (wid >= a.rows * a.H) return;
@@ -232,6 +235,7 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
 // ------------------------------------------------------------------ SwiGLU
 __global__ void swiglu_kernel(const float* __restrict__ part, int S, int rows, int F,
                               __half* __restrict__ u) {
+  pdl_enter();
   size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   size_t n = (size_t)rows * F;
   if (i >= n) return;
@@ -248,6 +252,7 @@ __global__ void swiglu_kernel(const float* __restrict__ part, int S, int rows, i
 }
 
 __global__ void set_pos_kernel(KvHeader* hdr, int lane, int value) {
+  pdl_enter();
   if (lane < 0) {
     for (int i = 0; i < kMaxLanes; ++i) hdr->pos[i] = value;
   } else {
@@ -256,6 +261,7 @@ __global__ void set_pos_kernel(KvHeader* hdr, int lane, int value) {
 }
 
 __global__ void advance_pos_kernel(KvHeader* hdr, int n_lanes) {
+  pdl_enter();
   int i = threadIdx.x;
   if (i < n_lanes) hdr->pos[i] += 1;
 }
@@ -264,14 +270,21 @@ __global__ void advance_pos_kernel(KvHeader* hdr, int n_lanes) {
 
 tl_status launch_embed(const EmbedArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
-  embed_kernel<<<a.rows, 256, 0, s>>>(a);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(embed_kernel, a.rows, 256, 0, s, a);
   return ok();
 }
 
 tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
-  residual_norm_kernel<<<a.rows, NORM_THREADS, 0, s>>>(a);
+  switch (a.d / NORM_THREADS) {
+    case 1: TL_LAUNCH_PDL(residual_norm_kernel<1>, a.rows, NORM_THREADS, 0, s, a); break;
+    case 2: TL_LAUNCH_PDL(residual_norm_kernel<2>, a.rows, NORM_THREADS, 0, s, a); break;
+    case 4: TL_LAUNCH_PDL(residual_norm_kernel<4>, a.rows, NORM_THREADS, 0, s, a); break;
+    case 8: TL_LAUNCH_PDL(residual_norm_kernel<8>, a.rows, NORM_THREADS, 0, s, a); break;
+    case 16: TL_LAUNCH_PDL(residual_norm_kernel<16>, a.rows, NORM_THREADS, 0, s, a); break;
+    case 32: TL_LAUNCH_PDL(residual_norm_kernel<32>, a.rows, NORM_THREADS, 0, s, a); break;
+    default: return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs d/256 in {1,2,4,...,32}", a.d);
+  }
   TL_LAUNCH_CHECK();
   return ok();
 }
@@ -279,28 +292,24 @@ tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
 tl_status launch_rope_kv(const RopeKvArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
   long warps = (long)a.rows * a.H;
-  rope_kv_kernel<<<(unsigned)((warps * 32 + 127) / 128), 128, 0, s>>>(a);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(rope_kv_kernel, (unsigned)((warps * 32 + 127) / 128), 128, 0, s, a);
   return ok();
 }
 
 tl_status launch_swiglu(const float* part, int S, int rows, int F, __half* u, cudaStream_t s) {
   if (rows == 0) return ok();
   size_t n = (size_t)rows * F;
-  swiglu_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, rows, F, u);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(swiglu_kernel, (unsigned)((n + 255) / 256), 256, 0, s, part, S, rows, F, u);
   return ok();
 }
 
 tl_status launch_set_pos(KvHeader* hdr, int lane, int value, cudaStream_t s) {
-  set_pos_kernel<<<1, 1, 0, s>>>(hdr, lane, value);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(set_pos_kernel, 1, 1, 0, s, hdr, lane, value);
   return ok();
 }
 
 tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s) {
-  advance_pos_kernel<<<1, kMaxLanes, 0, s>>>(hdr, n_lanes);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(advance_pos_kernel, 1, kMaxLanes, 0, s, hdr, n_lanes);
   return ok();
 }
 

@@ -19,7 +19,7 @@
 // Each output column (token) is computed independently of the others and the
 // split count depends only on (N, K, T-class), so a token's result does not
 // depend on which other tokens share the launch.
-#include "tl_internal.cuh"
+#include "tl_launch.cuh"
 
 namespace tl {
 namespace {
@@ -48,6 +48,7 @@ __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b
 
 template <int NT>
 __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
+  pdl_enter();
   __shared__ __align__(16) __half xs[NT][KC + 8];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,6 +198,34 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
   const int n_groups = (krange + a.G - 1) / a.G + 1;
   __half* ss = xs + 8 * xstride;              // [128][n_groups] scales of this CTA
 
+  // Weights and scales are constants of the model: stage the scales and issue
+  // the first batch of weight loads before waiting for the previous kernel, so
+  // their latency overlaps its tail.
+  for (int i = threadIdx.x; i < GV_ROWS * n_groups; i += GV_THREADS) {
+    const int r = i / n_groups, gg = i % n_groups;
+    const int row = m0 + r;
+    const __half* sp = row < a.n_split ? a.s0 + (size_t)row * gpr
+                                       : a.s1 + (size_t)(row - a.n_split) * gpr;
+    ss[i] = g_lo + gg < gpr ? sp[g_lo + gg] : __float2half_rn(0.f);
+  }
+  const int rowA = m0 + warp * 16 + g;
+  const uint2* wr[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int row = rowA + 8 * r;
+    const uint32_t* base = row < a.n_split ? a.w0 + (size_t)row * (a.K / 8)
+                                           : a.w1 + (size_t)(row - a.n_split) * (a.K / 8);
+    wr[r] = reinterpret_cast<const uint2*>(base + c0 * 8) + t;   // words 2t, 2t+1 of chunk 0
+  }
+  uint2 cur[GV_BATCH][2], nxt[GV_BATCH][2];
+#pragma unroll
+  for (int b = 0; b < GV_BATCH; ++b) {
+    const bool in = b < per;
+    nxt[b][0] = in ? __ldg(wr[0] + b * 4) : make_uint2(0u, 0u);
+    nxt[b][1] = in ? __ldg(wr[1] + b * 4) : make_uint2(0u, 0u);
+  }
+  pdl_enter();   // the activations below come from the previous kernel
+
   // stage x (rows >= T are zero), permuting each 8-k group to 0 4 1 5 2 6 3 7
   for (int i = threadIdx.x; i < 8 * (krange / 8); i += GV_THREADS) {
     const int r = i / (krange / 8), q = i % (krange / 8);
@@ -228,35 +257,11 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
     d[0] = make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
     d[1] = make_uint2(*reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
   }
-  for (int i = threadIdx.x; i < GV_ROWS * n_groups; i += GV_THREADS) {
-    const int r = i / n_groups, gg = i % n_groups;
-    const int row = m0 + r;
-    const __half* sp = row < a.n_split ? a.s0 + (size_t)row * gpr
-                                       : a.s1 + (size_t)(row - a.n_split) * gpr;
-    ss[i] = g_lo + gg < gpr ? sp[g_lo + gg] : __float2half_rn(0.f);
-  }
-
-  const int rowA = m0 + warp * 16 + g;
-  const uint2* wr[2];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int row = rowA + 8 * r;
-    const uint32_t* base = row < a.n_split ? a.w0 + (size_t)row * (a.K / 8)
-                                           : a.w1 + (size_t)(row - a.n_split) * (a.K / 8);
-    wr[r] = reinterpret_cast<const uint2*>(base + c0 * 8) + t;   // words 2t, 2t+1 of chunk 0
-  }
   const __half* srow0 = ss + (warp * 16 + g) * n_groups;
   const __half* srow1 = srow0 + 8 * n_groups;
   __syncthreads();
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  uint2 cur[GV_BATCH][2], nxt[GV_BATCH][2];
-#pragma unroll
-  for (int b = 0; b < GV_BATCH; ++b) {
-    const bool in = b < per;
-    nxt[b][0] = in ? __ldg(wr[0] + b * 4) : make_uint2(0u, 0u);
-    nxt[b][1] = in ? __ldg(wr[1] + b * 4) : make_uint2(0u, 0u);
-  }
   for (int cb = 0; cb < per; cb += GV_BATCH) {
 #pragma unroll
     for (int b = 0; b < GV_BATCH; ++b) {
@@ -307,10 +312,31 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
     out[(size_t)(tk + 1) * a.N + rowA] = acc[1];
     out[(size_t)(tk + 1) * a.N + rowA + 8] = acc[3];
   }
+  if (a.h == nullptr) return;
+  // last split of this row block: residual add of all partial sums, split order
+  __shared__ int gv_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int ticket = atomicAdd(&a.tickets[blockIdx.x], 1);
+    gv_last = ticket == a.splits - 1;
+    if (gv_last) a.tickets[blockIdx.x] = 0;
+  }
+  __syncthreads();
+  if (!gv_last) return;
+  __threadfence();
+  for (int i = threadIdx.x; i < a.T * GV_ROWS; i += GV_THREADS) {
+    const int tt = i / GV_ROWS, n = m0 + i % GV_ROWS;
+    float v = a.h[(size_t)tt * a.N + n];
+    float sum = 0.f;
+    for (int sp = 0; sp < a.splits; ++sp) sum += __ldcg(a.part + ((size_t)sp * a.T + tt) * a.N + n);
+    a.h[(size_t)tt * a.N + n] = v + sum;
+  }
 }
 
 __global__ void split_sum_kernel(const float* __restrict__ part, int S, long n,
                                  float* __restrict__ y) {
+  pdl_enter();
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   float acc = part[i];
@@ -337,8 +363,7 @@ int gemm_mma_splits(int N, int K, int T) {
 
 tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s) {
   if (n == 0) return ok();
-  split_sum_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(part, S, n, y);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(split_sum_kernel, (unsigned)((n + 255) / 256), 256, 0, s, part, S, n, y);
   return ok();
 }
 
@@ -346,12 +371,14 @@ bool gemv_eligible(int N, int K, int T) { return T <= 8 && N % GV_ROWS == 0 && K
 
 // Decode split count: each split covers at most 2048 k (the staged activations
 // then fit in 33 KB of shared memory) and at least 4 chunks; splits double
-// until there are two CTAs per SM.  Depends on (N, K) only.
+// while the grid still fits one wave of two CTAs per SM.  Depends on (N, K)
+// only.
 int gemv_splits(int N, int K) {
   const int n_chunks = K / KC;
   int s = 1;
   while (n_chunks / s > 32 && n_chunks % (2 * s) == 0) s *= 2;
-  while ((N / GV_ROWS) * s < 2 * 148 && n_chunks % (2 * s) == 0 && n_chunks / (2 * s) >= 4) s *= 2;
+  while ((N / GV_ROWS) * 2 * s <= 2 * 148 && n_chunks % (2 * s) == 0 && n_chunks / (2 * s) >= 4)
+    s *= 2;
   return s;
 }
 
@@ -368,14 +395,14 @@ tl_status launch_gemv(const GemmArgs& a, cudaStream_t s) {
   const size_t smem = (size_t)8 * (krange + 4) * 2 + (size_t)GV_ROWS * n_groups * 2;
   if (smem > 48 * 1024) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV split too wide");
   dim3 grid(a.N / GV_ROWS, 1, a.splits);
-  gemv_w4_kernel<<<grid, GV_THREADS, smem, s>>>(a);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(gemv_w4_kernel, grid, GV_THREADS, smem, s, a);
   return ok();
 }
 
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (gemv_eligible(a.N, a.K, a.T)) return launch_gemv(a, s);
-  if (a.x_part) return set_error(TL_ERR_UNSUPPORTED, "SwiGLU staging needs the decode GEMV");
+  if (a.x_part || a.h)
+    return set_error(TL_ERR_UNSUPPORTED, "fused staging / residual needs the decode GEMV");
   if (gemm_tc_eligible(a.N, a.K, a.T)) return launch_gemm_tc(a, s);
   return launch_gemm_mma(a, s);
 }
@@ -385,12 +412,11 @@ tl_status launch_gemm_mma(const GemmArgs& a, cudaStream_t s) {
   const int nt = token_tile(a.T);
   dim3 grid(a.N / ROWS_CTA, (a.T + nt - 1) / nt, a.splits);
   switch (nt) {
-    case 8: gemm_w4_mma_kernel<8><<<grid, THREADS, 0, s>>>(a); break;
-    case 16: gemm_w4_mma_kernel<16><<<grid, THREADS, 0, s>>>(a); break;
-    case 32: gemm_w4_mma_kernel<32><<<grid, THREADS, 0, s>>>(a); break;
-    default: gemm_w4_mma_kernel<64><<<grid, THREADS, 0, s>>>(a); break;
+    case 8: TL_LAUNCH_PDL(gemm_w4_mma_kernel<8>, grid, THREADS, 0, s, a); break;
+    case 16: TL_LAUNCH_PDL(gemm_w4_mma_kernel<16>, grid, THREADS, 0, s, a); break;
+    case 32: TL_LAUNCH_PDL(gemm_w4_mma_kernel<32>, grid, THREADS, 0, s, a); break;
+    default: TL_LAUNCH_PDL(gemm_w4_mma_kernel<64>, grid, THREADS, 0, s, a); break;
   }
-  TL_LAUNCH_CHECK();
   return ok();
 }
 

@@ -8,29 +8,41 @@
 //   * a TMA warp loads the activation tile x[BN tokens][64 k] (fp16, 128-byte
 //     swizzled, rows past T read as zero) and the packed weight tile
 //     [128 rows][8 words] into a shared-memory stage;
-//   * four dequantisation warps (one TMEM lane quadrant each, one thread per
-//     weight row) turn the row's 64 codes into fp16 code*scale pairs and store
-//     them straight into tensor memory with tcgen05.st: the weight tile is the
-//     A operand of the MMA and never passes through shared memory;
+//   * sixteen dequantisation warps (four groups of four, one warp per TMEM
+//     lane quadrant in each group; group g takes k blocks i with i % 4 == g;
+//     one thread per weight row) turn the row's 64 codes into fp16 code*scale
+//     pairs and store them straight into tensor memory with tcgen05.st: the
+//     weight tile is the A operand of the MMA and never passes through shared
+//     memory;
 //   * one thread issues four tcgen05.mma kind::f16 (M 128, N BN, K 16), A from
 //     TMEM, B from the swizzled shared-memory tile, fp32 accumulation in TMEM,
 //     and commits to the stage's "empty" barrier.
-// The same four warps then read the accumulator back with tcgen05.ld and store
-// it as fp32 partial sums.  Every wait on an mbarrier is bounded: when a wait
+// The same warps then read the accumulator back with tcgen05.ld and store it as
+// fp32 partial sums, and signal an "epilogue done" barrier that the MMA warp
+// waits on before it frees TMEM.  A CTA owns all of TMEM and 8 (5 for 256
+// tokens) pipeline stages; split-K counts are chosen so that one wave of CTAs
+// covers the 148 SMs.  Every wait on an mbarrier is bounded: when a wait
 // runs out the CTA records TL_ERR_TIMEOUT in the status word, stops issuing
 // work, waits (bounded) for its copies in flight, frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include "tl_internal.cuh"
+#include "tl_launch.cuh"
 
 namespace tl {
 namespace {
 
 constexpr int BM = 128;            // weight rows per CTA (MMA M)
 constexpr int BK = 64;             // k per stage
-constexpr int STAGES = 4;
-constexpr int THREADS = 256;       // warp 0 TMA, warp 1 MMA, warps 4..7 dequant + epilogue
+constexpr int DQ_GROUPS = 4;       // dequantisation groups, each 4 warps (one per TMEM quadrant)
+constexpr int DQ_WARPS = 4 * DQ_GROUPS;
+constexpr int TMA_WARP = DQ_WARPS, MMA_WARP = DQ_WARPS + 1;
+constexpr int THREADS = 32 * (DQ_WARPS + 2);
+constexpr int TMEM_COLS = 512;     // the whole of TMEM: one CTA per SM
+constexpr size_t kMinSmem = 120 * 1024;   // also keeps it to one CTA per SM
+template <int BN> struct TcCfg {
+  static constexpr int STAGES = BN >= 256 ? 5 : 8;
+};
 constexpr int A_COLS = BK / 2;     // TMEM columns per A stage (two fp16 per column)
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a bounded wait gives up after 2 s
 
@@ -59,24 +71,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 }
 
 // Bounded wait for the phase with the given parity to complete: false after
-// kWaitLimitNs of global time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// limit_ns of global time.
+__device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+// Bounded wait for the phase with the given parity to complete: false after
+// limit_ns of global time.  The clock is read only once the first try fails.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
-  uint64_t start = 0;
-  for (uint32_t i = 0;; ++i) {
-    uint32_t done;
-    asm volatile(
-        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-        " selp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(addr), "r"(parity)
-        : "memory");
-    if (done) return true;
-    if ((i & 255) == 0) {
-      const uint64_t now = globaltimer_ns();
-      if (i == 0) start = now;
-      else if (now - start > kWaitLimitNs) return false;
-    }
+  if (mbar_try(addr, parity)) return true;
+  const uint64_t start = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(addr, parity)) return true;
+    if ((i & 63) == 0 && globaltimer_ns() - start > limit_ns) return false;
   }
 }
 
@@ -128,7 +144,8 @@ __device__ __forceinline__ uint32_t dequant_code_pair(uint32_t w, uint32_t sel) 
 
 struct TcArgs {
   int N, K, G, T, n_split;   // n_split % 128 == 0
-  int kblocks_per_split;
+  int splits;                // split z covers k blocks [z*nkb/S, (z+1)*nkb/S)
+  int max_groups;            // scale groups staged per CTA (shared-memory sizing)
   const __half* s0;
   const __half* s1;
   float* part;
@@ -140,25 +157,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                       const __grid_constant__ CUtensorMap map_w0,
                       const __grid_constant__ CUtensorMap map_w1, TcArgs a) {
+  constexpr int STAGES = TcCfg<BN>::STAGES;
   constexpr uint32_t B_BYTES = BN * 128;          // BN rows x 64 fp16
   constexpr uint32_t W_BYTES = BM * 32;           // 128 rows x 8 words
-  constexpr uint32_t TMEM_COLS = (BN + STAGES * A_COLS) <= 256 ? 256 : 512;
+  static_assert(BN + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // 1024-align the dynamic shared memory base
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sB = smem;                                        // STAGES x B_BYTES
   uint8_t* sW = sB + STAGES * B_BYTES;                       // STAGES x W_BYTES
   __half* sScale = reinterpret_cast<__half*>(sW + STAGES * W_BYTES);   // [BM][groups]
-  const int kb_begin = blockIdx.z * a.kblocks_per_split;
-  const int nkb = a.kblocks_per_split;
-  const int groups = (nkb * BK + a.G - 1) / a.G;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sScale + BM * groups + 8);
+  const int nkb_total = a.K / BK;
+  const int kb_begin = (int)(((long)blockIdx.z * nkb_total) / a.splits);
+  const int nkb = (int)(((long)(blockIdx.z + 1) * nkb_total) / a.splits) - kb_begin;
+  const int g_first = (kb_begin * BK) / a.G;
+  const int groups = ((kb_begin + nkb) * BK - 1) / a.G - g_first + 1;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sScale + BM * a.max_groups + 8);
   bars = reinterpret_cast<uint64_t*>(((uintptr_t)bars + 7) & ~(uintptr_t)7);
   uint64_t* full = bars;                 // TMA landed
   uint64_t* empty = bars + STAGES;       // MMA done with the stage
   uint64_t* afull = bars + 2 * STAGES;   // A stage written to TMEM
   uint64_t* accb = bars + 3 * STAGES;    // accumulator complete
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accb + 1);
+  uint64_t* epib = accb + 1;             // epilogue finished reading TMEM
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epib + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,35 +197,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&afull[s], 4);
     }
     mbar_init(accb, 1);
+    mbar_init(epib, DQ_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(map_w) : "memory");
   }
-  if (warp == 1) {
+  __syncwarp();
+  if (warp == MMA_WARP) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(tmem_slot)),
                  "r"(TMEM_COLS));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
-  // scales of this CTA's rows and k range -> shared memory
-  {
-    const int gpr = a.K / a.G;
-    const int g0 = (kb_begin * BK) / a.G;
-    for (int i = threadIdx.x; i < BM * groups; i += THREADS) {
-      int r = i / groups, g = i % groups;
-      sScale[r * groups + g] =
-          g0 + g < gpr ? scales[(size_t)(wrow0 + r) * gpr + g0 + g] : __float2half_rn(0.f);
-    }
-  }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem_base = *tmem_slot;
+  // everything above is CTA-local; from here on the kernel reads what the
+  // previous kernel wrote (the activations), so wait for it here
+  pdl_enter();
   const uint32_t acc_col = 0;
   const uint32_t a_col0 = BN;
 
-  if (warp == 0) {
+  if (warp == TMA_WARP) {
     // ---------------------------------------------------------------- TMA
     if (lane == 0) {
       int issued = 0;
@@ -228,36 +244,63 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int i = 0; i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
       }
     }
-  } else if (warp == 1) {
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
     // ---------------------------------------------------------------- MMA
     if (lane == 0) {
       const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      // k blocks are issued in batches of up to MMA_BATCH that are already
+      // dequantised: one tcgen05.fence per batch instead of per k block
+      constexpr int MMA_BATCH = 4;
       bool ok = true;
-      for (int i = 0; i < nkb && ok; ++i) {
-        const int s = i % STAGES;
-        if (!mbar_wait(&full[s], (i / STAGES) & 1) || !mbar_wait(&afull[s], (i / STAGES) & 1) ||
-            *(volatile int*)abort_flag) {
+      for (int i0 = 0; i0 < nkb && ok; i0 += MMA_BATCH) {
+        const int cnt = min(MMA_BATCH, nkb - i0);
+        for (int j = 0; j < cnt; ++j) {
+          const int i = i0 + j, s = i % STAGES;
+          if (!mbar_wait(&full[s], (i / STAGES) & 1) || !mbar_wait(&afull[s], (i / STAGES) & 1)) {
+            ok = false;
+            break;
+          }
+        }
+        if (!ok || *(volatile int*)abort_flag) {
           atomicExch(abort_flag, 1);
           ok = false;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_BYTES));
-        const uint32_t a_tm = tmem_base + a_col0 + s * A_COLS;
+        for (int j = 0; j < cnt; ++j) {
+          const int i = i0 + j, s = i % STAGES;
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_BYTES));
+          const uint32_t a_tm = tmem_base + a_col0 + s * A_COLS;
 #pragma unroll
-        for (int j = 0; j < BK / 16; ++j)
-          mma_ts(tmem_base + acc_col, a_tm + j * 8, bdesc + (uint64_t)(2 * j), idesc,
-                 (i > 0 || j > 0) ? 1u : 0u);
-        mma_commit(&empty[s]);
+          for (int k = 0; k < BK / 16; ++k)
+            mma_ts(tmem_base + acc_col, a_tm + k * 8, bdesc + (uint64_t)(2 * k), idesc,
+                   (i > 0 || k > 0) ? 1u : 0u);
+          mma_commit(&empty[s]);
+        }
       }
       mma_commit(accb);   // arrives once all issued MMAs are complete
     }
-  } else if (warp >= 4) {
+    __syncwarp();
+  } else {
     // ---------------------------------------------------------------- dequant + epilogue
     const int quad = warp & 3;
+    const int parity = warp >> 2;               // group: takes k blocks i with i % DQ_GROUPS == parity
     const int r = quad * 32 + lane;             // weight row within the tile = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    for (int i = 0; i < nkb; ++i) {
+    // scales of this CTA's rows and k range -> shared memory (the TMA warp is
+    // already streaming; only the dequantisation warps wait for the scales)
+    {
+      const int gpr = a.K / a.G;
+      const int g0 = g_first;
+      for (int i = threadIdx.x; i < BM * groups; i += 32 * DQ_WARPS) {
+        const int rr = i / groups, gg = i % groups;
+        sScale[rr * groups + gg] =
+            g0 + gg < gpr ? scales[(size_t)(wrow0 + rr) * gpr + g0 + gg] : __float2half_rn(0.f);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * DQ_WARPS) : "memory");
+    }
+    for (int i = parity; i < nkb; i += DQ_GROUPS) {
       const int s = i % STAGES;
       if (!mbar_wait(&full[s], (i / STAGES) & 1) || *(volatile int*)abort_flag) {
         atomicExch(abort_flag, 1);
@@ -266,7 +309,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint4* wp = reinterpret_cast<const uint4*>(sW + s * W_BYTES + r * 32);
       const uint4 wa = wp[0], wb = wp[1];
       const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-      const int g = ((kb_begin + i) * BK) / a.G - (kb_begin * BK) / a.G;
+      const int g = ((kb_begin + i) * BK) / a.G - g_first;
       const __half sc = sScale[r * groups + g];
       const __half2 s2 = __halves2half2(sc, sc);
       uint32_t v[32];
@@ -300,8 +343,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (ok) {
       float* out = a.part + (size_t)blockIdx.z * a.T * a.N + (size_t)(m0 + r);
+      // this group's 32-token chunks: cc = parity, parity + 2, ...
 #pragma unroll 1
-      for (int cc = 0; cc < BN / 32; ++cc) {
+      for (int cc = parity; cc < BN / 32; cc += DQ_GROUPS) {
         if (t0 + cc * 32 >= a.T) break;   // warp-uniform
         uint32_t u[32];
         asm volatile(
@@ -316,23 +360,48 @@ __global__ void __launch_bounds__(THREADS, 1)
               "=r"(u[31])
             : "r"(tmem_base + lane_addr + acc_col + cc * 32));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        const int tn = min(32, a.T - (t0 + cc * 32));
+        float* o = out + (size_t)(t0 + cc * 32) * a.N;
+        if (tn == 32) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int t = t0 + cc * 32 + e;
-          if (t < a.T) out[(size_t)t * a.N] = __uint_as_float(u[e]);
+          for (int e = 0; e < 32; ++e) __stcg(o + (size_t)e * a.N, __uint_as_float(u[e]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (e < tn) __stcg(o + (size_t)e * a.N, __uint_as_float(u[e]));
         }
       }
     }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncwarp();
+    if (lane == 0) mbar_arrive(epib);
   }
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
-  if (*(volatile int*)abort_flag && threadIdx.x == 0 && a.status)
-    atomicCAS(a.status, 0, kDevTimeout);
-  if (warp == 1) {
+  if (warp == MMA_WARP) {
+    // free TMEM only once every epilogue warp has finished reading it
+    bool done = true;
+    if (lane == 0) done = mbar_wait(epib, 0);
+    done = __shfl_sync(0xffffffffu, done ? 1 : 0, 0) != 0;
+    if (!done && lane == 0) atomicExch(abort_flag, 1);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(TMEM_COLS));
   }
+  if (warp == MMA_WARP && lane == 0 && *(volatile int*)abort_flag && a.status)
+    atomicCAS(a.status, 0, kDevTimeout);
+}
+
+// A wait that can never complete: one barrier with an arrival count of 1 that
+// nobody arrives on.  The bounded wait gives up after limit_ns and records
+// TL_ERR_TIMEOUT, exercising the same path the GEMM pipeline uses.
+__global__ void bounded_wait_check_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, limit_ns)) atomicCAS(status, 0, kDevTimeout);
 }
 
 // ---------------------------------------------------------------- host side
@@ -370,10 +439,11 @@ int tc_tile_n(int T) {
 }
 
 template <int BN>
-size_t tc_smem_bytes(int kblocks_per_split, int G) {
-  int groups = (kblocks_per_split * BK + G - 1) / G + 1;
-  return 1024 + (size_t)STAGES * (BN * 128 + BM * 32) + (size_t)BM * groups * 2 + 16 +
-         (4 * STAGES + 1) * 8 + 16;
+size_t tc_smem_bytes(int max_groups) {
+  constexpr int STAGES = TcCfg<BN>::STAGES;
+  size_t b = 1024 + (size_t)STAGES * (BN * 128 + BM * 32) + (size_t)BM * max_groups * 2 + 16 +
+             (4 * STAGES + 2) * 8 + 16;
+  return b < kMinSmem ? kMinSmem : b;
 }
 
 template <int BN>
@@ -396,19 +466,30 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.G = g.G;
   a.T = g.T;
   a.n_split = g.n_split;
-  a.kblocks_per_split = (g.K / BK) / g.splits;
+  a.splits = g.splits;
+  {
+    // largest number of scale groups any split touches (+1 for an unaligned start)
+    const int nkb = g.K / BK;
+    const int per = (nkb + g.splits - 1) / g.splits;
+    a.max_groups = (per * BK + g.G - 1) / g.G + 1;
+  }
   a.s0 = g.s0;
   a.s1 = g.s1;
   a.part = g.part;
   a.status = g.status;
-  const size_t smem = tc_smem_bytes<BN>(a.kblocks_per_split, g.G);
+  const size_t smem = tc_smem_bytes<BN>(a.max_groups);
   dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
-  gemm_w4_tc_kernel<BN><<<grid, THREADS, smem, s>>>(mx, mw0, mw1, a);
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(gemm_w4_tc_kernel<BN>, grid, THREADS, smem, s, mx, mw0, mw1, a);
   return ok();
 }
 
 }  // namespace
+
+tl_status launch_bounded_wait_check(int* status, uint64_t limit_ns, cudaStream_t s) {
+  bounded_wait_check_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  TL_LAUNCH_CHECK();
+  return ok();
+}
 
 // One-time set-up (driver entry point, shared-memory limit); called outside
 // any stream capture.
@@ -426,14 +507,14 @@ tl_status gemm_tc_init() {
   return ok();
 }
 
-// Split-K factor for the tensor-core kernel: enough CTAs to cover the SMs
-// once, at least 4 k blocks per split.
+// Split-K factor for the tensor-core kernel: one CTA per SM, so as many splits
+// as fit the 148 SMs in one wave, each at least 3 k blocks long.
 int gemm_tc_splits(int N, int K, int T) {
   const int nkb = K / BK;
   const int tiles = (N / BM) * ((T + tc_tile_n(T) - 1) / tc_tile_n(T));
-  int s = 1;
-  while (tiles * s < 148 && s * 2 <= 16 && nkb % (s * 2) == 0 && nkb / (s * 2) >= 4) s *= 2;
-  return s;
+  int s = tiles >= 148 ? 1 : 148 / tiles;
+  if (s > nkb / 3) s = nkb / 3;
+  return s < 1 ? 1 : s;
 }
 
 bool gemm_tc_eligible(int N, int K, int T) { return T >= 64 && N % BM == 0 && K % BK == 0; }

@@ -83,6 +83,12 @@ struct GemmArgs {
   // gate|up partial sums) instead of x
   const float* x_part;
   int x_S, x_F;
+  // decode GEMV only: when h is set, the last CTA of each 128-row block (an
+  // atomic ticket in `tickets`, reset after use) adds the S partial sums in
+  // split order to h[t][n] (the residual stream) instead of leaving them for
+  // a later kernel
+  float* h;
+  int* tickets;
 };
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
 // kernel for T >= 64, the mma.sync register-dequant kernel below that.
@@ -95,6 +101,7 @@ bool gemm_tc_eligible(int N, int K, int T);
 int gemm_tc_splits(int N, int K, int T);
 tl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t s);
 tl_status gemm_tc_init();
+tl_status launch_bounded_wait_check(int* status, uint64_t limit_ns, cudaStream_t s);
 // y[t][n] = sum_{s < S} part[s][t][n], in order s = 0, 1, ...
 tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s);
 
@@ -155,10 +162,9 @@ tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s);
 tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
                               int T, int H, int hd, cudaStream_t s);
 struct DecodeAttnArgs {
-  const __half* q;           // [rows][d] (unfused path)
   __half* out;               // [rows][d]
   int rows, H, hd, d;
-  // fused path: q/k/v from the QKV split-K partials, RoPE, KV append, merge
+  // q/k/v come from the QKV split-K partials; RoPE, KV append and merge
   const float* qkv_part;     // [S][rows][3d]
   int qkv_S;
   const float2* rope_cs;     // [max_ctx][hd/2]
@@ -171,7 +177,6 @@ struct DecodeAttnArgs {
   float* scratch;            // [rows][H][max_chunks][hd + 2]
   int max_chunks;
 };
-tl_status launch_attn_decode(const DecodeAttnArgs& a, cudaStream_t s);
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
 
 }  // namespace tl

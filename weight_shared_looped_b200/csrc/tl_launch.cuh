@@ -1,0 +1,46 @@
+// Programmatic dependent launch for the forward kernels.
+//
+// Every forward kernel begins with pdl_enter(): griddepcontrol.wait blocks
+// until the kernel it depends on (the previous one in the stream or graph) has
+// completed and its memory is visible, and only then touches memory; after
+// that, griddepcontrol.launch_dependents lets the next kernel be scheduled
+// while this one runs.  Ordering is therefore exactly stream ordering; what
+// overlaps is the next kernel's launch and CTA scheduling.  Without the launch
+// attribute both instructions are no-ops.
+#pragma once
+
+#include "tl_internal.cuh"
+
+namespace tl {
+
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+#define TL_LAUNCH_PDL(kernel, grid, block, smem, stream, ...)                                \
+  do {                                                                                      \
+    cudaError_t e_ = ::tl::launch_pdl(kernel, dim3(grid), dim3(block), (size_t)(smem),      \
+                                      stream, __VA_ARGS__);                                 \
+    if (e_ != cudaSuccess)                                                                  \
+      return ::tl::set_error(TL_ERR_CUDA, "launch of %s failed: %s", #kernel,              \
+                             cudaGetErrorString(e_));                                       \
+  } while (0)
+
+}  // namespace tl
