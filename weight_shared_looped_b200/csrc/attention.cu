@@ -10,7 +10,7 @@
 // cache INT8").  The context is split into fixed 64-key chunks (a function of
 // the position only) whose partial results are merged in chunk order, so a
 // lane's output does not depend on the other lanes.
-#include "tl_internal.cuh"
+#include "tl_launch.cuh"
 
 namespace tl {
 namespace {
@@ -54,6 +54,7 @@ __global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __re
                                                               const __half* __restrict__ v,
                                                               __half* __restrict__ out, int T,
                                                               int H, float scale_log2) {
+  pdl_enter();
   constexpr int LD = HD + 8;                 // halves per smem row (16-byte aligned, no conflicts)
   __shared__ __align__(16) __half Ks[FK][LD];
   __shared__ __align__(16) __half Vs[FK][LD];
@@ -203,118 +204,6 @@ __global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __re
 }
 
 // ------------------------------------------------------------------ decode
-// grid (max_chunks, H, rows); 4 warps, 16 keys each.
-template <int HD>
-__global__ void __launch_bounds__(128) attn_decode_partial_kernel(DecodeAttnArgs a) {
-  constexpr int DPL = HD / 32;
-  __shared__ float sc[kDecodeChunk];
-  __shared__ float wacc[4][HD];
-  __shared__ float wl[4];
-  const int chunk = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
-  const int lane_id = a.lane_of_row[row];
-  const int n_keys = a.hdr->pos[lane_id] + 1;   // the current token is already appended
-  const int n_chunks = (n_keys + kDecodeChunk - 1) / kDecodeChunk;
-  if (chunk >= n_chunks) return;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const float scale = rsqrtf((float)HD);
-
-  float qv[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e)
-    qv[e] = __half2float(a.q[(size_t)row * a.d + head * HD + lane * DPL + e]) * scale;
-
-  const char* layer =
-      a.kv_base + (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
-  const size_t head_off = (size_t)head * a.max_ctx;
-  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
-  const __half* ksc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
-  const __half* vsc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
-
-  auto load_row = [&](int which, int pos, float* out) {
-    const size_t eoff = (head_off + pos) * HD + lane * DPL;
-    if (!a.kv_int8) {
-      const __half* p = reinterpret_cast<const __half*>(layer + which * a.kv_region_bytes) + eoff;
-#pragma unroll
-      for (int e = 0; e < DPL; e += 2) {
-        float2 f = __half22float2(*reinterpret_cast<const __half2*>(p + e));
-        out[e] = f.x;
-        out[e + 1] = f.y;
-      }
-    } else {
-      const int8_t* p = reinterpret_cast<const int8_t*>(layer + which * a.kv_region_bytes) + eoff;
-      const float s = __half2float((which == 0 ? ksc : vsc)[head_off + pos]);
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) out[e] = (float)p[e] * s;
-    }
-  };
-
-  const int base = chunk * kDecodeChunk;
-  for (int i = 0; i < kDecodeChunk / 4; ++i) {
-    const int j = warp * (kDecodeChunk / 4) + i;
-    const int pos = base + j;
-    float s = -INFINITY;
-    if (pos < n_keys) {
-      float kr[DPL];
-      load_row(0, pos, kr);
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) dot = fmaf(qv[e], kr[e], dot);
-      s = warp_sum(dot);
-    }
-    if (lane == 0) sc[j] = s;
-  }
-  __syncthreads();
-  float m = -INFINITY;
-  for (int j = 0; j < kDecodeChunk; ++j) m = fmaxf(m, sc[j]);
-  float acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  float lsum = 0.f;
-  for (int i = 0; i < kDecodeChunk / 4; ++i) {
-    const int j = warp * (kDecodeChunk / 4) + i;
-    const int pos = base + j;
-    if (pos >= n_keys) break;
-    const float p = __expf(sc[j] - m);
-    lsum += p;
-    float vr[DPL];
-    load_row(1, pos, vr);
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(p, vr[e], acc[e]);
-  }
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
-  if (lane == 0) wl[warp] = lsum;
-  __syncthreads();
-  float* dst = a.scratch + (((size_t)row * a.H + head) * a.max_chunks + chunk) * (HD + 2);
-  for (int e = threadIdx.x; e < HD; e += 128)
-    dst[e] = wacc[0][e] + wacc[1][e] + wacc[2][e] + wacc[3][e];
-  if (threadIdx.x == 0) {
-    dst[HD] = m;
-    dst[HD + 1] = wl[0] + wl[1] + wl[2] + wl[3];
-  }
-}
-
-// grid (H, rows); merge the chunks of one (row, head) in chunk order.
-template <int HD>
-__global__ void __launch_bounds__(HD) attn_decode_merge_kernel(DecodeAttnArgs a) {
-  const int head = blockIdx.x, row = blockIdx.y;
-  const int lane_id = a.lane_of_row[row];
-  const int n_keys = a.hdr->pos[lane_id] + 1;
-  const int n_chunks = (n_keys + kDecodeChunk - 1) / kDecodeChunk;
-  const float* src = a.scratch + ((size_t)row * a.H + head) * a.max_chunks * (HD + 2);
-  float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, src[c * (HD + 2) + HD]);
-  float L = 0.f, o = 0.f;
-  const int e = threadIdx.x;
-  for (int c = 0; c < n_chunks; ++c) {
-    const float* p = src + c * (HD + 2);
-    const float w = __expf(p[HD] - M);
-    L = fmaf(p[HD + 1], w, L);
-    o = fmaf(p[e], w, o);
-  }
-  a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
-}
-
 // Fused decode attention for one (row, head, 64-key chunk):
 //   * q = sum of the QKV split-K partials, RoPE at the lane's position;
 //   * the CTA holding the lane's newest position also forms k and v, applies
@@ -328,32 +217,86 @@ template <int HD>
 __global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a) {
   constexpr int DPL = HD / 32;
   constexpr int HALF = HD / 2;
+  constexpr int ROWB = HD * 2;                 // bytes of one fp16 row (int8 rows use half)
+  __shared__ __align__(16) unsigned char kv_s[2][kDecodeChunk * ROWB];   // staged K, V rows
+  __shared__ float ks_s[kDecodeChunk], vs_s[kDecodeChunk];                // INT8 scales
   __shared__ float qs[HD], kn[HD], vn[HD];
   __shared__ float sc[kDecodeChunk];
-  __shared__ float wacc[4][HD];
+  __shared__ float wacc[4][HD > kDecodeChunk ? HD : kDecodeChunk];
   __shared__ float wl[4];
   __shared__ float red[4];
   __shared__ int is_last;
+  (void)DPL;
   const int chunk = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
+  // Positions, the lane map, the RoPE table and the cache rows before the
+  // newest position were all written by earlier steps: read them (and start
+  // copying this chunk's K/V rows into shared memory) before waiting for the
+  // QKV projection that produces this token's q, k and v.
   const int lane_id = a.lane_of_row[row];
   const int pos = a.hdr->pos[lane_id];
   const int n_keys = pos + 1;
   const int n_chunks = (n_keys + kDecodeChunk - 1) / kDecodeChunk;
-  if (chunk >= n_chunks) return;
+  if (chunk >= n_chunks) {
+    pdl_enter();
+    return;
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool owner = chunk == n_chunks - 1;    // holds position pos
+  const int base = chunk * kDecodeChunk;
+  const int nk = min(kDecodeChunk, n_keys - base);          // keys in this chunk
+  const int n_old = owner ? nk - 1 : nk;                    // rows already in the cache
+  char* layer = const_cast<char*>(a.kv_base) +
+                (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
+  const size_t head_off = (size_t)head * a.max_ctx;
+  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
+  const int esz = a.kv_int8 ? 1 : 2;
+  {
+    const int chunks16 = HD * esz / 16;                      // 16-byte pieces per row
+    for (int which = 0; which < 2; ++which) {
+      const char* src = layer + which * a.kv_region_bytes + (head_off + base) * HD * esz;
+      for (int i = threadIdx.x; i < n_old * chunks16; i += 128) {
+        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(kv_s[which] + i * 16);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + i * 16)
+                     : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (a.kv_int8 && threadIdx.x < n_old) {
+      const __half* ksc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
+      const __half* vsc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
+      ks_s[threadIdx.x] = __half2float(ksc[head_off + base + threadIdx.x]);
+      vs_s[threadIdx.x] = __half2float(vsc[head_off + base + threadIdx.x]);
+    }
+  }
+  const int i = threadIdx.x;
+  float2 cs = make_float2(1.f, 0.f);
+  if (i < HD) cs = a.rope_cs[(size_t)pos * HALF + (i % HALF)];
+  pdl_enter();
+
+  // q (and k, v for the owner) from the QKV partial sums, all splits in flight
   const size_t split_stride = (size_t)a.rows * 3 * a.d;
   const float* prow = a.qkv_part + (size_t)row * 3 * a.d + (size_t)head * HD;
-
-  // q (and k, v for the owner) from the partial sums
-  for (int i = threadIdx.x; i < HD; i += 128) {
+  if (i < HD) {
+    float pq[8], pk[8], pv[8];
     float sq = 0.f, sk = 0.f, sv = 0.f;
-    for (int sp = 0; sp < a.qkv_S; ++sp) {
-      const float* p = prow + sp * split_stride;
-      sq += p[i];
-      if (owner) {
-        sk += p[a.d + i];
-        sv += p[2 * a.d + i];
+    for (int s0 = 0; s0 < a.qkv_S; s0 += 8) {
+      const int cnt = min(8, a.qkv_S - s0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < cnt) {
+          const float* p = prow + (size_t)(s0 + j) * split_stride;
+          pq[j] = p[i];
+          pk[j] = owner ? p[a.d + i] : 0.f;
+          pv[j] = owner ? p[2 * a.d + i] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < cnt) {
+          sq += pq[j];
+          sk += pk[j];
+          sv += pv[j];
+        }
       }
     }
     qs[i] = sq;
@@ -362,9 +305,7 @@ __global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a
   }
   __syncthreads();
   float qr = 0.f, kr = 0.f;
-  const int i = threadIdx.x;
   if (i < HD) {
-    const float2 cs = a.rope_cs[(size_t)pos * HALF + (i % HALF)];
     if (i < HALF) {
       qr = qs[i] * cs.x - qs[i + HALF] * cs.y;
       kr = kn[i] * cs.x - kn[i + HALF] * cs.y;
@@ -374,23 +315,22 @@ __global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a
     }
   }
   __syncthreads();
-  const char* layer_c =
-      a.kv_base + (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
-  char* layer = const_cast<char*>(layer_c);
-  const size_t head_off = (size_t)head * a.max_ctx;
-  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
   if (i < HD) {
     // the query is rounded to fp16 as in the unfused path
     qs[i] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
   }
   if (owner) {
-    // append k (after RoPE) and v at position pos
+    // append k (after RoPE) and v at position pos, in the cache and in the
+    // staged rows
+    const int jr = nk - 1;
     const __half kh = __float2half_rn(kr);
     const __half vh = __float2half_rn(i < HD ? vn[i] : 0.f);
     if (!a.kv_int8) {
       if (i < HD) {
         reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + i] = kh;
         reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = vh;
+        reinterpret_cast<__half*>(kv_s[0])[jr * HD + i] = kh;
+        reinterpret_cast<__half*>(kv_s[1])[jr * HD + i] = vh;
       }
     } else {
       float km = i < HD ? fabsf(__half2float(kh)) : 0.f;
@@ -406,89 +346,117 @@ __global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a
       vm = fmaxf(fmaxf(wl[0], wl[1]), fmaxf(wl[2], wl[3]));
       const __half ksh = __float2half_rn(__fdiv_rn(km, 127.0f));
       const __half vsh = __float2half_rn(__fdiv_rn(vm, 127.0f));
-      const float ks = __half2float(ksh), vs = __half2float(vsh);
+      const float ksf = __half2float(ksh), vsf = __half2float(vsh);
       if (i < HD) {
         const float kx = __half2float(kh), vx = __half2float(vh);
-        const int kc = ks == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ks)), -127.f), 127.f);
-        const int vc = vs == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vs)), -127.f), 127.f);
+        const int kc = ksf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ksf)), -127.f), 127.f);
+        const int vc = vsf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vsf)), -127.f), 127.f);
         reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + i] = (int8_t)kc;
         reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = (int8_t)vc;
+        reinterpret_cast<int8_t*>(kv_s[0])[jr * HD + i] = (int8_t)kc;
+        reinterpret_cast<int8_t*>(kv_s[1])[jr * HD + i] = (int8_t)vc;
       }
       if (i == 0) {
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] =
             vsh;
+        ks_s[jr] = ksf;
+        vs_s[jr] = vsf;
       }
     }
   }
-  __syncthreads();   // the appended entry and qs are visible to the whole CTA
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();   // staged rows, the appended entry and qs are visible to the whole CTA
 
-  const __half* ksc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
-  const __half* vsc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
-  auto load_row = [&](int which, int p, float* out) {
-    const size_t eoff = (head_off + p) * HD + lane * DPL;
-    if (!a.kv_int8) {
-      const __half* src = reinterpret_cast<const __half*>(layer + which * a.kv_region_bytes) + eoff;
+  // scores: thread (j, half) takes key base + j over one half of head_dim
+  {
+    const int j = threadIdx.x % kDecodeChunk, hf = threadIdx.x / kDecodeChunk;
+    float dot = 0.f;
+    if (j < nk) {
+      const int d0 = hf * HALF;
+      if (!a.kv_int8) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __half*>(kv_s[0]) + j * HD + d0);
 #pragma unroll
-      for (int e = 0; e < DPL; e += 2) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(src + e));
-        out[e] = f.x;
-        out[e + 1] = f.y;
+        for (int c = 0; c < HALF / 8; ++c) {
+          const uint4 w = src[c];
+          const __half2* hp = reinterpret_cast<const __half2*>(&w);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __half22float2(hp[e]);
+            dot = fmaf(qs[d0 + c * 8 + 2 * e], f.x, dot);
+            dot = fmaf(qs[d0 + c * 8 + 2 * e + 1], f.y, dot);
+          }
+        }
+      } else {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const int8_t*>(kv_s[0]) + j * HD + d0);
+        float part = 0.f;
+#pragma unroll
+        for (int c = 0; c < HALF / 16; ++c) {
+          const uint4 w = src[c];
+          const int8_t* bp = reinterpret_cast<const int8_t*>(&w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) part = fmaf(qs[d0 + c * 16 + e], (float)bp[e], part);
+        }
+        dot = part * ks_s[j];
       }
-    } else {
-      const int8_t* src = reinterpret_cast<const int8_t*>(layer + which * a.kv_region_bytes) + eoff;
-      const float sc_ = __half2float((which == 0 ? ksc : vsc)[head_off + p]);
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) out[e] = (float)src[e] * sc_;
     }
-  };
-  float qv[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) qv[e] = qs[lane * DPL + e];
-  const int base = chunk * kDecodeChunk;
-  for (int j0 = 0; j0 < kDecodeChunk / 4; ++j0) {
-    const int j = warp * (kDecodeChunk / 4) + j0;
-    const int p = base + j;
-    float sv = -INFINITY;
-    if (p < n_keys) {
-      float kr2[DPL];
-      load_row(0, p, kr2);
-      float dot = 0.f;
-#pragma unroll
-      for (int e = 0; e < DPL; ++e) dot = fmaf(qv[e], kr2[e], dot);
-      sv = warp_sum(dot);
-    }
-    if (lane == 0) sc[j] = sv;
+    wacc[hf][j] = dot;
   }
+  __syncthreads();
+  if (threadIdx.x < kDecodeChunk)
+    sc[threadIdx.x] = threadIdx.x < nk ? wacc[0][threadIdx.x] + wacc[1][threadIdx.x] : -INFINITY;
   __syncthreads();
   float m = -INFINITY;
   for (int j = 0; j < kDecodeChunk; ++j) m = fmaxf(m, sc[j]);
-  float acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  float lsum = 0.f;
-  for (int j0 = 0; j0 < kDecodeChunk / 4; ++j0) {
-    const int j = warp * (kDecodeChunk / 4) + j0;
-    const int p = base + j;
-    if (p >= n_keys) break;
-    const float pr = __expf(sc[j] - m);
-    lsum += pr;
-    float vr[DPL];
-    load_row(1, p, vr);
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = fmaf(pr, vr[e], acc[e]);
+  __syncthreads();
+  if (threadIdx.x < kDecodeChunk) {
+    const int j = threadIdx.x;
+    sc[j] = j < nk ? __expf(sc[j] - m) : 0.f;
+    if (a.kv_int8) wacc[3][j] = j < nk ? vs_s[j] : 0.f;
   }
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
-  if (lane == 0) wl[warp] = lsum;
+  __syncthreads();
+  // P V: thread (e, ks) takes dimension e over key slice ks
+  constexpr int KSPLIT = 128 / HD;
+  constexpr int KPER = kDecodeChunk / KSPLIT;
+  {
+    const int e = threadIdx.x % HD, ks = threadIdx.x / HD;
+    float acc = 0.f;
+    const int j0 = ks * KPER;
+    if (!a.kv_int8) {
+      const __half* src = reinterpret_cast<const __half*>(kv_s[1]) + e;
+#pragma unroll 8
+      for (int jj = 0; jj < KPER; ++jj) {
+        const int j = j0 + jj;
+        if (j < nk) acc = fmaf(sc[j], __half2float(src[j * HD]), acc);
+      }
+    } else {
+      const int8_t* src = reinterpret_cast<const int8_t*>(kv_s[1]) + e;
+#pragma unroll 8
+      for (int jj = 0; jj < KPER; ++jj) {
+        const int j = j0 + jj;
+        if (j < nk) acc = fmaf(sc[j] * wacc[3][j], (float)src[j * HD], acc);
+      }
+    }
+    wacc[ks][e] = acc;     // (scores in wacc[0..1] are no longer needed)
+  }
+  if (threadIdx.x < 32) {
+    float l = sc[threadIdx.x] + sc[threadIdx.x + 32];
+    l = warp_sum(l);
+    if (threadIdx.x == 0) wl[0] = l;
+  }
   __syncthreads();
   float* part = a.scratch + ((size_t)row * a.H + head) * a.max_chunks * (HD + 2);
   float* dst = part + (size_t)chunk * (HD + 2);
-  for (int e = threadIdx.x; e < HD; e += 128)
-    dst[e] = wacc[0][e] + wacc[1][e] + wacc[2][e] + wacc[3][e];
+  for (int e = threadIdx.x; e < HD; e += 128) {
+    float o = wacc[0][e];
+    if (KSPLIT > 1) o += wacc[1][e];
+    dst[e] = o;
+  }
   if (threadIdx.x == 0) {
     dst[HD] = m;
-    dst[HD + 1] = wl[0] + wl[1] + wl[2] + wl[3];
+    dst[HD + 1] = wl[0];
   }
   // last CTA of this (row, head) merges
   __threadfence();
@@ -524,12 +492,11 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   dim3 grid((T + FQ - 1) / FQ, H);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
   if (hd == 128)
-    attn_prefill_tc_kernel<128><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 128, 0, s, q, k, v, out, T, H, scale_log2);
   else if (hd == 64)
-    attn_prefill_tc_kernel<64><<<grid, 128, 0, s>>>(q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<64>, grid, 128, 0, s, q, k, v, out, T, H, scale_log2);
   else
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", hd);
-  TL_LAUNCH_CHECK();
   return ok();
 }
 
@@ -537,30 +504,11 @@ tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
   dim3 grid(a.max_chunks, a.H, a.rows);
   if (a.hd == 128)
-    attn_decode_fused_kernel<128><<<grid, 128, 0, s>>>(a);
+    TL_LAUNCH_PDL(attn_decode_fused_kernel<128>, grid, 128, 0, s, a);
   else if (a.hd == 64)
-    attn_decode_fused_kernel<64><<<grid, 128, 0, s>>>(a);
+    TL_LAUNCH_PDL(attn_decode_fused_kernel<64>, grid, 128, 0, s, a);
   else
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
-  TL_LAUNCH_CHECK();
-  return ok();
-}
-
-tl_status launch_attn_decode(const DecodeAttnArgs& a, cudaStream_t s) {
-  if (a.rows == 0) return ok();
-  dim3 g1(a.max_chunks, a.H, a.rows), g2(a.H, a.rows);
-  if (a.hd == 128) {
-    attn_decode_partial_kernel<128><<<g1, 128, 0, s>>>(a);
-    TL_LAUNCH_CHECK();
-    attn_decode_merge_kernel<128><<<g2, 128, 0, s>>>(a);
-  } else if (a.hd == 64) {
-    attn_decode_partial_kernel<64><<<g1, 128, 0, s>>>(a);
-    TL_LAUNCH_CHECK();
-    attn_decode_merge_kernel<64><<<g2, 64, 0, s>>>(a);
-  } else {
-    return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
-  }
-  TL_LAUNCH_CHECK();
   return ok();
 }
 
