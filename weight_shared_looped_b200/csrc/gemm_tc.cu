@@ -3,27 +3,26 @@
 //   part[z][t][n] = sum over k in split z of x[t][k] * W[n][k],
 //   W[n][k] = code[n][k] * scale[n][k / G]  (group-wise symmetric INT4).
 //
-// One CTA computes 128 weight rows x BN tokens over a range of 64-wide k
-// blocks.  Per k block:
-//   * a TMA warp loads the activation tile x[BN tokens][64 k] (fp16, 128-byte
-//     swizzled, rows past T read as zero) and the packed weight tile
-//     [128 rows][8 words] into a shared-memory stage;
-//   * sixteen dequantisation warps (four groups of four, one warp per TMEM
-//     lane quadrant in each group; group g takes k blocks i with i % 4 == g;
-//     one thread per weight row) turn the row's 64 codes into fp16 code*scale
-//     pairs and store them straight into tensor memory with tcgen05.st: the
-//     weight tile is the A operand of the MMA and never passes through shared
-//     memory;
-//   * one thread issues four tcgen05.mma kind::f16 (M 128, N BN, K 16), A from
-//     TMEM, B from the swizzled shared-memory tile, fp32 accumulation in TMEM,
-//     and commits to the stage's "empty" barrier.
-// The same warps then read the accumulator back with tcgen05.ld and store it as
-// fp32 partial sums, and signal an "epilogue done" barrier that the MMA warp
-// waits on before it frees TMEM.  A CTA owns all of TMEM and 8 (5 for 256
-// tokens) pipeline stages; split-K counts are chosen so that one wave of CTAs
-// covers the 148 SMs.  Every wait on an mbarrier is bounded: when a wait
-// runs out the CTA records TL_ERR_TIMEOUT in the status word, stops issuing
-// work, waits (bounded) for its copies in flight, frees its TMEM and returns.
+// One CTA per SM computes 128 weight rows x BN tokens over a range of 64-wide
+// k blocks, with three decoupled rings:
+//   * packed weights (128 rows x 8 words per k block) loaded by TMA far ahead
+//     (the first loads are issued before waiting for the previous kernel: the
+//     weights are constants of the model);
+//   * the fp16 A tiles in tensor memory: sixteen dequantisation warps (four
+//     groups of four, one warp per TMEM lane quadrant; group g takes k blocks
+//     i with i % 4 == g; one thread per weight row) turn a row's 64 codes into
+//     fp16 code*scale pairs and store them with tcgen05.st, so the weight tile
+//     is the MMA's A operand and never passes through shared memory;
+//   * the activation tiles x[BN tokens][64 k] (fp16, 128-byte swizzled, rows
+//     past T read as zero) loaded by a second TMA warp.
+// One thread issues tcgen05.mma kind::f16 (M 128, N BN, K 16; A from TMEM, B
+// from shared memory, fp32 accumulation in TMEM) for batches of ready k blocks
+// and commits each k block to the rings it frees.  The dequantisation warps
+// then read the accumulator back with tcgen05.ld, store fp32 partial sums and
+// signal an "epilogue done" barrier that the MMA warp waits on before it frees
+// TMEM.  Every wait on an mbarrier is bounded: when a wait runs out the CTA
+// records TL_ERR_TIMEOUT, stops issuing work, waits (bounded) for its copies in
+// flight, frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -36,15 +35,19 @@ constexpr int BM = 128;            // weight rows per CTA (MMA M)
 constexpr int BK = 64;             // k per stage
 constexpr int DQ_GROUPS = 4;       // dequantisation groups, each 4 warps (one per TMEM quadrant)
 constexpr int DQ_WARPS = 4 * DQ_GROUPS;
-constexpr int TMA_WARP = DQ_WARPS, MMA_WARP = DQ_WARPS + 1;
-constexpr int THREADS = 32 * (DQ_WARPS + 2);
+constexpr int WTMA_WARP = DQ_WARPS, XTMA_WARP = DQ_WARPS + 1, MMA_WARP = DQ_WARPS + 2;
+constexpr int THREADS = 32 * (DQ_WARPS + 3);
 constexpr int TMEM_COLS = 512;     // the whole of TMEM: one CTA per SM
-constexpr size_t kMinSmem = 120 * 1024;   // also keeps it to one CTA per SM
-template <int BN> struct TcCfg {
-  static constexpr int STAGES = BN >= 256 ? 5 : 8;
-};
 constexpr int A_COLS = BK / 2;     // TMEM columns per A stage (two fp16 per column)
+constexpr int BATCH = DQ_GROUPS;   // k blocks per batch: one per dequantisation group
+constexpr size_t kMinSmem = 120 * 1024;   // also keeps it to one CTA per SM
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a bounded wait gives up after 2 s
+template <int BN> struct TcCfg {
+  static constexpr int W_STAGES = 2 * BATCH;                  // packed-weight ring (k blocks)
+  static constexpr int X_BATCHES = BN >= 128 ? 2 : 3;         // activation ring (batches)
+  static constexpr int A_BATCHES = (TMEM_COLS - BN) / (A_COLS * BATCH);   // TMEM A ring (batches)
+  static constexpr int D_BATCHES = A_BATCHES > X_BATCHES ? A_BATCHES : X_BATCHES;
+};
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
@@ -157,28 +160,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                       const __grid_constant__ CUtensorMap map_w0,
                       const __grid_constant__ CUtensorMap map_w1, TcArgs a) {
-  constexpr int STAGES = TcCfg<BN>::STAGES;
-  constexpr uint32_t B_BYTES = BN * 128;          // BN rows x 64 fp16
+  constexpr int WS = TcCfg<BN>::W_STAGES, XB = TcCfg<BN>::X_BATCHES;
+  constexpr int AB = TcCfg<BN>::A_BATCHES, DB = TcCfg<BN>::D_BATCHES;
+  constexpr uint32_t X_BYTES = BN * 128;          // BN rows x 64 fp16
   constexpr uint32_t W_BYTES = BM * 32;           // 128 rows x 8 words
-  static_assert(BN + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(BN + AB * BATCH * A_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(AB >= 2 && XB >= 2 && WS % DQ_GROUPS == 0, "ring depths");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  // 1024-align the dynamic shared memory base
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sB = smem;                                        // STAGES x B_BYTES
-  uint8_t* sW = sB + STAGES * B_BYTES;                       // STAGES x W_BYTES
-  __half* sScale = reinterpret_cast<__half*>(sW + STAGES * W_BYTES);   // [BM][groups]
+  uint8_t* sX = smem;                                        // XB*BATCH x X_BYTES
+  uint8_t* sW = sX + XB * BATCH * X_BYTES;                   // WS x W_BYTES
+  __half* sScale = reinterpret_cast<__half*>(sW + WS * W_BYTES);   // [BM][groups]
   const int nkb_total = a.K / BK;
   const int kb_begin = (int)(((long)blockIdx.z * nkb_total) / a.splits);
   const int nkb = (int)(((long)(blockIdx.z + 1) * nkb_total) / a.splits) - kb_begin;
+  const int nbatch = (nkb + BATCH - 1) / BATCH;
   const int g_first = (kb_begin * BK) / a.G;
   const int groups = ((kb_begin + nkb) * BK - 1) / a.G - g_first + 1;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sScale + BM * a.max_groups + 8);
   bars = reinterpret_cast<uint64_t*>(((uintptr_t)bars + 7) & ~(uintptr_t)7);
-  uint64_t* full = bars;                 // TMA landed
-  uint64_t* empty = bars + STAGES;       // MMA done with the stage
-  uint64_t* afull = bars + 2 * STAGES;   // A stage written to TMEM
-  uint64_t* accb = bars + 3 * STAGES;    // accumulator complete
-  uint64_t* epib = accb + 1;             // epilogue finished reading TMEM
+  uint64_t* wfull = bars;               // packed weights of a k block landed
+  uint64_t* wempty = wfull + WS;        // dequantisation done reading them
+  uint64_t* xfull = wempty + WS;        // activations of a batch landed
+  uint64_t* afull = xfull + XB;         // A tiles of a batch in TMEM (and its activations seen)
+  uint64_t* done = afull + AB;          // MMAs of a batch complete: frees its X and A slots
+  uint64_t* accb = done + DB;           // accumulator complete
+  uint64_t* epib = accb + 1;            // epilogue finished reading TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epib + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
@@ -191,11 +198,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   const __half* scales = second ? a.s1 : a.s0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 4);
+    for (int s = 0; s < WS; ++s) {
+      mbar_init(&wfull[s], 1);
+      mbar_init(&wempty[s], 4);
     }
+    for (int s = 0; s < XB; ++s) mbar_init(&xfull[s], 1);
+    for (int s = 0; s < AB; ++s) mbar_init(&afull[s], DQ_WARPS);
+    for (int s = 0; s < DB; ++s) mbar_init(&done[s], 1);
     mbar_init(accb, 1);
     mbar_init(epib, DQ_WARPS);
     *abort_flag = 0;
@@ -214,70 +223,77 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem_base = *tmem_slot;
-  // everything above is CTA-local; from here on the kernel reads what the
-  // previous kernel wrote (the activations), so wait for it here
-  pdl_enter();
   const uint32_t acc_col = 0;
   const uint32_t a_col0 = BN;
 
-  if (warp == TMA_WARP) {
-    // ---------------------------------------------------------------- TMA
+  if (warp == WTMA_WARP) {
+    // ---------------------------------------------------------------- weight TMA
+    // weights are constants of the model: no need to wait for the previous kernel
     if (lane == 0) {
       int issued = 0;
       for (int i = 0; i < nkb; ++i) {
-        const int s = i % STAGES;
-        if (i >= STAGES) {
-          if (!mbar_wait(&empty[s], ((i / STAGES) - 1) & 1)) {
-            atomicExch(abort_flag, 1);
-            break;
-          }
+        const int s = i % WS;
+        if (i >= WS && !mbar_wait(&wempty[s], ((i / WS) - 1) & 1)) {
+          atomicExch(abort_flag, 1);
+          break;
         }
         if (*(volatile int*)abort_flag) break;
-        mbar_expect_tx(&full[s], B_BYTES + W_BYTES);
-        const int kb = kb_begin + i;
-        tma_load_2d(sB + s * B_BYTES, &map_x, kb * BK, t0, &full[s]);
-        tma_load_2d(sW + s * W_BYTES, map_w, kb * (BK / 8), wrow0, &full[s]);
+        mbar_expect_tx(&wfull[s], W_BYTES);
+        tma_load_2d(sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
         issued = i + 1;
       }
-      // on abort, let every copy already issued land before the CTA exits
-      if (*(volatile int*)abort_flag) {
-        for (int i = 0; i < issued; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1);
+      if (*(volatile int*)abort_flag)
+        for (int i = 0; i < issued; ++i) mbar_wait(&wfull[i % WS], (i / WS) & 1);
+    }
+    __syncwarp();
+    pdl_enter();
+  } else if (warp == XTMA_WARP) {
+    // ---------------------------------------------------------------- activation TMA
+    pdl_enter();   // the activations come from the previous kernel
+    if (lane == 0) {
+      int issued = 0;
+      for (int b = 0; b < nbatch; ++b) {
+        if (b >= XB && !mbar_wait(&done[(b - XB) % DB], ((b - XB) / DB) & 1)) {
+          atomicExch(abort_flag, 1);
+          break;
+        }
+        if (*(volatile int*)abort_flag) break;
+        const int cnt = min(BATCH, nkb - b * BATCH);
+        uint64_t* bar = &xfull[b % XB];
+        mbar_expect_tx(bar, cnt * X_BYTES);
+        for (int j = 0; j < cnt; ++j)
+          tma_load_2d(sX + ((b % XB) * BATCH + j) * X_BYTES, &map_x,
+                      (kb_begin + b * BATCH + j) * BK, t0, bar);
+        issued = b + 1;
       }
+      if (*(volatile int*)abort_flag)
+        for (int b = 0; b < issued; ++b) mbar_wait(&xfull[b % XB], (b / XB) & 1);
     }
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ---------------------------------------------------------------- MMA
+    // per batch: one wait (A tiles written and activations seen), one fence,
+    // up to 16 MMAs, one commit
+    pdl_enter();
     if (lane == 0) {
       const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-      // k blocks are issued in batches of up to MMA_BATCH that are already
-      // dequantised: one tcgen05.fence per batch instead of per k block
-      constexpr int MMA_BATCH = 4;
-      bool ok = true;
-      for (int i0 = 0; i0 < nkb && ok; i0 += MMA_BATCH) {
-        const int cnt = min(MMA_BATCH, nkb - i0);
-        for (int j = 0; j < cnt; ++j) {
-          const int i = i0 + j, s = i % STAGES;
-          if (!mbar_wait(&full[s], (i / STAGES) & 1) || !mbar_wait(&afull[s], (i / STAGES) & 1)) {
-            ok = false;
-            break;
-          }
-        }
-        if (!ok || *(volatile int*)abort_flag) {
+      for (int b = 0; b < nbatch; ++b) {
+        if (!mbar_wait(&afull[b % AB], (b / AB) & 1) || *(volatile int*)abort_flag) {
           atomicExch(abort_flag, 1);
-          ok = false;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const int cnt = min(BATCH, nkb - b * BATCH);
         for (int j = 0; j < cnt; ++j) {
-          const int i = i0 + j, s = i % STAGES;
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sB + s * B_BYTES));
-          const uint32_t a_tm = tmem_base + a_col0 + s * A_COLS;
+          const int i = b * BATCH + j;
+          const uint64_t bdesc = smem_desc_sw128(smem_u32(sX + ((b % XB) * BATCH + j) * X_BYTES));
+          const uint32_t a_tm = tmem_base + a_col0 + ((b % AB) * BATCH + j) * A_COLS;
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_ts(tmem_base + acc_col, a_tm + k * 8, bdesc + (uint64_t)(2 * k), idesc,
                    (i > 0 || k > 0) ? 1u : 0u);
-          mma_commit(&empty[s]);
         }
+        mma_commit(&done[b % DB]);
       }
       mma_commit(accb);   // arrives once all issued MMAs are complete
     }
@@ -285,11 +301,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else {
     // ---------------------------------------------------------------- dequant + epilogue
     const int quad = warp & 3;
-    const int parity = warp >> 2;               // group: takes k blocks i with i % DQ_GROUPS == parity
+    const int grp = warp >> 2;                  // this group takes k block grp of every batch
     const int r = quad * 32 + lane;             // weight row within the tile = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    // scales of this CTA's rows and k range -> shared memory (the TMA warp is
-    // already streaming; only the dequantisation warps wait for the scales)
+    // scales of this CTA's rows and k range -> shared memory (constants: read
+    // before waiting for the previous kernel)
     {
       const int gpr = a.K / a.G;
       const int g0 = g_first;
@@ -300,52 +316,70 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * DQ_WARPS) : "memory");
     }
-    for (int i = parity; i < nkb; i += DQ_GROUPS) {
-      const int s = i % STAGES;
-      if (!mbar_wait(&full[s], (i / STAGES) & 1) || *(volatile int*)abort_flag) {
+    for (int b = 0; b < nbatch; ++b) {
+      const int i = b * BATCH + grp;
+      // the TMEM slot of this batch is free once batch b - AB is done
+      if (b >= AB && !mbar_wait(&done[(b - AB) % DB], ((b - AB) / DB) & 1)) {
         atomicExch(abort_flag, 1);
         break;
       }
-      const uint4* wp = reinterpret_cast<const uint4*>(sW + s * W_BYTES + r * 32);
-      const uint4 wa = wp[0], wb = wp[1];
-      const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-      const int g = ((kb_begin + i) * BK) / a.G - g_first;
-      const __half sc = sScale[r * groups + g];
-      const __half2 s2 = __halves2half2(sc, sc);
-      uint32_t v[32];
+      if (i < nkb) {
+        const int ws = i % WS;
+        if (!mbar_wait(&wfull[ws], (i / WS) & 1) || *(volatile int*)abort_flag) {
+          atomicExch(abort_flag, 1);
+          break;
+        }
+        const uint4* wp = reinterpret_cast<const uint4*>(sW + ws * W_BYTES + r * 32);
+        const uint4 wa = wp[0], wb = wp[1];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&wempty[ws]);   // the packed words are in registers
+        const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        const int g = ((kb_begin + i) * BK) / a.G - g_first;
+        const __half sc = sScale[r * groups + g];
+        const __half2 s2 = __halves2half2(sc, sc);
+        uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const uint32_t b = c & 3;
-        const uint32_t sel = b | 0x40u | (b << 8) | 0x4000u;
-        uint32_t code = dequant_code_pair(words[c >> 2], sel);
-        __half2 wv = __hmul2(*reinterpret_cast<__half2*>(&code), s2);
-        v[c] = *reinterpret_cast<uint32_t*>(&wv);
+        for (int c = 0; c < 32; ++c) {
+          const uint32_t bb = c & 3;
+          const uint32_t sel = bb | 0x40u | (bb << 8) | 0x4000u;
+          uint32_t code = dequant_code_pair(words[c >> 2], sel);
+          __half2 wv = __hmul2(*reinterpret_cast<__half2*>(&code), s2);
+          v[c] = *reinterpret_cast<uint32_t*>(&wv);
+        }
+        if (b >= AB) asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const uint32_t taddr = tmem_base + lane_addr + a_col0 + ((b % AB) * BATCH + grp) * A_COLS;
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+            "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+            "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+            "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+            "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+            "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+            "r"(v[29]), "r"(v[30]), "r"(v[31])
+            : "memory");
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       }
-      const uint32_t taddr = tmem_base + lane_addr + a_col0 + s * A_COLS;
-      asm volatile(
-          "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, "
-          "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
-          "%27, %28, %29, %30, %31, %32};" ::"r"(taddr),
-          "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
-          "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
-          "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
-          "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
-          "r"(v[29]), "r"(v[30]), "r"(v[31])
-          : "memory");
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      // the batch's activations must have landed before the MMA thread (which
+      // waits only on afull) reads them
+      if (!mbar_wait(&xfull[b % XB], (b / XB) & 1)) {
+        atomicExch(abort_flag, 1);
+        break;
+      }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[s]);
+      if (lane == 0) mbar_arrive(&afull[b % AB]);
     }
+    pdl_enter();
     // epilogue: accumulator rows = weight rows, columns = tokens
     const bool ok = mbar_wait(accb, 0) && !*(volatile int*)abort_flag;
     if (!ok) atomicExch(abort_flag, 1);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     if (ok) {
       float* out = a.part + (size_t)blockIdx.z * a.T * a.N + (size_t)(m0 + r);
-      // this group's 32-token chunks: cc = parity, parity + 2, ...
+      // this group's 32-token chunks: cc = grp, grp + DQ_GROUPS, ...
 #pragma unroll 1
-      for (int cc = parity; cc < BN / 32; cc += DQ_GROUPS) {
+      for (int cc = grp; cc < BN / 32; cc += DQ_GROUPS) {
         if (t0 + cc * 32 >= a.T) break;   // warp-uniform
         uint32_t u[32];
         asm volatile(
@@ -379,10 +413,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   if (warp == MMA_WARP) {
     // free TMEM only once every epilogue warp has finished reading it
-    bool done = true;
-    if (lane == 0) done = mbar_wait(epib, 0);
-    done = __shfl_sync(0xffffffffu, done ? 1 : 0, 0) != 0;
-    if (!done && lane == 0) atomicExch(abort_flag, 1);
+    bool ok2 = true;
+    if (lane == 0) ok2 = mbar_wait(epib, 0);
+    ok2 = __shfl_sync(0xffffffffu, ok2 ? 1 : 0, 0) != 0;
+    if (!ok2 && lane == 0) atomicExch(abort_flag, 1);
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(TMEM_COLS));
@@ -433,16 +467,14 @@ tl_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
   return ok();
 }
 
-int tc_tile_n(int T) {
-  if (T >= 256) return 256;
-  return T <= 64 ? 64 : 128;
-}
+int tc_tile_n(int T) { return T <= 64 ? 64 : 128; }
 
 template <int BN>
 size_t tc_smem_bytes(int max_groups) {
-  constexpr int STAGES = TcCfg<BN>::STAGES;
-  size_t b = 1024 + (size_t)STAGES * (BN * 128 + BM * 32) + (size_t)BM * max_groups * 2 + 16 +
-             (4 * STAGES + 2) * 8 + 16;
+  constexpr int WS = TcCfg<BN>::W_STAGES, XB = TcCfg<BN>::X_BATCHES;
+  constexpr int AB = TcCfg<BN>::A_BATCHES, DB = TcCfg<BN>::D_BATCHES;
+  size_t b = 1024 + (size_t)XB * BATCH * BN * 128 + (size_t)WS * BM * 32 +
+             (size_t)BM * max_groups * 2 + 16 + (2 * WS + XB + AB + DB + 2) * 8 + 16;
   return b < kMinSmem ? kMinSmem : b;
 }
 
@@ -478,6 +510,8 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.part = g.part;
   a.status = g.status;
   const size_t smem = tc_smem_bytes<BN>(a.max_groups);
+  if (smem > 232448)
+    return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs %zu bytes of shared memory", smem);
   dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
   TL_LAUNCH_PDL(gemm_w4_tc_kernel<BN>, grid, THREADS, smem, s, mx, mw0, mw1, a);
   return ok();
@@ -501,8 +535,6 @@ tl_status gemm_tc_init() {
                                232448));
   TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<256>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
   done = true;
   return ok();
 }
@@ -523,9 +555,7 @@ tl_status launch_gemm_tc(const GemmArgs& g, cudaStream_t s) {
   if (g.T == 0) return ok();
   if (g.n_split % BM != 0)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs row split %% 128 == 0");
-  const int bn = tc_tile_n(g.T);
-  if (bn == 256) return launch_tc_bn<256>(g, s);
-  if (bn == 128) return launch_tc_bn<128>(g, s);
+  if (tc_tile_n(g.T) == 128) return launch_tc_bn<128>(g, s);
   return launch_tc_bn<64>(g, s);
 }
 
