@@ -262,7 +262,6 @@ def run_ours(args, rank, world, dist):
     _build.build()
     import synthetic as syn
     import weight_shared_looped_b200 as tl
-    from oracle import tinyloop_oracle as o   # noqa: F401  (block_cfg helper only)
     from weight_shared_looped_b200.model import DeviceBlock, DeviceModel
 
     dev = int(os.environ.get("LOCAL_RANK", 0))
@@ -315,7 +314,7 @@ def run_ours(args, rank, world, dist):
         step()
     torch.cuda.synchronize()
     assert model.sync_status() == tl.TL_OK
-    with ClockSampler(gpu_uuid(torch, dev)) as clk:
+    with ClockSampler(gpu_uuid(torch, dev)) as clk, torch.cuda.nvtx.range("prefill"):
         t = timed(step, args.steps, 0)
     assert model.sync_status() == tl.TL_OK
     t = max_over_ranks(t, dist, "cuda")
@@ -409,7 +408,8 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
     dstep()
     kv.set_position(0, w.seq)
     it = iter(range(10 ** 9))
-    t = max_t(timed(dstep, w.steps, 0))
+    with torch.cuda.nvtx.range("decode_b1"):
+        t = max_t(timed(dstep, w.steps, 0))
     avg_ctx = w.seq + (w.steps + 1) / 2
     kv_bytes = 10 * avg_ctx * 2048 * 2 * 2
     step_bytes = 3 * blk_bytes + kv_bytes
@@ -437,7 +437,8 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
     dstep8()
     for b in range(8):
         kv.set_position(b, w.seq)
-    t = max_t(timed(dstep8, w.steps, 0))
+    with torch.cuda.nvtx.range("decode_b8"):
+        t = max_t(timed(dstep8, w.steps, 0))
     avg_ctx = w.seq + (w.steps + 1) / 2
     kv_bytes = 8 * 10 * avg_ctx * 16 * (2 * 128 + 2 * 2)
     step_bytes = 3 * blk_bytes + kv_bytes
@@ -468,7 +469,8 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
     dstep3()
     for b in range(3):
         kv.set_position(b, w.seq)
-    t = max_t(timed(dstep3, w.steps, 0))
+    with torch.cuda.nvtx.range("decode_b3"):
+        t = max_t(timed(dstep3, w.steps, 0))
     avg_ctx = w.seq + (w.steps + 1) / 2
     slots = sum(2 + L for L in w.L)
     kv_bytes = slots * avg_ctx * 2048 * 2 * 2
