@@ -321,7 +321,7 @@ def run_ours(args, rank, world, dist):
     value = job_value(seq * args.steps, world, t)
     ms_per_step = t / args.steps * 1e3
     n_layers = 2 + L
-    launches_per_fwd = 2 + 9 * n_layers
+    launches_per_fwd = 2 + 8 * n_layers   # embed, final norm; per layer norm, QKV, RoPE+KV, attention, O, norm, gate|up+SwiGLU, down
 
     # e2e: host (pinned) ids in, host y out, through the C-ABI call
     ids_h = torch.from_numpy(syn.prompt_ids(w).astype(np.int32)).pin_memory()

@@ -734,8 +734,13 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     dn.tickets = m->gemv_tickets;
     TL_TRY(launch_gemm(dn, s));
   } else {
-    TL_TRY(launch_gemm(g, s));
-    TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
+    if (gemm_tc_eligible(g.N, g.K, rows) && g.splits == 1 && m->F % 64 == 0) {
+      g.swiglu_u = m->u;   // the GEMM's epilogue forms silu(gate) * up
+      TL_TRY(launch_gemm(g, s));
+    } else {
+      TL_TRY(launch_gemm(g, s));
+      TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
+    }
     g = gemm_args(m, b, 3, m->u, rows);
     TL_TRY(launch_gemm(g, s));
   }

@@ -400,6 +400,13 @@ tl_status launch_gemv(const GemmArgs& a, cudaStream_t s) {
 }
 
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.swiglu_u) {
+    if (!gemm_tc_eligible(a.N, a.K, a.T) || a.splits != 1 || a.N != 2 * a.n_split ||
+        a.n_split % 64 != 0 || a.x_part || a.h)
+      return set_error(TL_ERR_UNSUPPORTED,
+                       "the fused SwiGLU epilogue needs the one-split tensor-core GEMM");
+    return launch_gemm_tc(a, s);
+  }
   if (gemv_eligible(a.N, a.K, a.T)) return launch_gemv(a, s);
   if (a.x_part || a.h)
     return set_error(TL_ERR_UNSUPPORTED, "fused staging / residual needs the decode GEMV");

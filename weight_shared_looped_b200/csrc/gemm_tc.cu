@@ -44,9 +44,8 @@ constexpr size_t kMinSmem = 120 * 1024;   // also keeps it to one CTA per SM
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a bounded wait gives up after 2 s
 template <int BN> struct TcCfg {
   static constexpr int W_STAGES = 2 * BATCH;                  // packed-weight ring (k blocks)
-  static constexpr int X_BATCHES = BN >= 128 ? 2 : 3;         // activation ring (batches)
+  static constexpr int X_STAGES = BN >= 128 ? 8 : 12;         // activation ring (k blocks)
   static constexpr int A_BATCHES = (TMEM_COLS - BN) / (A_COLS * BATCH);   // TMEM A ring (batches)
-  static constexpr int D_BATCHES = A_BATCHES > X_BATCHES ? A_BATCHES : X_BATCHES;
 };
 
 __device__ __forceinline__ uint64_t globaltimer_ns() {
@@ -119,12 +118,23 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   return d;
 }
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
+// The four K=16 MMAs of one 64-wide k block (A columns +8, B descriptor +2
+// (32 bytes) per step), then a commit that frees the block's activation slot.
+__device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, bool accumulate, uint64_t* bar) {
   asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
+      "{\n .reg .pred p, q;\n .reg .b64 b1, b2, b3;\n .reg .b32 a1, a2, a3;\n"
+      " setp.ne.b32 p, %4, 0;\n setp.eq.b32 q, %4, %4;\n"
+      " add.s64 b1, %2, 2;\n add.s64 b2, %2, 4;\n add.s64 b3, %2, 6;\n"
+      " add.u32 a1, %1, 8;\n add.u32 a2, %1, 16;\n add.u32 a3, %1, 24;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, q;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, q;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, q;\n"
+      " tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n}\n" ::"r"(
+          d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(smem_u32(bar))
+      : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -153,6 +163,7 @@ struct TcArgs {
   const __half* s1;
   float* part;
   int* status;
+  __half* swiglu_u;          // fused SwiGLU epilogue: fp16 [T][n_split] (N = 2 * n_split)
 };
 
 template <int BN>
@@ -160,16 +171,16 @@ __global__ void __launch_bounds__(THREADS, 1)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x,
                       const __grid_constant__ CUtensorMap map_w0,
                       const __grid_constant__ CUtensorMap map_w1, TcArgs a) {
-  constexpr int WS = TcCfg<BN>::W_STAGES, XB = TcCfg<BN>::X_BATCHES;
-  constexpr int AB = TcCfg<BN>::A_BATCHES, DB = TcCfg<BN>::D_BATCHES;
+  constexpr int WS = TcCfg<BN>::W_STAGES, XS = TcCfg<BN>::X_STAGES;
+  constexpr int AB = TcCfg<BN>::A_BATCHES;
   constexpr uint32_t X_BYTES = BN * 128;          // BN rows x 64 fp16
   constexpr uint32_t W_BYTES = BM * 32;           // 128 rows x 8 words
   static_assert(BN + AB * BATCH * A_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(AB >= 2 && XB >= 2 && WS % DQ_GROUPS == 0, "ring depths");
+  static_assert(AB >= 2 && XS >= 2 * BATCH && WS % DQ_GROUPS == 0, "ring depths");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-  uint8_t* sX = smem;                                        // XB*BATCH x X_BYTES
-  uint8_t* sW = sX + XB * BATCH * X_BYTES;                   // WS x W_BYTES
+  uint8_t* sX = smem;                                        // XS x X_BYTES
+  uint8_t* sW = sX + XS * X_BYTES;                           // WS x W_BYTES
   __half* sScale = reinterpret_cast<__half*>(sW + WS * W_BYTES);   // [BM][groups]
   const int nkb_total = a.K / BK;
   const int kb_begin = (int)(((long)blockIdx.z * nkb_total) / a.splits);
@@ -181,10 +192,11 @@ __global__ void __launch_bounds__(THREADS, 1)
   bars = reinterpret_cast<uint64_t*>(((uintptr_t)bars + 7) & ~(uintptr_t)7);
   uint64_t* wfull = bars;               // packed weights of a k block landed
   uint64_t* wempty = wfull + WS;        // dequantisation done reading them
-  uint64_t* xfull = wempty + WS;        // activations of a batch landed
-  uint64_t* afull = xfull + XB;         // A tiles of a batch in TMEM (and its activations seen)
-  uint64_t* done = afull + AB;          // MMAs of a batch complete: frees its X and A slots
-  uint64_t* accb = done + DB;           // accumulator complete
+  uint64_t* xfull = wempty + WS;        // activations of a k block landed
+  uint64_t* xempty = xfull + XS;        // MMAs of a k block complete: frees its X slot
+  uint64_t* afull = xempty + XS;        // A tiles of a batch in TMEM (and its activations seen)
+  uint64_t* done = afull + AB;          // MMAs of a batch complete: frees its A slots
+  uint64_t* accb = done + AB;           // accumulator complete
   uint64_t* epib = accb + 1;            // epilogue finished reading TMEM
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epib + 1);
   int* abort_flag = reinterpret_cast<int*>(tmem_slot + 1);
@@ -192,9 +204,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * BM;
   const int t0 = blockIdx.y * BN;
-  const bool second = m0 >= a.n_split;
+  // fused SwiGLU: tile rows [0, 64) are gate rows wrow0.., rows [64, 128) the
+  // same rows of up (two 64-row weight loads per k block)
+  const bool sw = a.swiglu_u != nullptr;
+  const bool second = !sw && m0 >= a.n_split;
   const CUtensorMap* map_w = second ? &map_w1 : &map_w0;
-  const int wrow0 = second ? m0 - a.n_split : m0;
+  const int wrow0 = sw ? blockIdx.x * (BM / 2) : second ? m0 - a.n_split : m0;
   const __half* scales = second ? a.s1 : a.s0;
 
   if (threadIdx.x == 0) {
@@ -202,15 +217,21 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&wfull[s], 1);
       mbar_init(&wempty[s], 4);
     }
-    for (int s = 0; s < XB; ++s) mbar_init(&xfull[s], 1);
-    for (int s = 0; s < AB; ++s) mbar_init(&afull[s], DQ_WARPS);
-    for (int s = 0; s < DB; ++s) mbar_init(&done[s], 1);
+    for (int s = 0; s < XS; ++s) {
+      mbar_init(&xfull[s], 1);
+      mbar_init(&xempty[s], 1);
+    }
+    for (int s = 0; s < AB; ++s) {
+      mbar_init(&afull[s], DQ_WARPS);
+      mbar_init(&done[s], 1);
+    }
     mbar_init(accb, 1);
     mbar_init(epib, DQ_WARPS);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(map_w) : "memory");
+    if (sw) asm volatile("prefetch.tensormap [%0];" ::"l"(&map_w1) : "memory");
   }
   __syncwarp();
   if (warp == MMA_WARP) {
@@ -239,11 +260,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (*(volatile int*)abort_flag) break;
         mbar_expect_tx(&wfull[s], W_BYTES);
-        tma_load_2d(sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
+        if (sw) {
+          tma_load_2d(sW + s * W_BYTES, &map_w0, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
+          tma_load_2d(sW + s * W_BYTES + (BM / 2) * 32, &map_w1, (kb_begin + i) * (BK / 8), wrow0,
+                      &wfull[s]);
+        } else {
+          tma_load_2d(sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
+        }
         issued = i + 1;
       }
       if (*(volatile int*)abort_flag)
-        for (int i = 0; i < issued; ++i) mbar_wait(&wfull[i % WS], (i / WS) & 1);
+        for (int i = issued > WS ? issued - WS : 0; i < issued; ++i)   // the ones still in flight
+          mbar_wait(&wfull[i % WS], (i / WS) & 1);
     }
     __syncwarp();
     pdl_enter();
@@ -252,31 +280,36 @@ __global__ void __launch_bounds__(THREADS, 1)
     pdl_enter();   // the activations come from the previous kernel
     if (lane == 0) {
       int issued = 0;
-      for (int b = 0; b < nbatch; ++b) {
-        if (b >= XB && !mbar_wait(&done[(b - XB) % DB], ((b - XB) / DB) & 1)) {
+      for (int i = 0; i < nkb; ++i) {
+        const int s = i % XS;
+        if (i >= XS && !mbar_wait(&xempty[s], ((i / XS) - 1) & 1)) {
           atomicExch(abort_flag, 1);
           break;
         }
         if (*(volatile int*)abort_flag) break;
-        const int cnt = min(BATCH, nkb - b * BATCH);
-        uint64_t* bar = &xfull[b % XB];
-        mbar_expect_tx(bar, cnt * X_BYTES);
-        for (int j = 0; j < cnt; ++j)
-          tma_load_2d(sX + ((b % XB) * BATCH + j) * X_BYTES, &map_x,
-                      (kb_begin + b * BATCH + j) * BK, t0, bar);
-        issued = b + 1;
+        mbar_expect_tx(&xfull[s], X_BYTES);
+        tma_load_2d(sX + s * X_BYTES, &map_x, (kb_begin + i) * BK, t0, &xfull[s]);
+        issued = i + 1;
       }
       if (*(volatile int*)abort_flag)
-        for (int b = 0; b < issued; ++b) mbar_wait(&xfull[b % XB], (b / XB) & 1);
+        for (int i = issued > XS ? issued - XS : 0; i < issued; ++i)   // the ones still in flight
+          mbar_wait(&xfull[i % XS], (i / XS) & 1);
     }
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ---------------------------------------------------------------- MMA
     // per batch: one wait (A tiles written and activations seen), one fence,
-    // up to 16 MMAs, one commit
+    // up to 16 MMAs, one commit per k block (frees its activation slot) and
+    // one per batch (frees its A slots)
     pdl_enter();
     if (lane == 0) {
       const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      // loop-invariant operands: the X ring's first descriptor (each slot adds
+      // X_BYTES >> 4 to the start-address field, which stays below 2^14) and
+      // the accumulator / A ring addresses in TMEM
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(sX));
+      const uint32_t d_tm = tmem_base + acc_col;
+      int xs = 0;   // X slot of k block i
       for (int b = 0; b < nbatch; ++b) {
         if (!mbar_wait(&afull[b % AB], (b / AB) & 1) || *(volatile int*)abort_flag) {
           atomicExch(abort_flag, 1);
@@ -284,16 +317,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const int cnt = min(BATCH, nkb - b * BATCH);
+        const uint32_t a_b = tmem_base + a_col0 + (b % AB) * BATCH * A_COLS;
         for (int j = 0; j < cnt; ++j) {
-          const int i = b * BATCH + j;
-          const uint64_t bdesc = smem_desc_sw128(smem_u32(sX + ((b % XB) * BATCH + j) * X_BYTES));
-          const uint32_t a_tm = tmem_base + a_col0 + ((b % AB) * BATCH + j) * A_COLS;
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k)
-            mma_ts(tmem_base + acc_col, a_tm + k * 8, bdesc + (uint64_t)(2 * k), idesc,
-                   (i > 0 || k > 0) ? 1u : 0u);
+          mma_kblock(d_tm, a_b + j * A_COLS, xdesc0 + (uint64_t)(xs * (X_BYTES >> 4)), idesc,
+                     (b | j) != 0, &xempty[xs]);
+          xs = xs + 1 == XS ? 0 : xs + 1;
         }
-        mma_commit(&done[b % DB]);
+        mma_commit(&done[b % AB]);
       }
       mma_commit(accb);   // arrives once all issued MMAs are complete
     }
@@ -311,15 +341,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int g0 = g_first;
       for (int i = threadIdx.x; i < BM * groups; i += 32 * DQ_WARPS) {
         const int rr = i / groups, gg = i % groups;
-        sScale[rr * groups + gg] =
-            g0 + gg < gpr ? scales[(size_t)(wrow0 + rr) * gpr + g0 + gg] : __float2half_rn(0.f);
+        const __half* sp = !sw ? scales + (size_t)(wrow0 + rr) * gpr
+                           : rr < BM / 2 ? a.s0 + (size_t)(wrow0 + rr) * gpr
+                                         : a.s1 + (size_t)(wrow0 + rr - BM / 2) * gpr;
+        sScale[rr * groups + gg] = g0 + gg < gpr ? sp[g0 + gg] : __float2half_rn(0.f);
       }
       asm volatile("bar.sync 1, %0;" ::"n"(32 * DQ_WARPS) : "memory");
     }
     for (int b = 0; b < nbatch; ++b) {
       const int i = b * BATCH + grp;
       // the TMEM slot of this batch is free once batch b - AB is done
-      if (b >= AB && !mbar_wait(&done[(b - AB) % DB], ((b - AB) / DB) & 1)) {
+      if (b >= AB && !mbar_wait(&done[(b - AB) % AB], ((b - AB) / AB) & 1)) {
         atomicExch(abort_flag, 1);
         break;
       }
@@ -359,12 +391,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             "r"(v[29]), "r"(v[30]), "r"(v[31])
             : "memory");
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-      }
-      // the batch's activations must have landed before the MMA thread (which
-      // waits only on afull) reads them
-      if (!mbar_wait(&xfull[b % XB], (b / XB) & 1)) {
-        atomicExch(abort_flag, 1);
-        break;
+        // this k block's activations must have landed before the MMA thread
+        // (which waits only on afull) reads them
+        if (!mbar_wait(&xfull[i % XS], (i / XS) & 1)) {
+          atomicExch(abort_flag, 1);
+          break;
+        }
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
@@ -372,10 +404,66 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     pdl_enter();
     // epilogue: accumulator rows = weight rows, columns = tokens
-    const bool ok = mbar_wait(accb, 0) && !*(volatile int*)abort_flag;
+    bool ok = mbar_wait(accb, 0) && !*(volatile int*)abort_flag;
     if (!ok) atomicExch(abort_flag, 1);
+    {
+      // agree on ok across all dequantisation warps (the SwiGLU epilogue
+      // below synchronises groups of four warps)
+      uint32_t all;
+      asm volatile(
+          "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.red.and.pred q, 1, %2, p;\n"
+          " selp.u32 %0, 1, 0, q;\n}\n"
+          : "=r"(all)
+          : "r"(ok ? 1u : 0u), "n"(32 * DQ_WARPS)
+          : "memory");
+      ok = all != 0;
+    }
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    if (ok) {
+    if (ok && sw) {
+      // tile rows [0, 64) hold gate, [64, 128) up for the same 64 features;
+      // quadrants 2 and 3 pass up through shared memory (the activation ring
+      // is idle once the accumulator is complete) to quadrants 0 and 1
+      float* xch = reinterpret_cast<float*>(sX) + grp * 32 * (BM / 2);   // [32 tokens][64]
+      const int j = r & (BM / 2 - 1);
+      const int F = a.n_split;
+#pragma unroll 1
+      for (int cc = grp; cc < BN / 32; cc += DQ_GROUPS) {
+        if (t0 + cc * 32 >= a.T) break;   // uniform across the group
+        uint32_t u[32];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, "
+            "%10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, "
+            "%27, %28, %29, %30, %31}, [%32];"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+              "=r"(u[7]), "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]),
+              "=r"(u[13]), "=r"(u[14]), "=r"(u[15]), "=r"(u[16]), "=r"(u[17]), "=r"(u[18]),
+              "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]), "=r"(u[24]),
+              "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]),
+              "=r"(u[31])
+            : "r"(tmem_base + lane_addr + acc_col + cc * 32));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+        if (quad >= 2) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) xch[e * (BM / 2) + j] = __uint_as_float(u[e]);
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "n"(128) : "memory");
+        if (quad < 2) {
+          const int tn = min(32, a.T - (t0 + cc * 32));
+          __half* o = a.swiglu_u + (size_t)(t0 + cc * 32) * F + wrow0 + j;
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (e < tn) {
+              // the same arithmetic as the separate SwiGLU kernel on one split
+              const float gs = 0.f + __uint_as_float(u[e]);
+              const float us = 0.f + xch[e * (BM / 2) + j];
+              const float silu = gs / (1.0f + __expf(-gs));
+              o[(size_t)e * F] = __float2half_rn(silu * us);
+            }
+          }
+        }
+        asm volatile("bar.sync %0, %1;" ::"r"(2 + grp), "n"(128) : "memory");
+      }
+    } else if (ok) {
       float* out = a.part + (size_t)blockIdx.z * a.T * a.N + (size_t)(m0 + r);
       // this group's 32-token chunks: cc = grp, grp + DQ_GROUPS, ...
 #pragma unroll 1
@@ -471,10 +559,10 @@ int tc_tile_n(int T) { return T <= 64 ? 64 : 128; }
 
 template <int BN>
 size_t tc_smem_bytes(int max_groups) {
-  constexpr int WS = TcCfg<BN>::W_STAGES, XB = TcCfg<BN>::X_BATCHES;
-  constexpr int AB = TcCfg<BN>::A_BATCHES, DB = TcCfg<BN>::D_BATCHES;
-  size_t b = 1024 + (size_t)XB * BATCH * BN * 128 + (size_t)WS * BM * 32 +
-             (size_t)BM * max_groups * 2 + 16 + (2 * WS + XB + AB + DB + 2) * 8 + 16;
+  constexpr int WS = TcCfg<BN>::W_STAGES, XS = TcCfg<BN>::X_STAGES;
+  constexpr int AB = TcCfg<BN>::A_BATCHES;
+  size_t b = 1024 + (size_t)XS * BN * 128 + (size_t)WS * BM * 32 +
+             (size_t)BM * max_groups * 2 + 16 + (2 * WS + 2 * XS + 2 * AB + 2) * 8 + 16;
   return b < kMinSmem ? kMinSmem : b;
 }
 
@@ -484,11 +572,12 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   TL_TRY(encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.x, g.K, g.T, (uint64_t)g.K * 2, BK, BN,
                    CU_TENSOR_MAP_SWIZZLE_128B));
   const int n1 = g.n_split, n2 = g.N - g.n_split;
+  const int box_rows = g.swiglu_u ? BM / 2 : BM;   // fused SwiGLU: 64 gate + 64 up rows
   TL_TRY(encode_2d(&mw0, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w0, g.K / 8, n1, (uint64_t)g.K / 8 * 4,
-                   BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE));
+                   BK / 8, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE));
   if (n2 > 0) {
     TL_TRY(encode_2d(&mw1, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w1, g.K / 8, n2,
-                     (uint64_t)g.K / 8 * 4, BK / 8, BM, CU_TENSOR_MAP_SWIZZLE_NONE));
+                     (uint64_t)g.K / 8 * 4, BK / 8, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE));
   } else {
     mw1 = mw0;
   }
@@ -509,6 +598,7 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.s1 = g.s1;
   a.part = g.part;
   a.status = g.status;
+  a.swiglu_u = g.swiglu_u;
   const size_t smem = tc_smem_bytes<BN>(a.max_groups);
   if (smem > 232448)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs %zu bytes of shared memory", smem);

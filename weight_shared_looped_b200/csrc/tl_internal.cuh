@@ -89,6 +89,11 @@ struct GemmArgs {
   // a later kernel
   float* h;
   int* tickets;
+  // tensor-core kernel with one split only, for [gate; up] weights (n_split =
+  // F, N = 2F): when swiglu_u is set, each CTA takes 64 gate rows and the same
+  // 64 up rows and writes swiglu_u[t][f] = fp16(silu(gate) * up) (fp16 [T][F])
+  // instead of partial sums
+  __half* swiglu_u;
 };
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
 // kernel for T >= 64, the mma.sync register-dequant kernel below that.
