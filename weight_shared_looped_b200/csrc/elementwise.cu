@@ -47,74 +47,129 @@ __global__ void embed_kernel(EmbedArgs a) {
 }
 
 // ------------------------------------------------------------------ residual + RMSNorm
-constexpr int NORM_THREADS = 256;
+// A row of d columns is split over a thread-block cluster of C CTAs (C = d/512
+// capped at 8; consecutive blockIdx.x form a cluster), each CTA d/C columns,
+// each thread VPT float4 vectors (VPT = 1, or 2 for d = 8192).  The split-K
+// partial sums are loaded eight splits at a time (independent loads in
+// flight) and added in split order.  The sum of squares is reduced per thread,
+// per warp (xor tree), over the CTA's warps and over the cluster's CTAs (read
+// through distributed shared memory) in a fixed order that depends only on d.
+constexpr int NORM_MAX_THREADS = 128;
 
-// PER = d / 256 elements per thread.  Partial sums are loaded four splits at a
-// time (independent loads in flight) and added in split order.
-template <int PER>
-__global__ void __launch_bounds__(NORM_THREADS) residual_norm_kernel(NormArgs a) {
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+
+__device__ __forceinline__ float cluster_read_f32(const float* local, uint32_t rank) {
+  uint32_t addr = (uint32_t)__cvta_generic_to_shared(local), remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void add4(float4& a, const float4 b) {
+  a.x += b.x;
+  a.y += b.y;
+  a.z += b.z;
+  a.w += b.w;
+}
+
+template <int VPT>
+__global__ void __launch_bounds__(NORM_MAX_THREADS) residual_norm_kernel(NormArgs a, int C) {
   pdl_enter();
-  __shared__ float red[NORM_THREADS / 32];
-  const int row = blockIdx.x;
+  __shared__ float red[NORM_MAX_THREADS / 32];
+  __shared__ float cta_sum;
+  const int row = blockIdx.x / C;
+  const int crank = blockIdx.x % C;
+  const int cols = a.d / C;
+  const int nthr = blockDim.x;
+  const int nw = nthr / 32;
   float* h = a.h + (size_t)row * a.d;
   const int out_row = a.out_row ? a.out_row[row] : row;
-  float v[PER];
-  const bool add = row < a.n_add && a.S > 0;
+  int col[VPT];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) v[e] = h[threadIdx.x + e * NORM_THREADS];
-  if (add) {
+  for (int e = 0; e < VPT; ++e) col[e] = crank * cols + (e * nthr + threadIdx.x) * 4;
+  float4 v[VPT];
+#pragma unroll
+  for (int e = 0; e < VPT; ++e) v[e] = *reinterpret_cast<const float4*>(h + col[e]);
+  if (row < a.n_add && a.S > 0) {
     const size_t sstride = (size_t)a.part_rows * a.d;
-    const float* p0 = a.part + (size_t)row * a.d + threadIdx.x;
-    int sp = 0;
-    for (; sp + 4 <= a.S; sp += 4) {
-      float t[4][PER];
+    const float* p0 = a.part + (size_t)row * a.d;
+    for (int sp = 0; sp < a.S; sp += 8) {
+      const int n = min(8, a.S - sp);
+      float4 t[8][VPT];
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+      for (int q = 0; q < 8; ++q)
 #pragma unroll
-        for (int e = 0; e < PER; ++e) t[q][e] = p0[(sp + q) * sstride + e * NORM_THREADS];
+        for (int e = 0; e < VPT; ++e)
+          if (q < n) t[q][e] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + col[e]));
 #pragma unroll
-      for (int e = 0; e < PER; ++e) v[e] = (((v[e] + t[0][e]) + t[1][e]) + t[2][e]) + t[3][e];
+      for (int q = 0; q < 8; ++q)
+#pragma unroll
+        for (int e = 0; e < VPT; ++e)
+          if (q < n) add4(v[e], t[q][e]);
     }
-    for (; sp < a.S; ++sp)
 #pragma unroll
-      for (int e = 0; e < PER; ++e) v[e] += p0[sp * sstride + e * NORM_THREADS];
-#pragma unroll
-    for (int e = 0; e < PER; ++e) h[threadIdx.x + e * NORM_THREADS] = v[e];
+    for (int e = 0; e < VPT; ++e) *reinterpret_cast<float4*>(h + col[e]) = v[e];
   }
   if (a.trace) {
     float* tr = a.trace + (size_t)out_row * a.d;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) tr[threadIdx.x + e * NORM_THREADS] = v[e];
+    for (int e = 0; e < VPT; ++e) *reinterpret_cast<float4*>(tr + col[e]) = v[e];
   }
+  // row-uniform, hence uniform across the cluster: every CTA reaches the
+  // cluster barriers below
   const bool want_x = row < a.n_next;
   const bool want_y = row >= a.fin_lo && row < a.fin_hi;
-  if (!want_x && !want_y) return;
   float ss = 0.0f;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) ss = fmaf(v[e], v[e], ss);
+  for (int e = 0; e < VPT; ++e) {
+    ss = fmaf(v[e].x, v[e].x, ss);
+    ss = fmaf(v[e].y, v[e].y, ss);
+    ss = fmaf(v[e].z, v[e].z, ss);
+    ss = fmaf(v[e].w, v[e].w, ss);
+  }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
+  if (threadIdx.x == 0) {
+    float c = 0.0f;
+    for (int w = 0; w < nw; ++w) c += red[w];
+    cta_sum = c;
+  }
+  cluster_sync_all();   // every CTA's cta_sum is written
   float tot = 0.0f;
-#pragma unroll
-  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += red[w];
+  for (int q = 0; q < C; ++q) tot += cluster_read_f32(&cta_sum, (uint32_t)q);
+  cluster_sync_all();   // no CTA leaves while another still reads its cta_sum
+  if (!want_x && !want_y) return;
   const float r = rsqrtf(tot / (float)a.d + a.eps);
   if (want_x) {
     __half* x = a.x + (size_t)row * a.d;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const int i = threadIdx.x + e * NORM_THREADS;
-      x[i] = __float2half_rn(v[e] * r * a.gamma_next[i]);
+    for (int e = 0; e < VPT; ++e) {
+      const float4 g = *reinterpret_cast<const float4*>(a.gamma_next + col[e]);
+      const __half2 lo = __halves2half2(__float2half_rn(v[e].x * r * g.x), __float2half_rn(v[e].y * r * g.y));
+      const __half2 hi = __halves2half2(__float2half_rn(v[e].z * r * g.z), __float2half_rn(v[e].w * r * g.w));
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(x + col[e]) = pk;
     }
   } else {
     float* y = a.y + (size_t)out_row * a.d;
     bool bad = false;
 #pragma unroll
-    for (int e = 0; e < PER; ++e) {
-      const int i = threadIdx.x + e * NORM_THREADS;
-      const float o = v[e] * r * a.gamma_final[i];
-      bad |= !isfinite(o);
-      y[i] = o;
+    for (int e = 0; e < VPT; ++e) {
+      const float4 g = *reinterpret_cast<const float4*>(a.gamma_final + col[e]);
+      float4 o;
+      o.x = v[e].x * r * g.x;
+      o.y = v[e].y * r * g.y;
+      o.z = v[e].z * r * g.z;
+      o.w = v[e].w * r * g.w;
+      bad |= !isfinite(o.x) || !isfinite(o.y) || !isfinite(o.z) || !isfinite(o.w);
+      *reinterpret_cast<float4*>(y + col[e]) = o;
     }
     if (bad) set_status(a.status, TL_ERR_NUMERIC);
   }
@@ -276,15 +331,18 @@ tl_status launch_embed(const EmbedArgs& a, cudaStream_t s) {
 
 tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
-  switch (a.d / NORM_THREADS) {
-    case 1: TL_LAUNCH_PDL(residual_norm_kernel<1>, a.rows, NORM_THREADS, 0, s, a); break;
-    case 2: TL_LAUNCH_PDL(residual_norm_kernel<2>, a.rows, NORM_THREADS, 0, s, a); break;
-    case 4: TL_LAUNCH_PDL(residual_norm_kernel<4>, a.rows, NORM_THREADS, 0, s, a); break;
-    case 8: TL_LAUNCH_PDL(residual_norm_kernel<8>, a.rows, NORM_THREADS, 0, s, a); break;
-    case 16: TL_LAUNCH_PDL(residual_norm_kernel<16>, a.rows, NORM_THREADS, 0, s, a); break;
-    case 32: TL_LAUNCH_PDL(residual_norm_kernel<32>, a.rows, NORM_THREADS, 0, s, a); break;
-    default: return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs d/256 in {1,2,4,...,32}", a.d);
-  }
+  // d = 256 * 2^k: C = d / 512 CTAs per row (at least 1, at most 8), d / C
+  // columns per CTA, 4 * VPT per thread
+  if (a.d < 256 || a.d > 8192 || (a.d & (a.d - 1)) != 0)
+    return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs a power of two in [256, 8192]", a.d);
+  const int C = a.d <= 512 ? 1 : a.d / 512 > 8 ? 8 : a.d / 512;
+  const int cols = a.d / C;
+  const int vpt = cols > 512 ? 2 : 1;
+  const int threads = cols / (4 * vpt);
+  cudaError_t e = vpt == 1 ? launch_pdl_cluster(residual_norm_kernel<1>, dim3(a.rows * C), dim3(threads), 0, s, (unsigned)C, a, C)
+                           : launch_pdl_cluster(residual_norm_kernel<2>, dim3(a.rows * C), dim3(threads), 0, s, (unsigned)C, a, C);
+  if (e != cudaSuccess)
+    return set_error(TL_ERR_CUDA, "launch of residual_norm_kernel failed: %s", cudaGetErrorString(e));
   TL_LAUNCH_CHECK();
   return ok();
 }

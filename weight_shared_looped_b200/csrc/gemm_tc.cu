@@ -66,12 +66,6 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
 // Bounded wait for the phase with the given parity to complete: false after
 // limit_ns of global time.
 __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
@@ -98,12 +92,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   }
 }
 
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
+// The producer and MMA warps run their loops with all 32 lanes converged and
+// issue each TMA copy, MMA and commit from one lane chosen by elect.sync: a
+// lone active lane issues far more slowly while the dequantisation warps on
+// the same SM sub-partition keep its issue slots busy.
+__device__ __forceinline__ void tma_issue_elect(uint64_t* bar, uint32_t bytes, void* dst,
+                                                const CUtensorMap* map, int x, int y) {
   asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3, "
+      "{%4, %5}], [%0];\n}\n" ::"r"(smem_u32(bar)),
+      "r"(bytes), "r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Two tiles of one stage (64 gate rows and 64 up rows) on one barrier.
+__device__ __forceinline__ void tma_issue2_elect(uint64_t* bar, uint32_t bytes, void* dst0,
+                                                 const CUtensorMap* map0, void* dst1,
+                                                 const CUtensorMap* map1, int x, int y) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3, "
+      "{%6, %7}], [%0];\n"
+      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5, "
+      "{%6, %7}], [%0];\n}\n" ::"r"(smem_u32(bar)),
+      "r"(bytes), "r"(smem_u32(dst0)), "l"(map0), "r"(smem_u32(dst1)), "l"(map1), "r"(x), "r"(y)
       : "memory");
 }
 
@@ -119,29 +134,43 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
 }
 
 // The four K=16 MMAs of one 64-wide k block (A columns +8, B descriptor +2
-// (32 bytes) per step), then a commit that frees the block's activation slot.
+// (32 bytes) per step), then a commit that frees the block's activation slot;
+// called by the whole warp, issued by the lane elect.sync picks (the same lane
+// every time, so its commits track its own MMAs).
 __device__ __forceinline__ void mma_kblock(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                            uint32_t idesc, bool accumulate, uint64_t* bar) {
   asm volatile(
-      "{\n .reg .pred p, q;\n .reg .b64 b1, b2, b3;\n .reg .b32 a1, a2, a3;\n"
-      " setp.ne.b32 p, %4, 0;\n setp.eq.b32 q, %4, %4;\n"
+      "{\n .reg .pred p, e;\n .reg .b64 b1, b2, b3;\n .reg .b32 a1, a2, a3;\n"
+      " setp.ne.b32 p, %4, 0;\n"
       " add.s64 b1, %2, 2;\n add.s64 b2, %2, 4;\n add.s64 b3, %2, 6;\n"
       " add.u32 a1, %1, 8;\n add.u32 a2, %1, 16;\n add.u32 a3, %1, 24;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, q;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, q;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, q;\n"
-      " tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n}\n" ::"r"(
+      " elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, 1;\n"
+      " @e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, 1;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n}\n" ::"r"(
           d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(smem_u32(bar))
       : "memory");
 }
 
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n}\n" ::"r"(
           smem_u32(bar))
       : "memory");
+}
+
+// Bounded wait (when needed) by lane 0 with the outcome (and the CTA's abort flag) broadcast
+// to the warp, so the warp stays converged.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const int* abort_flag,
+                                          bool needed) {
+  bool ok = true;
+  if ((threadIdx.x & 31) == 0)
+    ok = (!needed || mbar_wait(bar, parity)) && !*(volatile const int*)abort_flag;
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
 __device__ __forceinline__ uint32_t dequant_code_pair(uint32_t w, uint32_t sel) {
@@ -250,51 +279,41 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == WTMA_WARP) {
     // ---------------------------------------------------------------- weight TMA
     // weights are constants of the model: no need to wait for the previous kernel
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % WS;
-        if (i >= WS && !mbar_wait(&wempty[s], ((i / WS) - 1) & 1)) {
-          atomicExch(abort_flag, 1);
-          break;
-        }
-        if (*(volatile int*)abort_flag) break;
-        mbar_expect_tx(&wfull[s], W_BYTES);
-        if (sw) {
-          tma_load_2d(sW + s * W_BYTES, &map_w0, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
-          tma_load_2d(sW + s * W_BYTES + (BM / 2) * 32, &map_w1, (kb_begin + i) * (BK / 8), wrow0,
-                      &wfull[s]);
-        } else {
-          tma_load_2d(sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0, &wfull[s]);
-        }
-        issued = i + 1;
+    int issued = 0;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % WS;
+      if (!warp_wait(&wempty[s], ((i / WS) - 1) & 1, abort_flag, i >= WS)) {
+        if (lane == 0) atomicExch(abort_flag, 1);
+        break;
       }
-      if (*(volatile int*)abort_flag)
-        for (int i = issued > WS ? issued - WS : 0; i < issued; ++i)   // the ones still in flight
-          mbar_wait(&wfull[i % WS], (i / WS) & 1);
+      if (sw)
+        tma_issue2_elect(&wfull[s], W_BYTES, sW + s * W_BYTES, &map_w0,
+                         sW + s * W_BYTES + (BM / 2) * 32, &map_w1, (kb_begin + i) * (BK / 8), wrow0);
+      else
+        tma_issue_elect(&wfull[s], W_BYTES, sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0);
+      issued = i + 1;
     }
+    if (lane == 0 && *(volatile int*)abort_flag)
+      for (int i = issued > WS ? issued - WS : 0; i < issued; ++i)   // the ones still in flight
+        mbar_wait(&wfull[i % WS], (i / WS) & 1);
     __syncwarp();
     pdl_enter();
   } else if (warp == XTMA_WARP) {
     // ---------------------------------------------------------------- activation TMA
     pdl_enter();   // the activations come from the previous kernel
-    if (lane == 0) {
-      int issued = 0;
-      for (int i = 0; i < nkb; ++i) {
-        const int s = i % XS;
-        if (i >= XS && !mbar_wait(&xempty[s], ((i / XS) - 1) & 1)) {
-          atomicExch(abort_flag, 1);
-          break;
-        }
-        if (*(volatile int*)abort_flag) break;
-        mbar_expect_tx(&xfull[s], X_BYTES);
-        tma_load_2d(sX + s * X_BYTES, &map_x, (kb_begin + i) * BK, t0, &xfull[s]);
-        issued = i + 1;
+    int issued = 0;
+    for (int i = 0; i < nkb; ++i) {
+      const int s = i % XS;
+      if (!warp_wait(&xempty[s], ((i / XS) - 1) & 1, abort_flag, i >= XS)) {
+        if (lane == 0) atomicExch(abort_flag, 1);
+        break;
       }
-      if (*(volatile int*)abort_flag)
-        for (int i = issued > XS ? issued - XS : 0; i < issued; ++i)   // the ones still in flight
-          mbar_wait(&xfull[i % XS], (i / XS) & 1);
+      tma_issue_elect(&xfull[s], X_BYTES, sX + s * X_BYTES, &map_x, (kb_begin + i) * BK, t0);
+      issued = i + 1;
     }
+    if (lane == 0 && *(volatile int*)abort_flag)
+      for (int i = issued > XS ? issued - XS : 0; i < issued; ++i)   // the ones still in flight
+        mbar_wait(&xfull[i % XS], (i / XS) & 1);
     __syncwarp();
   } else if (warp == MMA_WARP) {
     // ---------------------------------------------------------------- MMA
@@ -302,31 +321,29 @@ __global__ void __launch_bounds__(THREADS, 1)
     // up to 16 MMAs, one commit per k block (frees its activation slot) and
     // one per batch (frees its A slots)
     pdl_enter();
-    if (lane == 0) {
-      const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
-      // loop-invariant operands: the X ring's first descriptor (each slot adds
-      // X_BYTES >> 4 to the start-address field, which stays below 2^14) and
-      // the accumulator / A ring addresses in TMEM
-      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(sX));
-      const uint32_t d_tm = tmem_base + acc_col;
-      int xs = 0;   // X slot of k block i
-      for (int b = 0; b < nbatch; ++b) {
-        if (!mbar_wait(&afull[b % AB], (b / AB) & 1) || *(volatile int*)abort_flag) {
-          atomicExch(abort_flag, 1);
-          break;
-        }
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const int cnt = min(BATCH, nkb - b * BATCH);
-        const uint32_t a_b = tmem_base + a_col0 + (b % AB) * BATCH * A_COLS;
-        for (int j = 0; j < cnt; ++j) {
-          mma_kblock(d_tm, a_b + j * A_COLS, xdesc0 + (uint64_t)(xs * (X_BYTES >> 4)), idesc,
-                     (b | j) != 0, &xempty[xs]);
-          xs = xs + 1 == XS ? 0 : xs + 1;
-        }
-        mma_commit(&done[b % AB]);
+    const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+    // loop-invariant operands: the X ring's first descriptor (each slot adds
+    // X_BYTES >> 4 to the start-address field, which stays below 2^14) and
+    // the accumulator / A ring addresses in TMEM
+    const uint64_t xdesc0 = smem_desc_sw128(smem_u32(sX));
+    const uint32_t d_tm = tmem_base + acc_col;
+    int xs = 0;   // X slot of k block i
+    for (int b = 0; b < nbatch; ++b) {
+      if (!warp_wait(&afull[b % AB], (b / AB) & 1, abort_flag, true)) {
+        if (lane == 0) atomicExch(abort_flag, 1);
+        break;
       }
-      mma_commit(accb);   // arrives once all issued MMAs are complete
+      asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+      const int cnt = min(BATCH, nkb - b * BATCH);
+      const uint32_t a_b = tmem_base + a_col0 + (b % AB) * BATCH * A_COLS;
+      for (int j = 0; j < cnt; ++j) {
+        mma_kblock(d_tm, a_b + j * A_COLS, xdesc0 + (uint64_t)(xs * (X_BYTES >> 4)), idesc,
+                   (b | j) != 0, &xempty[xs]);
+        xs = xs + 1 == XS ? 0 : xs + 1;
+      }
+      mma_commit_elect(&done[b % AB]);
     }
+    mma_commit_elect(accb);   // arrives once all issued MMAs are complete
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- dequant + epilogue
