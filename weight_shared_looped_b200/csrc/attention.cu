@@ -484,6 +484,280 @@ __global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a
   }
 }
 
+// ------------------------------------------------------------------ decode (cluster)
+// Decode attention for one (row, head) on a thread-block cluster of CL CTAs
+// (CL = ceil(max_ctx / 64) capped at 8, fixed per cache).  CTA r takes the
+// contiguous keys [r * per, (r + 1) * per) of the lane's n_keys = pos + 1
+// (per = ceil(n_keys / CL), which depends only on the lane's own position);
+// its cached K/V rows are copied into shared memory before the wait for the
+// QKV projection.  The CTA holding position pos forms k and v from the QKV
+// partial sums, applies RoPE to k and appends both to the cache.  Each CTA
+// keeps its max score, exponential sum and unnormalised P V; rank 0 merges
+// the CTAs in rank order through distributed shared memory.
+__device__ __forceinline__ void cl_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+__device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
+  uint32_t addr = (uint32_t)__cvta_generic_to_shared(local), remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+template <int HD>
+__global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs a, int CL,
+                                                                  int max_per) {
+  constexpr int HALF = HD / 2;
+  constexpr int KSPLIT = 128 / HD;              // key slices in the P V step
+  extern __shared__ __align__(16) unsigned char dsm[];
+  __shared__ float qs[HD], kn[HD], vn[HD];
+  __shared__ float acc_s[KSPLIT][HD];
+  __shared__ float stat_s[2];                    // this CTA's max score and exponential sum
+  __shared__ float red[4];
+  const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int esz = a.kv_int8 ? 1 : 2;
+  const int rowb = HD * esz;
+  unsigned char* kst = dsm;                                          // [max_per][rowb]
+  unsigned char* vst = dsm + (size_t)max_per * rowb;                 // [max_per][rowb]
+  float* ksc = reinterpret_cast<float*>(dsm + 2 * (size_t)max_per * rowb);
+  float* vsc = ksc + max_per;
+  float* pr = vsc + max_per;                                         // scores, then weights
+  // positions, the lane map, the RoPE table and the cached rows before pos
+  // were written by earlier steps
+  const int lane_id = a.lane_of_row[row];
+  const int pos = a.hdr->pos[lane_id];
+  const int n_keys = pos + 1;
+  const int per = (n_keys + CL - 1) / CL;
+  const int k0 = min(crank * per, n_keys), k1 = min(k0 + per, n_keys);
+  const int nk = k1 - k0;
+  const bool owner = nk > 0 && k1 == n_keys;     // holds position pos
+  const int n_old = owner ? nk - 1 : nk;
+  char* layer = const_cast<char*>(a.kv_base) +
+                (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
+  const size_t head_off = (size_t)head * a.max_ctx;
+  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
+  {
+    const int pieces = rowb / 16;
+    for (int which = 0; which < 2; ++which) {
+      const char* src = layer + which * a.kv_region_bytes + (head_off + k0) * rowb;
+      unsigned char* dst = which ? vst : kst;
+      for (int i = tid; i < n_old * pieces; i += 128) {
+        const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i * 16);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + i * 16)
+                     : "memory");
+      }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    if (a.kv_int8) {
+      const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
+      const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
+      for (int j = tid; j < n_old; j += 128) {
+        ksc[j] = __half2float(kq[head_off + k0 + j]);
+        vsc[j] = __half2float(vq[head_off + k0 + j]);
+      }
+    }
+  }
+  float2 cs = make_float2(1.f, 0.f);
+  if (tid < HD) cs = a.rope_cs[(size_t)pos * HALF + (tid % HALF)];
+  pdl_enter();
+
+  // q (and k, v in the owner) from the QKV partial sums, all splits in flight
+  const size_t split_stride = (size_t)a.rows * 3 * a.d;
+  const float* prow = a.qkv_part + (size_t)row * 3 * a.d + (size_t)head * HD;
+  if (tid < HD) {
+    float pq[8], pk[8], pv[8];
+    float sq = 0.f, sk = 0.f, sv = 0.f;
+    for (int s0 = 0; s0 < a.qkv_S; s0 += 8) {
+      const int cnt = min(8, a.qkv_S - s0);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < cnt) {
+          const float* q = prow + (size_t)(s0 + j) * split_stride;
+          pq[j] = q[tid];
+          pk[j] = owner ? q[a.d + tid] : 0.f;
+          pv[j] = owner ? q[2 * a.d + tid] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < cnt) {
+          sq += pq[j];
+          sk += pk[j];
+          sv += pv[j];
+        }
+      }
+    }
+    qs[tid] = sq;
+    kn[tid] = sk;
+    vn[tid] = sv;
+  }
+  __syncthreads();
+  float qr = 0.f, kr = 0.f;
+  if (tid < HD) {
+    if (tid < HALF) {
+      qr = qs[tid] * cs.x - qs[tid + HALF] * cs.y;
+      kr = kn[tid] * cs.x - kn[tid + HALF] * cs.y;
+    } else {
+      qr = qs[tid] * cs.x + qs[tid - HALF] * cs.y;
+      kr = kn[tid] * cs.x + kn[tid - HALF] * cs.y;
+    }
+  }
+  __syncthreads();
+  // the query is rounded to fp16 as in the prefill path
+  if (tid < HD) qs[tid] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
+
+  if (owner) {
+    // append k (after RoPE) and v at position pos, in the cache and in the
+    // staged rows
+    const int jr = nk - 1;
+    const __half kh = __float2half_rn(kr);
+    const __half vh = __float2half_rn(tid < HD ? vn[tid] : 0.f);
+    if (!a.kv_int8) {
+      if (tid < HD) {
+        reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + tid] = kh;
+        reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = vh;
+        reinterpret_cast<__half*>(kst)[jr * HD + tid] = kh;
+        reinterpret_cast<__half*>(vst)[jr * HD + tid] = vh;
+      }
+    } else {
+      __shared__ float kmax_s[4], vmax_s[4];
+      float km = tid < HD ? fabsf(__half2float(kh)) : 0.f;
+      float vm = tid < HD ? fabsf(__half2float(vh)) : 0.f;
+      km = warp_max(km);
+      vm = warp_max(vm);
+      if (lane == 0) {
+        kmax_s[warp] = km;
+        vmax_s[warp] = vm;
+      }
+      __syncthreads();
+      km = fmaxf(fmaxf(kmax_s[0], kmax_s[1]), fmaxf(kmax_s[2], kmax_s[3]));
+      vm = fmaxf(fmaxf(vmax_s[0], vmax_s[1]), fmaxf(vmax_s[2], vmax_s[3]));
+      const __half ksh = __float2half_rn(__fdiv_rn(km, 127.0f));
+      const __half vsh = __float2half_rn(__fdiv_rn(vm, 127.0f));
+      const float ksf = __half2float(ksh), vsf = __half2float(vsh);
+      if (tid < HD) {
+        const float kx = __half2float(kh), vx = __half2float(vh);
+        const int kc = ksf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ksf)), -127.f), 127.f);
+        const int vc = vsf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vsf)), -127.f), 127.f);
+        reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + tid] = (int8_t)kc;
+        reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = (int8_t)vc;
+        reinterpret_cast<int8_t*>(kst)[jr * HD + tid] = (int8_t)kc;
+        reinterpret_cast<int8_t*>(vst)[jr * HD + tid] = (int8_t)vc;
+      }
+      if (tid == 0) {
+        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
+        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] = vsh;
+        ksc[jr] = ksf;
+        vsc[jr] = vsf;
+      }
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();   // staged rows, the appended entry and q are visible to the whole CTA
+
+  // scores: one key per thread, four partial dot products
+  float lmax = -INFINITY;
+  for (int j = tid; j < nk; j += 128) {
+    float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+    if (!a.kv_int8) {
+      const uint4* src = reinterpret_cast<const uint4*>(kst + (size_t)j * rowb);
+#pragma unroll
+      for (int c = 0; c < HD / 8; ++c) {
+        const uint4 w = src[c];
+        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w.z));
+        const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&w.w));
+        d0 = fmaf(qs[c * 8 + 0], f0.x, fmaf(qs[c * 8 + 1], f0.y, d0));
+        d1 = fmaf(qs[c * 8 + 2], f1.x, fmaf(qs[c * 8 + 3], f1.y, d1));
+        d2 = fmaf(qs[c * 8 + 4], f2.x, fmaf(qs[c * 8 + 5], f2.y, d2));
+        d3 = fmaf(qs[c * 8 + 6], f3.x, fmaf(qs[c * 8 + 7], f3.y, d3));
+      }
+    } else {
+      const uint4* src = reinterpret_cast<const uint4*>(kst + (size_t)j * rowb);
+#pragma unroll
+      for (int c = 0; c < HD / 16; ++c) {
+        const uint4 w = src[c];
+        const int8_t* b = reinterpret_cast<const int8_t*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          d0 = fmaf(qs[c * 16 + e], (float)b[e], d0);
+          d1 = fmaf(qs[c * 16 + 4 + e], (float)b[4 + e], d1);
+          d2 = fmaf(qs[c * 16 + 8 + e], (float)b[8 + e], d2);
+          d3 = fmaf(qs[c * 16 + 12 + e], (float)b[12 + e], d3);
+        }
+      }
+    }
+    float sc = (d0 + d1) + (d2 + d3);
+    if (a.kv_int8) sc *= ksc[j];
+    pr[j] = sc;
+    lmax = fmaxf(lmax, sc);
+  }
+  lmax = warp_max(lmax);
+  if (lane == 0) red[warp] = lmax;
+  __syncthreads();
+  const float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();   // red is reused below
+  float lsum = 0.f;
+  for (int j = tid; j < nk; j += 128) {
+    const float e = __expf(pr[j] - m);
+    lsum += e;
+    pr[j] = a.kv_int8 ? e * vsc[j] : e;   // INT8: fold the V scale into the weight
+  }
+  lsum = warp_sum(lsum);
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();   // weights and partial sums visible
+  const float l = (red[0] + red[1]) + (red[2] + red[3]);
+  // P V: thread (e, ks) takes dimension e over keys j = ks, ks + KSPLIT, ...
+  {
+    const int e = tid % HD, ks = tid / HD;
+    float acc0 = 0.f, acc1 = 0.f;
+    int j = ks;
+    if (!a.kv_int8) {
+      const __half* src = reinterpret_cast<const __half*>(vst) + e;
+      for (; j + KSPLIT < nk; j += 2 * KSPLIT) {
+        acc0 = fmaf(pr[j], __half2float(src[(size_t)j * HD]), acc0);
+        acc1 = fmaf(pr[j + KSPLIT], __half2float(src[(size_t)(j + KSPLIT) * HD]), acc1);
+      }
+      if (j < nk) acc0 = fmaf(pr[j], __half2float(src[(size_t)j * HD]), acc0);
+    } else {
+      const int8_t* src = reinterpret_cast<const int8_t*>(vst) + e;
+      for (; j + KSPLIT < nk; j += 2 * KSPLIT) {
+        acc0 = fmaf(pr[j], (float)src[(size_t)j * HD], acc0);
+        acc1 = fmaf(pr[j + KSPLIT], (float)src[(size_t)(j + KSPLIT) * HD], acc1);
+      }
+      if (j < nk) acc0 = fmaf(pr[j], (float)src[(size_t)j * HD], acc0);
+    }
+    acc_s[ks][e] = acc0 + acc1;
+  }
+  if (tid == 0) {
+    stat_s[0] = nk > 0 ? m : -INFINITY;
+    stat_s[1] = nk > 0 ? l : 0.f;
+  }
+  cl_sync();   // every CTA's statistics and P V are in its shared memory
+  if (crank == 0) {
+    float M = -INFINITY;
+    for (int r = 0; r < CL; ++r) M = fmaxf(M, cl_ld(&stat_s[0], (uint32_t)r));
+    for (int e = tid; e < HD; e += 128) {
+      float L = 0.f, o = 0.f;
+      for (int r = 0; r < CL; ++r) {
+        const float mr = cl_ld(&stat_s[0], (uint32_t)r);
+        const float w = mr == -INFINITY ? 0.f : __expf(mr - M);
+        L = fmaf(cl_ld(&stat_s[1], (uint32_t)r), w, L);
+        float pv = 0.f;
+#pragma unroll
+        for (int q = 0; q < KSPLIT; ++q) pv += cl_ld(&acc_s[q][e], (uint32_t)r);
+        o = fmaf(pv, w, o);
+      }
+      a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
+    }
+  }
+  cl_sync();   // no CTA leaves while rank 0 still reads its shared memory
+}
+
 }  // namespace
 
 tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
@@ -500,16 +774,49 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   return ok();
 }
 
+// Cluster size and staged rows per CTA of the cluster decode kernel for a
+// cache of max_ctx positions; 0 when the staged rows would not fit.
+static int decode_cluster_size(int max_ctx) {
+  const int c = (max_ctx + 63) / 64;
+  return c < 1 ? 1 : c > 8 ? 8 : c;
+}
+static size_t decode_cluster_smem(int max_ctx, int hd, bool int8, int* max_per) {
+  const int cl = decode_cluster_size(max_ctx);
+  *max_per = (max_ctx + cl - 1) / cl;
+  const size_t rowb = (size_t)hd * (int8 ? 1 : 2);
+  return 2 * (size_t)*max_per * rowb + 3 * (size_t)*max_per * sizeof(float);
+}
+
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
+  if (a.hd != 128 && a.hd != 64)
+    return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
+  int max_per = 0;
+  const size_t smem = decode_cluster_smem(a.max_ctx, a.hd, a.kv_int8 != 0, &max_per);
+  if (smem + 8 * 1024 <= 227 * 1024) {
+    static bool attr_done = false;
+    if (!attr_done) {
+      TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+      attr_done = true;
+    }
+    const int cl = decode_cluster_size(a.max_ctx);
+    dim3 grid(cl, a.H, a.rows);
+    cudaError_t e = a.hd == 128
+        ? launch_pdl_cluster(attn_decode_cluster_kernel<128>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per)
+        : launch_pdl_cluster(attn_decode_cluster_kernel<64>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per);
+    if (e != cudaSuccess)
+      return set_error(TL_ERR_CUDA, "launch of attn_decode_cluster_kernel failed: %s", cudaGetErrorString(e));
+    return ok();
+  }
+  // long caches: 64-key chunks merged by the last CTA of each (row, head)
   dim3 grid(a.max_chunks, a.H, a.rows);
   if (a.hd == 128)
     TL_LAUNCH_PDL(attn_decode_fused_kernel<128>, grid, 128, 0, s, a);
-  else if (a.hd == 64)
-    TL_LAUNCH_PDL(attn_decode_fused_kernel<64>, grid, 128, 0, s, a);
   else
-    return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
+    TL_LAUNCH_PDL(attn_decode_fused_kernel<64>, grid, 128, 0, s, a);
   return ok();
 }
-
 }  // namespace tl
