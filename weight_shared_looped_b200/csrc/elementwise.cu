@@ -47,27 +47,14 @@ __global__ void embed_kernel(EmbedArgs a) {
 }
 
 // ------------------------------------------------------------------ residual + RMSNorm
-// A row of d columns is split over a thread-block cluster of C CTAs (C = d/512
-// capped at 8; consecutive blockIdx.x form a cluster), each CTA d/C columns,
-// each thread VPT float4 vectors (VPT = 1, or 2 for d = 8192).  The split-K
-// partial sums are loaded eight splits at a time (independent loads in
-// flight) and added in split order.  The sum of squares is reduced per thread,
-// per warp (xor tree), over the CTA's warps and over the cluster's CTAs (read
-// through distributed shared memory) in a fixed order that depends only on d.
-constexpr int NORM_MAX_THREADS = 128;
-
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
-                   "memory");
-}
-
-__device__ __forceinline__ float cluster_read_f32(const float* local, uint32_t rank) {
-  uint32_t addr = (uint32_t)__cvta_generic_to_shared(local), remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
-  return v;
-}
+// One CTA of d/8 threads per row, each thread two float4 vectors (columns
+// 4t.. and d/2 + 4t..).  The split-K partial sums are loaded four splits at a
+// time (independent loads in flight) and added in split order.  The sum of
+// squares is reduced per thread, per warp (xor tree) and over the warps in
+// order: a fixed order that depends only on d.  One CTA per row keeps the
+// grid small (a prefill of 128 rows is one CTA per SM) so that it shares the
+// SMs with the GEMM CTAs launched early next to it.
+constexpr int NORM_MAX_WARPS = 32;
 
 __device__ __forceinline__ void add4(float4& a, const float4 b) {
   a.x += b.x;
@@ -76,102 +63,89 @@ __device__ __forceinline__ void add4(float4& a, const float4 b) {
   a.w += b.w;
 }
 
-template <int VPT>
-__global__ void __launch_bounds__(NORM_MAX_THREADS) residual_norm_kernel(NormArgs a, int C) {
+__global__ void __launch_bounds__(1024) residual_norm_kernel(NormArgs a) {
   pdl_enter();
-  __shared__ float red[NORM_MAX_THREADS / 32];
-  __shared__ float cta_sum;
-  const int row = blockIdx.x / C;
-  const int crank = blockIdx.x % C;
-  const int cols = a.d / C;
-  const int nthr = blockDim.x;
-  const int nw = nthr / 32;
+  __shared__ float red[NORM_MAX_WARPS];
+  const int row = blockIdx.x;
+  const int nthr = blockDim.x, nw = nthr >> 5;
+  const int c0 = threadIdx.x * 4, c1 = a.d / 2 + threadIdx.x * 4;
   float* h = a.h + (size_t)row * a.d;
   const int out_row = a.out_row ? a.out_row[row] : row;
-  int col[VPT];
-#pragma unroll
-  for (int e = 0; e < VPT; ++e) col[e] = crank * cols + (e * nthr + threadIdx.x) * 4;
-  float4 v[VPT];
-#pragma unroll
-  for (int e = 0; e < VPT; ++e) v[e] = *reinterpret_cast<const float4*>(h + col[e]);
+  float4 v0 = *reinterpret_cast<const float4*>(h + c0);
+  float4 v1 = *reinterpret_cast<const float4*>(h + c1);
   if (row < a.n_add && a.S > 0) {
     const size_t sstride = (size_t)a.part_rows * a.d;
     const float* p0 = a.part + (size_t)row * a.d;
-    for (int sp = 0; sp < a.S; sp += 8) {
-      const int n = min(8, a.S - sp);
-      float4 t[8][VPT];
+    for (int sp = 0; sp < a.S; sp += 4) {
+      const int n = min(4, a.S - sp);
+      float4 t0[4], t1[4];
 #pragma unroll
-      for (int q = 0; q < 8; ++q)
+      for (int q = 0; q < 4; ++q) {
+        if (q < n) {
+          t0[q] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + c0));
+          t1[q] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + c1));
+        }
+      }
 #pragma unroll
-        for (int e = 0; e < VPT; ++e)
-          if (q < n) t[q][e] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + col[e]));
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-#pragma unroll
-        for (int e = 0; e < VPT; ++e)
-          if (q < n) add4(v[e], t[q][e]);
+      for (int q = 0; q < 4; ++q) {
+        if (q < n) {
+          add4(v0, t0[q]);
+          add4(v1, t1[q]);
+        }
+      }
     }
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) *reinterpret_cast<float4*>(h + col[e]) = v[e];
+    *reinterpret_cast<float4*>(h + c0) = v0;
+    *reinterpret_cast<float4*>(h + c1) = v1;
   }
   if (a.trace) {
     float* tr = a.trace + (size_t)out_row * a.d;
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) *reinterpret_cast<float4*>(tr + col[e]) = v[e];
+    *reinterpret_cast<float4*>(tr + c0) = v0;
+    *reinterpret_cast<float4*>(tr + c1) = v1;
   }
-  // row-uniform, hence uniform across the cluster: every CTA reaches the
-  // cluster barriers below
   const bool want_x = row < a.n_next;
   const bool want_y = row >= a.fin_lo && row < a.fin_hi;
+  if (!want_x && !want_y) return;
   float ss = 0.0f;
-#pragma unroll
-  for (int e = 0; e < VPT; ++e) {
-    ss = fmaf(v[e].x, v[e].x, ss);
-    ss = fmaf(v[e].y, v[e].y, ss);
-    ss = fmaf(v[e].z, v[e].z, ss);
-    ss = fmaf(v[e].w, v[e].w, ss);
-  }
+  ss = fmaf(v0.x, v0.x, ss);
+  ss = fmaf(v0.y, v0.y, ss);
+  ss = fmaf(v0.z, v0.z, ss);
+  ss = fmaf(v0.w, v0.w, ss);
+  ss = fmaf(v1.x, v1.x, ss);
+  ss = fmaf(v1.y, v1.y, ss);
+  ss = fmaf(v1.z, v1.z, ss);
+  ss = fmaf(v1.w, v1.w, ss);
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    float c = 0.0f;
-    for (int w = 0; w < nw; ++w) c += red[w];
-    cta_sum = c;
-  }
-  cluster_sync_all();   // every CTA's cta_sum is written
   float tot = 0.0f;
-  for (int q = 0; q < C; ++q) tot += cluster_read_f32(&cta_sum, (uint32_t)q);
-  cluster_sync_all();   // no CTA leaves while another still reads its cta_sum
-  if (!want_x && !want_y) return;
+  for (int w = 0; w < nw; ++w) tot += red[w];
   const float r = rsqrtf(tot / (float)a.d + a.eps);
+  auto out_x = [&](int c, const float4 v) {
+    const float4 g = *reinterpret_cast<const float4*>(a.gamma_next + c);
+    const __half2 lo = __halves2half2(__float2half_rn(v.x * r * g.x), __float2half_rn(v.y * r * g.y));
+    const __half2 hi = __halves2half2(__float2half_rn(v.z * r * g.z), __float2half_rn(v.w * r * g.w));
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+    pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(a.x + (size_t)row * a.d + c) = pk;
+  };
+  auto out_y = [&](int c, const float4 v) -> bool {
+    const float4 g = *reinterpret_cast<const float4*>(a.gamma_final + c);
+    float4 o;
+    o.x = v.x * r * g.x;
+    o.y = v.y * r * g.y;
+    o.z = v.z * r * g.z;
+    o.w = v.w * r * g.w;
+    *reinterpret_cast<float4*>(a.y + (size_t)out_row * a.d + c) = o;
+    return !isfinite(o.x) || !isfinite(o.y) || !isfinite(o.z) || !isfinite(o.w);
+  };
   if (want_x) {
-    __half* x = a.x + (size_t)row * a.d;
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) {
-      const float4 g = *reinterpret_cast<const float4*>(a.gamma_next + col[e]);
-      const __half2 lo = __halves2half2(__float2half_rn(v[e].x * r * g.x), __float2half_rn(v[e].y * r * g.y));
-      const __half2 hi = __halves2half2(__float2half_rn(v[e].z * r * g.z), __float2half_rn(v[e].w * r * g.w));
-      uint2 pk;
-      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
-      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
-      *reinterpret_cast<uint2*>(x + col[e]) = pk;
-    }
+    out_x(c0, v0);
+    out_x(c1, v1);
   } else {
-    float* y = a.y + (size_t)out_row * a.d;
-    bool bad = false;
-#pragma unroll
-    for (int e = 0; e < VPT; ++e) {
-      const float4 g = *reinterpret_cast<const float4*>(a.gamma_final + col[e]);
-      float4 o;
-      o.x = v[e].x * r * g.x;
-      o.y = v[e].y * r * g.y;
-      o.z = v[e].z * r * g.z;
-      o.w = v[e].w * r * g.w;
-      bad |= !isfinite(o.x) || !isfinite(o.y) || !isfinite(o.z) || !isfinite(o.w);
-      *reinterpret_cast<float4*>(y + col[e]) = o;
-    }
-    if (bad) set_status(a.status, TL_ERR_NUMERIC);
+    const bool bad0 = out_y(c0, v0);
+    const bool bad1 = out_y(c1, v1);
+    if (bad0 || bad1) set_status(a.status, TL_ERR_NUMERIC);
   }
 }
 
@@ -331,19 +305,10 @@ tl_status launch_embed(const EmbedArgs& a, cudaStream_t s) {
 
 tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
-  // d = 256 * 2^k: C = d / 512 CTAs per row (at least 1, at most 8), d / C
-  // columns per CTA, 4 * VPT per thread
+  // d = 256 * 2^k: d / 8 threads (32 .. 1024)
   if (a.d < 256 || a.d > 8192 || (a.d & (a.d - 1)) != 0)
     return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs a power of two in [256, 8192]", a.d);
-  const int C = a.d <= 512 ? 1 : a.d / 512 > 8 ? 8 : a.d / 512;
-  const int cols = a.d / C;
-  const int vpt = cols > 512 ? 2 : 1;
-  const int threads = cols / (4 * vpt);
-  cudaError_t e = vpt == 1 ? launch_pdl_cluster(residual_norm_kernel<1>, dim3(a.rows * C), dim3(threads), 0, s, (unsigned)C, a, C)
-                           : launch_pdl_cluster(residual_norm_kernel<2>, dim3(a.rows * C), dim3(threads), 0, s, (unsigned)C, a, C);
-  if (e != cudaSuccess)
-    return set_error(TL_ERR_CUDA, "launch of residual_norm_kernel failed: %s", cudaGetErrorString(e));
-  TL_LAUNCH_CHECK();
+  TL_LAUNCH_PDL(residual_norm_kernel, a.rows, a.d / 8, 0, s, a);
   return ok();
 }
 

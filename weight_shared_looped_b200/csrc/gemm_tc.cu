@@ -4,24 +4,32 @@
 //   W[n][k] = code[n][k] * scale[n][k / G]  (group-wise symmetric INT4).
 //
 // One CTA per SM computes 128 weight rows x BN tokens over a range of 64-wide
-// k blocks, with three decoupled rings:
-//   * packed weights (128 rows x 8 words per k block) loaded by TMA far ahead
-//     (the first loads are issued before waiting for the previous kernel: the
-//     weights are constants of the model);
-//   * the fp16 A tiles in tensor memory: sixteen dequantisation warps (four
-//     groups of four, one warp per TMEM lane quadrant; group g takes k blocks
-//     i with i % 4 == g; one thread per weight row) turn a row's 64 codes into
-//     fp16 code*scale pairs and store them with tcgen05.st, so the weight tile
-//     is the MMA's A operand and never passes through shared memory;
-//   * the activation tiles x[BN tokens][64 k] (fp16, 128-byte swizzled, rows
-//     past T read as zero) loaded by a second TMA warp.
-// One thread issues tcgen05.mma kind::f16 (M 128, N BN, K 16; A from TMEM, B
-// from shared memory, fp32 accumulation in TMEM) for batches of ready k blocks
-// and commits each k block to the rings it frees.  The dequantisation warps
-// then read the accumulator back with tcgen05.ld, store fp32 partial sums and
-// signal an "epilogue done" barrier that the MMA warp waits on before it frees
-// TMEM.  Every wait on an mbarrier is bounded: when a wait runs out the CTA
-// records TL_ERR_TIMEOUT, stops issuing work, waits (bounded) for its copies in
+// k blocks.  Warp roles:
+//   * sixteen dequantisation warps (four groups of four, one warp per TMEM
+//     lane quadrant; group g takes k blocks i with i % 4 == g; one thread per
+//     weight row) read their row's packed words and scale straight from global
+//     memory, two of their k blocks ahead in registers (the first before the
+//     wait for the previous kernel: weights are constants of the model), turn
+//     the 64 codes into fp16 code*scale pairs and store them with tcgen05.st,
+//     so the weight tile is the MMA's A operand and never passes through
+//     shared memory, which the activation tiles and the MMA keep busy;
+//   * one TMA warp streams the activation tiles x[BN tokens][64 k] (fp16,
+//     128-byte swizzled, rows past T read as zero) through a ring that the
+//     MMAs free one k block at a time;
+//   * a watcher warp waits for each batch's activation tiles and arrives on
+//     the batch's barrier, so neither the MMA warp nor the dequantisation
+//     warps wait on them;
+//   * the MMA warp issues tcgen05.mma kind::f16 (M 128, N BN, K 16; A from
+//     TMEM, B from shared memory, fp32 accumulation in TMEM) per batch of four
+//     k blocks.
+// The producer, watcher and MMA warps keep all lanes converged and issue from
+// one elect.sync-chosen lane: a lone active lane is starved of issue slots by
+// the dequantisation warps sharing its SM sub-partition.  The dequantisation
+// warps then read the accumulator back with tcgen05.ld, store fp32 partial
+// sums (or, for [gate; up] with one split, fp16 silu(gate) * up) and signal an
+// "epilogue done" barrier that the MMA warp waits on before it frees TMEM.
+// Every wait on an mbarrier is bounded: when a wait runs out the CTA records
+// TL_ERR_TIMEOUT, stops issuing work, waits (bounded) for its copies in
 // flight, frees its TMEM and returns.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -35,7 +43,7 @@ constexpr int BM = 128;            // weight rows per CTA (MMA M)
 constexpr int BK = 64;             // k per stage
 constexpr int DQ_GROUPS = 4;       // dequantisation groups, each 4 warps (one per TMEM quadrant)
 constexpr int DQ_WARPS = 4 * DQ_GROUPS;
-constexpr int WTMA_WARP = DQ_WARPS, XTMA_WARP = DQ_WARPS + 1, MMA_WARP = DQ_WARPS + 2;
+constexpr int XTMA_WARP = DQ_WARPS, MMA_WARP = DQ_WARPS + 1, XWAIT_WARP = DQ_WARPS + 2;
 constexpr int THREADS = 32 * (DQ_WARPS + 3);
 constexpr int TMEM_COLS = 512;     // the whole of TMEM: one CTA per SM
 constexpr int A_COLS = BK / 2;     // TMEM columns per A stage (two fp16 per column)
@@ -43,8 +51,7 @@ constexpr int BATCH = DQ_GROUPS;   // k blocks per batch: one per dequantisation
 constexpr size_t kMinSmem = 120 * 1024;   // also keeps it to one CTA per SM
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // a bounded wait gives up after 2 s
 template <int BN> struct TcCfg {
-  static constexpr int W_STAGES = 2 * BATCH;                  // packed-weight ring (k blocks)
-  static constexpr int X_STAGES = BN >= 128 ? 8 : 12;         // activation ring (k blocks)
+  static constexpr int X_STAGES = BN >= 128 ? 12 : 16;        // activation ring (k blocks)
   static constexpr int A_BATCHES = (TMEM_COLS - BN) / (A_COLS * BATCH);   // TMEM A ring (batches)
 };
 
@@ -107,21 +114,6 @@ __device__ __forceinline__ void tma_issue_elect(uint64_t* bar, uint32_t bytes, v
       : "memory");
 }
 
-// Two tiles of one stage (64 gate rows and 64 up rows) on one barrier.
-__device__ __forceinline__ void tma_issue2_elect(uint64_t* bar, uint32_t bytes, void* dst0,
-                                                 const CUtensorMap* map0, void* dst1,
-                                                 const CUtensorMap* map1, int x, int y) {
-  asm volatile(
-      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
-      " @e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
-      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%2], [%3, "
-      "{%6, %7}], [%0];\n"
-      " @e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5, "
-      "{%6, %7}], [%0];\n}\n" ::"r"(smem_u32(bar)),
-      "r"(bytes), "r"(smem_u32(dst0)), "l"(map0), "r"(smem_u32(dst1)), "l"(map1), "r"(x), "r"(y)
-      : "memory");
-}
-
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
   // K-major, 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart
   uint64_t d = 0;
@@ -173,21 +165,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-__device__ __forceinline__ uint32_t dequant_code_pair(uint32_t w, uint32_t sel) {
-  // byte b of w holds the codes of k = 2b (low nibble) and 2b + 1 (high nibble)
-  uint32_t x, h;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(w), "r"(0u), "r"(sel));
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
-  const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
-  const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
-  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);
-  return *reinterpret_cast<uint32_t*>(&r);
-}
-
 struct TcArgs {
   int N, K, G, T, n_split;   // n_split % 128 == 0
   int splits;                // split z covers k blocks [z*nkb/S, (z+1)*nkb/S)
-  int max_groups;            // scale groups staged per CTA (shared-memory sizing)
+  const uint32_t* w0;        // canonical INT4 words of rows [0, n_split)
+  const uint32_t* w1;        // rows [n_split, N)
   const __half* s0;
   const __half* s1;
   float* part;
@@ -195,35 +177,35 @@ struct TcArgs {
   __half* swiglu_u;          // fused SwiGLU epilogue: fp16 [T][n_split] (N = 2 * n_split)
 };
 
+// The elected lane arrives once on a barrier for the whole warp.
+__device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n"
+      " @e mbarrier.arrive.shared::cta.b64 _, [%0];\n}\n" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+// 80 registers x 608 threads leave room in the register file for a CTA of the
+// next (or previous) small kernel on the same SM while this one runs.
 template <int BN>
-__global__ void __launch_bounds__(THREADS, 1)
-    gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x,
-                      const __grid_constant__ CUtensorMap map_w0,
-                      const __grid_constant__ CUtensorMap map_w1, TcArgs a) {
-  constexpr int WS = TcCfg<BN>::W_STAGES, XS = TcCfg<BN>::X_STAGES;
+__global__ void __maxnreg__(80)
+    gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x, TcArgs a) {
+  constexpr int XS = TcCfg<BN>::X_STAGES;
   constexpr int AB = TcCfg<BN>::A_BATCHES;
   constexpr uint32_t X_BYTES = BN * 128;          // BN rows x 64 fp16
-  constexpr uint32_t W_BYTES = BM * 32;           // 128 rows x 8 words
   static_assert(BN + AB * BATCH * A_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(AB >= 2 && XS >= 2 * BATCH && WS % DQ_GROUPS == 0, "ring depths");
+  static_assert(AB >= 2 && XS >= 2 * BATCH, "ring depths");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sX = smem;                                        // XS x X_BYTES
-  uint8_t* sW = sX + XS * X_BYTES;                           // WS x W_BYTES
-  __half* sScale = reinterpret_cast<__half*>(sW + WS * W_BYTES);   // [BM][groups]
   const int nkb_total = a.K / BK;
   const int kb_begin = (int)(((long)blockIdx.z * nkb_total) / a.splits);
   const int nkb = (int)(((long)(blockIdx.z + 1) * nkb_total) / a.splits) - kb_begin;
   const int nbatch = (nkb + BATCH - 1) / BATCH;
-  const int g_first = (kb_begin * BK) / a.G;
-  const int groups = ((kb_begin + nkb) * BK - 1) / a.G - g_first + 1;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sScale + BM * a.max_groups + 8);
-  bars = reinterpret_cast<uint64_t*>(((uintptr_t)bars + 7) & ~(uintptr_t)7);
-  uint64_t* wfull = bars;               // packed weights of a k block landed
-  uint64_t* wempty = wfull + WS;        // dequantisation done reading them
-  uint64_t* xfull = wempty + WS;        // activations of a k block landed
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sX + XS * X_BYTES);
+  uint64_t* xfull = bars;               // activations of a k block landed
   uint64_t* xempty = xfull + XS;        // MMAs of a k block complete: frees its X slot
-  uint64_t* afull = xempty + XS;        // A tiles of a batch in TMEM (and its activations seen)
+  uint64_t* afull = xempty + XS;        // A tiles and activations of a batch ready
   uint64_t* done = afull + AB;          // MMAs of a batch complete: frees its A slots
   uint64_t* accb = done + AB;           // accumulator complete
   uint64_t* epib = accb + 1;            // epilogue finished reading TMEM
@@ -234,24 +216,18 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int m0 = blockIdx.x * BM;
   const int t0 = blockIdx.y * BN;
   // fused SwiGLU: tile rows [0, 64) are gate rows wrow0.., rows [64, 128) the
-  // same rows of up (two 64-row weight loads per k block)
+  // same rows of up
   const bool sw = a.swiglu_u != nullptr;
   const bool second = !sw && m0 >= a.n_split;
-  const CUtensorMap* map_w = second ? &map_w1 : &map_w0;
   const int wrow0 = sw ? blockIdx.x * (BM / 2) : second ? m0 - a.n_split : m0;
-  const __half* scales = second ? a.s1 : a.s0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < WS; ++s) {
-      mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 4);
-    }
     for (int s = 0; s < XS; ++s) {
       mbar_init(&xfull[s], 1);
       mbar_init(&xempty[s], 1);
     }
     for (int s = 0; s < AB; ++s) {
-      mbar_init(&afull[s], DQ_WARPS);
+      mbar_init(&afull[s], DQ_WARPS + 1);   // + the activation watcher
       mbar_init(&done[s], 1);
     }
     mbar_init(accb, 1);
@@ -259,8 +235,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(&map_x) : "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(map_w) : "memory");
-    if (sw) asm volatile("prefetch.tensormap [%0];" ::"l"(&map_w1) : "memory");
   }
   __syncwarp();
   if (warp == MMA_WARP) {
@@ -276,29 +250,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t acc_col = 0;
   const uint32_t a_col0 = BN;
 
-  if (warp == WTMA_WARP) {
-    // ---------------------------------------------------------------- weight TMA
-    // weights are constants of the model: no need to wait for the previous kernel
-    int issued = 0;
-    for (int i = 0; i < nkb; ++i) {
-      const int s = i % WS;
-      if (!warp_wait(&wempty[s], ((i / WS) - 1) & 1, abort_flag, i >= WS)) {
-        if (lane == 0) atomicExch(abort_flag, 1);
-        break;
-      }
-      if (sw)
-        tma_issue2_elect(&wfull[s], W_BYTES, sW + s * W_BYTES, &map_w0,
-                         sW + s * W_BYTES + (BM / 2) * 32, &map_w1, (kb_begin + i) * (BK / 8), wrow0);
-      else
-        tma_issue_elect(&wfull[s], W_BYTES, sW + s * W_BYTES, map_w, (kb_begin + i) * (BK / 8), wrow0);
-      issued = i + 1;
-    }
-    if (lane == 0 && *(volatile int*)abort_flag)
-      for (int i = issued > WS ? issued - WS : 0; i < issued; ++i)   // the ones still in flight
-        mbar_wait(&wfull[i % WS], (i / WS) & 1);
-    __syncwarp();
-    pdl_enter();
-  } else if (warp == XTMA_WARP) {
+  if (warp == XTMA_WARP) {
     // ---------------------------------------------------------------- activation TMA
     pdl_enter();   // the activations come from the previous kernel
     int issued = 0;
@@ -315,11 +267,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int i = issued > XS ? issued - XS : 0; i < issued; ++i)   // the ones still in flight
         mbar_wait(&xfull[i % XS], (i / XS) & 1);
     __syncwarp();
+  } else if (warp == XWAIT_WARP) {
+    // ---------------------------------------------------------------- activation watcher
+    // waits until a batch's activation tiles have landed and arrives on its
+    // afull barrier, so neither the MMA warp nor the dequantisation warps
+    // wait on them
+    pdl_enter();
+    for (int b = 0; b < nbatch; ++b) {
+      const int cnt = min(BATCH, nkb - b * BATCH);
+      bool okw = true;
+      for (int j = 0; j < cnt && okw; ++j) {
+        const int i = b * BATCH + j;
+        okw = warp_wait(&xfull[i % XS], (i / XS) & 1, abort_flag, true);
+      }
+      if (!okw) {
+        if (lane == 0) atomicExch(abort_flag, 1);
+        break;
+      }
+      mbar_arrive_elect(&afull[b % AB]);
+    }
+    __syncwarp();
   } else if (warp == MMA_WARP) {
     // ---------------------------------------------------------------- MMA
-    // per batch: one wait (A tiles written and activations seen), one fence,
-    // up to 16 MMAs, one commit per k block (frees its activation slot) and
-    // one per batch (frees its A slots)
+    // per batch: one wait (A tiles written and activations landed), one
+    // fence, up to 16 MMAs, one commit per k block (frees its activation
+    // slot) and one per batch (frees its A slots)
     pdl_enter();
     const uint32_t idesc = (1u << 4) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
     // loop-invariant operands: the X ring's first descriptor (each slot adds
@@ -351,50 +323,62 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int grp = warp >> 2;                  // this group takes k block grp of every batch
     const int r = quad * 32 + lane;             // weight row within the tile = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    // scales of this CTA's rows and k range -> shared memory (constants: read
-    // before waiting for the previous kernel)
-    {
-      const int gpr = a.K / a.G;
-      const int g0 = g_first;
-      for (int i = threadIdx.x; i < BM * groups; i += 32 * DQ_WARPS) {
-        const int rr = i / groups, gg = i % groups;
-        const __half* sp = !sw ? scales + (size_t)(wrow0 + rr) * gpr
-                           : rr < BM / 2 ? a.s0 + (size_t)(wrow0 + rr) * gpr
-                                         : a.s1 + (size_t)(wrow0 + rr - BM / 2) * gpr;
-        sScale[rr * groups + gg] = g0 + gg < gpr ? sp[g0 + gg] : __float2half_rn(0.f);
-      }
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * DQ_WARPS) : "memory");
+    // this thread's weight row (canonical INT4 words) and scale row
+    const size_t wpr = (size_t)a.K / 8, gpr = (size_t)a.K / a.G;
+    const uint32_t* wrow;
+    const __half* srow;
+    if (sw) {
+      const bool up = r >= BM / 2;
+      const size_t row = (size_t)wrow0 + (up ? r - BM / 2 : r);
+      wrow = (up ? a.w1 : a.w0) + row * wpr;
+      srow = (up ? a.s1 : a.s0) + row * gpr;
+    } else {
+      wrow = (second ? a.w1 : a.w0) + (size_t)(wrow0 + r) * wpr;
+      srow = (second ? a.s1 : a.s0) + (size_t)(wrow0 + r) * gpr;
     }
-    for (int b = 0; b < nbatch; ++b) {
+    // The packed words (32 bytes per row and k block) and the scale come
+    // straight from global memory through the read-only path, two of this
+    // group's k blocks ahead in registers (sets 0 and 1 alternate).  Weights
+    // are constants of the model: the first loads go out before the wait for
+    // the previous kernel.
+    uint4 wa0 = make_uint4(0u, 0u, 0u, 0u), wb0 = wa0, wa1 = wa0, wb1 = wa0;
+    __half sc0 = __float2half_rn(0.f), sc1 = sc0;
+    auto fetch = [&](int i, uint4& wa, uint4& wb, __half& sc) {
+      if (i < nkb) {
+        const uint4* p = reinterpret_cast<const uint4*>(wrow + (size_t)(kb_begin + i) * (BK / 8));
+        wa = __ldg(p);
+        wb = __ldg(p + 1);
+        sc = __ldg(srow + ((kb_begin + i) * BK) / a.G);
+      }
+    };
+    fetch(grp, wa0, wb0, sc0);
+    fetch(grp + BATCH, wa1, wb1, sc1);
+    const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
+    const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
+    // one k block of batch b: wait for the A slot, dequantise, store to TMEM,
+    // refill the register set with this group's k block two batches on
+    auto kblock = [&](int b, uint4& wa, uint4& wb, __half& sc) -> bool {
       const int i = b * BATCH + grp;
       // the TMEM slot of this batch is free once batch b - AB is done
-      if (b >= AB && !mbar_wait(&done[(b - AB) % AB], ((b - AB) / AB) & 1)) {
-        atomicExch(abort_flag, 1);
-        break;
-      }
+      // (a failure elsewhere surfaces here as a timed-out wait)
+      if (b >= AB && !mbar_wait(&done[(b - AB) % AB], ((b - AB) / AB) & 1)) return false;
       if (i < nkb) {
-        const int ws = i % WS;
-        if (!mbar_wait(&wfull[ws], (i / WS) & 1) || *(volatile int*)abort_flag) {
-          atomicExch(abort_flag, 1);
-          break;
-        }
-        const uint4* wp = reinterpret_cast<const uint4*>(sW + ws * W_BYTES + r * 32);
-        const uint4 wa = wp[0], wb = wp[1];
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&wempty[ws]);   // the packed words are in registers
         const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        const int g = ((kb_begin + i) * BK) / a.G - g_first;
-        const __half sc = sScale[r * groups + g];
         const __half2 s2 = __halves2half2(sc, sc);
         uint32_t v[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
+          // byte c/2... of word c/4: codes of k = 2c (low nibble), 2c + 1 (high)
           const uint32_t bb = c & 3;
-          const uint32_t sel = bb | 0x40u | (bb << 8) | 0x4000u;
-          uint32_t code = dequant_code_pair(words[c >> 2], sel);
-          __half2 wv = __hmul2(*reinterpret_cast<__half2*>(&code), s2);
+          uint32_t x, h;
+          asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(words[c >> 2]), "r"(0u),
+              "r"(bb | 0x40u | (bb << 8) | 0x4000u));
+          asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
+          __half2 cv = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);   // exact codes
+          __half2 wv = __hmul2(cv, s2);                                      // fp16(code * s)
           v[c] = *reinterpret_cast<uint32_t*>(&wv);
         }
+        fetch(i + 2 * BATCH, wa, wb, sc);
         if (b >= AB) asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t taddr = tmem_base + lane_addr + a_col0 + ((b % AB) * BATCH + grp) * A_COLS;
         asm volatile(
@@ -408,16 +392,19 @@ __global__ void __launch_bounds__(THREADS, 1)
             "r"(v[29]), "r"(v[30]), "r"(v[31])
             : "memory");
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        // this k block's activations must have landed before the MMA thread
-        // (which waits only on afull) reads them
-        if (!mbar_wait(&xfull[i % XS], (i / XS) & 1)) {
-          atomicExch(abort_flag, 1);
-          break;
-        }
       }
       asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(&afull[b % AB]);
+      return true;
+    };
+    // the dequantisation reads only weights and writes only TMEM: it may run
+    // ahead of the previous kernel; the epilogue's stores wait for it
+    for (int b = 0; b < nbatch; b += 2) {
+      if (!kblock(b, wa0, wb0, sc0) || (b + 1 < nbatch && !kblock(b + 1, wa1, wb1, sc1))) {
+        atomicExch(abort_flag, 1);
+        break;
+      }
     }
     pdl_enter();
     // epilogue: accumulator rows = weight rows, columns = tokens
@@ -575,29 +562,18 @@ tl_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, 
 int tc_tile_n(int T) { return T <= 64 ? 64 : 128; }
 
 template <int BN>
-size_t tc_smem_bytes(int max_groups) {
-  constexpr int WS = TcCfg<BN>::W_STAGES, XS = TcCfg<BN>::X_STAGES;
+size_t tc_smem_bytes() {
+  constexpr int XS = TcCfg<BN>::X_STAGES;
   constexpr int AB = TcCfg<BN>::A_BATCHES;
-  size_t b = 1024 + (size_t)XS * BN * 128 + (size_t)WS * BM * 32 +
-             (size_t)BM * max_groups * 2 + 16 + (2 * WS + 2 * XS + 2 * AB + 2) * 8 + 16;
+  size_t b = 1024 + (size_t)XS * BN * 128 + (2 * XS + 2 * AB + 2) * 8 + 16;
   return b < kMinSmem ? kMinSmem : b;
 }
 
 template <int BN>
 tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
-  CUtensorMap mx, mw0, mw1;
+  CUtensorMap mx;
   TL_TRY(encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.x, g.K, g.T, (uint64_t)g.K * 2, BK, BN,
                    CU_TENSOR_MAP_SWIZZLE_128B));
-  const int n1 = g.n_split, n2 = g.N - g.n_split;
-  const int box_rows = g.swiglu_u ? BM / 2 : BM;   // fused SwiGLU: 64 gate + 64 up rows
-  TL_TRY(encode_2d(&mw0, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w0, g.K / 8, n1, (uint64_t)g.K / 8 * 4,
-                   BK / 8, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE));
-  if (n2 > 0) {
-    TL_TRY(encode_2d(&mw1, CU_TENSOR_MAP_DATA_TYPE_UINT32, g.w1, g.K / 8, n2,
-                     (uint64_t)g.K / 8 * 4, BK / 8, box_rows, CU_TENSOR_MAP_SWIZZLE_NONE));
-  } else {
-    mw1 = mw0;
-  }
   TcArgs a;
   a.N = g.N;
   a.K = g.K;
@@ -605,22 +581,18 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.T = g.T;
   a.n_split = g.n_split;
   a.splits = g.splits;
-  {
-    // largest number of scale groups any split touches (+1 for an unaligned start)
-    const int nkb = g.K / BK;
-    const int per = (nkb + g.splits - 1) / g.splits;
-    a.max_groups = (per * BK + g.G - 1) / g.G + 1;
-  }
+  a.w0 = g.w0;
+  a.w1 = g.w1;
   a.s0 = g.s0;
   a.s1 = g.s1;
   a.part = g.part;
   a.status = g.status;
   a.swiglu_u = g.swiglu_u;
-  const size_t smem = tc_smem_bytes<BN>(a.max_groups);
+  const size_t smem = tc_smem_bytes<BN>();
   if (smem > 232448)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs %zu bytes of shared memory", smem);
   dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
-  TL_LAUNCH_PDL(gemm_w4_tc_kernel<BN>, grid, THREADS, smem, s, mx, mw0, mw1, a);
+  TL_LAUNCH_PDL(gemm_w4_tc_kernel<BN>, grid, THREADS, smem, s, mx, a);
   return ok();
 }
 
