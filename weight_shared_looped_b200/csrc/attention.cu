@@ -506,25 +506,42 @@ __device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
   return v;
 }
 
+// Four int8 codes of a word to float, exactly: each biased byte goes into the
+// low mantissa bits of 2^23 (prmt with the constant's upper bytes), then the
+// bias 2^23 + 128 is subtracted.
+__device__ __forceinline__ void int8x4_to_float(uint32_t w, float* f) {
+  const uint32_t u = w ^ 0x80808080u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t b;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(b) : "r"(u), "r"(0x4B000000u), "r"(0x7650u | (uint32_t)i));
+    f[i] = __uint_as_float(b) - 8388736.0f;
+  }
+}
+
+constexpr int DS_KEYS = 64;     // keys per stage of the streaming decode kernel
+constexpr int DS_STAGES = 3;    // stages in flight (cp.async ring)
+
 template <int HD>
 __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs a, int CL,
                                                                   int max_per) {
   constexpr int HALF = HD / 2;
-  constexpr int KSPLIT = 128 / HD;              // key slices in the P V step
+  constexpr int KSPLIT = 128 / HD;              // key slices in the P V step (1 or 2)
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ float qs[HD], kn[HD], vn[HD];
   __shared__ float acc_s[KSPLIT][HD];
+  __shared__ float pw[DS_KEYS];                  // weights of the current stage's keys
   __shared__ float stat_s[2];                    // this CTA's max score and exponential sum
   __shared__ float red[4];
   const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int esz = a.kv_int8 ? 1 : 2;
   const int rowb = HD * esz;
-  unsigned char* kst = dsm;                                          // [max_per][rowb]
-  unsigned char* vst = dsm + (size_t)max_per * rowb;                 // [max_per][rowb]
-  float* ksc = reinterpret_cast<float*>(dsm + 2 * (size_t)max_per * rowb);
+  const int stage_bytes = DS_KEYS * rowb;
+  unsigned char* kst = dsm;                                        // [DS_STAGES][DS_KEYS][rowb]
+  unsigned char* vst = dsm + (size_t)DS_STAGES * stage_bytes;      // [DS_STAGES][DS_KEYS][rowb]
+  float* ksc = reinterpret_cast<float*>(dsm + 2 * (size_t)DS_STAGES * stage_bytes);   // [max_per]
   float* vsc = ksc + max_per;
-  float* pr = vsc + max_per;                                         // scores, then weights
   // positions, the lane map, the RoPE table and the cached rows before pos
   // were written by earlier steps
   const int lane_id = a.lane_of_row[row];
@@ -535,29 +552,37 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
   const int nk = k1 - k0;
   const bool owner = nk > 0 && k1 == n_keys;     // holds position pos
   const int n_old = owner ? nk - 1 : nk;
+  const int nsub = (nk + DS_KEYS - 1) / DS_KEYS;
   char* layer = const_cast<char*>(a.kv_base) +
                 (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
   const size_t head_off = (size_t)head * a.max_ctx;
   const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
-  {
-    const int pieces = rowb / 16;
-    for (int which = 0; which < 2; ++which) {
-      const char* src = layer + which * a.kv_region_bytes + (head_off + k0) * rowb;
-      unsigned char* dst = which ? vst : kst;
-      for (int i = tid; i < n_old * pieces; i += 128) {
-        const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i * 16);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + i * 16)
-                     : "memory");
+  // copy the cached rows of stage `sub` into ring slot sub % DS_STAGES (one
+  // commit group per stage, empty past the end)
+  auto issue = [&](int sub) {
+    if (sub < nsub) {
+      const int lo = sub * DS_KEYS, cnt = min(DS_KEYS, n_old - lo);
+      const int pieces = rowb / 16;
+      for (int which = 0; which < 2; ++which) {
+        const char* src = layer + which * a.kv_region_bytes + (head_off + k0 + lo) * rowb;
+        unsigned char* dst = (which ? vst : kst) + (size_t)(sub % DS_STAGES) * stage_bytes;
+        for (int i = tid; i < cnt * pieces; i += 128) {
+          const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i * 16);
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + i * 16)
+                       : "memory");
+        }
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    if (a.kv_int8) {
-      const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
-      const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
-      for (int j = tid; j < n_old; j += 128) {
-        ksc[j] = __half2float(kq[head_off + k0 + j]);
-        vsc[j] = __half2float(vq[head_off + k0 + j]);
-      }
+  };
+#pragma unroll
+  for (int st = 0; st < DS_STAGES - 1; ++st) issue(st);
+  if (a.kv_int8) {
+    const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
+    const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
+    for (int j = tid; j < n_old; j += 128) {
+      ksc[j] = __half2float(kq[head_off + k0 + j]);
+      vsc[j] = __half2float(vq[head_off + k0 + j]);
     }
   }
   float2 cs = make_float2(1.f, 0.f);
@@ -608,26 +633,25 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
   __syncthreads();
   // the query is rounded to fp16 as in the prefill path
   if (tid < HD) qs[tid] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
-
+  // owner: the new entry (position pos = key nk - 1 of this CTA) is appended
+  // to the cache now and copied into its stage slot when that stage is read
+  uint32_t k_new = 0, v_new = 0;     // fp16 bits or int8 code of element tid
   if (owner) {
-    // append k (after RoPE) and v at position pos, in the cache and in the
-    // staged rows
-    const int jr = nk - 1;
     const __half kh = __float2half_rn(kr);
     const __half vh = __float2half_rn(tid < HD ? vn[tid] : 0.f);
     if (!a.kv_int8) {
       if (tid < HD) {
         reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + tid] = kh;
         reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = vh;
-        reinterpret_cast<__half*>(kst)[jr * HD + tid] = kh;
-        reinterpret_cast<__half*>(vst)[jr * HD + tid] = vh;
+        k_new = __half_as_ushort(kh);
+        v_new = __half_as_ushort(vh);
       }
     } else {
-      __shared__ float kmax_s[4], vmax_s[4];
       float km = tid < HD ? fabsf(__half2float(kh)) : 0.f;
       float vm = tid < HD ? fabsf(__half2float(vh)) : 0.f;
       km = warp_max(km);
       vm = warp_max(vm);
+      __shared__ float kmax_s[4], vmax_s[4];
       if (lane == 0) {
         kmax_s[warp] = km;
         vmax_s[warp] = vm;
@@ -644,95 +668,159 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
         const int vc = vsf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vsf)), -127.f), 127.f);
         reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + tid] = (int8_t)kc;
         reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = (int8_t)vc;
-        reinterpret_cast<int8_t*>(kst)[jr * HD + tid] = (int8_t)kc;
-        reinterpret_cast<int8_t*>(vst)[jr * HD + tid] = (int8_t)vc;
+        k_new = (uint32_t)(uint8_t)(int8_t)kc;
+        v_new = (uint32_t)(uint8_t)(int8_t)vc;
       }
       if (tid == 0) {
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] = vsh;
-        ksc[jr] = ksf;
-        vsc[jr] = vsf;
+        ksc[nk - 1] = ksf;
+        vsc[nk - 1] = vsf;
       }
     }
   }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();   // staged rows, the appended entry and q are visible to the whole CTA
 
-  // scores: one key per thread, four partial dot products
-  float lmax = -INFINITY;
-  for (int j = tid; j < nk; j += 128) {
-    float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-    if (!a.kv_int8) {
-      const uint4* src = reinterpret_cast<const uint4*>(kst + (size_t)j * rowb);
+  // streaming online softmax over the stages
+  constexpr int QD = HD / 4;                     // head_dim quarter of a score thread
+  constexpr int G4 = HD / 4, KS4 = 128 / G4;     // P V: 4-dim groups x key slices
+  __syncthreads();                               // qs final
+  const int qq = tid & 3;                        // this thread's quarter of head_dim
+  float qreg[QD];
 #pragma unroll
-      for (int c = 0; c < HD / 8; ++c) {
-        const uint4 w = src[c];
-        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
-        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
-        const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w.z));
-        const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&w.w));
-        d0 = fmaf(qs[c * 8 + 0], f0.x, fmaf(qs[c * 8 + 1], f0.y, d0));
-        d1 = fmaf(qs[c * 8 + 2], f1.x, fmaf(qs[c * 8 + 3], f1.y, d1));
-        d2 = fmaf(qs[c * 8 + 4], f2.x, fmaf(qs[c * 8 + 5], f2.y, d2));
-        d3 = fmaf(qs[c * 8 + 6], f3.x, fmaf(qs[c * 8 + 7], f3.y, d3));
+  for (int d = 0; d < QD; ++d) qreg[d] = qs[qq * QD + d];
+  float m = -INFINITY, l = 0.f;
+  float acc4[4] = {0.f, 0.f, 0.f, 0.f};          // dims 4g..4g+3 over key slice ks
+  const int g4 = tid % G4, ks4 = tid / G4;
+  for (int sub = 0; sub < nsub; ++sub) {
+    issue(sub + DS_STAGES - 1);                  // its slot was freed at the end of the last stage
+    asm volatile("cp.async.wait_group %0;" ::"n"(DS_STAGES - 1) : "memory");
+    const int slot = sub % DS_STAGES;
+    unsigned char* ks_ = kst + (size_t)slot * stage_bytes;
+    unsigned char* vs_ = vst + (size_t)slot * stage_bytes;
+    const int base = sub * DS_KEYS;
+    const int cnt = min(DS_KEYS, nk - base);
+    if (owner && nk - 1 - base >= 0 && nk - 1 - base < DS_KEYS && tid < HD) {
+      const int r = nk - 1 - base;
+      if (!a.kv_int8) {
+        reinterpret_cast<unsigned short*>(ks_)[r * HD + tid] = (unsigned short)k_new;
+        reinterpret_cast<unsigned short*>(vs_)[r * HD + tid] = (unsigned short)v_new;
+      } else {
+        ks_[r * HD + tid] = (unsigned char)k_new;
+        vs_[r * HD + tid] = (unsigned char)v_new;
       }
-    } else {
-      const uint4* src = reinterpret_cast<const uint4*>(kst + (size_t)j * rowb);
+    }
+    __syncthreads();   // the stage's rows (and the appended entry) are visible
+    // scores: four threads per key (one head_dim quarter each), q in registers
+    float sc[DS_KEYS / 32];
 #pragma unroll
-      for (int c = 0; c < HD / 16; ++c) {
-        const uint4 w = src[c];
-        const int8_t* b = reinterpret_cast<const int8_t*>(&w);
+    for (int ps = 0; ps < DS_KEYS / 32; ++ps) {
+      const int j = ps * 32 + (tid >> 2);
+      float d0 = 0.f, d1 = 0.f;
+      if (j < cnt) {
+        if (!a.kv_int8) {
+          const uint4* src = reinterpret_cast<const uint4*>(ks_ + (size_t)j * rowb + qq * QD * 2);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          d0 = fmaf(qs[c * 16 + e], (float)b[e], d0);
-          d1 = fmaf(qs[c * 16 + 4 + e], (float)b[4 + e], d1);
-          d2 = fmaf(qs[c * 16 + 8 + e], (float)b[8 + e], d2);
-          d3 = fmaf(qs[c * 16 + 12 + e], (float)b[12 + e], d3);
+          for (int c = 0; c < QD / 8; ++c) {
+            const uint4 w = src[c];
+            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
+            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
+            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w.z));
+            const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&w.w));
+            d0 = fmaf(qreg[c * 8 + 0], f0.x, fmaf(qreg[c * 8 + 1], f0.y, d0));
+            d1 = fmaf(qreg[c * 8 + 2], f1.x, fmaf(qreg[c * 8 + 3], f1.y, d1));
+            d0 = fmaf(qreg[c * 8 + 4], f2.x, fmaf(qreg[c * 8 + 5], f2.y, d0));
+            d1 = fmaf(qreg[c * 8 + 6], f3.x, fmaf(qreg[c * 8 + 7], f3.y, d1));
+          }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(ks_ + (size_t)j * rowb + qq * QD);
+#pragma unroll
+          for (int c = 0; c < QD / 16; ++c) {
+            const uint4 w = src[c];
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float f[4];
+              int8x4_to_float(ww[e], f);
+              d0 = fmaf(qreg[c * 16 + 4 * e + 0], f[0], d0);
+              d1 = fmaf(qreg[c * 16 + 4 * e + 1], f[1], d1);
+              d0 = fmaf(qreg[c * 16 + 4 * e + 2], f[2], d0);
+              d1 = fmaf(qreg[c * 16 + 4 * e + 3], f[3], d1);
+            }
+          }
         }
       }
+      float sj = d0 + d1;
+      sj += __shfl_xor_sync(0xffffffffu, sj, 1);
+      sj += __shfl_xor_sync(0xffffffffu, sj, 2);
+      sc[ps] = j < cnt ? (a.kv_int8 ? sj * ksc[base + j] : sj) : -INFINITY;
     }
-    float sc = (d0 + d1) + (d2 + d3);
-    if (a.kv_int8) sc *= ksc[j];
-    pr[j] = sc;
-    lmax = fmaxf(lmax, sc);
+    // stage max, new running max, weights
+    float smax = sc[0];
+#pragma unroll
+    for (int ps = 1; ps < DS_KEYS / 32; ++ps) smax = fmaxf(smax, sc[ps]);
+    smax = warp_max(smax);
+    if (lane == 0) red[warp] = smax;
+    __syncthreads();
+    smax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    const float m_new = fmaxf(m, smax);
+    const float alpha = m == -INFINITY ? 0.f : __expf(m - m_new);
+    float psum = 0.f;
+#pragma unroll
+    for (int ps = 0; ps < DS_KEYS / 32; ++ps) {
+      const int j = ps * 32 + (tid >> 2);
+      const float pj = j < cnt ? __expf(sc[ps] - m_new) : 0.f;
+      if (qq == 0) {
+        pw[j] = a.kv_int8 ? pj * (j < cnt ? vsc[base + j] : 0.f) : pj;   // INT8: V scale folded in
+        psum += pj;
+      }
+    }
+    psum = warp_sum(psum);
+    __syncthreads();   // pw visible; red free again
+    if (lane == 0) red[warp] = psum;
+    // P V: thread (g4, ks4) takes dims 4*g4 .. 4*g4+3 over keys ks4, ks4 + KS4, ...
+    {
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (!a.kv_int8) {
+        for (int j = ks4; j < cnt; j += KS4) {
+          const float w = pw[j];
+          const uint2 v = *reinterpret_cast<const uint2*>(vs_ + (size_t)j * rowb + g4 * 8);
+          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+          s4[0] = fmaf(w, f0.x, s4[0]);
+          s4[1] = fmaf(w, f0.y, s4[1]);
+          s4[2] = fmaf(w, f1.x, s4[2]);
+          s4[3] = fmaf(w, f1.y, s4[3]);
+        }
+      } else {
+        for (int j = ks4; j < cnt; j += KS4) {
+          const float w = pw[j];
+          float f[4];
+          int8x4_to_float(*reinterpret_cast<const uint32_t*>(vs_ + (size_t)j * rowb + g4 * 4), f);
+          s4[0] = fmaf(w, f[0], s4[0]);
+          s4[1] = fmaf(w, f[1], s4[1]);
+          s4[2] = fmaf(w, f[2], s4[2]);
+          s4[3] = fmaf(w, f[3], s4[3]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc4[c] = fmaf(acc4[c], alpha, s4[c]);
+    }
+    __syncthreads();   // red (sums) visible; the stage slot and pw may be reused
+    l = fmaf(l, alpha, (red[0] + red[1]) + (red[2] + red[3]));
+    m = m_new;
   }
-  lmax = warp_max(lmax);
-  if (lane == 0) red[warp] = lmax;
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  // combine the key slices in slice order: dims of slice 0 first, then add
+  __shared__ float sl_s[KS4][HD];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) sl_s[ks4][4 * g4 + c] = acc4[c];
   __syncthreads();
-  const float m = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();   // red is reused below
-  float lsum = 0.f;
-  for (int j = tid; j < nk; j += 128) {
-    const float e = __expf(pr[j] - m);
-    lsum += e;
-    pr[j] = a.kv_int8 ? e * vsc[j] : e;   // INT8: fold the V scale into the weight
+  float acc = 0.f;
+  if (tid < HD) {
+#pragma unroll
+    for (int q = 0; q < KS4; ++q) acc += sl_s[q][tid];
   }
-  lsum = warp_sum(lsum);
-  if (lane == 0) red[warp] = lsum;
-  __syncthreads();   // weights and partial sums visible
-  const float l = (red[0] + red[1]) + (red[2] + red[3]);
-  // P V: thread (e, ks) takes dimension e over keys j = ks, ks + KSPLIT, ...
-  {
-    const int e = tid % HD, ks = tid / HD;
-    float acc0 = 0.f, acc1 = 0.f;
-    int j = ks;
-    if (!a.kv_int8) {
-      const __half* src = reinterpret_cast<const __half*>(vst) + e;
-      for (; j + KSPLIT < nk; j += 2 * KSPLIT) {
-        acc0 = fmaf(pr[j], __half2float(src[(size_t)j * HD]), acc0);
-        acc1 = fmaf(pr[j + KSPLIT], __half2float(src[(size_t)(j + KSPLIT) * HD]), acc1);
-      }
-      if (j < nk) acc0 = fmaf(pr[j], __half2float(src[(size_t)j * HD]), acc0);
-    } else {
-      const int8_t* src = reinterpret_cast<const int8_t*>(vst) + e;
-      for (; j + KSPLIT < nk; j += 2 * KSPLIT) {
-        acc0 = fmaf(pr[j], (float)src[(size_t)j * HD], acc0);
-        acc1 = fmaf(pr[j + KSPLIT], (float)src[(size_t)(j + KSPLIT) * HD], acc1);
-      }
-      if (j < nk) acc0 = fmaf(pr[j], (float)src[(size_t)j * HD], acc0);
-    }
-    acc_s[ks][e] = acc0 + acc1;
-  }
+  if (tid < HD) acc_s[0][tid] = acc;
   if (tid == 0) {
     stat_s[0] = nk > 0 ? m : -INFINITY;
     stat_s[1] = nk > 0 ? l : 0.f;
@@ -747,10 +835,7 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
         const float mr = cl_ld(&stat_s[0], (uint32_t)r);
         const float w = mr == -INFINITY ? 0.f : __expf(mr - M);
         L = fmaf(cl_ld(&stat_s[1], (uint32_t)r), w, L);
-        float pv = 0.f;
-#pragma unroll
-        for (int q = 0; q < KSPLIT; ++q) pv += cl_ld(&acc_s[q][e], (uint32_t)r);
-        o = fmaf(pv, w, o);
+        o = fmaf(cl_ld(&acc_s[0][e], (uint32_t)r), w, o);
       }
       a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
     }
@@ -784,7 +869,7 @@ static size_t decode_cluster_smem(int max_ctx, int hd, bool int8, int* max_per) 
   const int cl = decode_cluster_size(max_ctx);
   *max_per = (max_ctx + cl - 1) / cl;
   const size_t rowb = (size_t)hd * (int8 ? 1 : 2);
-  return 2 * (size_t)*max_per * rowb + 3 * (size_t)*max_per * sizeof(float);
+  return 2 * (size_t)DS_STAGES * DS_KEYS * rowb + 2 * (size_t)*max_per * sizeof(float);
 }
 
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
