@@ -107,12 +107,9 @@ struct tl_model {
   __half* u;
   float* part;
   float* part2;          // decode: gate|up partials read by the down projection
-  int* attn_counters;    // decode: merge tickets [kMaxLanes][H], zero between launches
   int* gemv_tickets;     // decode: residual-add tickets per 128-row block, zero between launches
   float* y;
   int32_t* lane_map;
-  float* dec_scratch;
-  int max_chunks;
   int* status;
   float2* rope;
   std::map<std::string, GraphEntry> graphs_cache;
@@ -322,7 +319,6 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->F = ld.ffn;
   m->eps = ld.eps;
   m->Tmax = std::max(md.max_tokens, md.max_lanes);
-  m->max_chunks = (md.max_ctx + kDecodeChunk - 1) / kDecodeChunk;
   const int T = m->Tmax, d = m->d, F = m->F;
   size_t maxpart = 0;
   for (int t = 1; t <= T; ++t) maxpart = std::max(maxpart, part_floats(m.get(), t));
@@ -332,8 +328,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
     size_t bytes;
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
-  void* p_u; void* p_part; void* p_y; void* p_lid; void* p_dec; void* p_status; void* p_rope;
-  void* p_part2; void* p_ctr; void* p_gtk;
+  void* p_u; void* p_part; void* p_y; void* p_lid; void* p_status; void* p_rope;
+  void* p_part2; void* p_gtk;
   size_t part2_floats = 0;
   for (int t = 1; t <= md.max_lanes; ++t)
     part2_floats = std::max(part2_floats, (size_t)gemm_splits(2 * F, d, t) * t * 2 * F);
@@ -349,11 +345,9 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_u, (size_t)T * F * 2},
       {&p_part, maxpart * 4},
       {&p_part2, part2_floats * 4},
-      {&p_ctr, (size_t)kMaxLanes * m->H * 4},
       {&p_gtk, (size_t)1024 * 4},
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
-      {&p_dec, (size_t)kMaxLanes * m->H * m->max_chunks * (m->hd + 2) * 4},
       {&p_status, 256},
       {&p_rope, (size_t)md.max_ctx * (m->hd / 2) * sizeof(float2)},
   };
@@ -378,11 +372,9 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->u = (__half*)p_u;
   m->part = (float*)p_part;
   m->part2 = (float*)p_part2;
-  m->attn_counters = (int*)p_ctr;
   m->gemv_tickets = (int*)p_gtk;
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
-  m->dec_scratch = (float*)p_dec;
   m->status = (int*)p_status;
   m->rope = (float2*)p_rope;
   // RoPE table: angle = pos * theta^(-2i/hd), computed in double, rounded to fp32
@@ -401,7 +393,6 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
                                 cudaMemcpyHostToDevice);
     cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
-    if (e3 == cudaSuccess) e3 = cudaMemset(m->attn_counters, 0, (size_t)kMaxLanes * m->H * 4);
     if (e3 == cudaSuccess) e3 = cudaMemset(m->gemv_tickets, 0, (size_t)1024 * 4);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
@@ -694,12 +685,9 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     da.max_ctx = kv->max_ctx;
     da.kv_int8 = kv->dtype == TL_KV_INT8;
     da.lane_of_row = lane_of_row;
-    da.scratch = m->dec_scratch;
-    da.max_chunks = (kv->max_ctx + kDecodeChunk - 1) / kDecodeChunk;
     da.qkv_part = m->part;
     da.qkv_S = g.splits;
     da.rope_cs = m->rope;
-    da.counters = m->attn_counters;
     TL_TRY(launch_attn_decode_fused(da, s));
   }
   // O projection, residual, RMSNorm before the MLP (decode: the GEMV's last

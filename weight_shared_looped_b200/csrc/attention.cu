@@ -7,9 +7,10 @@
 // Decode: one query per (lane, head) against the lane's cached keys 0..pos,
 // FP16 or INT8 (code * fp16 scale) ("Production Roadmap", Stage 2: keep the
 // direct cached single-query path for decode; "Performance and Memory", "KV
-// cache INT8").  The context is split into fixed 64-key chunks (a function of
-// the position only) whose partial results are merged in chunk order, so a
-// lane's output does not depend on the other lanes.
+// cache INT8").  The context is split over the CTAs of a thread-block cluster
+// by a rule that depends only on the lane's position and the cache size, and
+// the partial results are merged in a fixed order, so a lane's output does not
+// depend on the other lanes.
 #include "tl_launch.cuh"
 
 namespace tl {
@@ -200,287 +201,6 @@ __global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __re
       *reinterpret_cast<uint32_t*>(out + (size_t)r0 * d + c) = pack_half2(o[nt][0] * i0, o[nt][1] * i0);
     if (r1 < T)
       *reinterpret_cast<uint32_t*>(out + (size_t)r1 * d + c) = pack_half2(o[nt][2] * i1, o[nt][3] * i1);
-  }
-}
-
-// ------------------------------------------------------------------ decode
-// Fused decode attention for one (row, head, 64-key chunk):
-//   * q = sum of the QKV split-K partials, RoPE at the lane's position;
-//   * the CTA holding the lane's newest position also forms k and v, applies
-//     RoPE to k and appends both to the cache (fp16, or INT8 codes + fp16 scale
-//     per (token, head)); positions before it are only read;
-//   * scores, max-subtracted exponentials and the weighted V sum of the chunk
-//     go to scratch; the last CTA of the (row, head) to finish (an atomic
-//     ticket, no waiting) merges all chunks in chunk order and writes the
-//     output, then resets the ticket for the next launch.
-template <int HD>
-__global__ void __launch_bounds__(128) attn_decode_fused_kernel(DecodeAttnArgs a) {
-  constexpr int DPL = HD / 32;
-  constexpr int HALF = HD / 2;
-  constexpr int ROWB = HD * 2;                 // bytes of one fp16 row (int8 rows use half)
-  __shared__ __align__(16) unsigned char kv_s[2][kDecodeChunk * ROWB];   // staged K, V rows
-  __shared__ float ks_s[kDecodeChunk], vs_s[kDecodeChunk];                // INT8 scales
-  __shared__ float qs[HD], kn[HD], vn[HD];
-  __shared__ float sc[kDecodeChunk];
-  __shared__ float wacc[4][HD > kDecodeChunk ? HD : kDecodeChunk];
-  __shared__ float wl[4];
-  __shared__ float red[4];
-  __shared__ int is_last;
-  (void)DPL;
-  const int chunk = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
-  // Positions, the lane map, the RoPE table and the cache rows before the
-  // newest position were all written by earlier steps: read them (and start
-  // copying this chunk's K/V rows into shared memory) before waiting for the
-  // QKV projection that produces this token's q, k and v.
-  const int lane_id = a.lane_of_row[row];
-  const int pos = a.hdr->pos[lane_id];
-  const int n_keys = pos + 1;
-  const int n_chunks = (n_keys + kDecodeChunk - 1) / kDecodeChunk;
-  if (chunk >= n_chunks) {
-    pdl_enter();
-    return;
-  }
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool owner = chunk == n_chunks - 1;    // holds position pos
-  const int base = chunk * kDecodeChunk;
-  const int nk = min(kDecodeChunk, n_keys - base);          // keys in this chunk
-  const int n_old = owner ? nk - 1 : nk;                    // rows already in the cache
-  char* layer = const_cast<char*>(a.kv_base) +
-                (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
-  const size_t head_off = (size_t)head * a.max_ctx;
-  const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
-  const int esz = a.kv_int8 ? 1 : 2;
-  {
-    const int chunks16 = HD * esz / 16;                      // 16-byte pieces per row
-    for (int which = 0; which < 2; ++which) {
-      const char* src = layer + which * a.kv_region_bytes + (head_off + base) * HD * esz;
-      for (int i = threadIdx.x; i < n_old * chunks16; i += 128) {
-        const uint32_t dst = (uint32_t)__cvta_generic_to_shared(kv_s[which] + i * 16);
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + i * 16)
-                     : "memory");
-      }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    if (a.kv_int8 && threadIdx.x < n_old) {
-      const __half* ksc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
-      const __half* vsc = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
-      ks_s[threadIdx.x] = __half2float(ksc[head_off + base + threadIdx.x]);
-      vs_s[threadIdx.x] = __half2float(vsc[head_off + base + threadIdx.x]);
-    }
-  }
-  const int i = threadIdx.x;
-  float2 cs = make_float2(1.f, 0.f);
-  if (i < HD) cs = a.rope_cs[(size_t)pos * HALF + (i % HALF)];
-  pdl_enter();
-
-  // q (and k, v for the owner) from the QKV partial sums, all splits in flight
-  const size_t split_stride = (size_t)a.rows * 3 * a.d;
-  const float* prow = a.qkv_part + (size_t)row * 3 * a.d + (size_t)head * HD;
-  if (i < HD) {
-    float pq[8], pk[8], pv[8];
-    float sq = 0.f, sk = 0.f, sv = 0.f;
-    for (int s0 = 0; s0 < a.qkv_S; s0 += 8) {
-      const int cnt = min(8, a.qkv_S - s0);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < cnt) {
-          const float* p = prow + (size_t)(s0 + j) * split_stride;
-          pq[j] = p[i];
-          pk[j] = owner ? p[a.d + i] : 0.f;
-          pv[j] = owner ? p[2 * a.d + i] : 0.f;
-        }
-      }
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j < cnt) {
-          sq += pq[j];
-          sk += pk[j];
-          sv += pv[j];
-        }
-      }
-    }
-    qs[i] = sq;
-    kn[i] = sk;
-    vn[i] = sv;
-  }
-  __syncthreads();
-  float qr = 0.f, kr = 0.f;
-  if (i < HD) {
-    if (i < HALF) {
-      qr = qs[i] * cs.x - qs[i + HALF] * cs.y;
-      kr = kn[i] * cs.x - kn[i + HALF] * cs.y;
-    } else {
-      qr = qs[i] * cs.x + qs[i - HALF] * cs.y;
-      kr = kn[i] * cs.x + kn[i - HALF] * cs.y;
-    }
-  }
-  __syncthreads();
-  if (i < HD) {
-    // the query is rounded to fp16 as in the unfused path
-    qs[i] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
-  }
-  if (owner) {
-    // append k (after RoPE) and v at position pos, in the cache and in the
-    // staged rows
-    const int jr = nk - 1;
-    const __half kh = __float2half_rn(kr);
-    const __half vh = __float2half_rn(i < HD ? vn[i] : 0.f);
-    if (!a.kv_int8) {
-      if (i < HD) {
-        reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + i] = kh;
-        reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = vh;
-        reinterpret_cast<__half*>(kv_s[0])[jr * HD + i] = kh;
-        reinterpret_cast<__half*>(kv_s[1])[jr * HD + i] = vh;
-      }
-    } else {
-      float km = i < HD ? fabsf(__half2float(kh)) : 0.f;
-      float vm = i < HD ? fabsf(__half2float(vh)) : 0.f;
-      km = warp_max(km);
-      vm = warp_max(vm);
-      if (lane == 0) {
-        red[warp] = km;
-        wl[warp] = vm;
-      }
-      __syncthreads();
-      km = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-      vm = fmaxf(fmaxf(wl[0], wl[1]), fmaxf(wl[2], wl[3]));
-      const __half ksh = __float2half_rn(__fdiv_rn(km, 127.0f));
-      const __half vsh = __float2half_rn(__fdiv_rn(vm, 127.0f));
-      const float ksf = __half2float(ksh), vsf = __half2float(vsh);
-      if (i < HD) {
-        const float kx = __half2float(kh), vx = __half2float(vh);
-        const int kc = ksf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ksf)), -127.f), 127.f);
-        const int vc = vsf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vsf)), -127.f), 127.f);
-        reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + i] = (int8_t)kc;
-        reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + i] = (int8_t)vc;
-        reinterpret_cast<int8_t*>(kv_s[0])[jr * HD + i] = (int8_t)kc;
-        reinterpret_cast<int8_t*>(kv_s[1])[jr * HD + i] = (int8_t)vc;
-      }
-      if (i == 0) {
-        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
-        reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] =
-            vsh;
-        ks_s[jr] = ksf;
-        vs_s[jr] = vsf;
-      }
-    }
-  }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();   // staged rows, the appended entry and qs are visible to the whole CTA
-
-  // scores: thread (j, half) takes key base + j over one half of head_dim
-  {
-    const int j = threadIdx.x % kDecodeChunk, hf = threadIdx.x / kDecodeChunk;
-    float dot = 0.f;
-    if (j < nk) {
-      const int d0 = hf * HALF;
-      if (!a.kv_int8) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const __half*>(kv_s[0]) + j * HD + d0);
-#pragma unroll
-        for (int c = 0; c < HALF / 8; ++c) {
-          const uint4 w = src[c];
-          const __half2* hp = reinterpret_cast<const __half2*>(&w);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __half22float2(hp[e]);
-            dot = fmaf(qs[d0 + c * 8 + 2 * e], f.x, dot);
-            dot = fmaf(qs[d0 + c * 8 + 2 * e + 1], f.y, dot);
-          }
-        }
-      } else {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const int8_t*>(kv_s[0]) + j * HD + d0);
-        float part = 0.f;
-#pragma unroll
-        for (int c = 0; c < HALF / 16; ++c) {
-          const uint4 w = src[c];
-          const int8_t* bp = reinterpret_cast<const int8_t*>(&w);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) part = fmaf(qs[d0 + c * 16 + e], (float)bp[e], part);
-        }
-        dot = part * ks_s[j];
-      }
-    }
-    wacc[hf][j] = dot;
-  }
-  __syncthreads();
-  if (threadIdx.x < kDecodeChunk)
-    sc[threadIdx.x] = threadIdx.x < nk ? wacc[0][threadIdx.x] + wacc[1][threadIdx.x] : -INFINITY;
-  __syncthreads();
-  float m = -INFINITY;
-  for (int j = 0; j < kDecodeChunk; ++j) m = fmaxf(m, sc[j]);
-  __syncthreads();
-  if (threadIdx.x < kDecodeChunk) {
-    const int j = threadIdx.x;
-    sc[j] = j < nk ? __expf(sc[j] - m) : 0.f;
-    if (a.kv_int8) wacc[3][j] = j < nk ? vs_s[j] : 0.f;
-  }
-  __syncthreads();
-  // P V: thread (e, ks) takes dimension e over key slice ks
-  constexpr int KSPLIT = 128 / HD;
-  constexpr int KPER = kDecodeChunk / KSPLIT;
-  {
-    const int e = threadIdx.x % HD, ks = threadIdx.x / HD;
-    float acc = 0.f;
-    const int j0 = ks * KPER;
-    if (!a.kv_int8) {
-      const __half* src = reinterpret_cast<const __half*>(kv_s[1]) + e;
-#pragma unroll 8
-      for (int jj = 0; jj < KPER; ++jj) {
-        const int j = j0 + jj;
-        if (j < nk) acc = fmaf(sc[j], __half2float(src[j * HD]), acc);
-      }
-    } else {
-      const int8_t* src = reinterpret_cast<const int8_t*>(kv_s[1]) + e;
-#pragma unroll 8
-      for (int jj = 0; jj < KPER; ++jj) {
-        const int j = j0 + jj;
-        if (j < nk) acc = fmaf(sc[j] * wacc[3][j], (float)src[j * HD], acc);
-      }
-    }
-    wacc[ks][e] = acc;     // (scores in wacc[0..1] are no longer needed)
-  }
-  if (threadIdx.x < 32) {
-    float l = sc[threadIdx.x] + sc[threadIdx.x + 32];
-    l = warp_sum(l);
-    if (threadIdx.x == 0) wl[0] = l;
-  }
-  __syncthreads();
-  float* part = a.scratch + ((size_t)row * a.H + head) * a.max_chunks * (HD + 2);
-  float* dst = part + (size_t)chunk * (HD + 2);
-  for (int e = threadIdx.x; e < HD; e += 128) {
-    float o = wacc[0][e];
-    if (KSPLIT > 1) o += wacc[1][e];
-    dst[e] = o;
-  }
-  if (threadIdx.x == 0) {
-    dst[HD] = m;
-    dst[HD + 1] = wl[0];
-  }
-  // last CTA of this (row, head) merges
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int* ctr = a.counters + (size_t)lane_id * a.H + head;
-    const int ticket = atomicAdd(ctr, 1);
-    is_last = ticket == n_chunks - 1;
-    if (is_last) *ctr = 0;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  float M = -INFINITY;
-  for (int c = 0; c < n_chunks; ++c) M = fmaxf(M, __ldcg(part + (size_t)c * (HD + 2) + HD));
-  for (int e = threadIdx.x; e < HD; e += 128) {
-    float L = 0.f, o = 0.f;
-    for (int c = 0; c < n_chunks; ++c) {
-      const float* pc = part + (size_t)c * (HD + 2);
-      const float w = __expf(__ldcg(pc + HD) - M);
-      L = fmaf(__ldcg(pc + HD + 1), w, L);
-      o = fmaf(__ldcg(pc + e), w, o);
-    }
-    a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
   }
 }
 
@@ -878,30 +598,23 @@ tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
   int max_per = 0;
   const size_t smem = decode_cluster_smem(a.max_ctx, a.hd, a.kv_int8 != 0, &max_per);
-  if (smem + 8 * 1024 <= 227 * 1024) {
-    static bool attr_done = false;
-    if (!attr_done) {
-      TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<128>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-      TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<64>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-      attr_done = true;
-    }
-    const int cl = decode_cluster_size(a.max_ctx);
-    dim3 grid(cl, a.H, a.rows);
-    cudaError_t e = a.hd == 128
-        ? launch_pdl_cluster(attn_decode_cluster_kernel<128>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per)
-        : launch_pdl_cluster(attn_decode_cluster_kernel<64>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per);
-    if (e != cudaSuccess)
-      return set_error(TL_ERR_CUDA, "launch of attn_decode_cluster_kernel failed: %s", cudaGetErrorString(e));
-    return ok();
+  if (smem > 200 * 1024)
+    return set_error(TL_ERR_UNSUPPORTED, "decode attention: %zu bytes of shared memory", smem);
+  static bool attr_done = false;
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    attr_done = true;
   }
-  // long caches: 64-key chunks merged by the last CTA of each (row, head)
-  dim3 grid(a.max_chunks, a.H, a.rows);
-  if (a.hd == 128)
-    TL_LAUNCH_PDL(attn_decode_fused_kernel<128>, grid, 128, 0, s, a);
-  else
-    TL_LAUNCH_PDL(attn_decode_fused_kernel<64>, grid, 128, 0, s, a);
+  const int cl = decode_cluster_size(a.max_ctx);
+  dim3 grid(cl, a.H, a.rows);
+  cudaError_t e = a.hd == 128
+      ? launch_pdl_cluster(attn_decode_cluster_kernel<128>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per)
+      : launch_pdl_cluster(attn_decode_cluster_kernel<64>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per);
+  if (e != cudaSuccess)
+    return set_error(TL_ERR_CUDA, "launch of attn_decode_cluster_kernel failed: %s", cudaGetErrorString(e));
   return ok();
 }
 }  // namespace tl

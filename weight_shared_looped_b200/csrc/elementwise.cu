@@ -167,25 +167,42 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
   }
   const size_t row3 = (size_t)row * 3 * a.d;
   const size_t split_stride = (size_t)a.rows * 3 * a.d;
-  float q[2][2], k[2][2], v[2][2];
+  float q[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, k[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  float v[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  // partial sums: all q/k/v elements of up to four splits in flight, added in
+  // split order
+  for (int s0 = 0; s0 < a.S; s0 += 4) {
+    const int ns = min(4, a.S - s0);
+    float t[4][2][2][3];
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          if (s < ns && p < npair) {
+            const float* ps = a.part + (size_t)(s0 + s) * split_stride + row3 +
+                              (size_t)head * a.hd + lane + 32 * p + hh * half;
+            t[s][p][hh][0] = __ldcg(ps);
+            t[s][p][hh][1] = __ldcg(ps + a.d);
+            t[s][p][hh][2] = __ldcg(ps + 2 * a.d);
+          }
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int p = 0; p < 2; ++p)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          if (s < ns && p < npair) {
+            q[p][hh] += t[s][p][hh][0];
+            k[p][hh] += t[s][p][hh][1];
+            v[p][hh] += t[s][p][hh][2];
+          }
+  }
 #pragma unroll
   for (int p = 0; p < 2; ++p) {
     if (p < npair) {
       int i = lane + 32 * p;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        size_t col = (size_t)head * a.hd + i + hh * half;
-        float sq = 0.f, sk = 0.f, sv = 0.f;
-        for (int s = 0; s < a.S; ++s) {
-          const float* ps = a.part + s * split_stride + row3;
-          sq += ps[col];
-          sk += ps[a.d + col];
-          sv += ps[2 * a.d + col];
-        }
-        q[p][hh] = sq;
-        k[p][hh] = sk;
-        v[p][hh] = sv;
-      }
       float2 cs = a.rope_cs[(size_t)pos * half + i];
       float q0 = q[p][0], q1 = q[p][1], k0 = k[p][0], k1 = k[p][1];
       q[p][0] = q0 * cs.x - q1 * cs.y;

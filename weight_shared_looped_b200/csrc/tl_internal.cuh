@@ -41,7 +41,6 @@ constexpr int kMaxLanes = 8;
 constexpr int kMaxL = 64;
 constexpr int kMaxLayers = 16 + kMaxL;   // pre-blocks + loop iterations
 constexpr int kKvHeaderBytes = 4096;
-constexpr int kDecodeChunk = 64;         // keys per decode-attention split (fixed by position)
 
 // Device status codes written by kernels (same numbers as tl_status).
 constexpr int kDevTimeout = TL_ERR_TIMEOUT;
@@ -173,14 +172,11 @@ struct DecodeAttnArgs {
   const float* qkv_part;     // [S][rows][3d]
   int qkv_S;
   const float2* rope_cs;     // [max_ctx][hd/2]
-  int* counters;             // [kMaxLanes][H], zero between launches
   const char* kv_base;
   const KvHeader* hdr;
   size_t layer_bytes, kv_region_bytes;
   int layer, max_ctx, kv_int8;
   const int32_t* lane_of_row;
-  float* scratch;            // [rows][H][max_chunks][hd + 2]
-  int max_chunks;
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
 
