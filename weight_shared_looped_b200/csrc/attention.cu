@@ -33,7 +33,8 @@ __device__ __forceinline__ float warp_max(float v) {
 // score fragment reused in registers as the A operand of P V; V fragments come
 // from shared memory through ldmatrix.trans.  Online softmax in base 2 with
 // the 1/sqrt(hd) scale folded into log2(e).
-constexpr int FQ = 64;   // queries per CTA (4 warps x 16)
+constexpr int ATT_WARPS = 4;   // warps per CTA, 16 queries each
+constexpr int FQ = 16 * ATT_WARPS;   // queries per CTA
 constexpr int FK = 64;   // keys per tile
 
 __device__ __forceinline__ void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
@@ -50,7 +51,7 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __restrict__ q,
+__global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const __half* __restrict__ q,
                                                               const __half* __restrict__ k,
                                                               const __half* __restrict__ v,
                                                               __half* __restrict__ out, int T,
@@ -92,7 +93,7 @@ __global__ void __launch_bounds__(128) attn_prefill_tc_kernel(const __half* __re
   const int q_hi = min(q0 + FQ, T) - 1;
   for (int k0 = 0; k0 <= q_hi; k0 += FK) {
     __syncthreads();
-    for (int i = threadIdx.x; i < FK * (HD / 8); i += 128) {
+    for (int i = threadIdx.x; i < FK * (HD / 8); i += 32 * ATT_WARPS) {
       const int r = i / (HD / 8), c = (i % (HD / 8)) * 8;
       uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
       if (k0 + r < T) {
@@ -571,9 +572,9 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   dim3 grid((T + FQ - 1) / FQ, H);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
   if (hd == 128)
-    TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 128, 0, s, q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 32 * ATT_WARPS, 0, s, q, k, v, out, T, H, scale_log2);
   else if (hd == 64)
-    TL_LAUNCH_PDL(attn_prefill_tc_kernel<64>, grid, 128, 0, s, q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<64>, grid, 32 * ATT_WARPS, 0, s, q, k, v, out, T, H, scale_log2);
   else
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", hd);
   return ok();

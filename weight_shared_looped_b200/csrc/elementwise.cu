@@ -32,24 +32,33 @@ __global__ void embed_kernel(EmbedArgs a) {
   const int row = blockIdx.x;
   const int src = a.src_row ? a.src_row[row] : row;
   float* h = a.h + (size_t)row * a.d;
+  const __half* e;
   if (a.ids) {
     int id = a.ids[src];
     if (id < 0 || id >= a.vocab) {
       set_status(a.status, TL_ERR_INVALID_ARG);
       id = 0;
     }
-    const __half* e = a.embed + (size_t)id * a.d;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) h[i] = __half2float(e[i]);
+    e = a.embed + (size_t)id * a.d;
   } else {
-    const __half* e = a.h_in + (size_t)src * a.d;
-    for (int i = threadIdx.x; i < a.d; i += blockDim.x) h[i] = __half2float(e[i]);
+    e = a.h_in + (size_t)src * a.d;
+  }
+  // eight halves per thread and step (d is a multiple of 256)
+  for (int i = threadIdx.x * 8; i < a.d; i += blockDim.x * 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(e + i);
+    const __half2* hp = reinterpret_cast<const __half2*>(&w);
+    const float2 f0 = __half22float2(hp[0]), f1 = __half22float2(hp[1]);
+    const float2 f2 = __half22float2(hp[2]), f3 = __half22float2(hp[3]);
+    *reinterpret_cast<float4*>(h + i) = make_float4(f0.x, f0.y, f1.x, f1.y);
+    *reinterpret_cast<float4*>(h + i + 4) = make_float4(f2.x, f2.y, f3.x, f3.y);
   }
 }
 
 // ------------------------------------------------------------------ residual + RMSNorm
 // One CTA of d/8 threads per row, each thread two float4 vectors (columns
-// 4t.. and d/2 + 4t..).  The split-K partial sums are loaded four splits at a
-// time (independent loads in flight) and added in split order.  The sum of
+// 4t.. and d/2 + 4t..).  The split-K partial sums are loaded up to eight
+// (d <= 2048) or four splits at a time (independent loads in flight) and added
+// in split order.  The sum of
 // squares is reduced per thread, per warp (xor tree) and over the warps in
 // order: a fixed order that depends only on d.  One CTA per row keeps the
 // grid small (a prefill of 128 rows is one CTA per SM) so that it shares the
@@ -63,7 +72,8 @@ __device__ __forceinline__ void add4(float4& a, const float4 b) {
   a.w += b.w;
 }
 
-__global__ void __launch_bounds__(1024) residual_norm_kernel(NormArgs a) {
+template <int MAXT, int SP>
+__global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
   pdl_enter();
   __shared__ float red[NORM_MAX_WARPS];
   const int row = blockIdx.x;
@@ -76,18 +86,18 @@ __global__ void __launch_bounds__(1024) residual_norm_kernel(NormArgs a) {
   if (row < a.n_add && a.S > 0) {
     const size_t sstride = (size_t)a.part_rows * a.d;
     const float* p0 = a.part + (size_t)row * a.d;
-    for (int sp = 0; sp < a.S; sp += 4) {
-      const int n = min(4, a.S - sp);
-      float4 t0[4], t1[4];
+    for (int sp = 0; sp < a.S; sp += SP) {
+      const int n = min(SP, a.S - sp);
+      float4 t0[SP], t1[SP];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < SP; ++q) {
         if (q < n) {
           t0[q] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + c0));
           t1[q] = __ldcg(reinterpret_cast<const float4*>(p0 + (sp + q) * sstride + c1));
         }
       }
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < SP; ++q) {
         if (q < n) {
           add4(v0, t0[q]);
           add4(v1, t1[q]);
@@ -325,7 +335,13 @@ tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
   // d = 256 * 2^k: d / 8 threads (32 .. 1024)
   if (a.d < 256 || a.d > 8192 || (a.d & (a.d - 1)) != 0)
     return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs a power of two in [256, 8192]", a.d);
-  TL_LAUNCH_PDL(residual_norm_kernel, a.rows, a.d / 8, 0, s, a);
+  // up to 2048 columns: 256 threads with registers for eight splits in flight
+  // (more would keep the CTA from fitting next to a GEMM CTA); wider rows:
+  // four splits at a time
+  if (a.d <= 2048)
+    TL_LAUNCH_PDL((residual_norm_kernel<256, 8>), a.rows, a.d / 8, 0, s, a);
+  else
+    TL_LAUNCH_PDL((residual_norm_kernel<1024, 4>), a.rows, a.d / 8, 0, s, a);
   return ok();
 }
 
