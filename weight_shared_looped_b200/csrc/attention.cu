@@ -50,6 +50,24 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 16-byte cp.async, zero-filled when `valid` is false (rows past T).
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, bool valid) {
+  const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src),
+               "r"(valid ? 16 : 0)
+               : "memory");
+}
+
+// Two key tiles are copied per round trip (with the Q tile in the first): a
+// seq-128 CTA loads everything it needs at once; longer sequences refill the
+// two slots after each pair of tiles.
+constexpr int ATT_RES = 2;   // key tiles resident in shared memory at once
+
+template <int HD>
+constexpr size_t attn_prefill_smem() {
+  return (size_t)(FQ + 2 * ATT_RES * FK) * (HD + 8) * sizeof(__half);
+}
+
 template <int HD>
 __global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const __half* __restrict__ q,
                                                               const __half* __restrict__ k,
@@ -58,8 +76,10 @@ __global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const _
                                                               int H, float scale_log2) {
   pdl_enter();
   constexpr int LD = HD + 8;                 // halves per smem row (16-byte aligned, no conflicts)
-  __shared__ __align__(16) __half Ks[FK][LD];
-  __shared__ __align__(16) __half Vs[FK][LD];
+  extern __shared__ __align__(16) __half att_smem[];
+  __half (*Qs)[LD] = reinterpret_cast<__half (*)[LD]>(att_smem);                        // [FQ][LD]
+  __half (*Kr)[FK][LD] = reinterpret_cast<__half (*)[FK][LD]>(att_smem + FQ * LD);        // [ATT_RES]
+  __half (*Vr)[FK][LD] = reinterpret_cast<__half (*)[FK][LD]>(att_smem + (FQ + ATT_RES * FK) * LD);
   const int head = blockIdx.y;
   const int q0 = blockIdx.x * FQ;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -68,42 +88,61 @@ __global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const _
   const int qw = q0 + warp * 16;             // first query of this warp
   constexpr int KS = HD / 16;                // k steps over head_dim
   constexpr int NT = HD / 8;                 // output n tiles over head_dim
-
-  // Q fragments (A operand, 16 x HD), rows qw+g and qw+g+8
-  uint32_t qa[KS][4];
-  {
-    const int r0 = qw + g, r1 = qw + g + 8;
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) {
-      const int c = ks * 16 + 2 * t;
-      auto ld = [&](int r, int col) -> uint32_t {
-        if (r >= T) return 0u;
-        return *reinterpret_cast<const uint32_t*>(q + (size_t)r * d + head * HD + col);
-      };
-      qa[ks][0] = ld(r0, c);
-      qa[ks][1] = ld(r1, c);
-      qa[ks][2] = ld(r0, c + 8);
-      qa[ks][3] = ld(r1, c + 8);
+  constexpr int CPR = HD / 8;                // 16-byte pieces per row
+  constexpr int NTH = 32 * ATT_WARPS;
+  const int q_hi = min(q0 + FQ, T) - 1;
+  const int ntiles = q_hi / FK + 1;
+  // copy key tiles [t0, t0 + ATT_RES) into the resident slots (one round trip)
+  auto issue = [&](int t0) {
+    for (int tt = 0; tt < ATT_RES; ++tt) {
+      const int kt = t0 + tt;
+      if (kt >= ntiles) break;
+      const int k0 = kt * FK;
+      for (int i = threadIdx.x; i < FK * CPR; i += NTH) {
+        const int r = i / CPR, c = (i % CPR) * 8;
+        const bool ok = k0 + r < T;
+        const size_t off = (size_t)(ok ? k0 + r : 0) * d + head * HD + c;
+        cp_async16_zfill(&Kr[tt][r][c], k + off, ok);
+        cp_async16_zfill(&Vr[tt][r][c], v + off, ok);
+      }
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  for (int i = threadIdx.x; i < FQ * CPR; i += NTH) {
+    const int r = i / CPR, c = (i % CPR) * 8;
+    const bool ok = q0 + r < T;
+    cp_async16_zfill(&Qs[r][c], q + (size_t)(ok ? q0 + r : 0) * d + head * HD + c, ok);
   }
+  issue(0);
+
+  uint32_t qa[KS][4];
   float o[NT][4];
 #pragma unroll
   for (int i = 0; i < NT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const int q_hi = min(q0 + FQ, T) - 1;
-  for (int k0 = 0; k0 <= q_hi; k0 += FK) {
-    __syncthreads();
-    for (int i = threadIdx.x; i < FK * (HD / 8); i += 32 * ATT_WARPS) {
-      const int r = i / (HD / 8), c = (i % (HD / 8)) * 8;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
-      if (k0 + r < T) {
-        kv = *reinterpret_cast<const uint4*>(k + (size_t)(k0 + r) * d + head * HD + c);
-        vv = *reinterpret_cast<const uint4*>(v + (size_t)(k0 + r) * d + head * HD + c);
+  for (int kt = 0; kt < ntiles; ++kt) {
+    const int k0 = kt * FK;
+    if (kt % ATT_RES == 0) {
+      if (kt > 0) {
+        __syncthreads();                     // every warp is done with the resident tiles
+        issue(kt);
       }
-      *reinterpret_cast<uint4*>(&Ks[r][c]) = kv;
-      *reinterpret_cast<uint4*>(&Vs[r][c]) = vv;
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
     }
-    __syncthreads();
+    if (kt == 0) {
+      // Q fragments (A operand, 16 x HD), rows qw+g and qw+g+8
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        const int c = ks * 16 + 2 * t;
+        qa[ks][0] = *reinterpret_cast<const uint32_t*>(&Qs[warp * 16 + g][c]);
+        qa[ks][1] = *reinterpret_cast<const uint32_t*>(&Qs[warp * 16 + g + 8][c]);
+        qa[ks][2] = *reinterpret_cast<const uint32_t*>(&Qs[warp * 16 + g][c + 8]);
+        qa[ks][3] = *reinterpret_cast<const uint32_t*>(&Qs[warp * 16 + g + 8][c + 8]);
+      }
+    }
+    const __half (*Ks)[LD] = Kr[kt % ATT_RES];
+    const __half (*Vs)[LD] = Vr[kt % ATT_RES];
     if (k0 > qw + 15) continue;              // this warp's queries all precede the tile
     // S = Q K^T : 16 x 64
     float sc[FK / 8][4];
@@ -571,10 +610,22 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   if (T == 0) return ok();
   dim3 grid((T + FQ - 1) / FQ, H);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
+  static bool attr_done = false;
+  if (!attr_done) {
+    TL_CUDA(cudaFuncSetAttribute(attn_prefill_tc_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)attn_prefill_smem<128>()));
+    TL_CUDA(cudaFuncSetAttribute(attn_prefill_tc_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)attn_prefill_smem<64>()));
+    attr_done = true;
+  }
   if (hd == 128)
-    TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 32 * ATT_WARPS, 0, s, q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 32 * ATT_WARPS, attn_prefill_smem<128>(), s,
+                  q, k, v, out, T, H, scale_log2);
   else if (hd == 64)
-    TL_LAUNCH_PDL(attn_prefill_tc_kernel<64>, grid, 32 * ATT_WARPS, 0, s, q, k, v, out, T, H, scale_log2);
+    TL_LAUNCH_PDL(attn_prefill_tc_kernel<64>, grid, 32 * ATT_WARPS, attn_prefill_smem<64>(), s,
+                  q, k, v, out, T, H, scale_log2);
   else
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", hd);
   return ok();
