@@ -74,13 +74,24 @@ __device__ __forceinline__ void add4(float4& a, const float4 b) {
 
 template <int MAXT, int SP>
 __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
-  pdl_enter();
   __shared__ float red[NORM_MAX_WARPS];
   const int row = blockIdx.x;
   const int nthr = blockDim.x, nw = nthr >> 5;
   const int c0 = threadIdx.x * 4, c1 = a.d / 2 + threadIdx.x * 4;
-  float* h = a.h + (size_t)row * a.d;
+  // the gains are constants of the model and the lane map an input of the
+  // call: read them before waiting for the previous kernel, so no load round
+  // trip follows the reduction
+  const bool want_x = row < a.n_next;
+  const bool want_y = row >= a.fin_lo && row < a.fin_hi;
+  const float* gam = want_x ? a.gamma_next : want_y ? a.gamma_final : nullptr;
+  float4 g0 = make_float4(0.f, 0.f, 0.f, 0.f), g1 = g0;
+  if (gam) {
+    g0 = *reinterpret_cast<const float4*>(gam + c0);
+    g1 = *reinterpret_cast<const float4*>(gam + c1);
+  }
   const int out_row = a.out_row ? a.out_row[row] : row;
+  pdl_enter();
+  float* h = a.h + (size_t)row * a.d;
   float4 v0 = *reinterpret_cast<const float4*>(h + c0);
   float4 v1 = *reinterpret_cast<const float4*>(h + c1);
   if (row < a.n_add && a.S > 0) {
@@ -112,8 +123,6 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
     *reinterpret_cast<float4*>(tr + c0) = v0;
     *reinterpret_cast<float4*>(tr + c1) = v1;
   }
-  const bool want_x = row < a.n_next;
-  const bool want_y = row >= a.fin_lo && row < a.fin_hi;
   if (!want_x && !want_y) return;
   float ss = 0.0f;
   ss = fmaf(v0.x, v0.x, ss);
@@ -130,8 +139,7 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
   float tot = 0.0f;
   for (int w = 0; w < nw; ++w) tot += red[w];
   const float r = rsqrtf(tot / (float)a.d + a.eps);
-  auto out_x = [&](int c, const float4 v) {
-    const float4 g = *reinterpret_cast<const float4*>(a.gamma_next + c);
+  auto out_x = [&](int c, const float4 v, const float4 g) {
     const __half2 lo = __halves2half2(__float2half_rn(v.x * r * g.x), __float2half_rn(v.y * r * g.y));
     const __half2 hi = __halves2half2(__float2half_rn(v.z * r * g.z), __float2half_rn(v.w * r * g.w));
     uint2 pk;
@@ -139,8 +147,7 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
     pk.y = *reinterpret_cast<const uint32_t*>(&hi);
     *reinterpret_cast<uint2*>(a.x + (size_t)row * a.d + c) = pk;
   };
-  auto out_y = [&](int c, const float4 v) -> bool {
-    const float4 g = *reinterpret_cast<const float4*>(a.gamma_final + c);
+  auto out_y = [&](int c, const float4 v, const float4 g) -> bool {
     float4 o;
     o.x = v.x * r * g.x;
     o.y = v.y * r * g.y;
@@ -150,11 +157,11 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
     return !isfinite(o.x) || !isfinite(o.y) || !isfinite(o.z) || !isfinite(o.w);
   };
   if (want_x) {
-    out_x(c0, v0);
-    out_x(c1, v1);
+    out_x(c0, v0, g0);
+    out_x(c1, v1, g1);
   } else {
-    const bool bad0 = out_y(c0, v0);
-    const bool bad1 = out_y(c1, v1);
+    const bool bad0 = out_y(c0, v0, g0);
+    const bool bad1 = out_y(c1, v1, g1);
     if (bad0 || bad1) set_status(a.status, TL_ERR_NUMERIC);
   }
 }
@@ -163,17 +170,33 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
 // One warp per (row, head).  Lane l handles rotate-half pairs (i, i + hd/2)
 // for i = l, l + 32 (hd = 128) or i = l (hd = 64).
 __global__ void rope_kv_kernel(RopeKvArgs a) {
-  pdl_enter();
   const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (wid >= a.rows * a.H) return;
+  const bool active = wid < a.rows * a.H;
   const int row = wid / a.H, head = wid % a.H;
   const int half = a.hd / 2;
   const int npair = half / 32;   // 1 or 2
   int kv_lane = a.lane, pos = row;
+  // prefill: the positions are the row indices, and the RoPE table and the
+  // cache's layer offsets are constants: read them before waiting for the QKV
+  // projection
+  float2 csp[2] = {make_float2(1.f, 0.f), make_float2(1.f, 0.f)};
+  int cum = 0;
+  if (active && !a.decode) {
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+      if (p < npair) csp[p] = a.rope_cs[(size_t)pos * half + lane + 32 * p];
+    if (a.kv_base) cum = a.hdr->cum_layers[kv_lane];
+  }
+  pdl_enter();
+  if (!active) return;
   if (a.decode) {
     kv_lane = a.lane_of_row[row];
     pos = a.hdr->pos[kv_lane];
+#pragma unroll
+    for (int p = 0; p < 2; ++p)
+      if (p < npair) csp[p] = a.rope_cs[(size_t)pos * half + lane + 32 * p];
+    if (a.kv_base) cum = a.hdr->cum_layers[kv_lane];
   }
   const size_t row3 = (size_t)row * 3 * a.d;
   const size_t split_stride = (size_t)a.rows * 3 * a.d;
@@ -213,7 +236,7 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
   for (int p = 0; p < 2; ++p) {
     if (p < npair) {
       int i = lane + 32 * p;
-      float2 cs = a.rope_cs[(size_t)pos * half + i];
+      const float2 cs = csp[p];
       float q0 = q[p][0], q1 = q[p][1], k0 = k[p][0], k1 = k[p][1];
       q[p][0] = q0 * cs.x - q1 * cs.y;
       q[p][1] = q1 * cs.x + q0 * cs.y;
@@ -241,7 +264,7 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
     }
   }
   if (!a.kv_base) return;
-  char* layer = a.kv_base + (size_t)(a.hdr->cum_layers[kv_lane] + a.layer) * a.layer_bytes;
+  char* layer = a.kv_base + (size_t)(cum + a.layer) * a.layer_bytes;
   const size_t eoff = ((size_t)head * a.max_ctx + pos) * a.hd;
   if (!a.kv_int8) {
     __half* K = reinterpret_cast<__half*>(layer) + eoff;
