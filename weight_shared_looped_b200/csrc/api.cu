@@ -690,18 +690,14 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     da.rope_cs = m->rope;
     TL_TRY(launch_attn_decode_fused(da, s));
   }
-  // O projection, residual, RMSNorm before the MLP (decode: the GEMV's last
-  // CTA per row block adds the residual, the norm reads h only)
+  // O projection, then the residual add of its split-K partial sums and the
+  // RMSNorm before the MLP in one norm kernel
   g = gemm_args(m, b, 1, m->attn, rows);
-  if (decode) {
-    g.h = m->h;
-    g.tickets = m->gemv_tickets;
-  }
   TL_TRY(launch_gemm(g, s));
   NormArgs n = norm_args(m, rows);
   n.part = m->part;
   n.part_rows = rows;
-  n.S = decode ? 0 : g.splits;
+  n.S = g.splits;
   n.n_add = rows;
   n.gamma_next = b->d.gamma_ffn;
   n.n_next = rows;
@@ -718,8 +714,6 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     dn.x_part = m->part2;
     dn.x_S = g.splits;
     dn.x_F = m->F;
-    dn.h = m->h;
-    dn.tickets = m->gemv_tickets;
     TL_TRY(launch_gemm(dn, s));
   } else {
     if (gemm_tc_eligible(g.N, g.K, rows) && g.splits == 1 && m->F % 64 == 0) {
@@ -812,7 +806,10 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
     TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, s));
     const int nxt = layer + 1 < n_layers ? active(layer + 1) : 0;
     NormArgs en = norm_args(m, trace ? B : act);
-    en.S = 0;   // the down projection already added its sums into h
+    // the down projection's split-K partial sums are added into h here
+    en.part = m->part;
+    en.part_rows = act;
+    en.S = gemm_splits(m->d, m->F, act);
     en.n_add = act;
     en.n_next = nxt;
     if (nxt > 0) en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
