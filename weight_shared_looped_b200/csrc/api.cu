@@ -107,7 +107,6 @@ struct tl_model {
   __half* u;
   float* part;
   float* part2;          // decode: gate|up partials read by the down projection
-  int* gemv_tickets;     // decode: residual-add tickets per 128-row block, zero between launches
   float* y;
   int32_t* lane_map;
   int* status;
@@ -329,7 +328,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
   void* p_u; void* p_part; void* p_y; void* p_lid; void* p_status; void* p_rope;
-  void* p_part2; void* p_gtk;
+  void* p_part2;
   size_t part2_floats = 0;
   for (int t = 1; t <= md.max_lanes; ++t)
     part2_floats = std::max(part2_floats, (size_t)gemm_splits(2 * F, d, t) * t * 2 * F);
@@ -345,7 +344,6 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_u, (size_t)T * F * 2},
       {&p_part, maxpart * 4},
       {&p_part2, part2_floats * 4},
-      {&p_gtk, (size_t)1024 * 4},
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
       {&p_status, 256},
@@ -372,7 +370,6 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->u = (__half*)p_u;
   m->part = (float*)p_part;
   m->part2 = (float*)p_part2;
-  m->gemv_tickets = (int*)p_gtk;
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
   m->status = (int*)p_status;
@@ -393,7 +390,6 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
                                 cudaMemcpyHostToDevice);
     cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
-    if (e3 == cudaSuccess) e3 = cudaMemset(m->gemv_tickets, 0, (size_t)1024 * 4);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
       return set_error(TL_ERR_CUDA, "model initialisation copy failed");

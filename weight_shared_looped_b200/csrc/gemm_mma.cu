@@ -312,26 +312,6 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
     out[(size_t)(tk + 1) * a.N + rowA] = acc[1];
     out[(size_t)(tk + 1) * a.N + rowA + 8] = acc[3];
   }
-  if (a.h == nullptr) return;
-  // last split of this row block: residual add of all partial sums, split order
-  __shared__ int gv_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int ticket = atomicAdd(&a.tickets[blockIdx.x], 1);
-    gv_last = ticket == a.splits - 1;
-    if (gv_last) a.tickets[blockIdx.x] = 0;
-  }
-  __syncthreads();
-  if (!gv_last) return;
-  __threadfence();
-  for (int i = threadIdx.x; i < a.T * GV_ROWS; i += GV_THREADS) {
-    const int tt = i / GV_ROWS, n = m0 + i % GV_ROWS;
-    float v = a.h[(size_t)tt * a.N + n];
-    float sum = 0.f;
-    for (int sp = 0; sp < a.splits; ++sp) sum += __ldcg(a.part + ((size_t)sp * a.T + tt) * a.N + n);
-    a.h[(size_t)tt * a.N + n] = v + sum;
-  }
 }
 
 __global__ void split_sum_kernel(const float* __restrict__ part, int S, long n,
@@ -402,14 +382,14 @@ tl_status launch_gemv(const GemmArgs& a, cudaStream_t s) {
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.swiglu_u) {
     if (!gemm_tc_eligible(a.N, a.K, a.T) || a.splits != 1 || a.N != 2 * a.n_split ||
-        a.n_split % 64 != 0 || a.x_part || a.h)
+        a.n_split % 64 != 0 || a.x_part)
       return set_error(TL_ERR_UNSUPPORTED,
                        "the fused SwiGLU epilogue needs the one-split tensor-core GEMM");
     return launch_gemm_tc(a, s);
   }
   if (gemv_eligible(a.N, a.K, a.T)) return launch_gemv(a, s);
-  if (a.x_part || a.h)
-    return set_error(TL_ERR_UNSUPPORTED, "fused staging / residual needs the decode GEMV");
+  if (a.x_part)
+    return set_error(TL_ERR_UNSUPPORTED, "fused SwiGLU staging needs the decode GEMV");
   if (gemm_tc_eligible(a.N, a.K, a.T)) return launch_gemm_tc(a, s);
   return launch_gemm_mma(a, s);
 }

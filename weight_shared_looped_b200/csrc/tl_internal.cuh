@@ -82,12 +82,6 @@ struct GemmArgs {
   // gate|up partial sums) instead of x
   const float* x_part;
   int x_S, x_F;
-  // decode GEMV only: when h is set, the last CTA of each 128-row block (an
-  // atomic ticket in `tickets`, reset after use) adds the S partial sums in
-  // split order to h[t][n] (the residual stream) instead of leaving them for
-  // a later kernel
-  float* h;
-  int* tickets;
   // tensor-core kernel with one split only, for [gate; up] weights (n_split =
   // F, N = 2F): when swiglu_u is set, each CTA takes 64 gate rows and the same
   // 64 up rows and writes swiglu_u[t][f] = fp16(silu(gate) * up) (fp16 [T][F])
