@@ -16,11 +16,6 @@
 namespace tl {
 namespace {
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -266,90 +261,180 @@ __device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
   return v;
 }
 
-// Four int8 codes of a word to float, exactly: each biased byte goes into the
-// low mantissa bits of 2^23 (prmt with the constant's upper bytes), then the
-// bias 2^23 + 128 is subtracted.
-__device__ __forceinline__ void int8x4_to_float(uint32_t w, float* f) {
-  const uint32_t u = w ^ 0x80808080u;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t b;
-    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(b) : "r"(u), "r"(0x4B000000u), "r"(0x7650u | (uint32_t)i));
-    f[i] = __uint_as_float(b) - 8388736.0f;
+constexpr int DS_KEYS = 64;     // keys per stage of the decode kernel
+
+// ------------------------------------------------------------------ decode (tensor cores)
+// Within a CTA both products run on the tensor cores (mma.sync m16n8k16, fp16 in, fp32 accumulate) in transposed
+// form, so that the single query fills the N = 8 side and keys or head_dim
+// elements fill all 16 rows:
+//   S^T = K q^T : A = 16 keys x 16 head_dim elements, B = q (column 0)
+//   O^T = V^T P^T : A = 16 head_dim elements x 16 keys, B = p (column 0)
+// In each 64-key stage warp w owns keys 16w..16w+15.  FP16 K and V tiles
+// come through ldmatrix (V transposed).  INT8 codes become exact fp16 values
+// in registers (code + 128 in the low mantissa bits of 1024, minus 1152); a
+// lane then reads whole 16-byte chunks of its rows, and the k (or m) index of
+// each element follows from where it sits in the chunk, the same order being
+// used for q and for the output columns.  The scores of a warp sit in lanes
+// 4g (keys g and g + 8); the weights reach the P V B operand through two
+// shuffles.  Each warp keeps its own running max and sum (base 2); the four
+// warps merge at the end, then rank 0 of the cluster merges the CTAs in rank
+// order.
+constexpr int DT_STAGES_I8 = 3;    // stage ring of the tensor-core decode kernel, INT8 cache
+constexpr int DT_STAGES_F16 = 2;   // and FP16 cache (twice the bytes per stage)
+
+template <int HD, bool I8>
+struct DecTc {
+  static constexpr int KB = HD * (I8 ? 1 : 2);          // bytes of a cached row
+  static constexpr int NCH = KB / 64;                   // 16-byte chunks per lane and key
+  static constexpr bool VPAD = I8 && HD == 64;          // 64-byte INT8 V rows: padded, not swizzled
+  static constexpr int ROWK = KB;                       // K stage row
+  static constexpr int ROWV = VPAD ? KB + 16 : KB;      // V stage row
+  static constexpr int NST = I8 ? DT_STAGES_I8 : DT_STAGES_F16;
+  static constexpr int EPC = I8 ? 4 : 2;                // k steps per chunk
+  static constexpr int KSTEP = NCH * EPC;               // = HD / 16
+  static constexpr size_t STAGE_BYTES = (size_t)DS_KEYS * (ROWK + ROWV);
+  // INT8: chunk of a K row read by quad lane t as its h-th chunk
+  __host__ __device__ static constexpr int chunk(int t, int h) {
+    return NCH == 1 ? t : 2 * t + (h & 1) + 8 * (h >> 1);
   }
+  // Stage rows are stored with their 16-byte chunks permuted (XOR with bits
+  // of the row index) so that each quarter-warp's INT8 reads and each
+  // ldmatrix's eight rows fall on distinct banks without padding.
+  __host__ __device__ static constexpr int kphys(int r, int c) {
+    return !I8 ? c ^ (r & 7) : NCH == 1 ? c : c ^ (r & 1);
+  }
+  __host__ __device__ static constexpr int vphys(int r, int c) {
+    return VPAD ? c : I8 ? c ^ (r & 6) : c ^ (r & 7);
+  }
+};
+
+__device__ __forceinline__ void lds128(uint32_t* w, uint32_t addr) {
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t* r, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void lds64(uint32_t* w, uint32_t addr) {
+  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(w[0]), "=r"(w[1]) : "r"(addr));
 }
 
-constexpr int DS_KEYS = 64;     // keys per stage of the streaming decode kernel
-constexpr int DS_STAGES = 3;    // stages in flight (cp.async ring)
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 
-template <int HD>
-__global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs a, int CL,
-                                                                  int max_per) {
+// four int8 codes (bytes 0..3 of w) -> fp16 pairs (0,1) and (2,3), exactly
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  uint32_t x0, x1;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x0) : "r"(u), "r"(0x64646464u), "r"(0x4140u));
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x1) : "r"(u), "r"(0x64646464u), "r"(0x4342u));
+  const __half2 bias = __float2half2_rn(1152.0f);
+  lo = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&x0), bias));
+  hi = h2_bits(__hsub2(*reinterpret_cast<__half2*>(&x1), bias));
+}
+
+// byte e of wa and byte e of wb (int8 codes) -> an fp16 pair, exactly
+template <int E>
+__device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t wa, uint32_t wb) {
+  uint32_t x, y;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(wa), "r"(wb), "r"((uint32_t)(E | ((E + 4) << 8))));
+  // low byte of each half: code ^ 0x80; high byte: 0x64
+  asm("lop3.b32 %0, %1, %2, %3, 0x6a;" : "=r"(y) : "r"(x), "r"(0x00FF00FFu), "r"(0x64806480u));
+  const __half2 bias = __float2half2_rn(1152.0f);
+  return h2_bits(__hsub2(*reinterpret_cast<__half2*>(&y), bias));
+}
+
+template <int HD, bool I8>
+__global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeAttnArgs a, int CL,
+                                                                       int sc_len) {
+  using T = DecTc<HD, I8>;
   constexpr int HALF = HD / 2;
-  constexpr int KSPLIT = 128 / HD;              // key slices in the P V step (1 or 2)
+  constexpr int MT = HD / 16;                    // P V m tiles of 16 head_dim elements
   extern __shared__ __align__(16) unsigned char dsm[];
   __shared__ float qs[HD], kn[HD], vn[HD];
-  __shared__ float acc_s[KSPLIT][HD];
-  __shared__ float pw[DS_KEYS];                  // weights of the current stage's keys
-  __shared__ float stat_s[2];                    // this CTA's max score and exponential sum
-  __shared__ float red[4];
+  __shared__ __align__(16) __half qh[HD];
+  __shared__ float wm[4], wl[4];
+  __shared__ float acc_s[HD];
+  __shared__ float stat_s[2];
+  __shared__ float kmax_s[4], vmax_s[4];
   const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int esz = a.kv_int8 ? 1 : 2;
-  const int rowb = HD * esz;
-  const int stage_bytes = DS_KEYS * rowb;
-  unsigned char* kst = dsm;                                        // [DS_STAGES][DS_KEYS][rowb]
-  unsigned char* vst = dsm + (size_t)DS_STAGES * stage_bytes;      // [DS_STAGES][DS_KEYS][rowb]
-  float* ksc = reinterpret_cast<float*>(dsm + 2 * (size_t)DS_STAGES * stage_bytes);   // [max_per]
-  float* vsc = ksc + max_per;
-  // positions, the lane map, the RoPE table and the cached rows before pos
-  // were written by earlier steps
+  const int g = lane >> 2, t = lane & 3;
+  unsigned char* kst = dsm;                                          // [NST][DS_KEYS][ROWK]
+  unsigned char* vst = dsm + (size_t)T::NST * DS_KEYS * T::ROWK;     // [NST][DS_KEYS][ROWV]
+  float* ksc = reinterpret_cast<float*>(dsm + (size_t)T::NST * T::STAGE_BYTES);   // [sc_len]
+  float* vsc = ksc + sc_len;
   const int lane_id = a.lane_of_row[row];
   const int pos = a.hdr->pos[lane_id];
   const int n_keys = pos + 1;
   const int per = (n_keys + CL - 1) / CL;
   const int k0 = min(crank * per, n_keys), k1 = min(k0 + per, n_keys);
   const int nk = k1 - k0;
-  const bool owner = nk > 0 && k1 == n_keys;     // holds position pos
+  const bool owner = nk > 0 && k1 == n_keys;
   const int n_old = owner ? nk - 1 : nk;
   const int nsub = (nk + DS_KEYS - 1) / DS_KEYS;
   char* layer = const_cast<char*>(a.kv_base) +
                 (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
   const size_t head_off = (size_t)head * a.max_ctx;
   const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
-  // copy the cached rows of stage `sub` into ring slot sub % DS_STAGES (one
-  // commit group per stage, empty past the end)
+  // stage `sub` into ring slot sub % NST: cached rows are copied, rows past
+  // this CTA's keys zero-filled; the owner's new row is left to the append
+  // below (no copy races with it).  Thread tid always copies chunk
+  // tid % PIECES of rows tid / PIECES + RPP * p, so its shared-memory offsets
+  // (chunk permutation included) are fixed.
+  constexpr int PIECES = T::KB / 16, RPP = 128 / PIECES, PASSES = DS_KEYS / RPP;
+  const int cr0 = tid / PIECES, cpc = tid % PIECES;
+  const uint32_t kdst0 = (uint32_t)__cvta_generic_to_shared(kst) + cr0 * T::ROWK + 16 * T::kphys(cr0, cpc);
+  const uint32_t vdst0 = (uint32_t)__cvta_generic_to_shared(vst) + cr0 * T::ROWV + 16 * T::vphys(cr0, cpc);
+  const char* ksrc0 = layer + (head_off + k0 + cr0) * (size_t)T::KB + 16 * cpc;
   auto issue = [&](int sub) {
     if (sub < nsub) {
-      const int lo = sub * DS_KEYS, cnt = min(DS_KEYS, n_old - lo);
-      const int pieces = rowb / 16;
-      for (int which = 0; which < 2; ++which) {
-        const char* src = layer + which * a.kv_region_bytes + (head_off + k0 + lo) * rowb;
-        unsigned char* dst = (which ? vst : kst) + (size_t)(sub % DS_STAGES) * stage_bytes;
-        for (int i = tid; i < cnt * pieces; i += 128) {
-          const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst + i * 16);
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src + i * 16)
-                       : "memory");
-        }
+      const int slot = sub % T::NST;
+      const uint32_t kd = kdst0 + slot * (DS_KEYS * T::ROWK);
+      const uint32_t vd = vdst0 + slot * (DS_KEYS * T::ROWV);
+      const char* ks = ksrc0 + (size_t)sub * (DS_KEYS * T::KB);
+      const char* vs = ks + a.kv_region_bytes;
+      const int rem = n_old - sub * DS_KEYS - cr0;   // row cr0 + RPP*p is cached iff RPP*p < rem
+#pragma unroll
+      for (int p = 0; p < PASSES; ++p) {
+        if (owner && RPP * p == rem) continue;       // the new key's row
+        const bool ok = RPP * p < rem;
+        const uint32_t n = ok ? 16 : 0;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(kd + p * RPP * T::ROWK),
+                     "l"(ok ? ks + p * RPP * T::KB : layer), "r"(n) : "memory");
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(vd + p * RPP * T::ROWV),
+                     "l"(ok ? vs + p * RPP * T::KB : layer), "r"(n) : "memory");
       }
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
 #pragma unroll
-  for (int st = 0; st < DS_STAGES - 1; ++st) issue(st);
-  if (a.kv_int8) {
-    const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes);
-    const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region);
-    for (int j = tid; j < n_old; j += 128) {
-      ksc[j] = __half2float(kq[head_off + k0 + j]);
-      vsc[j] = __half2float(vq[head_off + k0 + j]);
+  for (int st = 0; st < T::NST - 1; ++st) issue(st);
+  pdl_enter();
+
+  // the cached keys' scales, the RoPE pair and the QKV partial sums are all
+  // requested before any of them is used (one round trip)
+  constexpr int SCU = 4;                         // scale loads in flight per thread
+  const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes) + head_off + k0;
+  const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region) +
+                     head_off + k0;
+  __half ksr[SCU], vsr[SCU];
+  if (I8) {
+#pragma unroll
+    for (int u = 0; u < SCU; ++u) {
+      const int j = tid + 128 * u;
+      if (j < n_old) {
+        ksr[u] = kq[j];
+        vsr[u] = vq[j];
+      }
     }
   }
   float2 cs = make_float2(1.f, 0.f);
   if (tid < HD) cs = a.rope_cs[(size_t)pos * HALF + (tid % HALF)];
-  pdl_enter();
-
-  // q (and k, v in the owner) from the QKV partial sums, all splits in flight
   const size_t split_stride = (size_t)a.rows * 3 * a.d;
   const float* prow = a.qkv_part + (size_t)row * 3 * a.d + (size_t)head * HD;
   if (tid < HD) {
@@ -379,9 +464,24 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
     kn[tid] = sk;
     vn[tid] = sv;
   }
+  if (I8) {
+#pragma unroll
+    for (int u = 0; u < SCU; ++u) {
+      const int j = tid + 128 * u;
+      if (j < n_old) {
+        ksc[j] = __half2float(ksr[u]);
+        vsc[j] = __half2float(vsr[u]);
+      }
+    }
+    for (int j = tid + 128 * SCU; j < n_old; j += 128) {   // longer contexts
+      ksc[j] = __half2float(kq[j]);
+      vsc[j] = __half2float(vq[j]);
+    }
+  }
   __syncthreads();
-  float qr = 0.f, kr = 0.f;
+  float kr = 0.f;
   if (tid < HD) {
+    float qr;
     if (tid < HALF) {
       qr = qs[tid] * cs.x - qs[tid + HALF] * cs.y;
       kr = kn[tid] * cs.x - kn[tid + HALF] * cs.y;
@@ -389,17 +489,15 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
       qr = qs[tid] * cs.x + qs[tid - HALF] * cs.y;
       kr = kn[tid] * cs.x + kn[tid - HALF] * cs.y;
     }
+    qh[tid] = __float2half_rn(qr);               // the query in fp16, as in the prefill path
   }
-  __syncthreads();
-  // the query is rounded to fp16 as in the prefill path
-  if (tid < HD) qs[tid] = __half2float(__float2half_rn(qr)) * rsqrtf((float)HD);
-  // owner: the new entry (position pos = key nk - 1 of this CTA) is appended
-  // to the cache now and copied into its stage slot when that stage is read
+  // owner: the new entry (position pos = key n_old of this CTA) is appended
+  // to the cache now and written into its stage row when that stage is read
   uint32_t k_new = 0, v_new = 0;     // fp16 bits or int8 code of element tid
   if (owner) {
     const __half kh = __float2half_rn(kr);
     const __half vh = __float2half_rn(tid < HD ? vn[tid] : 0.f);
-    if (!a.kv_int8) {
+    if (!I8) {
       if (tid < HD) {
         reinterpret_cast<__half*>(layer)[(head_off + pos) * HD + tid] = kh;
         reinterpret_cast<__half*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = vh;
@@ -411,7 +509,6 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
       float vm = tid < HD ? fabsf(__half2float(vh)) : 0.f;
       km = warp_max(km);
       vm = warp_max(vm);
-      __shared__ float kmax_s[4], vmax_s[4];
       if (lane == 0) {
         kmax_s[warp] = km;
         vmax_s[warp] = vm;
@@ -434,171 +531,235 @@ __global__ void __launch_bounds__(128) attn_decode_cluster_kernel(DecodeAttnArgs
       if (tid == 0) {
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] = vsh;
-        ksc[nk - 1] = ksf;
-        vsc[nk - 1] = vsf;
+        ksc[n_old] = ksf;
+        vsc[n_old] = vsf;
       }
     }
   }
+  __syncthreads();   // qh final
 
-  // streaming online softmax over the stages
-  constexpr int QD = HD / 4;                     // head_dim quarter of a score thread
-  constexpr int G4 = HD / 4, KS4 = 128 / G4;     // P V: 4-dim groups x key slices
-  __syncthreads();                               // qs final
-  const int qq = tid & 3;                        // this thread's quarter of head_dim
-  float qreg[QD];
+  // q as the B operand of S^T (column 0: lanes g == 0).  k step ks covers
+  // head_dim elements lo, lo+1 (k indices 2t, 2t+1) and hi, hi+1 (2t+8, 2t+9):
+  // FP16: lo = 16ks + 2t, hi = lo + 8 (the ldmatrix order); INT8 (ks = 4h + e):
+  // lo = 16 chunk(t, h) + 4e, hi = lo + 2 (four consecutive codes of a word).
+  uint32_t qb[T::KSTEP][2];
 #pragma unroll
-  for (int d = 0; d < QD; ++d) qreg[d] = qs[qq * QD + d];
+  for (int ks = 0; ks < T::KSTEP; ++ks) {
+    const int lo = I8 ? 16 * T::chunk(t, ks / 4) + 4 * (ks % 4) : 16 * ks + 2 * t;
+    const int hi = I8 ? lo + 2 : lo + 8;
+    qb[ks][0] = g == 0 ? *reinterpret_cast<const uint32_t*>(&qh[lo]) : 0u;
+    qb[ks][1] = g == 0 ? *reinterpret_cast<const uint32_t*>(&qh[hi]) : 0u;
+  }
+  const float csc = rsqrtf((float)HD) * 1.4426950408889634f;   // 1/sqrt(hd) in base 2
   float m = -INFINITY, l = 0.f;
-  float acc4[4] = {0.f, 0.f, 0.f, 0.f};          // dims 4g..4g+3 over key slice ks
-  const int g4 = tid % G4, ks4 = tid / G4;
+  float o[MT][4];                                // O^T tiles; column 0 (lanes t == 0) is the output
+#pragma unroll
+  for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+  const int kw = 16 * warp;                      // this warp's first key in a stage
+  // slot-0 shared-memory addresses of this lane's reads
+  uint32_t k_addr, v_addr;
+  int kmask = 0, vmask = 0;
+  if constexpr (I8) {
+    k_addr = (uint32_t)__cvta_generic_to_shared(kst) + (kw + g) * T::ROWK;   // + chunk, + 8 rows
+    v_addr = (uint32_t)__cvta_generic_to_shared(vst) + (kw + 2 * t) * T::ROWV +
+             (T::VPAD ? (HD / 8) * g : 16 * T::vphys(2 * t, g));
+  } else {
+    // ldmatrix rows: K lane l -> key kw + (l & 7) + 8 ((l >> 3) & 1), chunk 2ks + (l >> 4);
+    // V lane l -> key kw + (l & 7) + 8 (l >> 4), chunk 2mt + ((l >> 3) & 1)
+    k_addr = (uint32_t)__cvta_generic_to_shared(kst) + (kw + (lane & 7) + 8 * ((lane >> 3) & 1)) * T::ROWK;
+    v_addr = (uint32_t)__cvta_generic_to_shared(vst) + (kw + (lane & 7) + 8 * (lane >> 4)) * T::ROWV;
+    kmask = (lane >> 4) ^ (lane & 7);            // chunk 2ks + (l >> 4) is stored at 2ks ^ kmask
+    vmask = ((lane >> 3) & 1) ^ (lane & 7);
+  }
   for (int sub = 0; sub < nsub; ++sub) {
-    issue(sub + DS_STAGES - 1);                  // its slot was freed at the end of the last stage
-    asm volatile("cp.async.wait_group %0;" ::"n"(DS_STAGES - 1) : "memory");
-    const int slot = sub % DS_STAGES;
-    unsigned char* ks_ = kst + (size_t)slot * stage_bytes;
-    unsigned char* vs_ = vst + (size_t)slot * stage_bytes;
+    asm volatile("cp.async.wait_group %0;" ::"n"(T::NST - 2) : "memory");
+    const int slot = sub % T::NST;
     const int base = sub * DS_KEYS;
     const int cnt = min(DS_KEYS, nk - base);
-    if (owner && nk - 1 - base >= 0 && nk - 1 - base < DS_KEYS && tid < HD) {
-      const int r = nk - 1 - base;
-      if (!a.kv_int8) {
-        reinterpret_cast<unsigned short*>(ks_)[r * HD + tid] = (unsigned short)k_new;
-        reinterpret_cast<unsigned short*>(vs_)[r * HD + tid] = (unsigned short)v_new;
+    if (owner && n_old >= base && n_old - base < DS_KEYS && tid < HD) {
+      const int r = n_old - base;
+      const int byte = tid * (I8 ? 1 : 2), c = byte >> 4, off = byte & 15;
+      unsigned char* kd = kst + (size_t)slot * DS_KEYS * T::ROWK + (size_t)r * T::ROWK + 16 * T::kphys(r, c) + off;
+      unsigned char* vd = vst + (size_t)slot * DS_KEYS * T::ROWV + (size_t)r * T::ROWV + 16 * T::vphys(r, c) + off;
+      if (!I8) {
+        *reinterpret_cast<unsigned short*>(kd) = (unsigned short)k_new;
+        *reinterpret_cast<unsigned short*>(vd) = (unsigned short)v_new;
       } else {
-        ks_[r * HD + tid] = (unsigned char)k_new;
-        vs_[r * HD + tid] = (unsigned char)v_new;
+        *kd = (unsigned char)k_new;
+        *vd = (unsigned char)v_new;
       }
     }
-    __syncthreads();   // the stage's rows (and the appended entry) are visible
-    // scores: four threads per key (one head_dim quarter each), q in registers
-    float sc[DS_KEYS / 32];
+    __syncthreads();   // stage sub visible; every warp is done with stage sub - 1
+    issue(sub + T::NST - 1);                     // into the slot of stage sub - 1
+    if (kw >= cnt) continue;                     // no key of this warp in the stage
+    // S^T = K q^T: lane 4g ends with the scores of keys kw + g (s[0]) and kw + g + 8 (s[2])
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    const uint32_t kb_ = k_addr + slot * (DS_KEYS * T::ROWK);
+    if constexpr (I8) {
 #pragma unroll
-    for (int ps = 0; ps < DS_KEYS / 32; ++ps) {
-      const int j = ps * 32 + (tid >> 2);
-      float d0 = 0.f, d1 = 0.f;
-      if (j < cnt) {
-        if (!a.kv_int8) {
-          const uint4* src = reinterpret_cast<const uint4*>(ks_ + (size_t)j * rowb + qq * QD * 2);
+      for (int h = 0; h < T::NCH; ++h) {
+        const int ph = 16 * T::kphys(g, T::chunk(t, h));   // rows kw+g, kw+g+8: same parity
+        uint32_t w0[4], w1[4];
+        lds128(w0, kb_ + ph);
+        lds128(w1, kb_ + 8 * T::ROWK + ph);
 #pragma unroll
-          for (int c = 0; c < QD / 8; ++c) {
-            const uint4 w = src[c];
-            const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&w.x));
-            const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&w.y));
-            const float2 f2 = __half22float2(*reinterpret_cast<const __half2*>(&w.z));
-            const float2 f3 = __half22float2(*reinterpret_cast<const __half2*>(&w.w));
-            d0 = fmaf(qreg[c * 8 + 0], f0.x, fmaf(qreg[c * 8 + 1], f0.y, d0));
-            d1 = fmaf(qreg[c * 8 + 2], f1.x, fmaf(qreg[c * 8 + 3], f1.y, d1));
-            d0 = fmaf(qreg[c * 8 + 4], f2.x, fmaf(qreg[c * 8 + 5], f2.y, d0));
-            d1 = fmaf(qreg[c * 8 + 6], f3.x, fmaf(qreg[c * 8 + 7], f3.y, d1));
-          }
-        } else {
-          const uint4* src = reinterpret_cast<const uint4*>(ks_ + (size_t)j * rowb + qq * QD);
-#pragma unroll
-          for (int c = 0; c < QD / 16; ++c) {
-            const uint4 w = src[c];
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float f[4];
-              int8x4_to_float(ww[e], f);
-              d0 = fmaf(qreg[c * 16 + 4 * e + 0], f[0], d0);
-              d1 = fmaf(qreg[c * 16 + 4 * e + 1], f[1], d1);
-              d0 = fmaf(qreg[c * 16 + 4 * e + 2], f[2], d0);
-              d1 = fmaf(qreg[c * 16 + 4 * e + 3], f[3], d1);
-            }
-          }
+        for (int e = 0; e < 4; ++e) {
+          uint32_t af[4];
+          i8x4_to_h2x2(w0[e], af[0], af[2]);
+          i8x4_to_h2x2(w1[e], af[1], af[3]);
+          mma_f16(s, af, qb[4 * h + e][0], qb[4 * h + e][1]);
         }
       }
-      float sj = d0 + d1;
-      sj += __shfl_xor_sync(0xffffffffu, sj, 1);
-      sj += __shfl_xor_sync(0xffffffffu, sj, 2);
-      sc[ps] = j < cnt ? (a.kv_int8 ? sj * ksc[base + j] : sj) : -INFINITY;
-    }
-    // stage max, new running max, weights
-    float smax = sc[0];
+    } else {
 #pragma unroll
-    for (int ps = 1; ps < DS_KEYS / 32; ++ps) smax = fmaxf(smax, sc[ps]);
-    smax = warp_max(smax);
-    if (lane == 0) red[warp] = smax;
-    __syncthreads();
-    smax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-    const float m_new = fmaxf(m, smax);
-    const float alpha = m == -INFINITY ? 0.f : __expf(m - m_new);
-    float psum = 0.f;
-#pragma unroll
-    for (int ps = 0; ps < DS_KEYS / 32; ++ps) {
-      const int j = ps * 32 + (tid >> 2);
-      const float pj = j < cnt ? __expf(sc[ps] - m_new) : 0.f;
-      if (qq == 0) {
-        pw[j] = a.kv_int8 ? pj * (j < cnt ? vsc[base + j] : 0.f) : pj;   // INT8: V scale folded in
-        psum += pj;
+      for (int ks = 0; ks < T::KSTEP; ++ks) {
+        uint32_t af[4];
+        ldsm_x4(af, kb_ + 16 * ((2 * ks) ^ kmask));
+        mma_f16(s, af, qb[ks][0], qb[ks][1]);
       }
     }
-    psum = warp_sum(psum);
-    __syncthreads();   // pw visible; red free again
-    if (lane == 0) red[warp] = psum;
-    // P V: thread (g4, ks4) takes dims 4*g4 .. 4*g4+3 over keys ks4, ks4 + KS4, ...
-    {
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (!a.kv_int8) {
-        for (int j = ks4; j < cnt; j += KS4) {
-          const float w = pw[j];
-          const uint2 v = *reinterpret_cast<const uint2*>(vs_ + (size_t)j * rowb + g4 * 8);
-          const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
-          const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
-          s4[0] = fmaf(w, f0.x, s4[0]);
-          s4[1] = fmaf(w, f0.y, s4[1]);
-          s4[2] = fmaf(w, f1.x, s4[2]);
-          s4[3] = fmaf(w, f1.y, s4[3]);
-        }
-      } else {
-        for (int j = ks4; j < cnt; j += KS4) {
-          const float w = pw[j];
-          float f[4];
-          int8x4_to_float(*reinterpret_cast<const uint32_t*>(vs_ + (size_t)j * rowb + g4 * 4), f);
-          s4[0] = fmaf(w, f[0], s4[0]);
-          s4[1] = fmaf(w, f[1], s4[1]);
-          s4[2] = fmaf(w, f[2], s4[2]);
-          s4[3] = fmaf(w, f[3], s4[3]);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) acc4[c] = fmaf(acc4[c], alpha, s4[c]);
+    // online softmax over the warp's 16 keys (lanes t == 0)
+    float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+    if constexpr (I8) {   // the scale arrays are padded to whole stages: no bound check
+      ks0 = ksc[base + kw + g];
+      ks1 = ksc[base + kw + g + 8];
+      vs0 = vsc[base + kw + g];
+      vs1 = vsc[base + kw + g + 8];
     }
-    __syncthreads();   // red (sums) visible; the stage slot and pw may be reused
-    l = fmaf(l, alpha, (red[0] + red[1]) + (red[2] + red[3]));
+    const bool v0 = t == 0 && kw + g < cnt, v1 = t == 0 && kw + g + 8 < cnt;
+    const float x0 = v0 ? s[0] * csc * ks0 : -INFINITY;
+    const float x1 = v1 ? s[2] * csc * ks1 : -INFINITY;
+    float mx = fmaxf(x0, x1);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    const float m_new = fmaxf(m, mx);
+    const float alpha = m == -INFINITY ? 0.f : exp2f(m - m_new);
+    const float p0 = v0 ? exp2f(x0 - m_new) : 0.f;
+    const float p1 = v1 ? exp2f(x1 - m_new) : 0.f;
+    l = fmaf(l, alpha, p0 + p1);
+    if (__any_sync(0xffffffffu, m_new != m)) {
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        o[i][0] *= alpha;
+        o[i][2] *= alpha;
+      }
+    }
     m = m_new;
+    // P^T as the B operand (column 0: lanes g == 0 hold keys 2t, 2t+1 | 2t+8, 2t+9)
+    // (the scales past the stage's keys are stale: select, do not multiply)
+    const uint32_t hp = pack_half2(I8 ? (v0 ? p0 * vs0 : 0.f) : p0, I8 ? (v1 ? p1 * vs1 : 0.f) : p1);   // keys g | g + 8
+    const uint32_t pu = __shfl_sync(0xffffffffu, hp, 8 * t);       // keys 2t | 2t + 8
+    const uint32_t pv = __shfl_sync(0xffffffffu, hp, 8 * t + 4);   // keys 2t + 1 | 2t + 9
+    uint32_t pb0, pb1;
+    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(pb0) : "r"(pu), "r"(pv));
+    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(pb1) : "r"(pu), "r"(pv));
+    if (g != 0) pb0 = pb1 = 0u;
+    // O^T += V^T P^T
+    const uint32_t vb = v_addr + slot * (DS_KEYS * T::ROWV);
+    if constexpr (!I8) {
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        uint32_t af[4];
+        ldsm_x4_trans(af, vb + 16 * ((2 * i) ^ vmask));
+        mma_f16(o[i], af, pb0, pb1);
+      }
+    } else {
+      constexpr int NW = HD / 32;                // words of a V row per lane
+      uint32_t ra[4], rb[4], rc[4], rd[4];
+      if constexpr (NW == 4) {
+        lds128(ra, vb);
+        lds128(rb, vb + T::ROWV);
+        lds128(rc, vb + 8 * T::ROWV);
+        lds128(rd, vb + 9 * T::ROWV);
+      } else {
+        lds64(ra, vb);
+        lds64(rb, vb + T::ROWV);
+        lds64(rc, vb + 8 * T::ROWV);
+        lds64(rd, vb + 9 * T::ROWV);
+      }
+      // tile i, row g + 8h <-> byte 2i + h of the lane's chunk
+#pragma unroll
+      for (int i = 0; i < MT; ++i) {
+        const int w = i >> 1;
+        uint32_t af[4];
+        if (i & 1) {
+          af[0] = i8pair_to_h2<2>(ra[w], rb[w]);
+          af[1] = i8pair_to_h2<3>(ra[w], rb[w]);
+          af[2] = i8pair_to_h2<2>(rc[w], rd[w]);
+          af[3] = i8pair_to_h2<3>(rc[w], rd[w]);
+        } else {
+          af[0] = i8pair_to_h2<0>(ra[w], rb[w]);
+          af[1] = i8pair_to_h2<1>(ra[w], rb[w]);
+          af[2] = i8pair_to_h2<0>(rc[w], rd[w]);
+          af[3] = i8pair_to_h2<1>(rc[w], rd[w]);
+        }
+        mma_f16(o[i], af, pb0, pb1);
+      }
+    }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
-  // combine the key slices in slice order: dims of slice 0 first, then add
-  __shared__ float sl_s[KS4][HD];
+  __syncthreads();   // the stage ring is free: it holds the four warps' P V now
+  float (*wo)[HD] = reinterpret_cast<float (*)[HD]>(dsm);
+  // this warp's totals (lanes t == 0), then the four warps in order
+  l += __shfl_xor_sync(0xffffffffu, l, 4);
+  l += __shfl_xor_sync(0xffffffffu, l, 8);
+  l += __shfl_xor_sync(0xffffffffu, l, 16);
+  if (t == 0) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) sl_s[ks4][4 * g4 + c] = acc4[c];
-  __syncthreads();
-  float acc = 0.f;
-  if (tid < HD) {
-#pragma unroll
-    for (int q = 0; q < KS4; ++q) acc += sl_s[q][tid];
+    for (int i = 0; i < MT; ++i) {
+      const int d0 = I8 ? (HD / 8) * g + 2 * i : 16 * i + g;   // output row g of tile i
+      const int d1 = I8 ? d0 + 1 : d0 + 8;                     // and row g + 8
+      wo[warp][d0] = o[i][0];
+      wo[warp][d1] = o[i][2];
+    }
+    if (g == 0) {
+      wm[warp] = m;
+      wl[warp] = l;
+    }
   }
-  if (tid < HD) acc_s[0][tid] = acc;
-  if (tid == 0) {
-    stat_s[0] = nk > 0 ? m : -INFINITY;
-    stat_s[1] = nk > 0 ? l : 0.f;
+  __syncthreads();
+  if (tid < HD) {
+    const float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+    float acc = 0.f, L = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const float wt = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - M);
+      acc = fmaf(wo[w][tid], wt, acc);
+      L = fmaf(wl[w], wt, L);
+    }
+    acc_s[tid] = acc;
+    if (tid == 0) {
+      stat_s[0] = M;
+      stat_s[1] = L;
+    }
   }
   cl_sync();   // every CTA's statistics and P V are in its shared memory
-  if (crank == 0) {
-    float M = -INFINITY;
-    for (int r = 0; r < CL; ++r) M = fmaxf(M, cl_ld(&stat_s[0], (uint32_t)r));
-    for (int e = tid; e < HD; e += 128) {
-      float L = 0.f, o = 0.f;
-      for (int r = 0; r < CL; ++r) {
-        const float mr = cl_ld(&stat_s[0], (uint32_t)r);
-        const float w = mr == -INFINITY ? 0.f : __expf(mr - M);
-        L = fmaf(cl_ld(&stat_s[1], (uint32_t)r), w, L);
-        o = fmaf(cl_ld(&acc_s[0][e], (uint32_t)r), w, o);
+  if (crank == 0 && tid < HD) {
+    // all remote reads are issued before any is used
+    float mr[8], lr[8], ar[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < CL) {
+        mr[r] = cl_ld(&stat_s[0], (uint32_t)r);
+        lr[r] = cl_ld(&stat_s[1], (uint32_t)r);
+        ar[r] = cl_ld(&acc_s[tid], (uint32_t)r);
       }
-      a.out[(size_t)row * a.d + head * HD + e] = __float2half_rn(o / L);
     }
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < CL) M = fmaxf(M, mr[r]);
+    float L = 0.f, acc = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < CL) {
+        const float w = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
+        L = fmaf(lr[r], w, L);
+        acc = fmaf(ar[r], w, acc);
+      }
+    }
+    a.out[(size_t)row * a.d + head * HD + tid] = __float2half_rn(acc / L);
   }
   cl_sync();   // no CTA leaves while rank 0 still reads its shared memory
 }
@@ -632,41 +793,50 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
 }
 
 // Cluster size and staged rows per CTA of the cluster decode kernel for a
-// cache of max_ctx positions; 0 when the staged rows would not fit.
+// cache of max_ctx positions.
 static int decode_cluster_size(int max_ctx) {
   const int c = (max_ctx + 63) / 64;
   return c < 1 ? 1 : c > 8 ? 8 : c;
 }
-static size_t decode_cluster_smem(int max_ctx, int hd, bool int8, int* max_per) {
-  const int cl = decode_cluster_size(max_ctx);
-  *max_per = (max_ctx + cl - 1) / cl;
-  const size_t rowb = (size_t)hd * (int8 ? 1 : 2);
-  return 2 * (size_t)DS_STAGES * DS_KEYS * rowb + 2 * (size_t)*max_per * sizeof(float);
+template <int HD, bool I8>
+static size_t decode_tc_smem(int max_per) {
+  return (size_t)DecTc<HD, I8>::NST * DecTc<HD, I8>::STAGE_BYTES +
+         (I8 ? 2 * (size_t)max_per * sizeof(float) : 0);
+}
+constexpr size_t kDecodeSmemCap = 200 * 1024;
+
+template <int HD, bool I8>
+static cudaError_t launch_decode_tc(const DecodeAttnArgs& a, int cl, int max_per, cudaStream_t s) {
+  static bool attr_done = false;
+  if (!attr_done) {
+    const cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel<HD, I8>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)kDecodeSmemCap);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  dim3 grid(cl, a.H, a.rows);
+  return launch_pdl_cluster(attn_decode_tc_kernel<HD, I8>, grid, dim3(128),
+                            decode_tc_smem<HD, I8>(max_per), s, (unsigned)cl, a, cl, max_per);
 }
 
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
   if (a.hd != 128 && a.hd != 64)
     return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
-  int max_per = 0;
-  const size_t smem = decode_cluster_smem(a.max_ctx, a.hd, a.kv_int8 != 0, &max_per);
-  if (smem > 200 * 1024)
-    return set_error(TL_ERR_UNSUPPORTED, "decode attention: %zu bytes of shared memory", smem);
-  static bool attr_done = false;
-  if (!attr_done) {
-    TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-    TL_CUDA(cudaFuncSetAttribute(attn_decode_cluster_kernel<64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
-    attr_done = true;
-  }
   const int cl = decode_cluster_size(a.max_ctx);
-  dim3 grid(cl, a.H, a.rows);
-  cudaError_t e = a.hd == 128
-      ? launch_pdl_cluster(attn_decode_cluster_kernel<128>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per)
-      : launch_pdl_cluster(attn_decode_cluster_kernel<64>, grid, dim3(128), smem, s, (unsigned)cl, a, cl, max_per);
+  // keys per CTA at most, rounded up to whole stages (the scale arrays are read a stage at a time)
+  const int max_per = ((a.max_ctx + cl - 1) / cl + DS_KEYS - 1) / DS_KEYS * DS_KEYS;
+  const bool i8 = a.kv_int8 != 0;
+  const size_t smem = a.hd == 128 ? (i8 ? decode_tc_smem<128, true>(max_per) : decode_tc_smem<128, false>(max_per))
+                                  : (i8 ? decode_tc_smem<64, true>(max_per) : decode_tc_smem<64, false>(max_per));
+  if (smem > kDecodeSmemCap)
+    return set_error(TL_ERR_UNSUPPORTED, "decode attention: %zu bytes of shared memory", smem);
+  const cudaError_t e =
+      a.hd == 128 ? (i8 ? launch_decode_tc<128, true>(a, cl, max_per, s) : launch_decode_tc<128, false>(a, cl, max_per, s))
+                  : (i8 ? launch_decode_tc<64, true>(a, cl, max_per, s) : launch_decode_tc<64, false>(a, cl, max_per, s));
   if (e != cudaSuccess)
-    return set_error(TL_ERR_CUDA, "launch of attn_decode_cluster_kernel failed: %s", cudaGetErrorString(e));
+    return set_error(TL_ERR_CUDA, "launch of attn_decode_tc_kernel failed: %s", cudaGetErrorString(e));
   return ok();
 }
 }  // namespace tl
