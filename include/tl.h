@@ -186,6 +186,15 @@ tl_status tl_model_device_bytes(const tl_model* model, size_t* bytes);
 /* Enable (default) or disable CUDA-graph replay of the forward calls. */
 tl_status tl_model_set_graphs(tl_model* model, int enable);
 
+/* Decode attention splits each lane's context into min(8, ceil(max_ctx / 64))
+ * equal chunks (max_ctx of the cache) and merges them in a fixed order; one
+ * CTA streams `chunks_per_cta` consecutive chunks.  0 (the default) picks, per
+ * call, the fewest chunks per CTA that run all (row, head) pairs in the fewest
+ * waves on this GPU.  The result is bit-identical for every value: this is a
+ * tuning and testing knob.  Frees the model's captured graphs.
+ * Errors: TL_ERR_INVALID_ARG for a NULL model or a value outside [0, 8]. */
+tl_status tl_model_set_decode_chunks(tl_model* model, int chunks_per_cta);
+
 /* ------------------------------------------------------------------------
  * KV cache.  Every layer application keeps its own K/V slot: n_pre slots for
  * the pre-blocks and one per loop iteration ("Performance and Memory", "KV

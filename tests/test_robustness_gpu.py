@@ -1,7 +1,8 @@
 """Robustness of the library on the GPU: repeated create/destroy cycles leave
 no device memory behind, and randomised prefill/decode calls (shapes, depths,
 lanes, prompt lengths, cache dtypes and sizes drawn from a seeded generator)
-match the oracle, 50 randomised cases in all.  The pages list leak detection
+match the oracle, 50 randomised cases in all, and the decode attention's
+output does not depend on how many context chunks one CTA streams.  The pages list leak detection
 with zero growth and a 50-iteration fuzzing pass among their verification
 coverage ("Current Status", Verification Coverage list)."""
 import gc
@@ -101,3 +102,46 @@ def test_random_decode_matches_oracle(model, it):
     for b in range(n):
         assert kv.position(b) == prompts[b] + steps
     kv.close()
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "int8"])
+def test_decode_chunks_per_cta_bit_identical(dtype):
+    """Decode attention splits each lane's context into chunks fixed by the
+    cache size (a 512-position cache: 8) and merges them in a fixed order.
+    Whether a CTA streams 1, 2, 3 or all 8 chunks, or the count chosen per call,
+    every output is bit-identical, and it matches the oracle."""
+    m = device_model("tiny", max_tokens=512, max_lanes=3, max_ctx=512)
+    L_per_lane = [2, 1, 3]
+    prompts = [300, 17, 450]          # several stages per chunk, ragged ends
+    steps = 3
+    om = oracle_model("tiny")
+    xs = [syn.hidden_input(W, n, name=f"chunks.prompt.{b}") for b, n in enumerate(prompts)]
+    hs = [np.stack([syn.hidden_input(W, 1, name=f"chunks.step.{s}.{b}")[0] for b in range(3)])
+          for s in range(steps)]
+    outs = {}
+    try:
+        for chunks in (1, 2, 3, 8, 0):
+            m.set_decode_chunks(chunks)
+            kv = m.new_kv(L_per_lane, max_ctx=512, dtype=dtype)
+            for b in range(3):
+                m.prefill(h_in=to_dev(xs[b], torch.float16), L=L_per_lane[b], kv=kv, lane=b)
+            outs[chunks] = [m.decode(kv, h_in=to_dev(hs[s], torch.float16),
+                                     L_per_lane=L_per_lane).cpu() for s in range(steps)]
+            assert m.sync_status() == tl.TL_OK
+            kv.close()
+        for chunks in (2, 3, 8, 0):
+            for s in range(steps):
+                assert torch.equal(outs[chunks][s], outs[1][s]), (chunks, s)
+        okv = []
+        for b in range(3):
+            k = om.new_kv(L_per_lane[b], dtype)
+            om.prefill(xs[b].astype(np.float64), L_per_lane[b], kv=k)
+            okv.append(k)
+        for s in range(steps):
+            for b in range(3):
+                r = om.decode_step(hs[s][b].astype(np.float64), L_per_lane[b], okv[b])
+                y = outs[0][s][b].numpy()
+                assert cosine(y, r) >= FINAL_COSINE, (s, b)
+                assert rel_l2(y, r) <= 2 * BLOCK_REL_L2, (s, b)
+    finally:
+        m.close()

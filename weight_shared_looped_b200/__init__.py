@@ -67,6 +67,7 @@ _SIGS = {
     "tl_model_destroy": ([P], I),
     "tl_model_device_bytes": ([P, ctypes.POINTER(SZ)], I),
     "tl_model_set_graphs": ([P, I], I),
+    "tl_model_set_decode_chunks": ([P, I], I),
     "tl_kv_layer_bytes": ([I, I, I, I, ctypes.POINTER(SZ)], I),
     "tl_kv_bytes": ([P, I, I, P, I, ctypes.POINTER(SZ)], I),
     "tl_kv_create": ([P, I, I, P, I, P, SZ, ctypes.POINTER(P)], I),
@@ -189,6 +190,10 @@ def tl_model_device_bytes(model: int) -> int:
 
 def tl_model_set_graphs(model: int, enable: bool) -> None:
     _check(lib.tl_model_set_graphs(model, 1 if enable else 0))
+
+
+def tl_model_set_decode_chunks(model: int, chunks_per_cta: int) -> None:
+    _check(lib.tl_model_set_decode_chunks(model, chunks_per_cta))
 
 
 # --------------------------------------------------------------------- KV cache

@@ -81,6 +81,11 @@ struct tl_kv {
   size_t layer_bytes, region_bytes;
 };
 
+struct RowMap {
+  int lane[kMaxLanes];   // lane of each decode row
+  int cum[kMaxLanes];    // cache layers of the lanes before it
+};
+
 struct GraphEntry {
   cudaGraphExec_t exec = nullptr;
   int32_t* lane_of_row = nullptr;   // device, decode graphs
@@ -94,6 +99,7 @@ struct tl_model {
   int d, H, hd, F, Tmax;
   float eps;
   bool graphs = true;
+  int decode_chunks = 0;   // context chunks per decode-attention CTA; 0 = automatic
   cudaStream_t cap_stream = nullptr;
   // workspace
   void* ws = nullptr;
@@ -425,6 +431,15 @@ TL_API tl_status tl_model_set_graphs(tl_model* model, int enable) {
   return ok();
 }
 
+TL_API tl_status tl_model_set_decode_chunks(tl_model* model, int chunks_per_cta) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG(chunks_per_cta >= 0 && chunks_per_cta <= 8, "chunks_per_cta = %d out of [0, 8]",
+               chunks_per_cta);
+  model->decode_chunks = chunks_per_cta;
+  free_graphs(model);   // captured decode graphs hold the old launch shape
+  return ok();
+}
+
 // ============================================================================
 // KV cache
 // ============================================================================
@@ -635,7 +650,8 @@ NormArgs norm_args(const tl_model* m, int rows) {
 // including the down projection; the residual add of the down projection is
 // done by the next norm).  `rows` rows are active.
 tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
-                             int lane, bool decode, const int32_t* lane_of_row, cudaStream_t s) {
+                             int lane, bool decode, const int32_t* lane_of_row, const RowMap* rm,
+                             cudaStream_t s) {
   // QKV
   GemmArgs g = gemm_args(m, b, 0, m->x, rows);
   TL_TRY(launch_gemm(g, s));
@@ -680,10 +696,14 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
     da.layer = layer;
     da.max_ctx = kv->max_ctx;
     da.kv_int8 = kv->dtype == TL_KV_INT8;
-    da.lane_of_row = lane_of_row;
+    for (int i = 0; i < kMaxLanes; ++i) {
+      da.row_lane[i] = rm->lane[i];
+      da.row_cum[i] = rm->cum[i];
+    }
     da.qkv_part = m->part;
     da.qkv_S = g.splits;
     da.rope_cs = m->rope;
+    da.chunks = m->decode_chunks;
     TL_TRY(launch_attn_decode_fused(da, s));
   }
   // O projection, then the residual add of its split-K partial sums and the
@@ -745,7 +765,7 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
   TL_TRY(launch_residual_norm(n, s));
   for (int layer = 0; layer < n_layers; ++layer) {
     const tl_block* b = block_at(m, layer);
-    TL_TRY(enqueue_block_body(m, b, layer, seq, kv, lane, false, nullptr, s));
+    TL_TRY(enqueue_block_body(m, b, layer, seq, kv, lane, false, nullptr, nullptr, s));
     NormArgs en = norm_args(m, seq);
     en.part = m->part;
     en.part_rows = seq;
@@ -769,7 +789,8 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
 // rows are lanes sorted by L descending; active rows at loop iteration i are
 // those with L > i (a prefix).
 tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int* L_sorted,
-                         const int32_t* lane_of_row, float* trace, cudaStream_t s) {
+                         const int32_t* lane_of_row, const RowMap* rm, float* trace,
+                         cudaStream_t s) {
   const int n_pre = (int)m->pre.size();
   const int Lmax = L_sorted[0];
   const int n_layers = n_pre + Lmax;
@@ -799,7 +820,7 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
   for (int layer = 0; layer < n_layers; ++layer) {
     const int act = active(layer);
     const tl_block* b = block_at(m, layer);
-    TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, s));
+    TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, rm, s));
     const int nxt = layer + 1 < n_layers ? active(layer + 1) : 0;
     NormArgs en = norm_args(m, trace ? B : act);
     // the down projection's split-K partial sums are added into h here
@@ -919,6 +940,15 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
                    [&](int a, int b) { return L_per_lane[a] > L_per_lane[b]; });
   int L_sorted[kMaxLanes];
   for (int i = 0; i < n_lanes; ++i) L_sorted[i] = L_per_lane[order[i]];
+  // each row's lane and the cache layers before that lane (the cache header's
+  // cum_layers), passed to the attention kernel by value
+  RowMap rm;
+  for (int i = 0; i < kMaxLanes; ++i) {
+    rm.lane[i] = order[i];
+    int cum = 0;
+    for (int b = 0; b < order[i] && b < kv->n_lanes; ++b) cum += (int)model->pre.size() + kv->L[b];
+    rm.cum[i] = cum;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   const int d = model->d;
   if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)n_lanes * 4, cudaMemcpyDefault, s));
@@ -931,13 +961,14 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
     TL_TRY(run_graph(
         model, key, kv->id, s,
         [&](cudaStream_t cs, int32_t* lmap) {
-          return enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, lmap, h_trace, cs);
+          return enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, lmap, &rm, h_trace, cs);
         },
         order));
   } else {
     // without graphs the lane map lives in the model workspace
     TL_CUDA(cudaMemcpyAsync(model->lane_map, order, sizeof(order), cudaMemcpyHostToDevice, s));
-    TL_TRY(enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, model->lane_map, h_trace, s));
+    TL_TRY(enqueue_decode(model, kv, use_ids, n_lanes, L_sorted, model->lane_map, &rm, h_trace,
+                          s));
   }
   TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)n_lanes * d * 4, cudaMemcpyDefault, s));
   for (int b = 0; b < n_lanes; ++b) kv->pos[b] += 1;

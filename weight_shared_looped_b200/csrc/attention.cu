@@ -11,6 +11,9 @@
 // by a rule that depends only on the lane's position and the cache size, and
 // the partial results are merged in a fixed order, so a lane's output does not
 // depend on the other lanes.
+#include <algorithm>
+#include <map>
+
 #include "tl_launch.cuh"
 
 namespace tl {
@@ -350,7 +353,7 @@ __device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t wa, uint32_t wb) {
 
 template <int HD, bool I8>
 __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeAttnArgs a, int CL,
-                                                                       int sc_len) {
+                                                                       int F, int sc_len) {
   using T = DecTc<HD, I8>;
   constexpr int HALF = HD / 2;
   constexpr int MT = HD / 16;                    // P V m tiles of 16 head_dim elements
@@ -358,27 +361,30 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   __shared__ float qs[HD], kn[HD], vn[HD];
   __shared__ __align__(16) __half qh[HD];
   __shared__ float wm[4], wl[4];
-  __shared__ float acc_s[HD];
-  __shared__ float stat_s[2];
   __shared__ float kmax_s[4], vmax_s[4];
-  const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;
+  const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;   // crank: rank in the cluster
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   unsigned char* kst = dsm;                                          // [NST][DS_KEYS][ROWK]
   unsigned char* vst = dsm + (size_t)T::NST * DS_KEYS * T::ROWK;     // [NST][DS_KEYS][ROWV]
-  float* ksc = reinterpret_cast<float*>(dsm + (size_t)T::NST * T::STAGE_BYTES);   // [sc_len]
-  float* vsc = ksc + sc_len;
-  const int lane_id = a.lane_of_row[row];
+  __half* ksc = reinterpret_cast<__half*>(dsm + (size_t)T::NST * T::STAGE_BYTES);   // [sc_len]
+  __half* vsc = ksc + sc_len;
+  float* part = reinterpret_cast<float*>(vsc + sc_len);   // [F][HD + 2]: chunk P V, max, sum
+  // This CTA takes chunks crank*F .. crank*F + F - 1 of the CL equal chunks of
+  // the lane's context, i.e. the contiguous keys [kA, kB).  Each chunk is
+  // streamed in 64-key stages from its own start and folded into its own
+  // (P V, max, sum), exactly as if one CTA took each chunk.
+  const int lane_id = a.row_lane[row];
   const int pos = a.hdr->pos[lane_id];
   const int n_keys = pos + 1;
   const int per = (n_keys + CL - 1) / CL;
-  const int k0 = min(crank * per, n_keys), k1 = min(k0 + per, n_keys);
-  const int nk = k1 - k0;
-  const bool owner = nk > 0 && k1 == n_keys;
-  const int n_old = owner ? nk - 1 : nk;
-  const int nsub = (nk + DS_KEYS - 1) / DS_KEYS;
-  char* layer = const_cast<char*>(a.kv_base) +
-                (size_t)(a.hdr->cum_layers[lane_id] + a.layer) * a.layer_bytes;
+  const int kA = min(crank * F * per, n_keys), kB = min(kA + F * per, n_keys);
+  const int nkc = kB - kA;
+  const bool owner = nkc > 0 && kB == n_keys;
+  const int n_old = owner ? nkc - 1 : nkc;       // keys of [kA, kB) already cached
+  const int NSF = (per + DS_KEYS - 1) / DS_KEYS; // stages of a full chunk
+  const int nstage = nkc / per * NSF + (nkc % per + DS_KEYS - 1) / DS_KEYS;
+  char* layer = const_cast<char*>(a.kv_base) + (size_t)(a.row_cum[row] + a.layer) * a.layer_bytes;
   const size_t head_off = (size_t)head * a.max_ctx;
   const size_t scale_region = (a.layer_bytes - 2 * a.kv_region_bytes) / 2;
   // stage `sub` into ring slot sub % NST: cached rows are copied, rows past
@@ -390,18 +396,30 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   const int cr0 = tid / PIECES, cpc = tid % PIECES;
   const uint32_t kdst0 = (uint32_t)__cvta_generic_to_shared(kst) + cr0 * T::ROWK + 16 * T::kphys(cr0, cpc);
   const uint32_t vdst0 = (uint32_t)__cvta_generic_to_shared(vst) + cr0 * T::ROWV + 16 * T::vphys(cr0, cpc);
-  const char* ksrc0 = layer + (head_off + k0 + cr0) * (size_t)T::KB + 16 * cpc;
-  auto issue = [&](int sub) {
-    if (sub < nsub) {
-      const int slot = sub % T::NST;
+  const char* ksrc0 = layer + (head_off + kA + cr0) * (size_t)T::KB + 16 * cpc;
+  // stage s of the CTA: chunk s / NSF, its keys [lo, lo + cnt) relative to kA
+  auto stage_keys = [&](int s, int& lo, int& cnt, int& nkj) {
+    const int j = s / NSF, sub = s - j * NSF;
+    nkj = min(per, nkc - j * per);
+    lo = j * per + sub * DS_KEYS;
+    cnt = min(DS_KEYS, nkj - sub * DS_KEYS);
+  };
+  auto issue = [&](int s) {
+    if (s < nstage) {
+      int lo, cnt, nkj;
+      stage_keys(s, lo, cnt, nkj);
+      const int slot = s % T::NST;
       const uint32_t kd = kdst0 + slot * (DS_KEYS * T::ROWK);
       const uint32_t vd = vdst0 + slot * (DS_KEYS * T::ROWV);
-      const char* ks = ksrc0 + (size_t)sub * (DS_KEYS * T::KB);
+      const char* ks = ksrc0 + (size_t)lo * T::KB;
       const char* vs = ks + a.kv_region_bytes;
-      const int rem = n_old - sub * DS_KEYS - cr0;   // row cr0 + RPP*p is cached iff RPP*p < rem
+      // the new key (if in this stage) is row cr0 + rnew; row cr0 + RPP*p is
+      // cached iff RPP*p < rem
+      const int rnew = owner && n_old - lo < cnt ? n_old - lo - cr0 : -DS_KEYS;
+      const int rem = min(cnt, n_old - lo) - cr0;
 #pragma unroll
       for (int p = 0; p < PASSES; ++p) {
-        if (owner && RPP * p == rem) continue;       // the new key's row
+        if (RPP * p == rnew) continue;               // the new key's row
         const bool ok = RPP * p < rem;
         const uint32_t n = ok ? 16 : 0;
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(kd + p * RPP * T::ROWK),
@@ -419,9 +437,9 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   // the cached keys' scales, the RoPE pair and the QKV partial sums are all
   // requested before any of them is used (one round trip)
   constexpr int SCU = 4;                         // scale loads in flight per thread
-  const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes) + head_off + k0;
+  const __half* kq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes) + head_off + kA;
   const __half* vq = reinterpret_cast<const __half*>(layer + 2 * a.kv_region_bytes + scale_region) +
-                     head_off + k0;
+                     head_off + kA;
   __half ksr[SCU], vsr[SCU];
   if (I8) {
 #pragma unroll
@@ -469,15 +487,17 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
     for (int u = 0; u < SCU; ++u) {
       const int j = tid + 128 * u;
       if (j < n_old) {
-        ksc[j] = __half2float(ksr[u]);
-        vsc[j] = __half2float(vsr[u]);
+        ksc[j] = ksr[u];
+        vsc[j] = vsr[u];
       }
     }
     for (int j = tid + 128 * SCU; j < n_old; j += 128) {   // longer contexts
-      ksc[j] = __half2float(kq[j]);
-      vsc[j] = __half2float(vq[j]);
+      ksc[j] = kq[j];
+      vsc[j] = vq[j];
     }
   }
+  for (int i = tid; i < F * (HD + 2); i += 128)   // chunks without keys stay empty
+    part[i] = i % (HD + 2) == HD ? -INFINITY : 0.f;
   __syncthreads();
   float kr = 0.f;
   if (tid < HD) {
@@ -531,8 +551,8 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
       if (tid == 0) {
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes)[head_off + pos] = ksh;
         reinterpret_cast<__half*>(layer + 2 * a.kv_region_bytes + scale_region)[head_off + pos] = vsh;
-        ksc[n_old] = ksf;
-        vsc[n_old] = vsf;
+        ksc[n_old] = ksh;
+        vsc[n_old] = vsh;
       }
     }
   }
@@ -571,12 +591,12 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
     kmask = (lane >> 4) ^ (lane & 7);            // chunk 2ks + (l >> 4) is stored at 2ks ^ kmask
     vmask = ((lane >> 3) & 1) ^ (lane & 7);
   }
-  for (int sub = 0; sub < nsub; ++sub) {
+  for (int st = 0; st < nstage; ++st) {
     asm volatile("cp.async.wait_group %0;" ::"n"(T::NST - 2) : "memory");
-    const int slot = sub % T::NST;
-    const int base = sub * DS_KEYS;
-    const int cnt = min(DS_KEYS, nk - base);
-    if (owner && n_old >= base && n_old - base < DS_KEYS && tid < HD) {
+    const int slot = st % T::NST;
+    int base, cnt, nkj;
+    stage_keys(st, base, cnt, nkj);
+    if (owner && n_old >= base && n_old - base < cnt && tid < HD) {
       const int r = n_old - base;
       const int byte = tid * (I8 ? 1 : 2), c = byte >> 4, off = byte & 15;
       unsigned char* kd = kst + (size_t)slot * DS_KEYS * T::ROWK + (size_t)r * T::ROWK + 16 * T::kphys(r, c) + off;
@@ -589,174 +609,187 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
         *vd = (unsigned char)v_new;
       }
     }
-    __syncthreads();   // stage sub visible; every warp is done with stage sub - 1
-    issue(sub + T::NST - 1);                     // into the slot of stage sub - 1
-    if (kw >= cnt) continue;                     // no key of this warp in the stage
-    // S^T = K q^T: lane 4g ends with the scores of keys kw + g (s[0]) and kw + g + 8 (s[2])
-    float s[4] = {0.f, 0.f, 0.f, 0.f};
-    const uint32_t kb_ = k_addr + slot * (DS_KEYS * T::ROWK);
-    if constexpr (I8) {
+    __syncthreads();   // stage st visible; every warp is done with stage st - 1
+    issue(st + T::NST - 1);                      // into the slot of stage st - 1
+    if (kw < cnt) {                              // some key of this warp in the stage
+      // S^T = K q^T: lane 4g ends with the scores of keys kw + g (s[0]) and kw + g + 8 (s[2])
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint32_t kb_ = k_addr + slot * (DS_KEYS * T::ROWK);
+      if constexpr (I8) {
 #pragma unroll
-      for (int h = 0; h < T::NCH; ++h) {
-        const int ph = 16 * T::kphys(g, T::chunk(t, h));   // rows kw+g, kw+g+8: same parity
-        uint32_t w0[4], w1[4];
-        lds128(w0, kb_ + ph);
-        lds128(w1, kb_ + 8 * T::ROWK + ph);
+        for (int h = 0; h < T::NCH; ++h) {
+          const int ph = 16 * T::kphys(g, T::chunk(t, h));   // rows kw+g, kw+g+8: same parity
+          uint32_t w0[4], w1[4];
+          lds128(w0, kb_ + ph);
+          lds128(w1, kb_ + 8 * T::ROWK + ph);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t af[4];
-          i8x4_to_h2x2(w0[e], af[0], af[2]);
-          i8x4_to_h2x2(w1[e], af[1], af[3]);
-          mma_f16(s, af, qb[4 * h + e][0], qb[4 * h + e][1]);
+          for (int e = 0; e < 4; ++e) {
+            uint32_t af[4];
+            i8x4_to_h2x2(w0[e], af[0], af[2]);
+            i8x4_to_h2x2(w1[e], af[1], af[3]);
+            mma_f16(s, af, qb[4 * h + e][0], qb[4 * h + e][1]);
+          }
         }
-      }
-    } else {
-#pragma unroll
-      for (int ks = 0; ks < T::KSTEP; ++ks) {
-        uint32_t af[4];
-        ldsm_x4(af, kb_ + 16 * ((2 * ks) ^ kmask));
-        mma_f16(s, af, qb[ks][0], qb[ks][1]);
-      }
-    }
-    // online softmax over the warp's 16 keys (lanes t == 0)
-    float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
-    if constexpr (I8) {   // the scale arrays are padded to whole stages: no bound check
-      ks0 = ksc[base + kw + g];
-      ks1 = ksc[base + kw + g + 8];
-      vs0 = vsc[base + kw + g];
-      vs1 = vsc[base + kw + g + 8];
-    }
-    const bool v0 = t == 0 && kw + g < cnt, v1 = t == 0 && kw + g + 8 < cnt;
-    const float x0 = v0 ? s[0] * csc * ks0 : -INFINITY;
-    const float x1 = v1 ? s[2] * csc * ks1 : -INFINITY;
-    float mx = fmaxf(x0, x1);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-    const float m_new = fmaxf(m, mx);
-    const float alpha = m == -INFINITY ? 0.f : exp2f(m - m_new);
-    const float p0 = v0 ? exp2f(x0 - m_new) : 0.f;
-    const float p1 = v1 ? exp2f(x1 - m_new) : 0.f;
-    l = fmaf(l, alpha, p0 + p1);
-    if (__any_sync(0xffffffffu, m_new != m)) {
-#pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        o[i][0] *= alpha;
-        o[i][2] *= alpha;
-      }
-    }
-    m = m_new;
-    // P^T as the B operand (column 0: lanes g == 0 hold keys 2t, 2t+1 | 2t+8, 2t+9)
-    // (the scales past the stage's keys are stale: select, do not multiply)
-    const uint32_t hp = pack_half2(I8 ? (v0 ? p0 * vs0 : 0.f) : p0, I8 ? (v1 ? p1 * vs1 : 0.f) : p1);   // keys g | g + 8
-    const uint32_t pu = __shfl_sync(0xffffffffu, hp, 8 * t);       // keys 2t | 2t + 8
-    const uint32_t pv = __shfl_sync(0xffffffffu, hp, 8 * t + 4);   // keys 2t + 1 | 2t + 9
-    uint32_t pb0, pb1;
-    asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(pb0) : "r"(pu), "r"(pv));
-    asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(pb1) : "r"(pu), "r"(pv));
-    if (g != 0) pb0 = pb1 = 0u;
-    // O^T += V^T P^T
-    const uint32_t vb = v_addr + slot * (DS_KEYS * T::ROWV);
-    if constexpr (!I8) {
-#pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        uint32_t af[4];
-        ldsm_x4_trans(af, vb + 16 * ((2 * i) ^ vmask));
-        mma_f16(o[i], af, pb0, pb1);
-      }
-    } else {
-      constexpr int NW = HD / 32;                // words of a V row per lane
-      uint32_t ra[4], rb[4], rc[4], rd[4];
-      if constexpr (NW == 4) {
-        lds128(ra, vb);
-        lds128(rb, vb + T::ROWV);
-        lds128(rc, vb + 8 * T::ROWV);
-        lds128(rd, vb + 9 * T::ROWV);
       } else {
-        lds64(ra, vb);
-        lds64(rb, vb + T::ROWV);
-        lds64(rc, vb + 8 * T::ROWV);
-        lds64(rd, vb + 9 * T::ROWV);
-      }
-      // tile i, row g + 8h <-> byte 2i + h of the lane's chunk
 #pragma unroll
-      for (int i = 0; i < MT; ++i) {
-        const int w = i >> 1;
-        uint32_t af[4];
-        if (i & 1) {
-          af[0] = i8pair_to_h2<2>(ra[w], rb[w]);
-          af[1] = i8pair_to_h2<3>(ra[w], rb[w]);
-          af[2] = i8pair_to_h2<2>(rc[w], rd[w]);
-          af[3] = i8pair_to_h2<3>(rc[w], rd[w]);
-        } else {
-          af[0] = i8pair_to_h2<0>(ra[w], rb[w]);
-          af[1] = i8pair_to_h2<1>(ra[w], rb[w]);
-          af[2] = i8pair_to_h2<0>(rc[w], rd[w]);
-          af[3] = i8pair_to_h2<1>(rc[w], rd[w]);
+        for (int ks = 0; ks < T::KSTEP; ++ks) {
+          uint32_t af[4];
+          ldsm_x4(af, kb_ + 16 * ((2 * ks) ^ kmask));
+          mma_f16(s, af, qb[ks][0], qb[ks][1]);
         }
-        mma_f16(o[i], af, pb0, pb1);
       }
+      // online softmax over the warp's 16 keys (lanes t == 0)
+      float ks0 = 1.f, ks1 = 1.f, vs0 = 1.f, vs1 = 1.f;
+      if constexpr (I8) {   // the scale arrays are padded to whole stages: no bound check
+        ks0 = __half2float(ksc[base + kw + g]);
+        ks1 = __half2float(ksc[base + kw + g + 8]);
+        vs0 = __half2float(vsc[base + kw + g]);
+        vs1 = __half2float(vsc[base + kw + g + 8]);
+      }
+      const bool v0 = t == 0 && kw + g < cnt, v1 = t == 0 && kw + g + 8 < cnt;
+      const float x0 = v0 ? s[0] * csc * ks0 : -INFINITY;
+      const float x1 = v1 ? s[2] * csc * ks1 : -INFINITY;
+      float mx = fmaxf(x0, x1);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m, mx);
+      const float alpha = m == -INFINITY ? 0.f : exp2f(m - m_new);
+      const float p0 = v0 ? exp2f(x0 - m_new) : 0.f;
+      const float p1 = v1 ? exp2f(x1 - m_new) : 0.f;
+      l = fmaf(l, alpha, p0 + p1);
+      if (__any_sync(0xffffffffu, m_new != m)) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          o[i][0] *= alpha;
+          o[i][2] *= alpha;
+        }
+      }
+      m = m_new;
+      // P^T as the B operand (column 0: lanes g == 0 hold keys 2t, 2t+1 | 2t+8, 2t+9)
+      // (the scales past the stage's keys are stale: select, do not multiply)
+      const uint32_t hp = pack_half2(I8 ? (v0 ? p0 * vs0 : 0.f) : p0, I8 ? (v1 ? p1 * vs1 : 0.f) : p1);   // keys g | g + 8
+      const uint32_t pu = __shfl_sync(0xffffffffu, hp, 8 * t);       // keys 2t | 2t + 8
+      const uint32_t pv = __shfl_sync(0xffffffffu, hp, 8 * t + 4);   // keys 2t + 1 | 2t + 9
+      uint32_t pb0, pb1;
+      asm("prmt.b32 %0, %1, %2, 0x5410;" : "=r"(pb0) : "r"(pu), "r"(pv));
+      asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(pb1) : "r"(pu), "r"(pv));
+      if (g != 0) pb0 = pb1 = 0u;
+      // O^T += V^T P^T
+      const uint32_t vb = v_addr + slot * (DS_KEYS * T::ROWV);
+      if constexpr (!I8) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          uint32_t af[4];
+          ldsm_x4_trans(af, vb + 16 * ((2 * i) ^ vmask));
+          mma_f16(o[i], af, pb0, pb1);
+        }
+      } else {
+        constexpr int NW = HD / 32;                // words of a V row per lane
+        uint32_t ra[4], rb[4], rc[4], rd[4];
+        if constexpr (NW == 4) {
+          lds128(ra, vb);
+          lds128(rb, vb + T::ROWV);
+          lds128(rc, vb + 8 * T::ROWV);
+          lds128(rd, vb + 9 * T::ROWV);
+        } else {
+          lds64(ra, vb);
+          lds64(rb, vb + T::ROWV);
+          lds64(rc, vb + 8 * T::ROWV);
+          lds64(rd, vb + 9 * T::ROWV);
+        }
+        // tile i, row g + 8h <-> byte 2i + h of the lane's chunk
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          const int w = i >> 1;
+          uint32_t af[4];
+          if (i & 1) {
+            af[0] = i8pair_to_h2<2>(ra[w], rb[w]);
+            af[1] = i8pair_to_h2<3>(ra[w], rb[w]);
+            af[2] = i8pair_to_h2<2>(rc[w], rd[w]);
+            af[3] = i8pair_to_h2<3>(rc[w], rd[w]);
+          } else {
+            af[0] = i8pair_to_h2<0>(ra[w], rb[w]);
+            af[1] = i8pair_to_h2<1>(ra[w], rb[w]);
+            af[2] = i8pair_to_h2<0>(rc[w], rd[w]);
+            af[3] = i8pair_to_h2<1>(rc[w], rd[w]);
+          }
+          mma_f16(o[i], af, pb0, pb1);
+        }
+      }
+    }
+    if ((st - st / NSF * NSF + 1) * DS_KEYS >= nkj) {
+      // last stage of chunk st / NSF: the four warps' states are merged, in
+      // warp order, into the chunk's (P V, max, sum); the stage's K slot is
+      // free until the next iteration's barrier and holds the warp states
+      __syncthreads();
+      float (*wo)[HD] = reinterpret_cast<float (*)[HD]>(kst + (size_t)slot * DS_KEYS * T::ROWK);
+      float lw = l;
+      lw += __shfl_xor_sync(0xffffffffu, lw, 4);
+      lw += __shfl_xor_sync(0xffffffffu, lw, 8);
+      lw += __shfl_xor_sync(0xffffffffu, lw, 16);
+      if (t == 0) {
+#pragma unroll
+        for (int i = 0; i < MT; ++i) {
+          const int d0 = I8 ? (HD / 8) * g + 2 * i : 16 * i + g;   // output row g of tile i
+          const int d1 = I8 ? d0 + 1 : d0 + 8;                     // and row g + 8
+          wo[warp][d0] = o[i][0];
+          wo[warp][d1] = o[i][2];
+        }
+        if (g == 0) {
+          wm[warp] = m;
+          wl[warp] = lw;
+        }
+      }
+      __syncthreads();
+      if (tid < HD) {
+        const float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
+        float acc = 0.f, L = 0.f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float wt = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - M);
+          acc = fmaf(wo[w][tid], wt, acc);
+          L = fmaf(wl[w], wt, L);
+        }
+        float* pj = part + (st / NSF) * (HD + 2);
+        pj[tid] = acc;
+        if (tid == 0) {
+          pj[HD] = M;
+          pj[HD + 1] = L;
+        }
+      }
+      m = -INFINITY;
+      l = 0.f;
+#pragma unroll
+      for (int i = 0; i < MT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
     }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();   // the stage ring is free: it holds the four warps' P V now
-  float (*wo)[HD] = reinterpret_cast<float (*)[HD]>(dsm);
-  // this warp's totals (lanes t == 0), then the four warps in order
-  l += __shfl_xor_sync(0xffffffffu, l, 4);
-  l += __shfl_xor_sync(0xffffffffu, l, 8);
-  l += __shfl_xor_sync(0xffffffffu, l, 16);
-  if (t == 0) {
-#pragma unroll
-    for (int i = 0; i < MT; ++i) {
-      const int d0 = I8 ? (HD / 8) * g + 2 * i : 16 * i + g;   // output row g of tile i
-      const int d1 = I8 ? d0 + 1 : d0 + 8;                     // and row g + 8
-      wo[warp][d0] = o[i][0];
-      wo[warp][d1] = o[i][2];
-    }
-    if (g == 0) {
-      wm[warp] = m;
-      wl[warp] = l;
-    }
-  }
-  __syncthreads();
-  if (tid < HD) {
-    const float M = fmaxf(fmaxf(wm[0], wm[1]), fmaxf(wm[2], wm[3]));
-    float acc = 0.f, L = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float wt = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - M);
-      acc = fmaf(wo[w][tid], wt, acc);
-      L = fmaf(wl[w], wt, L);
-    }
-    acc_s[tid] = acc;
-    if (tid == 0) {
-      stat_s[0] = M;
-      stat_s[1] = L;
-    }
-  }
-  cl_sync();   // every CTA's statistics and P V are in its shared memory
+  cl_sync();   // every CTA's chunk results are in its shared memory
   if (crank == 0 && tid < HD) {
-    // all remote reads are issued before any is used
+    // chunk c sits in CTA c / F, slot c % F; all remote reads are issued
+    // before any is used, then the chunks are merged in order
     float mr[8], lr[8], ar[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (r < CL) {
-        mr[r] = cl_ld(&stat_s[0], (uint32_t)r);
-        lr[r] = cl_ld(&stat_s[1], (uint32_t)r);
-        ar[r] = cl_ld(&acc_s[tid], (uint32_t)r);
+    for (int c = 0; c < 8; ++c) {
+      if (c < CL) {
+        const float* pc = part + (c % F) * (HD + 2);
+        mr[c] = cl_ld(pc + HD, (uint32_t)(c / F));
+        lr[c] = cl_ld(pc + HD + 1, (uint32_t)(c / F));
+        ar[c] = cl_ld(pc + tid, (uint32_t)(c / F));
       }
     }
     float M = -INFINITY;
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-      if (r < CL) M = fmaxf(M, mr[r]);
+    for (int c = 0; c < 8; ++c)
+      if (c < CL) M = fmaxf(M, mr[c]);
     float L = 0.f, acc = 0.f;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      if (r < CL) {
-        const float w = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
-        L = fmaf(lr[r], w, L);
-        acc = fmaf(ar[r], w, acc);
+    for (int c = 0; c < 8; ++c) {
+      if (c < CL) {
+        const float w = mr[c] == -INFINITY ? 0.f : exp2f(mr[c] - M);
+        L = fmaf(lr[c], w, L);
+        acc = fmaf(ar[c], w, acc);
       }
     }
     a.out[(size_t)row * a.d + head * HD + tid] = __float2half_rn(acc / L);
@@ -792,51 +825,97 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   return ok();
 }
 
-// Cluster size and staged rows per CTA of the cluster decode kernel for a
-// cache of max_ctx positions.
+// Chunks of the decode split for a cache of max_ctx positions: ceil(max_ctx /
+// 64) capped at 8.  It depends on the cache alone, so a lane's arithmetic does
+// not depend on the batch; how many chunks one CTA takes (below) does not
+// change that arithmetic.
 static int decode_cluster_size(int max_ctx) {
   const int c = (max_ctx + 63) / 64;
   return c < 1 ? 1 : c > 8 ? 8 : c;
 }
 template <int HD, bool I8>
-static size_t decode_tc_smem(int max_per) {
+static size_t decode_tc_smem(int sc_len, int F) {
   return (size_t)DecTc<HD, I8>::NST * DecTc<HD, I8>::STAGE_BYTES +
-         (I8 ? 2 * (size_t)max_per * sizeof(float) : 0);
+         2 * (size_t)sc_len * sizeof(__half) + (size_t)F * (HD + 2) * sizeof(float);
 }
 constexpr size_t kDecodeSmemCap = 200 * 1024;
 
+// Clusters of `pc` CTAs of the decode kernel that fit on the GPU at once.
 template <int HD, bool I8>
-static cudaError_t launch_decode_tc(const DecodeAttnArgs& a, int cl, int max_per, cudaStream_t s) {
+static int decode_active_clusters(int pc, size_t smem) {
+  static std::map<std::pair<int, size_t>, int> cache;
+  auto it = cache.find({pc, smem});
+  if (it != cache.end()) return it->second;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pc, 1, 1);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = pc;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (const void*)attn_decode_tc_kernel<HD, I8>, &cfg) !=
+          cudaSuccess ||
+      n < 1) {
+    cudaGetLastError();
+    n = 1;
+  }
+  cache[{pc, smem}] = n;
+  return n;
+}
+
+template <int HD, bool I8>
+static tl_status launch_decode_tc(const DecodeAttnArgs& a, cudaStream_t s) {
   static bool attr_done = false;
   if (!attr_done) {
-    const cudaError_t e = cudaFuncSetAttribute(attn_decode_tc_kernel<HD, I8>,
-                                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kDecodeSmemCap);
-    if (e != cudaSuccess) return e;
+    TL_CUDA(cudaFuncSetAttribute(attn_decode_tc_kernel<HD, I8>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmemCap));
     attr_done = true;
   }
-  dim3 grid(cl, a.H, a.rows);
-  return launch_pdl_cluster(attn_decode_tc_kernel<HD, I8>, grid, dim3(128),
-                            decode_tc_smem<HD, I8>(max_per), s, (unsigned)cl, a, cl, max_per);
+  const int cl = decode_cluster_size(a.max_ctx);
+  const int max_per = (a.max_ctx + cl - 1) / cl;   // keys of a chunk at most
+  // chunks per CTA: the fewest that run every (row, head) cluster in the
+  // fewest waves
+  int best_f = 0, best_waves = 0;
+  size_t best_smem = 0;
+  int best_sc = 0;
+  for (int f = a.chunks > 0 ? std::min(a.chunks, cl) : 1; f <= cl; f *= 2) {
+    const int sc_len = I8 ? (f * max_per + DS_KEYS + 7) / 8 * 8 : 0;   // a stage past the last key
+    const size_t smem = decode_tc_smem<HD, I8>(sc_len, f);
+    if (smem > kDecodeSmemCap) break;
+    const int pc = (cl + f - 1) / f;
+    const int active = decode_active_clusters<HD, I8>(pc, smem);
+    const int waves = (a.rows * a.H + active - 1) / active;
+    if (best_f == 0 || waves < best_waves) {
+      best_f = f;
+      best_waves = waves;
+      best_smem = smem;
+      best_sc = sc_len;
+    }
+    if (a.chunks > 0) break;   // fixed by the caller
+  }
+  if (best_f == 0)
+    return set_error(TL_ERR_UNSUPPORTED, "decode attention: a cache of %d positions needs too much shared memory",
+                     a.max_ctx);
+  const int pc = (cl + best_f - 1) / best_f;
+  dim3 grid(pc, a.H, a.rows);
+  const cudaError_t e = launch_pdl_cluster(attn_decode_tc_kernel<HD, I8>, grid, dim3(128), best_smem, s,
+                                           (unsigned)pc, a, cl, best_f, best_sc);
+  if (e != cudaSuccess)
+    return set_error(TL_ERR_CUDA, "launch of attn_decode_tc_kernel failed: %s", cudaGetErrorString(e));
+  return ok();
 }
 
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s) {
   if (a.rows == 0) return ok();
-  if (a.hd != 128 && a.hd != 64)
-    return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
-  const int cl = decode_cluster_size(a.max_ctx);
-  // keys per CTA at most, rounded up to whole stages (the scale arrays are read a stage at a time)
-  const int max_per = ((a.max_ctx + cl - 1) / cl + DS_KEYS - 1) / DS_KEYS * DS_KEYS;
+  if (a.rows > kMaxLanes) return set_error(TL_ERR_INVALID_ARG, "decode attention: %d rows", a.rows);
   const bool i8 = a.kv_int8 != 0;
-  const size_t smem = a.hd == 128 ? (i8 ? decode_tc_smem<128, true>(max_per) : decode_tc_smem<128, false>(max_per))
-                                  : (i8 ? decode_tc_smem<64, true>(max_per) : decode_tc_smem<64, false>(max_per));
-  if (smem > kDecodeSmemCap)
-    return set_error(TL_ERR_UNSUPPORTED, "decode attention: %zu bytes of shared memory", smem);
-  const cudaError_t e =
-      a.hd == 128 ? (i8 ? launch_decode_tc<128, true>(a, cl, max_per, s) : launch_decode_tc<128, false>(a, cl, max_per, s))
-                  : (i8 ? launch_decode_tc<64, true>(a, cl, max_per, s) : launch_decode_tc<64, false>(a, cl, max_per, s));
-  if (e != cudaSuccess)
-    return set_error(TL_ERR_CUDA, "launch of attn_decode_tc_kernel failed: %s", cudaGetErrorString(e));
-  return ok();
+  if (a.hd == 128) return i8 ? launch_decode_tc<128, true>(a, s) : launch_decode_tc<128, false>(a, s);
+  if (a.hd == 64) return i8 ? launch_decode_tc<64, true>(a, s) : launch_decode_tc<64, false>(a, s);
+  return set_error(TL_ERR_UNSUPPORTED, "head_dim %d not supported", a.hd);
 }
 }  // namespace tl

@@ -170,7 +170,9 @@ struct DecodeAttnArgs {
   const KvHeader* hdr;
   size_t layer_bytes, kv_region_bytes;
   int layer, max_ctx, kv_int8;
-  const int32_t* lane_of_row;
+  int row_lane[kMaxLanes];   // lane of each row
+  int row_cum[kMaxLanes];    // cache layers of the lanes before that lane
+  int chunks;                // context chunks per CTA; 0 = fewest waves
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
 

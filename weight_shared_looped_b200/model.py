@@ -12,8 +12,8 @@ import torch
 from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_decode_step,
                tl_kv_bytes, tl_kv_create, tl_kv_destroy, tl_kv_layer_ptrs, tl_kv_position,
                tl_kv_reset, tl_kv_set_position, tl_model_create, tl_model_destroy,
-               tl_model_device_bytes, tl_model_set_graphs, tl_pack_weights, tl_packed_bytes,
-               tl_prefill, tl_sync_status)
+               tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
+               tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status)
 
 MATRICES = ("qkv", "o", "gate", "up", "down")
 
@@ -79,6 +79,10 @@ class DeviceModel:
 
     def set_graphs(self, on: bool) -> None:
         tl_model_set_graphs(self.handle, on)
+
+    def set_decode_chunks(self, chunks_per_cta: int) -> None:
+        """Context chunks one decode-attention CTA streams (0 = automatic)."""
+        tl_model_set_decode_chunks(self.handle, chunks_per_cta)
 
     def new_kv(self, L_per_lane: Sequence[int], max_ctx: int, dtype: str = "fp16") -> "DeviceKV":
         return DeviceKV(self, L_per_lane, max_ctx, dtype)
