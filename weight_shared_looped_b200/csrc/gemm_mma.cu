@@ -165,20 +165,30 @@ __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
 // B use the same one, so each lane owns two whole packed words (16 k) of its
 // two rows per 64-wide chunk: lane (g, t) loads words 2t and 2t+1 of rows g
 // and g+8 (8 distinct bytes each, no duplicate loads).  A word's nibble pairs
-// (i, i+4) come out of one lop3 each after a shift: (w >> 4i) & 0x000F000F |
-// 0x6400_6400 is the fp16 pair (1024 + u_i, 1024 + u_{i+4}), and one HSUB2 of
-// 1032 leaves the exact codes.  The activations are staged once per CTA with
+// (i, i+4) come out of one lop3 each: w & 0x000F000F | 0x6400_6400 is the fp16
+// pair (1024 + u_0, 1024 + u_4), less 1032 the exact codes; w & 0x00F000F0 |
+// 0x6400_6400 is (1024 + 16 u_1, 1024 + 16 u_5), and one HFMA2 (x / 16 - 72)
+// gives those codes exactly; w >> 8 yields pairs (2, 6) and (3, 7) the same
+// way (one shift per word).  The activations are staged once per CTA with
 // every 8-k group stored in the order 0 4 1 5 2 6 3 7, so the matching B pairs
 // are adjacent and one 8-byte shared load feeds a k step.
 constexpr int GV_ROWS = 128;      // 8 warps x 16 rows
 constexpr int GV_THREADS = 256;
 constexpr int GV_BATCH = 8;       // 64-k chunks loaded ahead per batch
 
-__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {
+__device__ __forceinline__ uint32_t nib_pair(uint32_t w) {   // nibbles 0 and 4
   uint32_t h;
   asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(w), "r"(0x000F000Fu), "r"(0x64006400u));
   __half2 r = __hsub2(*reinterpret_cast<__half2*>(&h),
                       __halves2half2(__float2half_rn(1032.0f), __float2half_rn(1032.0f)));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t nib_pair_hi(uint32_t w) {   // nibbles 1 and 5
+  uint32_t h;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(w), "r"(0x00F000F0u), "r"(0x64006400u));
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&h),
+                      __halves2half2(__float2half_rn(0.0625f), __float2half_rn(0.0625f)),
+                      __halves2half2(__float2half_rn(-72.0f), __float2half_rn(-72.0f)));
   return *reinterpret_cast<uint32_t*>(&r);
 }
 
@@ -288,8 +298,8 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
         uint32_t A[4];
         A[0] = nib_pair(w0 >> sh);
         A[1] = nib_pair(w1 >> sh);
-        A[2] = nib_pair(w0 >> (sh + 4));
-        A[3] = nib_pair(w1 >> (sh + 4));
+        A[2] = nib_pair_hi(w0 >> sh);
+        A[3] = nib_pair_hi(w1 >> sh);
         const uint2 bx =
             *reinterpret_cast<const uint2*>(xs + g * xstride + c * KC + 16 * t + 4 * j);
         mma16816(cacc, A, bx.x, bx.y);
