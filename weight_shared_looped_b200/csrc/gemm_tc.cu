@@ -185,10 +185,12 @@ __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
       : "memory");
 }
 
-// 80 registers x 608 threads leave room in the register file for a CTA of the
-// next (or previous) small kernel on the same SM while this one runs.
+// 96 registers x 608 threads (58 K of the 64 K register file) still leave
+// room for a small CTA of the next or previous kernel on the same SM; at 80
+// the compiler schedules the weight loads less freely (gate|up 4% slower),
+// and more registers or a third register set of weights gain nothing.
 template <int BN>
-__global__ void __maxnreg__(80)
+__global__ void __maxnreg__(96)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x, TcArgs a) {
   constexpr int XS = TcCfg<BN>::X_STAGES;
   constexpr int AB = TcCfg<BN>::A_BATCHES;
