@@ -243,15 +243,16 @@ __global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const _
 }
 
 // ------------------------------------------------------------------ decode (cluster)
-// Decode attention for one (row, head) on a thread-block cluster of CL CTAs
-// (CL = ceil(max_ctx / 64) capped at 8, fixed per cache).  CTA r takes the
-// contiguous keys [r * per, (r + 1) * per) of the lane's n_keys = pos + 1
-// (per = ceil(n_keys / CL), which depends only on the lane's own position);
-// its cached K/V rows are copied into shared memory before the wait for the
-// QKV projection.  The CTA holding position pos forms k and v from the QKV
-// partial sums, applies RoPE to k and appends both to the cache.  Each CTA
-// keeps its max score, exponential sum and unnormalised P V; rank 0 merges
-// the CTAs in rank order through distributed shared memory.
+// Decode attention for one (row, head) on a thread-block cluster.  The lane's
+// n_keys = pos + 1 keys are split into CL = min(8, ceil(max_ctx / 64)) chunks
+// (fixed per cache) of per = ceil(n_keys / CL) contiguous keys, which depends
+// only on the lane's own position; a CTA of the cluster streams F consecutive
+// chunks (F chosen at launch, the arithmetic being the same for every F), its
+// first cached K/V rows copied into shared memory before the wait for the QKV
+// projection.  The CTA holding position pos forms k and v from the QKV
+// partial sums, applies RoPE to k and appends both to the cache.  Each chunk
+// ends with its max score, exponential sum and unnormalised P V; rank 0
+// merges the chunks in order through distributed shared memory.
 __device__ __forceinline__ void cl_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
                    "memory");
