@@ -13,6 +13,7 @@
 // depend on the other lanes.
 #include <algorithm>
 #include <map>
+#include <mutex>
 
 #include "tl_launch.cuh"
 
@@ -844,7 +845,9 @@ constexpr size_t kDecodeSmemCap = 200 * 1024;
 // Clusters of `pc` CTAs of the decode kernel that fit on the GPU at once.
 template <int HD, bool I8>
 static int decode_active_clusters(int pc, size_t smem) {
+  static std::mutex mu;
   static std::map<std::pair<int, size_t>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
   auto it = cache.find({pc, smem});
   if (it != cache.end()) return it->second;
   cudaLaunchConfig_t cfg = {};
