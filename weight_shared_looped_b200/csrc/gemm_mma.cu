@@ -203,20 +203,30 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
   const int krange = per * KC;
   const int xstride = krange + 4;             // halves; row stride = 2 (mod 32) words
   __half* xs = gv_smem;                       // [8][xstride], k-permuted
-  const int gpr = a.K / a.G;
-  const int g_lo = (c0 * KC) / a.G;
-  const int n_groups = (krange + a.G - 1) / a.G + 1;
+  const int gsh = __ffs(a.G) - 1;            // the group size is 64 or 128
+  const int gpr = a.K >> gsh;
+  const int g_lo = (c0 * KC) >> gsh;
+  const int n_groups = ((krange + a.G - 1) >> gsh) + 1;
   __half* ss = xs + 8 * xstride;              // [128][n_groups] scales of this CTA
 
   // Weights and scales are constants of the model: stage the scales and issue
   // the first batch of weight loads before waiting for the previous kernel, so
-  // their latency overlaps its tail.
-  for (int i = threadIdx.x; i < GV_ROWS * n_groups; i += GV_THREADS) {
-    const int r = i / n_groups, gg = i % n_groups;
-    const int row = m0 + r;
-    const __half* sp = row < a.n_split ? a.s0 + (size_t)row * gpr
-                                       : a.s1 + (size_t)(row - a.n_split) * gpr;
-    ss[i] = g_lo + gg < gpr ? sp[g_lo + gg] : __float2half_rn(0.f);
+  // their latency overlaps its tail.  (Loops are laid out so that no index
+  // needs an integer division.)
+  constexpr int SROWS = GV_ROWS / (GV_THREADS / 32);   // rows per warp
+  for (int g0 = 0; g0 < n_groups; g0 += 32) {
+    const int gg = g0 + lane;
+    __half sv[SROWS];
+#pragma unroll
+    for (int k = 0; k < SROWS; ++k) {       // all loads in flight before any store
+      const int row = m0 + warp + k * (GV_THREADS / 32);
+      const __half* sp = row < a.n_split ? a.s0 + (size_t)row * gpr
+                                         : a.s1 + (size_t)(row - a.n_split) * gpr;
+      sv[k] = gg < n_groups && g_lo + gg < gpr ? sp[g_lo + gg] : __float2half_rn(0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < SROWS; ++k)
+      if (gg < n_groups) ss[(warp + k * (GV_THREADS / 32)) * n_groups + gg] = sv[k];
   }
   const int rowA = m0 + warp * 16 + g;
   const uint2* wr[2];
@@ -236,12 +246,33 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
   }
   pdl_enter();   // the activations below come from the previous kernel
 
-  // stage x (rows >= T are zero), permuting each 8-k group to 0 4 1 5 2 6 3 7
-  for (int i = threadIdx.x; i < 8 * (krange / 8); i += GV_THREADS) {
-    const int r = i / (krange / 8), q = i % (krange / 8);
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (r < a.T) {
-      if (a.x_part) {
+  // stage x (rows >= T are zero), permuting each 8-k group to 0 4 1 5 2 6 3 7;
+  // item i is token row i / Q, 8-k group i % Q
+  const int Q = krange / 8, n_items = 8 * Q;
+  const int qsh = (Q & (Q - 1)) == 0 ? __ffs(Q) - 1 : -1;
+  auto item = [&](int i, int& r, int& q) {
+    if (qsh >= 0) {
+      r = i >> qsh;
+      q = i & (Q - 1);
+    } else {
+      r = i / Q;
+      q = i - r * Q;
+    }
+  };
+  auto put = [&](int r, int q, uint4 v) {
+    const __half* e = reinterpret_cast<const __half*>(&v);
+    __half2 p0 = __halves2half2(e[0], e[4]), p1 = __halves2half2(e[1], e[5]);
+    __half2 p2 = __halves2half2(e[2], e[6]), p3 = __halves2half2(e[3], e[7]);
+    uint2* d = reinterpret_cast<uint2*>(xs + r * xstride + q * 8);   // 8-byte aligned
+    d[0] = make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
+    d[1] = make_uint2(*reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+  };
+  if (a.x_part) {
+    for (int i = threadIdx.x; i < n_items; i += GV_THREADS) {
+      int r, q;
+      item(i, r, q);
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (r < a.T) {
         // SwiGLU of the gate|up partial sums, rounded to fp16 like the unfused path
         __half hv[8];
         const size_t stride = (size_t)a.T * 2 * a.x_F;
@@ -256,16 +287,30 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
           hv[e] = __float2half_rn(gs / (1.0f + __expf(-gs)) * us);
         }
         v = *reinterpret_cast<const uint4*>(hv);
-      } else {
-        v = *reinterpret_cast<const uint4*>(a.x + (size_t)r * a.K + c0 * KC + q * 8);
       }
+      put(r, q, v);
     }
-    const __half* e = reinterpret_cast<const __half*>(&v);
-    __half2 p0 = __halves2half2(e[0], e[4]), p1 = __halves2half2(e[1], e[5]);
-    __half2 p2 = __halves2half2(e[2], e[6]), p3 = __halves2half2(e[3], e[7]);
-    uint2* d = reinterpret_cast<uint2*>(xs + r * xstride + q * 8);   // 8-byte aligned
-    d[0] = make_uint2(*reinterpret_cast<uint32_t*>(&p0), *reinterpret_cast<uint32_t*>(&p1));
-    d[1] = make_uint2(*reinterpret_cast<uint32_t*>(&p2), *reinterpret_cast<uint32_t*>(&p3));
+  } else {
+    // four items per thread at a time, all loads in flight before any store
+    for (int i0 = threadIdx.x; i0 < n_items; i0 += 4 * GV_THREADS) {
+      uint4 v[4];
+      int rr[4], qq[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * GV_THREADS;
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+        rr[u] = 0;
+        qq[u] = 0;
+        if (i < n_items) {
+          item(i, rr[u], qq[u]);
+          if (rr[u] < a.T)
+            v[u] = *reinterpret_cast<const uint4*>(a.x + (size_t)rr[u] * a.K + c0 * KC + qq[u] * 8);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (i0 + u * GV_THREADS < n_items) put(rr[u], qq[u], v[u]);
+    }
   }
   const __half* srow0 = ss + (warp * 16 + g) * n_groups;
   const __half* srow1 = srow0 + 8 * n_groups;
@@ -304,8 +349,9 @@ __global__ void __launch_bounds__(GV_THREADS) gemv_w4_kernel(GemmArgs a) {
             *reinterpret_cast<const uint2*>(xs + g * xstride + c * KC + 16 * t + 4 * j);
         mma16816(cacc, A, bx.x, bx.y);
       }
-      const float s0 = __half2float(srow0[((c0 + c) * KC) / a.G - g_lo]);
-      const float s1 = __half2float(srow1[((c0 + c) * KC) / a.G - g_lo]);
+      const int sidx = (((c0 + c) * KC) >> gsh) - g_lo;
+      const float s0 = __half2float(srow0[sidx]);
+      const float s1 = __half2float(srow1[sidx]);
       acc[0] = fmaf(cacc[0], s0, acc[0]);
       acc[1] = fmaf(cacc[1], s0, acc[1]);
       acc[2] = fmaf(cacc[2], s1, acc[2]);
