@@ -60,7 +60,8 @@ __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
   const int c_begin = blockIdx.z * per_split;
   const int c_end = c_begin + per_split;
   const int wpr = a.K / 8;
-  const int gpr = a.K / a.G;
+  const int gsh = __ffs(a.G) - 1;             // the group size is 64 or 128
+  const int gpr = a.K >> gsh;
 
   const uint32_t* wr[2];
   const __half* sr[2];
@@ -112,8 +113,8 @@ __global__ void __launch_bounds__(THREADS) gemm_w4_mma_kernel(GemmArgs a) {
         nxt[r][1] = __ldg(p + 1);
       }
     }
-    const float s0 = __half2float(sr[0][(c * KC) / a.G]);
-    const float s1 = __half2float(sr[1][(c * KC) / a.G]);
+    const float s0 = __half2float(sr[0][(c * KC) >> gsh]);
+    const float s1 = __half2float(sr[1][(c * KC) >> gsh]);
     __syncthreads();
 
     float cacc[NT / 8][4];

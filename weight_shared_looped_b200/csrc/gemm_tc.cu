@@ -326,7 +326,8 @@ __global__ void __maxnreg__(96)
     const int r = quad * 32 + lane;             // weight row within the tile = TMEM lane
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     // this thread's weight row (canonical INT4 words) and scale row
-    const size_t wpr = (size_t)a.K / 8, gpr = (size_t)a.K / a.G;
+    const int gsh = __ffs(a.G) - 1;             // the group size is 64 or 128
+    const size_t wpr = (size_t)a.K / 8, gpr = (size_t)a.K >> gsh;
     const uint32_t* wrow;
     const __half* srow;
     if (sw) {
@@ -350,7 +351,7 @@ __global__ void __maxnreg__(96)
         const uint4* p = reinterpret_cast<const uint4*>(wrow + (size_t)(kb_begin + i) * (BK / 8));
         wa = __ldg(p);
         wb = __ldg(p + 1);
-        sc = __ldg(srow + ((kb_begin + i) * BK) / a.G);
+        sc = __ldg(srow + (((kb_begin + i) * BK) >> gsh));
       }
     };
     fetch(grp, wa0, wb0, sc0);
