@@ -400,16 +400,21 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   const uint32_t vdst0 = (uint32_t)__cvta_generic_to_shared(vst) + cr0 * T::ROWV + 16 * T::vphys(cr0, cpc);
   const char* ksrc0 = layer + (head_off + kA + cr0) * (size_t)T::KB + 16 * cpc;
   // stage s of the CTA: chunk s / NSF, its keys [lo, lo + cnt) relative to kA
-  auto stage_keys = [&](int s, int& lo, int& cnt, int& nkj) {
-    const int j = s / NSF, sub = s - j * NSF;
+  auto stage_keys = [&](int s, int& lo, int& cnt, int& nkj, int& j) {
+    int sub = s;                                 // j = s / NSF, sub = s % NSF (F <= 8 steps)
+    j = 0;
+    while (sub >= NSF) {
+      sub -= NSF;
+      ++j;
+    }
     nkj = min(per, nkc - j * per);
     lo = j * per + sub * DS_KEYS;
     cnt = min(DS_KEYS, nkj - sub * DS_KEYS);
   };
   auto issue = [&](int s) {
     if (s < nstage) {
-      int lo, cnt, nkj;
-      stage_keys(s, lo, cnt, nkj);
+      int lo, cnt, nkj, j;
+      stage_keys(s, lo, cnt, nkj, j);
       const int slot = s % T::NST;
       const uint32_t kd = kdst0 + slot * (DS_KEYS * T::ROWK);
       const uint32_t vd = vdst0 + slot * (DS_KEYS * T::ROWV);
@@ -596,8 +601,8 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   for (int st = 0; st < nstage; ++st) {
     asm volatile("cp.async.wait_group %0;" ::"n"(T::NST - 2) : "memory");
     const int slot = st % T::NST;
-    int base, cnt, nkj;
-    stage_keys(st, base, cnt, nkj);
+    int base, cnt, nkj, jc;
+    stage_keys(st, base, cnt, nkj, jc);
     if (owner && n_old >= base && n_old - base < cnt && tid < HD) {
       const int r = n_old - base;
       const int byte = tid * (I8 ? 1 : 2), c = byte >> 4, off = byte & 15;
@@ -720,8 +725,8 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
         }
       }
     }
-    if ((st - st / NSF * NSF + 1) * DS_KEYS >= nkj) {
-      // last stage of chunk st / NSF: the four warps' states are merged, in
+    if (base + cnt - jc * per == nkj) {
+      // last stage of chunk jc: the four warps' states are merged, in
       // warp order, into the chunk's (P V, max, sum); the stage's K slot is
       // free until the next iteration's barrier and holds the warp states
       __syncthreads();
@@ -753,7 +758,7 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
           acc = fmaf(wo[w][tid], wt, acc);
           L = fmaf(wl[w], wt, L);
         }
-        float* pj = part + (st / NSF) * (HD + 2);
+        float* pj = part + jc * (HD + 2);
         pj[tid] = acc;
         if (tid == 0) {
           pj[HD] = M;
