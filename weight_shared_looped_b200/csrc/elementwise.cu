@@ -235,7 +235,6 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
 #pragma unroll
   for (int p = 0; p < 2; ++p) {
     if (p < npair) {
-      int i = lane + 32 * p;
       const float2 cs = csp[p];
       float q0 = q[p][0], q1 = q[p][1], k0 = k[p][0], k1 = k[p][1];
       q[p][0] = q0 * cs.x - q1 * cs.y;
