@@ -357,10 +357,12 @@ tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s) {
   // d = 256 * 2^k: d / 8 threads (32 .. 1024)
   if (a.d < 256 || a.d > 8192 || (a.d & (a.d - 1)) != 0)
     return set_error(TL_ERR_UNSUPPORTED, "d_model %d: the norm needs a power of two in [256, 8192]", a.d);
-  // up to 2048 columns: 256 threads with registers for eight splits in flight
-  // (more would keep the CTA from fitting next to a GEMM CTA); wider rows:
-  // four splits at a time
-  if (a.d <= 2048)
+  // up to 2048 columns: 256 threads with eight splits in flight, or sixteen
+  // for the prefill projections' 9-16 splits (one round trip instead of two;
+  // at decode the larger kernel measured slower); wider rows: four at a time
+  if (a.d <= 2048 && a.rows > 8 && a.S > 8 && a.S <= 16)
+    TL_LAUNCH_PDL((residual_norm_kernel<256, 16>), a.rows, a.d / 8, 0, s, a);
+  else if (a.d <= 2048)
     TL_LAUNCH_PDL((residual_norm_kernel<256, 8>), a.rows, a.d / 8, 0, s, a);
   else
     TL_LAUNCH_PDL((residual_norm_kernel<1024, 4>), a.rows, a.d / 8, 0, s, a);
