@@ -269,9 +269,9 @@ __device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
 constexpr int DS_KEYS = 64;     // keys per stage of the decode kernel
 
 // ------------------------------------------------------------------ decode (tensor cores)
-// Within a CTA both products run on the tensor cores (mma.sync m16n8k16, fp16 in, fp32 accumulate) in transposed
-// form, so that the single query fills the N = 8 side and keys or head_dim
-// elements fill all 16 rows:
+// Within a CTA both products run on the tensor cores (mma.sync m16n8k16,
+// fp16 in, fp32 accumulate) in transposed form, so that the single query fills
+// the N = 8 side and keys or head_dim elements fill all 16 rows:
 //   S^T = K q^T : A = 16 keys x 16 head_dim elements, B = q (column 0)
 //   O^T = V^T P^T : A = 16 head_dim elements x 16 keys, B = p (column 0)
 // In each 64-key stage warp w owns keys 16w..16w+15.  FP16 K and V tiles
@@ -282,8 +282,8 @@ constexpr int DS_KEYS = 64;     // keys per stage of the decode kernel
 // used for q and for the output columns.  The scores of a warp sit in lanes
 // 4g (keys g and g + 8); the weights reach the P V B operand through two
 // shuffles.  Each warp keeps its own running max and sum (base 2); the four
-// warps merge at the end, then rank 0 of the cluster merges the CTAs in rank
-// order.
+// warps merge at the end of every chunk, then rank 0 of the cluster merges the
+// chunks in order.
 constexpr int DT_STAGES_I8 = 3;    // stage ring of the tensor-core decode kernel, INT8 cache
 constexpr int DT_STAGES_F16 = 2;   // and FP16 cache (twice the bytes per stage)
 
