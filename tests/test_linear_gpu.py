@@ -37,6 +37,8 @@ def _run(words, scales, x, N, K, group):
 @pytest.mark.parametrize("N,K,T,group", [
     (64, 64, 1, 64), (128, 256, 8, 64), (256, 2048, 5, 128), (6144, 2048, 3, 128),
     (2048, 8192, 8, 128), (768, 256, 37, 64), (1536, 256, 16, 64),
+    # chunk counts that are not powers of two (3 and 5 chunks of 64 k; odd scale groups per row)
+    (128, 192, 3, 64), (256, 320, 8, 64),
 ])
 def test_linear_mma_kernel(N, K, T, group):
     words, scales, x, ref = _case(N, K, T, group, seed=N + K + T)
