@@ -204,6 +204,14 @@ def test_invalid_calls_rejected_before_launch(model):
     assert kv.position(0) == 4
     with pytest.raises(tl.TLError):
         model.decode(kv, h_in=x[:1], L_per_lane=[0])
+    with pytest.raises(tl.TLError) as e:
+        model.prefill(h_in=x[:0], L=1)                        # empty prompt
+    assert e.value.status == tl.TL_ERR_INVALID_ARG
+    for bad in (-1, 9):                                       # chunks per decode-attention CTA
+        with pytest.raises(tl.TLError) as e:
+            model.set_decode_chunks(bad)
+        assert e.value.status == tl.TL_ERR_INVALID_ARG
+    model.set_decode_chunks(0)
     assert model.sync_status() == tl.TL_OK
     kv.close()
 
