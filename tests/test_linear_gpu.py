@@ -51,6 +51,9 @@ def test_linear_mma_kernel(N, K, T, group):
     (128, 64, 64, 64), (256, 256, 100, 64), (768, 256, 128, 64), (2048, 2048, 128, 128),
     (6144, 2048, 128, 128), (2048, 8192, 128, 128), (16384, 2048, 128, 128),
     (1024, 2048, 256, 128), (512, 1024, 300, 128), (2048, 2048, 1024, 128),
+    # 64 tokens (64-wide token tile: its activation ring is deeper than the
+    # TMEM weight ring) over many k blocks
+    (2048, 8192, 64, 128), (6144, 2048, 64, 128),
 ])
 def test_linear_tc_kernel(N, K, T, group):
     words, scales, x, ref = _case(N, K, T, group, seed=N + K + T)

@@ -16,9 +16,10 @@
 //   * one TMA warp streams the activation tiles x[BN tokens][64 k] (fp16,
 //     128-byte swizzled, rows past T read as zero) through a ring that the
 //     MMAs free one k block at a time;
-//   * a watcher warp waits for each batch's activation tiles and arrives on
-//     the batch's barrier, so neither the MMA warp nor the dequantisation
-//     warps wait on them;
+//   * a watcher warp waits for each batch's activation tiles (and for the
+//     A slot's previous batch to be complete) and arrives on the batch's
+//     barrier, so neither the MMA warp nor the dequantisation warps wait on
+//     them;
 //   * the MMA warp issues tcgen05.mma kind::f16 (M 128, N BN, K 16; A from
 //     TMEM, B from shared memory, fp32 accumulation in TMEM) per batch of four
 //     k blocks.
@@ -282,6 +283,11 @@ __global__ void __maxnreg__(96)
         const int i = b * BATCH + j;
         okw = warp_wait(&xfull[i % XS], (i / XS) & 1, abort_flag, true);
       }
+      // when the activation ring holds more k blocks than the A ring
+      // (XS > AB * BATCH), batch b's tiles can land before the A slot's phase
+      // for batch b - AB has completed; arriving then would count towards that
+      // phase, so first wait for it
+      if (okw && b >= AB) okw = warp_wait(&afull[b % AB], ((b - AB) / AB) & 1, abort_flag, true);
       if (!okw) {
         if (lane == 0) atomicExch(abort_flag, 1);
         break;
