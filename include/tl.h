@@ -115,6 +115,22 @@ tl_status tl_unpack_codes(const uint32_t* packed, int N, int K, int bits,
 tl_status tl_kv_quant_int8(const uint16_t* x, int rows, int hd, int8_t* codes,
                            uint16_t* scales, tl_stream stream);
 
+/* Causal self-attention of a prefill (test hook): the block's attention step
+ * on its own, with the kernel the block's prefill uses (a tiled kernel with an
+ * online softmax: "Production Roadmap", Stage 2, Attention workstream, the
+ * tiled prefill kernel; "TinyLoop Framework", table of validated H100
+ * numbers, "Full prefill attention" row).  Per head h and query t,
+ *   out[t, h] = sum over j <= t of softmax_j(q[t, h] . k[j, h] / sqrt(hd)) v[j, h]
+ * with q and k taken as given (the block rotates them before this step).
+ * Scores, running maxima, exponentials and sums in fp32; the softmax weights
+ * enter the P.V product as fp16; out is rounded to fp16.
+ *   q, k, v   device fp16 [T, H * hd], head h in columns [h*hd, (h+1)*hd)
+ *   out       device fp16 [T, H * hd]   (written; must not overlap q, k, v)
+ * Requirements: 0 <= T <= 8192, 1 <= H <= 256, hd 64 or 128 (other values:
+ * TL_ERR_UNSUPPORTED), every pointer 16-byte aligned.  T = 0 does nothing. */
+tl_status tl_attention_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               int T, int H, int hd, uint16_t* out, tl_stream stream);
+
 /* ------------------------------------------------------------------------
  * Blocks.  One pre-norm transformer block: RMSNorm -> fused QKV -> RoPE on q
  * and k -> causal attention -> O projection + residual -> RMSNorm -> SwiGLU

@@ -83,6 +83,30 @@ def test_pack_rejects_before_launch(args, status):
     assert tl.lib.tl_last_error()
 
 
+@pytest.mark.parametrize("T,H,hd,status", [
+    (-1, 2, 64, tl.TL_ERR_INVALID_ARG),
+    (8193, 2, 64, tl.TL_ERR_INVALID_ARG),
+    (4, 0, 64, tl.TL_ERR_INVALID_ARG),
+    (4, 257, 64, tl.TL_ERR_INVALID_ARG),
+    (4, 2, 96, tl.TL_ERR_UNSUPPORTED),
+    (4, 2, 32, tl.TL_ERR_UNSUPPORTED),
+])
+def test_attention_prefill_rejects_before_launch(T, H, hd, status):
+    p = ctypes.c_void_p(16)
+    assert tl.lib.tl_attention_prefill(p, p, p, T, H, hd, p, None) == status
+    assert tl.lib.tl_last_error()
+
+
+def test_attention_prefill_pointer_checks():
+    p, odd = ctypes.c_void_p(16), ctypes.c_void_p(24)   # 24: 8-byte but not 16-byte aligned
+    f = tl.lib.tl_attention_prefill
+    assert f(None, p, p, 4, 2, 64, p, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, p, p, 4, 2, 64, None, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, odd, p, 4, 2, 128, p, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, p, p, 4, 2, 64, odd, None) == tl.TL_ERR_INVALID_ARG
+    assert f(None, None, None, 0, 2, 64, None, None) == tl.TL_OK   # empty: no-op
+
+
 def test_null_pointers_rejected():
     assert tl.lib.tl_pack_weights(None, 8, 64, 4, 64, None, None, None) == tl.TL_ERR_INVALID_ARG
     assert tl.lib.tl_kv_quant_int8(None, 4, 128, None, None, None) == tl.TL_ERR_INVALID_ARG

@@ -61,6 +61,7 @@ _SIGS = {
     "tl_pack_weights": ([P, I, I, I, I, P, P, P], I),
     "tl_unpack_codes": ([P, I, I, I, P, P], I),
     "tl_kv_quant_int8": ([P, I, I, P, P, P], I),
+    "tl_attention_prefill": ([P, P, P, I, I, I, P, P], I),
     "tl_block_create": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(P)], I),
     "tl_block_destroy": ([P], I),
     "tl_model_create": ([ctypes.POINTER(ModelDesc), ctypes.POINTER(P)], I),
@@ -147,6 +148,13 @@ def tl_unpack_codes(packed, N: int, K: int, bits: int, codes, stream=None) -> No
 def tl_kv_quant_int8(x, codes, scales, stream=None) -> None:
     rows, hd = (x.shape[0], x.shape[1]) if x.dim() == 2 else (0, x.shape[-1])
     _check(lib.tl_kv_quant_int8(_ptr(x), rows, hd, _ptr(codes), _ptr(scales), _stream(stream)))
+
+
+def tl_attention_prefill(q, k, v, H: int, hd: int, out, stream=None) -> None:
+    """q, k, v, out: fp16 [T, H * hd] (or [T, H, hd]) device tensors."""
+    T = q.shape[0]
+    _check(lib.tl_attention_prefill(_ptr(q), _ptr(k), _ptr(v), T, H, hd, _ptr(out),
+                                    _stream(stream)))
 
 
 # --------------------------------------------------------------------- blocks / model

@@ -175,6 +175,21 @@ TL_API tl_status tl_kv_quant_int8(const uint16_t* x, int rows, int hd, int8_t* c
                               reinterpret_cast<__half*>(scales), (cudaStream_t)stream);
 }
 
+TL_API tl_status tl_attention_prefill(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                      int T, int H, int hd, uint16_t* out, tl_stream stream) {
+  TL_CHECK_ARG(T >= 0 && T <= 8192, "T = %d out of [0, 8192]", T);
+  TL_CHECK_ARG(H >= 1 && H <= 256, "H = %d out of [1, 256]", H);
+  if (hd != 64 && hd != 128)
+    return set_error(TL_ERR_UNSUPPORTED, "head_dim = %d: only 64 and 128 are supported", hd);
+  if (T == 0) return ok();
+  TL_CHECK_ARG(q && k && v && out, "NULL device pointer");
+  const uintptr_t any = (uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)out;
+  TL_CHECK_ARG((any & 15) == 0, "q, k, v and out must be 16-byte aligned");
+  return launch_attn_prefill(reinterpret_cast<const __half*>(q), reinterpret_cast<const __half*>(k),
+                             reinterpret_cast<const __half*>(v), reinterpret_cast<__half*>(out), T,
+                             H, hd, (cudaStream_t)stream);
+}
+
 // ============================================================================
 // Blocks
 // ============================================================================
