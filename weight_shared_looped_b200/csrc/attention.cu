@@ -14,6 +14,7 @@
 #include <algorithm>
 #include <map>
 #include <mutex>
+#include <tuple>
 
 #include "tl_launch.cuh"
 
@@ -811,16 +812,16 @@ tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v,
   if (T == 0) return ok();
   dim3 grid((T + FQ - 1) / FQ, H);
   const float scale_log2 = 1.4426950408889634f / sqrtf((float)hd);
-  static bool attr_done = false;
-  if (!attr_done) {
+  static std::atomic<uint64_t> attr_done{0};
+  TL_TRY(once_per_device(attr_done, []() -> tl_status {
     TL_CUDA(cudaFuncSetAttribute(attn_prefill_tc_kernel<128>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)attn_prefill_smem<128>()));
     TL_CUDA(cudaFuncSetAttribute(attn_prefill_tc_kernel<64>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)attn_prefill_smem<64>()));
-    attr_done = true;
-  }
+    return ok();
+  }));
   if (hd == 128)
     TL_LAUNCH_PDL(attn_prefill_tc_kernel<128>, grid, 32 * ATT_WARPS, attn_prefill_smem<128>(), s,
                   q, k, v, out, T, H, scale_log2);
@@ -851,9 +852,15 @@ constexpr size_t kDecodeSmemCap = 200 * 1024;
 template <int HD, bool I8>
 static int decode_active_clusters(int pc, size_t smem) {
   static std::mutex mu;
-  static std::map<std::pair<int, size_t>, int> cache;
+  static std::map<std::tuple<int, int, size_t>, int> cache;   // (device, pc, smem)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    dev = -1;
+  }
+  const auto key = std::make_tuple(dev, pc, smem);
   std::lock_guard<std::mutex> lock(mu);
-  auto it = cache.find({pc, smem});
+  auto it = cache.find(key);
   if (it != cache.end()) return it->second;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pc, 1, 1);
@@ -873,18 +880,18 @@ static int decode_active_clusters(int pc, size_t smem) {
     cudaGetLastError();
     n = 1;
   }
-  cache[{pc, smem}] = n;
+  cache[key] = n;
   return n;
 }
 
 template <int HD, bool I8>
 static tl_status launch_decode_tc(const DecodeAttnArgs& a, cudaStream_t s) {
-  static bool attr_done = false;
-  if (!attr_done) {
+  static std::atomic<uint64_t> attr_done{0};
+  TL_TRY(once_per_device(attr_done, []() -> tl_status {
     TL_CUDA(cudaFuncSetAttribute(attn_decode_tc_kernel<HD, I8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmemCap));
-    attr_done = true;
-  }
+    return ok();
+  }));
   const int cl = decode_cluster_size(a.max_ctx);
   const int max_per = (a.max_ctx + cl - 1) / cl;   // keys of a chunk at most
   // chunks per CTA: the fewest that run every (row, head) cluster in the

@@ -613,18 +613,18 @@ tl_status launch_bounded_wait_check(int* status, uint64_t limit_ns, cudaStream_t
   return ok();
 }
 
-// One-time set-up (driver entry point, shared-memory limit); called outside
-// any stream capture.
+// Set-up once per device (driver entry point, shared-memory limit); called
+// outside any stream capture.
 tl_status gemm_tc_init() {
-  static bool done = false;
-  if (done) return ok();
-  TL_TRY(get_encoder());
-  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               232448));
-  TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-  done = true;
-  return ok();
+  static std::atomic<uint64_t> done{0};
+  return once_per_device(done, []() -> tl_status {
+    TL_TRY(get_encoder());
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    return ok();
+  });
 }
 
 // Split-K factor for the tensor-core kernel: one CTA per SM, so as many splits

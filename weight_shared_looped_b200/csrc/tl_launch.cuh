@@ -9,9 +9,27 @@
 // attribute both instructions are no-ops.
 #pragma once
 
+#include <atomic>
+
 #include "tl_internal.cuh"
 
 namespace tl {
+
+// One-time host set-up per device: kernel attributes such as the dynamic
+// shared-memory limit belong to the device's context, so a process that
+// drives several GPUs sets them on each.  Bit d of `done` records device d
+// (devices past 63 repeat the set-up on every call).  Concurrent first calls
+// may both run `f`; it only sets attributes, so that is harmless.
+template <typename Fn>
+inline tl_status once_per_device(std::atomic<uint64_t>& done, Fn f) {
+  int dev = 0;
+  TL_CUDA(cudaGetDevice(&dev));
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit != 0 && (done.load(std::memory_order_acquire) & bit) != 0) return ok();
+  TL_TRY(f());
+  done.fetch_or(bit, std::memory_order_release);
+  return ok();
+}
 
 __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
