@@ -44,3 +44,18 @@ def test_reference_arm_other_ranks_exit_without_work():
     r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
+
+
+def test_roofline_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
+    """The per-launch DRAM bytes from a committed ncu summary are reported only
+    while the kernel source hashes to the value the summary recorded."""
+    (tmp_path / "profiles").mkdir()
+    (tmp_path / "k.cu").write_text("kernel v1\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h = bench.source_hash("k.cu")
+    (tmp_path / "profiles" / "k.md").write_text(
+        f"# summary\n\nsource_sha256_16: {h}\ndram_bytes_per_launch: 17884160\n")
+    assert bench.ncu_traffic("k.md", ["k.cu"]) == 17884160.0
+    (tmp_path / "k.cu").write_text("kernel v2\n")          # the kernel changed since the capture
+    assert bench.ncu_traffic("k.md", ["k.cu"]) is None
+    assert bench.ncu_traffic("missing.md", ["k.cu"]) is None
