@@ -1,6 +1,7 @@
-"""bench.py's reference arm (the CPU oracle timed on the host) keeps the
-benchmark's one-line JSON contract, and under a multi-rank launch only rank 0
-does the work and prints."""
+"""Host logic of bench.py: the reference arm (the CPU oracle timed on the host)
+keeps the benchmark's one-line JSON contract, and under a multi-rank launch
+only rank 0 does the work and prints; the roofline's DRAM traffic is taken
+from a committed ncu summary only while the kernel source is unchanged."""
 import json
 import os
 import subprocess
