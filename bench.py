@@ -136,11 +136,15 @@ def oracle_threads():
     return os.cpu_count()
 
 
-def cpu_baseline_prefill(seconds: float = 10.0):
-    """The oracle's full seq-128 L=8 forward on the host cores, repeated for
-    about `seconds` (at least 2 forwards) after one untimed forward."""
+def cpu_baseline(seconds: float = 8.0):
+    """The oracle as it stands, on the host cores: full seq-128 L=8 forwards
+    for about `seconds` (at least 2, after one untimed forward); the cached
+    decode step of the batch-1 FP16-KV workload over its first 8 steps (the
+    256-token prompt prefill untimed); and the INT4 and INT3 packers on one
+    407M block."""
     import numpy as np
     import synthetic as syn
+    from oracle import tinyloop_oracle as o
     from oracle.workloads import build_oracle_model
     w = syn.WORKLOADS["prefill407m"]
     om = build_oracle_model("prefill407m")
@@ -151,10 +155,32 @@ def cpu_baseline_prefill(seconds: float = 10.0):
         om.prefill(ids, w.L[0])
         n += 1
     dt = time.perf_counter() - t0
+    # cached decode: prompt 256 (untimed), then 8 timed steps
+    wd = syn.WORKLOADS["decode407m"]
+    kv = om.new_kv(wd.L[0], "fp16")
+    om.prefill(syn.prompt_ids(wd), wd.L[0], kv=kv)
+    steps = syn.decode_ids(wd)
+    t1 = time.perf_counter()
+    for s in range(8):
+        om.decode_step(np.int64(steps[s]), wd.L[0], kv)
+    dec_ms = (time.perf_counter() - t1) / 8 * 1e3
+    # packers: quantise + pack the five matrices of one block
+    wts = syn.block_weights(w.shape, w.seed, "loop")
+    pack_ms = {}
+    for bits in (4, 3):
+        t2 = time.perf_counter()
+        o.pack_block(wts, bits, w.group)
+        pack_ms[bits] = (time.perf_counter() - t2) * 1e3
     return {"value": round(w.seq * n / dt, 2), "unit": "tokens/s", "cores": oracle_threads(),
             "kind": "oracle",
+            "decode_ms_per_step": round(dec_ms, 2),
+            "decode_tok_s": round(1e3 / dec_ms, 2),
+            "pack_int4_ms_per_block": round(pack_ms[4], 1),
+            "pack_int3_ms_per_block": round(pack_ms[3], 1),
             "sample": f"{n} full forwards (seq 128, L=8, fp64 numpy oracle), {dt:.1f} s; "
-                      f"model build untimed"}
+                      f"8 cached decode steps after a 256-token prompt (batch 1, FP16 KV, "
+                      f"L=8); one INT4 and one INT3 pack of a 407M block; model build and "
+                      f"prompt prefill untimed"}
 
 
 def run_reference(args, rank, world):
@@ -306,7 +332,9 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
-        return sum(a.elapsed_time(b) for a, b in evs) / 1e3   # seconds
+        per = [a.elapsed_time(b) for a, b in evs]
+        timed.last_median_ms = statistics.median(per)
+        return sum(per) / 1e3   # seconds
 
     # headline: prefill forward
     for _ in range(max(args.warmup, 3)):
@@ -317,6 +345,7 @@ def run_ours(args, rank, world, dist):
     with ClockSampler(gpu_uuid(torch, dev)) as clk, torch.cuda.nvtx.range("prefill"):
         t = timed(step, args.steps, 0)
     assert model.sync_status() == tl.TL_OK
+    median_ms = max_over_ranks(timed.last_median_ms, dist, "cuda")
     t = max_over_ranks(t, dist, "cuda")
     value = job_value(seq * args.steps, world, t)
     ms_per_step = t / args.steps * 1e3
@@ -389,39 +418,96 @@ def run_ours(args, rank, world, dist):
             "forward_tflops": round(172.5e9 * args.steps / (t / world) / 1e12, 2),
             "forward_frac": round(172.5e9 * args.steps / (t / world) / 1e12 / pk["bf16_tflops"], 4)}
 
+    l2 = l2_probe(tl, torch, dist)
     decode = None
     if not args.no_decode:
         decode = run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
-                            cfg)
+                            cfg, l2["gbs"])
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "ms_per_step_median": round(median_ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "l2": "flushed before every timed step (256 MiB write)",
                        "parallelism": "replicas" if world > 1 else "single",
                        "graphs": "one CUDA graph per (seq, L)"},
             "roofline": roof, "e2e": e2e, "gpu_launches": launches_per_fwd * args.steps,
+            "l2_probe": l2,
             "clocks": clk.summary()}
     if decode is not None:
         line["decode"] = decode
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline_prefill()
+        line["cpu_baseline"] = cpu_baseline()
     elif rank == 0:
         line["cpu_baseline"] = None
     model.close()
     return line
 
 
-def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg):
+def l2_probe(tl, torch, dist, mib: int = 32, passes: int = 64):
+    """L2 read bandwidth: tl_read_probe over a buffer well inside the L2 (one
+    untimed pass makes it resident), timed with CUDA events on the launching
+    stream, best of 5."""
+    buf = torch.empty(mib << 20, dtype=torch.uint8, device="cuda")
+    buf.fill_(1)
+    sink = torch.zeros(2, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    tl.tl_read_probe(buf, 1, sink)
+    best = None
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        tl.tl_read_probe(buf, passes, sink)
+        b.record(stream)
+        torch.cuda.synchronize()
+        t = a.elapsed_time(b) / 1e3
+        best = t if best is None else min(best, t)
+    assert int(sink[1].item()) == passes
+    best = max_over_ranks(best, dist, "cuda")
+    gbs = (mib << 20) * passes / best / 1e9
+    return {"gbs": round(gbs, 1), "bytes": mib << 20, "passes": passes,
+            "how": "tl_read_probe (128-bit loads over every SM) on an L2-resident buffer, "
+                   "CUDA events, best of 5"}
+
+
+def block_bytes(tl, bits: int, d: int = 2048, f: int = 8192, group: int = 128) -> int:
+    """Packed bytes (codes + fp16 scales) of one block, from the library's
+    own size query."""
+    total = 0
+    for n, k in ((3 * d, d), (d, d), (f, d), (f, d), (d, f)):
+        c, sc = tl.tl_packed_bytes(n, k, bits, group)
+        total += c + sc
+    return total
+
+
+def decode_roofline(t_step, hbm_bytes, l2_bytes, hbm_gbs, l2_gbs):
+    """The decode roofline: t = HBM bytes / HBM bandwidth + L2 bytes / L2
+    bandwidth (the loop block's re-reads within a step come from L2)."""
+    t_roof = hbm_bytes / (hbm_gbs * 1e9) + l2_bytes / (l2_gbs * 1e9)
+    return {"hbm_bytes_per_step": int(hbm_bytes), "l2_bytes_per_step": int(l2_bytes),
+            "roofline_us": round(t_roof * 1e6, 2),
+            "frac_roofline": round(t_roof / t_step, 4),
+            "frac_hbm": round(hbm_bytes / t_step / 1e9 / hbm_gbs, 4)}
+
+
+def loop_read_bytes(tl, blk) -> int:
+    """Bytes the decode kernels read per application of an INT3 block: the
+    library reads an INT4 copy of the INT3 codes (same scales)."""
+    return block_bytes(tl, 4)
+
+
+def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg, l2_gbs):
     """KV-cached decode throughput: B=1 FP16 KV (prompt 256, 128 steps), B=8
     INT8 KV at context 2048 (64 steps), mixed-depth INT3 lanes (ctx 1024, 32
     steps).  Each timed step is one tl_decode_step; caches are filled by GPU
-    prefill of seeded prompt ids."""
+    prefill of seeded prompt ids.  L2 is flushed before every step, so each
+    step reads the model's weights once from HBM; the loop block's further
+    iterations re-read them from L2."""
     from weight_shared_looped_b200.model import DeviceBlock, DeviceModel
     out = {}
     hbm = pk["hbm_gbs"]
-    blk_bytes = 34.6e6
+    blk_bytes = block_bytes(tl, 4)
 
     def ids_t(x):
         return torch.from_numpy(np.ascontiguousarray(x, dtype=np.int32)).cuda()
@@ -446,13 +532,14 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
     it = iter(range(10 ** 9))
     with torch.cuda.nvtx.range("decode_b1"):
         t = max_t(timed(dstep, w.steps, 0))
+    med = timed.last_median_ms
     avg_ctx = w.seq + (w.steps + 1) / 2
     kv_bytes = 10 * avg_ctx * 2048 * 2 * 2
-    step_bytes = 3 * blk_bytes + kv_bytes
     out["b1_fp16kv"] = {"tok_s": round(w.steps * world / t, 1),
                         "ms_per_step": round(t / w.steps * 1e3, 4),
-                        "hbm_bytes_per_step": int(step_bytes),
-                        "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                        "ms_per_step_median": round(med, 4),
+                        **decode_roofline(t / w.steps, 3 * blk_bytes + kv_bytes, 7 * blk_bytes,
+                                          hbm, l2_gbs),
                         "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
     kv.close()
     torch.cuda.synchronize()
@@ -475,13 +562,14 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
         kv.set_position(b, w.seq)
     with torch.cuda.nvtx.range("decode_b8"):
         t = max_t(timed(dstep8, w.steps, 0))
+    med = timed.last_median_ms
     avg_ctx = w.seq + (w.steps + 1) / 2
     kv_bytes = 8 * 10 * avg_ctx * 16 * (2 * 128 + 2 * 2)
-    step_bytes = 3 * blk_bytes + kv_bytes
     out["b8_int8kv_ctx2048"] = {"tok_s": round(8 * w.steps * world / t, 1),
                                 "ms_per_step": round(t / w.steps * 1e3, 4),
-                                "hbm_bytes_per_step": int(step_bytes),
-                                "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                                "ms_per_step_median": round(med, 4),
+                                **decode_roofline(t / w.steps, 3 * blk_bytes + kv_bytes,
+                                                  7 * blk_bytes, hbm, l2_gbs),
                                 "workload": "batch 8, context 2048 + 64 steps, L=8, INT8 KV"}
     kv.close()
     torch.cuda.synchronize()
@@ -507,14 +595,17 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
         kv.set_position(b, w.seq)
     with torch.cuda.nvtx.range("decode_b3"):
         t = max_t(timed(dstep3, w.steps, 0))
+    med = timed.last_median_ms
     avg_ctx = w.seq + (w.steps + 1) / 2
     slots = sum(2 + L for L in w.L)
     kv_bytes = slots * avg_ctx * 2048 * 2 * 2
-    step_bytes = 2 * blk_bytes + 28.2e6 + kv_bytes
+    loop_bytes = loop_read_bytes(tl, loop3)
     out["b3_int3_mixedL"] = {"tok_s": round(3 * w.steps * world / t, 1),
                              "ms_per_step": round(t / w.steps * 1e3, 4),
-                             "hbm_bytes_per_step": int(step_bytes),
-                             "frac_hbm": round(step_bytes / (t / w.steps) / 1e9 / hbm, 4),
+                             "ms_per_step_median": round(med, 4),
+                             **decode_roofline(t / w.steps, 2 * blk_bytes + loop_bytes + kv_bytes,
+                                               (max(w.L) - 1) * loop_bytes, hbm, l2_gbs),
+                             "loop_block_bytes_read": loop_bytes,
                              "workload": "lanes L=[4,16,32], INT3 loop block, context 1024 + "
                                          "32 steps, FP16 KV"}
     kv.close()

@@ -299,7 +299,9 @@ tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
  *   y               device fp32 [T, N]   (written)
  *   workspace       device scratch of tl_linear_workspace_bytes(N, K, T) bytes
  *                   (may be NULL when that size is 0)
- * Requirements: N % 64 == 0, K % 64 == 0, group in {64, 128}, 1 <= T <= 8192.
+ * Requirements: N % 64 == 0, K % 64 == 0, group in {64, 128}, K % group == 0,
+ * 1 <= T <= 8192; anything else returns TL_ERR_INVALID_ARG (TL_ERR_UNSUPPORTED
+ * for another group size) before any launch.
  * bits must be 4 (an INT3 matrix is converted by tl_block_create). */
 tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes);
 tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K,
@@ -317,7 +319,10 @@ tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K
  * Allocates nothing.  All calls share the buffer, so calls that overlap on the
  * GPU race; each call overwrites what it reads, so nothing needs clearing.
  * The first call on a device looks up the buffer's device address; make it
- * before any stream capture. */
+ * before any stream capture.  The address is kept for the life of the process:
+ * a cudaDeviceReset (or anything else that replaces the device's primary
+ * context) after that first call is not supported.  Shape requirements and
+ * errors are those of tl_linear. */
 tl_status tl_linear_noalloc(const uint32_t* packed, const uint16_t* scales, int N,
                             int K, int group, const uint16_t* x, int T, float* y,
                             tl_stream stream);
@@ -328,6 +333,23 @@ tl_status tl_linear_noalloc(const uint32_t* packed, const uint16_t* scales, int 
  * status word; read it with tl_sync_status.  The kernel returns normally: no
  * trap, no fault, the context stays usable. */
 tl_status tl_check_bounded_wait(tl_model* model, unsigned limit_us, tl_stream stream);
+
+/* Measurement hook: read-bandwidth probe.  Reads `bytes` of device memory at
+ * `buf` `passes` times with 128-bit loads spread evenly over every SM, folding
+ * the words into a value that decides one store to `sink` (so no load is
+ * dropped).  A buffer well under the L2 size stays resident after the first
+ * pass, so timing this call with CUDA events measures L2 read bandwidth: the
+ * denominator of the L2 term of the decode roofline, t = HBM bytes / HBM
+ * bandwidth + L2 bytes / L2 bandwidth, which charges the loop block's re-reads
+ * within a step (iterations 2..L reuse the same weights: "TinyLoop Framework",
+ * "What Makes It Different") at L2 speed.  A buffer several times the L2 size
+ * measures HBM read bandwidth instead.
+ *   buf    device pointer, 16-byte aligned; bytes a positive multiple of 16
+ *   sink   device pointer, uint32 [2] (written: sink[1] = passes)
+ *   passes 1 .. 4096
+ * No result is computed; errors are TL_ERR_INVALID_ARG before any launch. */
+tl_status tl_read_probe(const void* buf, size_t bytes, int passes, uint32_t* sink,
+                        tl_stream stream);
 
 /* Synchronise `stream`, then return and clear the model's device status word
  * (TL_OK, TL_ERR_TIMEOUT or TL_ERR_NUMERIC). */

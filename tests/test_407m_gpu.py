@@ -77,6 +77,31 @@ def test_cached_decode_407m_matches_uncached(m407):
     kv.close()
 
 
+def test_cached_decode_407m_per_block_traces(m407):
+    """Every block output of the first decode steps after a 256-token prompt
+    (FP16 KV) against the oracle's cached decode of the same prompt, at the
+    per-block tolerance; both sides run free from the same ids."""
+    w = syn.WORKLOADS["decode407m"]
+    L, n_layers, S = w.L[0], w.n_pre + w.L[0], 3
+    prompt, steps = syn.prompt_ids(w), syn.decode_ids(w)
+    kv = m407.new_kv([L], max_ctx=w.max_ctx, dtype="fp16")
+    m407.prefill(_ids(prompt), L=L, kv=kv, lane=0)
+    om = oracle_model("prefill407m")
+    okv = om.new_kv(L, "fp16")
+    om.prefill(prompt, L, kv=okv)
+    for s in range(S):
+        tr = torch.empty(n_layers, 1, w.shape.d_model, dtype=torch.float32, device="cuda")
+        y = m407.decode(kv, _ids(steps[s:s + 1]), L_per_lane=[L], h_trace=tr)
+        assert m407.sync_status() == tl.TL_OK
+        rtr = []
+        ry = om.decode_step(np.int64(steps[s]), L, okv, trace=rtr)
+        trc = tr.cpu().numpy()
+        errs = [rel_l2(trc[i, 0], rtr[i][0]) for i in range(n_layers)]
+        assert max(errs) <= BLOCK_REL_L2, (s, errs)
+        assert cosine(y[0].cpu().numpy(), ry) >= FINAL_COSINE, s
+    kv.close()
+
+
 def _raw_view(kv, ptr, shape, dtype):
     """A torch view of one region of the caller-owned KV buffer."""
     off = ptr - kv.buffer.data_ptr()
@@ -130,7 +155,7 @@ def test_long_context_int8_decode(m407):
         okv = om.new_kv(L, "int8")
         for layer, (kc, ks, vc, vs) in enumerate(ctx[lane]):
             okv[layer].load_stored(o.kv_dequant_int8(kc, ks), o.kv_dequant_int8(vc, vs))
-        for s in range(2):
+        for s in range(4):
             r = om.decode_step(np.int64(ids[s, lane]), L, okv)
             assert cosine(y[s, lane], r) >= FINAL_COSINE, (lane, s)
             assert rel_l2(y[s, lane], r) <= 2 * BLOCK_REL_L2, (lane, s)

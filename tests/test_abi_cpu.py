@@ -159,3 +159,35 @@ def test_model_create_validation():
         out = ctypes.c_void_p()
         assert tl.lib.tl_model_create(ctypes.byref(d), ctypes.byref(out)) == tl.TL_ERR_INVALID_ARG
     tl.lib.tl_block_destroy(blk)
+
+
+@pytest.mark.parametrize("N,K,group,T,status", [
+    (64, 192, 128, 1, tl.TL_ERR_INVALID_ARG),    # K % group == 64: half a scale group per row
+    (64, 320, 128, 16, tl.TL_ERR_INVALID_ARG),
+    (64, 96, 64, 1, tl.TL_ERR_INVALID_ARG),      # K % 64
+    (96, 128, 64, 1, tl.TL_ERR_INVALID_ARG),     # N % 64
+    (64, 128, 32, 1, tl.TL_ERR_UNSUPPORTED),     # group
+    (64, 128, 64, 0, tl.TL_ERR_INVALID_ARG),     # T
+    (64, 128, 64, 8193, tl.TL_ERR_INVALID_ARG),
+])
+def test_linear_entry_points_reject_before_launch(N, K, group, T, status):
+    """Both linear-layer entry points reject a shape whose rows do not hold
+    whole scale groups before anything is launched (no GPU is touched: the
+    pointers are placeholders)."""
+    p = ctypes.c_void_p(256)
+    assert tl.lib.tl_linear(p, p, N, K, group, p, T, p, p, None) == status
+    assert tl.lib.tl_last_error()
+    assert tl.lib.tl_linear_noalloc(p, p, N, K, group, p, T, p, None) == status
+    assert tl.lib.tl_last_error()
+
+
+def test_read_probe_rejects_before_launch():
+    p, odd = ctypes.c_void_p(256), ctypes.c_void_p(264)
+    f = tl.lib.tl_read_probe
+    assert f(None, 1024, 1, p, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, 1024, 1, None, None) == tl.TL_ERR_INVALID_ARG
+    assert f(odd, 1024, 1, p, None) == tl.TL_ERR_INVALID_ARG      # 8-byte aligned only
+    assert f(p, 1000, 1, p, None) == tl.TL_ERR_INVALID_ARG        # not a multiple of 16
+    assert f(p, 0, 1, p, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, 1024, 0, p, None) == tl.TL_ERR_INVALID_ARG
+    assert f(p, 1024, 4097, p, None) == tl.TL_ERR_INVALID_ARG

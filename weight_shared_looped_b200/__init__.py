@@ -85,6 +85,7 @@ _SIGS = {
     "tl_linear": ([P, P, I, I, I, P, I, P, P, P], I),
     "tl_linear_noalloc": ([P, P, I, I, I, P, I, P, P], I),
     "tl_check_bounded_wait": ([P, ctypes.c_uint, P], I),
+    "tl_read_probe": ([P, SZ, I, P, P], I),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -291,6 +292,12 @@ def tl_linear_noalloc(packed, scales, N: int, K: int, group: int, x, y, stream=N
     T = x.shape[0]
     _check(lib.tl_linear_noalloc(_ptr(packed), _ptr(scales), N, K, group, _ptr(x), T, _ptr(y),
                                  _stream(stream)))
+
+
+def tl_read_probe(buf, passes: int, sink, stream=None) -> None:
+    """Read `buf` (a 16-byte aligned device tensor) `passes` times."""
+    nbytes = buf.numel() * buf.element_size()
+    _check(lib.tl_read_probe(_ptr(buf), nbytes, passes, _ptr(sink), _stream(stream)))
 
 
 def tl_check_bounded_wait(model: int, limit_us: int, stream=None) -> None:

@@ -993,16 +993,18 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
 // ============================================================================
 // Linear-layer hook
 // ============================================================================
-namespace {
+namespace tl {
 tl_status check_linear(int N, int K, int group, int T) {
   TL_CHECK_ARG(N >= 64 && N % 64 == 0, "N = %d must be a positive multiple of 64", N);
   TL_CHECK_ARG(K >= 64 && K % 64 == 0, "K = %d must be a positive multiple of 64", K);
   if (group != 64 && group != 128)
     return set_error(TL_ERR_UNSUPPORTED, "group = %d: only 64 and 128 are supported", group);
+  // every row holds K / group whole scale groups (as tl_pack_weights requires)
+  TL_CHECK_ARG(K % group == 0, "K = %d is not a multiple of group %d", K, group);
   TL_CHECK_ARG(T >= 1 && T <= 8192, "T = %d out of [1, 8192]", T);
   return ok();
 }
-}  // namespace
+}  // namespace tl
 
 TL_API tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes) {
   TL_CHECK_ARG(bytes, "bytes is NULL");

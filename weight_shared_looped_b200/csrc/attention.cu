@@ -16,6 +16,7 @@
 #include <mutex>
 #include <tuple>
 
+#include "kv_quant.cuh"
 #include "tl_launch.cuh"
 
 namespace tl {
@@ -544,13 +545,13 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
       __syncthreads();
       km = fmaxf(fmaxf(kmax_s[0], kmax_s[1]), fmaxf(kmax_s[2], kmax_s[3]));
       vm = fmaxf(fmaxf(vmax_s[0], vmax_s[1]), fmaxf(vmax_s[2], vmax_s[3]));
-      const __half ksh = __float2half_rn(__fdiv_rn(km, 127.0f));
-      const __half vsh = __float2half_rn(__fdiv_rn(vm, 127.0f));
+      const __half ksh = kv_int8_scale(km);
+      const __half vsh = kv_int8_scale(vm);
       const float ksf = __half2float(ksh), vsf = __half2float(vsh);
       if (tid < HD) {
         const float kx = __half2float(kh), vx = __half2float(vh);
-        const int kc = ksf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ksf)), -127.f), 127.f);
-        const int vc = vsf == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vsf)), -127.f), 127.f);
+        const int kc = kv_int8_code(kx, ksf);
+        const int vc = kv_int8_code(vx, vsf);
         reinterpret_cast<int8_t*>(layer)[(head_off + pos) * HD + tid] = (int8_t)kc;
         reinterpret_cast<int8_t*>(layer + a.kv_region_bytes)[(head_off + pos) * HD + tid] = (int8_t)vc;
         k_new = (uint32_t)(uint8_t)(int8_t)kc;

@@ -6,6 +6,7 @@
 //
 // Every reduction runs in a fixed order that depends only on the row length,
 // so a row's result never depends on how many rows share the launch.
+#include "kv_quant.cuh"
 #include "tl_launch.cuh"
 
 namespace tl {
@@ -281,8 +282,8 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
   } else {
     kmax = warp_max(kmax);
     vmax = warp_max(vmax);
-    __half ksh = __float2half_rn(__fdiv_rn(kmax, 127.0f));
-    __half vsh = __float2half_rn(__fdiv_rn(vmax, 127.0f));
+    const __half ksh = kv_int8_scale(kmax);
+    const __half vsh = kv_int8_scale(vmax);
     float ks = __half2float(ksh), vs = __half2float(vsh);
     int8_t* K = reinterpret_cast<int8_t*>(layer) + eoff;
     int8_t* V = reinterpret_cast<int8_t*>(layer + a.kv_region_bytes) + eoff;
@@ -296,10 +297,8 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float kx = __half2float(kh[p][hh]), vx = __half2float(vh[p][hh]);
-          int kc = ks == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(kx, ks)), -127.f), 127.f);
-          int vc = vs == 0.f ? 0 : (int)fminf(fmaxf(rintf(__fdiv_rn(vx, vs)), -127.f), 127.f);
-          K[i + hh * half] = (int8_t)kc;
-          V[i + hh * half] = (int8_t)vc;
+          K[i + hh * half] = kv_int8_code(kx, ks);
+          V[i + hh * half] = kv_int8_code(vx, vs);
         }
       }
     }

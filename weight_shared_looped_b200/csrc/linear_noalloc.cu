@@ -60,11 +60,7 @@ using namespace tl;
 extern "C" __attribute__((visibility("default"))) tl_status tl_linear_noalloc(
     const uint32_t* packed, const uint16_t* scales, int N, int K, int group, const uint16_t* x,
     int T, float* y, tl_stream stream) {
-  TL_CHECK_ARG(N >= 64 && N % 64 == 0, "N = %d must be a positive multiple of 64", N);
-  TL_CHECK_ARG(K >= 64 && K % 64 == 0, "K = %d must be a positive multiple of 64", K);
-  if (group != 64 && group != 128)
-    return set_error(TL_ERR_UNSUPPORTED, "group = %d: only 64 and 128 are supported", group);
-  TL_CHECK_ARG(T >= 1 && T <= 8192, "T = %d out of [1, 8192]", T);
+  TL_TRY(check_linear(N, K, group, T));
   TL_CHECK_ARG(packed && scales && x && y, "NULL device pointer");
   const int S = gemm_splits(N, K, T);
   const size_t need = S > 1 ? (size_t)S * T * N * sizeof(float) : 0;

@@ -10,6 +10,7 @@
 // Every integer decision is an IEEE fp32 operation (correctly rounded division
 // __fdiv_rn, rintf ties-to-even, __float2half_rn), so the codes are a pure
 // function of the inputs.
+#include "kv_quant.cuh"
 #include "tl_internal.cuh"
 
 namespace tl {
@@ -141,12 +142,12 @@ __global__ void kv_quant_int8_kernel(const __half* __restrict__ x, int rows, int
     m = fmaxf(m, fabsf(v[e]));
   }
   m = warp_max(m);
-  __half sh = __float2half_rn(__fdiv_rn(m, 127.0f));
-  float s = __half2float(sh);
+  const __half sh = kv_int8_scale(m);
+  const float s = __half2float(sh);
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     int i = lane + 32 * e;
-    if (i < hd) codes[row * hd + i] = (int8_t)quant_code(v[e], s, -127.0f, 127.0f);
+    if (i < hd) codes[row * hd + i] = kv_int8_code(v[e], s);
   }
   if (lane == 0) scales[row] = sh;
 }

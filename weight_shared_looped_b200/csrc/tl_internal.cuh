@@ -88,6 +88,10 @@ struct GemmArgs {
   // instead of partial sums
   __half* swiglu_u;
 };
+// Shape checks shared by the linear-layer entry points (tl_linear and
+// tl_linear_noalloc): N, K multiples of 64, group 64 or 128 dividing K,
+// 1 <= T <= 8192.
+tl_status check_linear(int N, int K, int group, int T);
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
 // kernel for T >= 64, the mma.sync register-dequant kernel below that.
 int gemm_splits(int N, int K, int T);
@@ -175,5 +179,9 @@ struct DecodeAttnArgs {
   int chunks;                // context chunks per CTA; 0 = fewest waves
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
+
+// read-bandwidth probe (probe.cu)
+tl_status launch_read_probe(const void* buf, size_t bytes, int passes, uint32_t* sink,
+                            cudaStream_t s);
 
 }  // namespace tl
