@@ -345,6 +345,10 @@ class KVSlot:
         self._v[:v_values.shape[0]] = v_values
         self.n = k_values.shape[0]
 
+    def truncate(self, n: int) -> None:
+        """Keep positions 0..n-1 (entries past them are dropped)."""
+        self.n = min(self.n, n)
+
     @property
     def k(self) -> np.ndarray:
         return self._k[:self.n]
@@ -376,40 +380,133 @@ class LoopedModel:
     def embed(self, ids: np.ndarray) -> np.ndarray:
         return self.embed16[np.asarray(ids)].astype(F64)
 
+    def _exit_check(self, h: np.ndarray, layer: int, frozen: np.ndarray, loops: np.ndarray,
+                    exit_tau: Optional[float]) -> None:
+        """Per-iteration safety check ("Current Status", architecture-unique
+        features table, per-iteration safety check row: the residual stream's
+        L2 norm is computed every iteration and the loop stops above a
+        threshold, L checkpoints per token).  Reading: the check looks at the
+        residual stream leaving each loop iteration; a token whose norm exceeds
+        the threshold runs no further residual updates (its stream is frozen,
+        and the later iterations' K/V slots receive what the frozen stream
+        produces); its loop count is the iterations it ran."""
+        it = layer - len(self.pre)          # the loop iteration about to run
+        if exit_tau is None or it < 1:
+            return
+        norms = np.sqrt(np.sum(h * h, axis=-1))
+        newly = ~frozen & (norms > exit_tau)
+        loops[newly] = it
+        frozen |= newly
+
     def prefill(self, x_in: np.ndarray, L: int, kv: Optional[List[KVSlot]] = None,
-                trace: Optional[List[np.ndarray]] = None) -> np.ndarray:
+                trace: Optional[List[np.ndarray]] = None, exit_tau: Optional[float] = None,
+                info: Optional[dict] = None) -> np.ndarray:
         """Causal forward over T tokens at positions 0..T-1.  ``x_in`` is int ids
         [T] or hidden states [T, d].  With ``kv`` (one KVSlot per layer) the
         K/V of every layer are appended.  ``trace`` receives the residual
-        stream after every block application.  Returns the final-norm output."""
+        stream after every block application.  ``exit_tau`` enables the
+        per-iteration residual-norm check (``info["loops"]`` receives each
+        token's loop count).  Returns the final-norm output."""
         x_in = np.asarray(x_in)
         h = self.embed(x_in) if x_in.ndim == 1 else x_in.astype(F64)
         pos = np.arange(h.shape[0])
+        frozen = np.zeros(h.shape[0], bool)
+        loops = np.full(h.shape[0], L)
         for layer, blk in enumerate(self.schedule(L)):
+            self._exit_check(h, layer, frozen, loops, exit_tau)
             q, k, v = blk.qkv(h, pos)
             if kv is not None:
                 kv[layer].append(k, v)
-            h = blk.finish(h, causal_attention(q, k, v, pos))
+            h = np.where(frozen[:, None], h, blk.finish(h, causal_attention(q, k, v, pos)))
             if trace is not None:
                 trace.append(h.copy())
+        if info is not None:
+            info["loops"] = loops
+        return rmsnorm(h, self.gamma_final, self.cfg["eps"])
+
+    def extend(self, x_in, L: int, kv: List[KVSlot], trace: Optional[List[np.ndarray]] = None,
+               exit_tau: Optional[float] = None, info: Optional[dict] = None) -> np.ndarray:
+        """Cached forward of n tokens of one lane at positions p .. p+n-1, p =
+        len(kv[0]) (the verify pass of self-speculative decode: "Current
+        Status", speculative and adaptive decode table, self-speculative row:
+        L=2 draft, L=8 verify, same weights).  Every layer appends the n
+        tokens' K/V in the cache's storage dtype, then each token attends over
+        the stored entries up to its own position.  ``x_in``: ids [n] or
+        hidden states [n, d].  Returns the final-norm outputs [n, d]."""
+        x_in = np.asarray(x_in)
+        h = self.embed(x_in) if x_in.ndim == 1 else x_in.reshape(-1, self.cfg["d_model"]).astype(F64)
+        pos = np.arange(len(kv[0]), len(kv[0]) + h.shape[0])
+        frozen = np.zeros(h.shape[0], bool)
+        loops = np.full(h.shape[0], L)
+        for layer, blk in enumerate(self.schedule(L)):
+            self._exit_check(h, layer, frozen, loops, exit_tau)
+            q, k, v = blk.qkv(h, pos)
+            slot = kv[layer]
+            slot.append(k, v)
+            h = np.where(frozen[:, None], h,
+                         blk.finish(h, causal_attention(q, slot.k, slot.v, pos)))   # keys 0..pos
+            if trace is not None:
+                trace.append(h.copy())
+        if info is not None:
+            info["loops"] = loops
         return rmsnorm(h, self.gamma_final, self.cfg["eps"])
 
     def decode_step(self, x_in, L: int, kv: List[KVSlot],
-                    trace: Optional[List[np.ndarray]] = None) -> np.ndarray:
+                    trace: Optional[List[np.ndarray]] = None, exit_tau: Optional[float] = None,
+                    info: Optional[dict] = None) -> np.ndarray:
         """One cached decode step for one lane at position len(kv[0]): append
         this token's K/V to every layer's slot, attend over the stored
         entries.  Returns the final-norm output [d]."""
         x_in = np.asarray(x_in)
-        h = self.embed(x_in.reshape(1)) if x_in.ndim == 0 else x_in.reshape(1, -1).astype(F64)
-        pos = np.array([len(kv[0])])
-        for layer, blk in enumerate(self.schedule(L)):
-            q, k, v = blk.qkv(h, pos)
-            slot = kv[layer]
-            slot.append(k, v)
-            h = blk.finish(h, causal_attention(q, slot.k, slot.v, pos))   # keys 0..pos
-            if trace is not None:
-                trace.append(h.copy())
-        return rmsnorm(h, self.gamma_final, self.cfg["eps"])[0]
+        x1 = x_in.reshape(1) if x_in.ndim == 0 else x_in.reshape(1, -1)
+        return self.extend(x1, L, kv, trace=trace, exit_tau=exit_tau, info=info)[0]
+
+    def greedy_head(self, y: np.ndarray) -> np.ndarray:
+        """Greedy next tokens from final-norm outputs y [n, d] through the tied
+        embedding (logits = y . E^T, the head a self-speculative step needs to
+        compare draft and verify tokens); the lowest id wins a tie."""
+        logits = np.asarray(y, F64).reshape(-1, self.cfg["d_model"]) @ self.embed16.astype(F64).T
+        return np.argmax(logits, axis=-1)
+
+    def greedy_decode(self, token: int, n: int, L: int, kv: List[KVSlot]) -> List[int]:
+        """n greedy decode steps at depth L from the input token `token`;
+        returns the n generated tokens."""
+        out = []
+        for _ in range(n):
+            token = int(self.greedy_head(self.decode_step(np.int64(token), L, kv))[0])
+            out.append(token)
+        return out
+
+    def spec_step(self, token: int, K: int, L_draft: int, L_verify: int,
+                  kv: List[KVSlot]) -> List[int]:
+        """One greedy self-speculative step with one weight set and one cache
+        ("TinyLoop Framework", "What Makes It Different": draft and verify
+        reuse the same weights; "Current Status", self-speculative row: L=2
+        draft, L=8 verify).  From the input token x at position p:
+          draft   K decode steps at L_draft: d_1 .. d_K (each the greedy head
+                  of the previous step's output; they write positions
+                  p .. p+K-1 of the first n_pre + L_draft slots);
+          verify  rewind to p, extend [x, d_1 .. d_K] at L_verify (positions
+                  p .. p+K of every slot), greedy head: v_1 .. v_{K+1};
+          accept  m = the longest prefix with d_i == v_i; the emitted tokens
+                  are d_1 .. d_m, v_{m+1}; the cache keeps positions up to
+                  p + m (the entries past it are dropped).
+        The emitted tokens equal m + 1 greedy decode steps at L_verify."""
+        p = len(kv[0])
+        drafts, t = [], token
+        for _ in range(K):
+            t = int(self.greedy_head(self.decode_step(np.int64(t), L_draft, kv))[0])
+            drafts.append(t)
+        for slot in kv:
+            slot.truncate(p)
+        y = self.extend(np.array([token] + drafts, np.int64), L_verify, kv)
+        ver = [int(v) for v in self.greedy_head(y)]
+        m = 0
+        while m < K and drafts[m] == ver[m]:
+            m += 1
+        for slot in kv:
+            slot.truncate(p + m + 1)
+        return drafts[:m] + [ver[m]]
 
     def new_kv(self, L: int, dtype: str) -> List[KVSlot]:
         return [KVSlot(dtype) for _ in range(len(self.pre) + L)]

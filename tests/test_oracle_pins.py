@@ -480,3 +480,127 @@ def test_planted_mistake_is_caught(monkeypatch, idx):
     else:
         monkeypatch.setattr(o, name, fn)
     assert not _pins_pass()
+
+
+# ---------------------------------------------------------------- cached extend (verify pass)
+
+def test_extend_equals_sequential_decode_steps():
+    """n tokens in one cached call equal n single-token steps: the causal mask
+    by absolute position and the append-then-attend order are the same."""
+    m = _tiny_model()
+    ids = np.array([3, 17, 5, 11, 0, 19, 8], np.int64)
+    for dtype in ("exact", "fp16", "int8"):
+        kv_a, kv_b = m.new_kv(3, dtype), m.new_kv(3, dtype)
+        m.prefill(ids[:3], 3, kv=kv_a)
+        m.prefill(ids[:3], 3, kv=kv_b)
+        ya = m.extend(ids[3:], 3, kv_a)
+        yb = np.stack([m.decode_step(np.int64(t), 3, kv_b) for t in ids[3:]])
+        assert np.allclose(ya, yb, rtol=0, atol=1e-12), dtype
+        for sa, sb in zip(kv_a, kv_b):
+            assert len(sa) == len(sb) == len(ids)
+            assert np.allclose(sa.k, sb.k, atol=1e-12) and np.allclose(sa.v, sb.v, atol=1e-12)
+
+
+def test_extend_from_empty_exact_cache_is_the_uncached_forward():
+    m = _tiny_model()
+    ids = np.array([1, 2, 3, 4, 5, 6], np.int64)
+    y = m.extend(ids, 2, m.new_kv(2, "exact"))
+    assert np.allclose(y, m.prefill(ids, 2), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- per-iteration residual-norm exit
+
+def test_exit_threshold_infinite_changes_nothing():
+    m = _tiny_model()
+    ids = np.array([4, 9, 13, 2], np.int64)
+    info = {}
+    a = m.prefill(ids, 4, exit_tau=float("inf"), info=info)
+    assert np.array_equal(a, m.prefill(ids, 4))
+    assert list(info["loops"]) == [4, 4, 4, 4]
+
+
+def test_exit_threshold_zero_stops_after_the_first_iteration():
+    """Every norm is above 0: each token keeps the stream of its first loop
+    iteration, so the output is the L = 1 forward's."""
+    m = _tiny_model()
+    ids = np.array([4, 9, 13, 2, 7], np.int64)
+    info = {}
+    y = m.prefill(ids, 5, exit_tau=0.0, info=info)
+    assert np.array_equal(y, m.prefill(ids, 1))
+    assert list(info["loops"]) == [1] * 5
+
+
+def test_exit_loop_counts_are_the_first_norm_crossings():
+    """Before a token freezes its stream is the exit-free one, so its loop
+    count is the first iteration j >= 1 whose input (the stream leaving
+    iteration j - 1) has an L2 norm above the threshold; checked against the
+    exit-free trace by brute force, with a threshold between the norms."""
+    m = _tiny_model(n_pre=1)
+    ids = np.array([4, 9, 13, 2, 7, 1, 18], np.int64)
+    L = 6
+    trace = []
+    m.prefill(ids, L, trace=trace)
+    norms = np.array([[math.sqrt(sum(x * x for x in row)) for row in trace[1 + j]] for j in range(L)])
+    flat = np.sort(norms[:L - 1].ravel())
+    tau = float((flat[len(flat) // 2] + flat[len(flat) // 2 + 1]) / 2)
+    want = []
+    for t in range(len(ids)):
+        cross = [j for j in range(1, L) if norms[j - 1, t] > tau]
+        want.append(cross[0] if cross else L)
+    info = {}
+    m.prefill(ids, L, exit_tau=tau, info=info)
+    assert list(info["loops"]) == want
+    assert 1 < len(set(want))          # the threshold splits the tokens
+
+
+def test_exit_in_decode_equals_the_shallower_step():
+    """A decode token frozen after j iterations outputs what a depth-j step
+    from the same cache outputs (only its own stream reaches the output)."""
+    m = _tiny_model()
+    ids = np.array([3, 17, 5, 11], np.int64)
+    L = 5
+    for tau in (0.5, 2.0, 4.0, 1e9):
+        kv = m.new_kv(L, "fp16")
+        m.prefill(ids, L, kv=kv)
+        snap = [(s.k.copy(), s.v.copy()) for s in kv]
+        info = {}
+        y = m.decode_step(np.int64(6), L, kv, exit_tau=tau, info=info)
+        j = int(info["loops"][0])
+        kv2 = m.new_kv(j, "fp16")
+        for slot, (k, v) in zip(kv2, snap):
+            slot.load_stored(k, v)
+        assert np.array_equal(y, m.decode_step(np.int64(6), j, kv2)), tau
+
+
+# ---------------------------------------------------------------- greedy head and self-speculative step
+
+def test_greedy_head_brute_force():
+    m = _tiny_model()
+    y = np.random.default_rng(3).standard_normal((5, 8))
+    E = m.embed16.astype(np.float64)
+    for r in range(5):
+        scores = [sum(y[r, i] * E[v, i] for i in range(8)) for v in range(E.shape[0])]
+        assert m.greedy_head(y[r:r + 1])[0] == max(range(len(scores)), key=lambda v: (scores[v], -v))
+
+
+@pytest.mark.parametrize("K,L_draft", [(1, 1), (3, 1), (4, 2), (7, 2), (3, 3)])
+def test_spec_step_emits_the_greedy_decode_tokens(K, L_draft):
+    """Greedy self-speculative decoding with an exact verify emits exactly the
+    tokens greedy decoding at the verify depth emits, whatever the draft."""
+    L = 3
+    m = _tiny_model()
+    prompt = np.array([3, 17, 5, 11], np.int64)
+    kv_s, kv_g = m.new_kv(L, "fp16"), m.new_kv(L, "fp16")
+    m.prefill(prompt[:-1], L, kv=kv_s)
+    m.prefill(prompt[:-1], L, kv=kv_g)
+    tok, got = int(prompt[-1]), []
+    while len(got) < 12:
+        out = m.spec_step(tok, K, L_draft, L, kv_s)
+        assert 1 <= len(out) <= K + 1
+        got += out
+        tok = out[-1]
+        assert len(kv_s[0]) == len(prompt) - 1 + len(got)
+    want = m.greedy_decode(int(prompt[-1]), len(got), L, kv_g)
+    assert got == want
+    if L_draft == L:                    # the draft is the verify model: all accepted
+        assert len(m.spec_step(tok, K, L, L, kv_s)) == K + 1
