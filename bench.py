@@ -492,9 +492,9 @@ def decode_roofline(t_step, hbm_bytes, l2_bytes, hbm_gbs, l2_gbs):
 
 
 def loop_read_bytes(tl, blk) -> int:
-    """Bytes the decode kernels read per application of an INT3 block: the
-    library reads an INT4 copy of the INT3 codes (same scales)."""
-    return block_bytes(tl, 4)
+    """Bytes the decode kernels read per application of an INT3 block: its
+    canonical 10-codes-per-word rows and fp16 scales (read natively)."""
+    return block_bytes(tl, 3)
 
 
 def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg, l2_gbs):

@@ -164,9 +164,15 @@ typedef struct tl_block tl_block;
 
 /* Validate a block description and wrap it.  The block references the caller's
  * device memory (no copy); that memory must outlive the block and every model
- * built from it. */
+ * built from it.  Every kernel reads the canonical packed words directly, INT3
+ * included ("Current Status", core inference table, INT3 GEMM row: 10 values
+ * per 32-bit word), so an INT3 block costs its 3.2 bits per weight and
+ * nothing more. */
 tl_status tl_block_create(const tl_block_desc* desc, tl_block** out);
 tl_status tl_block_destroy(tl_block* block);
+
+/* Library-owned device bytes of a block (0: a block allocates nothing). */
+tl_status tl_block_device_bytes(const tl_block* block, size_t* bytes);
 
 /* ------------------------------------------------------------------------
  * Models.  Weight memory is tied to unique blocks, not to effective depth
@@ -289,6 +295,51 @@ tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
                          int n_lanes, float* y_out, float* h_trace,
                          tl_stream stream);
 
+/* Cached forward of `n` consecutive tokens of one lane at its current
+ * position p (positions p .. p+n-1), at loop count L: the verify pass of
+ * self-speculative decode ("Current Status", speculative and adaptive decode
+ * table, self-speculative row: L=2 draft, L=8 verify with the same weights;
+ * "TinyLoop Framework", "What Makes It Different": draft and verify reuse the
+ * same weights).  Every layer appends the n tokens' K/V to the lane's cache
+ * before any of them attends, and token i attends over positions 0 .. p+i.
+ * Each token is computed exactly as a one-token decode step at its position
+ * would be: the result is bit-identical to n successive decode steps.
+ *   ids / h_in  int32 [n] or fp16 [n, d] (exactly one; host or device)
+ *   y_out       fp32 [n, d]  (host or device)
+ *   h_trace     NULL or fp32 [n_pre + L, n, d]
+ * Requirements: 1 <= n <= 8 (and <= the model's max_tokens), 1 <= L <= the
+ * lane's loop slots, p + n <= the cache context.  The lane's position
+ * becomes p + n. */
+tl_status tl_extend(tl_model* model, tl_kv* kv, int lane, const int32_t* ids,
+                    const uint16_t* h_in, int n, int L, float* y_out, float* h_trace,
+                    tl_stream stream);
+
+/* Greedy next tokens through the tied embedding (the model's embedding used as
+ * its output head; the looped forward itself has no logits):
+ *   ids[r] = argmax over v of y[r] . E[v]   (fp32 sums; the lowest v wins a tie)
+ *   y    device fp32 [n, d] final-norm outputs;  ids  device int32 [n]
+ * Requirements: an embedding in the model, 1 <= n <= 8. */
+tl_status tl_greedy_head(tl_model* model, const float* y, int n, int32_t* ids,
+                         tl_stream stream);
+
+/* One greedy self-speculative step of one lane with one weight set and one
+ * cache ("Current Status", self-speculative row; "TinyLoop Framework", "What
+ * Makes It Different").  From the input token `token` at the lane's position
+ * p: K draft tokens d_1..d_K by K one-token steps at L_draft, each the greedy
+ * head of the previous output; then the lane goes back to p and one extend of
+ * [token, d_1 .. d_K] at L_verify gives the verify tokens v_1 .. v_{K+1}; the
+ * longest prefix with d_i == v_i (m tokens) is accepted.  Writes
+ * d_1 .. d_m, v_{m+1} to tokens_out (host int32 [K + 1]) and m + 1 to *n_out
+ * (host); the lane's position becomes p + m + 1 (entries past it are
+ * overwritten later).  The emitted tokens are those m + 1 greedy decode steps
+ * at L_verify would emit.  Synchronises `stream` once (the acceptance is
+ * decided on the host).
+ * Requirements: 1 <= K <= 7, L_draft and L_verify within the lane's slots,
+ * p + K + 1 <= the cache context, 0 <= token < vocab, an embedding. */
+tl_status tl_spec_step(tl_model* model, tl_kv* kv, int lane, int32_t token, int K,
+                       int L_draft, int L_verify, int32_t* tokens_out, int* n_out,
+                       tl_stream stream);
+
 /* ------------------------------------------------------------------------
  * Quantised-weight linear layer (test and measurement hook).  The GEMM every
  * block projection uses:  y[t, n] = sum_k x[t, k] * code[n, k] * scale[n, k/G]
@@ -301,8 +352,8 @@ tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
  *                   (may be NULL when that size is 0)
  * Requirements: N % 64 == 0, K % 64 == 0, group in {64, 128}, K % group == 0,
  * 1 <= T <= 8192; anything else returns TL_ERR_INVALID_ARG (TL_ERR_UNSUPPORTED
- * for another group size) before any launch.
- * bits must be 4 (an INT3 matrix is converted by tl_block_create). */
+ * for another group size) before any launch.  T <= 8 with K % 128 == 0 runs
+ * the decode projection kernel and needs no workspace (size 0). */
 tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes);
 tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N, int K,
                     int group, const uint16_t* x, int T, float* y,

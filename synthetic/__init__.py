@@ -94,6 +94,10 @@ WORKLOADS: Dict[str, Workload] = {
     "tiny": Workload("tiny", SHAPE_TINY, n_pre=0, group=64, bits_pre=4, bits_loop=4,
                      L=(2,), seq=16, steps=0, kv_dtype="none", input_kind="hidden",
                      max_ctx=16),
+    # the tiny block with an INT3 loop block (10 codes per word, group 64)
+    "tiny_int3": Workload("tiny_int3", SHAPE_TINY, n_pre=0, group=64, bits_pre=4, bits_loop=3,
+                          L=(2,), seq=16, steps=0, kv_dtype="none", input_kind="hidden",
+                          max_ctx=16),
     # 407M-shaped prefill, seq 128, L=8, no logits
     "prefill407m": Workload("prefill407m", SHAPE_407M, n_pre=2, group=128, bits_pre=4,
                             bits_loop=4, L=(8,), seq=128, steps=0, kv_dtype="none",

@@ -191,3 +191,14 @@ def test_read_probe_rejects_before_launch():
     assert f(p, 0, 1, p, None) == tl.TL_ERR_INVALID_ARG
     assert f(p, 1024, 0, p, None) == tl.TL_ERR_INVALID_ARG
     assert f(p, 1024, 4097, p, None) == tl.TL_ERR_INVALID_ARG
+
+
+def test_int3_block_wraps_without_device_work():
+    """An INT3 block is wrapped like an INT4 one: no copy, no device work, no
+    library-owned bytes (every kernel reads the canonical INT3 words)."""
+    out = ctypes.c_void_p()
+    assert tl.lib.tl_block_create(ctypes.byref(_desc(bits=3)), ctypes.byref(out)) == tl.TL_OK
+    n = ctypes.c_size_t(7)
+    assert tl.lib.tl_block_device_bytes(out, ctypes.byref(n)) == tl.TL_OK
+    assert n.value == 0
+    assert tl.lib.tl_block_destroy(out) == tl.TL_OK

@@ -1,0 +1,212 @@
+"""CPU model of the decode projection kernel's operand layout (gemv_dec.cu):
+the code pairs each lane extracts from its packed words (the lop3 / prmt /
+HFMA2 bit tricks, emulated bit for bit on fp16 values), the k step and slot
+each pair feeds, and the position the staging step writes each activation to.
+Summing A x B over every lane, k step and slot of a chunk must give the plain
+dot product of the codes with the activations, for INT4 and INT3 rows, for
+every lane and chunk position (the INT3 groups may straddle a lane's codes).
+The slot and position tables are read from the kernel source, so a change
+there is checked here."""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tinyloop_oracle as o
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = open(os.path.join(ROOT, "weight_shared_looped_b200", "csrc", "gemv_dec.cu")).read()
+
+
+def _f16(bits):
+    return np.array([bits & 0xFFFF], dtype=np.uint16).view(np.float16)[0]
+
+
+def _halves(x):
+    return float(_f16(x)), float(_f16(x >> 16))
+
+
+def _hfma2(x, m, a):
+    lo, hi = _halves(x)
+    r = [np.float16(np.float64(v) * mm + aa) for v, mm, aa in ((lo, m[0], a[0]), (hi, m[1], a[1]))]
+    return float(r[0]), float(r[1])
+
+
+def _lop3_ea(a, b, c):
+    return ((a & b) | c) & 0xFFFFFFFF
+
+
+def _prmt(a, b, sel):
+    src = [(a >> (8 * i)) & 0xFF for i in range(4)] + [(b >> (8 * i)) & 0xFF for i in range(4)]
+    return sum(src[(sel >> (4 * i)) & 7] << (8 * i) for i in range(4))
+
+
+def _const(pattern):
+    m = re.search(pattern, SRC)
+    assert m, pattern
+    return m
+
+
+# ---------------------------------------------------------------- the kernel's extraction steps
+def int4_pairs(w):
+    w8 = w >> 8
+    lo = lambda x: _hfma2(_lop3_ea(x, 0x000F000F, 0x64006400), (1.0, 1.0), (-1032.0, -1032.0))
+    hi = lambda x: _hfma2(_lop3_ea(x, 0x00F000F0, 0x64006400), (0.0625, 0.0625), (-72.0, -72.0))
+    return [lo(w), hi(w), lo(w8), hi(w8)]
+
+
+def int3_pair_i6(w, i):
+    return _hfma2(_lop3_ea(w >> (3 * i), 0x001C0007, 0x64006400), (1.0, 0.25), (-1028.0, -260.0))
+
+
+def int3_pair_c4(a, b):
+    return _hfma2(_lop3_ea(_prmt(a, b, 0x0501), 0x00700070, 0x64006400), (0.0625, 0.0625),
+                  (-68.0, -68.0))
+
+
+def int3_pair_c5(a, b):
+    return _hfma2(_lop3_ea(_prmt(a, b, 0x6521), 0x03800380, 0x64006400), (0.0078125, 0.0078125),
+                  (-12.0, -12.0))
+
+
+def test_extraction_constants_match_the_kernel():
+    for c in ("0x001C0007u, 0x64006400u", "h2c(1.f, 0.25f), h2c(-1028.f, -260.f)",
+              "prmt(a, b, 0x0501u), 0x00700070u", "h2c(-68.f, -68.f)",
+              "prmt(a, b, 0x6521u), 0x03800380u", "h2c(-12.f, -12.f)",
+              "lop3_ea(w, 0x000F000Fu, 0x64006400u), one, lo_b",
+              "lop3_ea(w, 0x00F000F0u, 0x64006400u), sixteenth, hi_b"):
+        assert c in SRC, c
+
+
+# ---------------------------------------------------------------- slot / position tables
+def int3_slot(L, t):
+    q, i = divmod(L, 10)
+    return {0: (2 * q, 2 * t), 6: (2 * q, 2 * t + 1), 1: (2 * q, 2 * t + 8), 7: (2 * q, 2 * t + 9),
+            2: (2 * q + 1, 2 * t), 8: (2 * q + 1, 2 * t + 1), 3: (2 * q + 1, 2 * t + 8),
+            9: (2 * q + 1, 2 * t + 9), 4: (8 + (q >> 1), 2 * t + (q & 1)),
+            5: (8 + (q >> 1), 2 * t + 8 + (q & 1))}[i]
+
+
+def test_int3_slot_table_matches_the_kernel():
+    for i, (j, s) in {0: ("2 * q", "2 * t"), 6: ("2 * q", "2 * t + 1"), 1: ("2 * q", "2 * t + 8"),
+                      7: ("2 * q", "2 * t + 9"), 2: ("2 * q + 1", "2 * t"),
+                      8: ("2 * q + 1", "2 * t + 1"), 3: ("2 * q + 1", "2 * t + 8"),
+                      9: ("2 * q + 1", "2 * t + 9"), 4: ("8 + (q >> 1)", "2 * t + (q & 1)")}.items():
+        assert f"case {i}: j = {j}; return {s};" in SRC, i
+
+
+def xpos(k, bits):
+    if bits == 4:
+        c, r = divmod(k, 128)
+        t, q, e = r >> 5, (r >> 3) & 3, k & 7
+        j = 2 * q + ((e >> 1) & 1)
+        s = 2 * t + (8 if e & 1 else 0) + (1 if e >= 4 else 0)
+        return c * 128 + 16 * j + s
+    c, r = divmod(k, 160)
+    t, L = divmod(r, 40)
+    j, s = int3_slot(L, t)
+    return c * 160 + 16 * j + s
+
+
+@pytest.mark.parametrize("bits,K", [(4, 256), (3, 480)])
+def test_staging_positions_are_a_permutation(bits, K):
+    pos = [xpos(k, bits) for k in range(K)]
+    assert sorted(pos) == list(range(K))
+
+
+def test_int4_staging_half2_stores_match_xpos():
+    # the staging writes (e0,e4) at base, (e1,e5) at +8, (e2,e6) at +16, (e3,e7) at +24
+    for k0 in range(0, 512, 8):
+        base = xpos(k0, 4)
+        for e, off in ((0, 0), (4, 1), (1, 8), (5, 9), (2, 16), (6, 17), (3, 24), (7, 25)):
+            assert xpos(k0 + e, 4) == base + off
+
+
+# ---------------------------------------------------------------- one chunk, all lanes
+def _lane_fragments_int4(words):
+    """words: the lane's 4 packed words of one row -> {k step: (pair (2t,2t+1), pair (2t+8,2t+9))}"""
+    frags = {}
+    for q in range(4):
+        p = int4_pairs(int(words[q]))
+        frags[2 * q] = (p[0], p[1])
+        frags[2 * q + 1] = (p[2], p[3])
+    return frags
+
+
+def _lane_fragments_int3(words, scales_of_L):
+    """Like the INT4 case; INT3 pairs are scaled in fp16 by their codes' group scales."""
+    def sc(pair, La, Lb):
+        return (float(np.float16(pair[0] * scales_of_L(La))), float(np.float16(pair[1] * scales_of_L(Lb))))
+    frags = {}
+    for q in range(4):
+        w, L = int(words[q]), 10 * q
+        frags[2 * q] = (sc(int3_pair_i6(w, 0), L, L + 6), sc(int3_pair_i6(w, 1), L + 1, L + 7))
+        frags[2 * q + 1] = (sc(int3_pair_i6(w, 2), L + 2, L + 8), sc(int3_pair_i6(w, 3), L + 3, L + 9))
+    w = [int(x) for x in words]
+    frags[8] = (sc(int3_pair_c4(w[0], w[1]), 4, 14), sc(int3_pair_c5(w[0], w[1]), 5, 15))
+    frags[9] = (sc(int3_pair_c4(w[2], w[3]), 24, 34), sc(int3_pair_c5(w[2], w[3]), 25, 35))
+    return frags
+
+
+def _mma_dot(frags_per_lane, xs_chunk, cw):
+    """Sum over k steps and slots of A[slot] * B[slot], B read where ldmatrix reads it:
+    k step j, slot s at position 16 j + s of the chunk's staged row."""
+    total = 0.0
+    for t, frags in enumerate(frags_per_lane):
+        for j, (pa, pb) in frags.items():
+            for slot, v in ((2 * t, pa[0]), (2 * t + 1, pa[1]), (2 * t + 8, pb[0]), (2 * t + 9, pb[1])):
+                total += v * xs_chunk[16 * j + slot]
+    return total
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_int4_chunk_dot_product(seed):
+    rng = np.random.default_rng(seed)
+    K = 256
+    codes = rng.integers(-8, 8, size=(1, K)).astype(np.int8)
+    codes[0, :8] = [-8, 7, -8, 7, 0, -1, 1, 3]
+    words = o.pack_codes(codes, 4)[0]
+    x = rng.standard_normal(K).astype(np.float16).astype(np.float64)
+    xs = np.zeros(K)
+    for k in range(K):
+        xs[xpos(k, 4)] = x[k]
+    for c in range(K // 128):
+        frags = [_lane_fragments_int4(words[16 * c + 4 * t:16 * c + 4 * t + 4]) for t in range(4)]
+        got = _mma_dot(frags, xs[128 * c:128 * c + 128], 128)
+        want = float(codes[0, 128 * c:128 * c + 128].astype(np.float64) @ x[128 * c:128 * c + 128])
+        assert abs(got - want) <= 1e-9 * max(1.0, abs(want)), (c, got, want)
+
+
+@pytest.mark.parametrize("G", [64, 128])
+@pytest.mark.parametrize("seed", range(3))
+def test_int3_chunk_dot_product_with_straddling_groups(G, seed):
+    rng = np.random.default_rng(100 + seed)
+    K = 2048                                              # 205 words padded to 208: 13 chunks
+    w = rng.standard_normal((1, K)).astype(np.float32) * 0.02
+    codes, scales = o.quantize_groupwise(w, 3, G)
+    words = o.pack_codes(codes, 3)[0]
+    nvec = len(words) // 4
+    nch = (nvec + 3) // 4
+    x = np.zeros(nch * 160)
+    x[:K] = rng.standard_normal(K).astype(np.float16).astype(np.float64)
+    xs = np.zeros(nch * 160)
+    for k in range(nch * 160):
+        xs[xpos(k, 3)] = x[k]
+    s = scales[0].astype(np.float64)
+    gpr = K // G
+    want_total = got_total = 0.0
+    for c in range(nch):
+        frags = []
+        for t in range(4):
+            vi = 4 * c + t
+            lw = words[4 * vi:4 * vi + 4] if vi < nvec else np.zeros(4, np.uint32)
+            k0 = 160 * c + 40 * t
+            ga = min(k0 // G, gpr - 1)
+            gb = min(ga + 1, gpr - 1)
+            bnd = (k0 // G + 1) * G - k0
+            frags.append(_lane_fragments_int3(lw, lambda L: s[ga] if L < bnd else s[gb]))
+        got_total += _mma_dot(frags, xs[160 * c:160 * c + 160], 160)
+    deq = np.array([float(np.float16(codes[0, k] * s[k // G])) for k in range(K)])
+    want_total = float(deq @ x[:K])
+    assert abs(got_total - want_total) <= 1e-9 * max(1.0, abs(want_total)), (got_total, want_total)

@@ -124,14 +124,13 @@ def test_tcgen05_gemm_byte_to_code_pair():
         assert np.array_equal(c_hi, codes[:, 2 * bb + 1].astype(np.float64))
 
 
-def test_gemv_nibble_pairs():
-    src = _src("gemm_mma.cu")
-    assert '"r"(w), "r"(0x000F000Fu), "r"(0x64006400u)' in src
-    assert '"r"(w), "r"(0x00F000F0u), "r"(0x64006400u)' in src
-    assert "__float2half_rn(1032.0f), __float2half_rn(1032.0f)" in src
-    assert "__float2half_rn(0.0625f), __float2half_rn(0.0625f)" in src
-    assert "__float2half_rn(-72.0f), __float2half_rn(-72.0f)" in src
-    assert "const int sh = (j & 1) * 8;" in src
+def test_decode_projection_nibble_pairs():
+    src = _src("gemv_dec.cu")
+    assert "lop3_ea(w, 0x000F000Fu, 0x64006400u), one, lo_b" in src
+    assert "lop3_ea(w, 0x00F000F0u, 0x64006400u), sixteenth, hi_b" in src
+    assert "lop3_ea(w8, 0x000F000Fu, 0x64006400u), one, lo_b" in src
+    assert "const uint32_t w8 = w >> 8;" in src
+    assert "h2c(-1032.f, -1032.f), hi_b = h2c(-72.f, -72.f)" in src
     rng = np.random.default_rng(1)
     words, codes = _int4_words(rng, 1 << 16)
     # pairs (0, 4), (1, 5) from w; (2, 6), (3, 7) from w >> 8
@@ -139,10 +138,57 @@ def test_gemv_nibble_pairs():
         w = words >> U32(sh)
         lo_a, hi_a = halves(lop3(w, U32(0x000F000F), U32(0x64006400), 0xEA))
         lo_b, hi_b = halves(lop3(w, U32(0x00F000F0), U32(0x64006400), 0xEA))
-        assert np.array_equal(hsub(lo_a, 1032.0), codes[:, k0])
-        assert np.array_equal(hsub(hi_a, 1032.0), codes[:, k0 + 4])
+        assert np.array_equal(hfma(lo_a, 1.0, -1032.0), codes[:, k0])
+        assert np.array_equal(hfma(hi_a, 1.0, -1032.0), codes[:, k0 + 4])
         assert np.array_equal(hfma(lo_b, 0.0625, -72.0), codes[:, k1])
         assert np.array_equal(hfma(hi_b, 0.0625, -72.0), codes[:, k1 + 4])
+
+
+def _int3_words(rng, n):
+    codes = rng.integers(-4, 4, size=(n, 10)).astype(np.int8)
+    codes[: 8 ** 2] = np.stack(np.meshgrid(np.arange(-4, 4), np.arange(-4, 4)), -1).reshape(-1, 2).repeat(5, 1)
+    return o.pack_codes(codes, 3)[:, 0], codes
+
+
+def test_decode_projection_int3_pairs():
+    """The decode kernel's INT3 pairs: codes (i, i + 6) of a word, and codes 4
+    and 5 of two words, over every code value in every position."""
+    src = _src("gemv_dec.cu")
+    for c in ["lop3_ea(w >> (3 * I), 0x001C0007u, 0x64006400u)", "h2c(1.f, 0.25f), h2c(-1028.f, -260.f)",
+              "lop3_ea(prmt(a, b, 0x0501u), 0x00700070u, 0x64006400u)", "h2c(0.0625f, 0.0625f), h2c(-68.f, -68.f)",
+              "lop3_ea(prmt(a, b, 0x6521u), 0x03800380u, 0x64006400u)",
+              "h2c(0.0078125f, 0.0078125f), h2c(-12.f, -12.f)"]:
+        assert c in src, c
+    rng = np.random.default_rng(5)
+    words, codes = _int3_words(rng, 1 << 14)
+    for i in range(4):
+        lo, hi = halves(lop3(words >> U32(3 * i), U32(0x001C0007), U32(0x64006400), 0xEA))
+        assert np.array_equal(hfma(lo, 1.0, -1028.0), codes[:, i])
+        assert np.array_equal(hfma(hi, 0.25, -260.0), codes[:, i + 6])
+    wa, wb = words, np.roll(words, 1)
+    ca, cb = codes, np.roll(codes, 1, axis=0)
+    lo, hi = halves(lop3(prmt(wa, wb, 0x0501), U32(0x00700070), U32(0x64006400), 0xEA))
+    assert np.array_equal(hfma(lo, 0.0625, -68.0), ca[:, 4])
+    assert np.array_equal(hfma(hi, 0.0625, -68.0), cb[:, 4])
+    lo, hi = halves(lop3(prmt(wa, wb, 0x6521), U32(0x03800380), U32(0x64006400), 0xEA))
+    assert np.array_equal(hfma(lo, 0.0078125, -12.0), ca[:, 5])
+    assert np.array_equal(hfma(hi, 0.0078125, -12.0), cb[:, 5])
+
+
+def test_tcgen05_gemm_int3_consecutive_pairs():
+    """The tensor-core GEMM's INT3 pairs (codes 2c, 2c + 1 of a word at an even
+    position i): shift, 6-bit mask, multiply by 1 + 2^13, lop3, less 1028."""
+    src = _src("gemm_tc.cu")
+    for c in ["const uint32_t y = ((v[q] >> (3 * i)) & 0x3Fu) * 8193u;",
+              '"r"(y), "r"(0x00070007u), "r"(0x64006400u)', "__float2half_rn(1028.0f)"]:
+        assert c in src, c
+    rng = np.random.default_rng(6)
+    words, codes = _int3_words(rng, 1 << 14)
+    for i in (0, 2, 4, 6, 8):
+        y = (((words >> U32(3 * i)) & U32(0x3F)) * U32(8193)).astype(U32)
+        lo, hi = halves(lop3(y, U32(0x00070007), U32(0x64006400), 0xEA))
+        assert np.array_equal(hsub(lo, 1028.0), codes[:, i])
+        assert np.array_equal(hsub(hi, 1028.0), codes[:, i + 1])
 
 
 def _int8_words(rng, n):

@@ -64,3 +64,28 @@ def test_linear_tc_kernel(N, K, T, group):
     err = np.linalg.norm(y - ref) / np.linalg.norm(ref)
     assert err <= 1e-3, err
     assert np.abs(y - ref).max() <= 5e-3 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("N,K,T,group", [
+    (64, 128, 1, 64), (128, 256, 8, 64), (2048, 2048, 1, 128), (6144, 2048, 3, 128),
+    (16384, 2048, 8, 128), (2048, 8192, 5, 128), (768, 1024, 7, 64), (192, 384, 2, 128),
+])
+def test_linear_decode_projection_kernel(N, K, T, group):
+    """Decode-sized calls (T <= 8, K % 128 == 0) run the decode projection
+    kernel: no split-K, the eight warps of a CTA split K and add in warp order;
+    exact codes with the group scale applied to fp32 sums (G = 64: one sum per
+    group), so only the summation order differs from the exact product."""
+    assert tl.tl_linear_workspace_bytes(N, K, T) == 0
+    words, scales, x, ref = _case(N, K, T, group, seed=N + K + T + 7)
+    y = _run(words, scales, x, N, K, group)
+    assert np.abs(y - ref).max() <= 1e-5 * np.abs(ref).max() + 1e-6
+
+
+def test_linear_decode_projection_rows_independent():
+    """A token's result does not depend on the other tokens of the call."""
+    N, K, group = 2048, 2048, 128
+    words, scales, x, _ = _case(N, K, 8, group, seed=99)
+    y8 = _run(words, scales, x, N, K, group)
+    for t in (0, 3, 7):
+        y1 = _run(words, scales, x[t:t + 1], N, K, group)
+        assert np.array_equal(y1[0], y8[t])

@@ -64,6 +64,7 @@ _SIGS = {
     "tl_attention_prefill": ([P, P, P, I, I, I, P, P], I),
     "tl_block_create": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(P)], I),
     "tl_block_destroy": ([P], I),
+    "tl_block_device_bytes": ([P, ctypes.POINTER(SZ)], I),
     "tl_model_create": ([ctypes.POINTER(ModelDesc), ctypes.POINTER(P)], I),
     "tl_model_destroy": ([P], I),
     "tl_model_device_bytes": ([P, ctypes.POINTER(SZ)], I),
@@ -81,6 +82,9 @@ _SIGS = {
     "tl_prefill": ([P, P, P, I, I, P, I, P, P, P], I),
     "tl_decode_step": ([P, P, P, P, P, I, P, P, P], I),
     "tl_sync_status": ([P, P], I),
+    "tl_extend": ([P, P, I, P, P, I, I, P, P, P], I),
+    "tl_greedy_head": ([P, P, I, P, P], I),
+    "tl_spec_step": ([P, P, I, ctypes.c_int32, I, I, I, P, ctypes.POINTER(I), P], I),
     "tl_linear_workspace_bytes": ([I, I, I, ctypes.POINTER(SZ)], I),
     "tl_linear": ([P, P, I, I, I, P, I, P, P, P], I),
     "tl_linear_noalloc": ([P, P, I, I, I, P, I, P, P], I),
@@ -175,6 +179,12 @@ def tl_block_create(cfg: dict, packed: dict) -> int:
 
 def tl_block_destroy(block: int) -> None:
     _check(lib.tl_block_destroy(block))
+
+
+def tl_block_device_bytes(block: int) -> int:
+    b = SZ()
+    _check(lib.tl_block_device_bytes(block, ctypes.byref(b)))
+    return b.value
 
 
 def tl_model_create(pre: Sequence[int], loop: int, embed, vocab: int, gamma_final,
@@ -273,6 +283,27 @@ def tl_decode_step(model: int, kv: int, ids=None, h_in=None, *, L_per_lane: Sequ
     arr = _int_array(L_per_lane)
     _check(lib.tl_decode_step(model, kv, _ptr(ids), _ptr(h_in), ctypes.cast(arr, P),
                               len(L_per_lane), _ptr(y_out), _ptr(h_trace), _stream(stream)))
+
+
+def tl_extend(model: int, kv: int, lane: int, ids=None, h_in=None, *, L: int, y_out,
+              h_trace=None, stream=None) -> None:
+    n = (ids if ids is not None else h_in).shape[0]
+    _check(lib.tl_extend(model, kv, lane, _ptr(ids), _ptr(h_in), n, L, _ptr(y_out),
+                         _ptr(h_trace), _stream(stream)))
+
+
+def tl_greedy_head(model: int, y, ids, stream=None) -> None:
+    _check(lib.tl_greedy_head(model, _ptr(y), y.shape[0], _ptr(ids), _stream(stream)))
+
+
+def tl_spec_step(model: int, kv: int, lane: int, token: int, K: int, L_draft: int,
+                 L_verify: int, stream=None):
+    """Returns the emitted tokens (a list of 1 .. K + 1 ids)."""
+    out = (ctypes.c_int32 * (K + 1))()
+    n = I()
+    _check(lib.tl_spec_step(model, kv, lane, token, K, L_draft, L_verify,
+                            ctypes.cast(out, P), ctypes.byref(n), _stream(stream)))
+    return list(out[:n.value])
 
 
 def tl_linear_workspace_bytes(N: int, K: int, T: int) -> int:

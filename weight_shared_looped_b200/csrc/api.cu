@@ -64,11 +64,7 @@ using namespace tl;
 // Objects
 // ============================================================================
 struct tl_block {
-  tl_block_desc d;
-  // INT4 canonical words the GEMM kernels read: the caller's words for an
-  // INT4 block, a library-owned INT4 copy of the same codes for an INT3 block.
-  const uint32_t* w4[5];
-  std::vector<void*> owned;
+  tl_block_desc d;   // every kernel reads the caller's canonical words (INT4 or INT3)
 };
 
 struct tl_kv {
@@ -84,6 +80,7 @@ struct tl_kv {
 struct RowMap {
   int lane[kMaxLanes];   // lane of each decode row
   int cum[kMaxLanes];    // cache layers of the lanes before it
+  int off[kMaxLanes];    // the row's position = its lane's position + off
 };
 
 struct GraphEntry {
@@ -112,9 +109,13 @@ struct tl_model {
   __half *q, *k, *v;
   __half* u;
   float* part;
-  float* part2;          // decode: gate|up partials read by the down projection
   float* y;
   int32_t* lane_map;
+  int32_t* ident_map;    // rows 0..7 -> 0..7 (extend, speculative steps)
+  int32_t* spec_ids;     // speculative step: the input token and the drafts [16]
+  int32_t* spec_ver;     // speculative step: the verify tokens [16]
+  float* head_ps;        // greedy head partials [head_parts()][8]
+  int* head_pv;
   int* status;
   float2* rope;
   std::map<std::string, GraphEntry> graphs_cache;
@@ -216,45 +217,18 @@ TL_API tl_status tl_block_create(const tl_block_desc* desc, tl_block** out) {
                "NULL weight pointer in block description");
   std::unique_ptr<tl_block> b(new tl_block());
   b->d = d;
-  const uint32_t* src[5] = {d.w_qkv, d.w_o, d.w_gate, d.w_up, d.w_down};
-  const int Ns[5] = {3 * d.d_model, d.d_model, d.ffn, d.ffn, d.d_model};
-  const int Ks[5] = {d.d_model, d.d_model, d.d_model, d.d_model, d.ffn};
-  if (d.bits == 4) {
-    for (int i = 0; i < 5; ++i) b->w4[i] = src[i];
-  } else {
-    cudaStream_t s;
-    TL_CUDA(cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking));
-    for (int i = 0; i < 5; ++i) {
-      void* p = nullptr;
-      if (cudaMalloc(&p, (size_t)Ns[i] * (Ks[i] / 8) * 4) != cudaSuccess) {
-        for (void* q : b->owned) cudaFree(q);
-        cudaStreamDestroy(s);
-        return set_error(TL_ERR_OOM, "cannot allocate the INT4 copy of an INT3 matrix");
-      }
-      b->owned.push_back(p);
-      tl_status st = launch_int3_to_int4(src[i], Ns[i], Ks[i], (uint32_t*)p, s);
-      if (st != TL_OK) {
-        for (void* q : b->owned) cudaFree(q);
-        cudaStreamDestroy(s);
-        return st;
-      }
-      b->w4[i] = (const uint32_t*)p;
-    }
-    cudaError_t e = cudaStreamSynchronize(s);
-    cudaStreamDestroy(s);
-    if (e != cudaSuccess) {
-      for (void* q : b->owned) cudaFree(q);
-      return set_error(TL_ERR_CUDA, "INT3 conversion failed: %s", cudaGetErrorString(e));
-    }
-  }
   *out = b.release();
   return ok();
 }
 
 TL_API tl_status tl_block_destroy(tl_block* block) {
-  if (!block) return ok();
-  for (void* p : block->owned) cudaFree(p);
   delete block;
+  return ok();
+}
+
+TL_API tl_status tl_block_device_bytes(const tl_block* block, size_t* bytes) {
+  TL_CHECK_ARG(block && bytes, "NULL argument");
+  *bytes = 0;   // a block references the caller's packed words; it allocates nothing
   return ok();
 }
 
@@ -270,7 +244,9 @@ struct GemmShape {
 size_t part_floats(const tl_model* m, int T) {
   const GemmShape gs[4] = {{3 * m->d, m->d}, {m->d, m->d}, {2 * m->F, m->d}, {m->d, m->F}};
   size_t best = 0;
-  for (auto& g : gs) best = std::max(best, (size_t)gemm_splits(g.N, g.K, T) * T * g.N);
+  for (auto& g : gs)
+    for (int bits = 3; bits <= 4; ++bits)
+      best = std::max(best, (size_t)gemm_splits(g.N, g.K, T, bits) * T * g.N);
   return best;
 }
 
@@ -349,10 +325,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
   void* p_u; void* p_part; void* p_y; void* p_lid; void* p_status; void* p_rope;
-  void* p_part2;
-  size_t part2_floats = 0;
-  for (int t = 1; t <= md.max_lanes; ++t)
-    part2_floats = std::max(part2_floats, (size_t)gemm_splits(2 * F, d, t) * t * 2 * F);
+  void* p_ident; void* p_sids; void* p_sver; void* p_hps; void* p_hpv;
   Slot slots[] = {
       {&p_ids, (size_t)T * 4},
       {&p_hin, (size_t)T * d * 2},
@@ -364,9 +337,13 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_v, (size_t)T * d * 2},
       {&p_u, (size_t)T * F * 2},
       {&p_part, maxpart * 4},
-      {&p_part2, part2_floats * 4},
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
+      {&p_ident, (size_t)kMaxLanes * 4},
+      {&p_sids, 16 * 4},
+      {&p_sver, 16 * 4},
+      {&p_hps, (size_t)head_parts() * 8 * 4},
+      {&p_hpv, (size_t)head_parts() * 8 * 4},
       {&p_status, 256},
       {&p_rope, (size_t)md.max_ctx * (m->hd / 2) * sizeof(float2)},
   };
@@ -390,9 +367,13 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->v = (__half*)p_v;
   m->u = (__half*)p_u;
   m->part = (float*)p_part;
-  m->part2 = (float*)p_part2;
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
+  m->ident_map = (int32_t*)p_ident;
+  m->spec_ids = (int32_t*)p_sids;
+  m->spec_ver = (int32_t*)p_sver;
+  m->head_ps = (float*)p_hps;
+  m->head_pv = (int*)p_hpv;
   m->status = (int*)p_status;
   m->rope = (float2*)p_rope;
   // RoPE table: angle = pos * theta^(-2i/hd), computed in double, rounded to fp32
@@ -410,6 +391,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
     cudaError_t e1 = cudaMemcpy(m->rope, tab.data(), tab.size() * sizeof(float2),
                                 cudaMemcpyHostToDevice);
     cudaError_t e2 = cudaMemcpy(m->lane_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
+    if (e2 == cudaSuccess)
+      e2 = cudaMemcpy(m->ident_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
@@ -610,40 +593,41 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
   const tl_block_desc& d = b->d;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
+  a.bits = d.bits;
   a.G = d.group;
   a.x = x;
   a.T = T;
   a.part = m->part;
   switch (which) {
     case 0:  // QKV
-      a.w0 = a.w1 = b->w4[0];
+      a.w0 = a.w1 = d.w_qkv;
       a.s0 = a.s1 = (const __half*)d.s_qkv;
       a.N = a.n_split = 3 * m->d;
       a.K = m->d;
       break;
     case 1:  // O
-      a.w0 = a.w1 = b->w4[1];
+      a.w0 = a.w1 = d.w_o;
       a.s0 = a.s1 = (const __half*)d.s_o;
       a.N = a.n_split = m->d;
       a.K = m->d;
       break;
     case 2:  // gate | up
-      a.w0 = b->w4[2];
+      a.w0 = d.w_gate;
       a.s0 = (const __half*)d.s_gate;
-      a.w1 = b->w4[3];
+      a.w1 = d.w_up;
       a.s1 = (const __half*)d.s_up;
       a.n_split = m->F;
       a.N = 2 * m->F;
       a.K = m->d;
       break;
     default:  // down
-      a.w0 = a.w1 = b->w4[4];
+      a.w0 = a.w1 = d.w_down;
       a.s0 = a.s1 = (const __half*)d.s_down;
       a.N = a.n_split = m->d;
       a.K = m->F;
       break;
   }
-  a.splits = gemm_splits(a.N, a.K, T);
+  a.splits = gemm_splits(a.N, a.K, T, a.bits);
   a.status = m->status;
   return a;
 }
@@ -661,66 +645,38 @@ NormArgs norm_args(const tl_model* m, int rows) {
   return n;
 }
 
-// One block application (everything after the input RMSNorm, up to and
-// including the down projection; the residual add of the down projection is
-// done by the next norm).  `rows` rows are active.
+// One prefill block application (everything after the input RMSNorm, up to
+// and including the down projection; the residual add of the down projection
+// is done by the next norm).
 tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
-                             int lane, bool decode, const int32_t* lane_of_row, const RowMap* rm,
-                             cudaStream_t s) {
+                             int lane, cudaStream_t s) {
   // QKV
   GemmArgs g = gemm_args(m, b, 0, m->x, rows);
   TL_TRY(launch_gemm(g, s));
-  if (!decode) {
-    RopeKvArgs r;
-    memset(&r, 0, sizeof(r));
-    r.part = m->part;
-    r.S = g.splits;
-    r.rows = rows;
-    r.d = m->d;
-    r.H = m->H;
-    r.hd = m->hd;
-    r.rope_cs = m->rope;
-    r.q = m->q;
-    r.k = m->k;
-    r.v = m->v;
-    if (kv) {
-      r.kv_base = kv->buffer + kKvHeaderBytes;
-      r.hdr = (const KvHeader*)kv->buffer;
-      r.layer_bytes = kv->layer_bytes;
-      r.kv_region_bytes = kv->region_bytes;
-      r.layer = layer;
-      r.max_ctx = kv->max_ctx;
-      r.kv_int8 = kv->dtype == TL_KV_INT8;
-    }
-    r.lane = lane;
-    TL_TRY(launch_rope_kv(r, s));
-    TL_TRY(launch_attn_prefill(m->q, m->k, m->v, m->attn, rows, m->H, m->hd, s));
-  } else {
-    // RoPE, KV append, split attention and merge in one launch
-    DecodeAttnArgs da;
-    memset(&da, 0, sizeof(da));
-    da.out = m->attn;
-    da.rows = rows;
-    da.H = m->H;
-    da.hd = m->hd;
-    da.d = m->d;
-    da.kv_base = kv->buffer + kKvHeaderBytes;
-    da.hdr = (const KvHeader*)kv->buffer;
-    da.layer_bytes = kv->layer_bytes;
-    da.kv_region_bytes = kv->region_bytes;
-    da.layer = layer;
-    da.max_ctx = kv->max_ctx;
-    da.kv_int8 = kv->dtype == TL_KV_INT8;
-    for (int i = 0; i < kMaxLanes; ++i) {
-      da.row_lane[i] = rm->lane[i];
-      da.row_cum[i] = rm->cum[i];
-    }
-    da.qkv_part = m->part;
-    da.qkv_S = g.splits;
-    da.rope_cs = m->rope;
-    da.chunks = m->decode_chunks;
-    TL_TRY(launch_attn_decode_fused(da, s));
+  RopeKvArgs r;
+  memset(&r, 0, sizeof(r));
+  r.part = m->part;
+  r.S = g.splits;
+  r.rows = rows;
+  r.d = m->d;
+  r.H = m->H;
+  r.hd = m->hd;
+  r.rope_cs = m->rope;
+  r.q = m->q;
+  r.k = m->k;
+  r.v = m->v;
+  if (kv) {
+    r.kv_base = kv->buffer + kKvHeaderBytes;
+    r.hdr = (const KvHeader*)kv->buffer;
+    r.layer_bytes = kv->layer_bytes;
+    r.kv_region_bytes = kv->region_bytes;
+    r.layer = layer;
+    r.max_ctx = kv->max_ctx;
+    r.kv_int8 = kv->dtype == TL_KV_INT8;
   }
+  r.lane = lane;
+  TL_TRY(launch_rope_kv(r, s));
+  TL_TRY(launch_attn_prefill(m->q, m->k, m->v, m->attn, rows, m->H, m->hd, s));
   // O projection, then the residual add of its split-K partial sums and the
   // RMSNorm before the MLP in one norm kernel
   g = gemm_args(m, b, 1, m->attn, rows);
@@ -732,31 +688,124 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   n.n_add = rows;
   n.gamma_next = b->d.gamma_ffn;
   n.n_next = rows;
-  n.out_row = lane_of_row;
   TL_TRY(launch_residual_norm(n, s));
   // SwiGLU MLP
   g = gemm_args(m, b, 2, m->x, rows);
-  if (decode) {
-    // gate|up partials go to their own buffer; the down projection's
-    // activation staging forms silu(gate) * up from them
-    g.part = m->part2;
+  if (gemm_tc_eligible(g.N, g.K, rows, g.bits) && g.splits == 1 && m->F % 64 == 0) {
+    g.swiglu_u = m->u;   // the GEMM's epilogue forms silu(gate) * up
     TL_TRY(launch_gemm(g, s));
-    GemmArgs dn = gemm_args(m, b, 3, m->u, rows);
-    dn.x_part = m->part2;
-    dn.x_S = g.splits;
-    dn.x_F = m->F;
-    TL_TRY(launch_gemm(dn, s));
   } else {
-    if (gemm_tc_eligible(g.N, g.K, rows) && g.splits == 1 && m->F % 64 == 0) {
-      g.swiglu_u = m->u;   // the GEMM's epilogue forms silu(gate) * up
-      TL_TRY(launch_gemm(g, s));
-    } else {
-      TL_TRY(launch_gemm(g, s));
-      TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
-    }
-    g = gemm_args(m, b, 3, m->u, rows);
     TL_TRY(launch_gemm(g, s));
+    TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
   }
+  g = gemm_args(m, b, 3, m->u, rows);
+  TL_TRY(launch_gemm(g, s));
+  return ok();
+}
+
+// One decode block application for `rows` active rows: four decode
+// projections (the QKV and gate/up ones form their own pre-norm from the
+// residual stream; the O and down ones add into it) around the fused decode
+// attention.  `trace` (null or [trace_rows][d], rows by lane) receives the
+// residual stream after the block for every row, active or not.
+tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
+                               const RowMap* rm, const int32_t* lane_of_row, float* trace,
+                               int trace_rows, bool split_attn, cudaStream_t s) {
+  const tl_block_desc& bd = b->d;
+  const int d = m->d, F = m->F;
+  DecGemvArgs p;
+  memset(&p, 0, sizeof(p));
+  p.G = bd.group;
+  p.bits = bd.bits;
+  p.T = rows;
+  p.eps = m->eps;
+  // QKV: q, k, v sums -> part [1][rows][3d]
+  p.w0 = bd.w_qkv;
+  p.s0 = (const __half*)bd.s_qkv;
+  p.N = 3 * d;
+  p.K = d;
+  p.h = m->h;
+  p.gamma = bd.gamma_attn;
+  p.epi = DEC_EPI_OUT;
+  p.out = m->part;
+  TL_TRY(launch_dec_gemv(p, s));
+  // RoPE, KV append, split attention and merge in one launch
+  DecodeAttnArgs da;
+  memset(&da, 0, sizeof(da));
+  da.out = m->attn;
+  da.rows = rows;
+  da.H = m->H;
+  da.hd = m->hd;
+  da.d = d;
+  da.kv_base = kv->buffer + kKvHeaderBytes;
+  da.hdr = (const KvHeader*)kv->buffer;
+  da.layer_bytes = kv->layer_bytes;
+  da.kv_region_bytes = kv->region_bytes;
+  da.layer = layer;
+  da.max_ctx = kv->max_ctx;
+  da.kv_int8 = kv->dtype == TL_KV_INT8;
+  for (int i = 0; i < kMaxLanes; ++i) {
+    da.row_lane[i] = rm->lane[i];
+    da.row_cum[i] = rm->cum[i];
+    da.row_off[i] = rm->off[i];
+  }
+  da.qkv_part = m->part;
+  da.qkv_S = 1;
+  da.rope_cs = m->rope;
+  da.chunks = m->decode_chunks;
+  if (!split_attn) {
+    da.mode = 0;
+    TL_TRY(launch_attn_decode_fused(da, s));
+  } else {
+    // several tokens of one lane: every entry is appended before any row attends
+    da.mode = 1;
+    TL_TRY(launch_attn_decode_fused(da, s));
+    da.mode = 2;
+    TL_TRY(launch_attn_decode_fused(da, s));
+  }
+  // O projection, added into the residual stream
+  p.w0 = bd.w_o;
+  p.s0 = (const __half*)bd.s_o;
+  p.N = d;
+  p.K = d;
+  p.h = nullptr;
+  p.gamma = nullptr;
+  p.x = m->attn;
+  p.epi = DEC_EPI_RESID;
+  p.out = nullptr;
+  p.hres = m->h;
+  TL_TRY(launch_dec_gemv(p, s));
+  // gate | up with the pre-norm, SwiGLU in the epilogue
+  p.w0 = bd.w_gate;
+  p.s0 = (const __half*)bd.s_gate;
+  p.w1 = bd.w_up;
+  p.s1 = (const __half*)bd.s_up;
+  p.N = F;
+  p.K = d;
+  p.x = nullptr;
+  p.h = m->h;
+  p.gamma = bd.gamma_ffn;
+  p.epi = DEC_EPI_SWIGLU;
+  p.hres = nullptr;
+  p.u = m->u;
+  TL_TRY(launch_dec_gemv(p, s));
+  // down projection, added into the residual stream (and the trace)
+  p.w0 = bd.w_down;
+  p.s0 = (const __half*)bd.s_down;
+  p.w1 = nullptr;
+  p.s1 = nullptr;
+  p.N = d;
+  p.K = F;
+  p.h = nullptr;
+  p.gamma = nullptr;
+  p.x = m->u;
+  p.epi = DEC_EPI_RESID;
+  p.u = nullptr;
+  p.hres = m->h;
+  p.trace = trace;
+  p.out_row = lane_of_row;
+  p.trace_rows = trace_rows;
+  TL_TRY(launch_dec_gemv(p, s));
   return ok();
 }
 
@@ -780,11 +829,11 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
   TL_TRY(launch_residual_norm(n, s));
   for (int layer = 0; layer < n_layers; ++layer) {
     const tl_block* b = block_at(m, layer);
-    TL_TRY(enqueue_block_body(m, b, layer, seq, kv, lane, false, nullptr, nullptr, s));
+    TL_TRY(enqueue_block_body(m, b, layer, seq, kv, lane, s));
     NormArgs en = norm_args(m, seq);
     en.part = m->part;
     en.part_rows = seq;
-    en.S = gemm_splits(m->d, m->F, seq);
+    en.S = gemm_splits(m->d, m->F, seq, b->d.bits);
     en.n_add = seq;
     if (layer + 1 < n_layers) {
       en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
@@ -827,32 +876,58 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
   e.h = m->h;
   e.status = m->status;
   TL_TRY(launch_embed(e, s));
-  NormArgs n = norm_args(m, B);
-  n.gamma_next = block_at(m, 0)->d.gamma_attn;
-  n.n_next = B;
-  n.out_row = lane_of_row;
-  TL_TRY(launch_residual_norm(n, s));
   for (int layer = 0; layer < n_layers; ++layer) {
     const int act = active(layer);
-    const tl_block* b = block_at(m, layer);
-    TL_TRY(enqueue_block_body(m, b, layer, act, kv, -1, true, lane_of_row, rm, s));
-    const int nxt = layer + 1 < n_layers ? active(layer + 1) : 0;
-    NormArgs en = norm_args(m, trace ? B : act);
-    // the down projection's split-K partial sums are added into h here
-    en.part = m->part;
-    en.part_rows = act;
-    en.S = gemm_splits(m->d, m->F, act);
-    en.n_add = act;
-    en.n_next = nxt;
-    if (nxt > 0) en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
-    en.gamma_final = m->desc.gamma_final;
-    en.fin_lo = nxt;
-    en.fin_hi = act;
-    en.out_row = lane_of_row;
-    if (trace) en.trace = trace + (size_t)layer * B * m->d;
-    TL_TRY(launch_residual_norm(en, s));
+    TL_TRY(enqueue_decode_layer(m, block_at(m, layer), layer, act, kv, rm, lane_of_row,
+                                trace ? trace + (size_t)layer * B * m->d : nullptr, B, false, s));
   }
+  // final RMSNorm of every row (a row's residual stream stops changing after
+  // its last iteration)
+  NormArgs fin = norm_args(m, B);
+  fin.gamma_final = m->desc.gamma_final;
+  fin.fin_lo = 0;
+  fin.fin_hi = B;
+  fin.out_row = lane_of_row;
+  TL_TRY(launch_residual_norm(fin, s));
   TL_TRY(launch_advance_pos((KvHeader*)kv->buffer, B, s));
+  return ok();
+}
+
+// n consecutive tokens of one lane at its current position: a decode step
+// whose rows are those tokens (row r at position pos + r), the attention split
+// into an append pass and an attend pass.  Each row's arithmetic is that of a
+// one-token decode step at its position.
+tl_status enqueue_extend(tl_model* m, tl_kv* kv, int lane, bool use_ids, int n, int L,
+                         float* trace, cudaStream_t s) {
+  RowMap rm;
+  int cum = 0;
+  for (int b = 0; b < lane; ++b) cum += (int)m->pre.size() + kv->L[b];
+  for (int i = 0; i < kMaxLanes; ++i) {
+    rm.lane[i] = lane;
+    rm.cum[i] = cum;
+    rm.off[i] = i;
+  }
+  EmbedArgs e;
+  memset(&e, 0, sizeof(e));
+  e.ids = use_ids ? m->ids : nullptr;
+  e.h_in = m->hin;
+  e.embed = (const __half*)m->desc.embed;
+  e.vocab = m->desc.vocab;
+  e.d = m->d;
+  e.rows = n;
+  e.h = m->h;
+  e.status = m->status;
+  TL_TRY(launch_embed(e, s));
+  const int n_layers = (int)m->pre.size() + L;
+  for (int layer = 0; layer < n_layers; ++layer)
+    TL_TRY(enqueue_decode_layer(m, block_at(m, layer), layer, n, kv, &rm, m->ident_map,
+                                trace ? trace + (size_t)layer * n * m->d : nullptr, n, true, s));
+  NormArgs fin = norm_args(m, n);
+  fin.gamma_final = m->desc.gamma_final;
+  fin.fin_lo = 0;
+  fin.fin_hi = n;
+  TL_TRY(launch_residual_norm(fin, s));
+  TL_TRY(launch_add_pos((KvHeader*)kv->buffer, lane, n, s));
   return ok();
 }
 
@@ -959,6 +1034,7 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
   // cum_layers), passed to the attention kernel by value
   RowMap rm;
   for (int i = 0; i < kMaxLanes; ++i) {
+    rm.off[i] = 0;
     rm.lane[i] = order[i];
     int cum = 0;
     for (int b = 0; b < order[i] && b < kv->n_lanes; ++b) cum += (int)model->pre.size() + kv->L[b];
@@ -990,6 +1066,108 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
   return ok();
 }
 
+namespace {
+
+tl_status check_extend(tl_model* model, tl_kv* kv, int lane, int n, int L) {
+  TL_CHECK_ARG(model && kv, "NULL model or kv");
+  TL_CHECK_ARG(kv->model == model, "kv was created for another model");
+  TL_CHECK_ARG(lane >= 0 && lane < kv->n_lanes, "lane = %d out of [0, %d)", lane, kv->n_lanes);
+  TL_CHECK_ARG(n >= 1 && n <= kMaxLanes && n <= model->Tmax, "n = %d out of [1, %d]", n,
+               std::min(kMaxLanes, model->Tmax));
+  TL_CHECK_ARG(L >= 1 && L <= kv->L[lane], "L = %d out of [1, %d] for lane %d", L, kv->L[lane], lane);
+  TL_CHECK_ARG(kv->pos[lane] + n <= kv->max_ctx, "lane %d: %d + %d positions exceed %d", lane,
+               kv->pos[lane], n, kv->max_ctx);
+  return ok();
+}
+
+// enqueue an extend of n tokens whose inputs already sit in the model's ids
+// (use_ids) or hin buffer; output in model->y [n][d]
+tl_status run_extend(tl_model* model, tl_kv* kv, int lane, bool use_ids, int n, int L,
+                     float* h_trace, cudaStream_t s) {
+  char key[256];
+  snprintf(key, sizeof(key), "E|%llu|%d|%d|%d|%d|%p", (unsigned long long)kv->id, lane, n, L,
+           use_ids ? 1 : 0, (void*)h_trace);
+  TL_TRY(run_graph(model, key, kv->id, s, [&](cudaStream_t cs, int32_t*) {
+    return enqueue_extend(model, kv, lane, use_ids, n, L, h_trace, cs);
+  }));
+  kv->pos[lane] += n;
+  return ok();
+}
+
+tl_status set_lane_pos(tl_kv* kv, int lane, int pos, cudaStream_t s) {
+  TL_TRY(launch_set_pos((KvHeader*)kv->buffer, lane, pos, s));
+  kv->pos[lane] = pos;
+  return ok();
+}
+
+}  // namespace
+
+TL_API tl_status tl_extend(tl_model* model, tl_kv* kv, int lane, const int32_t* ids,
+                           const uint16_t* h_in, int n, int L, float* y_out, float* h_trace,
+                           tl_stream stream) {
+  TL_TRY(check_extend(model, kv, lane, n, L));
+  TL_CHECK_ARG((ids == nullptr) != (h_in == nullptr), "give exactly one of ids and h_in");
+  TL_CHECK_ARG(ids == nullptr || model->desc.embed != nullptr, "ids given but no embedding");
+  TL_CHECK_ARG(y_out != nullptr, "y_out is NULL");
+  cudaStream_t s = (cudaStream_t)stream;
+  const int d = model->d;
+  if (ids) TL_CUDA(cudaMemcpyAsync(model->ids, ids, (size_t)n * 4, cudaMemcpyDefault, s));
+  else TL_CUDA(cudaMemcpyAsync(model->hin, h_in, (size_t)n * d * 2, cudaMemcpyDefault, s));
+  TL_TRY(run_extend(model, kv, lane, ids != nullptr, n, L, h_trace, s));
+  TL_CUDA(cudaMemcpyAsync(y_out, model->y, (size_t)n * d * 4, cudaMemcpyDefault, s));
+  return ok();
+}
+
+TL_API tl_status tl_greedy_head(tl_model* model, const float* y, int n, int32_t* ids,
+                                tl_stream stream) {
+  TL_CHECK_ARG(model && y && ids, "NULL argument");
+  TL_CHECK_ARG(model->desc.embed != nullptr, "the model has no embedding to use as its head");
+  TL_CHECK_ARG(n >= 1 && n <= 8, "n = %d out of [1, 8]", n);
+  return launch_greedy_head(y, n, (const __half*)model->desc.embed, model->desc.vocab, model->d,
+                            model->head_ps, model->head_pv, ids, (cudaStream_t)stream);
+}
+
+TL_API tl_status tl_spec_step(tl_model* model, tl_kv* kv, int lane, int32_t token, int K,
+                              int L_draft, int L_verify, int32_t* tokens_out, int* n_out,
+                              tl_stream stream) {
+  TL_CHECK_ARG(tokens_out && n_out, "NULL output");
+  TL_CHECK_ARG(K >= 1 && K <= kMaxLanes - 1, "K = %d out of [1, %d]", K, kMaxLanes - 1);
+  TL_TRY(check_extend(model, kv, lane, K + 1, L_verify));
+  TL_CHECK_ARG(L_draft >= 1 && L_draft <= kv->L[lane], "L_draft = %d out of [1, %d]", L_draft,
+               kv->L[lane]);
+  TL_CHECK_ARG(model->desc.embed != nullptr, "the model has no embedding to use as its head");
+  TL_CHECK_ARG(token >= 0 && token < model->desc.vocab, "token %d out of the vocabulary", token);
+  cudaStream_t s = (cudaStream_t)stream;
+  const int p = kv->pos[lane];
+  const __half* E = (const __half*)model->desc.embed;
+  // draft: K one-token steps at L_draft, each input the previous greedy token
+  TL_TRY(launch_set_i32(model->spec_ids, token, s));
+  for (int i = 0; i < K; ++i) {
+    TL_CUDA(cudaMemcpyAsync(model->ids, model->spec_ids + i, 4, cudaMemcpyDeviceToDevice, s));
+    TL_TRY(run_extend(model, kv, lane, true, 1, L_draft, nullptr, s));
+    TL_TRY(launch_greedy_head(model->y, 1, E, model->desc.vocab, model->d, model->head_ps,
+                              model->head_pv, model->spec_ids + i + 1, s));
+  }
+  // verify: back to p, the input token and the K drafts at L_verify
+  TL_TRY(set_lane_pos(kv, lane, p, s));
+  TL_CUDA(cudaMemcpyAsync(model->ids, model->spec_ids, (size_t)(K + 1) * 4,
+                          cudaMemcpyDeviceToDevice, s));
+  TL_TRY(run_extend(model, kv, lane, true, K + 1, L_verify, nullptr, s));
+  TL_TRY(launch_greedy_head(model->y, K + 1, E, model->desc.vocab, model->d, model->head_ps,
+                            model->head_pv, model->spec_ver, s));
+  int32_t drafts[kMaxLanes + 1], ver[kMaxLanes + 1];
+  TL_CUDA(cudaMemcpyAsync(drafts, model->spec_ids, (size_t)(K + 1) * 4, cudaMemcpyDeviceToHost, s));
+  TL_CUDA(cudaMemcpyAsync(ver, model->spec_ver, (size_t)(K + 1) * 4, cudaMemcpyDeviceToHost, s));
+  TL_CUDA(cudaStreamSynchronize(s));
+  // accept the longest matching prefix, then the verify token after it
+  int m = 0;
+  while (m < K && drafts[m + 1] == ver[m]) ++m;
+  for (int i = 0; i < m; ++i) tokens_out[i] = drafts[i + 1];
+  tokens_out[m] = ver[m];
+  *n_out = m + 1;
+  return set_lane_pos(kv, lane, p + m + 1, s);
+}
+
 // ============================================================================
 // Linear-layer hook
 // ============================================================================
@@ -1006,10 +1184,53 @@ tl_status check_linear(int N, int K, int group, int T) {
 }
 }  // namespace tl
 
+namespace tl {
+// Split count of the linear-layer hook: decode-sized calls run the decode
+// projection kernel (no split-K), the rest launch_gemm's kernels.
+int linear_splits(int N, int K, int T) {
+  return dec_gemv_eligible(N, K, T, 4) ? 1 : gemm_splits(N, K, T);
+}
+
+tl_status launch_linear(const uint32_t* packed, const uint16_t* scales, int N, int K, int group,
+                        const uint16_t* x, int T, float* y, float* scratch, cudaStream_t s) {
+  if (dec_gemv_eligible(N, K, T, 4)) {
+    DecGemvArgs p;
+    memset(&p, 0, sizeof(p));
+    p.w0 = packed;
+    p.s0 = (const __half*)scales;
+    p.N = N;
+    p.K = K;
+    p.G = group;
+    p.bits = 4;
+    p.T = T;
+    p.x = (const __half*)x;
+    p.epi = DEC_EPI_OUT;
+    p.out = y;
+    return launch_dec_gemv(p, s);
+  }
+  const int S = gemm_splits(N, K, T);
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.bits = 4;
+  a.w0 = a.w1 = packed;
+  a.s0 = a.s1 = (const __half*)scales;
+  a.n_split = a.N = N;
+  a.K = K;
+  a.G = group;
+  a.x = (const __half*)x;
+  a.T = T;
+  a.splits = S;
+  a.part = S > 1 ? scratch : y;
+  TL_TRY(launch_gemm(a, s));
+  if (S > 1) TL_TRY(launch_split_sum(scratch, S, (long)T * N, y, s));
+  return ok();
+}
+}  // namespace tl
+
 TL_API tl_status tl_linear_workspace_bytes(int N, int K, int T, size_t* bytes) {
   TL_CHECK_ARG(bytes, "bytes is NULL");
   TL_TRY(check_linear(N, K, 64, T));
-  const int S = gemm_splits(N, K, T);
+  const int S = linear_splits(N, K, T);
   *bytes = S > 1 ? (size_t)S * T * N * 4 : 0;
   return ok();
 }
@@ -1020,24 +1241,11 @@ TL_API tl_status tl_linear(const uint32_t* packed, const uint16_t* scales, int N
   TL_TRY(check_linear(N, K, group, T));
   TL_CHECK_ARG(packed && scales && x && y, "NULL device pointer");
   TL_TRY(gemm_tc_init());
-  const int S = gemm_splits(N, K, T);
+  const int S = linear_splits(N, K, T);
   TL_CHECK_ARG(S == 1 || workspace, "workspace is NULL but %zu bytes are needed",
                (size_t)S * T * N * 4);
-  GemmArgs a;
-  memset(&a, 0, sizeof(a));
-  a.w0 = a.w1 = packed;
-  a.s0 = a.s1 = (const __half*)scales;
-  a.n_split = a.N = N;
-  a.K = K;
-  a.G = group;
-  a.x = (const __half*)x;
-  a.T = T;
-  a.splits = S;
-  a.part = S > 1 ? (float*)workspace : y;
-  cudaStream_t s = (cudaStream_t)stream;
-  TL_TRY(launch_gemm(a, s));
-  if (S > 1) TL_TRY(launch_split_sum((const float*)workspace, S, (long)T * N, y, s));
-  return ok();
+  return launch_linear(packed, scales, N, K, group, x, T, y, (float*)workspace,
+                       (cudaStream_t)stream);
 }
 
 TL_API tl_status tl_check_bounded_wait(tl_model* model, unsigned limit_us, tl_stream stream) {

@@ -378,13 +378,20 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   // the lane's context, i.e. the contiguous keys [kA, kB).  Each chunk is
   // streamed in 64-key stages from its own start and folded into its own
   // (P V, max, sum), exactly as if one CTA took each chunk.
+  // Launch modes: 0 = append the row's new entry and attend (one decode
+  // token per lane); 1 = append only; 2 = attend only, every key (the new one
+  // included) read from the cache.  Modes 1 then 2 serve several consecutive
+  // tokens of one lane (row_off = 0, 1, ...): every token's entry is in the
+  // cache before any token attends, and each row's arithmetic is that of a
+  // mode-0 decode step at its position.
   const int lane_id = a.row_lane[row];
-  const int pos = a.hdr->pos[lane_id];
+  const int pos = a.hdr->pos[lane_id] + a.row_off[row];
   const int n_keys = pos + 1;
   const int per = (n_keys + CL - 1) / CL;
   const int kA = min(crank * F * per, n_keys), kB = min(kA + F * per, n_keys);
   const int nkc = kB - kA;
-  const bool owner = nkc > 0 && kB == n_keys;
+  const bool owner = a.mode != 2 && nkc > 0 && kB == n_keys;
+  if (a.mode == 1 && !owner) return;   // nothing to append here, nothing copied yet
   const int n_old = owner ? nkc - 1 : nkc;       // keys of [kA, kB) already cached
   const int NSF = (per + DS_KEYS - 1) / DS_KEYS; // stages of a full chunk
   const int nstage = nkc / per * NSF + (nkc % per + DS_KEYS - 1) / DS_KEYS;
@@ -439,9 +446,18 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
+  // the first stages are copied before the wait for the previous kernel: they
+  // hold entries of earlier steps only -- except in mode 2, where the
+  // previous kernel appended some of them, and mode 1, which copies nothing
+  if (a.mode == 0) {
 #pragma unroll
-  for (int st = 0; st < T::NST - 1; ++st) issue(st);
+    for (int st = 0; st < T::NST - 1; ++st) issue(st);
+  }
   pdl_enter();
+  if (a.mode == 2) {
+#pragma unroll
+    for (int st = 0; st < T::NST - 1; ++st) issue(st);
+  }
 
   // the cached keys' scales, the RoPE pair and the QKV partial sums are all
   // requested before any of them is used (one round trip)
@@ -565,6 +581,7 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
       }
     }
   }
+  if (a.mode == 1) return;   // append only: the entry is in the cache
   __syncthreads();   // qh final
 
   // q as the B operand of S^T (column 0: lanes g == 0).  k step ks covers

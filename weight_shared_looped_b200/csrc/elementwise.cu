@@ -337,6 +337,16 @@ __global__ void set_pos_kernel(KvHeader* hdr, int lane, int value) {
   }
 }
 
+__global__ void add_pos_kernel(KvHeader* hdr, int lane, int n) {
+  pdl_enter();
+  hdr->pos[lane] += n;
+}
+
+__global__ void set_i32_kernel(int32_t* p, int value) {
+  pdl_enter();
+  *p = value;
+}
+
 __global__ void advance_pos_kernel(KvHeader* hdr, int n_lanes) {
   pdl_enter();
   int i = threadIdx.x;
@@ -384,6 +394,16 @@ tl_status launch_swiglu(const float* part, int S, int rows, int F, __half* u, cu
 
 tl_status launch_set_pos(KvHeader* hdr, int lane, int value, cudaStream_t s) {
   TL_LAUNCH_PDL(set_pos_kernel, 1, 1, 0, s, hdr, lane, value);
+  return ok();
+}
+
+tl_status launch_add_pos(KvHeader* hdr, int lane, int n, cudaStream_t s) {
+  TL_LAUNCH_PDL(add_pos_kernel, 1, 1, 0, s, hdr, lane, n);
+  return ok();
+}
+
+tl_status launch_set_i32(int32_t* p, int value, cudaStream_t s) {
+  TL_LAUNCH_PDL(set_i32_kernel, 1, 1, 0, s, p, value);
   return ok();
 }
 

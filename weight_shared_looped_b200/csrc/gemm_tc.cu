@@ -1,7 +1,8 @@
 // Quantised-weight GEMM on the 5th-generation tensor cores (tcgen05), for
 // prefill-sized token counts:
 //   part[z][t][n] = sum over k in split z of x[t][k] * W[n][k],
-//   W[n][k] = code[n][k] * scale[n][k / G]  (group-wise symmetric INT4).
+//   W[n][k] = code[n][k] * scale[n][k / G]  (group-wise symmetric INT4, or INT3
+//   read straight from its canonical 10-codes-per-word rows).
 //
 // One CTA per SM computes 128 weight rows x BN tokens over a range of 64-wide
 // k blocks.  Warp roles:
@@ -168,6 +169,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
 
 struct TcArgs {
   int N, K, G, T, n_split;   // n_split % 128 == 0
+  int wpr;                   // packed words per row (K / 8 for INT4, the padded INT3 row)
   int splits;                // split z covers k blocks [z*nkb/S, (z+1)*nkb/S)
   const uint32_t* w0;        // canonical INT4 words of rows [0, n_split)
   const uint32_t* w1;        // rows [n_split, N)
@@ -186,11 +188,33 @@ __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
       : "memory");
 }
 
+// INT3 k block: the 64 codes k0 .. k0 + 63 of one row, k0 = 64m, start at code
+// O = k0 mod 10 (0, 4, 8, 2 or 6) of word v[0] of the row's words v[0..7].  O
+// is even, so codes 2c and 2c + 1 always share a word: a shift and a mask
+// leave the pair at bits 0-5, one multiply by 1 + 2^13 copies it to bits
+// 13-18, and a lop3 keeps code 2c at bits 0-2 and code 2c + 1 at bits 16-18
+// under the fp16 exponent of 1024; 1024 + u less 1028 is the exact code, then
+// the fp16 product with the scale (as for INT4).
+template <int O>
+__device__ __forceinline__ void int3_kblock(const uint32_t* v, __half2 s2, uint32_t* out) {
+  const __half2 bias = __halves2half2(__float2half_rn(1028.0f), __float2half_rn(1028.0f));
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const int p = O + 2 * c, q = p / 10, i = p % 10;   // compile-time: i even, i <= 8
+    const uint32_t y = ((v[q] >> (3 * i)) & 0x3Fu) * 8193u;
+    uint32_t h;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(y), "r"(0x00070007u), "r"(0x64006400u));
+    __half2 cv = __hsub2(*reinterpret_cast<__half2*>(&h), bias);
+    __half2 wv = __hmul2(cv, s2);
+    out[c] = *reinterpret_cast<uint32_t*>(&wv);
+  }
+}
+
 // 96 registers x 608 threads (58 K of the 64 K register file) still leave
 // room for a small CTA of the next or previous kernel on the same SM; at 80
 // the compiler schedules the weight loads less freely (gate|up 4% slower),
 // and more registers or a third register set of weights gain nothing.
-template <int BN>
+template <int BN, int BITS>
 __global__ void __maxnreg__(96)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x, TcArgs a) {
   constexpr int XS = TcCfg<BN>::X_STAGES;
@@ -333,7 +357,7 @@ __global__ void __maxnreg__(96)
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     // this thread's weight row (canonical INT4 words) and scale row
     const int gsh = __ffs(a.G) - 1;             // the group size is 64 or 128
-    const size_t wpr = (size_t)a.K / 8, gpr = (size_t)a.K >> gsh;
+    const size_t wpr = (size_t)a.wpr, gpr = (size_t)a.K >> gsh;
     const uint32_t* wrow;
     const __half* srow;
     if (sw) {
@@ -345,49 +369,85 @@ __global__ void __maxnreg__(96)
       wrow = (second ? a.w1 : a.w0) + (size_t)(wrow0 + r) * wpr;
       srow = (second ? a.s1 : a.s0) + (size_t)(wrow0 + r) * gpr;
     }
-    // The packed words (32 bytes per row and k block) and the scale come
+    // The packed words of this row's k block (INT4: 32 bytes; INT3: the three
+    // aligned 16-byte vectors holding its 7 or 8 words) and its scale come
     // straight from global memory through the read-only path, two of this
     // group's k blocks ahead in registers (sets 0 and 1 alternate).  Weights
     // are constants of the model: the first loads go out before the wait for
     // the previous kernel.
-    uint4 wa0 = make_uint4(0u, 0u, 0u, 0u), wb0 = wa0, wa1 = wa0, wb1 = wa0;
-    __half sc0 = __float2half_rn(0.f), sc1 = sc0;
-    auto fetch = [&](int i, uint4& wa, uint4& wb, __half& sc) {
+    struct WSet {
+      uint4 a, b, c;
+      __half sc;
+    };
+    WSet set0, set1;
+    set0.a = set0.b = set0.c = make_uint4(0u, 0u, 0u, 0u);
+    set0.sc = __float2half_rn(0.f);
+    set1 = set0;
+    auto fetch = [&](int i, WSet& w) {
       if (i < nkb) {
-        const uint4* p = reinterpret_cast<const uint4*>(wrow + (size_t)(kb_begin + i) * (BK / 8));
-        wa = __ldg(p);
-        wb = __ldg(p + 1);
-        sc = __ldg(srow + (((kb_begin + i) * BK) >> gsh));
+        const int k0 = (kb_begin + i) * BK;
+        if (BITS == 4) {
+          const uint4* p = reinterpret_cast<const uint4*>(wrow + (size_t)k0 / 8);
+          w.a = __ldg(p);
+          w.b = __ldg(p + 1);
+        } else {
+          const int base = (k0 / 10) & ~3;
+          const uint4* p = reinterpret_cast<const uint4*>(wrow + base);
+          w.a = __ldg(p);
+          w.b = __ldg(p + 1);
+          w.c = base + 8 < (int)wpr ? __ldg(p + 2) : make_uint4(0u, 0u, 0u, 0u);
+        }
+        w.sc = __ldg(srow + (k0 >> gsh));
       }
     };
-    fetch(grp, wa0, wb0, sc0);
-    fetch(grp + BATCH, wa1, wb1, sc1);
+    fetch(grp, set0);
+    fetch(grp + BATCH, set1);
     const __half2 mul = __halves2half2(__float2half_rn(1.0f), __float2half_rn(0.0625f));
     const __half2 add = __halves2half2(__float2half_rn(-1032.0f), __float2half_rn(-72.0f));
     // one k block of batch b: wait for the A slot, dequantise, store to TMEM,
     // refill the register set with this group's k block two batches on
-    auto kblock = [&](int b, uint4& wa, uint4& wb, __half& sc) -> bool {
+    auto kblock = [&](int b, WSet& ws) -> bool {
       const int i = b * BATCH + grp;
       // the TMEM slot of this batch is free once batch b - AB is done
       // (a failure elsewhere surfaces here as a timed-out wait)
       if (b >= AB && !mbar_wait(&done[(b - AB) % AB], ((b - AB) / AB) & 1)) return false;
       if (i < nkb) {
-        const uint32_t words[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-        const __half2 s2 = __halves2half2(sc, sc);
+        const __half2 s2 = __halves2half2(ws.sc, ws.sc);
         uint32_t v[32];
+        if (BITS == 4) {
+          const uint32_t words[8] = {ws.a.x, ws.a.y, ws.a.z, ws.a.w, ws.b.x, ws.b.y, ws.b.z, ws.b.w};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          // byte c/2... of word c/4: codes of k = 2c (low nibble), 2c + 1 (high)
-          const uint32_t bb = c & 3;
-          uint32_t x, h;
-          asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(words[c >> 2]), "r"(0u),
-              "r"(bb | 0x40u | (bb << 8) | 0x4000u));
-          asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
-          __half2 cv = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);   // exact codes
-          __half2 wv = __hmul2(cv, s2);                                      // fp16(code * s)
-          v[c] = *reinterpret_cast<uint32_t*>(&wv);
+          for (int c = 0; c < 32; ++c) {
+            // byte c/2... of word c/4: codes of k = 2c (low nibble), 2c + 1 (high)
+            const uint32_t bb = c & 3;
+            uint32_t x, h;
+            asm("prmt.b32 %0, %1, %2, %3;" : "=r"(x) : "r"(words[c >> 2]), "r"(0u),
+                "r"(bb | 0x40u | (bb << 8) | 0x4000u));
+            asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
+            __half2 cv = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);   // exact codes
+            __half2 wv = __hmul2(cv, s2);                                      // fp16(code * s)
+            v[c] = *reinterpret_cast<uint32_t*>(&wv);
+          }
+        } else {
+          // the 8 words from the first code's word on (d = its offset in the
+          // aligned vectors), then the k block's alignment case
+          const int k0 = (kb_begin + i) * BK;
+          const int d = (k0 / 10) & 3;
+          const uint32_t u[12] = {ws.a.x, ws.a.y, ws.a.z, ws.a.w, ws.b.x, ws.b.y,
+                                  ws.b.z, ws.b.w, ws.c.x, ws.c.y, ws.c.z, ws.c.w};
+          uint32_t w8[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            w8[j] = d == 0 ? u[j] : d == 1 ? u[j + 1] : d == 2 ? u[j + 2] : u[j + 3];
+          switch (k0 % 10) {
+            case 0: int3_kblock<0>(w8, s2, v); break;
+            case 2: int3_kblock<2>(w8, s2, v); break;
+            case 4: int3_kblock<4>(w8, s2, v); break;
+            case 6: int3_kblock<6>(w8, s2, v); break;
+            default: int3_kblock<8>(w8, s2, v); break;
+          }
         }
-        fetch(i + 2 * BATCH, wa, wb, sc);
+        fetch(i + 2 * BATCH, ws);
         if (b >= AB) asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
         const uint32_t taddr = tmem_base + lane_addr + a_col0 + ((b % AB) * BATCH + grp) * A_COLS;
         asm volatile(
@@ -410,7 +470,7 @@ __global__ void __maxnreg__(96)
     // the dequantisation reads only weights and writes only TMEM: it may run
     // ahead of the previous kernel; the epilogue's stores wait for it
     for (int b = 0; b < nbatch; b += 2) {
-      if (!kblock(b, wa0, wb0, sc0) || (b + 1 < nbatch && !kblock(b + 1, wa1, wb1, sc1))) {
+      if (!kblock(b, set0) || (b + 1 < nbatch && !kblock(b + 1, set1))) {
         atomicExch(abort_flag, 1);
         break;
       }
@@ -578,7 +638,7 @@ size_t tc_smem_bytes() {
   return b < kMinSmem ? kMinSmem : b;
 }
 
-template <int BN>
+template <int BN, int BITS>
 tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   CUtensorMap mx;
   TL_TRY(encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.x, g.K, g.T, (uint64_t)g.K * 2, BK, BN,
@@ -588,6 +648,7 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.K = g.K;
   a.G = g.G;
   a.T = g.T;
+  a.wpr = BITS == 4 ? g.K / 8 : ((g.K + 9) / 10 + 3) / 4 * 4;
   a.n_split = g.n_split;
   a.splits = g.splits;
   a.w0 = g.w0;
@@ -601,7 +662,7 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   if (smem > 232448)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs %zu bytes of shared memory", smem);
   dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
-  TL_LAUNCH_PDL(gemm_w4_tc_kernel<BN>, grid, THREADS, smem, s, mx, a);
+  TL_LAUNCH_PDL((gemm_w4_tc_kernel<BN, BITS>), grid, THREADS, smem, s, mx, a);
   return ok();
 }
 
@@ -619,9 +680,13 @@ tl_status gemm_tc_init() {
   static std::atomic<uint64_t> done{0};
   return once_per_device(done, []() -> tl_status {
     TL_TRY(get_encoder());
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 4>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 3>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 3>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
     return ok();
   });
@@ -637,14 +702,20 @@ int gemm_tc_splits(int N, int K, int T) {
   return s < 1 ? 1 : s;
 }
 
-bool gemm_tc_eligible(int N, int K, int T) { return T >= 64 && N % BM == 0 && K % BK == 0; }
+// INT4 below 64 tokens runs the mma.sync kernel; INT3 runs here at every
+// token count (rows past T are read as zero).
+bool gemm_tc_eligible(int N, int K, int T, int bits) {
+  return (T >= 64 || bits == 3) && T >= 1 && N % BM == 0 && K % BK == 0;
+}
 
 tl_status launch_gemm_tc(const GemmArgs& g, cudaStream_t s) {
   if (g.T == 0) return ok();
   if (g.n_split % BM != 0)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs row split %% 128 == 0");
-  if (tc_tile_n(g.T) == 128) return launch_tc_bn<128>(g, s);
-  return launch_tc_bn<64>(g, s);
+  if (g.bits == 3)
+    return tc_tile_n(g.T) == 128 ? launch_tc_bn<128, 3>(g, s) : launch_tc_bn<64, 3>(g, s);
+  if (tc_tile_n(g.T) == 128) return launch_tc_bn<128, 4>(g, s);
+  return launch_tc_bn<64, 4>(g, s);
 }
 
 }  // namespace tl

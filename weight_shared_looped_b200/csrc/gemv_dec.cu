@@ -1,0 +1,540 @@
+// Decode-sized quantised-weight projections (T <= 8 tokens), one launch per
+// projection, with the neighbouring row-wise work folded in:
+//   y[t][n] = sum over k of x[t][k] * W[n][k],   W[n][k] = code[n][k] * scale[n][k / G]
+// for canonical INT4 (8 codes per word) or INT3 (10 codes per word) weights.
+//
+// A CTA owns MT tiles of 16 weight rows over the whole of K; its eight warps
+// split K (MT = 1: eight k ranges; MT = 2: four per tile), so no split-K
+// partial sums leave the CTA: the warps' results are added in shared memory in
+// warp order, a fixed order that depends only on (N, K, MT).  Every token
+// column is computed independently of the others, so a token's result does
+// not depend on which other tokens share the launch.
+//
+// Weights are the A operand of mma.sync m16n8k16 (16 rows x 16 k), tokens the
+// B operand (8 columns).  Lane (g, t) of a warp reads one 16-byte vector of
+// packed words of row g and one of row g + 8 per chunk:
+//   INT4: chunk = 128 k; the lane's vector holds k = 32t .. 32t + 31 of the
+//         chunk; each word yields its code pairs (0,4) (1,5) (2,6) (3,7) with
+//         one lop3 (and one shift per word) and one HFMA2, as exact fp16
+//         integers; with G = 128 a chunk is one scale group, whose fp32 sum is
+//         scaled once per chunk; with G = 64 lanes t = 0, 1 hold the chunk's
+//         first group and t = 2, 3 its second, so each k step runs twice, once
+//         per group with the other lanes' A registers zero, into two fp32 sums;
+//   INT3: chunk = 16 words = 160 codes (the canonical rows are padded to
+//         whole 16-byte vectors); the lane's vector holds codes 40t .. 40t + 39
+//         of the chunk; code pairs (i, i + 6) of a word come out of one shift
+//         and one lop3, codes 4 and 5 pair across two words through one prmt;
+//         a lane's 40 codes may straddle a scale group, so the pair is scaled
+//         in fp16 before the MMA (fp16(code * scale), as the tensor-core
+//         prefill GEMM does).
+// The k order inside an MMA is free as long as A and B agree, so the
+// activations are staged in shared memory in the order the lanes' codes come
+// out, and ldmatrix feeds them to the B operand.
+//
+// Folded work (template EPI / NORM):
+//   NORM   the CTA forms its activations itself: x = fp16(rmsnorm(h) * gamma)
+//          from the fp32 residual stream (the pre-norm before the QKV and the
+//          gate/up projections), so no separate norm kernel runs at decode;
+//   EPI_OUT   y -> out (fp32 [T][N]);
+//   EPI_RESID y is added into the fp32 residual stream h (the O and down
+//             projections; each element has exactly one writer), and the
+//             down projection writes the per-layer trace;
+//   EPI_SWIGLU tile 0 holds 16 gate rows and tile 1 the same 16 up rows:
+//             u = fp16(silu(gate) * up).
+// Weights, scales and gains are constants of the model: they are requested
+// before the wait for the previous kernel, so their latency overlaps its tail.
+#include "tl_launch.cuh"
+
+namespace tl {
+namespace {
+
+constexpr int DG_THREADS = 256;
+constexpr int DG_WARPS = 8;
+constexpr int DG_MAXC = 8;          // most chunks whose words one lane holds in flight
+
+enum { EPI_OUT = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
+
+template <int BITS>
+struct DgFmt {
+  static constexpr int CW = BITS == 4 ? 128 : 160;   // codes per chunk (one row)
+};
+
+__device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t* r, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t lop3_ea(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));   // (a & b) | c
+  return d;
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t x, __half2 m, __half2 a) {
+  __half2 r = __hfma2(*reinterpret_cast<__half2*>(&x), m, a);
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t hmul2_bits(uint32_t x, uint32_t s) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2*>(&x), *reinterpret_cast<__half2*>(&s));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+__device__ __forceinline__ uint32_t h2bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 h2c(float lo, float hi) {
+  return __halves2half2(__float2half_rn(lo), __float2half_rn(hi));
+}
+
+// ---- INT4: the four exact fp16 code pairs of one word (nibbles (0,4) (1,5) (2,6) (3,7))
+__device__ __forceinline__ void int4_pairs(uint32_t w, uint32_t* p) {
+  const __half2 one = h2c(1.f, 1.f), sixteenth = h2c(0.0625f, 0.0625f);
+  const __half2 lo_b = h2c(-1032.f, -1032.f), hi_b = h2c(-72.f, -72.f);
+  const uint32_t w8 = w >> 8;
+  p[0] = hfma2_bits(lop3_ea(w, 0x000F000Fu, 0x64006400u), one, lo_b);          // 1024 + u - 1032
+  p[1] = hfma2_bits(lop3_ea(w, 0x00F000F0u, 0x64006400u), sixteenth, hi_b);    // (1024 + 16u)/16 - 72
+  p[2] = hfma2_bits(lop3_ea(w8, 0x000F000Fu, 0x64006400u), one, lo_b);
+  p[3] = hfma2_bits(lop3_ea(w8, 0x00F000F0u, 0x64006400u), sixteenth, hi_b);
+}
+
+// ---- INT3: codes (i, i + 6) of one word: bits 3i and 3i + 18 after a shift
+// by 3i land at bits 0-2 (1024 + u) and 18-20 (1024 + 4u of the upper half)
+template <int I>
+__device__ __forceinline__ uint32_t int3_pair_i6(uint32_t w) {
+  const uint32_t x = lop3_ea(w >> (3 * I), 0x001C0007u, 0x64006400u);
+  return hfma2_bits(x, h2c(1.f, 0.25f), h2c(-1028.f, -260.f));
+}
+// code 4 of words a and b (bits 12-14: bits 4-6 of byte 1)
+__device__ __forceinline__ uint32_t int3_pair_c4(uint32_t a, uint32_t b) {
+  const uint32_t x = lop3_ea(prmt(a, b, 0x0501u), 0x00700070u, 0x64006400u);
+  return hfma2_bits(x, h2c(0.0625f, 0.0625f), h2c(-68.f, -68.f));
+}
+// code 5 of words a and b (bits 15-17: bit 7 of byte 1 and bits 0-1 of byte 2)
+__device__ __forceinline__ uint32_t int3_pair_c5(uint32_t a, uint32_t b) {
+  const uint32_t x = lop3_ea(prmt(a, b, 0x6521u), 0x03800380u, 0x64006400u);
+  return hfma2_bits(x, h2c(0.0078125f, 0.0078125f), h2c(-12.f, -12.f));
+}
+
+// Position, in a staged activation row, of element k of the original row.
+// INT4: k = 128c + 32t + 8q + e -> k step 2q + ((e >> 1) & 1), slot 2t + 8 (e odd) + (e >= 4).
+// INT3: k = 160c + 40t + L (L = 10q + i) -> see int3_slot.
+__device__ __forceinline__ int int3_slot(int L, int t, int& j) {
+  const int q = L / 10, i = L - 10 * q;
+  switch (i) {
+    case 0: j = 2 * q; return 2 * t;
+    case 6: j = 2 * q; return 2 * t + 1;
+    case 1: j = 2 * q; return 2 * t + 8;
+    case 7: j = 2 * q; return 2 * t + 9;
+    case 2: j = 2 * q + 1; return 2 * t;
+    case 8: j = 2 * q + 1; return 2 * t + 1;
+    case 3: j = 2 * q + 1; return 2 * t + 8;
+    case 9: j = 2 * q + 1; return 2 * t + 9;
+    case 4: j = 8 + (q >> 1); return 2 * t + (q & 1);
+    default: j = 8 + (q >> 1); return 2 * t + 8 + (q & 1);   // i == 5
+  }
+}
+
+template <int BITS>
+__device__ __forceinline__ int xpos(int k) {
+  if (BITS == 4) {
+    const int c = k >> 7, r = k & 127, t = r >> 5, q = (r >> 3) & 3, e = k & 7;
+    const int j = 2 * q + ((e >> 1) & 1);
+    const int s = 2 * t + ((e & 1) ? 8 : 0) + (e >= 4 ? 1 : 0);
+    return c * 128 + 16 * j + s;
+  } else {
+    const int c = k / 160, r = k - 160 * c, t = r / 40, L = r - 40 * t;
+    int j;
+    const int s = int3_slot(L, t, j);
+    return c * 160 + 16 * j + s;
+  }
+}
+
+struct DgArgs {
+  const uint32_t* w0;   // canonical packed rows: tile m of CTA b is rows (b*MT + m)*16 ..
+  const __half* s0;     //   (EPI_SWIGLU: w0 = gate, w1 = up, both rows b*16 ..)
+  const uint32_t* w1;
+  const __half* s1;
+  int N, K, G, wpr;     // output rows (per matrix), K, group, packed words per row
+  int T;                // active token rows (1..8)
+  const __half* x;      // fp16 [T][K] activations (when !NORM)
+  const float* h;       // fp32 [T][K] residual stream (NORM)
+  const float* gamma;   // fp32 [K] (NORM)
+  float eps;
+  float* out;           // EPI_OUT: fp32 [T][N]
+  float* hres;          // EPI_RESID: fp32 [rows][N], += y
+  __half* u;            // EPI_SWIGLU: fp16 [T][N]
+  float* trace;         // EPI_RESID, optional: fp32 [trace_rows][N] rows indexed by out_row
+  const int32_t* out_row;
+  int trace_rows;       // rows T .. trace_rows-1 are copied from hres unchanged
+};
+
+// MC: chunks a lane holds in flight (its k range takes ceil(chunks / (8 / MT))
+// of them; larger ranges run in batches of MC)
+template <int BITS, int MT, bool NORM, int EPI, int MC>
+__global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(DgArgs a) {
+  using Fm = DgFmt<BITS>;
+  constexpr int CW = Fm::CW;
+  constexpr int W = DG_WARPS / MT;                 // warps (k ranges) per tile
+  extern __shared__ __align__(16) unsigned char dg_smem[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int m = warp / W, ks = warp - m * W;
+  const int nvec = a.wpr >> 2;                     // 16-byte vectors per packed row
+  const int nch = (nvec + 3) >> 2;                 // chunks per row
+  const int c_lo = ks * nch / W, c_hi = (ks + 1) * nch / W;
+  const int xw = nch * CW + 8;                     // staged row, halves (stride/16 odd)
+  __half* xs = reinterpret_cast<__half*>(dg_smem);                         // [T][xw]
+  float* red = reinterpret_cast<float*>(dg_smem + (size_t)a.T * xw * 2);  // [MT][W][16][8]
+  __shared__ __align__(16) uint32_t zero16[4];
+  __shared__ float nred[8][DG_WARPS];
+  const int gsh = __ffs(a.G) - 1;
+  const int gpr = a.K >> gsh;
+  const bool g64 = BITS == 4 && a.G == 64;
+
+  // this tile's rows g and g + 8
+  int row0;
+  const uint32_t* wm;
+  const __half* sm;
+  if (EPI == EPI_SWIGLU) {
+    row0 = blockIdx.x * 16;
+    wm = m == 0 ? a.w0 : a.w1;
+    sm = m == 0 ? a.s0 : a.s1;
+  } else {
+    row0 = (blockIdx.x * MT + m) * 16;
+    wm = a.w0;
+    sm = a.s0;
+  }
+  const uint4* wr0 = reinterpret_cast<const uint4*>(wm + (size_t)(row0 + g) * a.wpr);
+  const uint4* wr1 = reinterpret_cast<const uint4*>(wm + (size_t)(row0 + g + 8) * a.wpr);
+  const __half* sr0 = sm + (size_t)(row0 + g) * gpr;
+  const __half* sr1 = sm + (size_t)(row0 + g + 8) * gpr;
+
+  // ---- constants first: this lane's packed words and scales of its first chunks
+  // sv[i]: rows g, g + 8 of the first scale group ([0], [1]) and of the second
+  // ([2], [3]): INT4 G = 128 one group per chunk; INT4 G = 64 the chunk's two
+  // groups; INT3 the group of the lane's first code and the next one
+  uint4 wv[MC][2];
+  __half sv[MC][4];
+  auto fetch = [&](int cb) {
+#pragma unroll
+    for (int i = 0; i < MC; ++i) {
+      const int c = cb + i;
+      const int vi = 4 * c + t;
+      const bool in = c < c_hi && vi < nvec;
+      wv[i][0] = in ? __ldg(wr0 + vi) : make_uint4(0u, 0u, 0u, 0u);
+      wv[i][1] = in ? __ldg(wr1 + vi) : make_uint4(0u, 0u, 0u, 0u);
+      if (c < c_hi) {
+        int ga, gb;
+        if (BITS == 4) {
+          ga = g64 ? 2 * c : c;
+          gb = ga + 1;
+        } else {
+          ga = min((c * CW + 40 * t) >> gsh, gpr - 1);
+          gb = min(ga + 1, gpr - 1);
+        }
+        sv[i][0] = __ldg(sr0 + ga);
+        sv[i][1] = __ldg(sr1 + ga);
+        if (BITS == 3 || g64) {
+          sv[i][2] = __ldg(sr0 + gb);
+          sv[i][3] = __ldg(sr1 + gb);
+        }
+      }
+    }
+  };
+  fetch(c_lo);
+  if (tid == 0) zero16[0] = zero16[1] = zero16[2] = zero16[3] = 0u;
+  pdl_enter();   // activations and the residual stream come from the previous kernels
+
+  // ---- stage the activations (permuted) into xs; padding codes see zeros
+  const int kpad = nch * CW;
+  if (NORM) {
+    // x = fp16(h * rsqrt(mean(h^2) + eps) * gamma) per token row, the sum of
+    // squares in a fixed order (per thread, xor tree, warps in order)
+    for (int b = 0; b < a.T; ++b) {
+      const float* hr = a.h + (size_t)b * a.K;
+      float ss = 0.f;
+      for (int k = 4 * tid; k < a.K; k += 4 * DG_THREADS) {
+        const float4 v = *reinterpret_cast<const float4*>(hr + k);
+        ss = fmaf(v.x, v.x, ss);
+        ss = fmaf(v.y, v.y, ss);
+        ss = fmaf(v.z, v.z, ss);
+        ss = fmaf(v.w, v.w, ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      if (lane == 0) nred[b][warp] = ss;
+    }
+    __syncthreads();
+    for (int b = 0; b < a.T; ++b) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < DG_WARPS; ++w) tot += nred[b][w];
+      const float r = rsqrtf(tot / (float)a.K + a.eps);
+      const float* hr = a.h + (size_t)b * a.K;
+      __half* xr = xs + (size_t)b * xw;
+      for (int k = 4 * tid; k < a.K; k += 4 * DG_THREADS) {
+        const float4 v = *reinterpret_cast<const float4*>(hr + k);
+        const float4 gm = __ldg(reinterpret_cast<const float4*>(a.gamma + k));
+        xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
+        xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
+        xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
+        xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+      }
+      for (int k = a.K + tid; k < kpad; k += DG_THREADS) xr[xpos<BITS>(k)] = __float2half_rn(0.f);
+    }
+  } else {
+    for (int b = 0; b < a.T; ++b) {
+      const __half* src = a.x + (size_t)b * a.K;
+      __half* xr = xs + (size_t)b * xw;
+      if (BITS == 4) {
+        // eight consecutive k -> four half2 stores
+        for (int k = 8 * tid; k < a.K; k += 8 * DG_THREADS) {
+          const uint4 v = *reinterpret_cast<const uint4*>(src + k);
+          const __half* e = reinterpret_cast<const __half*>(&v);
+          const int base = xpos<4>(k);   // position of element 0 (k-step 2q, slot 2t)
+          *reinterpret_cast<__half2*>(xr + base) = __halves2half2(e[0], e[4]);
+          *reinterpret_cast<__half2*>(xr + base + 8) = __halves2half2(e[1], e[5]);
+          *reinterpret_cast<__half2*>(xr + base + 16) = __halves2half2(e[2], e[6]);
+          *reinterpret_cast<__half2*>(xr + base + 24) = __halves2half2(e[3], e[7]);
+        }
+      } else {
+        for (int k = tid; k < kpad; k += DG_THREADS)
+          xr[xpos<BITS>(k)] = k < a.K ? src[k] : __float2half_rn(0.f);
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- the MMAs: this warp's chunks of its tile
+  // ldmatrix rows: lane l supplies token row l & 7 (a zero block for rows >= T)
+  const int lr = lane & 7, lq = lane >> 3;
+  const uint32_t zaddr = (uint32_t)__cvta_generic_to_shared(zero16);
+  const bool lrow_ok = lr < a.T;
+  const uint32_t lbase =
+      lrow_ok ? (uint32_t)__cvta_generic_to_shared(xs + (size_t)lr * xw + 8 * lq) : zaddr;
+  const uint32_t lmul = lrow_ok ? 2u : 0u;   // bytes per staged element (0: stay on the zero block)
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int cb = c_lo; cb < c_hi; cb += MC) {
+    if (cb != c_lo) fetch(cb);
+#pragma unroll
+    for (int i = 0; i < MC; ++i) {
+      const int c = cb + i;
+      if (c >= c_hi) break;
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&wv[i][0]);   // row g
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&wv[i][1]);   // row g + 8
+      const uint32_t xb = lbase + lmul * (uint32_t)(c * CW);
+      if (BITS == 4) {
+        float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb2[4] = {0.f, 0.f, 0.f, 0.f};
+        const bool first = t < 2;   // G = 64: this lane's codes are in the chunk's first group
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t p0[4], p1[4];
+          int4_pairs(w0[q], p0);
+          int4_pairs(w1[q], p1);
+          uint32_t b[4];
+          ldsm_x4(b, xb + lmul * (uint32_t)(32 * q));   // k steps 2q and 2q + 1
+          const uint32_t A0[4] = {p0[0], p1[0], p0[1], p1[1]};
+          const uint32_t A1[4] = {p0[2], p1[2], p0[3], p1[3]};
+          if (!g64) {
+            mma16816(ca, A0, b[0], b[1]);
+            mma16816(ca, A1, b[2], b[3]);
+          } else {
+            const uint32_t z[4] = {0u, 0u, 0u, 0u};
+            mma16816(ca, first ? A0 : z, b[0], b[1]);
+            mma16816(ca, first ? A1 : z, b[2], b[3]);
+            mma16816(cb2, first ? z : A0, b[0], b[1]);
+            mma16816(cb2, first ? z : A1, b[2], b[3]);
+          }
+        }
+        const float f0 = __half2float(sv[i][0]), f1 = __half2float(sv[i][1]);
+        acc[0] = fmaf(ca[0], f0, acc[0]);
+        acc[1] = fmaf(ca[1], f0, acc[1]);
+        acc[2] = fmaf(ca[2], f1, acc[2]);
+        acc[3] = fmaf(ca[3], f1, acc[3]);
+        if (g64) {
+          const float e0 = __half2float(sv[i][2]), e1 = __half2float(sv[i][3]);
+          acc[0] = fmaf(cb2[0], e0, acc[0]);
+          acc[1] = fmaf(cb2[1], e0, acc[1]);
+          acc[2] = fmaf(cb2[2], e1, acc[2]);
+          acc[3] = fmaf(cb2[3], e1, acc[3]);
+        }
+      } else {
+        // INT3: the lane's codes 40t + L with L < bnd are in the lower scale
+        // group; bnd is a multiple of 8 (chunk, lane and group starts all
+        // are), so each octet of codes L = 8o .. 8o + 7 has one scale
+        const int k0 = c * CW + 40 * t;
+        const int bnd = (((k0 >> gsh) + 1) << gsh) - k0;
+        __half so0[5], so1[5];
+#pragma unroll
+        for (int oc = 0; oc < 5; ++oc) {
+          so0[oc] = 8 * oc < bnd ? sv[i][0] : sv[i][2];
+          so1[oc] = 8 * oc < bnd ? sv[i][1] : sv[i][3];
+        }
+#define TL_SC(p, La, Lb, so) hmul2_bits((p), h2bits(__halves2half2(so[(La) >> 3], so[(Lb) >> 3])))
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t b[4];
+          ldsm_x4(b, xb + lmul * (uint32_t)(32 * q));   // k steps 2q, 2q + 1
+          const int L = 10 * q;
+          const uint32_t A0[4] = {TL_SC(int3_pair_i6<0>(w0[q]), L, L + 6, so0),
+                                  TL_SC(int3_pair_i6<0>(w1[q]), L, L + 6, so1),
+                                  TL_SC(int3_pair_i6<1>(w0[q]), L + 1, L + 7, so0),
+                                  TL_SC(int3_pair_i6<1>(w1[q]), L + 1, L + 7, so1)};
+          const uint32_t A1[4] = {TL_SC(int3_pair_i6<2>(w0[q]), L + 2, L + 8, so0),
+                                  TL_SC(int3_pair_i6<2>(w1[q]), L + 2, L + 8, so1),
+                                  TL_SC(int3_pair_i6<3>(w0[q]), L + 3, L + 9, so0),
+                                  TL_SC(int3_pair_i6<3>(w1[q]), L + 3, L + 9, so1)};
+          mma16816(acc, A0, b[0], b[1]);
+          mma16816(acc, A1, b[2], b[3]);
+        }
+        {
+          uint32_t b[4];
+          ldsm_x4(b, xb + lmul * 128u);                  // k steps 8 and 9
+          const uint32_t A0[4] = {TL_SC(int3_pair_c4(w0[0], w0[1]), 4, 14, so0),
+                                  TL_SC(int3_pair_c4(w1[0], w1[1]), 4, 14, so1),
+                                  TL_SC(int3_pair_c5(w0[0], w0[1]), 5, 15, so0),
+                                  TL_SC(int3_pair_c5(w1[0], w1[1]), 5, 15, so1)};
+          const uint32_t A1[4] = {TL_SC(int3_pair_c4(w0[2], w0[3]), 24, 34, so0),
+                                  TL_SC(int3_pair_c4(w1[2], w1[3]), 24, 34, so1),
+                                  TL_SC(int3_pair_c5(w0[2], w0[3]), 25, 35, so0),
+                                  TL_SC(int3_pair_c5(w1[2], w1[3]), 25, 35, so1)};
+          mma16816(acc, A0, b[0], b[1]);
+          mma16816(acc, A1, b[2], b[3]);
+        }
+#undef TL_SC
+      }
+    }
+  }
+
+  // ---- the warps' sums, added in warp order
+  float* rw = red + ((size_t)(m * W + ks) * 16) * 8;      // [16 rows][8 tokens]
+  rw[g * 8 + 2 * t] = acc[0];
+  rw[g * 8 + 2 * t + 1] = acc[1];
+  rw[(g + 8) * 8 + 2 * t] = acc[2];
+  rw[(g + 8) * 8 + 2 * t + 1] = acc[3];
+  __syncthreads();
+  if (EPI == EPI_SWIGLU) {
+    if (tid < 16 * 8) {
+      const int r = tid >> 3, b = tid & 7;
+      if (b < a.T) {
+        float gs = 0.f, us = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) {
+          gs += red[((0 * W + w) * 16 + r) * 8 + b];
+          us += red[((1 * W + w) * 16 + r) * 8 + b];
+        }
+        const float silu = gs / (1.0f + __expf(-gs));
+        a.u[(size_t)b * a.N + row0 + r] = __float2half_rn(silu * us);
+      }
+    }
+  } else {
+    for (int i = tid; i < MT * 16 * 8; i += DG_THREADS) {
+      const int mm = i >> 7, r = (i >> 3) & 15, b = i & 7;
+      const int n = (blockIdx.x * MT + mm) * 16 + r;
+      float y = 0.f;
+#pragma unroll
+      for (int w = 0; w < W; ++w) y += red[((mm * W + w) * 16 + r) * 8 + b];
+      if (EPI == EPI_OUT) {
+        if (b < a.T) a.out[(size_t)b * a.N + n] = y;
+      } else {
+        if (b < a.T) {
+          float* hp = a.hres + (size_t)b * a.N + n;
+          const float hn = *hp + y;
+          *hp = hn;
+          if (a.trace) a.trace[(size_t)a.out_row[b] * a.N + n] = hn;
+        } else if (a.trace && b < a.trace_rows) {
+          // lanes that ran fewer iterations keep their last value in the trace
+          a.trace[(size_t)a.out_row[b] * a.N + n] = a.hres[(size_t)b * a.N + n];
+        }
+      }
+    }
+  }
+}
+
+template <int BITS, int MT, bool NORM, int EPI, int MC>
+tl_status launch_dg_mc(const DgArgs& a, int grid, size_t smem, cudaStream_t s) {
+  static std::atomic<uint64_t> attr_done{0};
+  TL_TRY(once_per_device(attr_done, []() -> tl_status {
+    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, MC>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    return ok();
+  }));
+  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, MC>), grid, DG_THREADS, smem, s, a);
+  return ok();
+}
+
+template <int BITS, int MT, bool NORM, int EPI>
+tl_status launch_dg(const DgArgs& a, int grid, cudaStream_t s) {
+  const int nvec = a.wpr / 4, nch = (nvec + 3) / 4;
+  const size_t xw = (size_t)nch * DgFmt<BITS>::CW + 8;
+  const size_t smem = (size_t)a.T * xw * 2 + (size_t)DG_WARPS * 16 * 8 * 4;
+  if (smem > 200 * 1024)
+    return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: K = %d x %d tokens needs too much shared memory",
+                     a.K, a.T);
+  const int per = (nch + DG_WARPS / MT - 1) / (DG_WARPS / MT);   // chunks of the longest k range
+  if (per <= 2) return launch_dg_mc<BITS, MT, NORM, EPI, 2>(a, grid, smem, s);
+  if (per <= 4) return launch_dg_mc<BITS, MT, NORM, EPI, 4>(a, grid, smem, s);
+  return launch_dg_mc<BITS, MT, NORM, EPI, DG_MAXC>(a, grid, smem, s);
+}
+
+}  // namespace
+
+bool dec_gemv_eligible(int N, int K, int T, int bits) {
+  return T >= 1 && T <= 8 && N % 16 == 0 && (bits == 3 || K % 128 == 0);
+}
+
+tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
+  if (d.T == 0) return ok();
+  if (d.T < 0 || d.T > 8) return set_error(TL_ERR_INVALID_ARG, "decode GEMV: %d tokens", d.T);
+  DgArgs a;
+  a.w0 = d.w0;
+  a.s0 = d.s0;
+  a.w1 = d.w1;
+  a.s1 = d.s1;
+  a.N = d.N;
+  a.K = d.K;
+  a.G = d.G;
+  a.wpr = d.bits == 4 ? d.K / 8 : ((d.K + 9) / 10 + 3) / 4 * 4;
+  a.T = d.T;
+  a.x = d.x;
+  a.h = d.h;
+  a.gamma = d.gamma;
+  a.eps = d.eps;
+  a.out = d.out;
+  a.hres = d.hres;
+  a.u = d.u;
+  a.trace = d.trace;
+  a.out_row = d.out_row;
+  a.trace_rows = d.trace_rows;
+  if (!dec_gemv_eligible(d.N, d.K, d.T, d.bits))
+    return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: shape N %d K %d", d.N, d.K);
+  const bool norm = d.h != nullptr;
+  switch (d.epi) {
+    case DEC_EPI_SWIGLU:
+      if (!norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: SwiGLU needs the norm prologue");
+      return d.bits == 4 ? launch_dg<4, 2, true, EPI_SWIGLU>(a, d.N / 16, s)
+                         : launch_dg<3, 2, true, EPI_SWIGLU>(a, d.N / 16, s);
+    case DEC_EPI_RESID:
+      if (norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: residual epilogue takes x");
+      return d.bits == 4 ? launch_dg<4, 1, false, EPI_RESID>(a, d.N / 16, s)
+                         : launch_dg<3, 1, false, EPI_RESID>(a, d.N / 16, s);
+    default:
+      if (norm)
+        return d.bits == 4 ? launch_dg<4, 1, true, EPI_OUT>(a, d.N / 16, s)
+                           : launch_dg<3, 1, true, EPI_OUT>(a, d.N / 16, s);
+      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT>(a, d.N / 16, s)
+                         : launch_dg<3, 1, false, EPI_OUT>(a, d.N / 16, s);
+  }
+}
+
+}  // namespace tl

@@ -62,7 +62,7 @@ extern "C" __attribute__((visibility("default"))) tl_status tl_linear_noalloc(
     int T, float* y, tl_stream stream) {
   TL_TRY(check_linear(N, K, group, T));
   TL_CHECK_ARG(packed && scales && x && y, "NULL device pointer");
-  const int S = gemm_splits(N, K, T);
+  const int S = linear_splits(N, K, T);
   const size_t need = S > 1 ? (size_t)S * T * N * sizeof(float) : 0;
   if (need > kNoAllocScratchBytes)
     return set_error(TL_ERR_INVALID_ARG,
@@ -72,19 +72,6 @@ extern "C" __attribute__((visibility("default"))) tl_status tl_linear_noalloc(
   TL_TRY(gemm_tc_init());
   void* scratch = nullptr;
   if (S > 1) TL_TRY(scratch_address(&scratch));
-  GemmArgs a;
-  memset(&a, 0, sizeof(a));
-  a.w0 = a.w1 = packed;
-  a.s0 = a.s1 = (const __half*)scales;
-  a.n_split = a.N = N;
-  a.K = K;
-  a.G = group;
-  a.x = (const __half*)x;
-  a.T = T;
-  a.splits = S;
-  a.part = S > 1 ? (float*)scratch : y;
-  cudaStream_t s = (cudaStream_t)stream;
-  TL_TRY(launch_gemm(a, s));
-  if (S > 1) TL_TRY(launch_split_sum((const float*)scratch, S, (long)T * N, y, s));
-  return ok();
+  return launch_linear(packed, scales, N, K, group, x, T, y, (float*)scratch,
+                       (cudaStream_t)stream);
 }

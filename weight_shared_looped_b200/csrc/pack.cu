@@ -107,25 +107,6 @@ __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int K, int bi
   }
 }
 
-// INT3 canonical -> INT4 canonical with identical codes (u4 = code + 8).
-__global__ void int3_to_int4_kernel(const uint32_t* __restrict__ src, int K, int wpr3,
-                                    long n_words4, uint32_t* __restrict__ dst) {
-  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n_words4) return;
-  int wpr4 = K / 8;
-  long row = i / wpr4;
-  int j = (int)(i % wpr4);
-  const uint32_t* r = src + row * wpr3;
-  uint32_t word = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    int k = 8 * j + e;
-    uint32_t u3 = (r[k / 10] >> (3 * (k % 10))) & 7u;
-    word |= (u3 + 4u) << (4 * e);   // code = u3 - 4, u4 = code + 8
-  }
-  dst[i] = word;
-}
-
 // One warp per row of hd <= 256 fp16 values.
 __global__ void kv_quant_int8_kernel(const __half* __restrict__ x, int rows, int hd,
                                      int8_t* __restrict__ codes, __half* __restrict__ scales) {
@@ -182,14 +163,6 @@ tl_status launch_unpack(const uint32_t* packed, int N, int K, int bits, int8_t* 
   int wpr = bits == 4 ? K / 8 : ((K + 9) / 10 + 3) / 4 * 4;
   long n_words = (long)N * wpr;
   unpack_kernel<<<blocks_for(n_words, 256), 256, 0, s>>>(packed, K, bits, wpr, n_words, codes);
-  TL_LAUNCH_CHECK();
-  return ok();
-}
-
-tl_status launch_int3_to_int4(const uint32_t* src, int N, int K, uint32_t* dst, cudaStream_t s) {
-  int wpr3 = ((K + 9) / 10 + 3) / 4 * 4;
-  long n_words4 = (long)N * (K / 8);
-  int3_to_int4_kernel<<<blocks_for(n_words4, 256), 256, 0, s>>>(src, K, wpr3, n_words4, dst);
   TL_LAUNCH_CHECK();
   return ok();
 }

@@ -61,12 +61,11 @@ tl_status launch_unpack(const uint32_t* packed, int N, int K, int bits, int8_t* 
                         cudaStream_t s);
 tl_status launch_kv_quant_int8(const __half* x, int rows, int hd, int8_t* codes, __half* scales,
                                cudaStream_t s);
-// INT3 canonical rows -> INT4 canonical rows (same codes), for the GEMM kernels
-tl_status launch_int3_to_int4(const uint32_t* src, int N, int K, uint32_t* dst, cudaStream_t s);
 
 // quantised-weight GEMM (gemm_mma.cu): part[z][t][n] = sum_{k in split z} x[t][k] * W[n][k]
 struct GemmArgs {
-  const uint32_t* w0;   // INT4 canonical words, rows [0, n_split)
+  int bits;             // 4, or 3 (canonical INT3 rows, tensor-core kernel only)
+  const uint32_t* w0;   // canonical packed words, rows [0, n_split)
   const __half* s0;
   const uint32_t* w1;   // rows [n_split, N) (may equal w0 when n_split == N)
   const __half* s1;
@@ -77,11 +76,6 @@ struct GemmArgs {
   float* part;          // fp32 [S][T][N]
   int splits;           // S (from gemm_splits)
   int* status;          // device status word for bounded-wait timeouts (may be null)
-  // decode GEMV only: when x_part is set the activations are
-  // silu(sum_s x_part[s][t][k]) * sum_s x_part[s][t][x_F + k] (SwiGLU of the
-  // gate|up partial sums) instead of x
-  const float* x_part;
-  int x_S, x_F;
   // tensor-core kernel with one split only, for [gate; up] weights (n_split =
   // F, N = 2F): when swiglu_u is set, each CTA takes 64 gate rows and the same
   // 64 up rows and writes swiglu_u[t][f] = fp16(silu(gate) * up) (fp16 [T][F])
@@ -93,19 +87,50 @@ struct GemmArgs {
 // 1 <= T <= 8192.
 tl_status check_linear(int N, int K, int group, int T);
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
-// kernel for T >= 64, the mma.sync register-dequant kernel below that.
-int gemm_splits(int N, int K, int T);
+// kernel for T >= 64, the mma.sync register-dequant kernel below that (the
+// decode projections use launch_dec_gemv instead).
+int gemm_splits(int N, int K, int T, int bits = 4);
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s);
 // the two kernels
 int gemm_mma_splits(int N, int K, int T);
 tl_status launch_gemm_mma(const GemmArgs& a, cudaStream_t s);
-bool gemm_tc_eligible(int N, int K, int T);
+bool gemm_tc_eligible(int N, int K, int T, int bits = 4);
 int gemm_tc_splits(int N, int K, int T);
 tl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t s);
 tl_status gemm_tc_init();
 tl_status launch_bounded_wait_check(int* status, uint64_t limit_ns, cudaStream_t s);
 // y[t][n] = sum_{s < S} part[s][t][n], in order s = 0, 1, ...
 tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStream_t s);
+
+// decode-sized projections (gemv_dec.cu): T <= 8 tokens, no split-K, the
+// pre-norm, residual add and SwiGLU folded in (see the file's header)
+enum DecEpi { DEC_EPI_OUT = 0, DEC_EPI_RESID = 1, DEC_EPI_SWIGLU = 2 };
+struct DecGemvArgs {
+  const uint32_t* w0;   // canonical packed words (bits 3 or 4) [N][wpr]
+  const __half* s0;     // fp16 scales [N][K/G]
+  const uint32_t* w1;   // DEC_EPI_SWIGLU: the up matrix (w0 = gate)
+  const __half* s1;
+  int N, K, G, bits, T;
+  const __half* x;      // fp16 [T][K] activations, or null with h set
+  const float* h;       // fp32 [T][K] residual stream: x = fp16(rmsnorm(h) * gamma)
+  const float* gamma;
+  float eps;
+  int epi;              // DecEpi
+  float* out;           // DEC_EPI_OUT: fp32 [T][N]
+  float* hres;          // DEC_EPI_RESID: fp32 residual [rows][N], += y
+  __half* u;            // DEC_EPI_SWIGLU: fp16 [T][N]
+  float* trace;         // DEC_EPI_RESID: null or fp32 [trace_rows][N] (rows by out_row)
+  const int32_t* out_row;
+  int trace_rows;
+};
+bool dec_gemv_eligible(int N, int K, int T, int bits);
+tl_status launch_dec_gemv(const DecGemvArgs& a, cudaStream_t s);
+// The linear-layer hook's kernels: the decode projection kernel for T <= 8
+// (no split-K), launch_gemm otherwise (split-K sums in `scratch`, then added
+// in split order into y).  linear_splits gives the split count.
+int linear_splits(int N, int K, int T);
+tl_status launch_linear(const uint32_t* packed, const uint16_t* scales, int N, int K, int group,
+                        const uint16_t* x, int T, float* y, float* scratch, cudaStream_t s);
 
 // elementwise (elementwise.cu)
 struct EmbedArgs {
@@ -159,6 +184,14 @@ tl_status launch_rope_kv(const RopeKvArgs& a, cudaStream_t s);
 tl_status launch_swiglu(const float* part, int S, int rows, int F, __half* u, cudaStream_t s);
 tl_status launch_set_pos(KvHeader* hdr, int lane, int value, cudaStream_t s);
 tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s);
+tl_status launch_add_pos(KvHeader* hdr, int lane, int n, cudaStream_t s);   // pos[lane] += n
+tl_status launch_set_i32(int32_t* p, int value, cudaStream_t s);
+
+// greedy head over the tied embedding (head.cu): ids[r] = argmax_v y[r] . E[v]
+// (lowest v on a tie), n <= 8 rows; part_s / part_v: head_parts() * 8 each
+int head_parts();
+tl_status launch_greedy_head(const float* y, int n, const __half* E, int V, int d, float* part_s,
+                             int* part_v, int32_t* ids, cudaStream_t s);
 
 // attention (attention.cu)
 tl_status launch_attn_prefill(const __half* q, const __half* k, const __half* v, __half* out,
@@ -176,6 +209,8 @@ struct DecodeAttnArgs {
   int layer, max_ctx, kv_int8;
   int row_lane[kMaxLanes];   // lane of each row
   int row_cum[kMaxLanes];    // cache layers of the lanes before that lane
+  int row_off[kMaxLanes];    // position of the row's token = the lane's position + row_off
+  int mode;                  // 0 append + attend, 1 append only, 2 attend only
   int chunks;                // context chunks per CTA; 0 = fewest waves
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);

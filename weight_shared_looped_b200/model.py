@@ -13,7 +13,8 @@ from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_dec
                tl_kv_bytes, tl_kv_create, tl_kv_destroy, tl_kv_layer_ptrs, tl_kv_position,
                tl_kv_reset, tl_kv_set_position, tl_model_create, tl_model_destroy,
                tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
-               tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status)
+               tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status, tl_extend,
+               tl_greedy_head, tl_spec_step)
 
 MATRICES = ("qkv", "o", "gate", "up", "down")
 
@@ -105,6 +106,25 @@ class DeviceModel:
         tl_decode_step(self.handle, kv.handle, ids, h_in, L_per_lane=L_per_lane, y_out=y_out,
                        h_trace=h_trace, stream=stream)
         return y_out
+
+    def extend(self, kv: "DeviceKV", ids=None, h_in=None, *, lane: int = 0, L: int, y_out=None,
+               h_trace=None, stream=None) -> torch.Tensor:
+        n = (ids if ids is not None else h_in).shape[0]
+        if y_out is None:
+            y_out = torch.empty(n, self.d, dtype=torch.float32, device="cuda")
+        tl_extend(self.handle, kv.handle, lane, ids, h_in, L=L, y_out=y_out, h_trace=h_trace,
+                  stream=stream)
+        return y_out
+
+    def greedy_head(self, y, stream=None) -> torch.Tensor:
+        ids = torch.empty(y.shape[0], dtype=torch.int32, device="cuda")
+        tl_greedy_head(self.handle, y, ids, stream=stream)
+        return ids
+
+    def spec_step(self, kv: "DeviceKV", token: int, *, lane: int = 0, K: int, L_draft: int,
+                  L_verify: int, stream=None):
+        return tl_spec_step(self.handle, kv.handle, lane, token, K, L_draft, L_verify,
+                            stream=stream)
 
     def sync_status(self, stream=None) -> int:
         return tl_sync_status(self.handle, stream)
