@@ -129,6 +129,53 @@ def unpack_codes(packed: np.ndarray, k: int, bits: int) -> np.ndarray:
     raise ValueError("bits must be 3 or 4")
 
 
+def sign_of_frac(w: np.ndarray, group: int, bits: int = 4) -> np.ndarray:
+    """The 1-bit sign-of-frac channel of group-wise quantised weights
+    ("Performance and Memory", "Cross-iteration stochastic rounding": INT4 +
+    1-bit sign-of-frac, +25 % storage; "Current Status", architecture-unique
+    features table, deterministic error cancellation row: even iterations use
+    the standard rounding, odd iterations apply the sign correction).
+    bit[n, k] = 1 when w / s lies above its code (the rounding went down), else
+    0; with the same fp32 quotient as quantize_groupwise.  Returns uint8 [N, K]."""
+    w = np.asarray(w, dtype=np.float32)
+    n, k = w.shape
+    codes, scale16 = quantize_groupwise(w, bits, group)
+    s = np.repeat(scale16.astype(np.float32), group, axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = (w / s).astype(np.float32)
+    return ((s != 0) & (ratio > codes.astype(np.float32))).astype(np.uint8)
+
+
+def pack_bits(bits: np.ndarray) -> np.ndarray:
+    """[N, K] bits -> uint32 [N, ceil(K/32)]; element 32j + i in bit i of word j
+    (bits past K are zero)."""
+    b = np.asarray(bits, dtype=np.uint64)
+    n, k = b.shape
+    nw = (k + 31) // 32
+    b = np.concatenate([b, np.zeros((n, nw * 32 - k), np.uint64)], axis=1).reshape(n, nw, 32)
+    word = np.zeros((n, nw), dtype=np.uint64)
+    for i in range(32):
+        word |= b[:, :, i] << np.uint64(i)
+    return word.astype(np.uint32)
+
+
+def unpack_bits(words: np.ndarray, k: int) -> np.ndarray:
+    w = np.asarray(words, dtype=np.uint64)
+    out = np.zeros((w.shape[0], w.shape[1], 32), dtype=np.uint8)
+    for i in range(32):
+        out[:, :, i] = (w >> np.uint64(i)) & np.uint64(1)
+    return out.reshape(w.shape[0], -1)[:, :k]
+
+
+def odd_iteration_codes(codes: np.ndarray, bits: np.ndarray) -> np.ndarray:
+    """The codes an odd loop iteration uses: each moved to its other rounding
+    neighbour, code + 1 where the bit is set, code - 1 where it is clear (so the
+    two neighbours bracket w / s; a code exactly equal to w / s moves down).
+    May leave the storage range by one (-9 .. 8): it is an arithmetic value,
+    never stored."""
+    return codes.astype(np.int16) + np.where(np.asarray(bits) != 0, 1, -1).astype(np.int16)
+
+
 def dequantize(codes: np.ndarray, scales16: np.ndarray, group: int) -> np.ndarray:
     """W[n, k] = code[n, k] * float(scale[n, k // group]), in fp64 (exact)."""
     s = np.repeat(scales16.astype(F64), group, axis=1)
@@ -251,9 +298,17 @@ class Block:
         d, f, g, bits = cfg["d_model"], cfg["ffn"], cfg["group"], cfg["bits"]
         shapes = {"qkv": (3 * d, d), "o": (d, d), "gate": (f, d), "up": (f, d), "down": (d, f)}
         self.W = {}
+        self.W_odd = None
         for name, (n, k) in shapes.items():
             codes = unpack_codes(packed[f"w_{name}"], k, bits)
             self.W[name] = dequantize(codes, packed[f"s_{name}"], g)
+            if f"sign_{name}" in packed:
+                # the cross-iteration rounding channel: odd loop iterations'
+                # weights (odd_iteration_codes x the same scales)
+                if self.W_odd is None:
+                    self.W_odd = {}
+                odd = odd_iteration_codes(codes, unpack_bits(packed[f"sign_{name}"], k))
+                self.W_odd[name] = dequantize(odd, packed[f"s_{name}"], g)
         self.gamma_attn = np.asarray(packed["gamma_attn"], F64)
         self.gamma_ffn = np.asarray(packed["gamma_ffn"], F64)
 
@@ -261,35 +316,45 @@ class Block:
     def from_fp32(cls, weights: Dict[str, np.ndarray], cfg: Dict) -> "Block":
         return cls(pack_block(weights, cfg["bits"], cfg["group"]), cfg)
 
-    def qkv(self, h: np.ndarray, positions: np.ndarray):
+    def weights(self, odd: bool = False) -> Dict[str, np.ndarray]:
+        """The weights of a loop iteration: the odd-iteration set when asked for
+        and present, else the standard one."""
+        return self.W_odd if odd and self.W_odd is not None else self.W
+
+    def qkv(self, h: np.ndarray, positions: np.ndarray, odd: bool = False):
         """RMSNorm -> QKV projection -> RoPE on q and k."""
         c = self.cfg
         t = h.shape[0]
         x = rmsnorm(h, self.gamma_attn, c["eps"])
-        qkv = x @ self.W["qkv"].T
+        qkv = x @ self.weights(odd)["qkv"].T
         d, nh, hd = c["d_model"], c["n_heads"], c["head_dim"]
         q = qkv[:, :d].reshape(t, nh, hd)
         k = qkv[:, d:2 * d].reshape(t, nh, hd)
         v = qkv[:, 2 * d:].reshape(t, nh, hd)
         return rope(q, positions, c["rope_theta"]), rope(k, positions, c["rope_theta"]), v
 
-    def finish(self, h: np.ndarray, attn: np.ndarray) -> np.ndarray:
+    def finish(self, h: np.ndarray, attn: np.ndarray, odd: bool = False) -> np.ndarray:
         """O projection + residual, then RMSNorm -> SwiGLU MLP + residual."""
         c = self.cfg
         t = h.shape[0]
-        h = h + attn.reshape(t, c["d_model"]) @ self.W["o"].T
+        W = self.weights(odd)
+        h = h + attn.reshape(t, c["d_model"]) @ W["o"].T
         x = rmsnorm(h, self.gamma_ffn, c["eps"])
-        u = silu(x @ self.W["gate"].T) * (x @ self.W["up"].T)
-        return h + u @ self.W["down"].T
+        u = silu(x @ W["gate"].T) * (x @ W["up"].T)
+        return h + u @ W["down"].T
 
 
-def pack_block(weights: Dict[str, np.ndarray], bits: int, group: int) -> Dict[str, np.ndarray]:
-    """Quantise and pack the five matrices of one block."""
+def pack_block(weights: Dict[str, np.ndarray], bits: int, group: int,
+               sign: bool = False) -> Dict[str, np.ndarray]:
+    """Quantise and pack the five matrices of one block (with the 1-bit
+    sign-of-frac channel of each when `sign`)."""
     out = {}
     for name in ("qkv", "o", "gate", "up", "down"):
         codes, scales = quantize_groupwise(weights[f"w_{name}"], bits, group)
         out[f"w_{name}"] = pack_codes(codes, bits)
         out[f"s_{name}"] = scales
+        if sign:
+            out[f"sign_{name}"] = pack_bits(sign_of_frac(weights[f"w_{name}"], group, bits))
     out["gamma_attn"] = weights["gamma_attn"]
     out["gamma_ffn"] = weights["gamma_ffn"]
     return out
@@ -371,6 +436,13 @@ class LoopedModel:
         self.gamma_final = np.asarray(gamma_final, F64)
         self.embed16 = embed16
         self.cfg = loop.cfg
+        self.cross_iter = False   # odd loop iterations use the loop block's odd weights
+
+    def odd(self, layer: int) -> bool:
+        """Whether layer `layer` is an odd loop iteration run with the odd
+        weights (cross-iteration rounding on, and the loop block has them)."""
+        it = layer - len(self.pre)
+        return self.cross_iter and it >= 0 and it % 2 == 1
 
     def schedule(self, L: int) -> List[Block]:
         """Block applied at each layer index: the pre-blocks, then the same
@@ -414,10 +486,11 @@ class LoopedModel:
         loops = np.full(h.shape[0], L)
         for layer, blk in enumerate(self.schedule(L)):
             self._exit_check(h, layer, frozen, loops, exit_tau)
-            q, k, v = blk.qkv(h, pos)
+            odd = self.odd(layer)
+            q, k, v = blk.qkv(h, pos, odd)
             if kv is not None:
                 kv[layer].append(k, v)
-            h = np.where(frozen[:, None], h, blk.finish(h, causal_attention(q, k, v, pos)))
+            h = np.where(frozen[:, None], h, blk.finish(h, causal_attention(q, k, v, pos), odd))
             if trace is not None:
                 trace.append(h.copy())
         if info is not None:
@@ -440,11 +513,12 @@ class LoopedModel:
         loops = np.full(h.shape[0], L)
         for layer, blk in enumerate(self.schedule(L)):
             self._exit_check(h, layer, frozen, loops, exit_tau)
-            q, k, v = blk.qkv(h, pos)
+            odd = self.odd(layer)
+            q, k, v = blk.qkv(h, pos, odd)
             slot = kv[layer]
             slot.append(k, v)
             h = np.where(frozen[:, None], h,
-                         blk.finish(h, causal_attention(q, slot.k, slot.v, pos)))   # keys 0..pos
+                         blk.finish(h, causal_attention(q, slot.k, slot.v, pos), odd))   # keys 0..pos
             if trace is not None:
                 trace.append(h.copy())
         if info is not None:

@@ -604,3 +604,76 @@ def test_spec_step_emits_the_greedy_decode_tokens(K, L_draft):
     assert got == want
     if L_draft == L:                    # the draft is the verify model: all accepted
         assert len(m.spec_step(tok, K, L, L, kv_s)) == K + 1
+
+
+# ---------------------------------------------------------------- cross-iteration rounding (sign of frac)
+
+def test_sign_of_frac_hand_worked():
+    """One group of eight weights with absmax 3.5, so s = fp16(3.5 / 7) = 0.5
+    exactly and w / s = 7, 2.4, -2.4, 0.52, -0.48, 0, 5.5, -6.5: codes round to
+    nearest (ties to even), the bit says the quotient lies above its code, and
+    odd iterations take the other neighbour."""
+    w = np.array([[3.5, 1.2, -1.2, 0.26, -0.24, 0.0, 2.75, -3.25]], np.float32)
+    codes, scales = o.quantize_groupwise(w, 4, 8)
+    assert float(scales[0, 0]) == 0.5
+    assert codes.tolist() == [[7, 2, -2, 1, 0, 0, 6, -6]]
+    bits = o.sign_of_frac(w, 8)
+    assert bits.tolist() == [[0, 1, 0, 0, 0, 0, 0, 0]]
+    assert o.odd_iteration_codes(codes, bits).tolist() == [[6, 3, -3, 0, -1, -1, 5, -7]]
+
+
+@pytest.mark.parametrize("group", [64, 128])
+def test_odd_codes_bracket_the_quotient(group):
+    rng = np.random.default_rng(21)
+    w = (rng.standard_normal((16, 512)) * 0.02).astype(np.float32)
+    w[3, :group] = 0.0                                     # an all-zero group: s = 0
+    codes, scales = o.quantize_groupwise(w, 4, group)
+    bits = o.sign_of_frac(w, group)
+    odd = o.odd_iteration_codes(codes, bits)
+    s = np.repeat(scales.astype(np.float32), group, axis=1)
+    nz = s != 0
+    r = (w[nz] / s[nz]).astype(np.float32)
+    assert np.all(np.abs(odd[nz] - codes[nz]) == 1)
+    assert np.all(np.minimum(codes[nz], odd[nz]) <= r) and np.all(r <= np.maximum(codes[nz], odd[nz]))
+    assert not bits[~nz].any()
+    # both roundings dequantise to zero in an all-zero group
+    assert np.all(o.dequantize(odd, scales, group)[3, :group] == 0)
+
+
+def test_bit_plane_layout():
+    bits = np.zeros((2, 64), np.uint8)
+    bits[0, 0] = bits[0, 33] = bits[1, 31] = 1
+    words = o.pack_bits(bits)
+    assert words.tolist() == [[1, 2], [1 << 31, 0]]
+    assert np.array_equal(o.unpack_bits(words, 64), bits)
+
+
+def _sign_model():
+    cfg = _tiny_cfg()
+    pre = [o.Block.from_fp32(_tiny_weights(31), cfg)]
+    w = _tiny_weights(32)
+    loop = o.Block(o.pack_block(w, 4, cfg["group"], sign=True), cfg)
+    gam = 1 + 0.1 * np.random.default_rng(33).standard_normal(8)
+    emb = (np.random.default_rng(34).standard_normal((20, 8))).astype(np.float16)
+    return o.LoopedModel(pre, loop, gam, emb), w
+
+
+def test_cross_iteration_rounding_model():
+    m, w = _sign_model()
+    ids = np.array([3, 9, 14, 2, 7], np.int64)
+    base = {L: m.prefill(ids, L) for L in (1, 2, 3)}
+    m.cross_iter = True
+    assert np.array_equal(m.prefill(ids, 1), base[1])     # no odd iteration yet
+    assert not np.allclose(m.prefill(ids, 2), base[2])
+    # an unrolled stack: pre-block, loop, odd-weight loop, loop
+    packed = o.pack_block(w, 4, m.loop.cfg["group"], sign=True)
+    odd_blk = o.Block(packed, m.loop.cfg)
+    odd_blk.W = odd_blk.W_odd
+    plain = o.Block(o.pack_block(w, 4, m.loop.cfg["group"]), m.loop.cfg)
+    deep = o.LoopedModel(m.pre + [plain, odd_blk], plain, m.gamma_final, m.embed16)
+    assert np.allclose(m.prefill(ids, 3), deep.prefill(ids, 1), rtol=0, atol=1e-12)
+    # without a sign channel the switch changes nothing
+    m2 = _tiny_model()
+    y = m2.prefill(ids, 3)
+    m2.cross_iter = True
+    assert np.array_equal(m2.prefill(ids, 3), y)
