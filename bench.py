@@ -497,6 +497,57 @@ def loop_read_bytes(tl, blk) -> int:
     return block_bytes(tl, 3)
 
 
+def run_spec(model, kv, w, torch, np, dist, world, K=4, L_draft=2, L_verify=8, n_steps=24):
+    """Greedy self-speculative steps (K drafts at L_draft, one verify extend of
+    K + 1 tokens at L_verify) from the 256-token prompt, against plain greedy
+    decoding (one-token extend at L_verify + head) from the same state.  Each
+    speculative step synchronises once (acceptance is decided on the host), so
+    both loops are timed with CUDA events around the whole loop."""
+    import synthetic as syn
+    stream = torch.cuda.current_stream()
+    base = w.seq
+    tok0 = int(syn.decode_ids(w)[0])
+
+    def spec_loop():
+        kv.set_position(0, base)
+        tok, n_tok = tok0, 0
+        for _ in range(n_steps):
+            out = model.spec_step(kv, tok, K=K, L_draft=L_draft, L_verify=L_verify)
+            n_tok += len(out)
+            tok = out[-1]
+        return n_tok
+
+    def greedy_loop(n):
+        kv.set_position(0, base)
+        tok = torch.tensor([tok0], dtype=torch.int32, device="cuda")
+        for _ in range(n):
+            y = model.extend(kv, tok, L=L_verify)
+            tok = model.greedy_head(y)
+
+    spec_loop()          # warm the graphs
+    greedy_loop(2)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    n_tok = spec_loop()
+    b.record(stream)
+    torch.cuda.synchronize()
+    t_spec = max_over_ranks(a.elapsed_time(b) / 1e3, dist, "cuda")
+    a.record(stream)
+    greedy_loop(n_tok)
+    b.record(stream)
+    torch.cuda.synchronize()
+    t_greedy = max_over_ranks(a.elapsed_time(b) / 1e3, dist, "cuda")
+    return {"tok_s": round(n_tok * world / t_spec, 1),
+            "greedy_tok_s": round(n_tok * world / t_greedy, 1),
+            "tokens_per_step": round(n_tok / n_steps, 3),
+            "acceptance": round((n_tok - n_steps) / (n_steps * K), 4),
+            "K": K, "L_draft": L_draft, "L_verify": L_verify, "steps": n_steps,
+            "workload": "batch 1, FP16 KV, after the 256-token prompt; greedy tokens through the "
+                        "tied fp16 embedding (50257 x 2048); synthetic random weights, so the "
+                        "acceptance is what such weights give, not a trained model's"}
+
+
 def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg, l2_gbs):
     """KV-cached decode throughput: B=1 FP16 KV (prompt 256, 128 steps), B=8
     INT8 KV at context 2048 (64 steps), mixed-depth INT3 lanes (ctx 1024, 32
@@ -541,8 +592,15 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
                         **decode_roofline(t / w.steps, 3 * blk_bytes + kv_bytes, 7 * blk_bytes,
                                           hbm, l2_gbs),
                         "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
+
+    # self-speculative decode on the same cache ("Current Status", self-speculative
+    # row: L=2 draft, L=8 verify, same weights): greedy tokens through the tied
+    # embedding head; draft + verify throughput, acceptance, and plain greedy
+    # decode with the same head for comparison
+    out["spec_L2_L8"] = run_spec(model, kv, w, torch, np, dist, world)
     kv.close()
     torch.cuda.synchronize()
+    kv = None
 
     # B = 8, INT8 KV, context 2048 -> 2112
     w = syn.WORKLOADS["longctx_int8"]

@@ -217,6 +217,28 @@ tl_status tl_model_set_graphs(tl_model* model, int enable);
  * Errors: TL_ERR_INVALID_ARG for a NULL model or a value outside [0, 8]. */
 tl_status tl_model_set_decode_chunks(tl_model* model, int chunks_per_cta);
 
+/* Per-iteration safety check ("Current Status", architecture-unique features
+ * table, per-iteration safety check row: the residual stream's L2 norm is
+ * computed every iteration, above a threshold the loop stops; L checkpoints
+ * per token).  With tau >= 0, a token (prefill, extend) or lane (decode)
+ * whose residual stream leaves loop iteration i - 1 with an L2 norm above tau
+ * runs no further residual updates: its stream stays frozen, its output is
+ * the final RMSNorm of the frozen stream, and the later iterations' KV slots
+ * still receive the K/V its frozen stream produces.  The check costs no extra
+ * pass: it reads the sum of squares the iteration's RMSNorm computes anyway.
+ * Per-lane loop counts thereby become data-dependent; a lane's result stays
+ * independent of the other lanes.  tau < 0 (the default) turns it off.
+ * Frees the model's captured graphs.  Errors: TL_ERR_INVALID_ARG for a NULL
+ * model, NaN or +infinity. */
+tl_status tl_model_set_exit_threshold(tl_model* model, float tau);
+
+/* Loop iterations each output row of the last forward call ran (after the
+ * stream's work): the loop count L unless the residual-norm check stopped it
+ * earlier.  Rows are tokens for tl_prefill / tl_extend and lanes for
+ * tl_decode_step.  Synchronises `stream`.
+ *   loops  host or device int32 [n] (written) */
+tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream);
+
 /* ------------------------------------------------------------------------
  * KV cache.  Every layer application keeps its own K/V slot: n_pre slots for
  * the pre-blocks and one per loop iteration ("Performance and Memory", "KV

@@ -210,3 +210,24 @@ def test_int3_chunk_dot_product_with_straddling_groups(G, seed):
     deq = np.array([float(np.float16(codes[0, k] * s[k // G])) for k in range(K)])
     want_total = float(deq @ x[:K])
     assert abs(got_total - want_total) <= 1e-9 * max(1.0, abs(want_total)), (got_total, want_total)
+
+
+def test_int3_word_slots_match_the_slot_table():
+    """The staging by packed word writes each of a word's ten codes where the
+    per-element slot table puts it (read from the kernel source)."""
+    src = SRC[SRC.index("void int3_word_slots("):]
+    src = src[:src.index("\n}\n")]
+    exprs = {}
+    for i in range(10):
+        m = re.search(r"pos\[%d\] = (.*);\s*// i = %d" % (i, i), src)
+        assert m, i
+        exprs[i] = m.group(1)
+    for c in range(3):
+        for t in range(4):
+            for q in range(4):
+                base = c * 160 + 2 * t
+                j0, j1, j8 = 16 * (2 * q), 16 * (2 * q + 1), 16 * (8 + (q >> 1))
+                for i in range(10):
+                    got = eval(exprs[i].replace("(q & 1)", str(q & 1)),
+                               {"base": base, "j0": j0, "j1": j1, "j8": j8})
+                    assert got == xpos(c * 160 + 40 * t + 10 * q + i, 3), (c, t, q, i)

@@ -36,7 +36,10 @@ def stage_keys(s, NSF, per, nkc):
     return lo, cnt, nkj, j
 
 
-def check(max_ctx, pos, F):
+def check(max_ctx, pos, F, mode=0):
+    """mode 0: the CTA holding key pos appends it (the decode step); mode 2:
+    every key, pos included, is copied from the cache (the attend pass after
+    an append pass)."""
     CL = cluster_size(max_ctx)
     n_keys = pos + 1
     per = (n_keys + CL - 1) // CL
@@ -48,7 +51,7 @@ def check(max_ctx, pos, F):
         kA = min(crank * F * per, n_keys)
         kB = min(kA + F * per, n_keys)
         nkc = kB - kA
-        owner = nkc > 0 and kB == n_keys
+        owner = mode != 2 and nkc > 0 and kB == n_keys
         n_old = nkc - 1 if owner else nkc
         NSF = (per + DS_KEYS - 1) // DS_KEYS
         nstage = nkc // per * NSF + (nkc % per + DS_KEYS - 1) // DS_KEYS
@@ -69,7 +72,7 @@ def check(max_ctx, pos, F):
                     assert key == pos
                     appends += 1
                 elif r < rem:                     # copied from the cache
-                    assert key < pos
+                    assert key < pos or (mode == 2 and key == pos)
                 else:                             # zero-filled (past the stage's keys)
                     assert r >= cnt
                 if r < cnt:
@@ -81,7 +84,7 @@ def check(max_ctx, pos, F):
                 ends.append(j)
         assert ends == [j for j in range(F) if min(per, nkc - j * per) > 0]
     assert reads == [1] * n_keys
-    assert appends == 1
+    assert appends == (1 if mode == 0 else 0)
 
 
 CTX = [1, 2, 16, 63, 64, 65, 100, 128, 200, 384, 511, 512, 513, 1056, 2048, 2112, 4096, 5000]
@@ -94,6 +97,7 @@ def test_stage_schedule_covers_each_key_once_for_every_F(max_ctx):
     for pos in sorted(p for p in positions if 0 <= p < max_ctx):
         for F in range(1, cluster_size(max_ctx) + 1):
             check(max_ctx, pos, F)
+            check(max_ctx, pos, F, mode=2)
 
 
 def test_chunk_count_follows_the_cache_size():
@@ -114,7 +118,8 @@ def test_model_follows_the_kernel_source():
         "const int c = (max_ctx + 63) / 64;",
         "const int per = (n_keys + CL - 1) / CL;",
         "const int kA = min(crank * F * per, n_keys), kB = min(kA + F * per, n_keys);",
-        "const bool owner = nkc > 0 && kB == n_keys;",
+        "const bool owner = a.mode != 2 && nkc > 0 && kB == n_keys;",
+        "const int pos = a.hdr->pos[lane_id] + a.row_off[row];",
         "const int n_old = owner ? nkc - 1 : nkc;",
         "const int NSF = (per + DS_KEYS - 1) / DS_KEYS;",
         "const int nstage = nkc / per * NSF + (nkc % per + DS_KEYS - 1) / DS_KEYS;",

@@ -70,6 +70,8 @@ _SIGS = {
     "tl_model_device_bytes": ([P, ctypes.POINTER(SZ)], I),
     "tl_model_set_graphs": ([P, I], I),
     "tl_model_set_decode_chunks": ([P, I], I),
+    "tl_model_set_exit_threshold": ([P, F], I),
+    "tl_loops_used": ([P, P, I, P], I),
     "tl_kv_layer_bytes": ([I, I, I, I, ctypes.POINTER(SZ)], I),
     "tl_kv_bytes": ([P, I, I, P, I, ctypes.POINTER(SZ)], I),
     "tl_kv_create": ([P, I, I, P, I, P, SZ, ctypes.POINTER(P)], I),
@@ -213,6 +215,16 @@ def tl_model_set_graphs(model: int, enable: bool) -> None:
 
 def tl_model_set_decode_chunks(model: int, chunks_per_cta: int) -> None:
     _check(lib.tl_model_set_decode_chunks(model, chunks_per_cta))
+
+
+def tl_model_set_exit_threshold(model: int, tau: float) -> None:
+    _check(lib.tl_model_set_exit_threshold(model, tau))
+
+
+def tl_loops_used(model: int, n: int, stream=None):
+    arr = (I * n)()
+    _check(lib.tl_loops_used(model, ctypes.cast(arr, P), n, _stream(stream)))
+    return list(arr)
 
 
 # --------------------------------------------------------------------- KV cache

@@ -97,6 +97,7 @@ struct tl_model {
   float eps;
   bool graphs = true;
   int decode_chunks = 0;   // context chunks per decode-attention CTA; 0 = automatic
+  float exit_tau = -1.f;   // per-iteration residual-norm check threshold; < 0 = off
   cudaStream_t cap_stream = nullptr;
   // workspace
   void* ws = nullptr;
@@ -114,6 +115,8 @@ struct tl_model {
   int32_t* ident_map;    // rows 0..7 -> 0..7 (extend, speculative steps)
   int32_t* spec_ids;     // speculative step: the input token and the drafts [16]
   int32_t* spec_ver;     // speculative step: the verify tokens [16]
+  int32_t* exit_it;      // per row: 0 while it runs, else the loop iterations it ran
+  int32_t* loops;        // per output row: loop iterations run by the last forward
   float* head_ps;        // greedy head partials [head_parts()][8]
   int* head_pv;
   int* status;
@@ -325,7 +328,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   };
   void* p_ids; void* p_hin; void* p_h; void* p_x; void* p_attn; void* p_q; void* p_k; void* p_v;
   void* p_u; void* p_part; void* p_y; void* p_lid; void* p_status; void* p_rope;
-  void* p_ident; void* p_sids; void* p_sver; void* p_hps; void* p_hpv;
+  void* p_ident; void* p_sids; void* p_sver; void* p_hps; void* p_hpv; void* p_exit; void* p_loops;
   Slot slots[] = {
       {&p_ids, (size_t)T * 4},
       {&p_hin, (size_t)T * d * 2},
@@ -340,6 +343,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
       {&p_y, (size_t)T * d * 4},
       {&p_lid, (size_t)kMaxLanes * 4},
       {&p_ident, (size_t)kMaxLanes * 4},
+      {&p_exit, (size_t)std::max(T, kMaxLanes) * 4},
+      {&p_loops, (size_t)std::max(T, kMaxLanes) * 4},
       {&p_sids, 16 * 4},
       {&p_sver, 16 * 4},
       {&p_hps, (size_t)head_parts() * 8 * 4},
@@ -370,6 +375,8 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
   m->y = (float*)p_y;
   m->lane_map = (int32_t*)p_lid;
   m->ident_map = (int32_t*)p_ident;
+  m->exit_it = (int32_t*)p_exit;
+  m->loops = (int32_t*)p_loops;
   m->spec_ids = (int32_t*)p_sids;
   m->spec_ver = (int32_t*)p_sver;
   m->head_ps = (float*)p_hps;
@@ -394,6 +401,7 @@ TL_API tl_status tl_model_create(const tl_model_desc* desc, tl_model** out) {
     if (e2 == cudaSuccess)
       e2 = cudaMemcpy(m->ident_map, ident, sizeof(ident), cudaMemcpyHostToDevice);
     cudaError_t e3 = cudaMemset(m->status, 0, 256);
+    if (e3 == cudaSuccess) e3 = cudaMemset(m->exit_it, 0, (size_t)std::max(T, kMaxLanes) * 4);
     if (e1 != cudaSuccess || e2 != cudaSuccess || e3 != cudaSuccess) {
       cudaFree(m->ws);
       return set_error(TL_ERR_CUDA, "model initialisation copy failed");
@@ -426,6 +434,23 @@ TL_API tl_status tl_model_set_graphs(tl_model* model, int enable) {
   TL_CHECK_ARG(model, "NULL model");
   model->graphs = enable != 0;
   if (!model->graphs) free_graphs(model);
+  return ok();
+}
+
+TL_API tl_status tl_model_set_exit_threshold(tl_model* model, float tau) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG(!std::isnan(tau) && tau != INFINITY, "tau must be a finite threshold or negative");
+  model->exit_tau = tau < 0.f ? -1.f : tau;
+  free_graphs(model);   // captured graphs hold the old threshold
+  return ok();
+}
+
+TL_API tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream) {
+  TL_CHECK_ARG(model && loops, "NULL argument");
+  TL_CHECK_ARG(n >= 1 && n <= std::max(model->Tmax, kMaxLanes), "n = %d out of range", n);
+  TL_CUDA(cudaMemcpyAsync(loops, model->loops, (size_t)n * 4, cudaMemcpyDefault,
+                          (cudaStream_t)stream));
+  TL_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
   return ok();
 }
 
@@ -632,6 +657,20 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
   return a;
 }
 
+// The residual-norm check for a kernel of layer `layer`: `check_iter` > 0
+// records rows above the threshold as having run check_iter iterations; loop
+// layers skip the residual updates of rows already stopped.
+ExitArgs exit_args(const tl_model* m, int layer, int check_iter) {
+  ExitArgs e;
+  memset(&e, 0, sizeof(e));
+  e.tau = m->exit_tau;
+  if (m->exit_tau < 0.f) return e;
+  e.exit_it = m->exit_it;
+  e.check_iter = check_iter;
+  e.skip = layer >= (int)m->pre.size() ? 1 : 0;
+  return e;
+}
+
 NormArgs norm_args(const tl_model* m, int rows) {
   NormArgs n;
   memset(&n, 0, sizeof(n));
@@ -688,6 +727,7 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   n.n_add = rows;
   n.gamma_next = b->d.gamma_ffn;
   n.n_next = rows;
+  n.ex = exit_args(m, layer, 0);
   TL_TRY(launch_residual_norm(n, s));
   // SwiGLU MLP
   g = gemm_args(m, b, 2, m->x, rows);
@@ -719,6 +759,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   p.bits = bd.bits;
   p.T = rows;
   p.eps = m->eps;
+  p.status = m->status;
   // QKV: q, k, v sums -> part [1][rows][3d]
   p.w0 = bd.w_qkv;
   p.s0 = (const __half*)bd.s_qkv;
@@ -728,7 +769,13 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   p.gamma = bd.gamma_attn;
   p.epi = DEC_EPI_OUT;
   p.out = m->part;
+  {
+    const int it = layer - (int)m->pre.size();   // the loop iteration this layer runs
+    p.ex = exit_args(m, layer, it >= 1 ? it : 0);
+    p.ex.skip = 0;
+  }
   TL_TRY(launch_dec_gemv(p, s));
+  p.ex = exit_args(m, layer, 0);
   // RoPE, KV append, split attention and merge in one launch
   DecodeAttnArgs da;
   memset(&da, 0, sizeof(da));
@@ -822,6 +869,7 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
   e.rows = seq;
   e.h = m->h;
   e.status = m->status;
+  e.exit_it = m->exit_it;
   TL_TRY(launch_embed(e, s));
   NormArgs n = norm_args(m, seq);
   n.gamma_next = block_at(m, 0)->d.gamma_attn;
@@ -835,6 +883,11 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
     en.part_rows = seq;
     en.S = gemm_splits(m->d, m->F, seq, b->d.bits);
     en.n_add = seq;
+    {
+      // the stream leaving this layer enters loop iteration it + 1
+      const int it = layer - (int)m->pre.size();
+      en.ex = exit_args(m, layer, it >= 0 && layer + 1 < n_layers ? it + 1 : 0);
+    }
     if (layer + 1 < n_layers) {
       en.gamma_next = block_at(m, layer + 1)->d.gamma_attn;
       en.n_next = seq;
@@ -842,6 +895,8 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
       en.gamma_final = m->desc.gamma_final;
       en.fin_lo = 0;
       en.fin_hi = seq;
+      en.loops_out = m->loops;
+      en.L_all = L;
     }
     if (trace) en.trace = trace + (size_t)layer * seq * m->d;
     TL_TRY(launch_residual_norm(en, s));
@@ -875,6 +930,7 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
   e.src_row = lane_of_row;
   e.h = m->h;
   e.status = m->status;
+  e.exit_it = m->exit_it;
   TL_TRY(launch_embed(e, s));
   for (int layer = 0; layer < n_layers; ++layer) {
     const int act = active(layer);
@@ -888,6 +944,9 @@ tl_status enqueue_decode(tl_model* m, tl_kv* kv, bool use_ids, int B, const int*
   fin.fin_lo = 0;
   fin.fin_hi = B;
   fin.out_row = lane_of_row;
+  fin.loops_out = m->loops;
+  fin.ex.exit_it = m->exit_tau >= 0.f ? m->exit_it : nullptr;
+  for (int i = 0; i < kMaxLanes; ++i) fin.L_row[i] = i < B ? L_sorted[i] : 0;
   TL_TRY(launch_residual_norm(fin, s));
   TL_TRY(launch_advance_pos((KvHeader*)kv->buffer, B, s));
   return ok();
@@ -917,6 +976,7 @@ tl_status enqueue_extend(tl_model* m, tl_kv* kv, int lane, bool use_ids, int n, 
   e.rows = n;
   e.h = m->h;
   e.status = m->status;
+  e.exit_it = m->exit_it;
   TL_TRY(launch_embed(e, s));
   const int n_layers = (int)m->pre.size() + L;
   for (int layer = 0; layer < n_layers; ++layer)
@@ -926,6 +986,9 @@ tl_status enqueue_extend(tl_model* m, tl_kv* kv, int lane, bool use_ids, int n, 
   fin.gamma_final = m->desc.gamma_final;
   fin.fin_lo = 0;
   fin.fin_hi = n;
+  fin.loops_out = m->loops;
+  fin.ex.exit_it = m->exit_tau >= 0.f ? m->exit_it : nullptr;
+  fin.L_all = L;
   TL_TRY(launch_residual_norm(fin, s));
   TL_TRY(launch_add_pos((KvHeader*)kv->buffer, lane, n, s));
   return ok();

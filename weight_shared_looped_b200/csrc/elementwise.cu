@@ -31,6 +31,7 @@ __device__ __forceinline__ void set_status(int* status, int code) {
 __global__ void embed_kernel(EmbedArgs a) {
   pdl_enter();
   const int row = blockIdx.x;
+  if (a.exit_it && threadIdx.x == 0) a.exit_it[row] = 0;
   const int src = a.src_row ? a.src_row[row] : row;
   float* h = a.h + (size_t)row * a.d;
   const __half* e;
@@ -95,7 +96,8 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
   float* h = a.h + (size_t)row * a.d;
   float4 v0 = *reinterpret_cast<const float4*>(h + c0);
   float4 v1 = *reinterpret_cast<const float4*>(h + c1);
-  if (row < a.n_add && a.S > 0) {
+  const bool frozen = a.ex.skip && a.ex.exit_it[row] != 0;   // stopped by the residual-norm check
+  if (row < a.n_add && a.S > 0 && !frozen) {
     const size_t sstride = (size_t)a.part_rows * a.d;
     const float* p0 = a.part + (size_t)row * a.d;
     for (int sp = 0; sp < a.S; sp += SP) {
@@ -140,6 +142,14 @@ __global__ void __launch_bounds__(MAXT) residual_norm_kernel(NormArgs a) {
   float tot = 0.0f;
   for (int w = 0; w < nw; ++w) tot += red[w];
   const float r = rsqrtf(tot / (float)a.d + a.eps);
+  // the residual-norm check on the stream entering the next loop iteration
+  if (a.ex.check_iter > 0 && threadIdx.x == 0 && row < a.n_next && a.ex.exit_it[row] == 0 &&
+      sqrtf(tot) > a.ex.tau)
+    a.ex.exit_it[row] = a.ex.check_iter;
+  if (a.loops_out && want_y && threadIdx.x == 0) {
+    const int e = a.ex.exit_it ? a.ex.exit_it[row] : 0;
+    a.loops_out[out_row] = e != 0 ? e : a.L_all > 0 ? a.L_all : a.L_row[row];
+  }
   auto out_x = [&](int c, const float4 v, const float4 g) {
     const __half2 lo = __halves2half2(__float2half_rn(v.x * r * g.x), __float2half_rn(v.y * r * g.y));
     const __half2 hi = __halves2half2(__float2half_rn(v.z * r * g.z), __float2half_rn(v.w * r * g.w));

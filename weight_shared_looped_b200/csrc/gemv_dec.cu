@@ -43,6 +43,9 @@
 //             u = fp16(silu(gate) * up).
 // Weights, scales and gains are constants of the model: they are requested
 // before the wait for the previous kernel, so their latency overlaps its tail.
+#include <algorithm>
+#include <cstring>
+
 #include "tl_launch.cuh"
 
 namespace tl {
@@ -50,7 +53,6 @@ namespace {
 
 constexpr int DG_THREADS = 256;
 constexpr int DG_WARPS = 8;
-constexpr int DG_MAXC = 8;          // most chunks whose words one lane holds in flight
 
 enum { EPI_OUT = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
 
@@ -144,6 +146,24 @@ __device__ __forceinline__ int int3_slot(int L, int t, int& j) {
   }
 }
 
+// INT3 staging by packed word: the ten codes L = 10q + i (i = 0..9) of the
+// word of lane t, word q of chunk c go to these positions of the staged row
+// (the slot table of int3_slot, unrolled with i known at compile time).
+__device__ __forceinline__ void int3_word_slots(int c, int t, int q, int* pos) {
+  const int base = c * 160 + 2 * t;
+  const int j0 = 16 * (2 * q), j1 = 16 * (2 * q + 1), j8 = 16 * (8 + (q >> 1));
+  pos[0] = base + j0;                 // i = 0
+  pos[1] = base + j0 + 8;             // i = 1
+  pos[2] = base + j1;                 // i = 2
+  pos[3] = base + j1 + 8;             // i = 3
+  pos[4] = base + j8 + (q & 1);       // i = 4
+  pos[5] = base + j8 + 8 + (q & 1);   // i = 5
+  pos[6] = base + j0 + 1;             // i = 6
+  pos[7] = base + j0 + 9;             // i = 7
+  pos[8] = base + j1 + 1;             // i = 8
+  pos[9] = base + j1 + 9;             // i = 9
+}
+
 template <int BITS>
 __device__ __forceinline__ int xpos(int k) {
   if (BITS == 4) {
@@ -160,12 +180,15 @@ __device__ __forceinline__ int xpos(int k) {
 }
 
 struct DgArgs {
-  const uint32_t* w0;   // canonical packed rows: tile m of CTA b is rows (b*MT + m)*16 ..
-  const __half* s0;     //   (EPI_SWIGLU: w0 = gate, w1 = up, both rows b*16 ..)
+  const uint32_t* w0;   // canonical packed rows; unit u is rows u*16 .. u*16+15
+  const __half* s0;     //   (EPI_SWIGLU: w0 = gate, w1 = up, both rows u*16 ..)
   const uint32_t* w1;
   const __half* s1;
   int N, K, G, wpr;     // output rows (per matrix), K, group, packed words per row
   int T;                // active token rows (1..8)
+  int n_units;          // N / 16
+  int stages;           // weight stages in shared memory
+  int row_stride;       // bytes per staged row (row bytes padded to 64 mod 128)
   const __half* x;      // fp16 [T][K] activations (when !NORM)
   const float* h;       // fp32 [T][K] residual stream (NORM)
   const float* gamma;   // fp32 [K] (NORM)
@@ -176,88 +199,194 @@ struct DgArgs {
   float* trace;         // EPI_RESID, optional: fp32 [trace_rows][N] rows indexed by out_row
   const int32_t* out_row;
   int trace_rows;       // rows T .. trace_rows-1 are copied from hres unchanged
+  int* status;          // a bounded wait that runs out records TL_ERR_TIMEOUT here
+  ExitArgs ex;          // the per-iteration residual-norm check
 };
 
-// MC: chunks a lane holds in flight (its k range takes ceil(chunks / (8 / MT))
-// of them; larger ranges run in batches of MC)
-template <int BITS, int MT, bool NORM, int EPI, int MC>
-__global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(DgArgs a) {
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ uint64_t dg_globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for an mbarrier phase: false once 2 s of global time have passed.
+__device__ __forceinline__ bool dg_wait(uint32_t bar, uint32_t parity) {
+  uint64_t start = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (i == 0) start = dg_globaltimer();
+    else if ((i & 63) == 0 && dg_globaltimer() - start > 2000000000ull) return false;
+  }
+}
+
+// The weights (and scales) of one unit into its stage: lane r of the calling
+// warp copies row r of the unit (one bulk copy per row, so that staged rows
+// sit 64 bytes off the 128-byte bank period), the scales one copy per tile.
+template <int MT>
+__device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigned char* stage,
+                                              uint32_t bar, int lane) {
+  const int rows = 16 * MT;
+  const uint32_t row_bytes = (uint32_t)a.wpr * 4;
+  const int gpr = a.K / a.G;
+  const uint32_t sc_bytes = 16u * gpr * 2;
+  if (lane == 0) {
+    const uint32_t total = rows * row_bytes + MT * sc_bytes;
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(total)
+                 : "memory");
+  }
+  __syncwarp();
+  const int r0 = unit * 16;
+  if (lane < rows) {
+    const int m = lane >> 4, r = lane & 15;
+    const uint32_t* src = (m == 0 ? a.w0 : a.w1) + (size_t)(r0 + r) * a.wpr;
+    const uint32_t dst = smem_u32(stage + (size_t)lane * a.row_stride);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(row_bytes), "r"(bar)
+        : "memory");
+  }
+  if (lane < MT) {
+    const __half* src = (lane == 0 ? a.s0 : a.s1) + (size_t)r0 * gpr;
+    const uint32_t dst = smem_u32(stage + (size_t)rows * a.row_stride + (size_t)lane * sc_bytes);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(src), "r"(sc_bytes), "r"(bar)
+        : "memory");
+  }
+}
+
+// One CTA per SM (at most): CTA c takes units c, c + gridDim.x, ...; a unit is
+// 16 weight rows (EPI_SWIGLU: 16 gate rows and the same 16 up rows).  The
+// units' packed words and scales stream through a ring of `stages` shared-
+// memory stages filled by bulk copies; the first stages are requested before
+// the wait for the previous kernel (weights are constants of the model), and
+// the CTA leaves room on its SM for the next kernel's CTA to do the same.
+// UM > 0: every unit of the CTA (at most UM) is resident at once, copied in
+// before the dependency wait; the warps compute them back to back into
+// per-unit sums and one reduction and one epilogue close the launch.  UM == 0:
+// the units stream through a ring of a.stages stages, one reduction per unit.
+template <int BITS, int MT, bool NORM, int EPI, int UM>
+__global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   using Fm = DgFmt<BITS>;
   constexpr int CW = Fm::CW;
   constexpr int W = DG_WARPS / MT;                 // warps (k ranges) per tile
-  extern __shared__ __align__(16) unsigned char dg_smem[];
+  extern __shared__ __align__(128) unsigned char dg_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
   const int m = warp / W, ks = warp - m * W;
   const int nvec = a.wpr >> 2;                     // 16-byte vectors per packed row
   const int nch = (nvec + 3) >> 2;                 // chunks per row
   const int c_lo = ks * nch / W, c_hi = (ks + 1) * nch / W;
-  const int xw = nch * CW + 8;                     // staged row, halves (stride/16 odd)
-  __half* xs = reinterpret_cast<__half*>(dg_smem);                         // [T][xw]
-  float* red = reinterpret_cast<float*>(dg_smem + (size_t)a.T * xw * 2);  // [MT][W][16][8]
-  __shared__ __align__(16) uint32_t zero16[4];
-  __shared__ float nred[8][DG_WARPS];
+  const int xw = nch * CW + 8;                     // staged activation row, halves
   const int gsh = __ffs(a.G) - 1;
   const int gpr = a.K >> gsh;
   const bool g64 = BITS == 4 && a.G == 64;
+  const size_t stage_bytes = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2;
+  unsigned char* stages = dg_smem;
+  __half* xs = reinterpret_cast<__half*>(dg_smem + (size_t)a.stages * stage_bytes);   // [T][xw]
+  float* red = reinterpret_cast<float*>(xs + (size_t)a.T * xw);      // [max(2, UM)][MT][W][16][8]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(red + (UM > 2 ? UM : 2) * DG_WARPS * 16 * 8);
+  __shared__ __align__(16) uint32_t zero16[4];
+  __shared__ float nred[8][DG_WARPS];
+  __shared__ int abort_flag;
+  const int n_my = (a.n_units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
 
-  // this tile's rows g and g + 8
-  int row0;
-  const uint32_t* wm;
-  const __half* sm;
-  if (EPI == EPI_SWIGLU) {
-    row0 = blockIdx.x * 16;
-    wm = m == 0 ? a.w0 : a.w1;
-    sm = m == 0 ? a.s0 : a.s1;
-  } else {
-    row0 = (blockIdx.x * MT + m) * 16;
-    wm = a.w0;
-    sm = a.s0;
+  if (tid == 0) {
+    for (int i = 0; i < a.stages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bars + i)));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    zero16[0] = zero16[1] = zero16[2] = zero16[3] = 0u;
+    abort_flag = 0;
   }
-  const uint4* wr0 = reinterpret_cast<const uint4*>(wm + (size_t)(row0 + g) * a.wpr);
-  const uint4* wr1 = reinterpret_cast<const uint4*>(wm + (size_t)(row0 + g + 8) * a.wpr);
-  const __half* sr0 = sm + (size_t)(row0 + g) * gpr;
-  const __half* sr1 = sm + (size_t)(row0 + g + 8) * gpr;
-
-  // ---- constants first: this lane's packed words and scales of its first chunks
-  // sv[i]: rows g, g + 8 of the first scale group ([0], [1]) and of the second
-  // ([2], [3]): INT4 G = 128 one group per chunk; INT4 G = 64 the chunk's two
-  // groups; INT3 the group of the lane's first code and the next one
-  uint4 wv[MC][2];
-  __half sv[MC][4];
-  auto fetch = [&](int cb) {
+  __syncthreads();
+  // the first units' weights: requested before the dependency wait
+  int issued = min(a.stages, n_my);   // units whose copies were issued (the same in every thread)
+  int stop = n_my;                    // the unit a timed-out wait stopped at
+  if (warp == 0)
+    for (int j = 0; j < a.stages && j < n_my; ++j)
+      dg_issue_unit<MT>(a, blockIdx.x + j * gridDim.x, stages + (size_t)j * stage_bytes,
+                        smem_u32(bars + j), lane);
+  // the gains are constants of the model: requested before the dependency
+  // wait (rows of d <= 2048 take two float4 per thread)
+  constexpr int NV = 2;
+  float4 gpre[NV];
+  const bool small_k = a.K <= 4 * DG_THREADS * NV;
+  if (NORM && BITS == 4 && small_k) {
 #pragma unroll
-    for (int i = 0; i < MC; ++i) {
-      const int c = cb + i;
-      const int vi = 4 * c + t;
-      const bool in = c < c_hi && vi < nvec;
-      wv[i][0] = in ? __ldg(wr0 + vi) : make_uint4(0u, 0u, 0u, 0u);
-      wv[i][1] = in ? __ldg(wr1 + vi) : make_uint4(0u, 0u, 0u, 0u);
-      if (c < c_hi) {
-        int ga, gb;
-        if (BITS == 4) {
-          ga = g64 ? 2 * c : c;
-          gb = ga + 1;
-        } else {
-          ga = min((c * CW + 40 * t) >> gsh, gpr - 1);
-          gb = min(ga + 1, gpr - 1);
-        }
-        sv[i][0] = __ldg(sr0 + ga);
-        sv[i][1] = __ldg(sr1 + ga);
-        if (BITS == 3 || g64) {
-          sv[i][2] = __ldg(sr0 + gb);
-          sv[i][3] = __ldg(sr1 + gb);
-        }
-      }
+    for (int i = 0; i < NV; ++i) {
+      const int k = 4 * tid + 4 * DG_THREADS * i;
+      gpre[i] = k < a.K ? __ldg(reinterpret_cast<const float4*>(a.gamma + k))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-  };
-  fetch(c_lo);
-  if (tid == 0) zero16[0] = zero16[1] = zero16[2] = zero16[3] = 0u;
+  }
   pdl_enter();   // activations and the residual stream come from the previous kernels
 
   // ---- stage the activations (permuted) into xs; padding codes see zeros
   const int kpad = nch * CW;
-  if (NORM) {
+  if (NORM && BITS == 4 && small_k && a.T <= 2) {
+    // one pass: the (at most two) rows stay in registers between the sum of
+    // squares and the scaling; same arithmetic and order as the general path
+    float4 hv[2][NV];
+#pragma unroll
+    for (int b = 0; b < 2; ++b)
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        const int k = 4 * tid + 4 * DG_THREADS * i;
+        hv[b][i] = b < a.T && k < a.K ? *reinterpret_cast<const float4*>(a.h + (size_t)b * a.K + k)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (b < a.T) {
+        float ss = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          ss = fmaf(hv[b][i].x, hv[b][i].x, ss);
+          ss = fmaf(hv[b][i].y, hv[b][i].y, ss);
+          ss = fmaf(hv[b][i].z, hv[b][i].z, ss);
+          ss = fmaf(hv[b][i].w, hv[b][i].w, ss);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        if (lane == 0) nred[b][warp] = ss;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      if (b < a.T) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < DG_WARPS; ++w) tot += nred[b][w];
+        if (a.ex.check_iter > 0 && blockIdx.x == 0 && tid == 0 && a.ex.exit_it[b] == 0 &&
+            sqrtf(tot) > a.ex.tau)
+          a.ex.exit_it[b] = a.ex.check_iter;
+        const float r = rsqrtf(tot / (float)a.K + a.eps);
+        __half* xr = xs + (size_t)b * xw;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          const int k = 4 * tid + 4 * DG_THREADS * i;
+          if (k < a.K) {
+            const float4 v = hv[b][i], gm = gpre[i];
+            xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
+            xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
+            xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
+            xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+          }
+        }
+        for (int k = a.K + tid; k < kpad; k += DG_THREADS) xr[xpos<BITS>(k)] = __float2half_rn(0.f);
+      }
+    }
+  } else if (NORM) {
     // x = fp16(h * rsqrt(mean(h^2) + eps) * gamma) per token row, the sum of
     // squares in a fixed order (per thread, xor tree, warps in order)
     for (int b = 0; b < a.T; ++b) {
@@ -279,18 +408,35 @@ __global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(D
       float tot = 0.f;
 #pragma unroll
       for (int w = 0; w < DG_WARPS; ++w) tot += nred[b][w];
+      // the residual-norm check on the stream entering this loop iteration
+      // (every CTA computes the same sum; CTA 0 records the decision)
+      if (a.ex.check_iter > 0 && blockIdx.x == 0 && tid == 0 && a.ex.exit_it[b] == 0 &&
+          sqrtf(tot) > a.ex.tau)
+        a.ex.exit_it[b] = a.ex.check_iter;
       const float r = rsqrtf(tot / (float)a.K + a.eps);
       const float* hr = a.h + (size_t)b * a.K;
       __half* xr = xs + (size_t)b * xw;
-      for (int k = 4 * tid; k < a.K; k += 4 * DG_THREADS) {
-        const float4 v = *reinterpret_cast<const float4*>(hr + k);
-        const float4 gm = __ldg(reinterpret_cast<const float4*>(a.gamma + k));
-        xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
-        xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
-        xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
-        xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+      if (BITS == 4) {
+        for (int k = 4 * tid; k < a.K; k += 4 * DG_THREADS) {
+          const float4 v = *reinterpret_cast<const float4*>(hr + k);
+          const float4 gm = __ldg(reinterpret_cast<const float4*>(a.gamma + k));
+          xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
+          xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
+          xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
+          xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+        }
+      } else {
+        for (int wd = tid; wd < nch * 16; wd += DG_THREADS) {
+          const int c = wd >> 4, t = (wd >> 2) & 3, q = wd & 3;
+          const int k0 = c * 160 + 40 * t + 10 * q;
+          int pos[10];
+          int3_word_slots(c, t, q, pos);
+#pragma unroll
+          for (int i = 0; i < 10; ++i)
+            xr[pos[i]] = k0 + i < a.K ? __float2half_rn(hr[k0 + i] * r * __ldg(a.gamma + k0 + i))
+                                      : __float2half_rn(0.f);
+        }
       }
-      for (int k = a.K + tid; k < kpad; k += DG_THREADS) xr[xpos<BITS>(k)] = __float2half_rn(0.f);
     }
   } else {
     for (int b = 0; b < a.T; ++b) {
@@ -308,32 +454,48 @@ __global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(D
           *reinterpret_cast<__half2*>(xr + base + 24) = __halves2half2(e[3], e[7]);
         }
       } else {
-        for (int k = tid; k < kpad; k += DG_THREADS)
-          xr[xpos<BITS>(k)] = k < a.K ? src[k] : __float2half_rn(0.f);
+        // one packed word (ten codes, ten consecutive k) per thread and step
+        for (int wd = tid; wd < nch * 16; wd += DG_THREADS) {
+          const int c = wd >> 4, t = (wd >> 2) & 3, q = wd & 3;
+          const int k0 = c * 160 + 40 * t + 10 * q;
+          int pos[10];
+          int3_word_slots(c, t, q, pos);
+#pragma unroll
+          for (int i = 0; i < 10; ++i)
+            xr[pos[i]] = k0 + i < a.K ? src[k0 + i] : __float2half_rn(0.f);
+        }
       }
     }
   }
   __syncthreads();
 
-  // ---- the MMAs: this warp's chunks of its tile
   // ldmatrix rows: lane l supplies token row l & 7 (a zero block for rows >= T)
   const int lr = lane & 7, lq = lane >> 3;
-  const uint32_t zaddr = (uint32_t)__cvta_generic_to_shared(zero16);
+  const uint32_t zaddr = smem_u32(zero16);
   const bool lrow_ok = lr < a.T;
-  const uint32_t lbase =
-      lrow_ok ? (uint32_t)__cvta_generic_to_shared(xs + (size_t)lr * xw + 8 * lq) : zaddr;
+  const uint32_t lbase = lrow_ok ? smem_u32(xs + (size_t)lr * xw + 8 * lq) : zaddr;
   const uint32_t lmul = lrow_ok ? 2u : 0u;   // bytes per staged element (0: stay on the zero block)
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int cb = c_lo; cb < c_hi; cb += MC) {
-    if (cb != c_lo) fetch(cb);
-#pragma unroll
-    for (int i = 0; i < MC; ++i) {
-      const int c = cb + i;
-      if (c >= c_hi) break;
-      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&wv[i][0]);   // row g
-      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&wv[i][1]);   // row g + 8
+
+  // this warp's chunks of its tile of the unit in `stage`, added into acc
+  auto unit_mma = [&](const unsigned char* stage, float* acc) {
+    // ---- the MMAs: this warp's chunks of its tile, words and scales from the stage
+    const unsigned char* wt0 = stage + (size_t)(16 * m + g) * a.row_stride;
+    const unsigned char* wt1 = wt0 + (size_t)8 * a.row_stride;
+    const __half* st0 = reinterpret_cast<const __half*>(stage + (size_t)16 * MT * a.row_stride +
+                                                        (size_t)m * 16 * gpr * 2) + (size_t)g * gpr;
+    const __half* st1 = st0 + (size_t)8 * gpr;
+    for (int c = c_lo; c < c_hi; ++c) {
+      const int vi = 4 * c + t;
+      uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+      if (vi < nvec) {
+        v0 = *reinterpret_cast<const uint4*>(wt0 + (size_t)vi * 16);
+        v1 = *reinterpret_cast<const uint4*>(wt1 + (size_t)vi * 16);
+      }
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&v0);   // row g
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&v1);   // row g + 8
       const uint32_t xb = lbase + lmul * (uint32_t)(c * CW);
       if (BITS == 4) {
+        const int ga = g64 ? 2 * c : c;
         float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb2[4] = {0.f, 0.f, 0.f, 0.f};
         const bool first = t < 2;   // G = 64: this lane's codes are in the chunk's first group
 #pragma unroll
@@ -356,13 +518,13 @@ __global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(D
             mma16816(cb2, first ? z : A1, b[2], b[3]);
           }
         }
-        const float f0 = __half2float(sv[i][0]), f1 = __half2float(sv[i][1]);
+        const float f0 = __half2float(st0[ga]), f1 = __half2float(st1[ga]);
         acc[0] = fmaf(ca[0], f0, acc[0]);
         acc[1] = fmaf(ca[1], f0, acc[1]);
         acc[2] = fmaf(ca[2], f1, acc[2]);
         acc[3] = fmaf(ca[3], f1, acc[3]);
         if (g64) {
-          const float e0 = __half2float(sv[i][2]), e1 = __half2float(sv[i][3]);
+          const float e0 = __half2float(st0[ga + 1]), e1 = __half2float(st1[ga + 1]);
           acc[0] = fmaf(cb2[0], e0, acc[0]);
           acc[1] = fmaf(cb2[1], e0, acc[1]);
           acc[2] = fmaf(cb2[2], e1, acc[2]);
@@ -373,12 +535,14 @@ __global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(D
         // group; bnd is a multiple of 8 (chunk, lane and group starts all
         // are), so each octet of codes L = 8o .. 8o + 7 has one scale
         const int k0 = c * CW + 40 * t;
+        const int ga = min(k0 >> gsh, gpr - 1), gb = min(ga + 1, gpr - 1);
         const int bnd = (((k0 >> gsh) + 1) << gsh) - k0;
+        const __half sa0 = st0[ga], sb0 = st0[gb], sa1 = st1[ga], sb1 = st1[gb];
         __half so0[5], so1[5];
 #pragma unroll
         for (int oc = 0; oc < 5; ++oc) {
-          so0[oc] = 8 * oc < bnd ? sv[i][0] : sv[i][2];
-          so1[oc] = 8 * oc < bnd ? sv[i][1] : sv[i][3];
+          so0[oc] = 8 * oc < bnd ? sa0 : sb0;
+          so1[oc] = 8 * oc < bnd ? sa1 : sb1;
         }
 #define TL_SC(p, La, Lb, so) hmul2_bits((p), h2bits(__halves2half2(so[(La) >> 3], so[(Lb) >> 3])))
 #pragma unroll
@@ -414,77 +578,181 @@ __global__ void __launch_bounds__(DG_THREADS, MC <= 4 ? 2 : 1) gemv_dec_kernel(D
 #undef TL_SC
       }
     }
-  }
 
-  // ---- the warps' sums, added in warp order
-  float* rw = red + ((size_t)(m * W + ks) * 16) * 8;      // [16 rows][8 tokens]
-  rw[g * 8 + 2 * t] = acc[0];
-  rw[g * 8 + 2 * t + 1] = acc[1];
-  rw[(g + 8) * 8 + 2 * t] = acc[2];
-  rw[(g + 8) * 8 + 2 * t + 1] = acc[3];
-  __syncthreads();
-  if (EPI == EPI_SWIGLU) {
-    if (tid < 16 * 8) {
-      const int r = tid >> 3, b = tid & 7;
-      if (b < a.T) {
-        float gs = 0.f, us = 0.f;
+  };
+  // the unit's outputs from the warps' sums in redj (threads tid < 128)
+  auto unit_epilogue = [&](int unit, const float* redj) {
+    if (EPI == EPI_SWIGLU) {
+      if (tid < 16 * 8) {
+        const int r = tid >> 3, b = tid & 7;
+        if (b < a.T) {
+          float gs = 0.f, us = 0.f;
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-          gs += red[((0 * W + w) * 16 + r) * 8 + b];
-          us += red[((1 * W + w) * 16 + r) * 8 + b];
+          for (int w = 0; w < W; ++w) {
+            gs += redj[((0 * W + w) * 16 + r) * 8 + b];
+            us += redj[((1 * W + w) * 16 + r) * 8 + b];
+          }
+          const float silu = gs / (1.0f + __expf(-gs));
+          a.u[(size_t)b * a.N + unit * 16 + r] = __float2half_rn(silu * us);
         }
-        const float silu = gs / (1.0f + __expf(-gs));
-        a.u[(size_t)b * a.N + row0 + r] = __float2half_rn(silu * us);
       }
+    } else {
+      if (tid < 16 * 8) {
+        const int r = tid >> 3, b = tid & 7;
+        const int n = unit * 16 + r;
+        float y = 0.f;
+#pragma unroll
+        for (int w = 0; w < W; ++w) y += redj[(w * 16 + r) * 8 + b];
+        if (EPI == EPI_OUT) {
+          if (b < a.T) a.out[(size_t)b * a.N + n] = y;
+        } else {
+          if (b < a.T) {
+            float* hp = a.hres + (size_t)b * a.N + n;
+            const bool frozen = a.ex.skip && a.ex.exit_it[b] != 0;   // stopped by the check
+            const float hn = frozen ? *hp : *hp + y;
+            *hp = hn;
+            if (a.trace) a.trace[(size_t)a.out_row[b] * a.N + n] = hn;
+          } else if (a.trace && b < a.trace_rows) {
+            // lanes that ran fewer iterations keep their last value in the trace
+            a.trace[(size_t)a.out_row[b] * a.N + n] = a.hres[(size_t)b * a.N + n];
+          }
+        }
+      }
+    }
+  };
+  if (UM > 0) {
+    // every unit resident: back to back, then one reduction
+    float acc[UM > 0 ? UM : 1][4];
+#pragma unroll
+    for (int u = 0; u < (UM > 0 ? UM : 1); ++u) {
+      acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+      if (u < n_my) {
+        if (!dg_wait(smem_u32(bars + u), 0u)) abort_flag = 1;
+        unit_mma(stages + (size_t)u * stage_bytes, acc[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < (UM > 0 ? UM : 1); ++u) {
+      if (u < n_my) {
+        float* rw = red + ((size_t)u * DG_WARPS + m * W + ks) * 16 * 8;
+        rw[g * 8 + 2 * t] = acc[u][0];
+        rw[g * 8 + 2 * t + 1] = acc[u][1];
+        rw[(g + 8) * 8 + 2 * t] = acc[u][2];
+        rw[(g + 8) * 8 + 2 * t + 1] = acc[u][3];
+      }
+    }
+    __syncthreads();
+    if (abort_flag) {
+      stop = 0;
+    } else {
+      for (int u = 0; u < n_my; ++u)
+        unit_epilogue(blockIdx.x + u * gridDim.x, red + (size_t)u * DG_WARPS * 16 * 8);
     }
   } else {
-    for (int i = tid; i < MT * 16 * 8; i += DG_THREADS) {
-      const int mm = i >> 7, r = (i >> 3) & 15, b = i & 7;
-      const int n = (blockIdx.x * MT + mm) * 16 + r;
-      float y = 0.f;
-#pragma unroll
-      for (int w = 0; w < W; ++w) y += red[((mm * W + w) * 16 + r) * 8 + b];
-      if (EPI == EPI_OUT) {
-        if (b < a.T) a.out[(size_t)b * a.N + n] = y;
-      } else {
-        if (b < a.T) {
-          float* hp = a.hres + (size_t)b * a.N + n;
-          const float hn = *hp + y;
-          *hp = hn;
-          if (a.trace) a.trace[(size_t)a.out_row[b] * a.N + n] = hn;
-        } else if (a.trace && b < a.trace_rows) {
-          // lanes that ran fewer iterations keep their last value in the trace
-          a.trace[(size_t)a.out_row[b] * a.N + n] = a.hres[(size_t)b * a.N + n];
-        }
-      }
+  for (int j = 0; j < n_my; ++j) {
+    const int unit = blockIdx.x + j * gridDim.x;
+    const int st = j % a.stages;
+    unsigned char* stage = stages + (size_t)st * stage_bytes;
+    if (!dg_wait(smem_u32(bars + st), (uint32_t)(j / a.stages) & 1u)) abort_flag = 1;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    unit_mma(stage, acc);
+    // ---- the warps' sums, added in warp order (red alternates between two halves)
+    float* redj = red + (size_t)(j & 1) * DG_WARPS * 16 * 8;
+    float* rw = redj + ((size_t)(m * W + ks) * 16) * 8;      // [16 rows][8 tokens]
+    rw[g * 8 + 2 * t] = acc[0];
+    rw[g * 8 + 2 * t + 1] = acc[1];
+    rw[(g + 8) * 8 + 2 * t] = acc[2];
+    rw[(g + 8) * 8 + 2 * t + 1] = acc[3];
+    __syncthreads();   // every warp is done with this stage and wrote its sums
+    if (abort_flag) {
+      stop = j;
+      break;
     }
+    // refill the stage with the unit `stages` ahead
+    if (j + a.stages < n_my) {
+      if (warp == 0)
+        dg_issue_unit<MT>(a, unit + a.stages * gridDim.x, stage, smem_u32(bars + st), lane);
+      ++issued;
+    }
+    unit_epilogue(unit, redj);
+  }
+  }
+  if (tid == 0 && abort_flag && a.status) atomicCAS(a.status, 0, (int)TL_ERR_TIMEOUT);
+  if (abort_flag && tid == 0) {
+    // wait (bounded) for the copies still in flight before the CTA leaves:
+    // units stop .. issued - 1
+    for (int jj = stop; jj < issued; ++jj)
+      dg_wait(smem_u32(bars + jj % a.stages), (uint32_t)(jj / a.stages) & 1u);
   }
 }
 
-template <int BITS, int MT, bool NORM, int EPI, int MC>
-tl_status launch_dg_mc(const DgArgs& a, int grid, size_t smem, cudaStream_t s) {
+int dg_sm_count() {
+  static std::atomic<int> cached{0};
+  int n = cached.load();
+  if (n > 0) return n;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    n = 148;
+  }
+  cached.store(n);
+  return n;
+}
+
+// Shared memory a CTA may take and still leave room on its SM for the next
+// kernel's CTA; a unit that does not fit with its activations takes more.
+constexpr size_t kDgSmemShare = 110 * 1024;
+// the most dynamic shared memory one CTA may take on sm_100 (232448 bytes in
+// all) less room for the kernel's static shared memory
+constexpr size_t kDgSmemMax = 232448 - 1024;
+
+template <int BITS, int MT, bool NORM, int EPI, int UM>
+tl_status launch_dg_um(const DgArgs& a, int grid, size_t smem, cudaStream_t s) {
   static std::atomic<uint64_t> attr_done{0};
   TL_TRY(once_per_device(attr_done, []() -> tl_status {
-    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, MC>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024));
+    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, UM>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDgSmemMax));
     return ok();
   }));
-  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, MC>), grid, DG_THREADS, smem, s, a);
+  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, UM>), grid, DG_THREADS, smem, s, a);
   return ok();
 }
 
 template <int BITS, int MT, bool NORM, int EPI>
-tl_status launch_dg(const DgArgs& a, int grid, cudaStream_t s) {
+tl_status launch_dg(DgArgs a, cudaStream_t s) {
   const int nvec = a.wpr / 4, nch = (nvec + 3) / 4;
   const size_t xw = (size_t)nch * DgFmt<BITS>::CW + 8;
-  const size_t smem = (size_t)a.T * xw * 2 + (size_t)DG_WARPS * 16 * 8 * 4;
-  if (smem > 200 * 1024)
+  const size_t row_bytes = (size_t)a.wpr * 4;
+  a.row_stride = (int)(row_bytes + ((64 + 128 - row_bytes % 128) % 128));
+  const size_t stage = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * (a.K / a.G) * 2;
+  const int grid = std::min(a.n_units, dg_sm_count());
+  const int per_cta = (a.n_units + grid - 1) / grid;
+  const size_t red_unit = (size_t)DG_WARPS * 16 * 8 * 4;
+  const size_t fixed0 = (size_t)a.T * xw * 2 + 8 * 8 + 128;
+  // every unit resident when they fit (one reduction per launch)
+  const int um = per_cta <= 1 ? 1 : per_cta <= 2 ? 2 : per_cta <= 4 ? 4 : per_cta <= 8 ? 8 : 0;
+  if (um > 0) {
+    const size_t smem = fixed0 + (size_t)std::max(um, 2) * red_unit + (size_t)per_cta * stage;
+    if (smem <= kDgSmemMax) {
+      a.stages = per_cta;
+      switch (um) {
+        case 1: return launch_dg_um<BITS, MT, NORM, EPI, 1>(a, grid, smem, s);
+        case 2: return launch_dg_um<BITS, MT, NORM, EPI, 2>(a, grid, smem, s);
+        case 4: return launch_dg_um<BITS, MT, NORM, EPI, 4>(a, grid, smem, s);
+        default: return launch_dg_um<BITS, MT, NORM, EPI, 8>(a, grid, smem, s);
+      }
+    }
+  }
+  // a ring of stages, within the share of the SM that leaves room for the next kernel
+  const size_t fixed = fixed0 + 2 * red_unit;
+  int stages = 1;
+  while (stages < per_cta && stages < 8 && fixed + (stages + 1) * stage <= kDgSmemShare) ++stages;
+  const size_t smem = fixed + stages * stage;
+  if (smem > kDgSmemMax)
     return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: K = %d x %d tokens needs too much shared memory",
                      a.K, a.T);
-  const int per = (nch + DG_WARPS / MT - 1) / (DG_WARPS / MT);   // chunks of the longest k range
-  if (per <= 2) return launch_dg_mc<BITS, MT, NORM, EPI, 2>(a, grid, smem, s);
-  if (per <= 4) return launch_dg_mc<BITS, MT, NORM, EPI, 4>(a, grid, smem, s);
-  return launch_dg_mc<BITS, MT, NORM, EPI, DG_MAXC>(a, grid, smem, s);
+  a.stages = stages;
+  return launch_dg_um<BITS, MT, NORM, EPI, 0>(a, grid, smem, s);
 }
 
 }  // namespace
@@ -496,16 +764,20 @@ bool dec_gemv_eligible(int N, int K, int T, int bits) {
 tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   if (d.T == 0) return ok();
   if (d.T < 0 || d.T > 8) return set_error(TL_ERR_INVALID_ARG, "decode GEMV: %d tokens", d.T);
+  if (!dec_gemv_eligible(d.N, d.K, d.T, d.bits))
+    return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: shape N %d K %d", d.N, d.K);
   DgArgs a;
+  memset(&a, 0, sizeof(a));
   a.w0 = d.w0;
   a.s0 = d.s0;
-  a.w1 = d.w1;
-  a.s1 = d.s1;
+  a.w1 = d.w1 ? d.w1 : d.w0;
+  a.s1 = d.s1 ? d.s1 : d.s0;
   a.N = d.N;
   a.K = d.K;
   a.G = d.G;
   a.wpr = d.bits == 4 ? d.K / 8 : ((d.K + 9) / 10 + 3) / 4 * 4;
   a.T = d.T;
+  a.n_units = d.N / 16;
   a.x = d.x;
   a.h = d.h;
   a.gamma = d.gamma;
@@ -516,24 +788,20 @@ tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   a.trace = d.trace;
   a.out_row = d.out_row;
   a.trace_rows = d.trace_rows;
-  if (!dec_gemv_eligible(d.N, d.K, d.T, d.bits))
-    return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: shape N %d K %d", d.N, d.K);
+  a.status = d.status;
+  a.ex = d.ex;
   const bool norm = d.h != nullptr;
   switch (d.epi) {
     case DEC_EPI_SWIGLU:
       if (!norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: SwiGLU needs the norm prologue");
-      return d.bits == 4 ? launch_dg<4, 2, true, EPI_SWIGLU>(a, d.N / 16, s)
-                         : launch_dg<3, 2, true, EPI_SWIGLU>(a, d.N / 16, s);
+      return d.bits == 4 ? launch_dg<4, 2, true, EPI_SWIGLU>(a, s) : launch_dg<3, 2, true, EPI_SWIGLU>(a, s);
     case DEC_EPI_RESID:
       if (norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: residual epilogue takes x");
-      return d.bits == 4 ? launch_dg<4, 1, false, EPI_RESID>(a, d.N / 16, s)
-                         : launch_dg<3, 1, false, EPI_RESID>(a, d.N / 16, s);
+      return d.bits == 4 ? launch_dg<4, 1, false, EPI_RESID>(a, s) : launch_dg<3, 1, false, EPI_RESID>(a, s);
     default:
       if (norm)
-        return d.bits == 4 ? launch_dg<4, 1, true, EPI_OUT>(a, d.N / 16, s)
-                           : launch_dg<3, 1, true, EPI_OUT>(a, d.N / 16, s);
-      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT>(a, d.N / 16, s)
-                         : launch_dg<3, 1, false, EPI_OUT>(a, d.N / 16, s);
+        return d.bits == 4 ? launch_dg<4, 1, true, EPI_OUT>(a, s) : launch_dg<3, 1, true, EPI_OUT>(a, s);
+      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT>(a, s) : launch_dg<3, 1, false, EPI_OUT>(a, s);
   }
 }
 

@@ -20,12 +20,17 @@ tl_status ok();
     if (!(cond)) return ::tl::set_error(TL_ERR_INVALID_ARG, __VA_ARGS__); \
   } while (0)
 
+// A failed runtime call is reported and its error taken out of the runtime's
+// last-error slot, so that a later, unrelated launch check does not report it
+// again (a sticky error stays with the context whatever is done here).
 #define TL_CUDA(call)                                                         \
   do {                                                                        \
     cudaError_t e_ = (call);                                                  \
-    if (e_ != cudaSuccess)                                                    \
+    if (e_ != cudaSuccess) {                                                  \
+      cudaGetLastError();                                                     \
       return ::tl::set_error(TL_ERR_CUDA, "%s failed: %s (%s:%d)", #call,    \
                              cudaGetErrorString(e_), __FILE__, __LINE__);    \
+    }                                                                         \
   } while (0)
 
 #define TL_LAUNCH_CHECK() TL_CUDA(cudaGetLastError())
@@ -50,6 +55,16 @@ constexpr int kDevNumeric = TL_ERR_NUMERIC;
 struct KvHeader {
   int32_t pos[kMaxLanes];         // cached tokens per lane
   int32_t cum_layers[kMaxLanes];  // layers of all lanes before this one
+};
+
+// Per-iteration residual-norm check (see tl_model_set_exit_threshold): a row
+// whose residual stream leaves loop iteration i - 1 with an L2 norm above tau
+// gets exit_it[row] = i and runs no further residual updates.
+struct ExitArgs {
+  float tau;                 // < 0: no check
+  int32_t* exit_it;          // [rows]: 0 while the row runs, else the iterations it ran
+  int check_iter;            // > 0: record check_iter for rows above tau (the norm's input row)
+  int skip;                  // 1: rows with exit_it != 0 keep their residual stream
 };
 
 // ---------------------------------------------------------------- kernels (host launchers)
@@ -122,6 +137,8 @@ struct DecGemvArgs {
   float* trace;         // DEC_EPI_RESID: null or fp32 [trace_rows][N] (rows by out_row)
   const int32_t* out_row;
   int trace_rows;
+  int* status;          // null, or the model status word (a bounded wait that runs out)
+  ExitArgs ex;          // norm prologue: record rows above tau; residual epilogue: skip them
 };
 bool dec_gemv_eligible(int N, int K, int T, int bits);
 tl_status launch_dec_gemv(const DecGemvArgs& a, cudaStream_t s);
@@ -141,8 +158,10 @@ struct EmbedArgs {
   const int32_t* src_row;    // row t reads input row src_row[t] (null = identity)
   float* h;                  // [rows][d]
   int* status;
+  int32_t* exit_it;          // null, or [rows]: cleared (every row starts its loop)
 };
 tl_status launch_embed(const EmbedArgs& a, cudaStream_t s);
+
 
 struct NormArgs {
   float* h;                  // [rows][d] residual
@@ -160,6 +179,10 @@ struct NormArgs {
   const int32_t* out_row;    // null = identity
   float eps;
   int* status;
+  ExitArgs ex;               // the residual-norm check (tau < 0: off)
+  int32_t* loops_out;        // null, or [out rows]: loops run by each row in [fin_lo, fin_hi)
+  int L_row[kMaxLanes];      // the row's loop count (rows < kMaxLanes) when L_all == 0
+  int L_all;                 // > 0: every row's loop count
 };
 tl_status launch_residual_norm(const NormArgs& a, cudaStream_t s);
 

@@ -14,7 +14,7 @@ from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_dec
                tl_kv_reset, tl_kv_set_position, tl_model_create, tl_model_destroy,
                tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
                tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status, tl_extend,
-               tl_greedy_head, tl_spec_step)
+               tl_greedy_head, tl_spec_step, tl_model_set_exit_threshold, tl_loops_used)
 
 MATRICES = ("qkv", "o", "gate", "up", "down")
 
@@ -84,6 +84,13 @@ class DeviceModel:
     def set_decode_chunks(self, chunks_per_cta: int) -> None:
         """Context chunks one decode-attention CTA streams (0 = automatic)."""
         tl_model_set_decode_chunks(self.handle, chunks_per_cta)
+
+    def set_exit_threshold(self, tau: float) -> None:
+        """Per-iteration residual-norm check threshold (< 0: off)."""
+        tl_model_set_exit_threshold(self.handle, tau)
+
+    def loops_used(self, n: int):
+        return tl_loops_used(self.handle, n)
 
     def new_kv(self, L_per_lane: Sequence[int], max_ctx: int, dtype: str = "fp16") -> "DeviceKV":
         return DeviceKV(self, L_per_lane, max_ctx, dtype)
