@@ -97,6 +97,29 @@ tl_status tl_packed_bytes(int N, int K, int bits, int group,
 tl_status tl_pack_weights(const float* w, int N, int K, int bits, int group,
                           uint32_t* packed, uint16_t* scales, tl_stream stream);
 
+/* The 1-bit sign-of-frac channel of cross-iteration rounding ("Performance
+ * and Memory", "Cross-iteration stochastic rounding": INT4 plus a 1-bit
+ * sign-of-frac channel, +25 % storage; "Current Status", architecture-unique
+ * features table, deterministic error cancellation row: even loop iterations
+ * use the standard rounding, odd iterations apply the sign correction).
+ * For element (n, k) with group scale s = the fp16 scale tl_pack_weights
+ * wrote and code c:  bit = 1 when s != 0 and the fp32 quotient w / s is
+ * greater than c (the rounding went down), else 0.  An odd loop iteration
+ * then uses code c + 1 where the bit is set and c - 1 where it is clear: the
+ * other neighbour of w / s.
+ * Layout: uint32 [N, ceil(K / 32)], row-major; element k of a row is bit
+ * k % 32 of word k / 32; bits past K are zero. */
+tl_status tl_sign_bits_bytes(int N, int K, size_t* bytes);
+
+/* Write the sign-of-frac bits of an fp32 [N, K] matrix (device pointers).
+ *   w       fp32 [N, K], the matrix given to tl_pack_weights
+ *   scales  fp16 [N, K/group], the scales tl_pack_weights wrote for it
+ *   sign    uint32 [N, ceil(K/32)] (written)
+ * Bit-exact with the definition above; same requirements as
+ * tl_pack_weights. */
+tl_status tl_pack_sign_bits(const float* w, int N, int K, int bits, int group,
+                            const uint16_t* scales, uint32_t* sign, tl_stream stream);
+
 /* Test hook: unpack canonical packed words back to int8 codes [N, K]
  * (device pointers). */
 tl_status tl_unpack_codes(const uint32_t* packed, int N, int K, int bits,
@@ -158,6 +181,15 @@ typedef struct tl_block_desc {
   const uint32_t* w_down; const uint16_t* s_down;  /* [d, F]  */
   const float* gamma_attn;                          /* [d] RMSNorm gain before QKV */
   const float* gamma_ffn;                           /* [d] RMSNorm gain before SwiGLU */
+  /* Optional sign-of-frac bits of the five matrices (tl_pack_sign_bits
+   * layout), all five or none (NULL): the odd-iteration weights of
+   * cross-iteration rounding, used when the block is a model's loop block
+   * and tl_model_set_cross_iter turned it on. */
+  const uint32_t* sign_qkv;
+  const uint32_t* sign_o;
+  const uint32_t* sign_gate;
+  const uint32_t* sign_up;
+  const uint32_t* sign_down;
 } tl_block_desc;
 
 typedef struct tl_block tl_block;
@@ -231,6 +263,18 @@ tl_status tl_model_set_decode_chunks(tl_model* model, int chunks_per_cta);
  * Frees the model's captured graphs.  Errors: TL_ERR_INVALID_ARG for a NULL
  * model, NaN or +infinity. */
 tl_status tl_model_set_exit_threshold(tl_model* model, float tau);
+
+/* Cross-iteration rounding ("Performance and Memory", "Cross-iteration
+ * stochastic rounding"; "Current Status", architecture-unique features
+ * table, deterministic error cancellation row): with on != 0, loop
+ * iterations 1, 3, 5, ... (counting from 0) of every forward call run the
+ * loop block with each code moved to its other rounding neighbour (code + 1
+ * where the block's sign bit is set, code - 1 where it is clear), same
+ * scales; iterations 0, 2, ... and the pre-blocks are unchanged.  Every kernel
+ * reads the bits next to the packed words; nothing is dequantised ahead.
+ * Frees the model's captured graphs.  Errors: TL_ERR_INVALID_ARG for a NULL
+ * model or when the loop block has no sign bits. */
+tl_status tl_model_set_cross_iter(tl_model* model, int on);
 
 /* Loop iterations each output row of the last forward call ran (after the
  * stream's work): the loop count L unless the residual-norm check stopped it

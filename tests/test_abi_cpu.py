@@ -40,7 +40,7 @@ def test_only_tl_symbols_exported():
 
 
 def test_abi_version():
-    assert tl.tl_abi_version() == 100
+    assert tl.tl_abi_version() == 101
 
 
 @pytest.mark.parametrize("K", [64, 256, 2048, 8192, 10, 11, 4000])

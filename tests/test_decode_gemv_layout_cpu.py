@@ -231,3 +231,161 @@ def test_int3_word_slots_match_the_slot_table():
                     got = eval(exprs[i].replace("(q & 1)", str(q & 1)),
                                {"base": base, "j0": j0, "j1": j1, "j8": j8})
                     assert got == xpos(c * 160 + 40 * t + 10 * q + i, 3), (c, t, q, i)
+
+
+# ---------------------------------------------------------------- cross-iteration rounding
+# The odd-iteration code is code + 1 where the sign-of-frac bit is set and
+# code - 1 where it is clear (oracle.odd_iteration_codes).  The kernels add
+# the fp16 pair pm1(x) (bits 15 and 31 of x -> +-1) to each exact code pair;
+# the bit manipulations below are the kernels', read from their sources.
+TC_SRC = open(os.path.join(ROOT, "weight_shared_looped_b200", "csrc", "gemm_tc.cu")).read()
+M32 = 0xFFFFFFFF
+
+
+def pm1(x):
+    return (1.0 if (x >> 15) & 1 else -1.0, 1.0 if (x >> 31) & 1 else -1.0)
+
+
+def int4_sign_fix(sw, q):
+    h = sw if q < 2 else sw >> 16
+    P = ((h & 0x0F0F) | ((h & 0xF0F0) << 12)) & M32
+    base = 7 if q & 1 else 15
+    return [pm1((P << (base - i)) & M32) for i in range(4)]
+
+
+def int3_sign_S(sg_row, vi):
+    wi, o = (5 * vi) >> 2, 8 * (vi & 3)
+    a = int(sg_row[wi]) if wi < len(sg_row) else 0
+    b = int(sg_row[wi + 1]) if wi + 1 < len(sg_row) else 0
+    return ((b << 32) | a) >> o
+
+
+def int3_sign_i6(S, q, I):
+    w = (S >> (10 * q)) & 0x3FF
+    return pm1(((w | (w << 10)) << (15 - I)) & M32)
+
+
+def int3_sign_c(S, o, shift):
+    u = (S >> o) & 0xC03
+    return pm1(((u | (u << 6)) << shift) & M32)
+
+
+def sign_spread(h16):
+    return (h16 & 0x5555) | ((h16 & 0xAAAA) << 15)
+
+
+def tc_sign_corr(gs, c):
+    return pm1((gs[c >> 3] << (15 - 2 * (c & 7))) & M32)
+
+
+def test_sign_constants_match_the_kernels():
+    for c in ('"r"(0x80008000u), "r"(0xBC00BC00u)', "lop3.b32 %0, %1, %2, %3, 0x6A;",
+              "const uint32_t P = (h & 0x0F0Fu) | ((h & 0xF0F0u) << 12);",
+              "const int base = (q & 1) ? 7 : 15;", "pm1(P << (base - i))",
+              "const uint32_t h = q < 2 ? sw : sw >> 16;",
+              "return pm1((w | (w << 10)) << (15 - I));", "(uint32_t)(S >> (10 * q)) & 0x3FFu",
+              "(uint32_t)(S >> o) & 0xC03u", "return pm1((u | (u << 6)) << 15);",
+              "return pm1((u | (u << 6)) << 14);",
+              "const int wi = (5 * vi) >> 2, o = 8 * (vi & 3);",
+              "int3_sign_c4(S0, 4)", "int3_sign_c5(S0, 24)"):
+        assert c in SRC, c
+    for c in ("return (h16 & 0x5555u) | ((h16 & 0xAAAAu) << 15);",
+              "pm1(gs[c >> 3] << (15 - 2 * (c & 7)))", "gs[1] = sign_spread(ws.sg.x >> 16);",
+              "gs[2] = sign_spread(ws.sg.y & 0xFFFFu);"):
+        assert c in TC_SRC, c
+
+
+def test_tc_sign_pairs():
+    """Pair c of a 64-code k block (codes 2c, 2c + 1) gets the bits 2c, 2c + 1."""
+    rng = np.random.default_rng(5)
+    for _ in range(50):
+        x, y = (int(v) for v in rng.integers(0, 2**32, size=2, dtype=np.uint64))
+        gs = [sign_spread(x & 0xFFFF), sign_spread(x >> 16), sign_spread(y & 0xFFFF),
+              sign_spread(y >> 16)]
+        bits = [((x | (y << 32)) >> k) & 1 for k in range(64)]
+        for c in range(32):
+            assert tc_sign_corr(gs, c) == (2.0 * bits[2 * c] - 1, 2.0 * bits[2 * c + 1] - 1), c
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_int4_chunk_dot_product_odd_iteration(seed):
+    rng = np.random.default_rng(40 + seed)
+    K = 256
+    codes = rng.integers(-8, 8, size=(1, K)).astype(np.int8)
+    bits = rng.integers(0, 2, size=(1, K)).astype(np.uint8)
+    words = o.pack_codes(codes, 4)[0]
+    sg = o.pack_bits(bits)[0]
+    odd = o.odd_iteration_codes(codes, bits)[0].astype(np.float64)
+    x = rng.standard_normal(K).astype(np.float16).astype(np.float64)
+    xs = np.zeros(K)
+    for k in range(K):
+        xs[xpos(k, 4)] = x[k]
+    for c in range(K // 128):
+        frags = []
+        for t in range(4):
+            vi = 4 * c + t
+            f = _lane_fragments_int4(words[4 * vi:4 * vi + 4])
+            for q in range(4):
+                corr = int4_sign_fix(int(sg[vi]), q)
+                a, b = f[2 * q], f[2 * q + 1]
+                f[2 * q] = ((a[0][0] + corr[0][0], a[0][1] + corr[0][1]),
+                            (a[1][0] + corr[1][0], a[1][1] + corr[1][1]))
+                f[2 * q + 1] = ((b[0][0] + corr[2][0], b[0][1] + corr[2][1]),
+                                (b[1][0] + corr[3][0], b[1][1] + corr[3][1]))
+            frags.append(f)
+        got = _mma_dot(frags, xs[128 * c:128 * c + 128], 128)
+        want = float(odd[128 * c:128 * c + 128] @ x[128 * c:128 * c + 128])
+        assert abs(got - want) <= 1e-9 * max(1.0, abs(want)), (c, got, want)
+
+
+@pytest.mark.parametrize("seed", range(2))
+def test_int3_chunk_dot_product_odd_iteration(seed):
+    rng = np.random.default_rng(60 + seed)
+    K, G = 2048, 64
+    w = rng.standard_normal((1, K)).astype(np.float32) * 0.02
+    codes, scales = o.quantize_groupwise(w, 3, G)
+    bits = o.sign_of_frac(w, G, 3)
+    words = o.pack_codes(codes, 3)[0]
+    sg = o.pack_bits(bits)[0]
+    odd = o.odd_iteration_codes(codes, bits)[0]
+    nvec = len(words) // 4
+    nch = (nvec + 3) // 4
+    x = np.zeros(nch * 160)
+    x[:K] = rng.standard_normal(K).astype(np.float16).astype(np.float64)
+    xs = np.zeros(nch * 160)
+    for k in range(nch * 160):
+        xs[xpos(k, 3)] = x[k]
+    s = scales[0].astype(np.float64)
+    gpr = K // G
+    total = 0.0
+    for c in range(nch):
+        frags = []
+        for t in range(4):
+            vi = 4 * c + t
+            lw = [int(v) for v in (words[4 * vi:4 * vi + 4] if vi < nvec else np.zeros(4, np.uint32))]
+            S = int3_sign_S(sg, vi)
+            k0 = 160 * c + 40 * t
+            ga = min(k0 // G, gpr - 1)
+            gb = min(ga + 1, gpr - 1)
+            bnd = (k0 // G + 1) * G - k0
+            sc = lambda L: s[ga] if L < bnd else s[gb]
+
+            def fx(pair, corr, La, Lb):
+                return (float(np.float16((pair[0] + corr[0]) * sc(La))),
+                        float(np.float16((pair[1] + corr[1]) * sc(Lb))))
+            f = {}
+            for q in range(4):
+                L = 10 * q
+                f[2 * q] = (fx(int3_pair_i6(lw[q], 0), int3_sign_i6(S, q, 0), L, L + 6),
+                            fx(int3_pair_i6(lw[q], 1), int3_sign_i6(S, q, 1), L + 1, L + 7))
+                f[2 * q + 1] = (fx(int3_pair_i6(lw[q], 2), int3_sign_i6(S, q, 2), L + 2, L + 8),
+                                fx(int3_pair_i6(lw[q], 3), int3_sign_i6(S, q, 3), L + 3, L + 9))
+            f[8] = (fx(int3_pair_c4(lw[0], lw[1]), int3_sign_c(S, 4, 15), 4, 14),
+                    fx(int3_pair_c5(lw[0], lw[1]), int3_sign_c(S, 4, 14), 5, 15))
+            f[9] = (fx(int3_pair_c4(lw[2], lw[3]), int3_sign_c(S, 24, 15), 24, 34),
+                    fx(int3_pair_c5(lw[2], lw[3]), int3_sign_c(S, 24, 14), 25, 35))
+            frags.append(f)
+        total += _mma_dot(frags, xs[160 * c:160 * c + 160], 160)
+    deq = np.array([float(np.float16(odd[k] * s[k // G])) for k in range(K)])
+    want = float(deq @ x[:K])
+    assert abs(total - want) <= 1e-9 * max(1.0, abs(want)), (total, want)

@@ -49,7 +49,7 @@ def _ring_depths():
     assert "A_BATCHES = (TMEM_COLS - BN) / (A_COLS * BATCH)" in src
     m = re.search(r"X_STAGES = BN >= 128 \? (\d+) : (\d+);", src)
     assert m
-    tiles = sorted(set(int(x) for x in re.findall(r"launch_tc_bn<(\d+), [34]>", src)))
+    tiles = sorted(set(int(x) for x in re.findall(r"launch_tc_bn<(\d+), [34], (?:true|false)>", src)))
     assert tiles == [64, 128], tiles
     out = {}
     for bn in tiles:

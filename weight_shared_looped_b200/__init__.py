@@ -44,7 +44,8 @@ class BlockDesc(ctypes.Structure):
                 ("group", I), ("eps", F), ("rope_theta", F),
                 ("w_qkv", P), ("s_qkv", P), ("w_o", P), ("s_o", P), ("w_gate", P), ("s_gate", P),
                 ("w_up", P), ("s_up", P), ("w_down", P), ("s_down", P),
-                ("gamma_attn", P), ("gamma_ffn", P)]
+                ("gamma_attn", P), ("gamma_ffn", P),
+                ("sign_qkv", P), ("sign_o", P), ("sign_gate", P), ("sign_up", P), ("sign_down", P)]
 
 
 class ModelDesc(ctypes.Structure):
@@ -60,6 +61,8 @@ _SIGS = {
     "tl_packed_bytes": ([I, I, I, I, ctypes.POINTER(SZ), ctypes.POINTER(SZ)], I),
     "tl_pack_weights": ([P, I, I, I, I, P, P, P], I),
     "tl_unpack_codes": ([P, I, I, I, P, P], I),
+    "tl_sign_bits_bytes": ([I, I, ctypes.POINTER(SZ)], I),
+    "tl_pack_sign_bits": ([P, I, I, I, I, P, P, P], I),
     "tl_kv_quant_int8": ([P, I, I, P, P, P], I),
     "tl_attention_prefill": ([P, P, P, I, I, I, P, P], I),
     "tl_block_create": ([ctypes.POINTER(BlockDesc), ctypes.POINTER(P)], I),
@@ -71,6 +74,7 @@ _SIGS = {
     "tl_model_set_graphs": ([P, I], I),
     "tl_model_set_decode_chunks": ([P, I], I),
     "tl_model_set_exit_threshold": ([P, F], I),
+    "tl_model_set_cross_iter": ([P, I], I),
     "tl_loops_used": ([P, P, I, P], I),
     "tl_kv_layer_bytes": ([I, I, I, I, ctypes.POINTER(SZ)], I),
     "tl_kv_bytes": ([P, I, I, P, I, ctypes.POINTER(SZ)], I),
@@ -148,6 +152,19 @@ def tl_pack_weights(w, bits: int, group: int, packed, scales, stream=None) -> No
                                _stream(stream)))
 
 
+def tl_sign_bits_bytes(N: int, K: int) -> int:
+    b = SZ()
+    _check(lib.tl_sign_bits_bytes(N, K, ctypes.byref(b)))
+    return b.value
+
+
+def tl_pack_sign_bits(w, bits: int, group: int, scales, sign, stream=None) -> None:
+    """Sign-of-frac bits of fp32 w [N, K] with the scales tl_pack_weights wrote."""
+    N, K = w.shape
+    _check(lib.tl_pack_sign_bits(_ptr(w), N, K, bits, group, _ptr(scales), _ptr(sign),
+                                 _stream(stream)))
+
+
 def tl_unpack_codes(packed, N: int, K: int, bits: int, codes, stream=None) -> None:
     _check(lib.tl_unpack_codes(_ptr(packed), N, K, bits, _ptr(codes), _stream(stream)))
 
@@ -168,12 +185,15 @@ def tl_attention_prefill(q, k, v, H: int, hd: int, out, stream=None) -> None:
 
 def tl_block_create(cfg: dict, packed: dict) -> int:
     """cfg: d_model, n_heads, head_dim, ffn, bits, group, eps, rope_theta;
-    packed: device tensors w_qkv, s_qkv, ..., gamma_attn, gamma_ffn."""
+    packed: device tensors w_qkv, s_qkv, ..., gamma_attn, gamma_ffn, and optionally
+    sign_qkv, ..., sign_down (the sign-of-frac bits of cross-iteration rounding)."""
     d = BlockDesc(cfg["d_model"], cfg["n_heads"], cfg["head_dim"], cfg["ffn"], cfg["bits"],
                   cfg["group"], cfg["eps"], cfg["rope_theta"],
                   *[_ptr(packed[k]) for k in ("w_qkv", "s_qkv", "w_o", "s_o", "w_gate", "s_gate",
                                               "w_up", "s_up", "w_down", "s_down", "gamma_attn",
-                                              "gamma_ffn")])
+                                              "gamma_ffn")],
+                  *[_ptr(packed.get(k)) for k in ("sign_qkv", "sign_o", "sign_gate", "sign_up",
+                                                  "sign_down")])
     out = P()
     _check(lib.tl_block_create(ctypes.byref(d), ctypes.byref(out)))
     return out.value
@@ -219,6 +239,10 @@ def tl_model_set_decode_chunks(model: int, chunks_per_cta: int) -> None:
 
 def tl_model_set_exit_threshold(model: int, tau: float) -> None:
     _check(lib.tl_model_set_exit_threshold(model, tau))
+
+
+def tl_model_set_cross_iter(model: int, on: bool) -> None:
+    _check(lib.tl_model_set_cross_iter(model, 1 if on else 0))
 
 
 def tl_loops_used(model: int, n: int, stream=None):

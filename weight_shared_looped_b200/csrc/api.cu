@@ -98,6 +98,7 @@ struct tl_model {
   bool graphs = true;
   int decode_chunks = 0;   // context chunks per decode-attention CTA; 0 = automatic
   float exit_tau = -1.f;   // per-iteration residual-norm check threshold; < 0 = off
+  bool cross_iter = false; // odd loop iterations take the loop block's other rounding neighbours
   cudaStream_t cap_stream = nullptr;
   // workspace
   void* ws = nullptr;
@@ -128,7 +129,7 @@ struct tl_model {
 // Misc
 // ============================================================================
 TL_API const char* tl_last_error(void) { return g_last_error.c_str(); }
-TL_API int tl_abi_version(void) { return 100; }
+TL_API int tl_abi_version(void) { return 101; }
 
 // ============================================================================
 // Packing
@@ -157,6 +158,20 @@ TL_API tl_status tl_pack_weights(const float* w, int N, int K, int bits, int gro
   TL_TRY(check_matrix(N, K, bits, group));
   TL_CHECK_ARG(w && packed && scales, "NULL device pointer");
   return launch_pack(w, N, K, bits, group, packed, scales, (cudaStream_t)stream);
+}
+
+TL_API tl_status tl_sign_bits_bytes(int N, int K, size_t* bytes) {
+  TL_CHECK_ARG(bytes != nullptr, "bytes is NULL");
+  TL_CHECK_ARG(N >= 1 && K >= 1, "matrix shape [%d, %d] must be positive", N, K);
+  *bytes = (size_t)N * ((K + 31) / 32) * 4;
+  return ok();
+}
+
+TL_API tl_status tl_pack_sign_bits(const float* w, int N, int K, int bits, int group,
+                                   const uint16_t* scales, uint32_t* sign, tl_stream stream) {
+  TL_TRY(check_matrix(N, K, bits, group));
+  TL_CHECK_ARG(w && scales && sign, "NULL device pointer");
+  return launch_pack_sign_bits(w, N, K, bits, group, scales, sign, (cudaStream_t)stream);
 }
 
 TL_API tl_status tl_unpack_codes(const uint32_t* packed, int N, int K, int bits, int8_t* codes,
@@ -218,6 +233,10 @@ TL_API tl_status tl_block_create(const tl_block_desc* desc, tl_block** out) {
   TL_CHECK_ARG(d.w_qkv && d.s_qkv && d.w_o && d.s_o && d.w_gate && d.s_gate && d.w_up &&
                    d.s_up && d.w_down && d.s_down && d.gamma_attn && d.gamma_ffn,
                "NULL weight pointer in block description");
+  const int n_sign = (d.sign_qkv != nullptr) + (d.sign_o != nullptr) + (d.sign_gate != nullptr) +
+                     (d.sign_up != nullptr) + (d.sign_down != nullptr);
+  TL_CHECK_ARG(n_sign == 0 || n_sign == 5,
+               "sign bits: give all five matrices' bits or none (%d given)", n_sign);
   std::unique_ptr<tl_block> b(new tl_block());
   b->d = d;
   *out = b.release();
@@ -445,6 +464,15 @@ TL_API tl_status tl_model_set_exit_threshold(tl_model* model, float tau) {
   return ok();
 }
 
+TL_API tl_status tl_model_set_cross_iter(tl_model* model, int on) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG(!on || model->loop->d.sign_qkv != nullptr,
+               "cross-iteration rounding needs a loop block with sign bits");
+  model->cross_iter = on != 0;
+  free_graphs(model);   // captured graphs hold the old weights of odd iterations
+  return ok();
+}
+
 TL_API tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream) {
   TL_CHECK_ARG(model && loops, "NULL argument");
   TL_CHECK_ARG(n >= 1 && n <= std::max(model->Tmax, kMaxLanes), "n = %d out of range", n);
@@ -614,7 +642,15 @@ const tl_block* block_at(const tl_model* m, int layer) {
   return layer < (int)m->pre.size() ? m->pre[layer] : m->loop;
 }
 
-GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half* x, int T) {
+// Whether layer `layer` is an odd loop iteration run with the other rounding
+// neighbours (cross-iteration rounding on).
+bool odd_iteration(const tl_model* m, int layer) {
+  const int it = layer - (int)m->pre.size();
+  return m->cross_iter && it >= 0 && (it & 1) == 1;
+}
+
+GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half* x, int T,
+                   bool odd) {
   const tl_block_desc& d = b->d;
   GemmArgs a;
   memset(&a, 0, sizeof(a));
@@ -627,12 +663,14 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
     case 0:  // QKV
       a.w0 = a.w1 = d.w_qkv;
       a.s0 = a.s1 = (const __half*)d.s_qkv;
+      a.g0 = a.g1 = d.sign_qkv;
       a.N = a.n_split = 3 * m->d;
       a.K = m->d;
       break;
     case 1:  // O
       a.w0 = a.w1 = d.w_o;
       a.s0 = a.s1 = (const __half*)d.s_o;
+      a.g0 = a.g1 = d.sign_o;
       a.N = a.n_split = m->d;
       a.K = m->d;
       break;
@@ -641,6 +679,8 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
       a.s0 = (const __half*)d.s_gate;
       a.w1 = d.w_up;
       a.s1 = (const __half*)d.s_up;
+      a.g0 = d.sign_gate;
+      a.g1 = d.sign_up;
       a.n_split = m->F;
       a.N = 2 * m->F;
       a.K = m->d;
@@ -648,11 +688,13 @@ GemmArgs gemm_args(const tl_model* m, const tl_block* b, int which, const __half
     default:  // down
       a.w0 = a.w1 = d.w_down;
       a.s0 = a.s1 = (const __half*)d.s_down;
+      a.g0 = a.g1 = d.sign_down;
       a.N = a.n_split = m->d;
       a.K = m->F;
       break;
   }
-  a.splits = gemm_splits(a.N, a.K, T, a.bits);
+  if (!odd) a.g0 = a.g1 = nullptr;
+  a.splits = gemm_splits(a.N, a.K, T, a.bits, a.g0 != nullptr);
   a.status = m->status;
   return a;
 }
@@ -689,8 +731,9 @@ NormArgs norm_args(const tl_model* m, int rows) {
 // is done by the next norm).
 tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
                              int lane, cudaStream_t s) {
+  const bool odd = odd_iteration(m, layer);
   // QKV
-  GemmArgs g = gemm_args(m, b, 0, m->x, rows);
+  GemmArgs g = gemm_args(m, b, 0, m->x, rows, odd);
   TL_TRY(launch_gemm(g, s));
   RopeKvArgs r;
   memset(&r, 0, sizeof(r));
@@ -718,7 +761,7 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   TL_TRY(launch_attn_prefill(m->q, m->k, m->v, m->attn, rows, m->H, m->hd, s));
   // O projection, then the residual add of its split-K partial sums and the
   // RMSNorm before the MLP in one norm kernel
-  g = gemm_args(m, b, 1, m->attn, rows);
+  g = gemm_args(m, b, 1, m->attn, rows, odd);
   TL_TRY(launch_gemm(g, s));
   NormArgs n = norm_args(m, rows);
   n.part = m->part;
@@ -730,15 +773,15 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   n.ex = exit_args(m, layer, 0);
   TL_TRY(launch_residual_norm(n, s));
   // SwiGLU MLP
-  g = gemm_args(m, b, 2, m->x, rows);
-  if (gemm_tc_eligible(g.N, g.K, rows, g.bits) && g.splits == 1 && m->F % 64 == 0) {
+  g = gemm_args(m, b, 2, m->x, rows, odd);
+  if (gemm_tc_eligible(g.N, g.K, rows, g.bits, g.g0 != nullptr) && g.splits == 1 && m->F % 64 == 0) {
     g.swiglu_u = m->u;   // the GEMM's epilogue forms silu(gate) * up
     TL_TRY(launch_gemm(g, s));
   } else {
     TL_TRY(launch_gemm(g, s));
     TL_TRY(launch_swiglu(m->part, g.splits, rows, m->F, m->u, s));
   }
-  g = gemm_args(m, b, 3, m->u, rows);
+  g = gemm_args(m, b, 3, m->u, rows, odd);
   TL_TRY(launch_gemm(g, s));
   return ok();
 }
@@ -753,6 +796,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
                                int trace_rows, bool split_attn, cudaStream_t s) {
   const tl_block_desc& bd = b->d;
   const int d = m->d, F = m->F;
+  const bool odd = odd_iteration(m, layer);
   DecGemvArgs p;
   memset(&p, 0, sizeof(p));
   p.G = bd.group;
@@ -763,6 +807,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   // QKV: q, k, v sums -> part [1][rows][3d]
   p.w0 = bd.w_qkv;
   p.s0 = (const __half*)bd.s_qkv;
+  p.g0 = odd ? bd.sign_qkv : nullptr;
   p.N = 3 * d;
   p.K = d;
   p.h = m->h;
@@ -813,6 +858,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   // O projection, added into the residual stream
   p.w0 = bd.w_o;
   p.s0 = (const __half*)bd.s_o;
+  p.g0 = odd ? bd.sign_o : nullptr;
   p.N = d;
   p.K = d;
   p.h = nullptr;
@@ -827,6 +873,8 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   p.s0 = (const __half*)bd.s_gate;
   p.w1 = bd.w_up;
   p.s1 = (const __half*)bd.s_up;
+  p.g0 = odd ? bd.sign_gate : nullptr;
+  p.g1 = odd ? bd.sign_up : nullptr;
   p.N = F;
   p.K = d;
   p.x = nullptr;
@@ -839,8 +887,10 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   // down projection, added into the residual stream (and the trace)
   p.w0 = bd.w_down;
   p.s0 = (const __half*)bd.s_down;
+  p.g0 = odd ? bd.sign_down : nullptr;
   p.w1 = nullptr;
   p.s1 = nullptr;
+  p.g1 = nullptr;
   p.N = d;
   p.K = F;
   p.h = nullptr;
@@ -881,7 +931,7 @@ tl_status enqueue_prefill(tl_model* m, bool use_ids, int seq, int L, tl_kv* kv, 
     NormArgs en = norm_args(m, seq);
     en.part = m->part;
     en.part_rows = seq;
-    en.S = gemm_splits(m->d, m->F, seq, b->d.bits);
+    en.S = gemm_splits(m->d, m->F, seq, b->d.bits, odd_iteration(m, layer));
     en.n_add = seq;
     {
       // the stream leaving this layer enters loop iteration it + 1

@@ -192,20 +192,22 @@ tl_status launch_split_sum(const float* part, int S, long n, float* y, cudaStrea
   return ok();
 }
 
-int gemm_splits(int N, int K, int T, int bits) {
-  return gemm_tc_eligible(N, K, T, bits) ? gemm_tc_splits(N, K, T) : gemm_mma_splits(N, K, T);
+int gemm_splits(int N, int K, int T, int bits, bool sign) {
+  return gemm_tc_eligible(N, K, T, bits, sign) ? gemm_tc_splits(N, K, T) : gemm_mma_splits(N, K, T);
 }
 
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.swiglu_u) {
-    if (!gemm_tc_eligible(a.N, a.K, a.T, a.bits) || a.splits != 1 || a.N != 2 * a.n_split ||
+    if (!gemm_tc_eligible(a.N, a.K, a.T, a.bits, a.g0 != nullptr) || a.splits != 1 ||
+        a.N != 2 * a.n_split ||
         a.n_split % 64 != 0)
       return set_error(TL_ERR_UNSUPPORTED,
                        "the fused SwiGLU epilogue needs the one-split tensor-core GEMM");
     return launch_gemm_tc(a, s);
   }
-  if (gemm_tc_eligible(a.N, a.K, a.T, a.bits)) return launch_gemm_tc(a, s);
-  if (a.bits == 3) return set_error(TL_ERR_UNSUPPORTED, "INT3 GEMM: N %% 128 and K %% 64 required");
+  if (gemm_tc_eligible(a.N, a.K, a.T, a.bits, a.g0 != nullptr)) return launch_gemm_tc(a, s);
+  if (a.bits == 3 || a.g0 != nullptr)
+    return set_error(TL_ERR_UNSUPPORTED, "INT3 or sign-bit GEMM: N %% 128 and K %% 64 required");
   return launch_gemm_mma(a, s);
 }
 

@@ -175,6 +175,8 @@ struct TcArgs {
   const uint32_t* w1;        // rows [n_split, N)
   const __half* s0;
   const __half* s1;
+  const uint32_t* g0;        // sign-of-frac bits [rows][K / 32] of w0's / w1's rows (SGN)
+  const uint32_t* g1;
   float* part;
   int* status;
   __half* swiglu_u;          // fused SwiGLU epilogue: fp16 [T][n_split] (N = 2 * n_split)
@@ -188,6 +190,25 @@ __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
       : "memory");
 }
 
+// Cross-iteration rounding: the odd-iteration code is code + 1 where the
+// sign-of-frac bit is set and code - 1 where it is clear.  A k block's 64
+// sign bits are two words; pair c (codes 2c, 2c + 1) has its bits at 2c and
+// 2c + 1.  sign_spread puts the bits of eight pairs of a half word 16 apart
+// (even bits stay, odd bits move up 15), so that one shift brings pair c's
+// bits to 15 and 31, and pm1 turns those into the fp16 pair (+-1, +-1).
+__device__ __forceinline__ uint32_t sign_spread(uint32_t h16) {
+  return (h16 & 0x5555u) | ((h16 & 0xAAAAu) << 15);
+}
+__device__ __forceinline__ uint32_t pm1(uint32_t x) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(x), "r"(0x80008000u), "r"(0xBC00BC00u));
+  return d;   // (x & 0x80008000) ^ 0xBC00BC00: bit set -> +1, clear -> -1
+}
+__device__ __forceinline__ __half2 sign_corr(const uint32_t* gs, int c) {
+  const uint32_t d = pm1(gs[c >> 3] << (15 - 2 * (c & 7)));
+  return *reinterpret_cast<const __half2*>(&d);
+}
+
 // INT3 k block: the 64 codes k0 .. k0 + 63 of one row, k0 = 64m, start at code
 // O = k0 mod 10 (0, 4, 8, 2 or 6) of word v[0] of the row's words v[0..7].  O
 // is even, so codes 2c and 2c + 1 always share a word: a shift and a mask
@@ -195,8 +216,9 @@ __device__ __forceinline__ void mbar_arrive_elect(uint64_t* bar) {
 // 13-18, and a lop3 keeps code 2c at bits 0-2 and code 2c + 1 at bits 16-18
 // under the fp16 exponent of 1024; 1024 + u less 1028 is the exact code, then
 // the fp16 product with the scale (as for INT4).
-template <int O>
-__device__ __forceinline__ void int3_kblock(const uint32_t* v, __half2 s2, uint32_t* out) {
+template <int O, bool SGN>
+__device__ __forceinline__ void int3_kblock(const uint32_t* v, __half2 s2, const uint32_t* gs,
+                                            uint32_t* out) {
   const __half2 bias = __halves2half2(__float2half_rn(1028.0f), __float2half_rn(1028.0f));
 #pragma unroll
   for (int c = 0; c < 32; ++c) {
@@ -205,6 +227,7 @@ __device__ __forceinline__ void int3_kblock(const uint32_t* v, __half2 s2, uint3
     uint32_t h;
     asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(y), "r"(0x00070007u), "r"(0x64006400u));
     __half2 cv = __hsub2(*reinterpret_cast<__half2*>(&h), bias);
+    if (SGN) cv = __hadd2(cv, sign_corr(gs, c));   // odd iteration: the other neighbour
     __half2 wv = __hmul2(cv, s2);
     out[c] = *reinterpret_cast<uint32_t*>(&wv);
   }
@@ -214,7 +237,7 @@ __device__ __forceinline__ void int3_kblock(const uint32_t* v, __half2 s2, uint3
 // room for a small CTA of the next or previous kernel on the same SM; at 80
 // the compiler schedules the weight loads less freely (gate|up 4% slower),
 // and more registers or a third register set of weights gain nothing.
-template <int BN, int BITS>
+template <int BN, int BITS, bool SGN>
 __global__ void __maxnreg__(96)
     gemm_w4_tc_kernel(const __grid_constant__ CUtensorMap map_x, TcArgs a) {
   constexpr int XS = TcCfg<BN>::X_STAGES;
@@ -360,14 +383,18 @@ __global__ void __maxnreg__(96)
     const size_t wpr = (size_t)a.wpr, gpr = (size_t)a.K >> gsh;
     const uint32_t* wrow;
     const __half* srow;
+    const uint32_t* grow = nullptr;   // the row's sign bits (SGN)
+    const size_t spr = (size_t)a.K >> 5;
     if (sw) {
       const bool up = r >= BM / 2;
       const size_t row = (size_t)wrow0 + (up ? r - BM / 2 : r);
       wrow = (up ? a.w1 : a.w0) + row * wpr;
       srow = (up ? a.s1 : a.s0) + row * gpr;
+      if (SGN) grow = (up ? a.g1 : a.g0) + row * spr;
     } else {
       wrow = (second ? a.w1 : a.w0) + (size_t)(wrow0 + r) * wpr;
       srow = (second ? a.s1 : a.s0) + (size_t)(wrow0 + r) * gpr;
+      if (SGN) grow = (second ? a.g1 : a.g0) + (size_t)(wrow0 + r) * spr;
     }
     // The packed words of this row's k block (INT4: 32 bytes; INT3: the three
     // aligned 16-byte vectors holding its 7 or 8 words) and its scale come
@@ -377,10 +404,12 @@ __global__ void __maxnreg__(96)
     // the previous kernel.
     struct WSet {
       uint4 a, b, c;
+      uint2 sg;   // the k block's 64 sign bits (SGN)
       __half sc;
     };
     WSet set0, set1;
     set0.a = set0.b = set0.c = make_uint4(0u, 0u, 0u, 0u);
+    set0.sg = make_uint2(0u, 0u);
     set0.sc = __float2half_rn(0.f);
     set1 = set0;
     auto fetch = [&](int i, WSet& w) {
@@ -398,6 +427,7 @@ __global__ void __maxnreg__(96)
           w.c = base + 8 < (int)wpr ? __ldg(p + 2) : make_uint4(0u, 0u, 0u, 0u);
         }
         w.sc = __ldg(srow + (k0 >> gsh));
+        if (SGN) w.sg = __ldg(reinterpret_cast<const uint2*>(grow + (k0 >> 5)));
       }
     };
     fetch(grp, set0);
@@ -413,6 +443,13 @@ __global__ void __maxnreg__(96)
       if (b >= AB && !mbar_wait(&done[(b - AB) % AB], ((b - AB) / AB) & 1)) return false;
       if (i < nkb) {
         const __half2 s2 = __halves2half2(ws.sc, ws.sc);
+        uint32_t gs[4] = {0u, 0u, 0u, 0u};
+        if (SGN) {
+          gs[0] = sign_spread(ws.sg.x & 0xFFFFu);
+          gs[1] = sign_spread(ws.sg.x >> 16);
+          gs[2] = sign_spread(ws.sg.y & 0xFFFFu);
+          gs[3] = sign_spread(ws.sg.y >> 16);
+        }
         uint32_t v[32];
         if (BITS == 4) {
           const uint32_t words[8] = {ws.a.x, ws.a.y, ws.a.z, ws.a.w, ws.b.x, ws.b.y, ws.b.z, ws.b.w};
@@ -425,6 +462,7 @@ __global__ void __maxnreg__(96)
                 "r"(bb | 0x40u | (bb << 8) | 0x4000u));
             asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(h) : "r"(x), "r"(0x00F0000Fu), "r"(0x64006400u));
             __half2 cv = __hfma2(*reinterpret_cast<__half2*>(&h), mul, add);   // exact codes
+            if (SGN) cv = __hadd2(cv, sign_corr(gs, c));   // odd iteration: the other neighbour
             __half2 wv = __hmul2(cv, s2);                                      // fp16(code * s)
             v[c] = *reinterpret_cast<uint32_t*>(&wv);
           }
@@ -440,11 +478,11 @@ __global__ void __maxnreg__(96)
           for (int j = 0; j < 8; ++j)
             w8[j] = d == 0 ? u[j] : d == 1 ? u[j + 1] : d == 2 ? u[j + 2] : u[j + 3];
           switch (k0 % 10) {
-            case 0: int3_kblock<0>(w8, s2, v); break;
-            case 2: int3_kblock<2>(w8, s2, v); break;
-            case 4: int3_kblock<4>(w8, s2, v); break;
-            case 6: int3_kblock<6>(w8, s2, v); break;
-            default: int3_kblock<8>(w8, s2, v); break;
+            case 0: int3_kblock<0, SGN>(w8, s2, gs, v); break;
+            case 2: int3_kblock<2, SGN>(w8, s2, gs, v); break;
+            case 4: int3_kblock<4, SGN>(w8, s2, gs, v); break;
+            case 6: int3_kblock<6, SGN>(w8, s2, gs, v); break;
+            default: int3_kblock<8, SGN>(w8, s2, gs, v); break;
           }
         }
         fetch(i + 2 * BATCH, ws);
@@ -638,7 +676,7 @@ size_t tc_smem_bytes() {
   return b < kMinSmem ? kMinSmem : b;
 }
 
-template <int BN, int BITS>
+template <int BN, int BITS, bool SGN>
 tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   CUtensorMap mx;
   TL_TRY(encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, g.x, g.K, g.T, (uint64_t)g.K * 2, BK, BN,
@@ -655,6 +693,8 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   a.w1 = g.w1;
   a.s0 = g.s0;
   a.s1 = g.s1;
+  a.g0 = g.g0;
+  a.g1 = g.g1 ? g.g1 : g.g0;
   a.part = g.part;
   a.status = g.status;
   a.swiglu_u = g.swiglu_u;
@@ -662,7 +702,7 @@ tl_status launch_tc_bn(const GemmArgs& g, cudaStream_t s) {
   if (smem > 232448)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs %zu bytes of shared memory", smem);
   dim3 grid(g.N / BM, (g.T + BN - 1) / BN, g.splits);
-  TL_LAUNCH_PDL((gemm_w4_tc_kernel<BN, BITS>), grid, THREADS, smem, s, mx, a);
+  TL_LAUNCH_PDL((gemm_w4_tc_kernel<BN, BITS, SGN>), grid, THREADS, smem, s, mx, a);
   return ok();
 }
 
@@ -680,13 +720,21 @@ tl_status gemm_tc_init() {
   static std::atomic<uint64_t> done{0};
   return once_per_device(done, []() -> tl_status {
     TL_TRY(get_encoder());
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 4>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 4, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 4>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 4, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 3>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 3, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
-    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 3>,
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 3, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 4, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 4, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<64, 3, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
+    TL_CUDA(cudaFuncSetAttribute(gemm_w4_tc_kernel<128, 3, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, 232448));
     return ok();
   });
@@ -704,18 +752,23 @@ int gemm_tc_splits(int N, int K, int T) {
 
 // INT4 below 64 tokens runs the mma.sync kernel; INT3 runs here at every
 // token count (rows past T are read as zero).
-bool gemm_tc_eligible(int N, int K, int T, int bits) {
-  return (T >= 64 || bits == 3) && T >= 1 && N % BM == 0 && K % BK == 0;
+bool gemm_tc_eligible(int N, int K, int T, int bits, bool sign) {
+  return (T >= 64 || bits == 3 || sign) && T >= 1 && N % BM == 0 && K % BK == 0;
 }
 
 tl_status launch_gemm_tc(const GemmArgs& g, cudaStream_t s) {
   if (g.T == 0) return ok();
   if (g.n_split % BM != 0)
     return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM needs row split %% 128 == 0");
-  if (g.bits == 3)
-    return tc_tile_n(g.T) == 128 ? launch_tc_bn<128, 3>(g, s) : launch_tc_bn<64, 3>(g, s);
-  if (tc_tile_n(g.T) == 128) return launch_tc_bn<128, 4>(g, s);
-  return launch_tc_bn<64, 4>(g, s);
+  if (g.g0 != nullptr && g.K % 64 != 0)
+    return set_error(TL_ERR_UNSUPPORTED, "tensor-core GEMM: sign bits need K %% 64 == 0");
+  const bool wide = tc_tile_n(g.T) == 128;
+  if (g.g0 != nullptr) {
+    if (g.bits == 3) return wide ? launch_tc_bn<128, 3, true>(g, s) : launch_tc_bn<64, 3, true>(g, s);
+    return wide ? launch_tc_bn<128, 4, true>(g, s) : launch_tc_bn<64, 4, true>(g, s);
+  }
+  if (g.bits == 3) return wide ? launch_tc_bn<128, 3, false>(g, s) : launch_tc_bn<64, 3, false>(g, s);
+  return wide ? launch_tc_bn<128, 4, false>(g, s) : launch_tc_bn<64, 4, false>(g, s);
 }
 
 }  // namespace tl

@@ -127,6 +127,48 @@ __device__ __forceinline__ uint32_t int3_pair_c5(uint32_t a, uint32_t b) {
   return hfma2_bits(x, h2c(0.0078125f, 0.0078125f), h2c(-12.f, -12.f));
 }
 
+// ---- cross-iteration rounding: the odd-iteration code is code + 1 where the
+// sign-of-frac bit is set and code - 1 where it is clear.  pm1 turns bits 15
+// and 31 of x into the fp16 pair (+-1, +-1); adding it to an exact code pair
+// is exact.
+__device__ __forceinline__ uint32_t pm1(uint32_t x) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(x), "r"(0x80008000u), "r"(0xBC00BC00u));
+  return d;   // (x & 0x80008000) ^ 0xBC00BC00: bit set -> +1, clear -> -1
+}
+__device__ __forceinline__ uint32_t hadd2_bits(uint32_t a, uint32_t b) {
+  __half2 r = __hadd2(*reinterpret_cast<__half2*>(&a), *reinterpret_cast<__half2*>(&b));
+  return *reinterpret_cast<uint32_t*>(&r);
+}
+// INT4: the pairs (i, i + 4), i = 0..3, of word q of a lane's vector have their
+// bits at i and i + 4 of byte q of the vector's sign word; spreading two bytes
+// as low nibbles at bits 0-3 / 8-11 and high nibbles at 16-19 / 24-27 puts
+// the pair's bits 16 apart, one shift away from bits 15 and 31.
+__device__ __forceinline__ void int4_sign_fix(uint32_t sw, int q, uint32_t* p) {
+  const uint32_t h = q < 2 ? sw : sw >> 16;
+  const uint32_t P = (h & 0x0F0Fu) | ((h & 0xF0F0u) << 12);
+  const int base = (q & 1) ? 7 : 15;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) p[i] = hadd2_bits(p[i], pm1(P << (base - i)));
+}
+// INT3: S holds the sign bits of a lane's 40 codes (bit L for code L =
+// 10 q + i).  Pair (i, i + 6) of word q: bits 10q + i and 10q + i + 6.
+template <int I>
+__device__ __forceinline__ uint32_t int3_sign_i6(uint64_t S, int q) {
+  const uint32_t w = (uint32_t)(S >> (10 * q)) & 0x3FFu;
+  return pm1((w | (w << 10)) << (15 - I));
+}
+// Pairs c4 (codes 4 and 14 of word pair (0, 1), or 24 and 34 of (2, 3)) and
+// c5 (5 and 15, or 25 and 35): bits o, o + 1, o + 10, o + 11 with o = 4 or 24.
+__device__ __forceinline__ uint32_t int3_sign_c4(uint64_t S, int o) {
+  const uint32_t u = (uint32_t)(S >> o) & 0xC03u;
+  return pm1((u | (u << 6)) << 15);
+}
+__device__ __forceinline__ uint32_t int3_sign_c5(uint64_t S, int o) {
+  const uint32_t u = (uint32_t)(S >> o) & 0xC03u;
+  return pm1((u | (u << 6)) << 14);
+}
+
 // Position, in a staged activation row, of element k of the original row.
 // INT4: k = 128c + 32t + 8q + e -> k step 2q + ((e >> 1) & 1), slot 2t + 8 (e odd) + (e >= 4).
 // INT3: k = 160c + 40t + L (L = 10q + i) -> see int3_slot.
@@ -184,6 +226,9 @@ struct DgArgs {
   const __half* s0;     //   (EPI_SWIGLU: w0 = gate, w1 = up, both rows u*16 ..)
   const uint32_t* w1;
   const __half* s1;
+  const uint32_t* g0;   // sign-of-frac bits of w0's / w1's rows [N][spr] (odd iterations)
+  const uint32_t* g1;
+  int spr;              // sign words per row (K / 32)
   int N, K, G, wpr;     // output rows (per matrix), K, group, packed words per row
   int T;                // active token rows (1..8)
   int n_units;          // N / 16
@@ -231,15 +276,16 @@ __device__ __forceinline__ bool dg_wait(uint32_t bar, uint32_t parity) {
 // The weights (and scales) of one unit into its stage: lane r of the calling
 // warp copies row r of the unit (one bulk copy per row, so that staged rows
 // sit 64 bytes off the 128-byte bank period), the scales one copy per tile.
-template <int MT>
+template <int MT, bool SGN>
 __device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigned char* stage,
                                               uint32_t bar, int lane) {
   const int rows = 16 * MT;
   const uint32_t row_bytes = (uint32_t)a.wpr * 4;
   const int gpr = a.K / a.G;
   const uint32_t sc_bytes = 16u * gpr * 2;
+  const uint32_t sg_bytes = SGN ? 16u * a.spr * 4 : 0u;   // a tile's sign rows, one copy
   if (lane == 0) {
-    const uint32_t total = rows * row_bytes + MT * sc_bytes;
+    const uint32_t total = rows * row_bytes + MT * (sc_bytes + sg_bytes);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(total)
                  : "memory");
   }
@@ -261,6 +307,15 @@ __device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigne
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(sc_bytes), "r"(bar)
         : "memory");
+    if (SGN) {
+      const uint32_t* gsrc = (lane == 0 ? a.g0 : a.g1) + (size_t)r0 * a.spr;
+      const uint32_t gdst = smem_u32(stage + (size_t)rows * a.row_stride + (size_t)MT * sc_bytes +
+                                     (size_t)lane * sg_bytes);
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(gdst),
+          "l"(gsrc), "r"(sg_bytes), "r"(bar)
+          : "memory");
+    }
   }
 }
 
@@ -274,7 +329,7 @@ __device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigne
 // before the dependency wait; the warps compute them back to back into
 // per-unit sums and one reduction and one epilogue close the launch.  UM == 0:
 // the units stream through a ring of a.stages stages, one reduction per unit.
-template <int BITS, int MT, bool NORM, int EPI, int UM>
+template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN>
 __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   using Fm = DgFmt<BITS>;
   constexpr int CW = Fm::CW;
@@ -290,7 +345,8 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   const int gsh = __ffs(a.G) - 1;
   const int gpr = a.K >> gsh;
   const bool g64 = BITS == 4 && a.G == 64;
-  const size_t stage_bytes = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2;
+  const size_t stage_bytes = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2 +
+                             (SGN ? (size_t)MT * 16 * a.spr * 4 : 0);
   unsigned char* stages = dg_smem;
   __half* xs = reinterpret_cast<__half*>(dg_smem + (size_t)a.stages * stage_bytes);   // [T][xw]
   float* red = reinterpret_cast<float*>(xs + (size_t)a.T * xw);      // [max(2, UM)][MT][W][16][8]
@@ -313,7 +369,7 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   int stop = n_my;                    // the unit a timed-out wait stopped at
   if (warp == 0)
     for (int j = 0; j < a.stages && j < n_my; ++j)
-      dg_issue_unit<MT>(a, blockIdx.x + j * gridDim.x, stages + (size_t)j * stage_bytes,
+      dg_issue_unit<MT, SGN>(a, blockIdx.x + j * gridDim.x, stages + (size_t)j * stage_bytes,
                         smem_u32(bars + j), lane);
   // the gains are constants of the model: requested before the dependency
   // wait (rows of d <= 2048 take two float4 per thread)
@@ -484,6 +540,11 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
     const __half* st0 = reinterpret_cast<const __half*>(stage + (size_t)16 * MT * a.row_stride +
                                                         (size_t)m * 16 * gpr * 2) + (size_t)g * gpr;
     const __half* st1 = st0 + (size_t)8 * gpr;
+    // the tile's sign rows (odd iterations): rows g and g + 8
+    const uint32_t* sg0 = reinterpret_cast<const uint32_t*>(
+        stage + (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2 +
+        (size_t)(m * 16 + g) * a.spr * 4);
+    const uint32_t* sg1 = sg0 + (size_t)8 * a.spr;
     for (int c = c_lo; c < c_hi; ++c) {
       const int vi = 4 * c + t;
       uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
@@ -495,6 +556,9 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
       const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&v1);   // row g + 8
       const uint32_t xb = lbase + lmul * (uint32_t)(c * CW);
       if (BITS == 4) {
+        // the vector's 32 codes have one sign word (rows g and g + 8)
+        const uint32_t sw0 = SGN && vi < nvec ? sg0[vi] : 0u;
+        const uint32_t sw1 = SGN && vi < nvec ? sg1[vi] : 0u;
         const int ga = g64 ? 2 * c : c;
         float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb2[4] = {0.f, 0.f, 0.f, 0.f};
         const bool first = t < 2;   // G = 64: this lane's codes are in the chunk's first group
@@ -503,6 +567,10 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
           uint32_t p0[4], p1[4];
           int4_pairs(w0[q], p0);
           int4_pairs(w1[q], p1);
+          if (SGN) {
+            int4_sign_fix(sw0, q, p0);
+            int4_sign_fix(sw1, q, p1);
+          }
           uint32_t b[4];
           ldsm_x4(b, xb + lmul * (uint32_t)(32 * q));   // k steps 2q and 2q + 1
           const uint32_t A0[4] = {p0[0], p1[0], p0[1], p1[1]};
@@ -544,38 +612,53 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
           so0[oc] = 8 * oc < bnd ? sa0 : sb0;
           so1[oc] = 8 * oc < bnd ? sa1 : sb1;
         }
+        // the sign bits of the lane's 40 codes (bit L for code L), rows g and g + 8
+        uint64_t S0 = 0, S1 = 0;
+        if (SGN) {
+          const int wi = (5 * vi) >> 2, o = 8 * (vi & 3);
+          const uint32_t a0 = wi < a.spr ? sg0[wi] : 0u, b0 = wi + 1 < a.spr ? sg0[wi + 1] : 0u;
+          const uint32_t a1 = wi < a.spr ? sg1[wi] : 0u, b1 = wi + 1 < a.spr ? sg1[wi + 1] : 0u;
+          S0 = ((((uint64_t)b0) << 32) | a0) >> o;
+          S1 = ((((uint64_t)b1) << 32) | a1) >> o;
+        }
+#define TL_FX(p, corr) (SGN ? hadd2_bits((p), (corr)) : (p))
 #define TL_SC(p, La, Lb, so) hmul2_bits((p), h2bits(__halves2half2(so[(La) >> 3], so[(Lb) >> 3])))
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t b[4];
           ldsm_x4(b, xb + lmul * (uint32_t)(32 * q));   // k steps 2q, 2q + 1
           const int L = 10 * q;
-          const uint32_t A0[4] = {TL_SC(int3_pair_i6<0>(w0[q]), L, L + 6, so0),
-                                  TL_SC(int3_pair_i6<0>(w1[q]), L, L + 6, so1),
-                                  TL_SC(int3_pair_i6<1>(w0[q]), L + 1, L + 7, so0),
-                                  TL_SC(int3_pair_i6<1>(w1[q]), L + 1, L + 7, so1)};
-          const uint32_t A1[4] = {TL_SC(int3_pair_i6<2>(w0[q]), L + 2, L + 8, so0),
-                                  TL_SC(int3_pair_i6<2>(w1[q]), L + 2, L + 8, so1),
-                                  TL_SC(int3_pair_i6<3>(w0[q]), L + 3, L + 9, so0),
-                                  TL_SC(int3_pair_i6<3>(w1[q]), L + 3, L + 9, so1)};
+          const uint32_t A0[4] = {
+              TL_SC(TL_FX(int3_pair_i6<0>(w0[q]), int3_sign_i6<0>(S0, q)), L, L + 6, so0),
+              TL_SC(TL_FX(int3_pair_i6<0>(w1[q]), int3_sign_i6<0>(S1, q)), L, L + 6, so1),
+              TL_SC(TL_FX(int3_pair_i6<1>(w0[q]), int3_sign_i6<1>(S0, q)), L + 1, L + 7, so0),
+              TL_SC(TL_FX(int3_pair_i6<1>(w1[q]), int3_sign_i6<1>(S1, q)), L + 1, L + 7, so1)};
+          const uint32_t A1[4] = {
+              TL_SC(TL_FX(int3_pair_i6<2>(w0[q]), int3_sign_i6<2>(S0, q)), L + 2, L + 8, so0),
+              TL_SC(TL_FX(int3_pair_i6<2>(w1[q]), int3_sign_i6<2>(S1, q)), L + 2, L + 8, so1),
+              TL_SC(TL_FX(int3_pair_i6<3>(w0[q]), int3_sign_i6<3>(S0, q)), L + 3, L + 9, so0),
+              TL_SC(TL_FX(int3_pair_i6<3>(w1[q]), int3_sign_i6<3>(S1, q)), L + 3, L + 9, so1)};
           mma16816(acc, A0, b[0], b[1]);
           mma16816(acc, A1, b[2], b[3]);
         }
         {
           uint32_t b[4];
           ldsm_x4(b, xb + lmul * 128u);                  // k steps 8 and 9
-          const uint32_t A0[4] = {TL_SC(int3_pair_c4(w0[0], w0[1]), 4, 14, so0),
-                                  TL_SC(int3_pair_c4(w1[0], w1[1]), 4, 14, so1),
-                                  TL_SC(int3_pair_c5(w0[0], w0[1]), 5, 15, so0),
-                                  TL_SC(int3_pair_c5(w1[0], w1[1]), 5, 15, so1)};
-          const uint32_t A1[4] = {TL_SC(int3_pair_c4(w0[2], w0[3]), 24, 34, so0),
-                                  TL_SC(int3_pair_c4(w1[2], w1[3]), 24, 34, so1),
-                                  TL_SC(int3_pair_c5(w0[2], w0[3]), 25, 35, so0),
-                                  TL_SC(int3_pair_c5(w1[2], w1[3]), 25, 35, so1)};
+          const uint32_t A0[4] = {
+              TL_SC(TL_FX(int3_pair_c4(w0[0], w0[1]), int3_sign_c4(S0, 4)), 4, 14, so0),
+              TL_SC(TL_FX(int3_pair_c4(w1[0], w1[1]), int3_sign_c4(S1, 4)), 4, 14, so1),
+              TL_SC(TL_FX(int3_pair_c5(w0[0], w0[1]), int3_sign_c5(S0, 4)), 5, 15, so0),
+              TL_SC(TL_FX(int3_pair_c5(w1[0], w1[1]), int3_sign_c5(S1, 4)), 5, 15, so1)};
+          const uint32_t A1[4] = {
+              TL_SC(TL_FX(int3_pair_c4(w0[2], w0[3]), int3_sign_c4(S0, 24)), 24, 34, so0),
+              TL_SC(TL_FX(int3_pair_c4(w1[2], w1[3]), int3_sign_c4(S1, 24)), 24, 34, so1),
+              TL_SC(TL_FX(int3_pair_c5(w0[2], w0[3]), int3_sign_c5(S0, 24)), 25, 35, so0),
+              TL_SC(TL_FX(int3_pair_c5(w1[2], w1[3]), int3_sign_c5(S1, 24)), 25, 35, so1)};
           mma16816(acc, A0, b[0], b[1]);
           mma16816(acc, A1, b[2], b[3]);
         }
 #undef TL_SC
+#undef TL_FX
       }
     }
 
@@ -671,7 +754,7 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
     // refill the stage with the unit `stages` ahead
     if (j + a.stages < n_my) {
       if (warp == 0)
-        dg_issue_unit<MT>(a, unit + a.stages * gridDim.x, stage, smem_u32(bars + st), lane);
+        dg_issue_unit<MT, SGN>(a, unit + a.stages * gridDim.x, stage, smem_u32(bars + st), lane);
       ++issued;
     }
     unit_epilogue(unit, redj);
@@ -706,25 +789,26 @@ constexpr size_t kDgSmemShare = 110 * 1024;
 // all) less room for the kernel's static shared memory
 constexpr size_t kDgSmemMax = 232448 - 1024;
 
-template <int BITS, int MT, bool NORM, int EPI, int UM>
+template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN>
 tl_status launch_dg_um(const DgArgs& a, int grid, size_t smem, cudaStream_t s) {
   static std::atomic<uint64_t> attr_done{0};
   TL_TRY(once_per_device(attr_done, []() -> tl_status {
-    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, UM>,
+    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDgSmemMax));
     return ok();
   }));
-  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, UM>), grid, DG_THREADS, smem, s, a);
+  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN>), grid, DG_THREADS, smem, s, a);
   return ok();
 }
 
-template <int BITS, int MT, bool NORM, int EPI>
+template <int BITS, int MT, bool NORM, int EPI, bool SGN>
 tl_status launch_dg(DgArgs a, cudaStream_t s) {
   const int nvec = a.wpr / 4, nch = (nvec + 3) / 4;
   const size_t xw = (size_t)nch * DgFmt<BITS>::CW + 8;
   const size_t row_bytes = (size_t)a.wpr * 4;
   a.row_stride = (int)(row_bytes + ((64 + 128 - row_bytes % 128) % 128));
-  const size_t stage = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * (a.K / a.G) * 2;
+  const size_t stage = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * (a.K / a.G) * 2 +
+                       (SGN ? (size_t)MT * 16 * a.spr * 4 : 0);
   const int grid = std::min(a.n_units, dg_sm_count());
   const int per_cta = (a.n_units + grid - 1) / grid;
   const size_t red_unit = (size_t)DG_WARPS * 16 * 8 * 4;
@@ -736,10 +820,10 @@ tl_status launch_dg(DgArgs a, cudaStream_t s) {
     if (smem <= kDgSmemMax) {
       a.stages = per_cta;
       switch (um) {
-        case 1: return launch_dg_um<BITS, MT, NORM, EPI, 1>(a, grid, smem, s);
-        case 2: return launch_dg_um<BITS, MT, NORM, EPI, 2>(a, grid, smem, s);
-        case 4: return launch_dg_um<BITS, MT, NORM, EPI, 4>(a, grid, smem, s);
-        default: return launch_dg_um<BITS, MT, NORM, EPI, 8>(a, grid, smem, s);
+        case 1: return launch_dg_um<BITS, MT, NORM, EPI, 1, SGN>(a, grid, smem, s);
+        case 2: return launch_dg_um<BITS, MT, NORM, EPI, 2, SGN>(a, grid, smem, s);
+        case 4: return launch_dg_um<BITS, MT, NORM, EPI, 4, SGN>(a, grid, smem, s);
+        default: return launch_dg_um<BITS, MT, NORM, EPI, 8, SGN>(a, grid, smem, s);
       }
     }
   }
@@ -752,7 +836,7 @@ tl_status launch_dg(DgArgs a, cudaStream_t s) {
     return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: K = %d x %d tokens needs too much shared memory",
                      a.K, a.T);
   a.stages = stages;
-  return launch_dg_um<BITS, MT, NORM, EPI, 0>(a, grid, smem, s);
+  return launch_dg_um<BITS, MT, NORM, EPI, 0, SGN>(a, grid, smem, s);
 }
 
 }  // namespace
@@ -772,6 +856,9 @@ tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   a.s0 = d.s0;
   a.w1 = d.w1 ? d.w1 : d.w0;
   a.s1 = d.s1 ? d.s1 : d.s0;
+  a.g0 = d.g0;
+  a.g1 = d.g1 ? d.g1 : d.g0;
+  a.spr = d.K / 32;
   a.N = d.N;
   a.K = d.K;
   a.G = d.G;
@@ -791,18 +878,25 @@ tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   a.status = d.status;
   a.ex = d.ex;
   const bool norm = d.h != nullptr;
+  const bool sg = d.g0 != nullptr;
+  if (sg && (d.K % 32 != 0 || (d.epi == DEC_EPI_SWIGLU && d.g1 == nullptr)))
+    return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: sign bits need K %% 32 == 0 (and both matrices')");
+#define TL_DG(B, MT_, NORM_, EPI_) \
+  (sg ? launch_dg<B, MT_, NORM_, EPI_, true>(a, s) : launch_dg<B, MT_, NORM_, EPI_, false>(a, s))
   switch (d.epi) {
     case DEC_EPI_SWIGLU:
       if (!norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: SwiGLU needs the norm prologue");
-      return d.bits == 4 ? launch_dg<4, 2, true, EPI_SWIGLU>(a, s) : launch_dg<3, 2, true, EPI_SWIGLU>(a, s);
+      return d.bits == 4 ? TL_DG(4, 2, true, EPI_SWIGLU) : TL_DG(3, 2, true, EPI_SWIGLU);
     case DEC_EPI_RESID:
       if (norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: residual epilogue takes x");
-      return d.bits == 4 ? launch_dg<4, 1, false, EPI_RESID>(a, s) : launch_dg<3, 1, false, EPI_RESID>(a, s);
+      return d.bits == 4 ? TL_DG(4, 1, false, EPI_RESID) : TL_DG(3, 1, false, EPI_RESID);
     default:
-      if (norm)
-        return d.bits == 4 ? launch_dg<4, 1, true, EPI_OUT>(a, s) : launch_dg<3, 1, true, EPI_OUT>(a, s);
-      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT>(a, s) : launch_dg<3, 1, false, EPI_OUT>(a, s);
+      if (norm) return d.bits == 4 ? TL_DG(4, 1, true, EPI_OUT) : TL_DG(3, 1, true, EPI_OUT);
+      if (sg) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: sign bits need the norm prologue here");
+      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT, false>(a, s)
+                         : launch_dg<3, 1, false, EPI_OUT, false>(a, s);
   }
+#undef TL_DG
 }
 
 }  // namespace tl

@@ -1,5 +1,5 @@
-// Weight packer (group-wise symmetric INT4 / INT3) and per-(token, head) INT8
-// KV quantisation.
+// Weight packer (group-wise symmetric INT4 / INT3, and the sign-of-frac bits
+// of cross-iteration rounding) and per-(token, head) INT8 KV quantisation.
 //
 // INT4 follows the low-bit body format of "TinyLoop Framework" ("What Makes It
 // Different": INT2/INT4 execution); INT3 follows "Current Status", core
@@ -87,6 +87,30 @@ __global__ void pack_int3_words_kernel(const float* __restrict__ w, int K, int G
   packed[i] = word;
 }
 
+// One thread per sign word: bit e of word j of a row is 1 when the fp32
+// quotient w / s of element 32 j + e lies above its code (the same quotient
+// and code as the packer's), 0 otherwise and past K.
+__global__ void pack_sign_bits_kernel(const float* __restrict__ w, int K, int G, int spr,
+                                      long n_words, float qmin, float qmax,
+                                      const __half* __restrict__ scales,
+                                      uint32_t* __restrict__ sign) {
+  long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_words) return;
+  long row = i / spr;
+  int j = (int)(i % spr);
+  uint32_t word = 0;
+  for (int e = 0; e < 32; ++e) {
+    const int k = 32 * j + e;
+    if (k >= K) break;
+    const float s = __half2float(scales[row * (K / G) + k / G]);
+    if (s == 0.0f) continue;
+    const float r = __fdiv_rn(w[row * (long)K + k], s);
+    const float c = fminf(fmaxf(rintf(r), qmin), qmax);
+    if (r > c) word |= 1u << e;
+  }
+  sign[i] = word;
+}
+
 __global__ void unpack_kernel(const uint32_t* __restrict__ packed, int K, int bits, int wpr,
                               long n_words, int8_t* __restrict__ codes) {
   long i = (long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -154,6 +178,17 @@ tl_status launch_pack(const float* w, int N, int K, int bits, int group, uint32_
     pack_int3_words_kernel<<<blocks_for(n_words, 256), 256, 0, s>>>(w, K, group, wpr, n_words,
                                                                      sc, packed);
   }
+  TL_LAUNCH_CHECK();
+  return ok();
+}
+
+tl_status launch_pack_sign_bits(const float* w, int N, int K, int bits, int group,
+                               const uint16_t* scales, uint32_t* sign, cudaStream_t s) {
+  const int spr = (K + 31) / 32;
+  const long n_words = (long)N * spr;
+  pack_sign_bits_kernel<<<blocks_for(n_words, 256), 256, 0, s>>>(
+      w, K, group, spr, n_words, bits == 4 ? -8.0f : -4.0f, bits == 4 ? 7.0f : 3.0f,
+      reinterpret_cast<const __half*>(scales), sign);
   TL_LAUNCH_CHECK();
   return ok();
 }

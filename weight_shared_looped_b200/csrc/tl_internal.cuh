@@ -74,6 +74,8 @@ tl_status launch_pack(const float* w, int N, int K, int bits, int group, uint32_
                       uint16_t* scales, cudaStream_t s);
 tl_status launch_unpack(const uint32_t* packed, int N, int K, int bits, int8_t* codes,
                         cudaStream_t s);
+tl_status launch_pack_sign_bits(const float* w, int N, int K, int bits, int group,
+                               const uint16_t* scales, uint32_t* sign, cudaStream_t s);
 tl_status launch_kv_quant_int8(const __half* x, int rows, int hd, int8_t* codes, __half* scales,
                                cudaStream_t s);
 
@@ -84,6 +86,11 @@ struct GemmArgs {
   const __half* s0;
   const uint32_t* w1;   // rows [n_split, N) (may equal w0 when n_split == N)
   const __half* s1;
+  // sign-of-frac bits of the rows of w0 / w1 (tl_pack_sign_bits layout): when
+  // set, the odd-iteration codes (code + 1 where the bit is set, code - 1
+  // where clear) are used; tensor-core kernel only
+  const uint32_t* g0;
+  const uint32_t* g1;
   int n_split;
   int N, K, G;
   const __half* x;      // fp16 [T][K]
@@ -104,12 +111,12 @@ tl_status check_linear(int N, int K, int group, int T);
 // Split count of the kernel launch_gemm picks for (N, K, T): the tensor-core
 // kernel for T >= 64, the mma.sync register-dequant kernel below that (the
 // decode projections use launch_dec_gemv instead).
-int gemm_splits(int N, int K, int T, int bits = 4);
+int gemm_splits(int N, int K, int T, int bits = 4, bool sign = false);
 tl_status launch_gemm(const GemmArgs& a, cudaStream_t s);
 // the two kernels
 int gemm_mma_splits(int N, int K, int T);
 tl_status launch_gemm_mma(const GemmArgs& a, cudaStream_t s);
-bool gemm_tc_eligible(int N, int K, int T, int bits = 4);
+bool gemm_tc_eligible(int N, int K, int T, int bits = 4, bool sign = false);
 int gemm_tc_splits(int N, int K, int T);
 tl_status launch_gemm_tc(const GemmArgs& a, cudaStream_t s);
 tl_status gemm_tc_init();
@@ -125,6 +132,8 @@ struct DecGemvArgs {
   const __half* s0;     // fp16 scales [N][K/G]
   const uint32_t* w1;   // DEC_EPI_SWIGLU: the up matrix (w0 = gate)
   const __half* s1;
+  const uint32_t* g0;   // null, or the sign-of-frac bits of w0's rows [N][K/32]: the
+  const uint32_t* g1;   //   odd-iteration codes (g1: of w1's rows); K % 128 == 0
   int N, K, G, bits, T;
   const __half* x;      // fp16 [T][K] activations, or null with h set
   const float* h;       // fp32 [T][K] residual stream: x = fp16(rmsnorm(h) * gamma)

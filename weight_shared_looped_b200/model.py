@@ -14,7 +14,8 @@ from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_dec
                tl_kv_reset, tl_kv_set_position, tl_model_create, tl_model_destroy,
                tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
                tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status, tl_extend,
-               tl_greedy_head, tl_spec_step, tl_model_set_exit_threshold, tl_loops_used)
+               tl_greedy_head, tl_spec_step, tl_model_set_exit_threshold, tl_loops_used,
+               tl_sign_bits_bytes, tl_pack_sign_bits, tl_model_set_cross_iter)
 
 MATRICES = ("qkv", "o", "gate", "up", "down")
 
@@ -28,10 +29,12 @@ def _dev(x, dtype=None, device="cuda"):
 
 class DeviceBlock:
     """One block packed on the device from fp32 weights (or from canonical
-    packed words and scales)."""
+    packed words and scales).  With `sign` (fp32 weights) or sign_* arrays in
+    `packed`, the block also carries the sign-of-frac bits of cross-iteration
+    rounding."""
 
     def __init__(self, cfg: Dict, weights: Optional[Dict] = None, packed: Optional[Dict] = None,
-                 stream=None):
+                 stream=None, sign: bool = False):
         self.cfg = dict(cfg)
         self.t: Dict[str, torch.Tensor] = {}
         bits, group = cfg["bits"], cfg["group"]
@@ -39,6 +42,8 @@ class DeviceBlock:
             if packed is not None:
                 self.t[f"w_{name}"] = _dev(packed[f"w_{name}"].view(np.int32), torch.int32)
                 self.t[f"s_{name}"] = _dev(packed[f"s_{name}"].view(np.int16), torch.int16)
+                if f"sign_{name}" in packed:
+                    self.t[f"sign_{name}"] = _dev(packed[f"sign_{name}"].view(np.int32), torch.int32)
             else:
                 w = _dev(weights[f"w_{name}"], torch.float32)
                 n, k = w.shape
@@ -48,6 +53,10 @@ class DeviceBlock:
                 tl_pack_weights(w, bits, group, pw, ps, stream)
                 self.t[f"w_{name}"] = pw.view(n, -1)
                 self.t[f"s_{name}"] = ps.view(n, -1)
+                if sign:
+                    sg = torch.empty(tl_sign_bits_bytes(n, k) // 4, dtype=torch.int32, device="cuda")
+                    tl_pack_sign_bits(w, bits, group, ps, sg, stream)
+                    self.t[f"sign_{name}"] = sg.view(n, -1)
                 del w
         src = packed if packed is not None else weights
         self.t["gamma_attn"] = _dev(src["gamma_attn"], torch.float32)
@@ -84,6 +93,11 @@ class DeviceModel:
     def set_decode_chunks(self, chunks_per_cta: int) -> None:
         """Context chunks one decode-attention CTA streams (0 = automatic)."""
         tl_model_set_decode_chunks(self.handle, chunks_per_cta)
+
+    def set_cross_iter(self, on: bool) -> None:
+        """Cross-iteration rounding: odd loop iterations take the other rounding
+        neighbour of every loop-block weight (needs a loop block with sign bits)."""
+        tl_model_set_cross_iter(self.handle, on)
 
     def set_exit_threshold(self, tau: float) -> None:
         """Per-iteration residual-norm check threshold (< 0: off)."""
