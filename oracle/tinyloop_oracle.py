@@ -437,6 +437,10 @@ class LoopedModel:
         self.embed16 = embed16
         self.cfg = loop.cfg
         self.cross_iter = False   # odd loop iterations use the loop block's odd weights
+        # per-iteration weight variants ("Current Status", architecture-unique
+        # features table, dual-bit and triple-bit weight swap rows): loop
+        # iteration i < len(iter_blocks) runs iter_blocks[i] (None: the loop block)
+        self.iter_blocks: List[Optional[Block]] = []
 
     def odd(self, layer: int) -> bool:
         """Whether layer `layer` is an odd loop iteration run with the odd
@@ -446,8 +450,11 @@ class LoopedModel:
 
     def schedule(self, L: int) -> List[Block]:
         """Block applied at each layer index: the pre-blocks, then the same
-        loop block object L times (weights shared, not copied)."""
-        return self.pre + [self.loop] * L
+        loop block object L times (weights shared, not copied), except the
+        iterations given a variant."""
+        its = [self.iter_blocks[i] if i < len(self.iter_blocks) and self.iter_blocks[i] is not None
+               else self.loop for i in range(L)]
+        return self.pre + its
 
     def embed(self, ids: np.ndarray) -> np.ndarray:
         return self.embed16[np.asarray(ids)].astype(F64)

@@ -677,3 +677,31 @@ def test_cross_iteration_rounding_model():
     y = m2.prefill(ids, 3)
     m2.cross_iter = True
     assert np.array_equal(m2.prefill(ids, 3), y)
+
+
+# ---------------------------------------------------------------- per-iteration weight variants
+
+def test_iteration_variants_are_an_unrolled_stack():
+    """Dual-bit weight swap ("Current Status", architecture-unique features
+    table: a low-bit copy of the loop block for the early iterations, the
+    higher-bit one later): with variants for iterations 0 and 1 the model is
+    the unrolled stack pre, v0, v1, loop, loop; without variants, or with the
+    loop block itself as the variant, nothing changes."""
+    m = _tiny_model()
+    ids = np.array([4, 1, 19, 7], np.int64)
+    base = m.prefill(ids, 4)
+    w = _tiny_weights(61)                        # the loop block's own weights at INT3
+    cfg3 = dict(_tiny_cfg(), bits=3)
+    low = o.Block.from_fp32(_tiny_weights(11 + 50), cfg3)
+    other = o.Block.from_fp32(w, _tiny_cfg())
+    m.iter_blocks = [low, other]
+    got = m.prefill(ids, 4)
+    deep = o.LoopedModel(m.pre + [low, other, m.loop], m.loop, m.gamma_final, m.embed16)
+    assert np.allclose(got, deep.prefill(ids, 1), rtol=0, atol=1e-12)
+    assert not np.allclose(got, base)
+    m.iter_blocks = [None, m.loop]
+    assert np.array_equal(m.prefill(ids, 4), base)
+    m.iter_blocks = [low] * 6                    # variants past L are never reached
+    assert np.allclose(m.prefill(ids, 2),
+                       o.LoopedModel(m.pre + [low], low, m.gamma_final, m.embed16).prefill(ids, 1),
+                       rtol=0, atol=1e-12)
