@@ -548,6 +548,60 @@ def run_spec(model, kv, w, torch, np, dist, world, K=4, L_draft=2, L_verify=8, n
                         "acceptance is what such weights give, not a trained model's"}
 
 
+def run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cfg, hbm, l2_gbs,
+                    blk_bytes, kv_bytes, ids_t):
+    """B = 1 decode (prompt 256, 128 steps, L = 8, FP16 KV) with loop-block
+    weight variants; the bytes per step count each variant's first read from
+    HBM and its further reads from L2."""
+    from weight_shared_looped_b200.model import DeviceBlock, DeviceModel
+    out = {}
+    wl = syn.block_weights(w.shape, w.seed, "loop")
+    signed = DeviceBlock(cfg(4), weights=wl, sign=True)
+    low = DeviceBlock(cfg(3), weights=wl)
+    sign_bytes = sum(tl.tl_sign_bits_bytes(n, k) for n, k in
+                     ((3 * 2048, 2048), (2048, 2048), (8192, 2048), (8192, 2048), (2048, 8192)))
+    low_bytes = block_bytes(tl, 3)
+    cases = {
+        # iterations 1, 3, 5, 7 also read the sign bits
+        "b1_cross_iter": (signed, [], True, 3 * blk_bytes + sign_bytes + kv_bytes,
+                          7 * blk_bytes + 3 * sign_bytes),
+        # iterations 0-3 read the INT3 copy, 4-7 the INT4 block
+        "b1_dual_bit_int3_int4": (blocks["loop"], [low] * 4, False,
+                                  3 * blk_bytes + low_bytes + kv_bytes,
+                                  3 * blk_bytes + 3 * low_bytes),
+    }
+    dids = [ids_t(syn.decode_ids(w)[i:i + 1]) for i in range(w.steps)]
+    for name, (loop_blk, variants, cross, hbm_b, l2_b) in cases.items():
+        m = DeviceModel([blocks["pre0"], blocks["pre1"]], loop_blk, syn.final_gain(w.shape, w.seed),
+                        syn.embedding(w.shape, w.seed), max_tokens=w.seq, max_lanes=1,
+                        max_ctx=w.max_ctx, max_L=8)
+        m.set_cross_iter(cross)
+        m.set_iteration_blocks(variants)
+        kv = m.new_kv([8], max_ctx=w.max_ctx)
+        m.prefill(ids_t(syn.prompt_ids(w)), L=8, kv=kv, lane=0)
+        y1 = torch.empty(1, 2048, dtype=torch.float32, device="cuda")
+        it = iter(range(10 ** 9))
+
+        def dstep():
+            m.decode(kv, dids[next(it) % w.steps], L_per_lane=[8], y_out=y1)
+
+        dstep()
+        kv.set_position(0, w.seq)
+        it = iter(range(10 ** 9))
+        t = max_over_ranks(timed(dstep, w.steps, 0), dist, "cuda")
+        out[name] = {"tok_s": round(w.steps * world / t, 1),
+                     "ms_per_step": round(t / w.steps * 1e3, 4),
+                     "ms_per_step_median": round(timed.last_median_ms, 4),
+                     **decode_roofline(t / w.steps, hbm_b, l2_b, hbm, l2_gbs),
+                     "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
+        kv.close()
+        m.close()
+        torch.cuda.synchronize()
+    signed.close()
+    low.close()
+    return out
+
+
 def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk, cfg, l2_gbs):
     """KV-cached decode throughput: B=1 FP16 KV (prompt 256, 128 steps), B=8
     INT8 KV at context 2048 (64 steps), mixed-depth INT3 lanes (ctx 1024, 32
@@ -592,6 +646,13 @@ def run_decode(model, blocks, syn, tl, torch, np, flush, timed, dist, world, pk,
                         **decode_roofline(t / w.steps, 3 * blk_bytes + kv_bytes, 7 * blk_bytes,
                                           hbm, l2_gbs),
                         "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
+
+    # the same B = 1 workload with per-iteration weight variants of the loop
+    # block ("Current Status", architecture-unique features table): cross-
+    # iteration rounding (odd iterations add the sign-of-frac bits) and the
+    # dual-bit swap (an INT3 copy for iterations 0-3, the INT4 block for 4-7)
+    out.update(run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cfg,
+                               hbm, l2_gbs, blk_bytes, kv_bytes, ids_t))
 
     # self-speculative decode on the same cache ("Current Status", self-speculative
     # row: L=2 draft, L=8 verify, same weights): greedy tokens through the tied

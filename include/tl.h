@@ -276,6 +276,21 @@ tl_status tl_model_set_exit_threshold(tl_model* model, float tau);
  * model or when the loop block has no sign bits. */
 tl_status tl_model_set_cross_iter(tl_model* model, int on);
 
+/* Per-iteration weight variants ("Current Status", architecture-unique
+ * features table, dual-bit and triple-bit weight swap rows: a low-bit copy of
+ * the loop block for the early iterations, a higher-bit one for the later
+ * iterations, optionally a third for iteration 0).  Loop iteration i < n runs
+ * blocks[i] instead of the loop block (NULL entries keep the loop block);
+ * iterations >= n and the pre-blocks are unchanged.  Each block must have the
+ * loop block's d_model, n_heads, head_dim, ffn, eps and rope_theta; its bits
+ * (3 or 4) and group may differ.  The blocks are referenced, not copied, and
+ * must outlive the model (or the next call).  n = 0 clears the variants.
+ * With cross-iteration rounding on, an odd iteration uses the sign bits of the
+ * block it runs, if that block has them.  Frees the model's captured graphs.
+ * Errors: TL_ERR_INVALID_ARG for a NULL model, n < 0 or n > max_L, a NULL
+ * `blocks` with n > 0, or a block of another shape. */
+tl_status tl_model_set_iteration_blocks(tl_model* model, tl_block* const* blocks, int n);
+
 /* Loop iterations each output row of the last forward call ran (after the
  * stream's work): the loop count L unless the residual-norm check stopped it
  * earlier.  Rows are tokens for tl_prefill / tl_extend and lanes for

@@ -75,6 +75,7 @@ _SIGS = {
     "tl_model_set_decode_chunks": ([P, I], I),
     "tl_model_set_exit_threshold": ([P, F], I),
     "tl_model_set_cross_iter": ([P, I], I),
+    "tl_model_set_iteration_blocks": ([P, P, I], I),
     "tl_loops_used": ([P, P, I, P], I),
     "tl_kv_layer_bytes": ([I, I, I, I, ctypes.POINTER(SZ)], I),
     "tl_kv_bytes": ([P, I, I, P, I, ctypes.POINTER(SZ)], I),
@@ -243,6 +244,13 @@ def tl_model_set_exit_threshold(model: int, tau: float) -> None:
 
 def tl_model_set_cross_iter(model: int, on: bool) -> None:
     _check(lib.tl_model_set_cross_iter(model, 1 if on else 0))
+
+
+def tl_model_set_iteration_blocks(model: int, blocks: Sequence[Optional[int]]) -> None:
+    """Loop iteration i < len(blocks) runs blocks[i] (None: the loop block)."""
+    arr = (P * max(1, len(blocks)))(*[b or None for b in blocks])
+    _check(lib.tl_model_set_iteration_blocks(model, ctypes.cast(arr, P) if blocks else None,
+                                             len(blocks)))
 
 
 def tl_loops_used(model: int, n: int, stream=None):

@@ -99,6 +99,7 @@ struct tl_model {
   int decode_chunks = 0;   // context chunks per decode-attention CTA; 0 = automatic
   float exit_tau = -1.f;   // per-iteration residual-norm check threshold; < 0 = off
   bool cross_iter = false; // odd loop iterations take the loop block's other rounding neighbours
+  std::vector<const tl_block*> iter_blocks;   // loop iteration i < size(): this block (if set)
   cudaStream_t cap_stream = nullptr;
   // workspace
   void* ws = nullptr;
@@ -473,6 +474,25 @@ TL_API tl_status tl_model_set_cross_iter(tl_model* model, int on) {
   return ok();
 }
 
+TL_API tl_status tl_model_set_iteration_blocks(tl_model* model, tl_block* const* blocks, int n) {
+  TL_CHECK_ARG(model, "NULL model");
+  TL_CHECK_ARG(n >= 0 && n <= model->desc.max_L, "n = %d out of [0, max_L = %d]", n,
+               model->desc.max_L);
+  TL_CHECK_ARG(n == 0 || blocks, "blocks is NULL");
+  const tl_block_desc& L = model->loop->d;
+  for (int i = 0; i < n; ++i) {
+    if (!blocks[i]) continue;
+    const tl_block_desc& b = blocks[i]->d;
+    TL_CHECK_ARG(b.d_model == L.d_model && b.n_heads == L.n_heads && b.head_dim == L.head_dim &&
+                     b.ffn == L.ffn && b.eps == L.eps && b.rope_theta == L.rope_theta,
+                 "iteration %d: the block's shape differs from the loop block's", i);
+  }
+  model->iter_blocks.assign(n, nullptr);
+  for (int i = 0; i < n; ++i) model->iter_blocks[i] = blocks[i];
+  free_graphs(model);   // captured graphs hold the old weights
+  return ok();
+}
+
 TL_API tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream) {
   TL_CHECK_ARG(model && loops, "NULL argument");
   TL_CHECK_ARG(n >= 1 && n <= std::max(model->Tmax, kMaxLanes), "n = %d out of range", n);
@@ -638,8 +658,12 @@ TL_API tl_status tl_kv_layer_ptrs(const tl_kv* kv, int lane, int layer, void** k
 // ============================================================================
 namespace {
 
+// The block layer `layer` runs: a pre-block, a per-iteration variant, or the
+// loop block.
 const tl_block* block_at(const tl_model* m, int layer) {
-  return layer < (int)m->pre.size() ? m->pre[layer] : m->loop;
+  if (layer < (int)m->pre.size()) return m->pre[layer];
+  const size_t it = (size_t)(layer - (int)m->pre.size());
+  return it < m->iter_blocks.size() && m->iter_blocks[it] ? m->iter_blocks[it] : m->loop;
 }
 
 // Whether layer `layer` is an odd loop iteration run with the other rounding

@@ -15,7 +15,8 @@ from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_dec
                tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
                tl_pack_weights, tl_packed_bytes, tl_prefill, tl_sync_status, tl_extend,
                tl_greedy_head, tl_spec_step, tl_model_set_exit_threshold, tl_loops_used,
-               tl_sign_bits_bytes, tl_pack_sign_bits, tl_model_set_cross_iter)
+               tl_sign_bits_bytes, tl_pack_sign_bits, tl_model_set_cross_iter,
+               tl_model_set_iteration_blocks)
 
 MATRICES = ("qkv", "o", "gate", "up", "down")
 
@@ -98,6 +99,12 @@ class DeviceModel:
         """Cross-iteration rounding: odd loop iterations take the other rounding
         neighbour of every loop-block weight (needs a loop block with sign bits)."""
         tl_model_set_cross_iter(self.handle, on)
+
+    def set_iteration_blocks(self, blocks: Sequence[Optional[DeviceBlock]]) -> None:
+        """Per-iteration weight variants: loop iteration i < len(blocks) runs
+        blocks[i] (None keeps the loop block)."""
+        tl_model_set_iteration_blocks(self.handle, [b.handle if b else None for b in blocks])
+        self._iter_blocks = list(blocks)   # referenced by the library: keep them alive
 
     def set_exit_threshold(self, tau: float) -> None:
         """Per-iteration residual-norm check threshold (< 0: off)."""
