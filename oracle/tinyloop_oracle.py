@@ -321,17 +321,24 @@ class Block:
         and present, else the standard one."""
         return self.W_odd if odd and self.W_odd is not None else self.W
 
-    def qkv(self, h: np.ndarray, positions: np.ndarray, odd: bool = False):
-        """RMSNorm -> QKV projection -> RoPE on q and k."""
+    def x_in(self, h: np.ndarray) -> np.ndarray:
+        """The input of the QKV projection: RMSNorm(h) * gamma_attn."""
+        return rmsnorm(h, self.gamma_attn, self.cfg["eps"])
+
+    def qkv_from_x(self, x: np.ndarray, positions: np.ndarray, odd: bool = False):
+        """QKV projection of x -> RoPE on q and k."""
         c = self.cfg
-        t = h.shape[0]
-        x = rmsnorm(h, self.gamma_attn, c["eps"])
+        t = x.shape[0]
         qkv = x @ self.weights(odd)["qkv"].T
         d, nh, hd = c["d_model"], c["n_heads"], c["head_dim"]
         q = qkv[:, :d].reshape(t, nh, hd)
         k = qkv[:, d:2 * d].reshape(t, nh, hd)
         v = qkv[:, 2 * d:].reshape(t, nh, hd)
         return rope(q, positions, c["rope_theta"]), rope(k, positions, c["rope_theta"]), v
+
+    def qkv(self, h: np.ndarray, positions: np.ndarray, odd: bool = False):
+        """RMSNorm -> QKV projection -> RoPE on q and k."""
+        return self.qkv_from_x(self.x_in(h), positions, odd)
 
     def finish(self, h: np.ndarray, attn: np.ndarray, odd: bool = False) -> np.ndarray:
         """O projection + residual, then RMSNorm -> SwiGLU MLP + residual."""
@@ -362,15 +369,26 @@ def pack_block(weights: Dict[str, np.ndarray], bits: int, group: int,
 
 class KVSlot:
     """K/V of one layer (one pre-block or one loop iteration) for one lane, in
-    the cache's storage dtype: "fp16", "int8" or "exact" (fp64, used only to
-    check the cached path against the uncached one without storage rounding).
-    Stored values are kept dequantised, positions 0..len-1."""
+    the cache's storage dtype: "fp16", "int8", "exact" (fp64, used only to
+    check the cached path against the uncached one without storage rounding)
+    or "h".  Stored values are kept dequantised, positions 0..len-1.
+
+    "h" is the store-h mode ("Current Status", KV cache mode table, Store-h
+    (FP16) and tensor-core reconstruction rows; "Claims & Data Sources", the
+    h-mode KV reconstruction from shared W_k / W_v row).  Reading: the slot
+    keeps, per position, the fp16 rounding of the input the layer's QKV
+    projection reads (x = RMSNorm(h) * gamma_attn: d values instead of the 2d
+    of K and V); K and V are rebuilt from those rows with the layer's own
+    W_k, W_v and RoPE whenever they are read, with no further rounding."""
 
     def __init__(self, dtype: str):
         self.dtype = dtype
         self._k: Optional[np.ndarray] = None
         self._v: Optional[np.ndarray] = None
         self.n = 0
+        self._x: Optional[np.ndarray] = None   # "h": the stored fp16 input rows
+        self._blk: Optional["Block"] = None
+        self._odd = False
 
     def _store(self, x: np.ndarray) -> np.ndarray:
         if self.dtype == "exact":
@@ -410,16 +428,32 @@ class KVSlot:
         self._v[:v_values.shape[0]] = v_values
         self.n = k_values.shape[0]
 
+    def append_x(self, x: np.ndarray, blk: "Block", odd: bool) -> None:
+        """Store-h: append T input rows x [T, d] (kept as fp16), to be projected
+        by `blk` (odd-iteration weights when `odd`)."""
+        x16 = np.asarray(x, F64).astype(np.float16)
+        self._x = x16 if self._x is None else np.concatenate([self._x[:self.n], x16])
+        self._blk, self._odd = blk, odd
+        self.n += x16.shape[0]
+
+    def _rebuild(self):
+        _, k, v = self._blk.qkv_from_x(self._x[:self.n].astype(F64), np.arange(self.n), self._odd)
+        return k, v
+
     def truncate(self, n: int) -> None:
         """Keep positions 0..n-1 (entries past them are dropped)."""
         self.n = min(self.n, n)
 
     @property
     def k(self) -> np.ndarray:
+        if self.dtype == "h":
+            return self._rebuild()[0]
         return self._k[:self.n]
 
     @property
     def v(self) -> np.ndarray:
+        if self.dtype == "h":
+            return self._rebuild()[1]
         return self._v[:self.n]
 
     def __len__(self) -> int:
@@ -496,7 +530,10 @@ class LoopedModel:
             odd = self.odd(layer)
             q, k, v = blk.qkv(h, pos, odd)
             if kv is not None:
-                kv[layer].append(k, v)
+                if kv[layer].dtype == "h":
+                    kv[layer].append_x(blk.x_in(h), blk, odd)
+                else:
+                    kv[layer].append(k, v)
             h = np.where(frozen[:, None], h, blk.finish(h, causal_attention(q, k, v, pos), odd))
             if trace is not None:
                 trace.append(h.copy())
@@ -523,7 +560,10 @@ class LoopedModel:
             odd = self.odd(layer)
             q, k, v = blk.qkv(h, pos, odd)
             slot = kv[layer]
-            slot.append(k, v)
+            if slot.dtype == "h":
+                slot.append_x(blk.x_in(h), blk, odd)
+            else:
+                slot.append(k, v)
             h = np.where(frozen[:, None], h,
                          blk.finish(h, causal_attention(q, slot.k, slot.v, pos), odd))   # keys 0..pos
             if trace is not None:

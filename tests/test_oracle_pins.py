@@ -266,8 +266,11 @@ def _tiny_weights(seed):
     return w
 
 
-def _block_brute(blk, h, pos0=0):
-    """One block by explicit loops over indices, from the dequantised weights."""
+def _block_brute(blk, h, pos0=0, kv_from_fp16_x=False):
+    """One block by explicit loops over indices, from the dequantised weights.
+    With kv_from_fp16_x, K and V are projected from the fp16 rounding of the
+    normalised input (the store-h cache's stored rows), q from the input
+    itself."""
     c = blk.cfg
     d, nh, hd, f = c["d_model"], c["n_heads"], c["head_dim"], c["ffn"]
     W = blk.W
@@ -286,11 +289,12 @@ def _block_brute(blk, h, pos0=0):
     for ti in range(t):
         x = norm(list(h[ti]), blk.gamma_attn)
         y = mv(W["qkv"], x)
+        ykv = mv(W["qkv"], [float(np.float16(e)) for e in x]) if kv_from_fp16_x else y
         for hh in range(nh):
             for e in range(hd):
                 q[ti][hh][e] = y[hh * hd + e]
-                k[ti][hh][e] = y[d + hh * hd + e]
-                v[ti][hh][e] = y[2 * d + hh * hd + e]
+                k[ti][hh][e] = ykv[d + hh * hd + e]
+                v[ti][hh][e] = ykv[2 * d + hh * hd + e]
         for arr in (q, k):
             for hh in range(nh):
                 vec = list(arr[ti][hh])
@@ -705,3 +709,52 @@ def test_iteration_variants_are_an_unrolled_stack():
     assert np.allclose(m.prefill(ids, 2),
                        o.LoopedModel(m.pre + [low], low, m.gamma_final, m.embed16).prefill(ids, 1),
                        rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- store-h KV
+
+def test_store_h_decode_brute_force():
+    """Store-h ("Current Status", KV cache mode table, Store-h rows): a
+    one-block model caches the fp16 rows x of each position; a decode step
+    rebuilds every position's K and V from them.  Against explicit loops over
+    the whole sequence with K, V projected from fp16(x) (q from x itself)."""
+    cfg = _tiny_cfg()
+    blk = o.Block.from_fp32(_tiny_weights(71), cfg)
+    gam = 1 + 0.1 * np.random.default_rng(72).standard_normal(8)
+    m = o.LoopedModel([], blk, gam)
+    h = np.random.default_rng(73).standard_normal((6, 8))
+    kv = m.new_kv(1, "h")
+    m.prefill(h[:5], 1, kv=kv)
+    tr = []
+    m.decode_step(h[5], 1, kv, trace=tr)
+    want = _block_brute(blk, h, kv_from_fp16_x=True)[5]
+    assert np.allclose(tr[0][0], want, rtol=0, atol=1e-12)
+    # the rounding of x is what the mode stores: the exact-cache result differs
+    kv_exact = m.new_kv(1, "exact")
+    m.prefill(h[:5], 1, kv=kv_exact)
+    tr_exact = []
+    m.decode_step(h[5], 1, kv_exact, trace=tr_exact)
+    assert np.allclose(tr_exact[0][0], _block_brute(blk, h)[5], rtol=0, atol=1e-12)
+    assert not np.array_equal(tr[0][0], tr_exact[0][0])
+    assert np.allclose(tr[0][0], tr_exact[0][0], rtol=0, atol=1e-2)
+    # the slot holds d fp16 values per position (K and V would take 2d)
+    assert kv[0]._x.dtype == np.float16 and kv[0]._x[:kv[0].n].shape == (6, 8)
+
+
+def test_store_h_cross_iteration_uses_odd_weights():
+    """An odd loop iteration's slot rebuilds K and V with that iteration's
+    weights."""
+    m, w = _sign_model()
+    m.cross_iter = True
+    ids = np.array([2, 5, 8, 13], np.int64)
+    kv_h, kv_e = m.new_kv(2, "h"), m.new_kv(2, "exact")
+    m.prefill(ids[:3], 2, kv=kv_h)
+    m.prefill(ids[:3], 2, kv=kv_e)
+    a = m.decode_step(ids[3], 2, kv_h)
+    b = m.decode_step(ids[3], 2, kv_e)
+    assert np.allclose(a, b, rtol=0, atol=5e-2)
+    for layer in (1, 2):
+        k_h = kv_h[layer].k
+        x16 = kv_h[layer]._x[:4].astype(np.float64)
+        _, k_want, _ = (m.loop.qkv_from_x(x16, np.arange(4), odd=(layer == 2)))
+        assert np.array_equal(k_h, k_want), layer
