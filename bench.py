@@ -571,13 +571,22 @@ def run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cf
                                   3 * blk_bytes + 3 * low_bytes),
     }
     dids = [ids_t(syn.decode_ids(w)[i:i + 1]) for i in range(w.steps)]
-    for name, (loop_blk, variants, cross, hbm_b, l2_b) in cases.items():
+    # store-h KV: the cache keeps the fp16 QKV-input rows, each step rebuilds K
+    # and V with the quantised-weight GEMM (its weight reads: W_k, W_v rows)
+    qkv_kv_bytes = 2 * (2048 * 2048 // 2 + 2048 * 16 * 2)
+    avg_ctx = w.seq + (w.steps + 1) / 2
+    cases["b1_store_h"] = (blocks["loop"], [], False, 3 * blk_bytes + kv_bytes / 2,
+                           7 * blk_bytes + 10 * qkv_kv_bytes, "h",
+                           round(10 * avg_ctx * 2 * 2048 * 2048 * 2 / 1e9, 2))
+    for name, case in cases.items():
+        loop_blk, variants, cross, hbm_b, l2_b = case[:5]
+        kv_dtype = case[5] if len(case) > 5 else "fp16"
         m = DeviceModel([blocks["pre0"], blocks["pre1"]], loop_blk, syn.final_gain(w.shape, w.seed),
                         syn.embedding(w.shape, w.seed), max_tokens=w.seq, max_lanes=1,
                         max_ctx=w.max_ctx, max_L=8)
         m.set_cross_iter(cross)
         m.set_iteration_blocks(variants)
-        kv = m.new_kv([8], max_ctx=w.max_ctx)
+        kv = m.new_kv([8], max_ctx=w.max_ctx, dtype=kv_dtype)
         m.prefill(ids_t(syn.prompt_ids(w)), L=8, kv=kv, lane=0)
         y1 = torch.empty(1, 2048, dtype=torch.float32, device="cuda")
         it = iter(range(10 ** 9))
@@ -594,6 +603,13 @@ def run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cf
                      "ms_per_step_median": round(timed.last_median_ms, 4),
                      **decode_roofline(t / w.steps, hbm_b, l2_b, hbm, l2_gbs),
                      "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
+        if kv_dtype == "h":
+            out[name]["workload"] = ("prompt 256 + 128 steps, L=8, store-h cache (fp16 QKV-input "
+                                     "rows; K and V rebuilt every step), batch 1, no CUDA graph")
+            out[name]["rebuild_gflop_per_step"] = case[6]
+            out[name]["cache_bytes"] = tl.tl_kv_bytes(m.handle, w.max_ctx, [8], tl.TL_KV_H)
+            out[name]["cache_bytes_fp16_kv"] = tl.tl_kv_bytes(m.handle, w.max_ctx, [8],
+                                                              tl.TL_KV_FP16)
         kv.close()
         m.close()
         torch.cuda.synchronize()

@@ -51,7 +51,10 @@ typedef enum tl_status {
 
 typedef enum tl_kv_dtype {
   TL_KV_FP16 = 0,  /* K and V as fp16 */
-  TL_KV_INT8 = 1   /* int8 codes + one fp16 scale per (token, head) */
+  TL_KV_INT8 = 1,  /* int8 codes + one fp16 scale per (token, head) */
+  TL_KV_H = 2      /* store-h: the fp16 input rows x of each block application;
+                    * K and V are rebuilt from them at every decode step (see
+                    * tl_kv_create) */
 } tl_kv_dtype;
 
 /* Description of the last failure on this thread ("" if none). */
@@ -311,11 +314,25 @@ tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream);
  * [H][max_ctx][hd] (fp16, or int8 codes), then for INT8 the scales K
  * [H][max_ctx], V [H][max_ctx] (fp16); every region starts on 256 bytes.
  * K is stored after RoPE.
+ *
+ * TL_KV_H (store-h: "Current Status", KV cache mode table, Store-h (FP16) and
+ * tensor-core reconstruction rows; "Claims & Data Sources", h-mode KV
+ * reconstruction from shared W_k / W_v): a slot holds, per position, the fp16
+ * row x = RMSNorm(h) * gamma_attn that the layer's QKV projection read
+ * ([max_ctx][d], d values instead of the 2d of K and V).  At every decode step
+ * each layer rebuilds the K and V of a lane's cached positions from those
+ * rows with the layer's own W_k, W_v (the quantised-weight GEMM on the tensor
+ * cores, RoPE after it) into a workspace that follows the slots in the same
+ * buffer (a header, one fp16 K/V layer per lane and the GEMM's partial sums),
+ * then attends over them.  Prefill and decode steps support it; tl_extend and
+ * tl_spec_step return TL_ERR_UNSUPPORTED, and decode steps run without CUDA
+ * graphs (the rebuild's size changes with every position).
  * ------------------------------------------------------------------------ */
 typedef struct tl_kv tl_kv;
 
 /* Bytes of one (lane, layer) slot: 2 * align256(H * max_ctx * hd * elem)
- * plus, for INT8, 2 * align256(H * max_ctx * 2) of fp16 scales.  Host-only. */
+ * plus, for INT8, 2 * align256(H * max_ctx * 2) of fp16 scales; for TL_KV_H
+ * align256(max_ctx * H * hd * 2).  Host-only. */
 tl_status tl_kv_layer_bytes(int n_heads, int head_dim, int max_ctx, tl_kv_dtype dtype,
                             size_t* bytes);
 
@@ -336,7 +353,8 @@ tl_status tl_kv_position(const tl_kv* kv, int lane, int* pos);
  * cache filled by the caller through tl_kv_layer_ptrs). */
 tl_status tl_kv_set_position(tl_kv* kv, int lane, int pos, tl_stream stream);
 /* Device pointers of one (lane, layer) slot: K, V ([H][max_ctx][hd]) and, for
- * INT8, the scales ([H][max_ctx]; NULL for FP16). */
+ * INT8, the scales ([H][max_ctx]; NULL for FP16).  TL_KV_H: *k receives the
+ * fp16 rows x [max_ctx][d]; *v and the scales are NULL. */
 tl_status tl_kv_layer_ptrs(const tl_kv* kv, int lane, int layer, void** k,
                            void** v, uint16_t** k_scale, uint16_t** v_scale);
 

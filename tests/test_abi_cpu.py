@@ -69,6 +69,14 @@ def test_kv_layer_bytes_match_pages_figures():
     assert round(fp16 / 1e6, 1) == 167.8 and round(int8 / 1e6, 1) == 85.2
 
 
+def test_store_h_slot_is_half_the_fp16_slot():
+    # store-h keeps d fp16 values per position instead of the 2d of K and V
+    # ("Current Status", KV cache mode table, Store-h (FP16): 43-50 % saving)
+    h = 10 * tl.tl_kv_layer_bytes(16, 128, 2048, tl.TL_KV_H)
+    fp16 = 10 * tl.tl_kv_layer_bytes(16, 128, 2048, tl.TL_KV_FP16)
+    assert h * 2 == fp16 and h == 10 * 2048 * 2048 * 2
+
+
 @pytest.mark.parametrize("args,status", [
     ((64, 128, 5, 64), tl.TL_ERR_UNSUPPORTED),     # bits
     ((64, 128, 4, 32), tl.TL_ERR_UNSUPPORTED),     # group

@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(HERE, "libtinyloop_b200.so")
 
 TL_OK, TL_ERR_INVALID_ARG, TL_ERR_CUDA, TL_ERR_OOM, TL_ERR_TIMEOUT, TL_ERR_UNSUPPORTED, \
     TL_ERR_NUMERIC = range(7)
-TL_KV_FP16, TL_KV_INT8 = 0, 1
+TL_KV_FP16, TL_KV_INT8, TL_KV_H = 0, 1, 2
 STATUS_NAMES = {0: "TL_OK", 1: "TL_ERR_INVALID_ARG", 2: "TL_ERR_CUDA", 3: "TL_ERR_OOM",
                 4: "TL_ERR_TIMEOUT", 5: "TL_ERR_UNSUPPORTED", 6: "TL_ERR_NUMERIC"}
 

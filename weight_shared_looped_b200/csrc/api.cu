@@ -75,6 +75,13 @@ struct tl_kv {
   int pos[kMaxLanes];
   char* buffer;
   size_t layer_bytes, region_bytes;
+  // store-h workspace (TL_KV_H), after the slots in the same buffer: a header
+  // whose cum_layers are 0, 1, 2, ..., one fp16 K/V layer per lane (the
+  // rebuilt entries) and the rebuild GEMM's partial sums
+  KvHeader* h_hdr = nullptr;
+  char* h_kv = nullptr;
+  float* h_part = nullptr;
+  size_t h_layer_bytes = 0, h_region_bytes = 0;
 };
 
 struct RowMap {
@@ -517,6 +524,11 @@ TL_API tl_status tl_model_set_decode_chunks(tl_model* model, int chunks_per_cta)
 namespace {
 
 void kv_geometry_hd(int H, int hd, int max_ctx, int dtype, size_t* layer, size_t* region) {
+  if (dtype == TL_KV_H) {   // the fp16 input rows x [max_ctx][H * hd]
+    *region = align256((size_t)max_ctx * H * hd * 2);
+    *layer = *region;
+    return;
+  }
   size_t esz = dtype == TL_KV_INT8 ? 1 : 2;
   size_t r = align256((size_t)H * max_ctx * hd * esz);
   size_t l = 2 * r;
@@ -529,6 +541,23 @@ void kv_geometry(const tl_model* m, int max_ctx, int dtype, size_t* layer, size_
   kv_geometry_hd(m->H, m->hd, max_ctx, dtype, layer, region);
 }
 
+// Store-h workspace bytes (after the slots): header, one fp16 K/V layer per
+// lane, and the rebuild GEMM's partial sums for up to kRebuildRows rows (the
+// largest split count x rows over every row count and weight format).
+constexpr int kRebuildRows = 512;   // positions per rebuild GEMM
+
+size_t h_workspace_bytes(const tl_model* m, int n_lanes, int max_ctx, size_t* layer16,
+                         size_t* region16, size_t* part_off) {
+  kv_geometry(m, max_ctx, TL_KV_FP16, layer16, region16);
+  size_t part = 0;
+  for (int T = 1; T <= std::min(max_ctx, kRebuildRows); ++T)
+    for (int bits = 3; bits <= 4; ++bits)
+      for (int sg = 0; sg <= 1; ++sg)
+        part = std::max(part, (size_t)gemm_splits(2 * m->d, m->d, T, bits, sg != 0) * T);
+  *part_off = kKvHeaderBytes + (size_t)n_lanes * *layer16;
+  return *part_off + align256(part * 2 * m->d * sizeof(float));
+}
+
 tl_status check_kv_args(const tl_model* m, int n_lanes, int max_ctx, const int* L, int dtype) {
   TL_CHECK_ARG(m, "NULL model");
   TL_CHECK_ARG(n_lanes >= 1 && n_lanes <= kMaxLanes, "n_lanes = %d out of [1, %d]", n_lanes,
@@ -539,7 +568,8 @@ tl_status check_kv_args(const tl_model* m, int n_lanes, int max_ctx, const int* 
   for (int b = 0; b < n_lanes; ++b)
     TL_CHECK_ARG(L[b] >= 1 && L[b] <= m->desc.max_L, "L_per_lane[%d] = %d out of [1, %d]", b,
                  L[b], m->desc.max_L);
-  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8, "unknown KV dtype %d", dtype);
+  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8 || dtype == TL_KV_H,
+               "unknown KV dtype %d", dtype);
   return ok();
 }
 
@@ -549,7 +579,8 @@ TL_API tl_status tl_kv_layer_bytes(int n_heads, int head_dim, int max_ctx, tl_kv
                                    size_t* bytes) {
   TL_CHECK_ARG(bytes, "bytes is NULL");
   TL_CHECK_ARG(n_heads >= 1 && head_dim >= 1 && max_ctx >= 1, "sizes must be positive");
-  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8, "unknown KV dtype %d", dtype);
+  TL_CHECK_ARG(dtype == TL_KV_FP16 || dtype == TL_KV_INT8 || dtype == TL_KV_H,
+               "unknown KV dtype %d", dtype);
   size_t region;
   kv_geometry_hd(n_heads, head_dim, max_ctx, dtype, bytes, &region);
   return ok();
@@ -564,6 +595,10 @@ TL_API tl_status tl_kv_bytes(const tl_model* model, int n_lanes, int max_ctx,
   size_t layers = 0;
   for (int b = 0; b < n_lanes; ++b) layers += (size_t)model->desc.n_pre + L_per_lane[b];
   *bytes = kKvHeaderBytes + layers * layer;
+  if (dtype == TL_KV_H) {
+    size_t l16, r16, poff;
+    *bytes += h_workspace_bytes(model, n_lanes, max_ctx, &l16, &r16, &poff);
+  }
   return ok();
 }
 
@@ -595,6 +630,19 @@ TL_API tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
     if (b < n_lanes) cum += model->desc.n_pre + L_per_lane[b];
   }
   TL_CUDA(cudaMemcpy(buffer, &hdr, sizeof(hdr), cudaMemcpyHostToDevice));
+  if (dtype == TL_KV_H) {
+    size_t layers = 0, poff = 0;
+    for (int b = 0; b < n_lanes; ++b) layers += (size_t)model->desc.n_pre + L_per_lane[b];
+    char* ws = (char*)buffer + kKvHeaderBytes + layers * kv->layer_bytes;
+    h_workspace_bytes(model, n_lanes, max_ctx, &kv->h_layer_bytes, &kv->h_region_bytes, &poff);
+    kv->h_hdr = (KvHeader*)ws;
+    kv->h_kv = ws + kKvHeaderBytes;
+    kv->h_part = (float*)(ws + poff);
+    KvHeader hh;
+    memset(&hh, 0, sizeof(hh));
+    for (int b = 0; b < kMaxLanes; ++b) hh.cum_layers[b] = b;   // lane b: rebuilt layer b
+    TL_CUDA(cudaMemcpy(kv->h_hdr, &hh, sizeof(hh), cudaMemcpyHostToDevice));
+  }
   *out = kv.release();
   return ok();
 }
@@ -641,7 +689,7 @@ TL_API tl_status tl_kv_layer_ptrs(const tl_kv* kv, int lane, int layer, void** k
   for (int b = 0; b < lane; ++b) cum += kv->model->desc.n_pre + kv->L[b];
   char* base = kv->buffer + kKvHeaderBytes + (size_t)(cum + layer) * kv->layer_bytes;
   *k = base;
-  *v = base + kv->region_bytes;
+  *v = kv->dtype == TL_KV_H ? nullptr : base + kv->region_bytes;
   if (kv->dtype == TL_KV_INT8) {
     size_t sreg = (kv->layer_bytes - 2 * kv->region_bytes) / 2;
     *k_scale = (uint16_t*)(base + 2 * kv->region_bytes);
@@ -756,6 +804,14 @@ NormArgs norm_args(const tl_model* m, int rows) {
 tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows, tl_kv* kv,
                              int lane, cudaStream_t s) {
   const bool odd = odd_iteration(m, layer);
+  const bool store_h = kv && kv->dtype == TL_KV_H;
+  if (store_h) {
+    // store-h: the QKV projection's input rows x go to the slot, positions 0..rows-1
+    int cum = 0;
+    for (int b = 0; b < lane; ++b) cum += (int)m->pre.size() + kv->L[b];
+    char* slot = kv->buffer + kKvHeaderBytes + (size_t)(cum + layer) * kv->layer_bytes;
+    TL_CUDA(cudaMemcpyAsync(slot, m->x, (size_t)rows * m->d * 2, cudaMemcpyDeviceToDevice, s));
+  }
   // QKV
   GemmArgs g = gemm_args(m, b, 0, m->x, rows, odd);
   TL_TRY(launch_gemm(g, s));
@@ -771,7 +827,7 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   r.q = m->q;
   r.k = m->k;
   r.v = m->v;
-  if (kv) {
+  if (kv && !store_h) {
     r.kv_base = kv->buffer + kKvHeaderBytes;
     r.hdr = (const KvHeader*)kv->buffer;
     r.layer_bytes = kv->layer_bytes;
@@ -810,6 +866,62 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   return ok();
 }
 
+// Store-h: rebuild the K/V of every row's lane at positions 0 .. pos - 1 from
+// the slot's fp16 input rows: the quantised-weight GEMM of those rows with the
+// W_k, W_v rows of the layer's QKV matrix (odd-iteration codes when `odd`),
+// then RoPE into the lane's layer of the workspace (fp16, the standard
+// layout the decode attention reads).
+tl_status rebuild_kv(tl_model* m, const tl_block_desc& bd, int layer, int rows, tl_kv* kv,
+                     const RowMap* rm, bool odd, cudaStream_t s) {
+  const int d = m->d;
+  const size_t wpr = (size_t)words_per_row(d, bd.bits), gpr = (size_t)(d / bd.group);
+  for (int i = 0; i < rows; ++i) {
+    const int lane = rm->lane[i];
+    const int pos = kv->pos[lane] + rm->off[i];
+    const __half* slot = (const __half*)(kv->buffer + kKvHeaderBytes +
+                                         (size_t)(rm->cum[i] + layer) * kv->layer_bytes);
+    // positions [p0, p0 + n): one GEMM and one RoPE pass each
+    for (int p0 = 0; p0 < pos; p0 += kRebuildRows) {
+      const int n = std::min(kRebuildRows, pos - p0);
+      GemmArgs g;
+      memset(&g, 0, sizeof(g));
+      g.bits = bd.bits;
+      g.G = bd.group;
+      g.x = slot + (size_t)p0 * d;
+      g.T = n;
+      g.part = kv->h_part;
+      g.w0 = g.w1 = bd.w_qkv + (size_t)d * wpr;   // rows d .. 3d: W_k, W_v
+      g.s0 = g.s1 = (const __half*)bd.s_qkv + (size_t)d * gpr;
+      if (odd && bd.sign_qkv) g.g0 = g.g1 = bd.sign_qkv + (size_t)d * (d / 32);
+      g.N = g.n_split = 2 * d;
+      g.K = d;
+      g.splits = gemm_splits(g.N, g.K, n, g.bits, g.g0 != nullptr);
+      g.status = m->status;
+      TL_TRY(launch_gemm(g, s));
+      RopeKvArgs r;
+      memset(&r, 0, sizeof(r));
+      r.part = kv->h_part;
+      r.S = g.splits;
+      r.rows = n;
+      r.pos0 = p0;
+      r.d = d;
+      r.H = m->H;
+      r.hd = m->hd;
+      r.rope_cs = m->rope;
+      r.kv_base = kv->h_kv;
+      r.hdr = kv->h_hdr;
+      r.layer_bytes = kv->h_layer_bytes;
+      r.kv_region_bytes = kv->h_region_bytes;
+      r.layer = 0;
+      r.max_ctx = kv->max_ctx;
+      r.lane = lane;
+      r.kv_only = 1;
+      TL_TRY(launch_rope_kv(r, s));
+    }
+  }
+  return ok();
+}
+
 // One decode block application for `rows` active rows: four decode
 // projections (the QKV and gate/up ones form their own pre-norm from the
 // residual stream; the O and down ones add into it) around the fused decode
@@ -821,6 +933,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   const tl_block_desc& bd = b->d;
   const int d = m->d, F = m->F;
   const bool odd = odd_iteration(m, layer);
+  const bool store_h = kv->dtype == TL_KV_H;
   DecGemvArgs p;
   memset(&p, 0, sizeof(p));
   p.G = bd.group;
@@ -838,6 +951,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   p.gamma = bd.gamma_attn;
   p.epi = DEC_EPI_OUT;
   p.out = m->part;
+  p.x_out = store_h ? m->x : nullptr;   // store-h: the rows to append to the slots
   {
     const int it = layer - (int)m->pre.size();   // the loop iteration this layer runs
     p.ex = exit_args(m, layer, it >= 1 ? it : 0);
@@ -845,6 +959,8 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   }
   TL_TRY(launch_dec_gemv(p, s));
   p.ex = exit_args(m, layer, 0);
+  p.x_out = nullptr;
+  if (store_h) TL_TRY(rebuild_kv(m, bd, layer, rows, kv, rm, odd, s));
   // RoPE, KV append, split attention and merge in one launch
   DecodeAttnArgs da;
   memset(&da, 0, sizeof(da));
@@ -869,6 +985,16 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   da.qkv_S = 1;
   da.rope_cs = m->rope;
   da.chunks = m->decode_chunks;
+  if (store_h) {
+    // attend over the rebuilt entries: lane b's are layer b of the workspace
+    da.kv_base = kv->h_kv;
+    da.layer_bytes = kv->h_layer_bytes;
+    da.kv_region_bytes = kv->h_region_bytes;
+    da.layer = 0;
+    da.kv_int8 = 0;
+    for (int i = 0; i < kMaxLanes; ++i) da.row_cum[i] = rm->lane[i];
+    da.late_prefetch = 1;
+  }
   if (!split_attn) {
     da.mode = 0;
     TL_TRY(launch_attn_decode_fused(da, s));
@@ -878,6 +1004,15 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
     TL_TRY(launch_attn_decode_fused(da, s));
     da.mode = 2;
     TL_TRY(launch_attn_decode_fused(da, s));
+  }
+  if (store_h) {
+    // this step's input rows join the slots at the rows' positions
+    for (int i = 0; i < rows; ++i) {
+      const int pos = kv->pos[rm->lane[i]] + rm->off[i];
+      char* slot = kv->buffer + kKvHeaderBytes + (size_t)(rm->cum[i] + layer) * kv->layer_bytes;
+      TL_CUDA(cudaMemcpyAsync(slot + (size_t)pos * d * 2, m->x + (size_t)i * d, (size_t)d * 2,
+                              cudaMemcpyDeviceToDevice, s));
+    }
   }
   // O projection, added into the residual stream
   p.w0 = bd.w_o;
@@ -1185,7 +1320,8 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
                     std::to_string(ids ? 1 : 0) + "|" + std::to_string((uintptr_t)h_trace);
   for (int b = 0; b < n_lanes; ++b) key += "|" + std::to_string(L_per_lane[b]);
   const bool use_ids = ids != nullptr;
-  if (model->graphs) {
+  // store-h: the rebuild's row counts follow the positions, so no graph
+  if (model->graphs && kv->dtype != TL_KV_H) {
     TL_TRY(run_graph(
         model, key, kv->id, s,
         [&](cudaStream_t cs, int32_t* lmap) {
@@ -1214,6 +1350,8 @@ tl_status check_extend(tl_model* model, tl_kv* kv, int lane, int n, int L) {
   TL_CHECK_ARG(L >= 1 && L <= kv->L[lane], "L = %d out of [1, %d] for lane %d", L, kv->L[lane], lane);
   TL_CHECK_ARG(kv->pos[lane] + n <= kv->max_ctx, "lane %d: %d + %d positions exceed %d", lane,
                kv->pos[lane], n, kv->max_ctx);
+  if (kv->dtype == TL_KV_H)
+    return set_error(TL_ERR_UNSUPPORTED, "extend and speculative steps need a K/V cache, not store-h");
   return ok();
 }
 

@@ -448,13 +448,14 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   };
   // the first stages are copied before the wait for the previous kernel: they
   // hold entries of earlier steps only -- except in mode 2, where the
-  // previous kernel appended some of them, and mode 1, which copies nothing
-  if (a.mode == 0) {
+  // previous kernel appended some of them, with late_prefetch, where the
+  // previous kernels rebuilt them, and in mode 1, which copies nothing
+  if (a.mode == 0 && !a.late_prefetch) {
 #pragma unroll
     for (int st = 0; st < T::NST - 1; ++st) issue(st);
   }
   pdl_enter();
-  if (a.mode == 2) {
+  if (a.mode == 2 || (a.mode == 0 && a.late_prefetch)) {
 #pragma unroll
     for (int st = 0; st < T::NST - 1; ++st) issue(st);
   }

@@ -187,7 +187,7 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
   const int row = wid / a.H, head = wid % a.H;
   const int half = a.hd / 2;
   const int npair = half / 32;   // 1 or 2
-  int kv_lane = a.lane, pos = row;
+  int kv_lane = a.lane, pos = a.pos0 + row;
   // prefill: the positions are the row indices, and the RoPE table and the
   // cache's layer offsets are constants: read them before waiting for the QKV
   // projection
@@ -209,8 +209,11 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
       if (p < npair) csp[p] = a.rope_cs[(size_t)pos * half + lane + 32 * p];
     if (a.kv_base) cum = a.hdr->cum_layers[kv_lane];
   }
-  const size_t row3 = (size_t)row * 3 * a.d;
-  const size_t split_stride = (size_t)a.rows * 3 * a.d;
+  // columns of the partial sums: q | k | v, or k | v only
+  const int ncol = a.kv_only ? 2 : 3;
+  const size_t koff = a.kv_only ? 0 : (size_t)a.d, voff = koff + a.d;
+  const size_t row3 = (size_t)row * ncol * a.d;
+  const size_t split_stride = (size_t)a.rows * ncol * a.d;
   float q[2][2] = {{0.f, 0.f}, {0.f, 0.f}}, k[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   float v[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   // partial sums: all q/k/v elements of up to four splits in flight, added in
@@ -227,9 +230,9 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
           if (s < ns && p < npair) {
             const float* ps = a.part + (size_t)(s0 + s) * split_stride + row3 +
                               (size_t)head * a.hd + lane + 32 * p + hh * half;
-            t[s][p][hh][0] = __ldcg(ps);
-            t[s][p][hh][1] = __ldcg(ps + a.d);
-            t[s][p][hh][2] = __ldcg(ps + 2 * a.d);
+            t[s][p][hh][0] = a.kv_only ? 0.f : __ldcg(ps);
+            t[s][p][hh][1] = __ldcg(ps + koff);
+            t[s][p][hh][2] = __ldcg(ps + voff);
           }
 #pragma unroll
     for (int s = 0; s < 4; ++s)
@@ -263,7 +266,7 @@ __global__ void rope_kv_kernel(RopeKvArgs a) {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         size_t col = (size_t)row * a.d + (size_t)head * a.hd + i + hh * half;
-        a.q[col] = __float2half_rn(q[p][hh]);
+        if (a.q) a.q[col] = __float2half_rn(q[p][hh]);
         kh[p][hh] = __float2half_rn(k[p][hh]);
         vh[p][hh] = __float2half_rn(v[p][hh]);
         if (a.k) a.k[col] = kh[p][hh];

@@ -237,6 +237,7 @@ struct DgArgs {
   const __half* x;      // fp16 [T][K] activations (when !NORM)
   const float* h;       // fp32 [T][K] residual stream (NORM)
   const float* gamma;   // fp32 [K] (NORM)
+  __half* x_out;        // NORM, optional: the fp16 activations x [T][K], natural order (CTA 0)
   float eps;
   float* out;           // EPI_OUT: fp32 [T][N]
   float* hres;          // EPI_RESID: fp32 [rows][N], += y
@@ -433,10 +434,17 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
           const int k = 4 * tid + 4 * DG_THREADS * i;
           if (k < a.K) {
             const float4 v = hv[b][i], gm = gpre[i];
-            xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
-            xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
-            xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
-            xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+            const __half x0 = __float2half_rn(v.x * r * gm.x), x1 = __float2half_rn(v.y * r * gm.y);
+            const __half x2 = __float2half_rn(v.z * r * gm.z), x3 = __float2half_rn(v.w * r * gm.w);
+            xr[xpos<BITS>(k)] = x0;
+            xr[xpos<BITS>(k + 1)] = x1;
+            xr[xpos<BITS>(k + 2)] = x2;
+            xr[xpos<BITS>(k + 3)] = x3;
+            if (a.x_out && blockIdx.x == 0) {
+              __half2* xo = reinterpret_cast<__half2*>(a.x_out + (size_t)b * a.K + k);
+              xo[0] = __halves2half2(x0, x1);
+              xo[1] = __halves2half2(x2, x3);
+            }
           }
         }
         for (int k = a.K + tid; k < kpad; k += DG_THREADS) xr[xpos<BITS>(k)] = __float2half_rn(0.f);
@@ -476,10 +484,17 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
         for (int k = 4 * tid; k < a.K; k += 4 * DG_THREADS) {
           const float4 v = *reinterpret_cast<const float4*>(hr + k);
           const float4 gm = __ldg(reinterpret_cast<const float4*>(a.gamma + k));
-          xr[xpos<BITS>(k)] = __float2half_rn(v.x * r * gm.x);
-          xr[xpos<BITS>(k + 1)] = __float2half_rn(v.y * r * gm.y);
-          xr[xpos<BITS>(k + 2)] = __float2half_rn(v.z * r * gm.z);
-          xr[xpos<BITS>(k + 3)] = __float2half_rn(v.w * r * gm.w);
+          const __half x0 = __float2half_rn(v.x * r * gm.x), x1 = __float2half_rn(v.y * r * gm.y);
+          const __half x2 = __float2half_rn(v.z * r * gm.z), x3 = __float2half_rn(v.w * r * gm.w);
+          xr[xpos<BITS>(k)] = x0;
+          xr[xpos<BITS>(k + 1)] = x1;
+          xr[xpos<BITS>(k + 2)] = x2;
+          xr[xpos<BITS>(k + 3)] = x3;
+          if (a.x_out && blockIdx.x == 0) {
+            __half2* xo = reinterpret_cast<__half2*>(a.x_out + (size_t)b * a.K + k);
+            xo[0] = __halves2half2(x0, x1);
+            xo[1] = __halves2half2(x2, x3);
+          }
         }
       } else {
         for (int wd = tid; wd < nch * 16; wd += DG_THREADS) {
@@ -488,9 +503,12 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
           int pos[10];
           int3_word_slots(c, t, q, pos);
 #pragma unroll
-          for (int i = 0; i < 10; ++i)
-            xr[pos[i]] = k0 + i < a.K ? __float2half_rn(hr[k0 + i] * r * __ldg(a.gamma + k0 + i))
-                                      : __float2half_rn(0.f);
+          for (int i = 0; i < 10; ++i) {
+            const __half xv = k0 + i < a.K ? __float2half_rn(hr[k0 + i] * r * __ldg(a.gamma + k0 + i))
+                                           : __float2half_rn(0.f);
+            xr[pos[i]] = xv;
+            if (a.x_out && blockIdx.x == 0 && k0 + i < a.K) a.x_out[(size_t)b * a.K + k0 + i] = xv;
+          }
         }
       }
     }
@@ -868,6 +886,7 @@ tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   a.x = d.x;
   a.h = d.h;
   a.gamma = d.gamma;
+  a.x_out = d.x_out;
   a.eps = d.eps;
   a.out = d.out;
   a.hres = d.hres;

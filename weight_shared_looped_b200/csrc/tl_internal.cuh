@@ -138,6 +138,7 @@ struct DecGemvArgs {
   const __half* x;      // fp16 [T][K] activations, or null with h set
   const float* h;       // fp32 [T][K] residual stream: x = fp16(rmsnorm(h) * gamma)
   const float* gamma;
+  __half* x_out;        // with h: null, or written with those fp16 x rows [T][K]
   float eps;
   int epi;              // DecEpi
   float* out;           // DEC_EPI_OUT: fp32 [T][N]
@@ -210,6 +211,8 @@ struct RopeKvArgs {
   const int32_t* lane_of_row;  // decode: lane of each row; null = prefill of `lane`
   int lane;
   int decode;                  // 1: position = hdr->pos[lane]; 0: position = row index
+  int kv_only;                 // 1: part holds [S][rows][2d] K|V sums only; no q is written
+  int pos0;                    // decode == 0: position = pos0 + row index
 };
 tl_status launch_rope_kv(const RopeKvArgs& a, cudaStream_t s);
 
@@ -243,6 +246,8 @@ struct DecodeAttnArgs {
   int row_cum[kMaxLanes];    // cache layers of the lanes before that lane
   int row_off[kMaxLanes];    // position of the row's token = the lane's position + row_off
   int mode;                  // 0 append + attend, 1 append only, 2 attend only
+  int late_prefetch;         // 1: the cached entries were written by the previous kernel
+                             //    (rebuilt K/V): no copy before the dependency wait
   int chunks;                // context chunks per CTA; 0 = fewest waves
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);

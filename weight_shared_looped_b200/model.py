@@ -9,7 +9,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 import torch
 
-from . import (TL_KV_FP16, TL_KV_INT8, tl_block_create, tl_block_destroy, tl_decode_step,
+from . import (TL_KV_FP16, TL_KV_INT8, TL_KV_H, tl_block_create, tl_block_destroy, tl_decode_step,
                tl_kv_bytes, tl_kv_create, tl_kv_destroy, tl_kv_layer_ptrs, tl_kv_position,
                tl_kv_reset, tl_kv_set_position, tl_model_create, tl_model_destroy,
                tl_model_device_bytes, tl_model_set_decode_chunks, tl_model_set_graphs,
@@ -167,7 +167,7 @@ class DeviceKV:
     def __init__(self, model: DeviceModel, L_per_lane: Sequence[int], max_ctx: int,
                  dtype: str = "fp16"):
         self.model = model
-        self.dtype = TL_KV_INT8 if dtype == "int8" else TL_KV_FP16
+        self.dtype = {"int8": TL_KV_INT8, "h": TL_KV_H}.get(dtype, TL_KV_FP16)
         self.L = list(L_per_lane)
         self.max_ctx = max_ctx
         nbytes = tl_kv_bytes(model.handle, max_ctx, self.L, self.dtype)
