@@ -389,3 +389,38 @@ def test_int3_chunk_dot_product_odd_iteration(seed):
     deq = np.array([float(np.float16(odd[k] * s[k // G])) for k in range(K)])
     want = float(deq @ x[:K])
     assert abs(total - want) <= 1e-9 * max(1.0, abs(want)), (total, want)
+
+
+# ---------------------------------------------------------------- staged row layout
+def dg_row(r):
+    return ((r & 1) << 3) | ((r & 8) >> 1) | ((r & 7) >> 1)
+
+
+def dg_row_off(r, rb):
+    pr = dg_row(r)
+    return (pr >> 3) * (8 * rb + 64) + (pr & 7) * rb
+
+
+def test_row_layout_matches_the_kernel():
+    assert "return ((r & 1) << 3) | ((r & 8) >> 1) | ((r & 7) >> 1);" in SRC
+    assert "return (size_t)8 * row_bytes + 64;" in SRC
+    assert "(size_t)(pr >> 3) * dg_grp_bytes(row_bytes) + (size_t)(pr & 7) * row_bytes" in SRC
+
+
+@pytest.mark.parametrize("rb", [1024, 4096, 832, 3280])   # INT4 and INT3 rows, K 2048 and 8192
+def test_staged_rows_are_bank_conflict_free(rb):
+    """Two bulk copies per 16-row tile (rows 0-7, rows 8-15 64 bytes after the
+    end of the first group): every 16-byte operand load of a quarter warp
+    (lanes 8p .. 8p + 7: MMA rows 2p, 2p + 1, vectors 4c .. 4c + 3) touches 32
+    distinct banks, for the rows g and for the rows g + 8."""
+    assert sorted(dg_row(r) for r in range(16)) == list(range(16))
+    for half in (0, 8):
+        for c in range(3):
+            for p in range(4):
+                banks = []
+                for lane in range(8 * p, 8 * p + 8):
+                    g, t = lane >> 2, lane & 3
+                    off = dg_row_off(g + half, rb) + 16 * (4 * c + t)
+                    assert off % 16 == 0
+                    banks += [(off // 4 + i) % 32 for i in range(4)]
+                assert len(set(banks)) == 32, (rb, half, c, p)

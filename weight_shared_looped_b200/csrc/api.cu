@@ -985,6 +985,7 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
   da.qkv_S = 1;
   da.rope_cs = m->rope;
   da.chunks = m->decode_chunks;
+  da.status = m->status;
   if (store_h) {
     // attend over the rebuilt entries: lane b's are layer b of the workspace
     da.kv_base = kv->h_kv;

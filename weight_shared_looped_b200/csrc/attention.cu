@@ -254,18 +254,54 @@ __global__ void __launch_bounds__(32 * ATT_WARPS) attn_prefill_tc_kernel(const _
 // first cached K/V rows copied into shared memory before the wait for the QKV
 // projection.  The CTA holding position pos forms k and v from the QKV
 // partial sums, applies RoPE to k and appends both to the cache.  Each chunk
-// ends with its max score, exponential sum and unnormalised P V; rank 0
-// merges the chunks in order through distributed shared memory.
+// ends with its max score, exponential sum and unnormalised P V, and rank 0
+// merges the chunks in order: either every CTA pushes its chunks into rank 0's
+// shared memory (distributed shared-memory stores, one mbarrier arrival per
+// CTA) and leaves, or, where the push target's shared memory would cost a wave
+// of clusters, rank 0 pulls them between two cluster barriers.  Both merges
+// do the same arithmetic.
 __device__ __forceinline__ void cl_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;" :::
                    "memory");
 }
-__device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
+__device__ __forceinline__ uint32_t cl_addr(const void* local, uint32_t rank) {
   uint32_t addr = (uint32_t)__cvta_generic_to_shared(local), remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ float cl_ld(const float* local, uint32_t rank) {
   float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cl_addr(local, rank)) : "memory");
   return v;
+}
+// a store into the shared memory of CTA `rank` of the cluster
+__device__ __forceinline__ void cl_st(float* local, uint32_t rank, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(cl_addr(local, rank)), "f"(v) : "memory");
+}
+// one arrival, with release semantics at cluster scope, on an mbarrier of CTA `rank`
+__device__ __forceinline__ void cl_arrive(uint64_t* bar, uint32_t rank) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr(bar, rank))
+               : "memory");
+}
+// bounded wait (2 s of global time) for phase 0 of a local mbarrier whose
+// arrivals come from the whole cluster
+__device__ __forceinline__ bool cl_wait0(uint64_t* bar) {
+  const uint32_t addr = (uint32_t)__cvta_generic_to_shared(bar);
+  uint64_t t0 = 0;
+  for (uint32_t i = 0;; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr)
+        : "memory");
+    if (done) return true;
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    if (i == 0) t0 = t;
+    else if (t - t0 > 2000000000ull) return false;
+  }
 }
 
 constexpr int DS_KEYS = 64;     // keys per stage of the decode kernel
@@ -357,7 +393,7 @@ __device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t wa, uint32_t wb) {
 
 template <int HD, bool I8>
 __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeAttnArgs a, int CL,
-                                                                       int F, int sc_len) {
+                                                                       int F, int sc_len, int push) {
   using T = DecTc<HD, I8>;
   constexpr int HALF = HD / 2;
   constexpr int MT = HD / 16;                    // P V m tiles of 16 head_dim elements
@@ -366,6 +402,8 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   __shared__ __align__(16) __half qh[HD];
   __shared__ float wm[4], wl[4];
   __shared__ float kmax_s[4], vmax_s[4];
+  __shared__ __align__(8) uint64_t mrg_bar;  // push merge, rank 0: one arrival per CTA of the cluster
+  __shared__ int mrg_ok;
   const int crank = blockIdx.x, head = blockIdx.y, row = blockIdx.z;   // crank: rank in the cluster
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, t = lane & 3;
@@ -374,6 +412,8 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   __half* ksc = reinterpret_cast<__half*>(dsm + (size_t)T::NST * T::STAGE_BYTES);   // [sc_len]
   __half* vsc = ksc + sc_len;
   float* part = reinterpret_cast<float*>(vsc + sc_len);   // [F][HD + 2]: chunk P V, max, sum
+  // push merge: rank 0's [CL][HD + 2] of every chunk's (P V, max, sum)
+  float* allp = part + (size_t)F * (HD + 2);
   // This CTA takes chunks crank*F .. crank*F + F - 1 of the CL equal chunks of
   // the lane's context, i.e. the contiguous keys [kA, kB).  Each chunk is
   // streamed in 64-key stages from its own start and folded into its own
@@ -392,6 +432,18 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
   const int nkc = kB - kA;
   const bool owner = a.mode != 2 && nkc > 0 && kB == n_keys;
   if (a.mode == 1 && !owner) return;   // nothing to append here, nothing copied yet
+  if (a.mode != 1 && push) {
+    // the push merge: rank 0's barrier counts one arrival per CTA; its
+    // initialisation is published by the cluster barrier arrival here and
+    // awaited before the first remote access at the end
+    if (crank == 0 && tid == 0) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(
+                       (uint32_t)__cvta_generic_to_shared(&mrg_bar)),
+                   "r"(gridDim.x));
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  }
   const int n_old = owner ? nkc - 1 : nkc;       // keys of [kA, kB) already cached
   const int NSF = (per + DS_KEYS - 1) / DS_KEYS; // stages of a full chunk
   const int nstage = nkc / per * NSF + (nkc % per + DS_KEYS - 1) / DS_KEYS;
@@ -792,10 +844,51 @@ __global__ void __launch_bounds__(128, I8 ? 4 : 3) attn_decode_tc_kernel(DecodeA
     }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
+  if (push) {
+    __syncthreads();   // this CTA's chunk results are complete
+    // push them into rank 0 (chunk c = crank * F + j goes to its slot c), then
+    // one arrival; every CTA but rank 0 is done after that
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");   // rank 0's barrier is set up
+    for (int j = 0; j < F; ++j) {
+      const int c = crank * F + j;
+      if (c < CL)
+        for (int i = tid; i < HD + 2; i += 128)
+          cl_st(allp + (size_t)c * (HD + 2) + i, 0u, part[j * (HD + 2) + i]);
+    }
+    __syncthreads();
+    if (tid == 0) cl_arrive(&mrg_bar, 0u);
+    if (crank != 0) return;
+    if (tid == 0) mrg_ok = cl_wait0(&mrg_bar) ? 1 : 0;
+    __syncthreads();
+    if (!mrg_ok) {
+      if (tid == 0 && a.status) atomicCAS(a.status, 0, (int)TL_ERR_TIMEOUT);
+      return;
+    }
+    if (tid < HD) {
+      // the chunks merged in order from rank 0's own shared memory
+      float M = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        if (c < CL) M = fmaxf(M, allp[c * (HD + 2) + HD]);
+      float L = 0.f, acc = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        if (c < CL) {
+          const float mc = allp[c * (HD + 2) + HD];
+          const float w = mc == -INFINITY ? 0.f : exp2f(mc - M);
+          L = fmaf(allp[c * (HD + 2) + HD + 1], w, L);
+          acc = fmaf(allp[c * (HD + 2) + tid], w, acc);
+        }
+      }
+      a.out[(size_t)row * a.d + head * HD + tid] = __float2half_rn(acc / L);
+    }
+    return;
+  }
   cl_sync();   // every CTA's chunk results are in its shared memory
   if (crank == 0 && tid < HD) {
-    // chunk c sits in CTA c / F, slot c % F; all remote reads are issued
-    // before any is used, then the chunks are merged in order
+    // pull merge: chunk c sits in CTA c / F, slot c % F; all remote reads are
+    // issued before any is used, then the chunks are merged in order (the same
+    // arithmetic as the push merge)
     float mr[8], lr[8], ar[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -861,9 +954,9 @@ static int decode_cluster_size(int max_ctx) {
   return c < 1 ? 1 : c > 8 ? 8 : c;
 }
 template <int HD, bool I8>
-static size_t decode_tc_smem(int sc_len, int F) {
+static size_t decode_tc_smem(int sc_len, int F, int push_cl) {
   return (size_t)DecTc<HD, I8>::NST * DecTc<HD, I8>::STAGE_BYTES +
-         2 * (size_t)sc_len * sizeof(__half) + (size_t)F * (HD + 2) * sizeof(float);
+         2 * (size_t)sc_len * sizeof(__half) + (size_t)(F + push_cl) * (HD + 2) * sizeof(float);
 }
 constexpr size_t kDecodeSmemCap = 200 * 1024;
 
@@ -915,21 +1008,26 @@ static tl_status launch_decode_tc(const DecodeAttnArgs& a, cudaStream_t s) {
   const int max_per = (a.max_ctx + cl - 1) / cl;   // keys of a chunk at most
   // chunks per CTA: the fewest that run every (row, head) cluster in the
   // fewest waves
-  int best_f = 0, best_waves = 0;
+  // fewest waves; on a tie the push merge (its rank 0 holds every chunk's
+  // record: more shared memory per CTA, one cluster barrier instead of two)
+  int best_f = 0, best_waves = 0, best_push = 0;
   size_t best_smem = 0;
   int best_sc = 0;
   for (int f = a.chunks > 0 ? std::min(a.chunks, cl) : 1; f <= cl; f *= 2) {
     const int sc_len = I8 ? (f * max_per + DS_KEYS + 7) / 8 * 8 : 0;   // a stage past the last key
-    const size_t smem = decode_tc_smem<HD, I8>(sc_len, f);
-    if (smem > kDecodeSmemCap) break;
-    const int pc = (cl + f - 1) / f;
-    const int active = decode_active_clusters<HD, I8>(pc, smem);
-    const int waves = (a.rows * a.H + active - 1) / active;
-    if (best_f == 0 || waves < best_waves) {
-      best_f = f;
-      best_waves = waves;
-      best_smem = smem;
-      best_sc = sc_len;
+    for (int push = 1; push >= 0; --push) {
+      const size_t smem = decode_tc_smem<HD, I8>(sc_len, f, push ? cl : 0);
+      if (smem > kDecodeSmemCap) continue;
+      const int pc = (cl + f - 1) / f;
+      const int active = decode_active_clusters<HD, I8>(pc, smem);
+      const int waves = (a.rows * a.H + active - 1) / active;
+      if (best_f == 0 || waves < best_waves) {
+        best_f = f;
+        best_waves = waves;
+        best_smem = smem;
+        best_sc = sc_len;
+        best_push = push;
+      }
     }
     if (a.chunks > 0) break;   // fixed by the caller
   }
@@ -939,7 +1037,7 @@ static tl_status launch_decode_tc(const DecodeAttnArgs& a, cudaStream_t s) {
   const int pc = (cl + best_f - 1) / best_f;
   dim3 grid(pc, a.H, a.rows);
   const cudaError_t e = launch_pdl_cluster(attn_decode_tc_kernel<HD, I8>, grid, dim3(128), best_smem, s,
-                                           (unsigned)pc, a, cl, best_f, best_sc);
+                                           (unsigned)pc, a, cl, best_f, best_sc, best_push);
   if (e != cudaSuccess)
     return set_error(TL_ERR_CUDA, "launch of attn_decode_tc_kernel failed: %s", cudaGetErrorString(e));
   return ok();

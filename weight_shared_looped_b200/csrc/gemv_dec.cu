@@ -233,7 +233,7 @@ struct DgArgs {
   int T;                // active token rows (1..8)
   int n_units;          // N / 16
   int stages;           // weight stages in shared memory
-  int row_stride;       // bytes per staged row (row bytes padded to 64 mod 128)
+  int row_bytes;        // bytes of one packed row (wpr * 4)
   const __half* x;      // fp16 [T][K] activations (when !NORM)
   const float* h;       // fp32 [T][K] residual stream (NORM)
   const float* gamma;   // fp32 [K] (NORM)
@@ -274,43 +274,57 @@ __device__ __forceinline__ bool dg_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
-// The weights (and scales) of one unit into its stage: lane r of the calling
-// warp copies row r of the unit (one bulk copy per row, so that staged rows
-// sit 64 bytes off the 128-byte bank period), the scales one copy per tile.
+// Stage layout of one 16-row tile: two groups of eight consecutive packed
+// rows (rows 0-7 and 8-15 of the tile), each group one bulk copy, the second
+// group 64 bytes further than the end of the first, so that the two rows any
+// quarter-warp reads (MMA rows 2p and 2p + 1 below) sit half a bank period
+// apart.  MMA row r of the tile (lane g = r & 7 holds rows g and g + 8) is
+// packed row dg_row(r): rows 2p, 2p + 1 of an MMA tile come from different
+// groups.  The epilogue writes row r's result to output row dg_row(r).
+__device__ __forceinline__ int dg_row(int r) { return ((r & 1) << 3) | ((r & 8) >> 1) | ((r & 7) >> 1); }
+__device__ __forceinline__ size_t dg_grp_bytes(int row_bytes) { return (size_t)8 * row_bytes + 64; }
+__device__ __forceinline__ size_t dg_row_off(int r, int row_bytes) {
+  const int pr = dg_row(r);
+  return (size_t)(pr >> 3) * dg_grp_bytes(row_bytes) + (size_t)(pr & 7) * row_bytes;
+}
+
+// The weights, scales (and sign rows) of one unit into its stage: lanes
+// 0 .. 2 MT - 1 of the calling warp copy the row groups, then one lane per
+// tile its scales (and its sign rows, one copy each).
 template <int MT, bool SGN>
 __device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigned char* stage,
                                               uint32_t bar, int lane) {
-  const int rows = 16 * MT;
-  const uint32_t row_bytes = (uint32_t)a.wpr * 4;
+  const uint32_t grp_copy = 8u * (uint32_t)a.row_bytes;
+  const size_t grp = dg_grp_bytes(a.row_bytes), tile = 2 * grp;
   const int gpr = a.K / a.G;
   const uint32_t sc_bytes = 16u * gpr * 2;
   const uint32_t sg_bytes = SGN ? 16u * a.spr * 4 : 0u;   // a tile's sign rows, one copy
   if (lane == 0) {
-    const uint32_t total = rows * row_bytes + MT * (sc_bytes + sg_bytes);
+    const uint32_t total = MT * (2 * grp_copy + sc_bytes + sg_bytes);
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(total)
                  : "memory");
   }
   __syncwarp();
   const int r0 = unit * 16;
-  if (lane < rows) {
-    const int m = lane >> 4, r = lane & 15;
-    const uint32_t* src = (m == 0 ? a.w0 : a.w1) + (size_t)(r0 + r) * a.wpr;
-    const uint32_t dst = smem_u32(stage + (size_t)lane * a.row_stride);
+  if (lane < 2 * MT) {
+    const int m = lane >> 1, q = lane & 1;   // tile m, rows 8q .. 8q + 7
+    const uint32_t* src = (m == 0 ? a.w0 : a.w1) + (size_t)(r0 + 8 * q) * a.wpr;
+    const uint32_t dst = smem_u32(stage + (size_t)m * tile + (size_t)q * grp);
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-        "l"(src), "r"(row_bytes), "r"(bar)
+        "l"(src), "r"(grp_copy), "r"(bar)
         : "memory");
   }
   if (lane < MT) {
     const __half* src = (lane == 0 ? a.s0 : a.s1) + (size_t)r0 * gpr;
-    const uint32_t dst = smem_u32(stage + (size_t)rows * a.row_stride + (size_t)lane * sc_bytes);
+    const uint32_t dst = smem_u32(stage + (size_t)MT * tile + (size_t)lane * sc_bytes);
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
         "l"(src), "r"(sc_bytes), "r"(bar)
         : "memory");
     if (SGN) {
       const uint32_t* gsrc = (lane == 0 ? a.g0 : a.g1) + (size_t)r0 * a.spr;
-      const uint32_t gdst = smem_u32(stage + (size_t)rows * a.row_stride + (size_t)MT * sc_bytes +
+      const uint32_t gdst = smem_u32(stage + (size_t)MT * tile + (size_t)MT * sc_bytes +
                                      (size_t)lane * sg_bytes);
       asm volatile(
           "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(gdst),
@@ -346,7 +360,8 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   const int gsh = __ffs(a.G) - 1;
   const int gpr = a.K >> gsh;
   const bool g64 = BITS == 4 && a.G == 64;
-  const size_t stage_bytes = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2 +
+  const size_t tile_bytes = 2 * dg_grp_bytes(a.row_bytes);
+  const size_t stage_bytes = (size_t)MT * tile_bytes + (size_t)MT * 16 * gpr * 2 +
                              (SGN ? (size_t)MT * 16 * a.spr * 4 : 0);
   unsigned char* stages = dg_smem;
   __half* xs = reinterpret_cast<__half*>(dg_smem + (size_t)a.stages * stage_bytes);   // [T][xw]
@@ -553,16 +568,20 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   // this warp's chunks of its tile of the unit in `stage`, added into acc
   auto unit_mma = [&](const unsigned char* stage, float* acc) {
     // ---- the MMAs: this warp's chunks of its tile, words and scales from the stage
-    const unsigned char* wt0 = stage + (size_t)(16 * m + g) * a.row_stride;
-    const unsigned char* wt1 = wt0 + (size_t)8 * a.row_stride;
-    const __half* st0 = reinterpret_cast<const __half*>(stage + (size_t)16 * MT * a.row_stride +
-                                                        (size_t)m * 16 * gpr * 2) + (size_t)g * gpr;
-    const __half* st1 = st0 + (size_t)8 * gpr;
-    // the tile's sign rows (odd iterations): rows g and g + 8
-    const uint32_t* sg0 = reinterpret_cast<const uint32_t*>(
-        stage + (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * gpr * 2 +
-        (size_t)(m * 16 + g) * a.spr * 4);
-    const uint32_t* sg1 = sg0 + (size_t)8 * a.spr;
+    // MMA rows g and g + 8 of tile m: packed rows dg_row(g), dg_row(g + 8)
+    const int pr0 = dg_row(g), pr1 = dg_row(g + 8);
+    const unsigned char* tile_base = stage + (size_t)m * tile_bytes;
+    const unsigned char* wt0 = tile_base + dg_row_off(g, a.row_bytes);
+    const unsigned char* wt1 = tile_base + dg_row_off(g + 8, a.row_bytes);
+    const __half* sct = reinterpret_cast<const __half*>(stage + (size_t)MT * tile_bytes +
+                                                        (size_t)m * 16 * gpr * 2);
+    const __half* st0 = sct + (size_t)pr0 * gpr;
+    const __half* st1 = sct + (size_t)pr1 * gpr;
+    // the tile's sign rows (odd iterations), same rows
+    const uint32_t* sgt = reinterpret_cast<const uint32_t*>(
+        stage + (size_t)MT * tile_bytes + (size_t)MT * 16 * gpr * 2 + (size_t)m * 16 * a.spr * 4);
+    const uint32_t* sg0 = sgt + (size_t)pr0 * a.spr;
+    const uint32_t* sg1 = sgt + (size_t)pr1 * a.spr;
     for (int c = c_lo; c < c_hi; ++c) {
       const int vi = 4 * c + t;
       uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
@@ -694,13 +713,13 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
             us += redj[((1 * W + w) * 16 + r) * 8 + b];
           }
           const float silu = gs / (1.0f + __expf(-gs));
-          a.u[(size_t)b * a.N + unit * 16 + r] = __float2half_rn(silu * us);
+          a.u[(size_t)b * a.N + unit * 16 + dg_row(r)] = __float2half_rn(silu * us);
         }
       }
     } else {
       if (tid < 16 * 8) {
         const int r = tid >> 3, b = tid & 7;
-        const int n = unit * 16 + r;
+        const int n = unit * 16 + dg_row(r);
         float y = 0.f;
 #pragma unroll
         for (int w = 0; w < W; ++w) y += redj[(w * 16 + r) * 8 + b];
@@ -824,8 +843,8 @@ tl_status launch_dg(DgArgs a, cudaStream_t s) {
   const int nvec = a.wpr / 4, nch = (nvec + 3) / 4;
   const size_t xw = (size_t)nch * DgFmt<BITS>::CW + 8;
   const size_t row_bytes = (size_t)a.wpr * 4;
-  a.row_stride = (int)(row_bytes + ((64 + 128 - row_bytes % 128) % 128));
-  const size_t stage = (size_t)16 * MT * a.row_stride + (size_t)MT * 16 * (a.K / a.G) * 2 +
+  a.row_bytes = (int)row_bytes;
+  const size_t stage = (size_t)MT * 2 * (8 * row_bytes + 64) + (size_t)MT * 16 * (a.K / a.G) * 2 +
                        (SGN ? (size_t)MT * 16 * a.spr * 4 : 0);
   const int grid = std::min(a.n_units, dg_sm_count());
   const int per_cta = (a.n_units + grid - 1) / grid;

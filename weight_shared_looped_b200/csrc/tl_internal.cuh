@@ -249,6 +249,7 @@ struct DecodeAttnArgs {
   int late_prefetch;         // 1: the cached entries were written by the previous kernel
                              //    (rebuilt K/V): no copy before the dependency wait
   int chunks;                // context chunks per CTA; 0 = fewest waves
+  int* status;               // null, or the status word a timed-out merge wait sets
 };
 tl_status launch_attn_decode_fused(const DecodeAttnArgs& a, cudaStream_t s);
 
