@@ -72,7 +72,7 @@ def test_linear_tc_kernel(N, K, T, group):
 ])
 def test_linear_decode_projection_kernel(N, K, T, group):
     """Decode-sized calls (T <= 8, K % 128 == 0) run the decode projection
-    kernel: no split-K, the eight warps of a CTA split K and add in warp order;
+    kernel: no split-K, the sixteen warps of a CTA split K and add in warp order;
     exact codes with the group scale applied to fp32 sums (G = 64: one sum per
     group), so only the summation order differs from the exact product."""
     assert tl.tl_linear_workspace_bytes(N, K, T) == 0

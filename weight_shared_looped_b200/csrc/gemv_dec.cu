@@ -3,8 +3,8 @@
 //   y[t][n] = sum over k of x[t][k] * W[n][k],   W[n][k] = code[n][k] * scale[n][k / G]
 // for canonical INT4 (8 codes per word) or INT3 (10 codes per word) weights.
 //
-// A CTA owns MT tiles of 16 weight rows over the whole of K; its eight warps
-// split K (MT = 1: eight k ranges; MT = 2: four per tile), so no split-K
+// A CTA owns MT tiles of 16 weight rows over the whole of K; its sixteen warps
+// split K (MT = 1: sixteen k ranges; MT = 2: eight per tile), so no split-K
 // partial sums leave the CTA: the warps' results are added in shared memory in
 // warp order, a fixed order that depends only on (N, K, MT).  Every token
 // column is computed independently of the others, so a token's result does
@@ -51,8 +51,8 @@
 namespace tl {
 namespace {
 
-constexpr int DG_THREADS = 256;
-constexpr int DG_WARPS = 8;
+constexpr int DG_THREADS = 512;   // sixteen warps: more MMA chains in flight per SM
+constexpr int DG_WARPS = 16;
 
 enum { EPI_OUT = 0, EPI_RESID = 1, EPI_SWIGLU = 2 };
 
