@@ -344,7 +344,7 @@ __device__ __forceinline__ void dg_issue_unit(const DgArgs& a, int unit, unsigne
 // before the dependency wait; the warps compute them back to back into
 // per-unit sums and one reduction and one epilogue close the launch.  UM == 0:
 // the units stream through a ring of a.stages stages, one reduction per unit.
-template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN>
+template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN, bool WIDE>
 __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
   using Fm = DgFmt<BITS>;
   constexpr int CW = Fm::CW;
@@ -465,6 +465,62 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
         for (int k = a.K + tid; k < kpad; k += DG_THREADS) xr[xpos<BITS>(k)] = __float2half_rn(0.f);
       }
     }
+  } else if (WIDE && NORM && BITS == 4 && a.K <= 4 * DG_THREADS) {
+    // three to eight rows of d <= 2048: one float4 of every row per thread,
+    // all rows' loads in flight together and kept in registers between the
+    // sum of squares and the scaling (same arithmetic and order per row as
+    // the general path)
+    float4 hv[8];
+    const int k = 4 * tid;
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+      hv[b] = b < a.T && k < a.K ? *reinterpret_cast<const float4*>(a.h + (size_t)b * a.K + k)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    float ss[8];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      ss[b] = fmaf(hv[b].x, hv[b].x, 0.f);
+      ss[b] = fmaf(hv[b].y, hv[b].y, ss[b]);
+      ss[b] = fmaf(hv[b].z, hv[b].z, ss[b]);
+      ss[b] = fmaf(hv[b].w, hv[b].w, ss[b]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) ss[b] += __shfl_xor_sync(0xffffffffu, ss[b], o);
+    if (lane == 0)
+#pragma unroll
+      for (int b = 0; b < 8; ++b)
+        if (b < a.T) nred[b][warp] = ss[b];
+    __syncthreads();
+    const float4 gm = gpre[0];
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      if (b < a.T) {
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < DG_WARPS; ++w) tot += nred[b][w];
+        if (a.ex.check_iter > 0 && blockIdx.x == 0 && tid == 0 && a.ex.exit_it[b] == 0 &&
+            sqrtf(tot) > a.ex.tau)
+          a.ex.exit_it[b] = a.ex.check_iter;
+        const float r = rsqrtf(tot / (float)a.K + a.eps);
+        if (k < a.K) {
+          const float4 v = hv[b];
+          __half* xr = xs + (size_t)b * xw;
+          const __half x0 = __float2half_rn(v.x * r * gm.x), x1 = __float2half_rn(v.y * r * gm.y);
+          const __half x2 = __float2half_rn(v.z * r * gm.z), x3 = __float2half_rn(v.w * r * gm.w);
+          xr[xpos<BITS>(k)] = x0;
+          xr[xpos<BITS>(k + 1)] = x1;
+          xr[xpos<BITS>(k + 2)] = x2;
+          xr[xpos<BITS>(k + 3)] = x3;
+          if (a.x_out && blockIdx.x == 0) {
+            __half2* xo = reinterpret_cast<__half2*>(a.x_out + (size_t)b * a.K + k);
+            xo[0] = __halves2half2(x0, x1);
+            xo[1] = __halves2half2(x2, x3);
+          }
+        }
+      }
+    }
   } else if (NORM) {
     // x = fp16(h * rsqrt(mean(h^2) + eps) * gamma) per token row, the sum of
     // squares in a fixed order (per thread, xor tree, warps in order)
@@ -524,6 +580,32 @@ __global__ void __launch_bounds__(DG_THREADS, 1) gemv_dec_kernel(DgArgs a) {
             xr[pos[i]] = xv;
             if (a.x_out && blockIdx.x == 0 && k0 + i < a.K) a.x_out[(size_t)b * a.K + k0 + i] = xv;
           }
+        }
+      }
+    }
+  } else if (WIDE && BITS == 4 && a.T > 2) {
+    // three to eight rows: the vectors of eight consecutive k of all rows
+    // ([T][K] contiguous), eight per thread in flight; each becomes four
+    // half2 stores
+    const int kv = a.K >> 3, total = a.T * kv;
+    for (int e0 = tid; e0 < total; e0 += 8 * DG_THREADS) {
+      uint4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * DG_THREADS;
+        if (e < total) v[i] = *reinterpret_cast<const uint4*>(a.x + (size_t)e * 8);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * DG_THREADS;
+        if (e < total) {
+          const int b = e / kv, k = (e - b * kv) * 8;
+          const __half* h8 = reinterpret_cast<const __half*>(&v[i]);
+          __half* xr = xs + (size_t)b * xw + xpos<4>(k);   // element 0: k step 2q, slot 2t
+          *reinterpret_cast<__half2*>(xr) = __halves2half2(h8[0], h8[4]);
+          *reinterpret_cast<__half2*>(xr + 8) = __halves2half2(h8[1], h8[5]);
+          *reinterpret_cast<__half2*>(xr + 16) = __halves2half2(h8[2], h8[6]);
+          *reinterpret_cast<__half2*>(xr + 24) = __halves2half2(h8[3], h8[7]);
         }
       }
     }
@@ -826,19 +908,19 @@ constexpr size_t kDgSmemShare = 110 * 1024;
 // all) less room for the kernel's static shared memory
 constexpr size_t kDgSmemMax = 232448 - 1024;
 
-template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN>
+template <int BITS, int MT, bool NORM, int EPI, int UM, bool SGN, bool WIDE>
 tl_status launch_dg_um(const DgArgs& a, int grid, size_t smem, cudaStream_t s) {
   static std::atomic<uint64_t> attr_done{0};
   TL_TRY(once_per_device(attr_done, []() -> tl_status {
-    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN>,
+    TL_CUDA(cudaFuncSetAttribute(gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN, WIDE>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDgSmemMax));
     return ok();
   }));
-  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN>), grid, DG_THREADS, smem, s, a);
+  TL_LAUNCH_PDL((gemv_dec_kernel<BITS, MT, NORM, EPI, UM, SGN, WIDE>), grid, DG_THREADS, smem, s, a);
   return ok();
 }
 
-template <int BITS, int MT, bool NORM, int EPI, bool SGN>
+template <int BITS, int MT, bool NORM, int EPI, bool SGN, bool WIDE>
 tl_status launch_dg(DgArgs a, cudaStream_t s) {
   const int nvec = a.wpr / 4, nch = (nvec + 3) / 4;
   const size_t xw = (size_t)nch * DgFmt<BITS>::CW + 8;
@@ -857,10 +939,10 @@ tl_status launch_dg(DgArgs a, cudaStream_t s) {
     if (smem <= kDgSmemMax) {
       a.stages = per_cta;
       switch (um) {
-        case 1: return launch_dg_um<BITS, MT, NORM, EPI, 1, SGN>(a, grid, smem, s);
-        case 2: return launch_dg_um<BITS, MT, NORM, EPI, 2, SGN>(a, grid, smem, s);
-        case 4: return launch_dg_um<BITS, MT, NORM, EPI, 4, SGN>(a, grid, smem, s);
-        default: return launch_dg_um<BITS, MT, NORM, EPI, 8, SGN>(a, grid, smem, s);
+        case 1: return launch_dg_um<BITS, MT, NORM, EPI, 1, SGN, WIDE>(a, grid, smem, s);
+        case 2: return launch_dg_um<BITS, MT, NORM, EPI, 2, SGN, WIDE>(a, grid, smem, s);
+        case 4: return launch_dg_um<BITS, MT, NORM, EPI, 4, SGN, WIDE>(a, grid, smem, s);
+        default: return launch_dg_um<BITS, MT, NORM, EPI, 8, SGN, WIDE>(a, grid, smem, s);
       }
     }
   }
@@ -873,7 +955,7 @@ tl_status launch_dg(DgArgs a, cudaStream_t s) {
     return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: K = %d x %d tokens needs too much shared memory",
                      a.K, a.T);
   a.stages = stages;
-  return launch_dg_um<BITS, MT, NORM, EPI, 0, SGN>(a, grid, smem, s);
+  return launch_dg_um<BITS, MT, NORM, EPI, 0, SGN, WIDE>(a, grid, smem, s);
 }
 
 }  // namespace
@@ -919,22 +1001,32 @@ tl_status launch_dec_gemv(const DecGemvArgs& d, cudaStream_t s) {
   const bool sg = d.g0 != nullptr;
   if (sg && (d.K % 32 != 0 || (d.epi == DEC_EPI_SWIGLU && d.g1 == nullptr)))
     return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: sign bits need K %% 32 == 0 (and both matrices')");
-#define TL_DG(B, MT_, NORM_, EPI_) \
-  (sg ? launch_dg<B, MT_, NORM_, EPI_, true>(a, s) : launch_dg<B, MT_, NORM_, EPI_, false>(a, s))
+  // INT4 launches of three to eight rows take kernels with the staging that
+  // keeps every row's loads in flight; one or two rows keep the compact one
+  const bool wide = d.T > 2;
+#define TL_DG4(MT_, NORM_, EPI_)                                                              \
+  (sg ? (wide ? launch_dg<4, MT_, NORM_, EPI_, true, true>(a, s)                            \
+              : launch_dg<4, MT_, NORM_, EPI_, true, false>(a, s))                          \
+      : (wide ? launch_dg<4, MT_, NORM_, EPI_, false, true>(a, s)                           \
+              : launch_dg<4, MT_, NORM_, EPI_, false, false>(a, s)))
+#define TL_DG3(MT_, NORM_, EPI_) \
+  (sg ? launch_dg<3, MT_, NORM_, EPI_, true, false>(a, s) : launch_dg<3, MT_, NORM_, EPI_, false, false>(a, s))
   switch (d.epi) {
     case DEC_EPI_SWIGLU:
       if (!norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: SwiGLU needs the norm prologue");
-      return d.bits == 4 ? TL_DG(4, 2, true, EPI_SWIGLU) : TL_DG(3, 2, true, EPI_SWIGLU);
+      return d.bits == 4 ? TL_DG4(2, true, EPI_SWIGLU) : TL_DG3(2, true, EPI_SWIGLU);
     case DEC_EPI_RESID:
       if (norm) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: residual epilogue takes x");
-      return d.bits == 4 ? TL_DG(4, 1, false, EPI_RESID) : TL_DG(3, 1, false, EPI_RESID);
+      return d.bits == 4 ? TL_DG4(1, false, EPI_RESID) : TL_DG3(1, false, EPI_RESID);
     default:
-      if (norm) return d.bits == 4 ? TL_DG(4, 1, true, EPI_OUT) : TL_DG(3, 1, true, EPI_OUT);
+      if (norm) return d.bits == 4 ? TL_DG4(1, true, EPI_OUT) : TL_DG3(1, true, EPI_OUT);
       if (sg) return set_error(TL_ERR_UNSUPPORTED, "decode GEMV: sign bits need the norm prologue here");
-      return d.bits == 4 ? launch_dg<4, 1, false, EPI_OUT, false>(a, s)
-                         : launch_dg<3, 1, false, EPI_OUT, false>(a, s);
+      return d.bits == 4 ? (wide ? launch_dg<4, 1, false, EPI_OUT, false, true>(a, s)
+                                 : launch_dg<4, 1, false, EPI_OUT, false, false>(a, s))
+                         : launch_dg<3, 1, false, EPI_OUT, false, false>(a, s);
   }
-#undef TL_DG
+#undef TL_DG4
+#undef TL_DG3
 }
 
 }  // namespace tl
