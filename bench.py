@@ -575,9 +575,10 @@ def run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cf
     # and V with the quantised-weight GEMM (its weight reads: W_k, W_v rows)
     qkv_kv_bytes = 2 * (2048 * 2048 // 2 + 2048 * 16 * 2)
     avg_ctx = w.seq + (w.steps + 1) / 2
+    bucket_rows = sum(min(w.max_ctx, (p + 127) // 128 * 128) for p in range(w.seq, w.seq + w.steps)) / w.steps
     cases["b1_store_h"] = (blocks["loop"], [], False, 3 * blk_bytes + kv_bytes / 2,
                            7 * blk_bytes + 10 * qkv_kv_bytes, "h",
-                           round(10 * avg_ctx * 2 * 2048 * 2048 * 2 / 1e9, 2))
+                           round(10 * bucket_rows * 2 * 2048 * 2048 * 2 / 1e9, 2))
     for name, case in cases.items():
         loop_blk, variants, cross, hbm_b, l2_b = case[:5]
         kv_dtype = case[5] if len(case) > 5 else "fp16"
@@ -605,7 +606,8 @@ def run_b1_variants(model, blocks, w, syn, tl, torch, np, timed, dist, world, cf
                      "workload": "prompt 256 + 128 steps, L=8, FP16 KV, batch 1"}
         if kv_dtype == "h":
             out[name]["workload"] = ("prompt 256 + 128 steps, L=8, store-h cache (fp16 QKV-input "
-                                     "rows; K and V rebuilt every step), batch 1, no CUDA graph")
+                                     "rows; K and V of every position below the step's 128-"
+                                     "position bucket rebuilt every step), batch 1")
             out[name]["rebuild_gflop_per_step"] = case[6]
             out[name]["cache_bytes"] = tl.tl_kv_bytes(m.handle, w.max_ctx, [8], tl.TL_KV_H)
             out[name]["cache_bytes_fp16_kv"] = tl.tl_kv_bytes(m.handle, w.max_ctx, [8],

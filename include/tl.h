@@ -325,8 +325,9 @@ tl_status tl_loops_used(tl_model* model, int* loops, int n, tl_stream stream);
  * cores, RoPE after it) into a workspace that follows the slots in the same
  * buffer (a header, one fp16 K/V layer per lane and the GEMM's partial sums),
  * then attends over them.  Prefill and decode steps support it; tl_extend and
- * tl_spec_step return TL_ERR_UNSUPPORTED, and decode steps run without CUDA
- * graphs (the rebuild's size changes with every position).
+ * tl_spec_step return TL_ERR_UNSUPPORTED.  A decode step rebuilds every
+ * position below the lane's position rounded up to a multiple of 128 (at most
+ * max_ctx), so its captured graph serves 128 consecutive steps.
  * ------------------------------------------------------------------------ */
 typedef struct tl_kv tl_kv;
 

@@ -866,6 +866,13 @@ tl_status enqueue_block_body(tl_model* m, const tl_block* b, int layer, int rows
   return ok();
 }
 
+// Store-h: positions rebuilt for a lane whose next token sits at
+// pos + off: pos + off rounded up to a multiple of 128, capped by the cache.
+int rebuild_rows(const tl_kv* kv, int lane, int off) {
+  const int p = kv->pos[lane] + off;
+  return p == 0 ? 0 : std::min(kv->max_ctx, (p + 127) / 128 * 128);
+}
+
 // Store-h: rebuild the K/V of every row's lane at positions 0 .. pos - 1 from
 // the slot's fp16 input rows: the quantised-weight GEMM of those rows with the
 // W_k, W_v rows of the layer's QKV matrix (odd-iteration codes when `odd`),
@@ -877,7 +884,12 @@ tl_status rebuild_kv(tl_model* m, const tl_block_desc& bd, int layer, int rows, 
   const size_t wpr = (size_t)words_per_row(d, bd.bits), gpr = (size_t)(d / bd.group);
   for (int i = 0; i < rows; ++i) {
     const int lane = rm->lane[i];
-    const int pos = kv->pos[lane] + rm->off[i];
+    // every position below the lane's bucket (the step's position rounded up
+    // to a multiple of 128, at most the cache size) is rebuilt: the launch
+    // shapes then change only every 128 steps, so a captured graph serves
+    // them; rows past the position are rebuilt from whatever the slot holds
+    // there and never read
+    const int pos = rebuild_rows(kv, lane, rm->off[i]);
     const __half* slot = (const __half*)(kv->buffer + kKvHeaderBytes +
                                          (size_t)(rm->cum[i] + layer) * kv->layer_bytes);
     // positions [p0, p0 + n): one GEMM and one RoPE pass each
@@ -1007,13 +1019,20 @@ tl_status enqueue_decode_layer(tl_model* m, const tl_block* b, int layer, int ro
     TL_TRY(launch_attn_decode_fused(da, s));
   }
   if (store_h) {
-    // this step's input rows join the slots at the rows' positions
+    // this step's input rows join the slots at the rows' positions (read on
+    // the device)
+    AppendRowsArgs ar;
+    memset(&ar, 0, sizeof(ar));
+    ar.x = m->x;
+    ar.rows = rows;
+    ar.d = d;
+    ar.hdr = (const KvHeader*)kv->buffer;
     for (int i = 0; i < rows; ++i) {
-      const int pos = kv->pos[rm->lane[i]] + rm->off[i];
-      char* slot = kv->buffer + kKvHeaderBytes + (size_t)(rm->cum[i] + layer) * kv->layer_bytes;
-      TL_CUDA(cudaMemcpyAsync(slot + (size_t)pos * d * 2, m->x + (size_t)i * d, (size_t)d * 2,
-                              cudaMemcpyDeviceToDevice, s));
+      ar.slot[i] = (__half*)(kv->buffer + kKvHeaderBytes + (size_t)(rm->cum[i] + layer) * kv->layer_bytes);
+      ar.lane[i] = rm->lane[i];
+      ar.off[i] = rm->off[i];
     }
+    TL_TRY(launch_append_rows(ar, s));
   }
   // O projection, added into the residual stream
   p.w0 = bd.w_o;
@@ -1321,8 +1340,11 @@ TL_API tl_status tl_decode_step(tl_model* model, tl_kv* kv, const int32_t* ids,
                     std::to_string(ids ? 1 : 0) + "|" + std::to_string((uintptr_t)h_trace);
   for (int b = 0; b < n_lanes; ++b) key += "|" + std::to_string(L_per_lane[b]);
   const bool use_ids = ids != nullptr;
-  // store-h: the rebuild's row counts follow the positions, so no graph
-  if (model->graphs && kv->dtype != TL_KV_H) {
+  // store-h: the rebuild's row counts change every 128 positions; they are
+  // part of the graph key
+  if (kv->dtype == TL_KV_H)
+    for (int b = 0; b < n_lanes; ++b) key += "|h" + std::to_string(rebuild_rows(kv, b, 0));
+  if (model->graphs) {
     TL_TRY(run_graph(
         model, key, kv->id, s,
         [&](cudaStream_t cs, int32_t* lmap) {

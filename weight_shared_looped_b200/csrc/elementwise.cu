@@ -415,6 +415,24 @@ tl_status launch_add_pos(KvHeader* hdr, int lane, int n, cudaStream_t s) {
   return ok();
 }
 
+namespace {
+__global__ void append_rows_kernel(AppendRowsArgs a) {
+  pdl_enter();
+  const int r = blockIdx.x;
+  const int pos = a.hdr->pos[a.lane[r]] + a.off[r];
+  const uint4* src = reinterpret_cast<const uint4*>(a.x + (size_t)r * a.d);
+  uint4* dst = reinterpret_cast<uint4*>(a.slot[r] + (size_t)pos * a.d);
+  for (int i = threadIdx.x; i < a.d / 8; i += blockDim.x) dst[i] = src[i];
+}
+}  // namespace
+
+tl_status launch_append_rows(const AppendRowsArgs& a, cudaStream_t s) {
+  if (a.rows == 0) return ok();
+  if (a.d % 8 != 0) return set_error(TL_ERR_UNSUPPORTED, "append rows: d %% 8");
+  TL_LAUNCH_PDL(append_rows_kernel, a.rows, 256, 0, s, a);
+  return ok();
+}
+
 tl_status launch_set_i32(int32_t* p, int value, cudaStream_t s) {
   TL_LAUNCH_PDL(set_i32_kernel, 1, 1, 0, s, p, value);
   return ok();

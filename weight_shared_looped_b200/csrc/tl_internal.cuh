@@ -221,6 +221,18 @@ tl_status launch_set_pos(KvHeader* hdr, int lane, int value, cudaStream_t s);
 tl_status launch_advance_pos(KvHeader* hdr, int n_lanes, cudaStream_t s);
 tl_status launch_add_pos(KvHeader* hdr, int lane, int n, cudaStream_t s);   // pos[lane] += n
 tl_status launch_set_i32(int32_t* p, int value, cudaStream_t s);
+// Store-h: row r of x [rows][d] (fp16) goes to row hdr->pos[lane[r]] + off[r]
+// of the slot slot[r] ([max_ctx][d]); the position is read on the device, so a
+// graph can replay the append at every step.
+struct AppendRowsArgs {
+  const __half* x;
+  int rows, d;
+  const KvHeader* hdr;
+  __half* slot[kMaxLanes];
+  int lane[kMaxLanes];
+  int off[kMaxLanes];
+};
+tl_status launch_append_rows(const AppendRowsArgs& a, cudaStream_t s);
 
 // greedy head over the tied embedding (head.cu): ids[r] = argmax_v y[r] . E[v]
 // (lowest v on a tie), n <= 8 rows; part_s / part_v: head_parts() * 8 each
