@@ -60,3 +60,23 @@ def test_roofline_traffic_only_for_the_profiled_source(tmp_path, monkeypatch):
     (tmp_path / "k.cu").write_text("kernel v2\n")          # the kernel changed since the capture
     assert bench.ncu_traffic("k.md", ["k.cu"]) is None
     assert bench.ncu_traffic("missing.md", ["k.cu"]) is None
+
+
+def test_decode_roofline_accounting():
+    """The decode roofline's byte counts: one 407M-shaped block is its packed
+    codes plus fp16 scales for QKV, O, gate, up and down (INT4: 67.1 M weights
+    at half a byte plus one 2-byte scale per 128; INT3: padded 10-codes-per-
+    word rows), and t = HBM bytes / HBM bandwidth + L2 bytes / L2 bandwidth."""
+    import weight_shared_looped_b200 as tl
+    d, f = 2048, 8192
+    n_w = 3 * d * d + d * d + 3 * f * d
+    assert bench.block_bytes(tl, 4) == n_w // 2 + n_w // 128 * 2 == 34603008
+    words3 = 4 * ((d // 10 + 1 + 3) // 4)            # K = 2048: 205 words, padded to 208
+    words3_f = 4 * ((f // 10 + 1 + 3) // 4)          # K = 8192: 820 words (already whole vectors)
+    rows_d, rows_f = 3 * d + d + 2 * f, d            # rows with K = d and with K = f
+    assert bench.block_bytes(tl, 3) == (rows_d * words3 + rows_f * words3_f) * 4 + n_w // 128 * 2
+    r = bench.decode_roofline(t_step=100e-6, hbm_bytes=6.4e8, l2_bytes=1.6e9, hbm_gbs=6400.0,
+                              l2_gbs=16000.0)
+    assert r["roofline_us"] == 200.0                 # 100 us of HBM + 100 us of L2
+    assert r["frac_roofline"] == 2.0 and r["frac_hbm"] == 1.0
+    assert r["hbm_bytes_per_step"] == 640000000 and r["l2_bytes_per_step"] == 1600000000
