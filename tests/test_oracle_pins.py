@@ -758,3 +758,106 @@ def test_store_h_cross_iteration_uses_odd_weights():
         x16 = kv_h[layer]._x[:4].astype(np.float64)
         _, k_want, _ = (m.loop.qkv_from_x(x16, np.arange(4), odd=(layer == 2)))
         assert np.array_equal(k_h, k_want), layer
+
+
+# ---------------------------------------------------------------- planted mistakes, loop variants
+
+def _variant_pins_pass():
+    """The pins of cross-iteration rounding, the iteration variants, store-h
+    and the residual-norm check; returns False if any fails."""
+    checks = [test_sign_of_frac_hand_worked, lambda: test_odd_codes_bracket_the_quotient(64),
+              test_bit_plane_layout, test_cross_iteration_rounding_model,
+              test_iteration_variants_are_an_unrolled_stack, test_store_h_decode_brute_force,
+              test_store_h_cross_iteration_uses_odd_weights, test_exit_threshold_infinite_changes_nothing,
+              test_exit_threshold_zero_stops_after_the_first_iteration,
+              test_exit_loop_counts_are_the_first_norm_crossings]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def _variant_mutants():
+    orig_sof, orig_odd_codes, orig_pack_bits = o.sign_of_frac, o.odd_iteration_codes, o.pack_bits
+
+    def sof_ties_up(w, group, bits=4):            # a quotient equal to its code counts as above
+        w = np.asarray(w, np.float32)
+        codes, s16 = o.quantize_groupwise(w, bits, group)
+        s = np.repeat(s16.astype(np.float32), group, axis=1)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            r = (w / s).astype(np.float32)
+        return ((s != 0) & (r >= codes.astype(np.float32))).astype(np.uint8)
+
+    def sof_inverted(w, group, bits=4):           # the bit says the rounding went up
+        return (1 - orig_sof(w, group, bits)).astype(np.uint8)
+
+    def odd_codes_swapped(codes, bits):           # -1 where set, +1 where clear
+        return orig_odd_codes(codes, 1 - (np.asarray(bits) != 0))
+
+    def pack_bits_reversed(bits):                 # element 32j + i in bit 31 - i
+        b = np.asarray(bits)
+        n, k = b.shape
+        nw = (k + 31) // 32
+        b = np.concatenate([b, np.zeros((n, nw * 32 - k), b.dtype)], axis=1).reshape(n, nw, 32)
+        return orig_pack_bits(b[:, :, ::-1].reshape(n, nw * 32))
+
+    def odd_even_parity(self, layer):             # even loop iterations take the odd weights
+        it = layer - len(self.pre)
+        return self.cross_iter and it >= 0 and it % 2 == 0
+
+    def schedule_no_variants(self, L):            # the variants ignored
+        return self.pre + [self.loop] * L
+
+    def exit_check_from_zero(self, h, layer, frozen, loops, exit_tau):   # also before iteration 0
+        it = layer - len(self.pre)
+        if exit_tau is None or it < 0:
+            return
+        newly = ~frozen & (np.sqrt(np.sum(h * h, axis=-1)) > exit_tau)
+        loops[newly] = it
+        frozen |= newly
+
+    def exit_count_plus_one(self, h, layer, frozen, loops, exit_tau):    # loop count off by one
+        it = layer - len(self.pre)
+        if exit_tau is None or it < 1:
+            return
+        newly = ~frozen & (np.sqrt(np.sum(h * h, axis=-1)) > exit_tau)
+        loops[newly] = it + 1
+        frozen |= newly
+
+    def append_x_unrounded(self, x, blk, odd):    # store-h rows kept in fp64
+        x = np.asarray(x, np.float64)
+        self._x = x if self._x is None else np.concatenate([self._x[:self.n], x])
+        self._blk, self._odd = blk, odd
+        self.n += x.shape[0]
+
+    def rebuild_even_weights(self):               # odd iterations rebuilt with the even weights
+        _, k, v = self._blk.qkv_from_x(self._x[:self.n].astype(np.float64), np.arange(self.n), False)
+        return k, v
+
+    return [("sign_of_frac", sof_ties_up), ("sign_of_frac", sof_inverted),
+            ("odd_iteration_codes", odd_codes_swapped), ("pack_bits", pack_bits_reversed),
+            ("LoopedModel.odd", odd_even_parity), ("LoopedModel.schedule", schedule_no_variants),
+            ("LoopedModel._exit_check", exit_check_from_zero),
+            ("LoopedModel._exit_check", exit_count_plus_one),
+            ("KVSlot.append_x", append_x_unrounded), ("KVSlot._rebuild", rebuild_even_weights)]
+
+
+def test_variant_pins_pass_unmutated():
+    assert _variant_pins_pass()
+
+
+@pytest.mark.parametrize("idx", range(10))
+def test_planted_variant_mistake_is_caught(monkeypatch, idx):
+    """Each plausible mistake planted in the oracle's cross-iteration rounding,
+    iteration variants, store-h cache or residual-norm check makes at least
+    one of their pins fail."""
+    name, fn = _variant_mutants()[idx]
+    if "." in name:
+        cls, attr = name.split(".")
+        monkeypatch.setattr(getattr(o, cls), attr, fn)
+    else:
+        monkeypatch.setattr(o, name, fn)
+    assert not _variant_pins_pass()
+
