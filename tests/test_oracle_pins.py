@@ -587,27 +587,49 @@ def test_greedy_head_brute_force():
         assert m.greedy_head(y[r:r + 1])[0] == max(range(len(scores)), key=lambda v: (scores[v], -v))
 
 
+def _spec_model():
+    """The tiny model with its projections five times stronger, so that the
+    block, not the token's own embedding, decides the greedy token: greedy
+    decoding then moves between tokens and shallow drafts get rejected."""
+    cfg = _tiny_cfg()
+
+    def wts(seed):
+        w = _tiny_weights(seed)
+        return {k: ((v * 5).astype(np.float32) if k.startswith("w_") else v) for k, v in w.items()}
+    pre = [o.Block.from_fp32(wts(11), cfg)]
+    loop = o.Block.from_fp32(wts(61), cfg)
+    gam = 1 + 0.1 * np.random.default_rng(11).standard_normal(8)
+    emb = (np.random.default_rng(12).standard_normal((20, 8))).astype(np.float16)
+    return o.LoopedModel(pre, loop, gam, emb)
+
+
 @pytest.mark.parametrize("K,L_draft", [(1, 1), (3, 1), (4, 2), (7, 2), (3, 3)])
 def test_spec_step_emits_the_greedy_decode_tokens(K, L_draft):
     """Greedy self-speculative decoding with an exact verify emits exactly the
-    tokens greedy decoding at the verify depth emits, whatever the draft."""
+    tokens greedy decoding at the verify depth emits, whatever the draft; a
+    shallower draft gets some of its tokens rejected on the way, a draft at
+    the verify depth none."""
     L = 3
-    m = _tiny_model()
+    m = _spec_model()
     prompt = np.array([3, 17, 5, 11], np.int64)
     kv_s, kv_g = m.new_kv(L, "fp16"), m.new_kv(L, "fp16")
     m.prefill(prompt[:-1], L, kv=kv_s)
     m.prefill(prompt[:-1], L, kv=kv_g)
-    tok, got = int(prompt[-1]), []
+    tok, got, lens = int(prompt[-1]), [], []
     while len(got) < 12:
         out = m.spec_step(tok, K, L_draft, L, kv_s)
         assert 1 <= len(out) <= K + 1
         got += out
+        lens.append(len(out))
         tok = out[-1]
         assert len(kv_s[0]) == len(prompt) - 1 + len(got)
     want = m.greedy_decode(int(prompt[-1]), len(got), L, kv_g)
     assert got == want
-    if L_draft == L:                    # the draft is the verify model: all accepted
-        assert len(m.spec_step(tok, K, L, L, kv_s)) == K + 1
+    assert len(set(want)) > 2                   # greedy decoding is not stuck on one token
+    if L_draft < L:
+        assert min(lens) < K + 1                # some draft was rejected
+    else:                                       # the draft is the verify model: all accepted
+        assert lens == [K + 1] * len(lens)
 
 
 # ---------------------------------------------------------------- cross-iteration rounding (sign of frac)
@@ -861,3 +883,58 @@ def test_planted_variant_mistake_is_caught(monkeypatch, idx):
         monkeypatch.setattr(o, name, fn)
     assert not _variant_pins_pass()
 
+
+
+# ---------------------------------------------------------------- planted mistakes, speculative step
+
+def _spec_pins_pass():
+    checks = [test_greedy_head_brute_force, lambda: test_spec_step_emits_the_greedy_decode_tokens(3, 1),
+              lambda: test_spec_step_emits_the_greedy_decode_tokens(4, 2),
+              lambda: test_spec_step_emits_the_greedy_decode_tokens(3, 3)]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def _spec_step_with(accept_mismatch: bool, keep: int):
+    """The self-speculative step with one planted mistake: accept the first
+    mismatching draft too, or keep `keep` entries fewer in the cache."""
+    def spec_step(self, token, K, L_draft, L_verify, kv):
+        p = len(kv[0])
+        drafts, t = [], token
+        for _ in range(K):
+            t = int(self.greedy_head(self.decode_step(np.int64(t), L_draft, kv))[0])
+            drafts.append(t)
+        for slot in kv:
+            slot.truncate(p)
+        ver = [int(v) for v in self.greedy_head(self.extend(np.array([token] + drafts, np.int64),
+                                                            L_verify, kv))]
+        m = 0
+        while m < K and drafts[m] == ver[m]:
+            m += 1
+        if accept_mismatch and m < K:
+            m += 1
+        for slot in kv:
+            slot.truncate(p + m + 1 - keep)
+        return drafts[:m] + [ver[m]]
+    return spec_step
+
+
+@pytest.mark.parametrize("mutant", ["argmin_head", "accept_mismatch", "cache_short"])
+def test_planted_spec_mistake_is_caught(monkeypatch, mutant):
+    """Each plausible mistake planted in the greedy head or the speculative
+    step makes at least one of their pins fail."""
+    assert _spec_pins_pass()
+    if mutant == "argmin_head":
+        def head(self, y):
+            logits = np.asarray(y, np.float64).reshape(-1, self.cfg["d_model"]) @ self.embed16.astype(np.float64).T
+            return np.argmin(logits, axis=-1)
+        monkeypatch.setattr(o.LoopedModel, "greedy_head", head)
+    elif mutant == "accept_mismatch":
+        monkeypatch.setattr(o.LoopedModel, "spec_step", _spec_step_with(True, 0))
+    else:
+        monkeypatch.setattr(o.LoopedModel, "spec_step", _spec_step_with(False, 1))
+    assert not _spec_pins_pass()
