@@ -938,3 +938,101 @@ def test_planted_spec_mistake_is_caught(monkeypatch, mutant):
     else:
         monkeypatch.setattr(o.LoopedModel, "spec_step", _spec_step_with(False, 1))
     assert not _spec_pins_pass()
+
+
+# ---------------------------------------------------------------- planted mistakes, integer outputs
+
+_HAND = [(4, [0.7, -0.35, 0.1, 0, 0.2499, -0.7, 0.05, 0.35], 0x2E66, [7, -4, 1, 0, 2, -7, 1, 4]),
+         (4, [7, 2.5, -2.5, 3.5, -0.5, 0.5, 1.5, 0], 0x3C00, [7, 2, -2, 4, 0, 0, 2, 0]),
+         (3, [3, 1.5, -1.5, 2.5, -0.5, 0.5, -3, 0], 0x3C00, [3, 2, -2, 2, 0, 0, -3, 0]),
+         (3, [-0.3, 0.1, 0.05, 0, 0, 0, 0, 0], 0x2E66, [-3, 1, 1, 0, 0, 0, 0, 0])]
+
+
+def _integer_pins_pass():
+    """The pins of the bit-exact outputs: quantisers, word layouts, INT8 KV."""
+    checks = [lambda h=h: test_quantize_hand_worked(*h) for h in _HAND]
+    checks += [test_pack_layout_int4_nibble_order, test_pack_layout_int3_ten_per_word,
+               lambda: test_quantize_properties(4, 64), lambda: test_quantize_properties(3, 128),
+               test_kv_int8_hand_worked, test_kv_int8_properties]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def _quantizer(scale_fn, round_fn, qmax_of):
+    """quantize_groupwise with its scale and rounding steps replaceable."""
+    def q(w, bits, group):
+        w = np.asarray(w, np.float32)
+        n, k = w.shape
+        qmax = np.float32(qmax_of(bits))
+        g = w.reshape(n, k // group, group)
+        absmax = np.max(np.abs(g), axis=2)
+        scale16 = (absmax / qmax).astype(np.float32).astype(np.float16)
+        s = scale_fn(absmax, qmax, scale16)[:, :, None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = (g / s).astype(np.float32)
+        ratio = np.where(s == 0, np.float32(0), ratio)
+        codes = np.clip(round_fn(ratio), -qmax - 1, qmax).astype(np.int8)
+        return codes.reshape(n, k), scale16
+    return q
+
+
+def _kv_quantizer(div, use_rounded):
+    def q(x16):
+        x = np.asarray(x16, np.float16).astype(np.float32)
+        absmax = np.max(np.abs(x), axis=-1)
+        scale16 = (absmax / np.float32(div)).astype(np.float32).astype(np.float16)
+        s = (scale16.astype(np.float32) if use_rounded else (absmax / np.float32(127)))[..., None]
+        with np.errstate(divide="ignore", invalid="ignore"):
+            ratio = (x / s).astype(np.float32)
+        ratio = np.where(s == 0, np.float32(0), ratio)
+        return np.clip(np.rint(ratio), -127, 127).astype(np.int8), scale16
+    return q
+
+
+def _integer_mutants():
+    rounded = lambda absmax, qmax, s16: s16.astype(np.float32)               # noqa: E731
+    unrounded = lambda absmax, qmax, s16: (absmax / qmax).astype(np.float32)  # noqa: E731
+    half_away = lambda r: np.sign(r) * np.floor(np.abs(r) + np.float32(0.5))   # noqa: E731
+    orig_pack = o.pack_codes
+
+    def pack_high_nibble_first(codes, bits):
+        if bits != 4:
+            return orig_pack(codes, bits)
+        c = np.asarray(codes).reshape(codes.shape[0], -1, 8)[:, :, ::-1]
+        return orig_pack(c.reshape(codes.shape), bits)
+
+    def pack_int3_zero_padding(codes, bits):
+        words = orig_pack(codes, bits)
+        if bits != 3:
+            return words
+        k = codes.shape[1]
+        w = words.astype(np.uint64)
+        for slot in range(k, words.shape[1] * 10):     # clear the padding slots (u = 4 -> 0)
+            j, i = divmod(slot, 10)
+            w[:, j] &= ~np.uint64(7 << (3 * i))
+        return w.astype(np.uint32)
+
+    return [("quantize_groupwise", _quantizer(unrounded, np.rint, o.QMAX.get)),
+            ("quantize_groupwise", _quantizer(rounded, half_away, o.QMAX.get)),
+            ("quantize_groupwise", _quantizer(rounded, np.rint, lambda b: o.QMAX[b] + 1)),
+            ("pack_codes", pack_high_nibble_first), ("pack_codes", pack_int3_zero_padding),
+            ("kv_quant_int8", _kv_quantizer(128, True)), ("kv_quant_int8", _kv_quantizer(127, False))]
+
+
+def test_integer_pins_pass_unmutated():
+    assert _integer_pins_pass()
+
+
+@pytest.mark.parametrize("idx", range(7))
+def test_planted_integer_mistake_is_caught(monkeypatch, idx):
+    """Each plausible mistake planted in a quantiser or a word layout (the
+    unrounded scale, round half away from zero, the wrong level count, the
+    nibble order, the INT3 padding code, the INT8 divisor, the unrounded INT8
+    scale) makes at least one pin of the bit-exact outputs fail."""
+    name, fn = _integer_mutants()[idx]
+    monkeypatch.setattr(o, name, fn)
+    assert not _integer_pins_pass()
