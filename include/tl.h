@@ -337,9 +337,21 @@ typedef struct tl_kv tl_kv;
 tl_status tl_kv_layer_bytes(int n_heads, int head_dim, int max_ctx, tl_kv_dtype dtype,
                             size_t* bytes);
 
+/* Bytes of the cache buffer for n_lanes lanes of max_ctx positions each, lane
+ * b running L_per_lane[b] loop iterations: the 4 KiB header, every lane's
+ * n_pre + L_b slots (tl_kv_layer_bytes each) and, for TL_KV_H, the rebuild
+ * workspace.  Host-only.  Errors: TL_ERR_INVALID_ARG for a NULL model,
+ * L_per_lane or bytes, n_lanes outside [1, 8], max_ctx outside [1, the
+ * model's max_ctx], an L outside [1, max_L] or an unknown dtype. */
 tl_status tl_kv_bytes(const tl_model* model, int n_lanes, int max_ctx,
                       const int* L_per_lane /* host [n_lanes] */,
                       tl_kv_dtype dtype, size_t* bytes);
+/* Lays a cache out in `buffer` (device, caller-owned, 256-byte aligned, at
+ * least tl_kv_bytes bytes) and sets every lane's position to 0.  The handle
+ * references the buffer and the model, which must outlive it; tl_kv_destroy
+ * releases the handle (and the model's graphs captured for it), never the
+ * buffer.  Errors: those of tl_kv_bytes; TL_ERR_INVALID_ARG for a NULL `out`,
+ * a NULL, misaligned or short buffer; TL_ERR_CUDA if the header upload fails. */
 tl_status tl_kv_create(const tl_model* model, int n_lanes, int max_ctx,
                        const int* L_per_lane /* host [n_lanes] */,
                        tl_kv_dtype dtype, void* buffer, size_t buffer_bytes,
