@@ -210,3 +210,42 @@ def test_int3_block_wraps_without_device_work():
     assert tl.lib.tl_block_device_bytes(out, ctypes.byref(n)) == tl.TL_OK
     assert n.value == 0
     assert tl.lib.tl_block_destroy(out) == tl.TL_OK
+
+
+@pytest.mark.parametrize("N,K", [(1, 1), (3, 31), (48, 256), (6144, 2048), (2048, 8192), (5, 100)])
+def test_sign_bits_bytes_match_oracle_plane(N, K):
+    """The sign plane is the oracle's bit-plane layout: uint32 [N, ceil(K/32)]."""
+    want = o.pack_bits(np.zeros((N, K), np.uint8)).nbytes
+    assert tl.tl_sign_bits_bytes(N, K) == want == N * ((K + 31) // 32) * 4
+
+
+def test_sign_plane_is_a_quarter_of_the_int4_codes():
+    """One bit per weight on top of four: the pages' "+25 % storage" for the
+    sign-of-frac channel ("Performance and Memory", "Cross-iteration stochastic
+    rounding"), for every matrix of the 407M-shaped block."""
+    d, f = 2048, 8192
+    for n, k in ((3 * d, d), (d, d), (f, d), (f, d), (d, f)):
+        codes, _ = tl.tl_packed_bytes(n, k, 4, 128)
+        assert tl.tl_sign_bits_bytes(n, k) * 4 == codes
+
+
+@pytest.mark.parametrize("args,status", [
+    ((64, 128, 5, 64), tl.TL_ERR_UNSUPPORTED),     # bits
+    ((64, 128, 4, 32), tl.TL_ERR_UNSUPPORTED),     # group
+    ((64, 96, 4, 64), tl.TL_ERR_INVALID_ARG),      # K % group
+    ((0, 128, 4, 64), tl.TL_ERR_INVALID_ARG),      # empty N
+])
+def test_pack_sign_bits_rejects_before_launch(args, status):
+    n, k, bits, group = args
+    p = ctypes.c_void_p(16)
+    assert tl.lib.tl_pack_sign_bits(p, n, k, bits, group, p, p, None) == status
+    assert tl.lib.tl_last_error()
+
+
+def test_sign_bits_null_arguments_rejected():
+    p = ctypes.c_void_p(16)
+    assert tl.lib.tl_pack_sign_bits(None, 64, 128, 4, 64, p, p, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_pack_sign_bits(p, 64, 128, 4, 64, None, p, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_pack_sign_bits(p, 64, 128, 4, 64, p, None, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_sign_bits_bytes(64, 128, None) == tl.TL_ERR_INVALID_ARG
+    assert tl.lib.tl_sign_bits_bytes(0, 128, ctypes.byref(ctypes.c_size_t())) == tl.TL_ERR_INVALID_ARG
