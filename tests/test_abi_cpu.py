@@ -249,3 +249,42 @@ def test_sign_bits_null_arguments_rejected():
     assert tl.lib.tl_pack_sign_bits(p, 64, 128, 4, 64, p, None, None) == tl.TL_ERR_INVALID_ARG
     assert tl.lib.tl_sign_bits_bytes(64, 128, None) == tl.TL_ERR_INVALID_ARG
     assert tl.lib.tl_sign_bits_bytes(0, 128, ctypes.byref(ctypes.c_size_t())) == tl.TL_ERR_INVALID_ARG
+
+
+def test_null_handles_rejected_before_any_work():
+    """Every call on a model, block or cache handle checks the handle first
+    (a NULL handle is TL_ERR_INVALID_ARG, nothing launched); destroying NULL
+    is a no-op."""
+    p = ctypes.c_void_p(16)
+    sz = ctypes.c_size_t()
+    i = ctypes.c_int()
+    one = (ctypes.c_int * 1)(1)
+    E = tl.TL_ERR_INVALID_ARG
+    L = tl.lib
+    calls = [
+        L.tl_block_device_bytes(None, ctypes.byref(sz)),
+        L.tl_model_device_bytes(None, ctypes.byref(sz)),
+        L.tl_model_set_graphs(None, 1),
+        L.tl_model_set_decode_chunks(None, 0),
+        L.tl_model_set_exit_threshold(None, 1.0),
+        L.tl_model_set_cross_iter(None, 1),
+        L.tl_model_set_iteration_blocks(None, None, 0),
+        L.tl_loops_used(None, p, 1, None),
+        L.tl_kv_bytes(None, 1, 16, ctypes.cast(one, ctypes.c_void_p), 0, ctypes.byref(sz)),
+        L.tl_kv_create(None, 1, 16, ctypes.cast(one, ctypes.c_void_p), 0, p, 1 << 20, None),
+        L.tl_kv_reset(None, 0, None),
+        L.tl_kv_position(None, 0, ctypes.byref(i)),
+        L.tl_kv_set_position(None, 0, 0, None),
+        L.tl_kv_layer_ptrs(None, 0, 0, ctypes.byref(ctypes.c_void_p()), ctypes.byref(ctypes.c_void_p()),
+                           ctypes.byref(ctypes.c_void_p()), ctypes.byref(ctypes.c_void_p())),
+        L.tl_decode_step(None, None, p, None, ctypes.cast(one, ctypes.c_void_p), 0, None, None, None),
+        L.tl_extend(None, None, 0, p, None, 1, 1, None, None, None),
+        L.tl_greedy_head(None, p, 1, p, None),
+        L.tl_spec_step(None, None, 0, 1, 2, 1, 2, p, ctypes.byref(i), None),
+        L.tl_check_bounded_wait(None, 1000, None),
+        L.tl_sync_status(None, None),
+    ]
+    assert calls == [E] * len(calls), calls
+    assert L.tl_block_destroy(None) == tl.TL_OK
+    assert L.tl_model_destroy(None) == tl.TL_OK
+    assert L.tl_kv_destroy(None) == tl.TL_OK
